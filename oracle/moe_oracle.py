@@ -1,0 +1,504 @@
+"""CPU oracle for the forward pass of one sparse MoE FFN layer (fp64, numpy).
+
+TEST INFRASTRUCTURE ONLY.  This module is the plain, slow, obviously correct
+statement of what the layer computes, used to check the CUDA library.  Only the
+tests, ``__graft_entry__.smoke()`` and the CPU-baseline leg of ``bench.py``
+may import it.  It shares no code with the CUDA path and imports nothing from
+the product package; the product path never calls it.
+
+Every function follows the pages it cites.  The pages (web articles) are:
+
+  [TKR]  "Top-k 路由（Top-k Routing）", compassingai.com concept page
+  [RAT]  "Mixture of Experts (MoE): 解释 MoE 的路由算法（Top-k / expert choice /
+         soft routing）与取舍", talentme M4-080
+  [GLO]  "Top-K Routing (MoE)", ayinedjimi-consultants glossary
+  [CMP]  "别只比较 Top-k：同一个数字，可能对应完全不同的专家工作量",
+         ailearn moe-comparison
+  [TINY] "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡",
+         f3dlife
+
+Arithmetic is float64 throughout, from the (bf16- or fp32-valued) inputs.
+Library primitives used as steps: numpy matmul, exp, and a stable argsort.
+
+Readings where the pages are silent (each one is listed in the design notes):
+  * ties in top-k / top-c go to the lower expert / token index;
+  * within a token, slot j holds the j-th largest key;
+  * rows of one expert are ordered by (token, slot) ascending, as torch.where
+    orders them in [TINY] section 5;
+  * under a capacity limit C = ceil(CF*T*k/E), the first C assignments of an
+    expert in (token, slot) order keep their slot, the rest are dropped and
+    contribute zero; gates are not renormalised after a drop;
+  * load f_e counts nominal (pre-capacity) routes over T*k;
+  * under sigmoid affinity the importance P_e is the mean of the affinities
+    normalised to sum 1 over experts;
+  * under expert choice the merge weight is the softmax probability, a token
+    taken by several experts sums their contributions, an untaken token gets 0;
+  * shared experts are added with weight 1.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+(worked examples of the pages, closed forms, brute force and reductions to
+dense/soft routing); none is "parity unpinned".
+"""
+
+from __future__ import annotations
+
+import math
+
+import numpy as np
+
+__all__ = [
+    "router_logits", "softmax_rows", "sigmoid", "routing_keys",
+    "topk_desc", "route_token_choice", "route_expert_choice",
+    "capacity", "dispatch_token_choice", "dispatch_expert_choice",
+    "swiglu_expert", "relu_expert", "expert_rows",
+    "combine", "balance_stats", "layer_forward", "layer_forward_rows",
+    "dense_masked_forward", "soft_routing_forward",
+]
+
+
+# --------------------------------------------------------------------------
+# Score: router logits and affinity
+# --------------------------------------------------------------------------
+
+def router_logits(x, Wg):
+    """s = W_g . x for every token: logits[t, e] = sum_d Wg[e, d] * x[t, d].
+
+    [TKR] "門控函式的數學形式" Step 1 (W_g in R^{N x d}); [TINY] section 4
+    (router = nn.Linear(D, E, bias=False), weight stored [E, D]).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    Wg = np.asarray(Wg, dtype=np.float64)
+    return x @ Wg.T
+
+
+def softmax_rows(s):
+    """Softmax over the experts of each token (max-subtracted for range).
+
+    [TKR] gate Step 2, variant (a); [TINY] section 4 (F.softmax over dim=-1).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    z = np.exp(s - s.max(axis=1, keepdims=True))
+    return z / z.sum(axis=1, keepdims=True)
+
+
+def sigmoid(s):
+    """Sigmoid affinity sigma(s) = 1 / (1 + e^{-s}), per expert.
+
+    [CMP] "评分、Top-k、合并权重和实际执行" Score step (DeepSeek-V3 uses a
+    Sigmoid affinity).
+    """
+    s = np.asarray(s, dtype=np.float64)
+    return 1.0 / (1.0 + np.exp(-s))
+
+
+def routing_keys(x, Wg, bias=None, score="softmax"):
+    """Per-token keys that top-k selection ranks.
+
+    Softmax: the logits themselves (softmax is monotone within a row, so the
+    top-k of probabilities and of logits coincide).  Sigmoid: sigma(s) + b,
+    the selection-only bias of [CMP] "Select" / [RAT] variant (d).
+    """
+    s = router_logits(x, Wg)
+    if score == "softmax":
+        return s
+    k = sigmoid(s)
+    if bias is not None:
+        k = k + np.asarray(bias, dtype=np.float64)[None, :]
+    return k
+
+
+def softmax_probs_of(x, Wg):
+    """Soft probabilities of every token (expert-choice keys), [TINY] section 4."""
+    return softmax_rows(router_logits(x, Wg))
+
+
+# --------------------------------------------------------------------------
+# Select: token choice top-k, expert choice top-c
+# --------------------------------------------------------------------------
+
+def topk_desc(keys, k):
+    """Indices of the k largest keys per row, largest first; ties -> lower index.
+
+    [TKR] gate "top_k_indices = argtopk"; [TINY] section 4 (torch.topk).  A
+    stable sort of -key keeps equal keys in index order.
+    """
+    keys = np.asarray(keys, dtype=np.float64)
+    order = np.argsort(-keys, axis=1, kind="stable")
+    return order[:, :k]
+
+
+def route_token_choice(logits, k, score="softmax", gate="renorm", bias=None):
+    """Token-choice routing from router logits.
+
+    Returns (ids[T,k] int, gates[T,k], probs_for_importance[T,E]).
+
+    * softmax + renorm (Mixtral, tiny): p = softmax(s); pick the k largest;
+      g_j = p_j / sum_sel p   -- [GLO] TopKRouter, [TINY] section 4,
+      [RAT] variant (a).  Equal to softmax over the selected logits
+      ([TKR] gate Step 2, variant (b)).
+    * softmax + raw (Switch): top-1 of softmax, gate = the softmax value,
+      no renormalisation -- [TKR] gate Step 2 note on Switch Transformer.
+    * sigmoid (+ optional selection-only bias): select on sigma(s) + b,
+      merge weight sigma(s_j) / sum_sel sigma(s)  (bias excluded) --
+      [CMP] "Select" / "Merge" steps, DeepSeek-V3 row of the family table.
+    """
+    s = np.asarray(logits, dtype=np.float64)
+    T, E = s.shape
+    if score == "softmax":
+        p = softmax_rows(s)
+        ids = topk_desc(s, k)
+        psel = np.take_along_axis(p, ids, axis=1)
+        imp = p
+    elif score == "sigmoid":
+        a = sigmoid(s)
+        key = a + (np.asarray(bias, dtype=np.float64)[None, :] if bias is not None else 0.0)
+        ids = topk_desc(key, k)
+        psel = np.take_along_axis(a, ids, axis=1)
+        imp = a / a.sum(axis=1, keepdims=True)
+    else:
+        raise ValueError(score)
+    if gate == "renorm":
+        g = psel / psel.sum(axis=1, keepdims=True)
+    elif gate == "raw":
+        g = psel
+    else:
+        raise ValueError(gate)
+    return ids.astype(np.int64), g, imp
+
+
+def route_expert_choice(logits, c):
+    """Expert-choice routing: every expert takes its c most probable tokens.
+
+    [TKR] "Token-Choice vs Expert-Choice" table (each expert picks top-C
+    tokens); [RAT] routing class (2).  p = softmax over experts per token;
+    per expert column, the c largest p (ties -> lower token id), reported in
+    ascending token order.  Returns (picked[E,c], probs[T,E]); the merge weight
+    of (t, e) is probs[t, e].
+    """
+    p = softmax_rows(logits)
+    T, E = p.shape
+    picked = np.empty((E, c), dtype=np.int64)
+    for e in range(E):
+        order = np.argsort(-p[:, e], kind="stable")[:c]
+        picked[e] = np.sort(order)
+    return picked, p
+
+
+# --------------------------------------------------------------------------
+# Execute: capacity and dispatch
+# --------------------------------------------------------------------------
+
+def capacity(capacity_factor, T, k, E):
+    """Expert buffer = CF * (tokens per batch / N) * k, rounded up.
+
+    [TKR] "容量因子" (capacity factor) formula.  The page gives no rounding;
+    ceil, evaluated in double as CF*T*k/E.
+    """
+    return int(math.ceil(float(capacity_factor) * T * k / E))
+
+
+def dispatch_token_choice(ids, E, cap=None):
+    """Group assignments by expert (the torch.where step of [TINY] section 5).
+
+    Assignment a = t*k + j is token t's j-th choice.  Rows of expert e are its
+    assignments in ascending a (token, then slot).  With a capacity `cap`
+    ([CMP] capacity + overflow table: Switch skips the expert for an
+    overflowing token), only the first `cap` of each expert keep a row.
+
+    Returns counts[E] (nominal), kept[E], offsets[E+1] (exclusive scan of kept),
+    row_src[A_kept] (assignment id per row), inv[T*k] (row per assignment, -1
+    if dropped).
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    T, k = ids.shape
+    flat = ids.reshape(-1)
+    counts = np.zeros(E, dtype=np.int64)
+    rank = np.empty_like(flat)
+    for a, e in enumerate(flat):              # plain running count per expert
+        rank[a] = counts[e]
+        counts[e] += 1
+    kept = counts.copy() if cap is None else np.minimum(counts, cap)
+    offsets = np.zeros(E + 1, dtype=np.int64)
+    offsets[1:] = np.cumsum(kept)
+    inv = np.full(T * k, -1, dtype=np.int64)
+    row_src = np.empty(int(offsets[-1]), dtype=np.int64)
+    for a, e in enumerate(flat):
+        if cap is None or rank[a] < cap:
+            r = offsets[e] + rank[a]
+            inv[a] = r
+            row_src[r] = a
+    return counts, kept, offsets, row_src, inv
+
+
+def dispatch_expert_choice(picked, T):
+    """Rows of expert e are its picked tokens in ascending token order.
+
+    Assignment id of (t, e) is t*E + e; inv[T*E] is the row of (t, e) or -1
+    (token t not picked by e).  Every expert has exactly c rows.
+    """
+    picked = np.asarray(picked, dtype=np.int64)
+    E, c = picked.shape
+    counts = np.full(E, c, dtype=np.int64)
+    offsets = np.arange(E + 1, dtype=np.int64) * c
+    row_src = np.empty(E * c, dtype=np.int64)
+    inv = np.full(T * E, -1, dtype=np.int64)
+    for e in range(E):
+        for i, t in enumerate(picked[e]):
+            r = e * c + i
+            row_src[r] = t * E + e
+            inv[t * E + e] = r
+    return counts, counts.copy(), offsets, row_src, inv
+
+
+# --------------------------------------------------------------------------
+# Expert compute
+# --------------------------------------------------------------------------
+
+def silu(z):
+    return z / (1.0 + np.exp(-z))
+
+
+def swiglu_expert(xr, Wgate, Wup, Wdown):
+    """One SwiGLU expert on a block of rows.
+
+    [TINY] section 3: gate = SiLU(x W_gate), value = x W_up,
+    hidden = gate (.) value, output = hidden W_down, with nn.Linear weights
+    gate/up [F, D] and down [D, F].
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    g = xr @ np.asarray(Wgate, dtype=np.float64).T
+    u = xr @ np.asarray(Wup, dtype=np.float64).T
+    return (silu(g) * u) @ np.asarray(Wdown, dtype=np.float64).T
+
+
+def relu_expert(xr, Wup, Wdown):
+    """Classic two-matrix FFN D -> F -> D with a ReLU in between.
+
+    [TINY] section 2-3 (the classic D -> 4D -> D FFN; the Switch-style layer
+    here uses ReLU as its activation).
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    h = np.maximum(xr @ np.asarray(Wup, dtype=np.float64).T, 0.0)
+    return h @ np.asarray(Wdown, dtype=np.float64).T
+
+
+def expert_rows(act, xr, e, W_gate, W_up, W_down):
+    if act == "swiglu":
+        return swiglu_expert(xr, W_gate[e], W_up[e], W_down[e])
+    if act == "relu":
+        return relu_expert(xr, W_up[e], W_down[e])
+    raise ValueError(act)
+
+
+# --------------------------------------------------------------------------
+# Merge: weighted combine back to token rows
+# --------------------------------------------------------------------------
+
+def combine(T, D, y_rows, inv, gates, K, shared=None):
+    """out[t] = sum_j gates[t, j] * y_rows[inv[t, j]]  (+ sum of shared outputs).
+
+    [TKR] "Combine" (output = sum of gate_score_i * y_i); [TINY] section 6:
+    accumulate (index_add), never assign.  A dropped or unpicked assignment
+    (inv = -1) contributes 0.  Shared experts add with weight 1.
+    """
+    out = np.zeros((T, D), dtype=np.float64)
+    inv = np.asarray(inv).reshape(T, K)
+    gates = np.asarray(gates, dtype=np.float64).reshape(T, K)
+    for t in range(T):
+        for j in range(K):
+            r = inv[t, j]
+            if r >= 0:
+                out[t] += gates[t, j] * y_rows[r]
+    if shared is not None:
+        for ys in shared:
+            out += ys
+    return out
+
+
+# --------------------------------------------------------------------------
+# Balance statistics
+# --------------------------------------------------------------------------
+
+def balance_stats(importance_rows, counts, n_kept, n_routes, alpha):
+    """Load statistics and the auxiliary balance loss.
+
+    P_e = mean_t importance_rows[t, e] (average routing probability, before
+    selection); f_e = counts_e / n_routes (share of routes each expert gets,
+    [TINY] section 8: one_hot(topk).mean over (tokens, k)); aux = alpha * E *
+    sum_e f_e P_e ([TKR] "負載均衡" formula, [TINY] section 8).  Also
+    max/mean of the counts ([CMP] "先数 assignments": [9,4,2,1] -> 2.25) and
+    the number of dropped routes (n_routes - n_kept).
+    """
+    counts = np.asarray(counts, dtype=np.float64)
+    E = counts.shape[0]
+    P = np.asarray(importance_rows, dtype=np.float64).mean(axis=0)
+    f = counts / float(n_routes)
+    aux = alpha * E * float(np.sum(f * P))
+    mean = counts.sum() / E
+    return {
+        "P": P, "f": f, "aux": aux,
+        "max_over_mean": float(counts.max() / mean) if mean > 0 else 0.0,
+        "n_dropped": int(n_routes - n_kept),
+    }
+
+
+# --------------------------------------------------------------------------
+# Whole layer
+# --------------------------------------------------------------------------
+
+def _np(a):
+    if a is None:
+        return None
+    if hasattr(a, "detach"):          # a torch tensor handed in by a test
+        a = a.detach().float().cpu().numpy()
+    return np.asarray(a, dtype=np.float64)
+
+
+def route(w, logits, bias=None):
+    """Score + select + merge weights from given logits (fp32 GPU logits in
+    the bit-exact checks, or the oracle's own fp64 logits).
+
+    `w` is a mapping/object with fields k, c, E, T, score, select, gate,
+    overflow, capacity_factor, aux_alpha.
+    """
+    g = _get(w)
+    if g["select"] == "token":
+        ids, gates, imp = route_token_choice(logits, g["k"], g["score"], g["gate"], bias)
+        cap = capacity(g["capacity_factor"], g["T"], g["k"], g["E"]) if g["overflow"] == "drop" else None
+        counts, kept, offsets, row_src, inv = dispatch_token_choice(ids, g["E"], cap)
+        K = g["k"]
+        n_routes = g["T"] * g["k"]
+    else:
+        picked, p = route_expert_choice(logits, g["c"])
+        ids, gates, imp = picked, p, p
+        counts, kept, offsets, row_src, inv = dispatch_expert_choice(picked, g["T"])
+        K = g["E"]
+        n_routes = g["E"] * g["c"]
+        cap = None
+    stats = balance_stats(imp, counts, int(kept.sum()), n_routes, g["aux_alpha"])
+    return dict(ids=ids, gates=gates, importance=imp, counts=counts, kept=kept,
+                offsets=offsets, row_src=row_src, inv=inv, K=K, cap=cap, stats=stats)
+
+
+def _get(w):
+    keys = ["T", "D", "E", "F", "k", "c", "score", "select", "gate", "overflow",
+            "capacity_factor", "act", "n_shared", "F_shared", "aux_alpha"]
+    if isinstance(w, dict):
+        return {k: w[k] for k in keys}
+    return {k: getattr(w, k) for k in keys}
+
+
+def layer_forward(w, x, Wg, bias, W_gate, W_up, W_down,
+                  Ws_gate=None, Ws_up=None, Ws_down=None, logits=None):
+    """The whole forward pass (Gate -> Dispatch -> Expert compute -> Combine,
+    [TKR] lifecycle; [CMP] Score -> Select -> Merge -> Execute).
+
+    `logits`, when given, replaces the router product (used to route from the
+    GPU's fp32 logits).  Returns a dict with the routing, the stats, the
+    per-row expert outputs and out[T, D].
+    """
+    g = _get(w)
+    x = _np(x)
+    s = router_logits(x, _np(Wg)) if logits is None else _np(logits)
+    r = route(g, s, _np(bias))
+    Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
+    D = g["D"]
+    y = np.zeros((len(r["row_src"]), D), dtype=np.float64)
+    off = r["offsets"]
+    K = r["K"]
+    for e in range(g["E"]):
+        rows = slice(off[e], off[e + 1])
+        if off[e + 1] == off[e]:
+            continue
+        src_tok = r["row_src"][rows] // K
+        y[rows] = expert_rows(g["act"], x[src_tok], e, Wgt, Wu, Wd)
+    shared = None
+    if g["n_shared"]:
+        Sg, Su, Sd = _np(Ws_gate), _np(Ws_up), _np(Ws_down)
+        shared = [swiglu_expert(x, Sg[i], Su[i], Sd[i]) for i in range(g["n_shared"])]
+    out = combine(g["T"], D, y, r["inv"], r["gates"], K, shared)
+    r.update(logits=s, y_rows=y, shared=shared, out=out)
+    return r
+
+
+def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
+                       Ws_gate=None, Ws_up=None, Ws_down=None, logits=None,
+                       weights_of=None):
+    """out[t] for a sample of tokens at full size.
+
+    Routing and dispatch are computed for the whole batch (a drop depends on
+    earlier tokens); only the sampled tokens' expert rows are evaluated.
+    `weights_of(e)` (optional) returns (W_gate[e], W_up[e], W_down[e]) as fp64
+    arrays, so that a caller can stream expert weights from device memory one
+    expert at a time.
+    """
+    g = _get(w)
+    x = _np(x)
+    s = router_logits(x, _np(Wg)) if logits is None else _np(logits)
+    r = route(g, s, _np(bias))
+    K = r["K"]
+    tokens = [int(t) for t in tokens]
+    need = {}
+    for t in tokens:
+        for j in range(K):
+            row = r["inv"][t * K + j]
+            if row >= 0:
+                e = j if g["select"] == "expert" else int(r["ids"][t, j])
+                need.setdefault(e, []).append((t, j))
+    if weights_of is None:
+        Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
+
+        def weights_of(e):
+            return (Wgt[e] if Wgt is not None else None), Wu[e], Wd[e]
+    out = {t: np.zeros(g["D"], dtype=np.float64) for t in tokens}
+    gates = np.asarray(r["gates"], dtype=np.float64).reshape(g["T"], K)
+    for e in sorted(need):
+        wg_e, wu_e, wd_e = weights_of(e)
+        ts = [t for t, _ in need[e]]
+        if g["act"] == "swiglu":
+            ye = swiglu_expert(x[ts], wg_e, wu_e, wd_e)
+        else:
+            ye = relu_expert(x[ts], wu_e, wd_e)
+        for i, (t, j) in enumerate(need[e]):
+            out[t] += gates[t, j] * ye[i]
+    if g["n_shared"]:
+        Sg, Su, Sd = _np(Ws_gate), _np(Ws_up), _np(Ws_down)
+        for i in range(g["n_shared"]):
+            ys = swiglu_expert(x[tokens], Sg[i], Su[i], Sd[i])
+            for n, t in enumerate(tokens):
+                out[t] += ys[n]
+    r.update(logits=s, out_rows=np.stack([out[t] for t in tokens]) if tokens else
+             np.zeros((0, g["D"])))
+    return r
+
+
+# --------------------------------------------------------------------------
+# Second paths (used only to pin the first)
+# --------------------------------------------------------------------------
+
+def dense_masked_forward(w, x, Wg, bias, W_gate, W_up, W_down):
+    """Every expert on every token, then keep only each token's selected
+    experts with their gates.  Equal to the dropless sparse layer."""
+    g = _get(w)
+    x = _np(x)
+    s = router_logits(x, _np(Wg))
+    ids, gates, _ = route_token_choice(s, g["k"], g["score"], g["gate"], _np(bias))
+    Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
+    T = x.shape[0]
+    allout = np.stack([expert_rows(g["act"], x, e, Wgt, Wu, Wd) for e in range(g["E"])], 1)
+    mask = np.zeros((T, g["E"]), dtype=np.float64)
+    for t in range(T):
+        for j in range(g["k"]):
+            mask[t, ids[t, j]] = gates[t, j]
+    return np.einsum("te,ted->td", mask, allout)
+
+
+def soft_routing_forward(w, x, Wg, W_gate, W_up, W_down):
+    """Soft routing y = sum_i g_i(x) E_i(x) over all experts with softmax g
+    ([RAT] routing class (3))."""
+    g = _get(w)
+    x = _np(x)
+    p = softmax_rows(router_logits(x, _np(Wg)))
+    Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
+    allout = np.stack([expert_rows(g["act"], x, e, Wgt, Wu, Wd) for e in range(g["E"])], 1)
+    return np.einsum("te,ted->td", p, allout)

@@ -1,0 +1,398 @@
+"""Pins of the CPU oracle to facts the pages and mathematics fix (no GPU).
+
+Each test ties one oracle function to something other than itself: a worked
+example printed on a page (fixtures in tests/golden/, each citing its page and
+section), a closed form, brute force over a tiny input, or a reduction of the
+layer to a textbook computation (a dense FFN, soft routing).
+"""
+
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+from oracle import moe_oracle as O
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def gold(name):
+    with open(os.path.join(GOLD, name)) as f:
+        return json.load(f)
+
+
+def cfg(**kw):
+    base = dict(T=8, D=6, E=4, F=5, k=2, c=0, score="softmax", select="token",
+                gate="renorm", overflow="dropless", capacity_factor=0.0,
+                act="swiglu", n_shared=0, F_shared=0, aux_alpha=1e-2)
+    base.update(kw)
+    return base
+
+
+def rand_layer(rng, c, with_bias=False):
+    x = rng.standard_normal((c["T"], c["D"]))
+    Wg = rng.standard_normal((c["E"], c["D"]))
+    Wgate = rng.standard_normal((c["E"], c["F"], c["D"])) / math.sqrt(c["D"])
+    Wup = rng.standard_normal((c["E"], c["F"], c["D"])) / math.sqrt(c["D"])
+    Wdown = rng.standard_normal((c["E"], c["D"], c["F"])) / math.sqrt(c["F"])
+    b = rng.standard_normal(c["E"]) * 0.3 if with_bias else None
+    return x, Wg, b, Wgate, Wup, Wdown
+
+
+# ---------------------------------------------------------------- router ----
+
+def test_router_logits_basis_vector_gives_weight_column():
+    # s = W_g . x with x the d-th basis vector is column d of W_g (shape [E, D]).
+    rng = np.random.default_rng(1)
+    Wg = rng.standard_normal((5, 7))
+    for d in range(7):
+        x = np.zeros((1, 7))
+        x[0, d] = 1.0
+        np.testing.assert_array_equal(O.router_logits(x, Wg)[0], Wg[:, d])
+
+
+def test_router_logits_is_linear_in_x():
+    rng = np.random.default_rng(2)
+    Wg = rng.standard_normal((3, 4))
+    a, b = rng.standard_normal((1, 4)), rng.standard_normal((1, 4))
+    np.testing.assert_allclose(O.router_logits(2 * a - b, Wg),
+                               2 * O.router_logits(a, Wg) - O.router_logits(b, Wg), atol=1e-12)
+
+
+def test_softmax_rows_are_distributions_and_shift_invariant():
+    rng = np.random.default_rng(3)
+    s = rng.standard_normal((6, 5)) * 4
+    p = O.softmax_rows(s)
+    np.testing.assert_allclose(p.sum(1), 1.0, atol=1e-15)
+    np.testing.assert_allclose(O.softmax_rows(s + 100.0), p, atol=1e-14)
+    # ratio of two probabilities is e^{s_i - s_j}
+    np.testing.assert_allclose(p[:, 0] / p[:, 1], np.exp(s[:, 0] - s[:, 1]), rtol=1e-12)
+
+
+def test_sigmoid_closed_forms():
+    assert O.sigmoid(np.array([0.0]))[0] == 0.5
+    np.testing.assert_allclose(O.sigmoid(np.array([math.log(3.0)])), [0.75], rtol=1e-15)
+    np.testing.assert_allclose(O.sigmoid(np.array([-math.log(3.0)])), [0.25], rtol=1e-15)
+
+
+# ------------------------------------------------------------ selection ----
+
+def test_page_router_example_top2_renormalised():
+    g = gold("tiny_moe_router_example.json")
+    logits = np.log(np.array([g["router_probs"]]))
+    ids, gates, probs = O.route_token_choice(logits, g["k"], "softmax", "renorm")
+    assert ids[0].tolist() == g["topk_indices"]
+    np.testing.assert_allclose(np.take_along_axis(probs, ids, 1)[0], g["topk_weights"], rtol=1e-12)
+    np.testing.assert_allclose(gates[0], g["renormalized"], rtol=1e-12)
+    ids_raw, gates_raw, _ = O.route_token_choice(logits, g["k"], "softmax", "raw")
+    np.testing.assert_allclose(gates_raw[0], g["topk_weights"], rtol=1e-12)
+
+
+@pytest.mark.parametrize("E,k", [(4, 2), (6, 3), (8, 1), (5, 5)])
+def test_topk_matches_bruteforce_enumeration(E, k):
+    # The chosen set maximises the key sum over all C(E, k) subsets, and its
+    # members come in descending key order.
+    rng = np.random.default_rng(10 + E * 7 + k)
+    keys = rng.standard_normal((40, E))
+    ids = O.topk_desc(keys, k)
+    for t in range(keys.shape[0]):
+        best = max(itertools.combinations(range(E), k), key=lambda S: sum(keys[t, list(S)]))
+        assert sorted(ids[t].tolist()) == sorted(best)
+        vals = keys[t, ids[t]]
+        assert np.all(vals[:-1] > vals[1:])
+
+
+def test_topk_ties_go_to_lower_index():
+    keys = np.array([[1.0, 3.0, 3.0, 0.0, 3.0]])
+    assert O.topk_desc(keys, 2)[0].tolist() == [1, 2]
+    assert O.topk_desc(keys, 3)[0].tolist() == [1, 2, 4]
+
+
+def test_renormalised_gates_equal_softmax_over_selected_logits():
+    # [TKR] gate Step 2: g_i = e^{s_i} / sum_{j in TopK} e^{s_j} (variant b)
+    # equals softmax over all experts followed by renormalisation (variant a).
+    rng = np.random.default_rng(4)
+    s = rng.standard_normal((20, 6)) * 2
+    ids, gates, _ = O.route_token_choice(s, 3, "softmax", "renorm")
+    for t in range(20):
+        sel = s[t, ids[t]]
+        direct = [math.exp(v) / sum(math.exp(u) for u in sel) for v in sel]
+        np.testing.assert_allclose(gates[t], direct, rtol=1e-12)
+    np.testing.assert_allclose(gates.sum(1), 1.0, atol=1e-15)
+
+
+def test_switch_raw_gate_is_top1_softmax_value():
+    rng = np.random.default_rng(5)
+    s = rng.standard_normal((30, 8))
+    ids, gates, probs = O.route_token_choice(s, 1, "softmax", "raw")
+    np.testing.assert_allclose(gates[:, 0], probs.max(1), rtol=1e-15)
+    assert np.all(gates <= 1.0)
+    assert np.all(ids[:, 0] == s.argmax(1))
+
+
+def test_sigmoid_bias_changes_selection_but_not_merge_weights():
+    # logits chosen so that sigma(s) ranks expert 0 > 1 > 2, while the bias
+    # lifts expert 2 above expert 1 for selection only.
+    s = np.array([[2.0, 1.0, 0.5]])
+    b = np.array([0.0, 0.0, 0.15])
+    ids, gates, _ = O.route_token_choice(s, 2, "sigmoid", "renorm", bias=b)
+    assert ids[0].tolist() == [0, 2]
+    a0, a2 = 1 / (1 + math.exp(-2.0)), 1 / (1 + math.exp(-0.5))
+    np.testing.assert_allclose(gates[0], [a0 / (a0 + a2), a2 / (a0 + a2)], rtol=1e-14)
+    ids_nb, _, _ = O.route_token_choice(s, 2, "sigmoid", "renorm", bias=None)
+    assert ids_nb[0].tolist() == [0, 1]
+
+
+def test_expert_choice_bruteforce_and_exact_counts():
+    rng = np.random.default_rng(6)
+    T, E, c = 7, 3, 2
+    s = rng.standard_normal((T, E)) * 2
+    picked, p = O.route_expert_choice(s, c)
+    assert picked.shape == (E, c)
+    for e in range(E):
+        best = max(itertools.combinations(range(T), c), key=lambda S: sum(p[list(S), e]))
+        assert picked[e].tolist() == sorted(best)
+    counts, kept, offsets, row_src, inv = O.dispatch_expert_choice(picked, T)
+    assert counts.tolist() == [c] * E and offsets.tolist() == [0, 2, 4, 6]
+
+
+# -------------------------------------------------------------- dispatch ----
+
+def test_page_dispatch_example():
+    g = gold("tiny_moe_dispatch_example.json")
+    ids = np.array(g["topk_indices"])
+    counts, kept, offsets, row_src, inv = O.dispatch_token_choice(ids, g["num_experts"])
+    e = g["expert_id"]
+    rows = row_src[offsets[e]:offsets[e + 1]]
+    k = ids.shape[1]
+    assert (rows // k).tolist() == g["token_indices"]
+    assert (rows % k).tolist() == g["route_slots"]
+    assert ((ids == e).tolist() == g["mask"])
+    # inverse permutation
+    for r, a in enumerate(row_src):
+        assert inv[a] == r
+
+
+def test_counts_sum_to_routes_and_permutation_is_bijection():
+    gt = gold("tiny_moe_route_totals.json")
+    for cnt in gt["printed_counts"]:
+        assert sum(cnt) == gt["routes"] == gt["N"] * gt["K"]
+    rng = np.random.default_rng(7)
+    s = rng.standard_normal((gt["N"], 4))
+    ids, _, _ = O.route_token_choice(s, gt["K"])
+    counts, kept, offsets, row_src, inv = O.dispatch_token_choice(ids, 4)
+    assert counts.sum() == gt["routes"]
+    assert sorted(row_src.tolist()) == list(range(gt["routes"]))
+    assert sorted(inv.tolist()) == list(range(gt["routes"]))
+
+
+def test_capacity_formula_and_switch_value():
+    # [TKR] capacity factor: buffer = CF * tokens/N * k; Switch workload: 80 slots.
+    assert O.capacity(1.25, 8192, 1, 128) == 80
+    assert O.capacity(1.0, 10, 2, 4) == 5
+    assert O.capacity(1.1, 10, 1, 4) == 3          # 2.75 rounds up
+
+
+def test_capacity_drops_later_assignments_first():
+    ids = np.array([[0], [0], [1], [0], [0]])
+    counts, kept, offsets, row_src, inv = O.dispatch_token_choice(ids, 2, cap=2)
+    assert counts.tolist() == [4, 1] and kept.tolist() == [2, 1]
+    assert inv.tolist() == [0, 1, 2, -1, -1]
+    assert row_src.tolist() == [0, 1, 2]
+
+
+# ----------------------------------------------------------- expert FFN ----
+
+def test_swiglu_closed_form_scalar():
+    # D = F = 1: out = w_down * SiLU(w_gate * x) * (w_up * x); SiLU(ln 3) = (3/4) ln 3.
+    x = np.array([[1.0]])
+    out = O.swiglu_expert(x, [[math.log(3.0)]], [[2.0]], [[0.5]])
+    np.testing.assert_allclose(out, [[0.5 * 0.75 * math.log(3.0) * 2.0]], rtol=1e-15)
+    # gate and up are not interchangeable: swapping them changes the result
+    out_sw = O.swiglu_expert(x, [[2.0]], [[math.log(3.0)]], [[0.5]])
+    assert abs(out_sw[0, 0] - out[0, 0]) > 0.1
+    # a zero gate pre-activation closes the gate
+    assert O.swiglu_expert(x, [[0.0]], [[5.0]], [[1.0]])[0, 0] == 0.0
+
+
+def _swiglu_by_loops(xv, Wgate, Wup, Wdown):
+    D, F = len(xv), len(Wgate)
+    h = []
+    for f in range(F):
+        a = sum(Wgate[f][d] * xv[d] for d in range(D))
+        u = sum(Wup[f][d] * xv[d] for d in range(D))
+        h.append(a / (1 + math.exp(-a)) * u)
+    return [sum(Wdown[d][f] * h[f] for f in range(F)) for d in range(D)]
+
+
+def test_single_expert_layer_is_the_dense_ffn():
+    c = cfg(E=1, k=1, T=3)
+    rng = np.random.default_rng(8)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    r = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    for t in range(c["T"]):
+        ref = _swiglu_by_loops(x[t].tolist(), Wgate[0].tolist(), Wup[0].tolist(), Wdown[0].tolist())
+        np.testing.assert_allclose(r["out"][t], ref, rtol=1e-12, atol=1e-14)
+
+
+def test_relu_expert_closed_form():
+    x = np.array([[1.0, -2.0]])
+    Wup = np.array([[1.0, 0.0], [0.0, 1.0], [1.0, 1.0]])      # pre-act [1, -2, -1]
+    Wdown = np.array([[1.0, 1.0, 1.0], [2.0, 0.0, 5.0]])
+    np.testing.assert_allclose(O.relu_expert(x, Wup, Wdown), [[1.0, 2.0]])
+
+
+# -------------------------------------------------------------- combine ----
+
+def test_page_combine_example_accumulates_both_experts():
+    g = gold("tiny_moe_combine_example.json")
+    # ReLU experts with W_up = I, W_down = (e+1) I: E_e(x) = (e+1) x for x > 0.
+    D, E = 3, 4
+    c = cfg(T=1, D=D, E=E, F=D, k=2, act="relu")
+    Wup = np.stack([np.eye(D)] * E)
+    Wdown = np.stack([(e + 1) * np.eye(D) for e in range(E)])
+    x = np.array([[0.5, 1.0, 2.0]])
+    # router probs [0.2, 0.1, 0.6, 0.1]: top-2 = experts 2, 0 -> 0.75, 0.25
+    logits = np.log(np.array([[0.2, 0.1, 0.6, 0.1]]))
+    r = O.layer_forward(c, x, np.zeros((E, D)), None, None, Wup, Wdown, logits=logits)
+    assert r["ids"][0].tolist() == g["experts"]
+    np.testing.assert_allclose(r["gates"][0], g["weights"], rtol=1e-12)
+    expect = sum(w * (e + 1) * x[0] for e, w in zip(g["experts"], g["weights"]))
+    np.testing.assert_allclose(r["out"][0], expect, rtol=1e-12)
+
+
+# ----------------------------------------------------- balance statistics ----
+
+def test_page_imbalance_example():
+    g = gold("moe_comparison_imbalance.json")
+    st = O.balance_stats(np.full((1, 4), 0.25), g["counts"], g["total"], g["total"], 1e-2)
+    assert sum(g["counts"]) == g["total"] and g["total"] / 4 == g["ideal_mean"]
+    assert st["max_over_mean"] == g["max_over_mean"]
+    assert st["n_dropped"] == 0
+
+
+@pytest.mark.parametrize("case", ["case_A", "case_B"])
+def test_page_importance_and_load_cases(case):
+    g = gold("tiny_moe_balance_cases.json")
+    cs = g[case]
+    c = cfg(T=2, E=2, k=1, D=1, F=1, aux_alpha=0.01)
+    r = O.route(c, np.log(np.array(cs["probs"])))
+    assert r["ids"][:, 0].tolist() == cs["routes"]
+    st = r["stats"]
+    np.testing.assert_allclose(st["P"], cs["importance"], rtol=1e-12)
+    np.testing.assert_allclose(st["f"], cs["load"], rtol=1e-12)
+    expect = 0.01 * 2 * sum(p * f for p, f in zip(cs["importance"], cs["load"]))
+    np.testing.assert_allclose(st["aux"], expect, rtol=1e-12)
+    # case A puts both routes on the expert with the larger importance: 1.02 alpha;
+    # case B balances the routes: exactly the reference value 1 * alpha.
+    np.testing.assert_allclose(st["aux"] / 0.01, {"case_A": 1.02, "case_B": 1.0}[case], rtol=1e-12)
+
+
+def test_balanced_reference_value_is_alpha():
+    g = gold("tiny_moe_balance_cases.json")
+    for E in (2, 4, 8):
+        st = O.balance_stats(np.full((5, E), 1.0 / E), [3] * E, 3 * E, 3 * E, 0.01)
+        np.testing.assert_allclose(st["aux"], 0.01 * g["balanced_reference_value"], rtol=1e-12)
+
+
+def test_load_counts_routes_over_tokens_times_k():
+    rng = np.random.default_rng(9)
+    c = cfg(T=50, E=6, k=2)
+    r = O.route(c, rng.standard_normal((50, 6)))
+    np.testing.assert_allclose(r["stats"]["f"].sum(), 1.0, atol=1e-15)
+    np.testing.assert_allclose(r["stats"]["P"].sum(), 1.0, atol=1e-14)
+
+
+# ---------------------------------------------------------- whole layer ----
+
+@pytest.mark.parametrize("score,act,bias", [("softmax", "swiglu", False),
+                                            ("softmax", "relu", False),
+                                            ("sigmoid", "swiglu", True)])
+def test_dropless_equals_dense_masked(score, act, bias):
+    c = cfg(T=12, D=8, E=5, F=7, k=2, score=score, act=act)
+    rng = np.random.default_rng(11)
+    x, Wg, b, Wgate, Wup, Wdown = rand_layer(rng, c, with_bias=bias)
+    r = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown)
+    dense = O.dense_masked_forward(c, x, Wg, b, Wgate, Wup, Wdown)
+    np.testing.assert_allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
+
+
+def test_topk_equal_E_with_renorm_is_soft_routing():
+    c = cfg(T=9, D=5, E=4, F=6, k=4)
+    rng = np.random.default_rng(12)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    r = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    soft = O.soft_routing_forward(c, x, Wg, Wgate, Wup, Wdown)
+    np.testing.assert_allclose(r["out"], soft, rtol=1e-12, atol=1e-13)
+
+
+def test_large_capacity_equals_dropless_and_overflow_rows_are_zero():
+    c = cfg(T=16, D=6, E=4, F=5, k=1, overflow="drop", capacity_factor=100.0, gate="raw")
+    rng = np.random.default_rng(13)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    Wg[0] += 3.0 * x.mean(0)          # make expert 0 popular
+    big = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    free = O.layer_forward(dict(c, overflow="dropless"), x, Wg, None, Wgate, Wup, Wdown)
+    np.testing.assert_allclose(big["out"], free["out"], rtol=1e-13, atol=1e-14)
+    small = O.layer_forward(dict(c, capacity_factor=1.0), x, Wg, None, Wgate, Wup, Wdown)
+    cap = O.capacity(1.0, 16, 1, 4)
+    assert small["cap"] == cap == 4
+    dropped = np.nonzero(small["inv"] < 0)[0]
+    assert len(dropped) == small["stats"]["n_dropped"] > 0
+    for t in dropped:                          # k = 1: assignment id == token id
+        assert np.all(small["out"][t] == 0.0)
+    kept = np.nonzero(small["inv"] >= 0)[0]
+    np.testing.assert_allclose(small["out"][kept], free["out"][kept], rtol=1e-13, atol=1e-14)
+    # the tokens kept by each expert are its earliest ones
+    for e in range(4):
+        toks = [t for t in range(16) if free["ids"][t, 0] == e]
+        assert [t for t in toks if small["inv"][t] >= 0] == toks[:cap]
+
+
+def test_expert_choice_c_equal_T_is_soft_routing_and_unpicked_rows_are_zero():
+    c = cfg(T=6, D=5, E=3, F=4, k=0, c=6, select="expert")
+    rng = np.random.default_rng(14)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    r = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    soft = O.soft_routing_forward(c, x, Wg, Wgate, Wup, Wdown)
+    np.testing.assert_allclose(r["out"], soft, rtol=1e-12, atol=1e-13)
+    c2 = dict(c, c=1)
+    r2 = O.layer_forward(c2, x, Wg, None, Wgate, Wup, Wdown)
+    picked = set(r2["ids"].reshape(-1).tolist())
+    assert r2["counts"].tolist() == [1, 1, 1]
+    for t in range(6):
+        if t not in picked:
+            assert np.all(r2["out"][t] == 0.0)
+    np.testing.assert_allclose(r2["stats"]["f"], [1 / 3] * 3, rtol=1e-15)
+
+
+def test_shared_expert_adds_with_weight_one():
+    c = cfg(T=5, D=4, E=3, F=3, k=1, n_shared=1, F_shared=6)
+    rng = np.random.default_rng(15)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    Sg, Su, Sd = (rng.standard_normal((1, 6, 4)), rng.standard_normal((1, 6, 4)),
+                  rng.standard_normal((1, 4, 6)))
+    r = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown, Sg, Su, Sd)
+    base = O.layer_forward(dict(c, n_shared=0), x, Wg, None, Wgate, Wup, Wdown)
+    for t in range(5):
+        ref = _swiglu_by_loops(x[t].tolist(), Sg[0].tolist(), Su[0].tolist(), Sd[0].tolist())
+        np.testing.assert_allclose(r["out"][t] - base["out"][t], ref, rtol=1e-11, atol=1e-13)
+
+
+@pytest.mark.parametrize("kw", [dict(), dict(overflow="drop", capacity_factor=1.0, k=1, gate="raw"),
+                                dict(select="expert", k=0, c=3),
+                                dict(score="sigmoid", n_shared=1, F_shared=4)])
+def test_sampled_rows_agree_with_full_layer(kw):
+    c = cfg(T=10, D=6, E=4, F=5, **kw)
+    rng = np.random.default_rng(16)
+    x, Wg, b, Wgate, Wup, Wdown = rand_layer(rng, c, with_bias=c["score"] == "sigmoid")
+    S = None
+    if c["n_shared"]:
+        S = (rng.standard_normal((1, 4, 6)), rng.standard_normal((1, 4, 6)),
+             rng.standard_normal((1, 6, 4)))
+    full = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown, *(S or ()))
+    rows = O.layer_forward_rows(c, [0, 3, 7, 9], x, Wg, b, Wgate, Wup, Wdown, *(S or ()))
+    np.testing.assert_allclose(rows["out_rows"], full["out"][[0, 3, 7, 9]], rtol=1e-12, atol=1e-14)
