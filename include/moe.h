@@ -1,0 +1,220 @@
+/*
+ * moe.h -- C ABI of the B200 (sm_100a) sparse Mixture-of-Experts FFN layer, forward pass.
+ *
+ * The layer, as the pages define it (Gate -> Dispatch -> Expert compute -> Combine):
+ *   "Top-k 路由（Top-k Routing）" (compassingai), "Top-k 路由的完整生命週期" and
+ *   "門控函式的數學形式" Steps 1-3;
+ *   "别只比较 Top-k" (ailearn moe-comparison), "评分、Top-k、合并权重和实际执行是四个连续但
+ *   不同的步骤" (Score -> Select -> Merge -> Execute);
+ *   "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡" (f3dlife),
+ *   sections 3-8.
+ *
+ * Conventions shared by every entry point
+ *   - All pointers named as device buffers are device pointers of the current CUDA device;
+ *     the caller allocates and owns them.  The library allocates, frees and synchronises
+ *     nothing (the one exception, moe_get_device_error, says so).  Work is enqueued on the
+ *     given stream and is asynchronous.
+ *   - Tensors are dense row-major.  Weights use the nn.Linear layout [out, in]:
+ *     W_g [E, D]; W_gate, W_up [E, F, D]; W_down [E, D, F]; shared [S, Fs, D] / [S, D, Fs].
+ *   - dtype MOE_BF16: activations and weights are bf16 (fp32 accumulation, bf16 out);
+ *     dtype MOE_F32: everything is fp32.  Router logits, probabilities and gates are fp32.
+ *   - Every device buffer handed in must be 16-byte aligned.
+ *   - Arguments are checked on the host before anything is launched: a bad argument returns
+ *     MOE_ERR_INVALID_ARG, a valid but unimplemented combination MOE_ERR_UNSUPPORTED, a too
+ *     small workspace MOE_ERR_WORKSPACE, a failed launch MOE_ERR_CUDA.  Device-side waits are
+ *     bounded: a wait that gives up records MOE_ERR_TIMEOUT in a device error word, read
+ *     with moe_get_device_error.
+ *   - Limits: 1 <= E <= 256; token choice 1 <= k <= min(E, 32); expert choice 1 <= c <= T;
+ *     T * max(k, E) < 2^31.  bf16: D, F and F_shared multiples of 64.  fp32: D multiple of 4.
+ */
+#ifndef MOE_B200_H
+#define MOE_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* moe_stream_t;   /* same type as cudaStream_t; NULL = legacy default stream */
+
+typedef enum {
+    MOE_OK = 0,
+    MOE_ERR_INVALID_ARG = 1,
+    MOE_ERR_UNSUPPORTED = 2,
+    MOE_ERR_WORKSPACE = 3,
+    MOE_ERR_CUDA = 4,
+    MOE_ERR_TIMEOUT = 5,
+    MOE_ERR_DEVICE = 6
+} moe_status_t;
+
+enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };   /* affinity */
+enum { MOE_TOKEN_CHOICE = 0, MOE_EXPERT_CHOICE = 1 };    /* who selects */
+enum { MOE_GATE_RENORM = 0, MOE_GATE_RAW = 1 };          /* merge weights */
+enum { MOE_DROPLESS = 0, MOE_CAPACITY_DROP = 1 };        /* overflow policy */
+enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU = 1 };           /* expert FFN */
+enum { MOE_F32 = 0, MOE_BF16 = 1 };                      /* operand dtype */
+
+/* Problem statement of one layer call.
+ *   T tokens, D hidden, E routed experts, F expert width;
+ *   k  : token choice, experts per token ("Top-k 路由" gate Step 2);
+ *   c  : expert choice, tokens per expert ("Top-k 路由" Token-Choice vs Expert-Choice table);
+ *   n_shared, F_shared : always-on shared experts (moe-comparison family table, DeepSeek rows);
+ *   score    : softmax over experts, or sigmoid affinity (moe-comparison "Score");
+ *   gate     : RENORM g_j = p_j / sum_sel p (Tiny MoE section 4), RAW g = p (Switch, top-1);
+ *              under sigmoid, RENORM uses the raw affinities, never the selection bias;
+ *   overflow : DROPLESS, or CAPACITY_DROP with C = ceil(capacity_factor * T * k / E) slots per
+ *              expert, evaluated in double ("Top-k 路由" capacity factor formula); the first C
+ *              assignments of an expert in (token, slot) order keep a slot, later ones add 0;
+ *   aux_alpha: alpha of the balance loss alpha * E * sum_e f_e P_e. */
+typedef struct moe_desc {
+    int32_t T, D, E, F;
+    int32_t k;
+    int32_t c;
+    int32_t n_shared, F_shared;
+    int32_t score, select, gate, overflow, act, dtype;
+    float capacity_factor;
+    float aux_alpha;
+} moe_desc_t;
+
+/* Scalars of the balance statistics (written to device memory by moe_balance_stats). */
+typedef struct moe_stats {
+    float aux;             /* alpha * E * sum_e f_e * P_e */
+    float max_over_mean;   /* max_e count_e / mean_e count_e (nominal counts) */
+    int32_t n_routes;      /* T*k (token choice) or E*c (expert choice) */
+    int32_t n_kept;        /* rows the experts execute */
+    int32_t n_dropped;     /* n_routes - n_kept */
+    int32_t reserved;
+} moe_stats_t;
+
+/* Device views into a moe_layer_forward workspace (see moe_layer_views). */
+typedef struct moe_layer_views {
+    int32_t* expert_ids;   /* TC [T,k] expert per slot, descending key; EC [E,c] token ids, ascending */
+    float* gates;          /* TC [T,k] merge weights;  EC [T,E] softmax probabilities */
+    float* logits;         /* [T,E] fp32 router logits */
+    float* importance;     /* [E]   P_e */
+    int32_t* counts;       /* [E]   nominal assignments per expert */
+    int32_t* offsets;      /* [E+1] first row of each expert in the grouped buffers */
+    int32_t* row_src;      /* [A]   assignment id of each row: t*k+j (TC) or t*E+e (EC) */
+    int32_t* inv;          /* TC [T*k], EC [T*E]: row of each assignment, -1 if dropped / not picked */
+    void* x_perm;          /* [A, D]  token rows grouped by expert */
+    void* h;               /* [A, F]  expert hidden activations */
+    void* y;               /* [A, D]  expert outputs, grouped */
+    void* y_shared;        /* [S, T, D] shared expert outputs (NULL when S = 0) */
+    void* h_shared;        /* [T, Fs] shared expert hidden (NULL when S = 0) */
+    int32_t* shared_offsets; /* [2] = {0, T} */
+    float* f;              /* [E] load f_e */
+    moe_stats_t* stats;    /* one moe_stats_t */
+    void* scratch;         /* scratch for the step entry points */
+    size_t scratch_bytes;
+    int64_t rows;          /* A: rows allocated for the grouped buffers */
+} moe_layer_views_t;
+
+/* Human-readable name of a status code (static string). */
+const char* moe_status_string(moe_status_t status);
+
+/* Library version as a static string. */
+const char* moe_version(void);
+
+/* A, the upper bound on rows the experts execute: T*k (dropless), min(T*k, E*C) (capacity
+ * drop), E*c (expert choice).  Grouped buffers (x_perm, h, y, row_src) need A rows. */
+moe_status_t moe_rows_max(const moe_desc_t* desc, int64_t* rows);
+
+/* C, the slots per expert under MOE_CAPACITY_DROP (0 otherwise). */
+moe_status_t moe_capacity(const moe_desc_t* desc, int32_t* capacity);
+
+/* Bytes of scratch that moe_route, moe_permute and moe_balance_stats need. */
+moe_status_t moe_scratch_size(const moe_desc_t* desc, size_t* bytes);
+
+/* Bytes of workspace moe_layer_forward needs (every intermediate plus scratch). */
+moe_status_t moe_workspace_size(const moe_desc_t* desc, size_t* bytes);
+
+/* Carves `ws` (moe_workspace_size bytes, 256-byte aligned) into the views above.  Host only. */
+moe_status_t moe_layer_views(const moe_desc_t* desc, void* ws, size_t ws_bytes,
+                             moe_layer_views_t* views);
+
+/* Score + Select + merge weights.
+ * "Top-k 路由" gate Steps 1-2; Tiny MoE section 4; moe-comparison "Score"/"Select"/"Merge".
+ *   x [T,D], Wg [E,D] (dtype); sel_bias [E] fp32 or NULL (added to sigmoid affinities for
+ *   selection only).
+ *   Token choice: expert_ids [T,k], gates [T,k]; slot j holds the j-th largest key (the logit
+ *   under softmax, sigmoid + bias under sigmoid), ties to the lower expert id.
+ *   Expert choice: expert_ids [E,c] = each expert's c most probable tokens (ties to the lower
+ *   token id) in ascending order; gates [T,E] = softmax probabilities (merge weights).
+ *   logits [T,E] (fp32) and importance [E] (P_e = mean_t of the softmax probabilities, or of
+ *   the sigmoid affinities normalised over experts) are optional (NULL).
+ *   scratch: moe_scratch_size bytes. */
+moe_status_t moe_route(const moe_desc_t* desc, const void* x, const void* Wg,
+                       const float* sel_bias, int32_t* expert_ids, float* gates,
+                       float* logits, float* importance,
+                       void* scratch, size_t scratch_bytes, moe_stream_t stream);
+
+/* Dispatch: counting-sort permutation of assignments into expert-contiguous rows.
+ * Tiny MoE section 5 (torch.where gives, per expert, its (token, slot) pairs in row-major
+ * order); "Top-k 路由" capacity factor; moe-comparison capacity/overflow table.
+ *   counts [E] nominal assignments; offsets [E+1] exclusive scan of kept rows;
+ *   row_src [A] assignment id per row; inv [T*k] (TC) / [T*E] (EC) row per assignment or -1;
+ *   x_perm [A, D] (dtype) rows gathered from x.  Rows of one expert are ordered by (token,
+ *   slot).  All outputs are deterministic.  scratch: moe_scratch_size bytes. */
+moe_status_t moe_permute(const moe_desc_t* desc, const int32_t* expert_ids, const void* x,
+                         void* x_perm, int32_t* counts, int32_t* offsets, int32_t* row_src,
+                         int32_t* inv, void* scratch, size_t scratch_bytes, moe_stream_t stream);
+
+/* Expert compute on grouped rows (Tiny MoE section 3, SwiGLU: down(SiLU(x W_gate^T) * x W_up^T);
+ * ReLU: down(ReLU(x W_up^T))).  Group g owns rows [offsets[g], offsets[g+1]) of `a`
+ * (offsets is a device array of n_groups+1 ints, read on the device).
+ *   a [a_rows, D], h [a_rows, F], y [a_rows, D] (dtype; h, y rows outside the groups are not
+ *   written).  W_gate (NULL for ReLU), W_up [n_groups, F, D], W_down [n_groups, D, F].
+ *   D comes from desc; act and dtype too.  For routed experts: n_groups = E, F = desc->F,
+ *   a = x_perm, a_rows = moe_rows_max.  For a shared expert: n_groups = 1, F = F_shared,
+ *   a = x, a_rows = T, offsets = {0, T}.
+ * moe_expert_up writes h, moe_expert_down reads h and writes y; moe_expert_ffn does both. */
+moe_status_t moe_expert_up(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                           const void* a, int64_t a_rows, const int32_t* offsets,
+                           const void* W_gate, const void* W_up, void* h, moe_stream_t stream);
+moe_status_t moe_expert_down(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                             const void* h, int64_t a_rows, const int32_t* offsets,
+                             const void* W_down, void* y, moe_stream_t stream);
+moe_status_t moe_expert_ffn(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                            const void* a, int64_t a_rows, const int32_t* offsets,
+                            const void* W_gate, const void* W_up, const void* W_down,
+                            void* h, void* y, moe_stream_t stream);
+
+/* Merge: out[t] = sum_j gates[t,j] * y[inv[t,j]] + sum_s y_shared[s,t], fp32 accumulation in
+ * slot order, no atomics; inv = -1 contributes 0.  "Top-k 路由" Combine; Tiny MoE section 6.
+ *   y [A, D] (dtype); inv, gates as produced by moe_permute / moe_route (K = k, or E under
+ *   expert choice); y_shared [n_shared, T, D] or NULL; out [T, D] (dtype). */
+moe_status_t moe_combine(const moe_desc_t* desc, const void* y, const int32_t* inv,
+                         const float* gates, const void* y_shared, void* out,
+                         moe_stream_t stream);
+
+/* Balance statistics ("Top-k 路由" load-balancing loss; Tiny MoE section 8; moe-comparison
+ * [9,4,2,1] imbalance example): f_e = counts_e / n_routes, aux = alpha * E * sum f_e P_e,
+ * max/mean of counts, kept and dropped routes.  counts [E] and offsets [E+1] from
+ * moe_permute, importance [E] from moe_route; f [E] and one moe_stats_t are written. */
+moe_status_t moe_balance_stats(const moe_desc_t* desc, const int32_t* counts,
+                               const int32_t* offsets, const float* importance, float* f,
+                               moe_stats_t* stats, moe_stream_t stream);
+
+/* The whole layer: route -> permute -> expert_ffn (+ shared experts) -> combine -> stats,
+ * enqueued on one stream with no host synchronisation.  Intermediates live in `ws`
+ * (moe_workspace_size bytes); moe_layer_views gives their addresses.
+ *   x [T,D], Wg [E,D], sel_bias [E] or NULL, routed weights as above, shared weights
+ *   [S,Fs,D], [S,Fs,D], [S,D,Fs] (NULL when S = 0), out [T,D]. */
+moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void* Wg,
+                               const float* sel_bias, const void* W_gate, const void* W_up,
+                               const void* W_down, const void* Ws_gate, const void* Ws_up,
+                               const void* Ws_down, void* out, void* ws, size_t ws_bytes,
+                               moe_stream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that kernels set when
+ * a bounded wait gives up (MOE_ERR_TIMEOUT) or a device-side check fires (MOE_ERR_DEVICE).
+ * *code receives the raw word (0 = none).  Returns MOE_OK when the word was 0. */
+moe_status_t moe_get_device_error(moe_stream_t stream, int32_t* code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H */

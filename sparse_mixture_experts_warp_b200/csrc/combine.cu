@@ -1,0 +1,161 @@
+// Combine (unpermute + weighted sum) and the balance statistics.
+//
+// Combine: "Top-k 路由（Top-k Routing）" (compassingai), Combine box (output = sum of
+// gate_score_i * y_i over the selected experts) and "門控函式的數學形式" Step 3;
+// "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡" (f3dlife), section 6
+// (contributions are accumulated, never assigned).  Each output row is produced by one warp
+// that walks the token's assignments in slot order through the inverse permutation, so the
+// sum has a fixed order and needs no atomics; a dropped or unpicked assignment (row -1) adds
+// nothing.  Shared experts ("别只比较 Top-k" family table, DeepSeek rows) add with weight 1.
+//
+// Statistics: "Top-k 路由" load-balancing loss L = alpha * N * sum_i f_i P_i; Tiny MoE section 8
+// (importance before top-k, load after top-k; E * sum p_e f_e = 1 at balance); "别只比较
+// Top-k" section "先数 assignments" (max/mean imbalance, [9,4,2,1] -> 2.25).
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kWarps = 8;
+constexpr int kMaxList = 256;      // assignments per token held in shared memory (K <= 256)
+
+template <bool BF16> struct Row;
+template <> struct Row<true> {     // 8 bf16 per 16 bytes
+  static constexpr int N = 8;
+  __device__ __forceinline__ static void acc(const uint4* p, float g, float* a) {
+    const uint4 u = __ldcs(p);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      a[2 * i] = fmaf(g, __uint_as_float(w[i] << 16), a[2 * i]);
+      a[2 * i + 1] = fmaf(g, __uint_as_float(w[i] & 0xffff0000u), a[2 * i + 1]);
+    }
+  }
+  __device__ __forceinline__ static void store(uint4* p, const float* a) {
+    uint32_t w[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      __nv_bfloat162 h = __floats2bfloat162_rn(a[2 * i], a[2 * i + 1]);
+      w[i] = *reinterpret_cast<uint32_t*>(&h);
+    }
+    *p = make_uint4(w[0], w[1], w[2], w[3]);
+  }
+};
+template <> struct Row<false> {    // 4 fp32 per 16 bytes
+  static constexpr int N = 4;
+  __device__ __forceinline__ static void acc(const uint4* p, float g, float* a) {
+    const float4 f = __ldcs(reinterpret_cast<const float4*>(p));
+    a[0] = fmaf(g, f.x, a[0]); a[1] = fmaf(g, f.y, a[1]);
+    a[2] = fmaf(g, f.z, a[2]); a[3] = fmaf(g, f.w, a[3]);
+  }
+  __device__ __forceinline__ static void store(uint4* p, const float* a) {
+    *reinterpret_cast<float4*>(p) = make_float4(a[0], a[1], a[2], a[3]);
+  }
+};
+
+template <bool BF16>
+__global__ void __launch_bounds__(kWarps * 32)
+combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
+               const float* __restrict__ gates, const uint4* __restrict__ ys, int S, int T,
+               int K, int nvec, uint4* __restrict__ out) {
+  using R = Row<BF16>;
+  __shared__ int s_row[kWarps][kMaxList];
+  __shared__ float s_g[kWarps][kMaxList];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + warp;
+  if (t >= T) return;
+  // Compact the token's live assignments, keeping slot order.
+  int n = 0;
+  for (int j0 = 0; j0 < K; j0 += 32) {
+    const int j = j0 + lane;
+    const int r = (j < K) ? inv[(int64_t)t * K + j] : -1;
+    const float g = (j < K && r >= 0) ? gates[(int64_t)t * K + j] : 0.f;
+    const unsigned live = __ballot_sync(0xffffffffu, r >= 0);
+    if (r >= 0) {
+      const int pos = n + __popc(live & ((1u << lane) - 1u));
+      s_row[warp][pos] = r;
+      s_g[warp][pos] = g;
+    }
+    n += __popc(live);
+  }
+  __syncwarp();
+  for (int v = lane; v < nvec; v += 32) {
+    float a[R::N];
+#pragma unroll
+    for (int i = 0; i < R::N; ++i) a[i] = 0.f;
+    for (int q = 0; q < n; ++q) R::acc(y + (int64_t)s_row[warp][q] * nvec + v, s_g[warp][q], a);
+    for (int s = 0; s < S; ++s) R::acc(ys + ((int64_t)s * T + t) * nvec + v, 1.0f, a);
+    R::store(out + (int64_t)t * nvec + v, a);
+  }
+}
+
+__global__ void __launch_bounds__(256)
+stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance, int E,
+             int n_routes, float alpha, float* f, moe_stats_t* st) {
+  __shared__ float s_fp[256];
+  __shared__ int s_max[256];
+  const int e = threadIdx.x;
+  float fp = 0.f;
+  int c = 0;
+  if (e < E) {
+    c = counts[e];
+    const float fe = (float)c / (float)n_routes;
+    f[e] = fe;
+    fp = fe * importance[e];
+  }
+  s_fp[e] = fp;
+  s_max[e] = c;
+  __syncthreads();
+  for (int h = 128; h > 0; h >>= 1) {       // fixed-order tree
+    if (e < h) {
+      s_fp[e] += s_fp[e + h];
+      s_max[e] = max(s_max[e], s_max[e + h]);
+    }
+    __syncthreads();
+  }
+  if (e == 0) {
+    const int kept = offsets[E];
+    moe_stats_t r;
+    r.aux = alpha * (float)E * s_fp[0];
+    const float mean = (float)n_routes / (float)E;
+    r.max_over_mean = mean > 0.f ? (float)s_max[0] / mean : 0.f;
+    r.n_routes = n_routes;
+    r.n_kept = kept;
+    r.n_dropped = n_routes - kept;
+    r.reserved = 0;
+    *st = r;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
+                           const float* gates, const void* y_shared, void* out,
+                           cudaStream_t s) {
+  if (d.T == 0) return cudaSuccess;
+  const int K = (d.select == MOE_EXPERT_CHOICE) ? d.E : d.k;
+  const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
+  const int nvec = d.D * esz / 16;
+  const int S = y_shared ? d.n_shared : 0;
+  const int blocks = (d.T + kWarps - 1) / kWarps;
+  if (d.dtype == MOE_BF16)
+    combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
+        K, nvec, static_cast<uint4*>(out));
+  else
+    combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(
+        static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
+        K, nvec, static_cast<uint4*>(out));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
+                                 const int32_t* offsets, const float* importance, float* f,
+                                 moe_stats_t* stats, cudaStream_t s) {
+  const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
+  stats_kernel<<<1, 256, 0, s>>>(counts, offsets, importance, d.E, n_routes, d.aux_alpha, f,
+                                 stats);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,75 @@
+// Shared device/host helpers of the sm_100a MoE library (no layer arithmetic here).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "moe.h"
+
+namespace moe {
+
+// Device error codes written into the library's device error word.
+enum : int {
+  DEVERR_NONE = 0,
+  DEVERR_TIMEOUT_TMA = 0x101,     // producer gave up waiting for a free stage
+  DEVERR_TIMEOUT_MMA = 0x102,     // MMA issuer gave up waiting for operands / accumulator
+  DEVERR_TIMEOUT_EPI = 0x103,     // epilogue gave up waiting for an accumulator
+  DEVERR_BOUNDS = 0x201,          // a device-side bounds check fired
+};
+
+// Address of the library's device error word on the current device.
+int* device_error_word();
+
+inline bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
+
+// route.cu
+cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
+                                       const float* bias, int32_t* ids, float* gates,
+                                       float* logits, float* imp_partials, int n_partials,
+                                       cudaStream_t s);
+cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
+                                        float* probs, float* probsT, float* logits,
+                                        float* imp_partials, int n_partials, cudaStream_t s);
+cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
+                             cudaStream_t s);
+cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
+                                     float* importance, cudaStream_t s);
+int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer
+
+// permute.cu
+int permute_blocks(const moe_desc_t& d);
+cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids, const void* x,
+                                        void* x_perm, int32_t* counts, int32_t* offsets,
+                                        int32_t* row_src, int32_t* inv, int32_t* block_hist,
+                                        int32_t cap, cudaStream_t s);
+cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* picked,
+                                         const void* x, void* x_perm, int32_t* counts,
+                                         int32_t* offsets, int32_t* row_src, int32_t* inv,
+                                         cudaStream_t s);
+
+// gemm_sm100.cu (bf16 grouped GEMM on tcgen05)
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2 };
+cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
+                                     const void* B0, const void* B1, int n_groups, int N,
+                                     const int32_t* offsets, void* out, cudaStream_t s);
+
+// ffn_simt.cu (fp32 experts)
+cudaError_t launch_ffn_up_f32(int act, const float* a, int64_t a_rows, int D, int F,
+                              const int32_t* offsets, int n_groups, const float* Wgate,
+                              const float* Wup, float* h, cudaStream_t s);
+cudaError_t launch_ffn_down_f32(const float* h, int64_t a_rows, int D, int F,
+                                const int32_t* offsets, int n_groups, const float* Wdown,
+                                float* y, cudaStream_t s);
+
+// combine.cu
+cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
+                           const float* gates, const void* y_shared, void* out,
+                           cudaStream_t s);
+cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
+                                 const int32_t* offsets, const float* importance, float* f,
+                                 moe_stats_t* stats, cudaStream_t s);
+
+}  // namespace moe

@@ -1,0 +1,535 @@
+// Grouped GEMM for the experts' projections on 5th-generation tensor cores (sm_100a).
+//
+// "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡" (f3dlife), section 3
+// (SwiGLU expert: hidden = SiLU(x W_gate) * (x W_up), output = hidden W_down) and sections 5/12
+// (production systems replace the per-expert loop by token permutation + grouped GEMM);
+// "别只比较 Top-k" (ailearn moe-comparison), Execute step (experts run as a Grouped GEMM).
+//
+// out[r, n] = epi( sum_k A[r, k] * B[g*N + n, k] ) for every row r of group g, where group g owns
+// rows [offsets[g], offsets[g+1]) of A.  A is [rows, K] bf16 row-major, B is the stacked
+// nn.Linear weights [G*N, K] bf16 row-major (both K-major operands), accumulation is fp32 in
+// tensor memory, out is bf16 [rows, N].
+//   EPI_SWIGLU: B0 = W_gate, B1 = W_up; one 128x256 MMA tile holds 128 gate columns and the
+//               same 128 up columns side by side in TMEM; out = SiLU(gate) * up.
+//   EPI_RELU:   out = max(acc, 0) with B0 = W_up.
+//   EPI_NONE:   out = acc with B0 = W_down.
+//
+// Design (one persistent CTA per SM, 192 threads, warp-specialised):
+//   warp 0 (one thread)  TMA producer: 128-byte-swizzled K-major boxes of A (128 x 64) and
+//                        B (2 x 128 x 64) into a 4-stage shared-memory ring, mbarrier
+//                        complete_tx; no multicast.
+//   warp 1 (one thread)  MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256 K=16,
+//                        fp32 accumulator in TMEM; tcgen05.commit frees ring stages and hands
+//                        finished accumulators to the epilogue.  Warp 1 also owns the TMEM
+//                        allocation (512 columns = two 256-column accumulators, so the epilogue
+//                        of tile i overlaps the main loop of tile i+1).
+//   warps 2-5            epilogue: tcgen05.ld 32x32b (warp w reads TMEM lanes 32*(w%4)..+31,
+//                        one output row per thread), activation, bf16 pack, 16-byte stores of
+//                        the rows that belong to the group (rows past the group end are
+//                        computed from neighbouring rows and discarded).
+// Tiles are enumerated group by group, n-tile by n-tile, with the m-tiles innermost, so the
+// CTAs that run at the same time share B tiles through L2 and each weight byte streams from
+// HBM about once.  The per-group row counts are read on the device (no host sync).
+// Every mbarrier wait is bounded (globaltimer); a wait that gives up records an error code in
+// the device error word and makes the CTA drain its in-flight copies and MMAs and exit.
+#include <cuda.h>
+#include <mutex>
+
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int BK = 64;                      // 64 bf16 = 128 bytes = one swizzle-atom row
+constexpr int MMA_N = 256;
+constexpr int MMA_K = 16;
+constexpr int STAGES = 4;
+constexpr int A_BYTES = BM * BK * 2;        // 16 KB
+constexpr int B_BYTES = MMA_N * BK * 2;     // 32 KB
+constexpr int ACC_COLS = MMA_N;             // fp32 accumulator columns per tile
+constexpr int TMEM_COLS = 2 * ACC_COLS;     // two accumulators
+constexpr int THREADS = 192;
+constexpr uint64_t TIMEOUT_NS = 2000000000ull;   // 2 s per wait
+constexpr uint64_t DRAIN_NS = 200000000ull;      // 0.2 s to drain after an abort
+
+// Instruction descriptor, kind::f16: D fp32 (bits 4-5 = 1), A bf16 (bits 7-9 = 1), B bf16
+// (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at 24-28.
+constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
+                            ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+struct GemmParams {
+  const int32_t* offsets;   // [G+1] device
+  __nv_bfloat16* out;       // [rows, N]
+  int* err;                 // device error word
+  int64_t rows;             // rows allocated in A and out
+  int64_t ldo;              // out row pitch (elements)
+  int G, N, K;
+  int n_out_tile;           // output columns per tile
+  int nt;                   // n-tiles per group
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+__device__ __forceinline__ uint64_t gtimer() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)),
+               "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+// Bounded wait for the phase of parity `parity` to complete.  Returns false when it gave up
+// (time limit, or another role already aborted).
+__device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                       int* err, int code, uint64_t limit) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const uint64_t t0 = gtimer();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort_flag) return false;
+    if (gtimer() - t0 > limit) {
+      *abort_flag = 1;
+      atomicCAS(err, 0, code);
+      return false;
+    }
+  }
+  return true;
+}
+
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
+__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);        // start address
+  d |= (uint64_t)1 << 16;                           // leading byte offset (unused here), 16 B
+  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)1 << 46;                           // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;                           // 128-byte swizzle
+  return d;
+}
+
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(kIdesc), "r"(acc));
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+  asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+  asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]),
+        "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]),
+        "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]),
+        "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]),
+        "=r"(r[31])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_wait_ld() {
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int EPI>
+__global__ void __launch_bounds__(THREADS, 1)
+grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB0,
+                    const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + STAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + STAGES;
+  uint64_t* tfull = bars + 2 * STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* grp_off = reinterpret_cast<int*>(tmem_holder + 2);   // [G+1]
+  int* tile_pre = grp_off + (p.G + 1);                      // [G+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&tfull[a], 1);
+      mbar_init(&tempty[a], 4 * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB0)) : "memory");
+    if (EPI == EPI_SWIGLU)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB1)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  if (warp == 2) {
+    // group row starts and the tile prefix (tiles of group g = ceil(rows_g / BM) * nt)
+    int carry = 0;
+    if (lane == 0) {
+      grp_off[0] = p.offsets[0];
+      tile_pre[0] = 0;
+    }
+    for (int g0 = 0; g0 < p.G; g0 += 32) {
+      const int g = g0 + lane;
+      int tiles = 0;
+      if (g < p.G) {
+        const int lo = p.offsets[g], hi = p.offsets[g + 1];
+        const int m = hi > lo ? hi - lo : 0;
+        tiles = ((m + BM - 1) / BM) * p.nt;
+        grp_off[g + 1] = hi;
+      }
+      int inc = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (g < p.G) tile_pre[g + 1] = carry + inc;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = tile_pre[p.G];
+  const int nkb = (p.K + BK - 1) / BK;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;     // per stage: has a load, parity of the last one
+      bool ok = true;
+      int g = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        while (tile >= tile_pre[g + 1]) ++g;
+        const int m = grp_off[g + 1] - grp_off[g];
+        const int mt = (m + BM - 1) / BM;
+        const int local = tile - tile_pre[g];
+        const int n_idx = local / mt, m_idx = local - n_idx * mt;
+        const int a_row = grp_off[g] + m_idx * BM;
+        const int b_row = g * p.N + n_idx * p.n_out_tile;
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
+                         TIMEOUT_NS)) {
+            ok = false;
+            break;
+          }
+          mbar_expect_tx(&full[stage], A_BYTES + B_BYTES);
+          const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, a_row);
+          if (EPI == EPI_SWIGLU) {
+            tma_load_2d(b_dst, &tmB0, &full[stage], kb * BK, b_row);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB1, &full[stage], kb * BK, b_row);
+          } else {
+            tma_load_2d(b_dst, &tmB0, &full[stage], kb * BK, b_row);
+            tma_load_2d(b_dst + B_BYTES / 2, &tmB0, &full[stage], kb * BK, b_row + 128);
+          }
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let the copies already in flight land before the CTA exits
+        for (int s = 0; s < STAGES; ++s)
+          if (issued & (1u << s))
+            mbar_wait(&full[s], (issued_par >> s) & 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
+                      DRAIN_NS);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ---------------- MMA issuer ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
+                       TIMEOUT_NS)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
+                         TIMEOUT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < BK / MMA_K; ++k) {
+            umma_bf16(d_tmem, sdesc_sw128(a0 + k * MMA_K * 2), sdesc_sw128(b0 + k * MMA_K * 2),
+                      (kb > 0 || k > 0) ? 1u : 0u);
+          }
+          umma_commit(&empty[stage]);       // frees the stage once these MMAs have read it
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit(&tfull[acc]);   // accumulator ready for the epilogue
+      }
+      // all MMAs issued by this thread complete before the CTA releases TMEM
+      umma_commit(drain);
+      mbar_wait(drain, 0u, abort_flag, p.err, DEVERR_TIMEOUT_MMA, ok ? TIMEOUT_NS : DRAIN_NS);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..5) ----------------
+    const int q = warp & 3;                  // TMEM lane quarter this warp may access
+    const int row = q * 32 + lane;
+    int g = 0, it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      while (tile >= tile_pre[g + 1]) ++g;
+      const int m = grp_off[g + 1] - grp_off[g];
+      const int mt = (m + BM - 1) / BM;
+      const int local = tile - tile_pre[g];
+      const int n_idx = local / mt, m_idx = local - n_idx * mt;
+      const int acc = it & 1;
+      const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
+      int okw = 1;
+      if (lane == 0)
+        okw = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err, DEVERR_TIMEOUT_EPI, TIMEOUT_NS);
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      tc_fence_after();
+      const int r = m_idx * BM + row;
+      const int64_t orow = (int64_t)grp_off[g] + r;
+      bool valid = r < m;
+      if (valid && (orow < 0 || orow >= p.rows)) {
+        atomicCAS(p.err, 0, DEVERR_BOUNDS);
+        valid = false;
+      }
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+      __nv_bfloat16* orow_ptr = p.out + orow * p.ldo + (int64_t)n_idx * p.n_out_tile;
+      if (EPI == EPI_SWIGLU) {
+#pragma unroll 1
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t gv[32], uv[32];
+          tmem_ld32(taddr + c, gv);
+          tmem_ld32(taddr + 128 + c, uv);
+          tmem_wait_ld();
+          const int col = n_idx * p.n_out_tile + c;
+          if (valid && col < p.N) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+              const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
+              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              pk[i] = pack_bf16(h0, h1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < MMA_N; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          const int col = n_idx * p.n_out_tile + c;
+          if (valid && col < p.N) {
+            uint32_t pk[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+              if (EPI == EPI_RELU) {
+                a0 = fmaxf(a0, 0.f);
+                a1 = fmaxf(a1, 0.f);
+              }
+              pk[i] = pack_bf16(a0, a1);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c);
+            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&tempty[acc]);
+    }
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------- host side ----------------
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2D bf16 tensor [rows, cols] row-major; box = 64 columns x box_rows rows, 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+template <int EPI>
+cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                       const GemmParams& p, int grid, size_t smem, cudaStream_t s) {
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  grouped_gemm_kernel<EPI><<<grid, THREADS, smem, s>>>(a, b0, b1, p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
+                                     const void* B0, const void* B1, int n_groups, int N,
+                                     const int32_t* offsets, void* out, cudaStream_t s) {
+  if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb0, tb1;
+  const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&tb0, B0, brows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+  if (epi == EPI_SWIGLU) {
+    if (!make_map(&tb1, B1, brows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
+  } else {
+    tb1 = tb0;
+  }
+  GemmParams p;
+  p.offsets = offsets;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  p.rows = a_rows;
+  p.ldo = N;
+  p.G = n_groups;
+  p.N = N;
+  p.K = K;
+  p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
+  p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
+  const int64_t max_tiles = ((a_rows + BM - 1) / BM + n_groups) * (int64_t)p.nt;
+  const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
+  const size_t smem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (2 * STAGES + 5) * 8 + 8 +
+                      (size_t)2 * (n_groups + 1) * sizeof(int);
+  switch (epi) {
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb0, tb1, p, grid, smem, s);
+    case EPI_RELU: return launch_epi<EPI_RELU>(ta, tb0, tb1, p, grid, smem, s);
+    default: return launch_epi<EPI_NONE>(ta, tb0, tb1, p, grid, smem, s);
+  }
+}
+
+}  // namespace moe

@@ -1,0 +1,401 @@
+// C ABI of the sm_100a sparse MoE FFN layer: argument validation, workspace carving and the
+// launch chain.  The layer follows "Top-k 路由（Top-k Routing）" (compassingai), lifecycle
+// Gate -> Dispatch -> Expert compute -> Combine, and "别只比较 Top-k" (ailearn
+// moe-comparison), Score -> Select -> Merge -> Execute.  No entry point allocates, frees or
+// synchronises (moe_get_device_error excepted); all work goes on the caller's stream.
+#include <math.h>
+#include <string.h>
+
+#include "common.cuh"
+
+namespace moe {
+
+static __device__ int g_device_error = 0;
+
+int* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+namespace {
+
+constexpr size_t kAlign = 256;
+inline size_t up(size_t v) { return (v + kAlign - 1) / kAlign * kAlign; }
+
+moe_status_t validate(const moe_desc_t* d) {
+  if (!d) return MOE_ERR_INVALID_ARG;
+  if (d->T < 0 || d->D <= 0 || d->E <= 0 || d->F <= 0) return MOE_ERR_INVALID_ARG;
+  if (d->score != MOE_SCORE_SOFTMAX && d->score != MOE_SCORE_SIGMOID) return MOE_ERR_INVALID_ARG;
+  if (d->select != MOE_TOKEN_CHOICE && d->select != MOE_EXPERT_CHOICE) return MOE_ERR_INVALID_ARG;
+  if (d->gate != MOE_GATE_RENORM && d->gate != MOE_GATE_RAW) return MOE_ERR_INVALID_ARG;
+  if (d->overflow != MOE_DROPLESS && d->overflow != MOE_CAPACITY_DROP) return MOE_ERR_INVALID_ARG;
+  if (d->act != MOE_ACT_SWIGLU && d->act != MOE_ACT_RELU) return MOE_ERR_INVALID_ARG;
+  if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
+  if (d->n_shared < 0 || (d->n_shared > 0 && d->F_shared <= 0)) return MOE_ERR_INVALID_ARG;
+  if (d->E > 256) return MOE_ERR_UNSUPPORTED;
+  if (d->select == MOE_TOKEN_CHOICE) {
+    if (d->k < 1 || d->k > d->E) return MOE_ERR_INVALID_ARG;
+    if (d->k > 32) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)d->T * d->k >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+    if (d->overflow == MOE_CAPACITY_DROP && !(d->capacity_factor > 0.f)) return MOE_ERR_INVALID_ARG;
+  } else {
+    if (d->c < 1 || d->c > d->T) return MOE_ERR_INVALID_ARG;
+    if (d->score != MOE_SCORE_SOFTMAX) return MOE_ERR_UNSUPPORTED;
+    if (d->overflow != MOE_DROPLESS) return MOE_ERR_UNSUPPORTED;
+    if ((int64_t)d->T * d->E >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
+  }
+  if (!(d->aux_alpha >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_BF16) {
+    if (d->D % 64 || d->F % 64) return MOE_ERR_UNSUPPORTED;
+    if (d->n_shared > 0 && d->F_shared % 64) return MOE_ERR_UNSUPPORTED;
+  } else {
+    if (d->D % 4) return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_OK;
+}
+
+int32_t capacity_of(const moe_desc_t* d) {
+  if (d->select != MOE_TOKEN_CHOICE || d->overflow != MOE_CAPACITY_DROP) return 0;
+  const double c = ceil((double)d->capacity_factor * (double)d->T * (double)d->k / (double)d->E);
+  return (int32_t)c;
+}
+
+int64_t rows_of(const moe_desc_t* d) {
+  if (d->select == MOE_EXPERT_CHOICE) return (int64_t)d->E * d->c;
+  const int64_t A = (int64_t)d->T * d->k;
+  if (d->overflow == MOE_CAPACITY_DROP) {
+    const int64_t cap = (int64_t)d->E * capacity_of(d);
+    return cap < A ? cap : A;
+  }
+  return A;
+}
+
+size_t esize(const moe_desc_t* d) { return d->dtype == MOE_BF16 ? 2 : 4; }
+
+size_t route_scratch(const moe_desc_t* d) {
+  size_t b = up((size_t)router_partials(*d) * d->E * sizeof(float));
+  if (d->select == MOE_EXPERT_CHOICE) b += up((size_t)d->E * d->T * sizeof(float));
+  return b;
+}
+size_t permute_scratch(const moe_desc_t* d) {
+  if (d->select == MOE_EXPERT_CHOICE) return 0;
+  return up((size_t)(permute_blocks(*d) > 0 ? permute_blocks(*d) : 1) * d->E * sizeof(int32_t));
+}
+size_t scratch_bytes(const moe_desc_t* d) {
+  const size_t a = route_scratch(d), b = permute_scratch(d);
+  return (a > b ? a : b) + kAlign;
+}
+
+// Workspace layout of moe_layer_forward; with base == nullptr only the size is computed.
+size_t carve(const moe_desc_t* d, uint8_t* base, moe_layer_views_t* v) {
+  const int64_t T = d->T, E = d->E, A = rows_of(d);
+  const bool ec = d->select == MOE_EXPERT_CHOICE;
+  const int64_t K = ec ? E : d->k;
+  const size_t es = esize(d);
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = base ? base + off : nullptr;
+    off += up(bytes ? bytes : 1);
+    return p;
+  };
+  moe_layer_views_t w;
+  memset(&w, 0, sizeof(w));
+  w.logits = static_cast<float*>(take(T * E * 4));
+  w.expert_ids = static_cast<int32_t*>(take((ec ? E * d->c : T * K) * 4));
+  w.gates = static_cast<float*>(take(T * K * 4));
+  w.importance = static_cast<float*>(take(E * 4));
+  w.counts = static_cast<int32_t*>(take(E * 4));
+  w.offsets = static_cast<int32_t*>(take((E + 1) * 4));
+  w.row_src = static_cast<int32_t*>(take(A * 4));
+  w.inv = static_cast<int32_t*>(take(T * K * 4));
+  w.x_perm = take(A * d->D * es);
+  w.h = take(A * d->F * es);
+  w.y = take(A * d->D * es);
+  if (d->n_shared > 0) {
+    w.h_shared = take(T * d->F_shared * es);
+    w.y_shared = take((int64_t)d->n_shared * T * d->D * es);
+    w.shared_offsets = static_cast<int32_t*>(take(2 * 4));
+  }
+  w.f = static_cast<float*>(take(E * 4));
+  w.stats = static_cast<moe_stats_t*>(take(sizeof(moe_stats_t)));
+  const size_t sb = scratch_bytes(d);
+  w.scratch = take(sb);
+  w.scratch_bytes = sb;
+  w.rows = A;
+  if (v) *v = w;
+  return off;
+}
+
+inline moe_status_t cuda_status(cudaError_t e) {
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+__global__ void set_offsets_kernel(int32_t* o, int T) {
+  o[0] = 0;
+  o[1] = T;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(moe_status_t s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "unsupported configuration";
+    case MOE_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case MOE_ERR_CUDA: return "CUDA launch error";
+    case MOE_ERR_TIMEOUT: return "device wait timed out";
+    case MOE_ERR_DEVICE: return "device-side check failed";
+  }
+  return "unknown status";
+}
+
+const char* moe_version(void) { return "moe-b200 0.1 (sm_100a)"; }
+
+moe_status_t moe_rows_max(const moe_desc_t* d, int64_t* rows) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!rows) return MOE_ERR_INVALID_ARG;
+  *rows = rows_of(d);
+  return MOE_OK;
+}
+
+moe_status_t moe_capacity(const moe_desc_t* d, int32_t* c) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!c) return MOE_ERR_INVALID_ARG;
+  *c = capacity_of(d);
+  return MOE_OK;
+}
+
+moe_status_t moe_scratch_size(const moe_desc_t* d, size_t* bytes) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = scratch_bytes(d);
+  return MOE_OK;
+}
+
+moe_status_t moe_workspace_size(const moe_desc_t* d, size_t* bytes) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  *bytes = carve(d, nullptr, nullptr);
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_views(const moe_desc_t* d, void* ws, size_t ws_bytes,
+                             moe_layer_views_t* v) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!ws || !v) return MOE_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < carve(d, nullptr, nullptr)) return MOE_ERR_WORKSPACE;
+  carve(d, static_cast<uint8_t*>(ws), v);
+  return MOE_OK;
+}
+
+moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const float* sel_bias,
+                       int32_t* expert_ids, float* gates, float* logits, float* importance,
+                       void* scratch, size_t scratch_bytes_, moe_stream_t stream) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (d->T == 0) return MOE_OK;
+  if (!x || !Wg || !expert_ids || !gates || !scratch) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(x) || !is_aligned16(Wg)) return MOE_ERR_INVALID_ARG;
+  if (scratch_bytes_ < scratch_bytes(d)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* sc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(scratch) + kAlign - 1) &
+                                           ~(uintptr_t)(kAlign - 1));
+  float* partials = reinterpret_cast<float*>(sc);
+  const int np = router_partials(*d);
+  cudaError_t e;
+  if (d->select == MOE_TOKEN_CHOICE) {
+    e = launch_router_token_choice(*d, x, Wg, d->score == MOE_SCORE_SIGMOID ? sel_bias : nullptr,
+                                   expert_ids, gates, logits, partials, np, s);
+  } else {
+    float* probsT = reinterpret_cast<float*>(sc + up((size_t)np * d->E * sizeof(float)));
+    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, np, s);
+    if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
+  }
+  if (e == cudaSuccess && importance)
+    e = launch_importance_reduce(partials, np, d->E, d->T, importance, s);
+  return cuda_status(e);
+}
+
+moe_status_t moe_permute(const moe_desc_t* d, const int32_t* expert_ids, const void* x,
+                         void* x_perm, int32_t* counts, int32_t* offsets, int32_t* row_src,
+                         int32_t* inv, void* scratch, size_t scratch_bytes_,
+                         moe_stream_t stream) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!expert_ids || !x || !x_perm || !counts || !offsets || !row_src || !inv)
+    return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(x) || !is_aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d->select == MOE_TOKEN_CHOICE) {
+    if (!scratch || scratch_bytes_ < scratch_bytes(d)) return MOE_ERR_WORKSPACE;
+    int32_t* hist = reinterpret_cast<int32_t*>(
+        (reinterpret_cast<uintptr_t>(scratch) + kAlign - 1) & ~(uintptr_t)(kAlign - 1));
+    e = launch_permute_token_choice(*d, expert_ids, x, x_perm, counts, offsets, row_src, inv,
+                                    hist, capacity_of(d), s);
+  } else {
+    e = launch_permute_expert_choice(*d, expert_ids, x, x_perm, counts, offsets, row_src, inv, s);
+  }
+  return cuda_status(e);
+}
+
+static moe_status_t check_ffn(const moe_desc_t* d, int32_t G, int32_t F, const void* a,
+                              int64_t a_rows, const int32_t* offsets) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (G < 1 || G > 1024 || F <= 0 || a_rows < 0 || !a || !offsets) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(a)) return MOE_ERR_INVALID_ARG;
+  if (d->dtype == MOE_BF16 && (F % 64)) return MOE_ERR_UNSUPPORTED;
+  if (a_rows >= ((int64_t)1 << 31)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+moe_status_t moe_expert_up(const moe_desc_t* d, int32_t G, int32_t F, const void* a,
+                           int64_t a_rows, const int32_t* offsets, const void* W_gate,
+                           const void* W_up, void* h, moe_stream_t stream) {
+  moe_status_t st = check_ffn(d, G, F, a, a_rows, offsets);
+  if (st != MOE_OK) return st;
+  if (!W_up || !h || (d->act == MOE_ACT_SWIGLU && !W_gate)) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(W_up) || !is_aligned16(h) || (W_gate && !is_aligned16(W_gate)))
+    return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d->dtype == MOE_BF16) {
+    if (d->act == MOE_ACT_SWIGLU)
+      e = launch_grouped_gemm_bf16(EPI_SWIGLU, a, a_rows, d->D, W_gate, W_up, G, F, offsets, h, s);
+    else
+      e = launch_grouped_gemm_bf16(EPI_RELU, a, a_rows, d->D, W_up, nullptr, G, F, offsets, h, s);
+  } else {
+    e = launch_ffn_up_f32(d->act, static_cast<const float*>(a), a_rows, d->D, F, offsets, G,
+                          static_cast<const float*>(W_gate), static_cast<const float*>(W_up),
+                          static_cast<float*>(h), s);
+  }
+  return cuda_status(e);
+}
+
+moe_status_t moe_expert_down(const moe_desc_t* d, int32_t G, int32_t F, const void* h,
+                             int64_t a_rows, const int32_t* offsets, const void* W_down, void* y,
+                             moe_stream_t stream) {
+  moe_status_t st = check_ffn(d, G, F, h, a_rows, offsets);
+  if (st != MOE_OK) return st;
+  if (!W_down || !y) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(W_down) || !is_aligned16(y)) return MOE_ERR_INVALID_ARG;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e;
+  if (d->dtype == MOE_BF16)
+    e = launch_grouped_gemm_bf16(EPI_NONE, h, a_rows, F, W_down, nullptr, G, d->D, offsets, y, s);
+  else
+    e = launch_ffn_down_f32(static_cast<const float*>(h), a_rows, d->D, F, offsets, G,
+                            static_cast<const float*>(W_down), static_cast<float*>(y), s);
+  return cuda_status(e);
+}
+
+moe_status_t moe_expert_ffn(const moe_desc_t* d, int32_t G, int32_t F, const void* a,
+                            int64_t a_rows, const int32_t* offsets, const void* W_gate,
+                            const void* W_up, const void* W_down, void* h, void* y,
+                            moe_stream_t stream) {
+  moe_status_t st = moe_expert_up(d, G, F, a, a_rows, offsets, W_gate, W_up, h, stream);
+  if (st != MOE_OK) return st;
+  return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
+}
+
+moe_status_t moe_combine(const moe_desc_t* d, const void* y, const int32_t* inv,
+                         const float* gates, const void* y_shared, void* out,
+                         moe_stream_t stream) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!y || !inv || !gates || !out) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(y) || !is_aligned16(out) || (y_shared && !is_aligned16(y_shared)))
+    return MOE_ERR_INVALID_ARG;
+  if (y_shared && d->n_shared == 0) return MOE_ERR_INVALID_ARG;
+  return cuda_status(launch_combine(*d, y, inv, gates, y_shared, out,
+                                    reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_balance_stats(const moe_desc_t* d, const int32_t* counts, const int32_t* offsets,
+                               const float* importance, float* f, moe_stats_t* stats,
+                               moe_stream_t stream) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!counts || !offsets || !importance || !f || !stats) return MOE_ERR_INVALID_ARG;
+  if (d->select == MOE_TOKEN_CHOICE ? d->T * d->k == 0 : d->E * d->c == 0) return MOE_OK;
+  return cuda_status(launch_balance_stats(*d, counts, offsets, importance, f, stats,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* Wg,
+                               const float* sel_bias, const void* W_gate, const void* W_up,
+                               const void* W_down, const void* Ws_gate, const void* Ws_up,
+                               const void* Ws_down, void* out, void* ws, size_t ws_bytes,
+                               moe_stream_t stream) {
+  moe_layer_views_t v;
+  moe_status_t st = moe_layer_views(d, ws, ws_bytes, &v);
+  if (st != MOE_OK) return st;
+  if (!x || !Wg || !W_up || !W_down || !out) return MOE_ERR_INVALID_ARG;
+  if (d->act == MOE_ACT_SWIGLU && !W_gate) return MOE_ERR_INVALID_ARG;
+  if (d->n_shared > 0 && (!Ws_gate || !Ws_up || !Ws_down)) return MOE_ERR_INVALID_ARG;
+  if (d->T == 0) return MOE_OK;
+  st = moe_route(d, x, Wg, sel_bias, v.expert_ids, v.gates, v.logits, v.importance, v.scratch,
+                 v.scratch_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_permute(d, v.expert_ids, x, v.x_perm, v.counts, v.offsets, v.row_src, v.inv,
+                   v.scratch, v.scratch_bytes, stream);
+  if (st != MOE_OK) return st;
+  st = moe_expert_ffn(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, W_down, v.h, v.y,
+                      stream);
+  if (st != MOE_OK) return st;
+  if (d->n_shared > 0) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    set_offsets_kernel<<<1, 1, 0, s>>>(v.shared_offsets, d->T);
+    if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
+    // shared experts always use SwiGLU
+    moe_desc_t ds = *d;
+    ds.act = MOE_ACT_SWIGLU;
+    const size_t es = esize(d);
+    const int64_t wstride_up = (int64_t)d->F_shared * d->D * es;
+    for (int i = 0; i < d->n_shared; ++i) {
+      const uint8_t* gw = static_cast<const uint8_t*>(Ws_gate) + i * wstride_up;
+      const uint8_t* uw = static_cast<const uint8_t*>(Ws_up) + i * wstride_up;
+      const uint8_t* dw = static_cast<const uint8_t*>(Ws_down) + i * wstride_up;
+      uint8_t* ys = static_cast<uint8_t*>(v.y_shared) + (int64_t)i * d->T * d->D * es;
+      st = moe_expert_ffn(&ds, 1, d->F_shared, x, d->T, v.shared_offsets, gw, uw, dw, v.h_shared,
+                          ys, stream);
+      if (st != MOE_OK) return st;
+    }
+  }
+  st = moe_combine(d, v.y, v.inv, v.gates, d->n_shared > 0 ? v.y_shared : nullptr, out, stream);
+  if (st != MOE_OK) return st;
+  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.f, v.stats, stream);
+}
+
+moe_status_t moe_get_device_error(moe_stream_t stream, int32_t* code) {
+  int* w = device_error_word();
+  if (!w) return MOE_ERR_CUDA;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess)
+    return MOE_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return MOE_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+      return MOE_ERR_CUDA;
+  }
+  if (code) *code = v;
+  if (v == 0) return MOE_OK;
+  return (v >= 0x100 && v < 0x200) ? MOE_ERR_TIMEOUT : MOE_ERR_DEVICE;
+}
+
+}  // extern "C"

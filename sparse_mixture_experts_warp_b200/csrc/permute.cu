@@ -1,0 +1,266 @@
+// Dispatch: a counting-sort permutation of (token, slot) assignments into expert-contiguous
+// rows, with an optional capacity clamp, and the gather of token rows into that order.
+//
+// "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡" (f3dlife),
+// section 5 (torch.where lists, per expert, its (token, route slot) pairs in row-major order);
+// "Top-k 路由（Top-k Routing）" (compassingai), capacity factor (expert buffer = CF * T/N * k);
+// "别只比较 Top-k" (ailearn moe-comparison), capacity + overflow row of the balance table
+// (an overflowing token skips the expert).
+//
+// Token choice, A = T*k assignments a = t*k + j, processed in blocks of kBlockItems:
+//   1. hist:   per block, per expert assignment counts                    -> block_hist[blk][E]
+//   2. scan:   per expert, exclusive scan over blocks (block bases) and total counts; kept =
+//              min(count, C); offsets = exclusive scan of kept over experts
+//   3. rank:   per block, the stable rank of each assignment within its expert, from
+//              __match_any_sync peer groups inside a warp, per-warp counts in shared memory and
+//              the block base -- no atomics decide any order; row = offsets[e] + rank, kept
+//              when rank < C
+//   4. gather: one warp per token reads x[t] once (16-byte loads) and writes it to each of its
+//              kept rows.
+// Expert choice: row e*c + i is the i-th picked token of expert e (already in token order).
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kThreads = 256;                // 8 warps
+constexpr int kChunksPerWarp = 4;            // 32 assignments per chunk
+constexpr int kBlockItems = kThreads * kChunksPerWarp;   // 1024 assignments per block
+constexpr int kWarpsPerBlock = kThreads / 32;
+
+__global__ void __launch_bounds__(kThreads)
+perm_hist_kernel(const int32_t* ids, int A, int E, int32_t* block_hist) {
+  extern __shared__ int s_hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
+  __syncthreads();
+  const int base = blockIdx.x * kBlockItems;
+  for (int i = threadIdx.x; i < kBlockItems; i += blockDim.x) {
+    const int a = base + i;
+    if (a < A) {
+      const int e = ids[a];
+      if (e >= 0 && e < E) atomicAdd(&s_hist[e], 1);   // counting only: order-free
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) block_hist[(int64_t)blockIdx.x * E + e] = s_hist[e];
+}
+
+// One block; thread e walks the blocks of expert e; then an exclusive scan over experts.
+__global__ void __launch_bounds__(1024)
+perm_scan_kernel(int32_t* block_hist, int nblk, int E, int cap, int32_t* counts,
+                 int32_t* offsets) {
+  __shared__ int s_warp[32];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E) {
+    for (int b = 0; b < nblk; ++b) {
+      const int v = block_hist[(int64_t)b * E + e];
+      block_hist[(int64_t)b * E + e] = total;    // becomes the block base of expert e
+      total += v;
+    }
+    counts[e] = total;
+  }
+  const int kept = (e < E) ? ((cap > 0 && total > cap) ? cap : total) : 0;
+  // exclusive scan of kept over experts
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int inc = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = (lane < nw) ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += n;
+    }
+    if (lane < nw) s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int before = (warp > 0) ? s_warp[warp - 1] : 0;
+  if (e < E) offsets[e] = before + inc - kept;
+  if (e == E - 1) offsets[E] = before + inc;
+}
+
+__global__ void __launch_bounds__(kThreads)
+perm_rank_kernel(const int32_t* ids, int A, int E, int cap, const int32_t* block_base,
+                 const int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  extern __shared__ int s_mem[];
+  int* s_cnt = s_mem;                             // [warps][E] per-warp counts, then bases
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kWarpsPerBlock * E; i += blockDim.x) s_cnt[i] = 0;
+  __syncthreads();
+  const int wbase = blockIdx.x * kBlockItems + warp * (32 * kChunksPerWarp);
+  int* my = s_cnt + warp * E;
+  const unsigned lt = (1u << lane) - 1u;
+  // pass 1: per-warp counts per expert
+  for (int ch = 0; ch < kChunksPerWarp; ++ch) {
+    const int a = wbase + ch * 32 + lane;
+    const int e = (a < A) ? ids[a] : -1;
+    const bool ok = (e >= 0 && e < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    if (ok && (peers & lt) == 0) my[e] += __popc(peers);   // leader of the peer group
+    __syncwarp();
+  }
+  __syncthreads();
+  // per expert: exclusive scan over warps, plus the block base
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int run = block_base[(int64_t)blockIdx.x * E + e];
+    for (int w = 0; w < kWarpsPerBlock; ++w) {
+      const int v = s_cnt[w * E + e];
+      s_cnt[w * E + e] = run;
+      run += v;
+    }
+  }
+  __syncthreads();
+  // pass 2: ranks
+  for (int ch = 0; ch < kChunksPerWarp; ++ch) {
+    const int a = wbase + ch * 32 + lane;
+    const int e = (a < A) ? ids[a] : -1;
+    const bool ok = (e >= 0 && e < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    int rank = 0;
+    if (ok) rank = my[e] + __popc(peers & lt);
+    __syncwarp();
+    if (ok && (peers & lt) == 0) my[e] += __popc(peers);
+    __syncwarp();
+    if (a < A) {
+      int row = -1;
+      if (ok && (cap <= 0 || rank < cap)) {
+        row = offsets[e] + rank;
+        row_src[row] = a;
+      }
+      inv[a] = row;
+    }
+  }
+}
+
+// One warp per token: copy x[t] (D elements of `esz` bytes) to each kept row.
+__global__ void __launch_bounds__(256)
+gather_tc_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_t* inv,
+                 uint4* __restrict__ xp) {
+  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (warp >= T) return;
+  int rows[8];
+  int nr = 0;
+  for (int j = 0; j < k && j < 8; ++j) {
+    const int r = inv[(int64_t)warp * k + j];
+    rows[j] = r;
+    nr = j + 1;
+  }
+  const uint4* src = x + (int64_t)warp * nvec;
+  int v = lane;
+  for (; v + 96 < nvec; v += 128) {
+    const uint4 a0 = __ldcs(src + v), a1 = __ldcs(src + v + 32), a2 = __ldcs(src + v + 64),
+                a3 = __ldcs(src + v + 96);
+    for (int j = 0; j < nr; ++j) {
+      if (rows[j] < 0) continue;
+      uint4* dst = xp + (int64_t)rows[j] * nvec;
+      dst[v] = a0; dst[v + 32] = a1; dst[v + 64] = a2; dst[v + 96] = a3;
+    }
+  }
+  for (; v < nvec; v += 32) {
+    const uint4 a0 = __ldcs(src + v);
+    for (int j = 0; j < nr; ++j) {
+      if (rows[j] < 0) continue;
+      xp[(int64_t)rows[j] * nvec + v] = a0;
+    }
+  }
+  // k > 8: remaining slots (not used by the shipped workloads, kept correct)
+  for (int j = 8; j < k; ++j) {
+    const int r = inv[(int64_t)warp * k + j];
+    if (r < 0) continue;
+    for (int u = lane; u < nvec; u += 32) xp[(int64_t)r * nvec + u] = src[u];
+  }
+}
+
+// Expert choice: row r = e*c + i takes token picked[r]; inv[t*E + e] = r.
+__global__ void ec_fill_kernel(int32_t* inv, int64_t n) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) inv[i] = -1;
+}
+
+__global__ void ec_index_kernel(const int32_t* picked, int E, int c, int T, int32_t* counts,
+                                int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  const int r = blockIdx.x * blockDim.x + threadIdx.x;
+  if (r <= E) {
+    offsets[r] = r * c;
+    if (r < E) counts[r] = c;
+  }
+  if (r < E * c) {
+    const int e = r / c;
+    const int t = picked[r];
+    if (t >= 0 && t < T) {
+      row_src[r] = t * E + e;
+      inv[(int64_t)t * E + e] = r;
+    } else {
+      row_src[r] = -1;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256)
+gather_rows_kernel(const uint4* __restrict__ x, int T, int nvec, const int32_t* picked, int rows,
+                   uint4* __restrict__ xp) {
+  const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+  if (r >= rows) return;
+  const int t = picked[r];
+  if (t < 0 || t >= T) return;
+  const uint4* src = x + (int64_t)t * nvec;
+  uint4* dst = xp + (int64_t)r * nvec;
+  for (int v = lane; v < nvec; v += 32) dst[v] = __ldg(src + v);
+}
+
+}  // namespace
+
+int permute_blocks(const moe_desc_t& d) {
+  const int64_t A = (int64_t)d.T * d.k;
+  return (int)((A + kBlockItems - 1) / kBlockItems);
+}
+
+cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids, const void* x,
+                                        void* x_perm, int32_t* counts, int32_t* offsets,
+                                        int32_t* row_src, int32_t* inv, int32_t* block_hist,
+                                        int32_t cap, cudaStream_t s) {
+  const int A = d.T * d.k;
+  const int nblk = permute_blocks(d);
+  const int E = d.E;
+  if (nblk > 0) {
+    perm_hist_kernel<<<nblk, kThreads, E * sizeof(int), s>>>(ids, A, E, block_hist);
+  }
+  perm_scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
+  if (nblk > 0) {
+    perm_rank_kernel<<<nblk, kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
+        ids, A, E, cap, block_hist, offsets, row_src, inv);
+    const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
+    const int nvec = d.D * esz / 16;
+    const int blocks = (d.T * 32 + 255) / 256;
+    gather_tc_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
+                                            static_cast<uint4*>(x_perm));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* picked,
+                                         const void* x, void* x_perm, int32_t* counts,
+                                         int32_t* offsets, int32_t* row_src, int32_t* inv,
+                                         cudaStream_t s) {
+  const int64_t n = (int64_t)d.T * d.E;
+  if (n > 0) ec_fill_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(inv, n);
+  const int rows = d.E * d.c;
+  const int m = (rows > d.E + 1 ? rows : d.E + 1);
+  ec_index_kernel<<<(m + 255) / 256, 256, 0, s>>>(picked, d.E, d.c, d.T, counts, offsets,
+                                                  row_src, inv);
+  const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
+  const int nvec = d.D * esz / 16;
+  if (rows > 0)
+    gather_rows_kernel<<<(rows * 32 + 255) / 256, 256, 0, s>>>(
+        static_cast<const uint4*>(x), d.T, nvec, picked, rows, static_cast<uint4*>(x_perm));
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,159 @@
+"""Helpers of the GPU parity tests: run the CUDA layer through the C ABI and compare it with
+the CPU oracle on the same seeded inputs.
+
+Tolerances (from the layer's arithmetic):
+  * routing (expert ids, counts, offsets, row order, inverse permutation, dropped sets) is
+    compared bit-exactly, the oracle routing from the GPU's own fp32 logits;
+  * router logits: per token max_e |gpu - oracle| / max_e |oracle| <= 1e-5 (fp32 accumulation
+    of exact bf16/fp32 products over D terms);
+  * gates / probabilities: relative 1e-5 (fp32 exp and division);
+  * layer output: max |gpu - oracle| / max |oracle| over the compared rows <= 2e-2 for bf16
+    operands (bf16 rounding of h, y and out, each 2^-9 relative), <= 1e-5 for fp32; rows the
+    method zeroes (dropped or unpicked tokens) must be exactly zero.
+"""
+
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import sparse_mixture_experts_warp_b200 as M
+from sparse_mixture_experts_warp_b200.workloads import make_inputs
+from oracle import moe_oracle as O
+
+TOL_OUT = {"bf16": 2e-2, "f32": 1e-5}
+TOL_LOGITS = 1e-5
+TOL_GATES = 1e-5
+
+
+def key_fn_for(w):
+    if w.select == "expert":
+        return lambda x, Wg, b: O.softmax_probs_of(x, Wg)
+    return lambda x, Wg, b: O.routing_keys(x, Wg, b, w.score)
+
+
+def inputs_for(w, seed=0, device="cuda"):
+    if w.select == "expert":
+        return make_inputs(w, seed, device, key_fn=key_fn_for(w), ec_gap=1e-6)
+    return make_inputs(w, seed, device, key_fn=key_fn_for(w), key_gap=1e-3)
+
+
+def np64(t):
+    if t is None:
+        return None
+    return t.detach().float().cpu().double().numpy()
+
+
+def run_layer(w, inp):
+    d = M.desc_of(w)
+    ws = M.empty_workspace(d, inp.x.device)
+    out = torch.empty_like(inp.x)
+    M.moe_layer_forward(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                        inp.Ws_gate, inp.Ws_up, inp.Ws_down, out, ws)
+    torch.cuda.synchronize()
+    err = M.get_device_error()
+    assert err == 0, f"device error word {err:#x}"
+    return out, M.layer_views(d, ws)
+
+
+def max_rel(a, b):
+    den = np.max(np.abs(b))
+    if den == 0:
+        return float(np.max(np.abs(a)))
+    return float(np.max(np.abs(a - b)) / den)
+
+
+def check_logits(w, inp, v, rows=None):
+    """GPU fp32 logits against the oracle's fp64 router product (optionally sampled rows)."""
+    x = np64(inp.x) if rows is None else np64(inp.x[torch.as_tensor(rows, device=inp.x.device)])
+    ref = O.router_logits(x, np64(inp.Wg))
+    got = v["logits"].double().cpu().numpy()
+    if rows is not None:
+        got = got[rows]
+    den = np.maximum(np.abs(ref).max(axis=1), 1e-30)
+    err = (np.abs(got - ref).max(axis=1) / den).max()
+    assert err <= TOL_LOGITS, f"router logits max rel err {err:.3e}"
+    return err
+
+
+def wdict(w):
+    return dict(T=w.T, D=w.D, E=w.E, F=w.F, k=w.k, c=w.c, score=w.score, select=w.select,
+                gate=w.gate, overflow=w.overflow, capacity_factor=w.capacity_factor, act=w.act,
+                n_shared=w.n_shared, F_shared=w.F_shared, aux_alpha=w.aux_alpha)
+
+
+def check_routing(w, inp, v):
+    """Routing, permutation and statistics bit-exact / within fp32 rounding, with the oracle
+    routing from the GPU's fp32 logits."""
+    logits = v["logits"].double().cpu().numpy()
+    ref = O.route(wdict(w), logits, np64(inp.bias))
+    ids = v["expert_ids"].cpu().numpy()
+    np.testing.assert_array_equal(ids, ref["ids"])
+    counts = v["counts"].cpu().numpy()
+    offsets = v["offsets"].cpu().numpy()
+    np.testing.assert_array_equal(counts, ref["counts"])
+    np.testing.assert_array_equal(offsets, ref["offsets"])
+    n = int(offsets[-1])
+    np.testing.assert_array_equal(v["row_src"].cpu().numpy()[:n], ref["row_src"])
+    np.testing.assert_array_equal(v["inv"].cpu().numpy().reshape(-1), ref["inv"])
+    gates = v["gates"].double().cpu().numpy()
+    np.testing.assert_allclose(gates, np.asarray(ref["gates"]).reshape(gates.shape),
+                               rtol=TOL_GATES, atol=1e-7)
+    # gathered rows are exact copies of their tokens
+    K = ref["K"]
+    if n:
+        src_tok = torch.as_tensor(ref["row_src"] // K, device=inp.x.device, dtype=torch.long)
+        assert torch.equal(v["x_perm"][:n], inp.x[src_tok])
+    st = ref["stats"]
+    np.testing.assert_allclose(v["importance"].double().cpu().numpy(), st["P"], rtol=1e-5,
+                               atol=1e-7)
+    np.testing.assert_allclose(v["f"].double().cpu().numpy(), st["f"], rtol=1e-6, atol=1e-9)
+    s = M.stats_of(v["stats"])
+    np.testing.assert_allclose(s["aux"], st["aux"], rtol=1e-5)
+    np.testing.assert_allclose(s["max_over_mean"], st["max_over_mean"], rtol=1e-6)
+    assert s["n_dropped"] == st["n_dropped"]
+    assert s["n_kept"] == int(ref["kept"].sum())
+    return ref
+
+
+def check_full_output(w, inp, out, ref_route):
+    """Whole-layer output against the oracle's fp64 evaluation (all rows)."""
+    r = O.layer_forward(wdict(w), np64(inp.x), np64(inp.Wg), np64(inp.bias), np64(inp.W_gate),
+                        np64(inp.W_up), np64(inp.W_down), np64(inp.Ws_gate), np64(inp.Ws_up),
+                        np64(inp.Ws_down), logits=None)
+    # the oracle routed from its own logits: gaps in the inputs make that routing identical
+    np.testing.assert_array_equal(r["ids"], ref_route["ids"])
+    got = out.double().cpu().numpy()
+    err = max_rel(got, r["out"])
+    assert err <= TOL_OUT[w.dtype], f"layer output max rel err {err:.3e}"
+    zero_rows = np.nonzero(np.all(r["out"] == 0.0, axis=1))[0]
+    assert np.all(got[zero_rows] == 0.0)
+    return err
+
+
+def expert_weights_streamer(inp):
+    """weights_of(e) for the oracle: one expert's weights copied to the host as fp64."""
+    def weights_of(e):
+        g = np64(inp.W_gate[e]) if inp.W_gate is not None else None
+        return g, np64(inp.W_up[e]), np64(inp.W_down[e])
+    return weights_of
+
+
+def check_sampled_output(w, inp, out, v, tokens):
+    """Sampled output rows at full size: oracle routes the whole batch from the GPU's logits
+    and evaluates only the sampled tokens' experts."""
+    logits = v["logits"].double().cpu().numpy()
+    tk = torch.as_tensor(tokens, device=inp.x.device, dtype=torch.long)
+    x_rows = np.zeros((w.T, w.D))
+    x_rows[tokens] = np64(inp.x[tk])
+    r = O.layer_forward_rows(wdict(w), tokens, x_rows, None, np64(inp.bias), None, None, None,
+                             np64(inp.Ws_gate), np64(inp.Ws_up), np64(inp.Ws_down),
+                             logits=logits, weights_of=expert_weights_streamer(inp))
+    got = out[tk].double().cpu().numpy()
+    ref = r["out_rows"]
+    err = max_rel(got, ref)
+    assert err <= TOL_OUT[w.dtype], f"sampled output max rel err {err:.3e}"
+    for i in range(len(tokens)):
+        if np.all(ref[i] == 0.0):
+            assert np.all(got[i] == 0.0)
+    return err

@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI (no GPU): the library loads, exports every function
+include/moe.h declares, sizes the grouped buffers and workspace, and rejects bad arguments
+before anything is launched."""
+
+import ctypes
+import math
+
+import pytest
+
+import sparse_mixture_experts_warp_b200 as M
+from sparse_mixture_experts_warp_b200.build import build
+from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, capacity_of, rows_max
+
+
+@pytest.fixture(scope="module", autouse=True)
+def built():
+    build()
+
+
+def test_library_exports_every_declared_function():
+    L = M.lib()
+    names = M.header_functions()
+    assert len(names) >= 15
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.moe_version().decode().startswith("moe-b200")
+
+
+def test_status_strings():
+    assert M.status_string(0) == "ok"
+    assert "invalid" in M.status_string(1)
+    assert "unsupported" in M.status_string(2)
+    assert "timed out" in M.status_string(5)
+
+
+@pytest.mark.parametrize("name", sorted(WORKLOADS))
+def test_rows_capacity_workspace(name):
+    w = WORKLOADS[name]
+    d = M.desc_of(w)
+    assert M.rows_max(d) == rows_max(w)
+    assert M.capacity(d) == capacity_of(w)
+    ws = M.workspace_size(d)
+    es = 2 if w.dtype == "bf16" else 4
+    A = rows_max(w)
+    # at least x_perm + h + y
+    assert ws >= A * (2 * w.D + w.F) * es
+    assert M.scratch_size(d) > 0
+
+
+def test_switch_capacity_is_80():
+    d = M.desc_of(WORKLOADS["switch"])
+    assert M.capacity(d) == 80 == math.ceil(1.25 * 8192 / 128)
+    assert M.rows_max(d) == min(8192, 128 * 80)
+
+
+def _bad(**kw):
+    d = M.desc_of(WORKLOADS["mixtral"])
+    for k, v in kw.items():
+        setattr(d, k, v)
+    return d
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(k=0), 1), (dict(k=9), 1), (dict(D=0), 1), (dict(E=0), 1), (dict(T=-1), 1),
+    (dict(score=7), 1), (dict(dtype=3), 1), (dict(E=300, k=2), 2), (dict(D=4100), 2),
+    (dict(F=100), 2), (dict(overflow=1, capacity_factor=0.0), 1),
+    (dict(select=1, c=0), 1), (dict(select=1, c=5000), 1), (dict(select=1, c=8, score=1), 2),
+])
+def test_invalid_descriptors_are_rejected(kw, status):
+    v = ctypes.c_size_t()
+    assert M.lib().moe_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == status
+
+
+def test_null_pointers_rejected_before_launch():
+    d = M.desc_of(WORKLOADS["mixtral"])
+    L = M.lib()
+    st = L.moe_route(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    st = L.moe_permute(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None)
+    assert st == 1
+    st = L.moe_combine(ctypes.byref(d), None, None, None, None, None, None)
+    assert st == 1
+    st = L.moe_expert_ffn(ctypes.byref(d), 8, 14336, None, 8192, None, None, None, None, None,
+                          None, None)
+    assert st == 1
+    # misaligned pointers are refused too
+    st = L.moe_combine(ctypes.byref(d), 0x1001, 0x2000, 0x3000, None, 0x4000, None)
+    assert st == 1
+
+
+def test_workspace_too_small_or_misaligned():
+    d = M.desc_of(WORKLOADS["tiny"])
+    need = M.workspace_size(d)
+    v = M.MoeLayerViews()
+    L = M.lib()
+    assert L.moe_layer_views(ctypes.byref(d), 0x10000, need - 1, ctypes.byref(v)) == 3
+    assert L.moe_layer_views(ctypes.byref(d), 0x10010, need, ctypes.byref(v)) == 3
+    assert L.moe_layer_views(ctypes.byref(d), 0x10000, need, ctypes.byref(v)) == 0
+    # views are laid out inside the workspace, 256-byte aligned, in range
+    ptrs = [v.logits, v.expert_ids, v.gates, v.importance, v.counts, v.offsets, v.row_src,
+            v.inv, v.x_perm, v.h, v.y, v.f, v.stats, v.scratch]
+    for p in ptrs:
+        assert 0x10000 <= p < 0x10000 + need and p % 256 == 0
+    assert len(set(ptrs)) == len(ptrs)
+    assert v.rows == 128
+
+
+def test_header_entry_points_cite_the_pages():
+    text = open(M.HEADER).read()
+    for title in ("Top-k 路由", "Tiny MoE", "moe-comparison"):
+        assert title in text
