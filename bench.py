@@ -1,0 +1,509 @@
+"""Throughput of the sparse MoE FFN layer forward pass on B200 (one JSON line on rank 0).
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl cuda|reference]
+
+A step is one pass of the whole layer -- route, permute, expert up (gate/up + SiLU*up),
+expert down, combine, balance statistics -- over one batch of synthetic tokens of the
+Mixtral-8x7B layer shape (T=4096, D=4096, E=8, top-2, SwiGLU F=14336, bf16), with inputs and
+weights resident in HBM.  The step calls the library's step entry points in the order
+moe_layer_forward chains them, with CUDA events between them for the per-kernel times.
+`e2e` times the public moe_layer_forward call with the step's tokens copied in from pinned
+host memory and the layer output copied back, every step.
+
+Multi-GPU: the layer does not shard (one GPU, no collectives); `--gpus N` under torchrun runs
+N independent replicas, one per GPU, each on its own batch; value = all ranks' tokens / the
+slowest rank's time (weak scaling).
+
+`--impl reference` times the CPU oracle (fp64) on the host cores on bounded samples of the
+same workload: each step routes the whole batch and evaluates a sample of its tokens.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, make_inputs, scaled  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at Mixtral-8x7B shape; % of tensor-core / HBM roofline"
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_traffic.json")
+GEMM_SRC = os.path.join(ROOT, "sparse_mixture_experts_warp_b200", "csrc", "gemm_sm100.cu")
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+STAGES = ["route", "permute", "expert_up", "expert_down", "combine", "stats"]
+
+
+# ------------------------------------------------------------------ helpers ----
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def load_peaks():
+    try:
+        with open(PEAKS_FILE) as f:
+            p = json.load(f)
+        return ({k: float(p[k]) for k in ("hbm_gbs", "bf16_tflops", "bf16_tflops_sustained")},
+                "measured")
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def file_sha(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def load_traffic(workload):
+    """DRAM bytes per launch of the gate/up grouped GEMM from a committed ncu capture; null
+    once the kernel source has changed since the capture."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            t = json.load(f)
+        if t.get("kernel_sha") != file_sha(GEMM_SRC):
+            return None
+        return t.get("bytes_per_launch", {}).get(workload)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """Samples the SM clock and clock-event reasons of one GPU in a thread (NVML, 20 ms)."""
+
+    REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
+               0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
+
+    def __init__(self, index):
+        self.index = index
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.error = None
+
+    def __enter__(self):
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self._nvml = pynvml
+            self._h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self._h, pynvml.NVML_CLOCK_SM)
+        except Exception as e:  # pragma: no cover - no NVML
+            self.error = str(e)
+            return self
+        self._thread = threading.Thread(target=self._run, daemon=True)
+        self._thread.start()
+        return self
+
+    def _run(self):
+        p = self._nvml
+        get_reasons = getattr(p, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(p, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append(p.nvmlDeviceGetClockInfo(self._h, p.NVML_CLOCK_SM))
+                r = get_reasons(self._h)
+                for bit, name in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(name)
+            except Exception as e:  # pragma: no cover
+                self.error = str(e)
+            self._stop.wait(0.02)
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self._thread:
+            self._thread.join()
+
+    def summary(self):
+        med = statistics.median(self.samples) if self.samples else None
+        out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+               "samples": len(self.samples)}
+        if self.error:
+            out["error"] = self.error
+        return out
+
+    def rejected(self):
+        if self.reasons & {"hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown"}:
+            return True
+        s = self.summary()
+        if s["sm_mhz"] and s["sm_max_mhz"] and not self.reasons:
+            return s["sm_mhz"] < 0.7 * s["sm_max_mhz"]        # a leftover clock lock
+        return False
+
+
+def launches_per_step(w):
+    """Kernels the library launches per layer step (its own kernels only)."""
+    n = 2 + (1 if w.select == "expert" else 0)            # router, importance reduce, ec select
+    n += 3 if w.select == "expert" else 4                  # permute
+    n += 2                                                 # grouped GEMM up + down
+    n += (1 + 2 * w.n_shared) if w.n_shared else 0         # shared experts (+ offsets kernel)
+    n += 2                                                 # combine, stats
+    return n
+
+
+def stage_work(w, rows_exec):
+    """Algorithmic bytes (HBM-bound stages) or FLOPs (GEMMs) per launch; rows_exec = A_exec."""
+    es = 2 if w.dtype == "bf16" else 4
+    T, D, E, F = w.T, w.D, w.E, w.F
+    K = w.E if w.select == "expert" else w.k
+    A = rows_exec
+    n_up = 2 if w.act == "swiglu" else 1
+    return {
+        # x and W_g read once; logits, ids and gates written
+        "route": ("hbm", T * D * es + E * D * es + T * E * 4 + T * K * 8),
+        # ids read; x read once; x_perm written; row_src and inv written
+        "permute": ("hbm", T * K * 4 + T * D * es + A * D * es + A * 4 + T * K * 4),
+        "expert_up": ("tensor", 2.0 * A * D * F * n_up),
+        "expert_down": ("tensor", 2.0 * A * F * D),
+        # expert rows read once; out written once; inv and gates read
+        "combine": ("hbm", A * D * es + T * D * es + T * K * 8),
+        "stats": ("hbm", E * 16),
+    }
+
+
+def workload_of(args):
+    w = WORKLOADS[args.workload]
+    if args.tokens:
+        w = scaled(w, T=args.tokens)
+    return w
+
+
+# -------------------------------------------------------------- CUDA arm ----
+
+def run_cuda(args, rank, world, local):
+    import torch.distributed as dist
+    import sparse_mixture_experts_warp_b200 as M
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    w = workload_of(args)
+    if w.n_shared:
+        raise SystemExit("the step benchmark covers workloads without shared experts")
+    inp = make_inputs(w, seed=rank, device=dev)
+    d = M.desc_of(w)
+    ws = M.empty_workspace(d, dev)
+    v = M.layer_views(d, ws)
+    scratch = v["scratch"]
+    out = torch.empty_like(inp.x)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(ev=None):
+        M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
+                    v["importance"], scratch, stream)
+        if ev is not None:
+            ev[1].record(stream)
+        M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
+                      v["row_src"], v["inv"], scratch, stream)
+        if ev is not None:
+            ev[2].record(stream)
+        M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
+                        stream)
+        if ev is not None:
+            ev[3].record(stream)
+        M.moe_expert_down(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], stream)
+        if ev is not None:
+            ev[4].record(stream)
+        M.moe_combine(d, v["y"], v["inv"], v["gates"], None, out, stream)
+        if ev is not None:
+            ev[5].record(stream)
+        M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
+                            stream)
+        if ev is not None:
+            ev[6].record(stream)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    nvml_index = local if "CUDA_VISIBLE_DEVICES" not in os.environ else \
+        int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
+
+    def timed():
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)]
+               for _ in range(args.steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier()
+        torch.cuda.synchronize(dev)
+        with ClockSampler(nvml_index) as clk:
+            start.record(stream)
+            for i in range(args.steps):
+                evs[i][0].record(stream)
+                step(evs[i])
+            end.record(stream)
+            torch.cuda.synchronize(dev)
+        barrier()
+        total = start.elapsed_time(end)
+        per_stage = {s: 0.0 for s in STAGES}
+        for i in range(args.steps):
+            for j, s in enumerate(STAGES):
+                per_stage[s] += evs[i][j].elapsed_time(evs[i][j + 1])
+        return total, {s: per_stage[s] / args.steps for s in STAGES}, clk
+
+    total_ms, per_stage, clk = timed()
+    remeasured = False
+    if clk.rejected():
+        total_ms, per_stage, clk = timed()
+        remeasured = True
+    total_ms = max_over_ranks(total_ms)
+    ms_per_step = total_ms / args.steps
+    value = w.T * world * args.steps / (total_ms / 1e3)
+
+    # e2e: the public call with host buffers, copies inside the timed region
+    x_host = inp.x.cpu().pin_memory()
+    out_host = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    x_dev = torch.empty_like(inp.x)
+
+    def e2e_step():
+        x_dev.copy_(x_host, non_blocking=True)
+        M.moe_layer_forward(d, x_dev, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                            inp.Ws_gate, inp.Ws_up, inp.Ws_down, out, ws, stream)
+        out_host.copy_(out, non_blocking=True)
+
+    for _ in range(args.warmup):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    barrier()
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s0.record(stream)
+    for _ in range(args.steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier()
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1))
+    e2e_value = w.T * world * args.steps / (e2e_ms / 1e3)
+    err = M.get_device_error(stream)
+    if err:
+        raise RuntimeError(f"device error word {err:#x}")
+
+    # roofline of the dominant kernel (gate/up grouped GEMM launch)
+    rows_exec = int(v["offsets"][-1].item())
+    work = stage_work(w, rows_exec)
+    peaks, peaks_kind = load_peaks()
+    power_capped = "sw_power_cap" in clk.reasons
+    tc_key = "bf16_tflops_sustained" if power_capped else "bf16_tflops"
+    tc_peak = peaks[tc_key]
+    stages = {}
+    for s in STAGES:
+        kind, amount = work[s]
+        t = per_stage[s] * 1e-3
+        if kind == "tensor":
+            ach = amount / t / 1e12
+            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "tflops": round(ach, 1),
+                         "frac": round(ach / tc_peak, 3)}
+        else:
+            ach = amount / t / 1e9
+            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "gbs": round(ach, 1),
+                         "frac": round(ach / peaks["hbm_gbs"], 3)}
+    up_flops = work["expert_up"][1]
+    achieved = up_flops / (per_stage["expert_up"] * 1e-3) / 1e12
+    gemm_flops = work["expert_up"][1] + work["expert_down"][1]
+    gemm_tflops = gemm_flops / ((per_stage["expert_up"] + per_stage["expert_down"]) * 1e-3) / 1e12
+    # whole-layer roofline: GEMM FLOPs at the tensor peak + HBM-bound stages' bytes at HBM peak
+    hbm_bytes = sum(work[s][1] for s in ("route", "permute", "combine", "stats"))
+    layer_roof_s = gemm_flops / (tc_peak * 1e12) + hbm_bytes / (peaks["hbm_gbs"] * 1e9)
+    roofline = {
+        "bound": "tensor",
+        "kernel": "grouped_gemm_kernel<EPI_SWIGLU> (expert up: gate+up, SiLU*up epilogue)",
+        "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
+        "frac": round(achieved / tc_peak, 3),
+        "traffic": load_traffic(args.workload),
+        "peak_source": f"{peaks_kind} {tc_key} (MEASURED_PEAKS.json)",
+        "flops_per_launch": up_flops,
+        "grouped_gemm_up_down_tflops": round(gemm_tflops, 1),
+        "layer_frac_of_roofline": round(layer_roof_s / (ms_per_step * 1e-3), 3),
+    }
+    res = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random-init)",
+        "config": {"workload": w.name, "model": w.description, "T": w.T,
+                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "global_batch": w.T * world,
+                   "seq_len": w.T,
+                   "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
+                   "rows_executed": rows_exec,
+                   "l2": "inputs larger than L2: %.2f GB of expert weights stream per step"
+                         % ((w.E * 3 * w.F * w.D * 2) / 1e9)},
+        "roofline": roofline, "stages": stages,
+        "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms / args.steps, 4),
+                "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
+                "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
+        "gpu_launches": launches_per_step(w) * args.steps,
+        "clocks": clk.summary(),
+    }
+    if remeasured:
+        res["clocks"]["remeasured"] = True
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        res["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+    if rank == 0:
+        print(json.dumps(res), flush=True)
+
+
+# ---------------------------------------------------------- oracle arm ----
+
+def _host_inputs(inp):
+    """The workload's tensors copied to host memory once (bf16/fp32 as generated)."""
+    def h(t):
+        return None if t is None else t.cpu()
+    return dict(x=h(inp.x), Wg=h(inp.Wg), bias=h(inp.bias), W_gate=h(inp.W_gate),
+                W_up=h(inp.W_up), W_down=h(inp.W_down), Ws_gate=h(inp.Ws_gate),
+                Ws_up=h(inp.Ws_up), Ws_down=h(inp.Ws_down))
+
+
+def oracle_step(w, host, tokens):
+    """One bounded oracle step: route the whole batch, evaluate the sampled tokens."""
+    from oracle import moe_oracle as O
+
+    def f64(t):
+        return None if t is None else t.float().double().numpy()
+
+    def weights_of(e):
+        g = f64(host["W_gate"][e]) if host["W_gate"] is not None else None
+        return g, f64(host["W_up"][e]), f64(host["W_down"][e])
+
+    wd = dict(T=w.T, D=w.D, E=w.E, F=w.F, k=w.k, c=w.c, score=w.score, select=w.select,
+              gate=w.gate, overflow=w.overflow, capacity_factor=w.capacity_factor, act=w.act,
+              n_shared=w.n_shared, F_shared=w.F_shared, aux_alpha=w.aux_alpha)
+    r = O.layer_forward_rows(wd, tokens, f64(host["x"]), f64(host["Wg"]), f64(host["bias"]),
+                             None, None, None, f64(host["Ws_gate"]), f64(host["Ws_up"]),
+                             f64(host["Ws_down"]), weights_of=weights_of)
+    return r["out_rows"]
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i["num_threads"] for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(w, inp, budget_s=15.0, sample=128):
+    import numpy as np
+    host = _host_inputs(inp)
+    rng = np.random.default_rng(0)
+    done, reps, t0 = 0, 0, time.perf_counter()
+    while True:
+        tokens = sorted(rng.choice(w.T, size=sample, replace=False).tolist())
+        oracle_step(w, host, tokens)
+        done += len(tokens)
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": round(done / dt, 2), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle",
+            "sample": f"{reps} x {sample} random tokens of one {w.name} batch (T={w.T}); each "
+                      f"repetition routes the whole batch and evaluates the sampled tokens' "
+                      f"experts in fp64 ({dt:.1f} s of CPU work)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    import numpy as np
+    w = workload_of(args)
+    device = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = make_inputs(w, seed=0, device=device)
+    host = _host_inputs(inp)
+    del inp
+    if device == "cuda":
+        torch.cuda.empty_cache()
+    rng = np.random.default_rng(0)
+    probe = sorted(rng.choice(w.T, size=16, replace=False).tolist())
+    t0 = time.perf_counter()
+    oracle_step(w, host, probe)
+    fixed = time.perf_counter() - t0
+    # per-step sample sized so that warm-up + steps take about args.ref_budget seconds
+    per_step = max(fixed, args.ref_budget / max(1, args.steps + args.warmup))
+    sample = int(max(8, min(w.T, 16 * per_step / max(fixed, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_step(w, host, sorted(rng.choice(w.T, size=sample, replace=False).tolist()))
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(w, host, sorted(rng.choice(w.T, size=sample, replace=False).tolist()))
+    dt = time.perf_counter() - t0
+    value = sample * args.steps / dt
+    desc = (f"each step routes one whole {w.name} batch (T={w.T}) and evaluates {sample} "
+            f"random tokens' experts in fp64")
+    res = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random-init)",
+        "config": {"workload": w.name, "model": w.description, "T": w.T,
+                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "global_batch": w.T,
+                   "seq_len": w.T, "parallelism": "CPU oracle (rank 0)"},
+        "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(),
+                         "kind": "oracle", "sample": desc},
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(res), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default="mixtral", choices=["mixtral", "switch", "ec"])
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="override the batch size T (smaller cases for profiling)")
+    ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0)
+    ap.add_argument("--ref-budget", type=float, default=90.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, rank, world)
+        return
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    try:
+        run_cuda(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

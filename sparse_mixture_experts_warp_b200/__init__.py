@@ -233,6 +233,7 @@ def layer_views(d: MoeDesc, ws: torch.Tensor) -> dict:
         y_shared=view(v.y_shared, dt, (d.n_shared, d.T, d.D)) if d.n_shared else None,
         f=view(v.f, torch.float32, (d.E,)),
         stats=view(v.stats, torch.uint8, (ctypes.sizeof(MoeStats),)),
+        scratch=view(v.scratch, torch.uint8, (v.scratch_bytes,)),
         rows=A,
     )
     return out
