@@ -161,6 +161,24 @@ moe_status_t moe_permute(const moe_desc_t* desc, const int32_t* expert_ids, cons
                          void* x_perm, int32_t* counts, int32_t* offsets, int32_t* row_src,
                          int32_t* inv, void* scratch, size_t scratch_bytes, moe_stream_t stream);
 
+/* moe_permute without scratch, for callers that cannot allocate device memory (a plugin handed
+ * only its input and output buffers by an engine whose allocator owns the device memory, or
+ * host code that must not call cudaMalloc at that point).  The pages have no counterpart: this
+ * is a property of the library, not of the method.
+ *   Same arguments, outputs and results as moe_permute, minus scratch.  Its scratch is a fixed
+ *   file-scope device array of MOE_PERMUTE_NOALLOC_MAX_INTS int32 (256 KiB) that every GPU
+ *   loading the library holds until exit.  Token choice needs ceil(T*k/1024)*E of them; larger
+ *   problems return MOE_ERR_UNSUPPORTED before anything is launched.  Allocates nothing (no
+ *   cudaMalloc, cudaFree or allocating library call).
+ *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
+ *   that device current and caches it: make that first call before any stream capture.
+ *   All calls share the array and each overwrites the last one's contents; calls whose work
+ *   overlaps on the GPU (other streams, other threads) race on it -- serialise them. */
+#define MOE_PERMUTE_NOALLOC_MAX_INTS 65536
+moe_status_t moe_permute_noalloc(const moe_desc_t* desc, const int32_t* expert_ids,
+                                 const void* x, void* x_perm, int32_t* counts, int32_t* offsets,
+                                 int32_t* row_src, int32_t* inv, moe_stream_t stream);
+
 /* Expert compute on grouped rows (Tiny MoE section 3, SwiGLU: down(SiLU(x W_gate^T) * x W_up^T);
  * ReLU: down(ReLU(x W_up^T))).  Group g owns rows [offsets[g], offsets[g+1]) of `a`
  * (offsets is a device array of n_groups+1 ints, read on the device).

@@ -20,7 +20,7 @@ __all__ = [
     "MoeDesc", "MoeStats", "MoeLayerViews", "MoeError", "lib", "library_path", "desc_of",
     "header_functions", "status_string", "rows_max", "capacity", "scratch_size",
     "workspace_size", "layer_views", "moe_route", "moe_permute", "moe_expert_up",
-    "moe_expert_down", "moe_expert_ffn", "moe_combine", "moe_balance_stats",
+    "moe_expert_down", "moe_expert_ffn", "moe_permute_noalloc", "moe_combine", "moe_balance_stats",
     "moe_layer_forward", "get_device_error", "empty_scratch", "empty_workspace",
 ]
 
@@ -86,6 +86,7 @@ _SIGS = {
     "moe_layer_views": ([_DP, _P, _SZ, ctypes.POINTER(MoeLayerViews)], ctypes.c_int),
     "moe_route": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_permute_noalloc": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_up": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_down": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -263,6 +264,14 @@ def moe_permute(d, expert_ids, x, x_perm, counts, offsets, row_src, inv, scratch
     _check("moe_permute", lib().moe_permute(
         ctypes.byref(d), _ptr(expert_ids), _ptr(x), _ptr(x_perm), _ptr(counts), _ptr(offsets),
         _ptr(row_src), _ptr(inv), _ptr(scratch), scratch.numel(), _stream(stream)))
+
+
+def moe_permute_noalloc(d, expert_ids, x, x_perm, counts, offsets, row_src, inv, stream=None):
+    """moe_permute for callers that cannot allocate: its scratch is a fixed device array inside
+    the library (see include/moe.h)."""
+    _check("moe_permute_noalloc", lib().moe_permute_noalloc(
+        ctypes.byref(d), _ptr(expert_ids), _ptr(x), _ptr(x_perm), _ptr(counts), _ptr(offsets),
+        _ptr(row_src), _ptr(inv), _stream(stream)))
 
 
 def moe_expert_up(d, n_groups, F, a, offsets, W_gate, W_up, h, stream=None):
