@@ -23,7 +23,9 @@ template <bool BF16> struct Row;
 template <> struct Row<true> {     // 8 bf16 per 16 bytes
   static constexpr int N = 8;
   __device__ __forceinline__ static void acc(const uint4* p, float g, float* a) {
-    const uint4 u = __ldcs(p);
+    acc_val(__ldcs(p), g, a);
+  }
+  __device__ __forceinline__ static void acc_val(const uint4 u, float g, float* a) {
     const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -44,7 +46,11 @@ template <> struct Row<true> {     // 8 bf16 per 16 bytes
 template <> struct Row<false> {    // 4 fp32 per 16 bytes
   static constexpr int N = 4;
   __device__ __forceinline__ static void acc(const uint4* p, float g, float* a) {
-    const float4 f = __ldcs(reinterpret_cast<const float4*>(p));
+    acc_val(__ldcs(p), g, a);
+  }
+  __device__ __forceinline__ static void acc_val(const uint4 u, float g, float* a) {
+    const float4 f = make_float4(__uint_as_float(u.x), __uint_as_float(u.y),
+                                 __uint_as_float(u.z), __uint_as_float(u.w));
     a[0] = fmaf(g, f.x, a[0]); a[1] = fmaf(g, f.y, a[1]);
     a[2] = fmaf(g, f.z, a[2]); a[3] = fmaf(g, f.w, a[3]);
   }
@@ -86,6 +92,56 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
     for (int q = 0; q < n; ++q) R::acc(y + (int64_t)s_row[warp][q] * nvec + v, s_g[warp][q], a);
     for (int s = 0; s < S; ++s) R::acc(ys + ((int64_t)s * T + t) * nvec + v, 1.0f, a);
     R::store(out + (int64_t)t * nvec + v, a);
+  }
+}
+
+
+// K <= 2 and no shared experts (Mixtral, Switch): each lane keeps 4 chunks x K rows of loads in
+// flight before accumulating, so a warp has up to 4 KB outstanding.
+template <bool BF16, int K>
+__global__ void __launch_bounds__(kWarps * 32)
+combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
+                       const float* __restrict__ gates, int T, int nvec,
+                       uint4* __restrict__ out) {
+  using R = Row<BF16>;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int t = blockIdx.x * kWarps + warp;
+  if (t >= T) return;
+  int row[K];
+  float g[K];
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    row[j] = inv[(int64_t)t * K + j];
+    g[j] = row[j] >= 0 ? gates[(int64_t)t * K + j] : 0.f;
+  }
+  int v = lane;
+  for (; v + 96 < nvec; v += 128) {
+    uint4 q[K][4];
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+        q[j][u] = row[j] >= 0 ? __ldcs(y + (int64_t)row[j] * nvec + v + 32 * u)
+                              : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float acc[R::N];
+#pragma unroll
+      for (int i = 0; i < R::N; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < K; ++j)
+        if (row[j] >= 0) R::acc_val(q[j][u], g[j], acc);
+      R::store(out + (int64_t)t * nvec + v + 32 * u, acc);
+    }
+  }
+  for (; v < nvec; v += 32) {
+    float acc[R::N];
+#pragma unroll
+    for (int i = 0; i < R::N; ++i) acc[i] = 0.f;
+#pragma unroll
+    for (int j = 0; j < K; ++j)
+      if (row[j] >= 0) R::acc(y + (int64_t)row[j] * nvec + v, g[j], acc);
+    R::store(out + (int64_t)t * nvec + v, acc);
   }
 }
 
@@ -138,6 +194,18 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
   const int nvec = d.D * esz / 16;
   const int S = y_shared ? d.n_shared : 0;
   const int blocks = (d.T + kWarps - 1) / kWarps;
+  if (S == 0 && d.select == MOE_TOKEN_CHOICE && d.k <= 2) {
+    const uint4* yy = static_cast<const uint4*>(y);
+    uint4* oo = static_cast<uint4*>(out);
+    if (d.dtype == MOE_BF16) {
+      if (K == 1) combine_small_k_kernel<true, 1><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      else combine_small_k_kernel<true, 2><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+    } else {
+      if (K == 1) combine_small_k_kernel<false, 1><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      else combine_small_k_kernel<false, 2><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+    }
+    return cudaGetLastError();
+  }
   if (d.dtype == MOE_BF16)
     combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,

@@ -28,16 +28,19 @@ inline bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p)
 // route.cu
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
-                                       float* logits, float* imp_partials, int n_partials,
+                                       float* logits, float* imp_partials, int* n_partials,
                                        cudaStream_t s);
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, int n_partials, cudaStream_t s);
+                                        float* imp_partials, int* n_partials, cudaStream_t s);
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s);
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
                                      float* importance, cudaStream_t s);
-int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer
+int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer (upper bound)
+
+// Streaming multiprocessors of the current device.
+int num_sms();
 
 // permute.cu
 int permute_blocks(const moe_desc_t& d);

@@ -14,25 +14,32 @@
 //   EPI_RELU:   out = max(acc, 0) with B0 = W_up.
 //   EPI_NONE:   out = acc with B0 = W_down.
 //
-// Design (one persistent CTA per SM, 192 threads, warp-specialised):
-//   warp 0 (one thread)  TMA producer: 128-byte-swizzled K-major boxes of A (128 x 64) and
-//                        B (2 x 128 x 64) into a 4-stage shared-memory ring, mbarrier
+// Design (one persistent CTA per SM, warp-specialised; two tile heights, see grouped_gemm_kernel):
+//   warp 0 (one thread)  TMA producer: 128-byte-swizzled K-major boxes of A (128 x 64, one or two
+//                        per stage) and B (2 x 128 x 64) into a shared-memory ring, mbarrier
 //                        complete_tx; no multicast.
-//   warp 1 (one thread)  MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256 K=16,
-//                        fp32 accumulator in TMEM; tcgen05.commit frees ring stages and hands
-//                        finished accumulators to the epilogue.  Warp 1 also owns the TMEM
-//                        allocation (512 columns = two 256-column accumulators, so the epilogue
-//                        of tile i overlaps the main loop of tile i+1).
-//   warps 2-5            epilogue: tcgen05.ld 32x32b (warp w reads TMEM lanes 32*(w%4)..+31,
-//                        one output row per thread), activation, bf16 pack, 16-byte stores of
-//                        the rows that belong to the group (rows past the group end are
-//                        computed from neighbouring rows and discarded).
+//   warp 1 (one thread)  MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256 K=16, fp32
+//                        accumulators in TMEM (512 columns); tcgen05.commit frees ring stages and
+//                        hands finished accumulators to the epilogue.  Warp 1 also owns the TMEM
+//                        allocation.
+//   warps 2..            epilogue: tcgen05.ld 32x32b (warp w reads TMEM lanes 32*(w%4)..+31, one
+//                        output row per thread), activation, bf16 pack, 16-byte stores of the rows
+//                        that belong to the group (rows past the group end are computed from
+//                        neighbouring rows and discarded).
+//   128-row tiles: 4 stages of 48 KB, two 256-column accumulators so the epilogue of tile i
+//   overlaps the main loop of tile i+1.  256-row tiles (the default): two M=128 MMAs per k-step
+//   share each B stage, which cuts L2->SMEM bytes per FLOP by a third (the 128-row tile needs
+//   ~96 B/clk/SM, more than the L2 can feed at full tensor rate); 3 stages of 64 KB, one
+//   512-column accumulator set; a tile with at most 128 live rows runs one half only, so the
+//   row waste stays that of 128-row tiles.
 // Tiles are enumerated group by group, n-tile by n-tile, with the m-tiles innermost, so the
 // CTAs that run at the same time share B tiles through L2 and each weight byte streams from
 // HBM about once.  The per-group row counts are read on the device (no host sync).
 // Every mbarrier wait is bounded (globaltimer); a wait that gives up records an error code in
 // the device error word and makes the CTA drain its in-flight copies and MMAs and exit.
 #include <cuda.h>
+#include <stdlib.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -49,7 +56,6 @@ constexpr int A_BYTES = BM * BK * 2;        // 16 KB
 constexpr int B_BYTES = MMA_N * BK * 2;     // 32 KB
 constexpr int ACC_COLS = MMA_N;             // fp32 accumulator columns per tile
 constexpr int TMEM_COLS = 2 * ACC_COLS;     // two accumulators
-constexpr int THREADS = 192;
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;   // 2 s per wait
 constexpr uint64_t DRAIN_NS = 200000000ull;      // 0.2 s to drain after an abort
 
@@ -177,22 +183,33 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-template <int EPI>
-__global__ void __launch_bounds__(THREADS, 1)
+// HALVES = 1: 128-row tiles, 4-stage ring of 48 KB, two 256-column TMEM accumulators (the
+//             epilogue of one tile overlaps the next tile's main loop), 4 epilogue warps.
+// HALVES = 2: 256-row tiles made of two M=128 MMAs that share every B stage (a third fewer
+//             L2->SMEM bytes per FLOP), 3-stage ring of 64 KB, one 512-column accumulator set,
+//             8 epilogue warps; a tile with <= 128 live rows loads and multiplies one half only.
+template <int EPI, int HALVES>
+__global__ void __launch_bounds__(64 + 128 * HALVES, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  constexpr int TBM = BM * HALVES;
+  constexpr int TSTAGES = HALVES == 1 ? STAGES : 3;
+  constexpr int TA_BYTES = TBM * BK * 2;
+  constexpr int NBUF = HALVES == 1 ? 2 : 1;          // TMEM accumulator buffers
+  constexpr int BUF_COLS = HALVES * ACC_COLS;        // columns per buffer
+  constexpr int N_EPI = 4 * HALVES;                  // epilogue warps
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
-  const uint32_t sB = sA + STAGES * A_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + STAGES * (A_BYTES + B_BYTES));
+  const uint32_t sB = sA + TSTAGES * TA_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TSTAGES * (TA_BYTES + B_BYTES));
   uint64_t* full = bars;
-  uint64_t* empty = bars + STAGES;
-  uint64_t* tfull = bars + 2 * STAGES;
-  uint64_t* tempty = tfull + 2;
-  uint64_t* drain = tempty + 2;
+  uint64_t* empty = bars + TSTAGES;
+  uint64_t* tfull = bars + 2 * TSTAGES;
+  uint64_t* tempty = tfull + NBUF;
+  uint64_t* drain = tempty + NBUF;
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
   int* grp_off = reinterpret_cast<int*>(tmem_holder + 2);   // [G+1]
@@ -201,13 +218,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
+    for (int s = 0; s < TSTAGES; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int a = 0; a < 2; ++a) {
+    for (int a = 0; a < NBUF; ++a) {
       mbar_init(&tfull[a], 1);
-      mbar_init(&tempty[a], 4 * 32);
+      mbar_init(&tempty[a], N_EPI * 32);
     }
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -240,7 +257,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       if (g < p.G) {
         const int lo = p.offsets[g], hi = p.offsets[g + 1];
         const int m = hi > lo ? hi - lo : 0;
-        tiles = ((m + BM - 1) / BM) * p.nt;
+        tiles = ((m + TBM - 1) / TBM) * p.nt;
         grp_off[g + 1] = hi;
       }
       int inc = tiles;
@@ -271,20 +288,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
         while (tile >= tile_pre[g + 1]) ++g;
         const int m = grp_off[g + 1] - grp_off[g];
-        const int mt = (m + BM - 1) / BM;
+        const int mt = (m + TBM - 1) / TBM;
         const int local = tile - tile_pre[g];
         const int n_idx = local / mt, m_idx = local - n_idx * mt;
-        const int a_row = grp_off[g] + m_idx * BM;
+        const int a_row = grp_off[g] + m_idx * TBM;
         const int b_row = g * p.N + n_idx * p.n_out_tile;
+        const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
                          TIMEOUT_NS)) {
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[stage], A_BYTES + B_BYTES);
-          const uint32_t a_dst = sA + stage * A_BYTES, b_dst = sB + stage * B_BYTES;
+          mbar_expect_tx(&full[stage], (two ? 2 * A_BYTES : A_BYTES) + B_BYTES);
+          const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * B_BYTES;
           tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, a_row);
+          if (two) tma_load_2d(a_dst + A_BYTES, &tmA, &full[stage], kb * BK, a_row + BM);
           if (EPI == EPI_SWIGLU) {
             tma_load_2d(b_dst, &tmB0, &full[stage], kb * BK, b_row);
             tma_load_2d(b_dst + B_BYTES / 2, &tmB1, &full[stage], kb * BK, b_row);
@@ -294,7 +313,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
-          if (++stage == STAGES) {
+          if (++stage == TSTAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -302,7 +321,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       if (!ok) {
         // let the copies already in flight land before the CTA exits
-        for (int s = 0; s < STAGES; ++s)
+        for (int s = 0; s < TSTAGES; ++s)
           if (issued & (1u << s))
             mbar_wait(&full[s], (issued_par >> s) & 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
                       DRAIN_NS);
@@ -314,17 +333,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       int stage = 0;
       uint32_t phase = 0;
       bool ok = true;
-      int it = 0;
+      int it = 0, g = 0;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
+        while (tile >= tile_pre[g + 1]) ++g;
+        const int m = grp_off[g + 1] - grp_off[g];
+        const int mt = (m + TBM - 1) / TBM;
+        const int m_idx = (tile - tile_pre[g]) % mt;
+        const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
+        const int acc = it % NBUF;
+        const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
                        TIMEOUT_NS)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * ACC_COLS);
+        const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BUF_COLS);
         for (int kb = 0; kb < nkb; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
                          TIMEOUT_NS)) {
@@ -332,14 +356,18 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
+          const uint32_t a0 = sA + stage * TA_BYTES, b0 = sB + stage * B_BYTES;
 #pragma unroll
           for (int k = 0; k < BK / MMA_K; ++k) {
-            umma_bf16(d_tmem, sdesc_sw128(a0 + k * MMA_K * 2), sdesc_sw128(b0 + k * MMA_K * 2),
-                      (kb > 0 || k > 0) ? 1u : 0u);
+            const uint64_t bdesc = sdesc_sw128(b0 + k * MMA_K * 2);
+            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+            umma_bf16(d_tmem, sdesc_sw128(a0 + k * MMA_K * 2), bdesc, accum);
+            if (two)
+              umma_bf16(d_tmem + ACC_COLS, sdesc_sw128(a0 + A_BYTES + k * MMA_K * 2), bdesc,
+                        accum);
           }
           umma_commit(&empty[stage]);       // frees the stage once these MMAs have read it
-          if (++stage == STAGES) {
+          if (++stage == TSTAGES) {
             stage = 0;
             phase ^= 1u;
           }
@@ -351,32 +379,40 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       mbar_wait(drain, 0u, abort_flag, p.err, DEVERR_TIMEOUT_MMA, ok ? TIMEOUT_NS : DRAIN_NS);
     }
   } else {
-    // ---------------- epilogue (warps 2..5) ----------------
+    // ---------------- epilogue (warps 2 .. 2 + N_EPI) ----------------
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
-    const int row = q * 32 + lane;
+    const int half = (warp - 2) / 4;         // which 128-row half of the tile
+    const int row = half * BM + q * 32 + lane;
     int g = 0, it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       while (tile >= tile_pre[g + 1]) ++g;
       const int m = grp_off[g + 1] - grp_off[g];
-      const int mt = (m + BM - 1) / BM;
+      const int mt = (m + TBM - 1) / TBM;
       const int local = tile - tile_pre[g];
       const int n_idx = local / mt, m_idx = local - n_idx * mt;
-      const int acc = it & 1;
-      const uint32_t acc_par = (uint32_t)(it >> 1) & 1u;
+      const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
+      const int acc = it % NBUF;
+      const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
       int okw = 1;
       if (lane == 0)
         okw = mbar_wait(&tfull[acc], acc_par, abort_flag, p.err, DEVERR_TIMEOUT_EPI, TIMEOUT_NS);
       okw = __shfl_sync(0xffffffffu, okw, 0);
       if (!okw) break;
       tc_fence_after();
-      const int r = m_idx * BM + row;
+      if (half == 1 && !two) {               // this half was not computed: nothing to drain
+        tc_fence_before();
+        mbar_arrive(&tempty[acc]);
+        continue;
+      }
+      const int r = m_idx * TBM + row;
       const int64_t orow = (int64_t)grp_off[g] + r;
       bool valid = r < m;
       if (valid && (orow < 0 || orow >= p.rows)) {
         atomicCAS(p.err, 0, DEVERR_BOUNDS);
         valid = false;
       }
-      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * ACC_COLS);
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) +
+                             (uint32_t)(acc * BUF_COLS + half * ACC_COLS);
       __nv_bfloat16* orow_ptr = p.out + orow * p.ldo + (int64_t)n_idx * p.n_out_tile;
       if (EPI == EPI_SWIGLU) {
 #pragma unroll 1
@@ -392,8 +428,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
               const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * u0;
-              const float h1 = g1 / (1.0f + __expf(-g1)) * u1;
+              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;   // SiLU(g) * u
+              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
               pk[i] = pack_bf16(h0, h1);
             }
             uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c);
@@ -478,6 +514,19 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tile height in 128-row halves: 256-row tiles (a third fewer L2 bytes per FLOP) for every
+// epilogue; measured on the Mixtral layer shape they beat 128-row tiles for both the gate/up and
+// the down projection.  MOE_GEMM_HALVES=1 selects the 128-row tile with its double TMEM buffer
+// (kept for comparison measurements; both heights are tested).
+int gemm_halves(int epi) {
+  (void)epi;
+  static int h = [] {
+    const char* v = getenv("MOE_GEMM_HALVES");
+    return (v && v[0] == '1') ? 1 : 2;
+  }();
+  return h;
+}
+
 int sm_count() {
   int dev = 0, n = 0;
   cudaGetDevice(&dev);
@@ -485,13 +534,13 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int EPI>
+template <int EPI, int HALVES>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI>,
+  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, HALVES>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<EPI><<<grid, THREADS, smem, s>>>(a, b0, b1, p);
+  grouped_gemm_kernel<EPI, HALVES><<<grid, 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
   return cudaGetLastError();
 }
 
@@ -521,14 +570,24 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.K = K;
   p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
   p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
-  const int64_t max_tiles = ((a_rows + BM - 1) / BM + n_groups) * (int64_t)p.nt;
+  const int halves = gemm_halves(epi);
+  const int tbm = BM * halves;
+  const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
-  const size_t smem = 1024 + (size_t)STAGES * (A_BYTES + B_BYTES) + (2 * STAGES + 5) * 8 + 8 +
-                      (size_t)2 * (n_groups + 1) * sizeof(int);
+  const int tstages = halves == 1 ? STAGES : 3;
+  const size_t smem = 1024 + (size_t)tstages * ((size_t)tbm * BK * 2 + B_BYTES) +
+                      (2 * tstages + 5) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
+  if (halves == 2) {
+    switch (epi) {
+      case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 2>(ta, tb0, tb1, p, grid, smem, s);
+      case EPI_RELU: return launch_epi<EPI_RELU, 2>(ta, tb0, tb1, p, grid, smem, s);
+      default: return launch_epi<EPI_NONE, 2>(ta, tb0, tb1, p, grid, smem, s);
+    }
+  }
   switch (epi) {
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU>(ta, tb0, tb1, p, grid, smem, s);
-    case EPI_RELU: return launch_epi<EPI_RELU>(ta, tb0, tb1, p, grid, smem, s);
-    default: return launch_epi<EPI_NONE>(ta, tb0, tb1, p, grid, smem, s);
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 1>(ta, tb0, tb1, p, grid, smem, s);
+    case EPI_RELU: return launch_epi<EPI_RELU, 1>(ta, tb0, tb1, p, grid, smem, s);
+    default: return launch_epi<EPI_NONE, 1>(ta, tb0, tb1, p, grid, smem, s);
   }
 }
 

@@ -12,6 +12,13 @@ namespace moe {
 
 static __device__ int g_device_error = 0;
 
+int num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+  return n > 0 ? n : 148;
+}
+
 int* device_error_word() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
@@ -214,14 +221,15 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
   uint8_t* sc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(scratch) + kAlign - 1) &
                                            ~(uintptr_t)(kAlign - 1));
   float* partials = reinterpret_cast<float*>(sc);
-  const int np = router_partials(*d);
+  int np = 0;
   cudaError_t e;
   if (d->select == MOE_TOKEN_CHOICE) {
     e = launch_router_token_choice(*d, x, Wg, d->score == MOE_SCORE_SIGMOID ? sel_bias : nullptr,
-                                   expert_ids, gates, logits, partials, np, s);
+                                   expert_ids, gates, logits, partials, &np, s);
   } else {
-    float* probsT = reinterpret_cast<float*>(sc + up((size_t)np * d->E * sizeof(float)));
-    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, np, s);
+    const size_t pbytes = up((size_t)router_partials(*d) * d->E * sizeof(float));
+    float* probsT = reinterpret_cast<float*>(sc + pbytes);
+    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, s);
     if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
   }
   if (e == cudaSuccess && importance)

@@ -139,6 +139,99 @@ perm_rank_kernel(const int32_t* ids, int A, int E, int cap, const int32_t* block
   }
 }
 
+
+// Small problems (A <= kFusedMaxItems): histogram, scans and stable ranks in ONE block of 32
+// warps.  The expert ids are first staged in shared memory with all loads in flight at once;
+// warp w owns the contiguous assignments [w*S, (w+1)*S); pass 1 counts them per expert (peer
+// groups from __match_any_sync, leader adds), the per-expert exclusive scan over warps gives
+// each warp its base, a block scan over experts gives the offsets, and pass 2 assigns ranks in
+// the same order.  One launch instead of three.
+constexpr int kFusedMaxItems = 1 << 15;
+
+__global__ void __launch_bounds__(1024)
+perm_index_fused_kernel(const int32_t* ids, int A, int E, int cap, int32_t* counts,
+                        int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  extern __shared__ int s_mem[];
+  int* s_cnt = s_mem;                    // [32][E]
+  int* s_off = s_mem + 32 * E;           // [E]
+  int* s_ids = s_mem + 33 * E;           // [A]
+  __shared__ int s_warp[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) s_cnt[i] = 0;
+  for (int i = threadIdx.x; i < A; i += blockDim.x) s_ids[i] = ids[i];
+  __syncthreads();
+  const int per = ((A + 32 * 32 - 1) / (32 * 32)) * 32;       // multiple of 32
+  const int lo = warp * per, hi = min(A, lo + per);
+  int* my = s_cnt + warp * E;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int a = base + lane;
+    const int e = (a < hi) ? s_ids[a] : -1;
+    const bool ok = (e >= 0 && e < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    if (ok && (peers & lt) == 0) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  int kept = 0;
+  const int e = threadIdx.x;
+  if (e < E) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int v = s_cnt[w * E + e];
+      s_cnt[w * E + e] = run;
+      run += v;
+    }
+    counts[e] = run;
+    kept = (cap > 0 && run > cap) ? cap : run;
+  }
+  // exclusive scan of kept over experts (E <= 1024)
+  int inc = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int n = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += n;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += n;
+    }
+    s_warp[lane] = wv;
+  }
+  __syncthreads();
+  const int excl = (warp > 0 ? s_warp[warp - 1] : 0) + inc - kept;
+  if (e < E) {
+    offsets[e] = excl;
+    s_off[e] = excl;
+  }
+  if (e == E - 1) offsets[E] = excl + kept;
+  __syncthreads();
+  for (int base = lo; base < hi; base += 32) {
+    const int a = base + lane;
+    const int ee = (a < hi) ? s_ids[a] : -1;
+    const bool ok = (ee >= 0 && ee < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? ee : -1);
+    int rank = 0;
+    if (ok) rank = my[ee] + __popc(peers & lt);
+    __syncwarp();
+    if (ok && (peers & lt) == 0) my[ee] += __popc(peers);
+    __syncwarp();
+    if (a < hi) {
+      int row = -1;
+      if (ok && (cap <= 0 || rank < cap)) {
+        row = s_off[ee] + rank;
+        row_src[row] = a;
+      }
+      inv[a] = row;
+    }
+  }
+}
+
 // One warp per token: copy x[t] (D elements of `esz` bytes) to each kept row.
 __global__ void __launch_bounds__(256)
 gather_tc_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_t* inv,
@@ -229,13 +322,19 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
   const int A = d.T * d.k;
   const int nblk = permute_blocks(d);
   const int E = d.E;
-  if (nblk > 0) {
+  if (A <= kFusedMaxItems) {
+    const size_t smem = ((size_t)33 * E + A) * sizeof(int);
+    if (smem > 48 * 1024)
+      cudaFuncSetAttribute(perm_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem);
+    perm_index_fused_kernel<<<1, 1024, smem, s>>>(ids, A, E, cap, counts, offsets, row_src, inv);
+  } else {
     perm_hist_kernel<<<nblk, kThreads, E * sizeof(int), s>>>(ids, A, E, block_hist);
-  }
-  perm_scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
-  if (nblk > 0) {
+    perm_scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
     perm_rank_kernel<<<nblk, kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
         ids, A, E, cap, block_hist, offsets, row_src, inv);
+  }
+  if (nblk > 0) {
     const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
     const int nvec = d.D * esz / 16;
     const int blocks = (d.T * 32 + 255) / 256;

@@ -337,11 +337,164 @@ ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
   }
 }
 
+
+// ---- fast path: bf16 token choice, E <= 8, D = 256 * NW with 4 <= NW <= 16 ----
+//
+// The router product is an HBM-bound contraction with N = E <= 8 experts: exactly the N of
+// mma.sync m16n8k16, so the FMAs (and the bf16 -> fp32 conversions a CUDA-core dot product
+// needs) go to the tensor cores and the kernel is left with streaming x.  One CTA of NW warps
+// owns a contiguous range of tokens; warp w owns the hidden slice [256w, 256w + 256).  The k
+// order inside the slice is permuted (the same permutation for x and W_g, which leaves the sum
+// unchanged) so that each thread's A fragments over the 16 k-steps are eight 16-byte chunks of
+// two token rows and its B fragments the same eight chunks of one W_g row: every global load is
+// a 16-byte vector load, and the 4 threads of a row read 64 contiguous bytes together.  Per 16-token batch a warp issues 16 MMAs; partial
+// logits of the NW warps are summed in a fixed order through shared memory, the next batch's
+// loads are already in flight while warps do the per-token affinity / top-k / gates.
+constexpr int kFastE = 8;        // MMA N: experts (zero-padded)
+constexpr int kFastTB = 16;      // MMA M: tokens per batch
+constexpr int kFastMaxNW = 16;
+
+__device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1,
+                                               uint32_t a2, uint32_t a3, uint32_t b0,
+                                               uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 "
+      "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two token rows (g, g + 8 of the batch): this thread's 8 chunks of 8 elements, chunk i at
+// element kbase + 32 i (kbase = 256 w + 8 tig), so the 4 threads of a row read 64 contiguous
+// bytes per load instruction.
+__device__ __forceinline__ void load_rows(uint4 (&r0)[8], uint4 (&r1)[8],
+                                          const __nv_bfloat16* x, int D, int t0, int t_end,
+                                          int g, int kbase) {
+  const int ta = t0 + g, tb = t0 + g + 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r0[i] = (ta < t_end)
+                ? __ldcs(reinterpret_cast<const uint4*>(x + (int64_t)ta * D + kbase + 32 * i))
+                : make_uint4(0u, 0u, 0u, 0u);
+    r1[i] = (tb < t_end)
+                ? __ldcs(reinterpret_cast<const uint4*>(x + (int64_t)tb * D + kbase + 32 * i))
+                : make_uint4(0u, 0u, 0u, 0u);
+  }
+}
+
+__device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float sv, bool live,
+                                             int lane, float& imp) {
+  const int E = a.E;
+  if (a.logits && live) a.logits[(int64_t)tok * E + lane] = sv;
+  float selw, key;
+  if (a.score == MOE_SCORE_SOFTMAX) {
+    const float m = warp_max(sv);
+    const float z = live ? expf(sv - m) : 0.f;
+    const float p = z / warp_sum(z);
+    selw = p;
+    key = sv;                    // softmax is monotone in the logit within a row
+    imp += p;
+  } else {
+    const float af = live ? 1.0f / (1.0f + expf(-sv)) : 0.f;
+    selw = af;
+    key = live ? af + (a.bias ? a.bias[lane] : 0.f) : -INFINITY;
+    imp += af / warp_sum(af);
+  }
+  bool taken = !live;
+  int my_id = -1;
+  float my_w = 0.f, wsum = 0.f;
+  for (int j = 0; j < a.k; ++j) {
+    float bk = taken ? -INFINITY : key;
+    int bi = taken ? 0x7fffffff : lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ok > bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+    }
+    const float wv = __shfl_sync(0xffffffffu, selw, bi & 31);
+    if (lane == bi) taken = true;
+    wsum += wv;
+    if (lane == j) { my_id = (bi < E) ? bi : -1; my_w = wv; }
+  }
+  if (lane < a.k) {
+    a.ids[(int64_t)tok * a.k + lane] = my_id;
+    a.gates[(int64_t)tok * a.k + lane] = (a.gate == MOE_GATE_RENORM) ? my_w / wsum : my_w;
+  }
+}
+
+__global__ void __launch_bounds__(kFastMaxNW * 32, 1)
+router_fast_kernel(RouterArgs a, int tokens_per_cta) {
+  __shared__ float s_red[kFastMaxNW][kFastTB][kFastE];
+  __shared__ float s_log[kFastTB][kFastE];
+  __shared__ float s_imp[kFastTB][kFastE];
+  const int NW = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, tig = lane & 3;
+  const int E = a.E;
+  const int kbase = warp * 256 + tig * 8;    // this thread's chunks: kbase + 32 i, i < 8
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+  const __nv_bfloat16* Wg = static_cast<const __nv_bfloat16*>(a.Wg);
+  uint4 wv[8];                               // W_g[g][kbase + 32 i .. + 8)
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    wv[i] = (g < E) ? __ldg(reinterpret_cast<const uint4*>(Wg + (int64_t)g * a.D + kbase + 32 * i))
+                    : make_uint4(0u, 0u, 0u, 0u);
+  const int t_begin = blockIdx.x * tokens_per_cta;
+  const int t_end = min(a.T, t_begin + tokens_per_cta);
+  float imp = 0.f;
+  uint4 r0[8], r1[8];
+  load_rows(r0, r1, x, a.D, t_begin, t_end, g, kbase);
+  for (int t0 = t_begin; t0 < t_end; t0 += kFastTB) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // k-steps 2i (chunk elements 0..3) and 2i+1 (chunk elements 4..7)
+      mma_16816_bf16(c, r0[i].x, r1[i].x, r0[i].y, r1[i].y, wv[i].x, wv[i].y);
+      mma_16816_bf16(c, r0[i].z, r1[i].z, r0[i].w, r1[i].w, wv[i].z, wv[i].w);
+    }
+    if (t0 + kFastTB < t_end) load_rows(r0, r1, x, a.D, t0 + kFastTB, t_end, g, kbase);
+    s_red[warp][g][2 * tig] = c[0];
+    s_red[warp][g][2 * tig + 1] = c[1];
+    s_red[warp][g + 8][2 * tig] = c[2];
+    s_red[warp][g + 8][2 * tig + 1] = c[3];
+    __syncthreads();
+    if (threadIdx.x < kFastTB * kFastE) {
+      const int j = threadIdx.x / kFastE, e = threadIdx.x % kFastE;
+      float sum = 0.f;
+      for (int ww = 0; ww < NW; ++ww) sum += s_red[ww][j][e];
+      s_log[j][e] = sum;
+    }
+    __syncthreads();
+    for (int jj = warp; jj < kFastTB; jj += NW) {
+      if (t0 + jj >= t_end) break;
+      const bool live = lane < E;
+      select_token(a, t0 + jj, live ? s_log[jj][lane] : -INFINITY, live, lane, imp);
+    }
+  }
+  // CTA importance partial: sum over the selection warps in a fixed order
+  const int n_sel = NW < kFastTB ? NW : kFastTB;
+  if (warp < n_sel && lane < kFastE) s_imp[warp][lane] = imp;
+  __syncthreads();
+  if (a.partials && threadIdx.x < E) {
+    float sum = 0.f;
+    for (int j = 0; j < n_sel; ++j) sum += s_imp[j][threadIdx.x];
+    a.partials[(int64_t)blockIdx.x * E + threadIdx.x] = sum;
+  }
+}
+
 }  // namespace
 
-int router_partials(const moe_desc_t& d) {
+// Rows of importance partials the generic kernel writes (one per warp).
+static int generic_partials(const moe_desc_t& d) {
   const int blocks = (d.T + kWarps * kTPW - 1) / (kWarps * kTPW);
   return blocks * kWarps;
+}
+
+int router_partials(const moe_desc_t& d) {
+  // capacity for either kernel: generic = one row per warp; fast = one row per CTA (<= 1024)
+  const int generic = generic_partials(d);
+  return generic > 1024 ? generic : 1024;
 }
 
 static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStream_t s) {
@@ -360,20 +513,34 @@ static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStre
   return cudaGetLastError();
 }
 
+static bool fast_router_ok(const moe_desc_t& d) {
+  return d.dtype == MOE_BF16 && d.select == MOE_TOKEN_CHOICE && d.E <= kFastE &&
+         d.D % 256 == 0 && d.D / 256 >= 4 && d.D / 256 <= kFastMaxNW && d.k <= 32;
+}
+
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
-                                       float* logits, float* imp_partials, int n_partials,
+                                       float* logits, float* imp_partials, int* n_partials,
                                        cudaStream_t s) {
-  (void)n_partials;
   RouterArgs a{x, Wg, bias, ids, gates, logits, nullptr, imp_partials,
                d.T, d.D, d.E, d.k, d.score, d.gate, 0};
+  if (fast_router_ok(d)) {
+    const int sms = num_sms() < 1024 ? num_sms() : 1024;
+    const int tpc = (d.T + sms - 1) / sms;
+    const int grid = tpc > 0 ? (d.T + tpc - 1) / tpc : 0;
+    *n_partials = grid;
+    if (grid == 0) return cudaSuccess;
+    router_fast_kernel<<<grid, (d.D / 256) * 32, 0, s>>>(a, tpc);
+    return cudaGetLastError();
+  }
+  *n_partials = generic_partials(d);
   return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, int n_partials, cudaStream_t s) {
-  (void)n_partials;
+                                        float* imp_partials, int* n_partials, cudaStream_t s) {
+  *n_partials = generic_partials(d);
   RouterArgs a{x, Wg, nullptr, nullptr, probs, logits, probsT, imp_partials,
                d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1};
   return launch_router(a, d.dtype == MOE_BF16, d.T, s);

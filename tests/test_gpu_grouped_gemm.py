@@ -83,3 +83,16 @@ def test_grouped_gemm_repeatable():
     M.moe_expert_ffn(d, G, 192, a, offsets, Wg, Wu, Wd, h, y)
     torch.cuda.synchronize()
     assert torch.equal(y1[:n], y[:n])
+
+
+def test_grouped_gemm_128_row_tiles_in_subprocess():
+    """The 128-row tile variant (double TMEM buffer) is selected per process by
+    MOE_GEMM_HALVES=1; run this file's ragged cases under it in a child process."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_GEMM_HALVES="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__,
+                        "-k", "ragged or repeatable"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]

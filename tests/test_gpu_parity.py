@@ -32,6 +32,14 @@ SMALL = {
     "switch_small": scaled(W["switch"], T=3000, D=256, E=16, F=512),
     "v3_small": scaled(W["v3"], T=300, D=512, E=64, F=256, F_shared=256),
     "ec_small": scaled(W["ec"], T=1000, D=256, E=16, F=256, c=125),
+    # the bf16 router fast path (E <= 8, D = 256 * NW, 4 <= NW <= 16), ragged token counts
+    "fast_router_T1": scaled(W["mixtral"], T=1, D=4096, F=256),
+    "fast_router_T37": scaled(W["mixtral"], T=37, D=1024, F=256),
+    "fast_router_T300_E6": scaled(W["mixtral"], T=300, D=2048, E=6, F=256),
+    "fast_router_switch_k1": scaled(W["switch"], T=500, D=1024, E=8, F=256),
+    "fast_router_sigmoid_shared": scaled(W["v3"], T=200, D=1024, E=8, k=2, F=256, F_shared=256),
+    # more than 65536 assignments: the multi-block permute path
+    "large_A": scaled(W["mixtral"], T=33000, D=128, F=128),
 }
 
 

@@ -65,6 +65,9 @@ def _compare(w, d, x, ids):
     ("mixtral", dict(T=700, D=512, F=1024)),
     ("switch", dict(T=3000, D=256, E=16, F=512)),     # capacity drop
     ("v3", dict(T=300, D=512, E=64, F=256, F_shared=256)),
+    # more than 65536 assignments: the histogram path that uses the fixed scratch array
+    ("mixtral", dict(T=40000, D=128, F=128)),
+    ("v3", dict(T=9000, D=128, E=64, F=128, F_shared=128)),
 ])
 def test_noalloc_permute_matches_permute_on_two_calls(name, shape):
     w = scaled(WORKLOADS[name], **shape)
