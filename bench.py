@@ -148,6 +148,28 @@ class ClockSampler:
         return False
 
 
+def barrier(world):
+    """Barrier across the replicas (no-op for one process)."""
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x, world, device):
+    """The largest value of x over all ranks (timings: the slowest replica sets the time)."""
+    if world == 1:
+        return float(x)
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank, world, steps, max_total_ms):
+    """Whole-job tokens/s: every replica's tokens over the slowest replica's time."""
+    return tokens_per_rank * world * steps / (max_total_ms / 1e3)
+
+
 def launches_per_step(w):
     """Kernels the library launches per layer step (its own kernels only)."""
     n = 2 + (1 if w.select == "expert" else 0)            # router, importance reduce, ec select
@@ -188,7 +210,6 @@ def workload_of(args):
 # -------------------------------------------------------------- CUDA arm ----
 
 def run_cuda(args, rank, world, local):
-    import torch.distributed as dist
     import sparse_mixture_experts_warp_b200 as M
 
     torch.cuda.set_device(local)
@@ -228,17 +249,6 @@ def run_cuda(args, rank, world, local):
         if ev is not None:
             ev[6].record(stream)
 
-    def barrier():
-        if world > 1:
-            dist.barrier()
-
-    def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
-
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
@@ -249,7 +259,7 @@ def run_cuda(args, rank, world, local):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)]
                for _ in range(args.steps)]
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier()
+        barrier(world)
         torch.cuda.synchronize(dev)
         with ClockSampler(nvml_index) as clk:
             start.record(stream)
@@ -258,7 +268,7 @@ def run_cuda(args, rank, world, local):
                 step(evs[i])
             end.record(stream)
             torch.cuda.synchronize(dev)
-        barrier()
+        barrier(world)
         total = start.elapsed_time(end)
         per_stage = {s: 0.0 for s in STAGES}
         for i in range(args.steps):
@@ -271,9 +281,9 @@ def run_cuda(args, rank, world, local):
     if clk.rejected():
         total_ms, per_stage, clk = timed()
         remeasured = True
-    total_ms = max_over_ranks(total_ms)
+    total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
-    value = w.T * world * args.steps / (total_ms / 1e3)
+    value = job_throughput(w.T, world, args.steps, total_ms)
 
     # e2e: the public call with host buffers, copies inside the timed region
     x_host = inp.x.cpu().pin_memory()
@@ -289,16 +299,16 @@ def run_cuda(args, rank, world, local):
     for _ in range(args.warmup):
         e2e_step()
     torch.cuda.synchronize(dev)
-    barrier()
+    barrier(world)
     s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     s0.record(stream)
     for _ in range(args.steps):
         e2e_step()
     s1.record(stream)
     torch.cuda.synchronize(dev)
-    barrier()
-    e2e_ms = max_over_ranks(s0.elapsed_time(s1))
-    e2e_value = w.T * world * args.steps / (e2e_ms / 1e3)
+    barrier(world)
+    e2e_ms = max_over_ranks(s0.elapsed_time(s1), world, dev)
+    e2e_value = job_throughput(w.T, world, args.steps, e2e_ms)
     err = M.get_device_error(stream)
     if err:
         raise RuntimeError(f"device error word {err:#x}")

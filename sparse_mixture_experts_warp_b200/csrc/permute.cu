@@ -232,6 +232,174 @@ perm_index_fused_kernel(const int32_t* ids, int A, int E, int cap, int32_t* coun
   }
 }
 
+
+// One-pass token-choice permute for small problems (E <= 8, k <= 8, A <= kOnePassMaxItems):
+// every CTA owns 32 consecutive tokens.  It first counts ALL assignments per expert (totals)
+// and those before its own tokens (its per-expert base) -- the ids are L2-resident and shared
+// by all CTAs, so this replaces a grid-wide scan.  Counting uses per-thread packed counters
+// (eight 8-bit counts in two registers) and a fixed-order block reduction.  Then it ranks its
+// own assignments stably (peer groups of __match_any_sync, per-warp prefix), writes inv /
+// row_src (CTA 0 also counts and offsets), and copies its tokens' rows into their expert rows
+// with four tokens' loads in flight per warp.  Counting is order-free and every rank is a
+// deterministic prefix: the result equals the multi-kernel path bit for bit.
+constexpr int kOnePassTokens = 32;
+constexpr int kOnePassMaxE = 8;
+constexpr int kOnePassMaxK = 8;
+constexpr int kOnePassMaxItems = 1 << 14;       // <= 64 ids per thread: 8-bit counts suffice
+
+__device__ __forceinline__ void count_packed(int e, uint32_t& lo, uint32_t& hi) {
+  const uint32_t inc = 1u << (8 * (e & 3));
+  if (e >= 0 && e < 4) lo += inc;
+  else if (e >= 4 && e < 8) hi += inc;
+}
+
+__global__ void __launch_bounds__(256)
+permute_onepass_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int cap,
+                       const uint4* __restrict__ x, int nvec, uint4* __restrict__ xp,
+                       int32_t* counts, int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  __shared__ int s_all[8][kOnePassMaxE];       // per warp: all assignments
+  __shared__ int s_pre[8][kOnePassMaxE];       // per warp: assignments before this CTA's
+  __shared__ int s_own[8][kOnePassMaxE];       // per warp: this CTA's, then exclusive bases
+  __shared__ int s_off[kOnePassMaxE];
+  __shared__ int s_row[kOnePassTokens * kOnePassMaxK];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const unsigned lt = (1u << lane) - 1u;
+  const int A = T * k;
+  const int a0 = blockIdx.x * kOnePassTokens * k;
+  const int a1 = min(A, a0 + kOnePassTokens * k);
+  // 1. packed per-thread counts of all ids and of the ids before a0
+  uint32_t all_lo = 0, all_hi = 0, pre_lo = 0, pre_hi = 0;
+  for (int base0 = threadIdx.x; base0 < A; base0 += 256 * 8) {
+    int ev[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int a = base0 + 256 * u;
+      ev[u] = (a < A) ? __ldg(ids + a) : -1;
+    }
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int a = base0 + 256 * u;
+      count_packed(ev[u], all_lo, all_hi);
+      if (a < a0) count_packed(ev[u], pre_lo, pre_hi);
+    }
+  }
+  // unpack and reduce over the warp (fixed butterfly), then over warps through shared memory
+  int call[kOnePassMaxE], cpre[kOnePassMaxE];
+#pragma unroll
+  for (int e = 0; e < kOnePassMaxE; ++e) {
+    const uint32_t wa = e < 4 ? all_lo : all_hi, wp = e < 4 ? pre_lo : pre_hi;
+    call[e] = (int)((wa >> (8 * (e & 3))) & 0xffu);
+    cpre[e] = (int)((wp >> (8 * (e & 3))) & 0xffu);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      call[e] += __shfl_xor_sync(0xffffffffu, call[e], o);
+      cpre[e] += __shfl_xor_sync(0xffffffffu, cpre[e], o);
+    }
+  }
+  if (lane < kOnePassMaxE) {
+    int va = 0, vp = 0;
+#pragma unroll
+    for (int e = 0; e < kOnePassMaxE; ++e)
+      if (lane == e) { va = call[e]; vp = cpre[e]; }
+    s_all[warp][lane] = va;
+    s_pre[warp][lane] = vp;
+    s_own[warp][lane] = 0;
+  }
+  __syncthreads();
+  // own assignments: chunk `warp` of the CTA's range (<= 8 chunks of 32)
+  const int oa = a0 + warp * 32 + lane;
+  const int oe = (oa < a1) ? ids[oa] : -1;
+  const bool ook = oe >= 0 && oe < E;
+  const unsigned opeers = __match_any_sync(0xffffffffu, ook ? oe : -1);
+  if (ook && (opeers & lt) == 0) s_own[warp][oe] = __popc(opeers);
+  __syncthreads();
+  // 2. per expert: totals, kept, bases; offsets = exclusive scan of kept (one warp)
+  if (warp == 0) {
+    int total = 0, pre = 0;
+    if (lane < E) {
+      for (int w = 0; w < 8; ++w) {
+        total += s_all[w][lane];
+        pre += s_pre[w][lane];
+      }
+      int run = pre;                               // exclusive bases of this CTA's warps
+      for (int w = 0; w < 8; ++w) {
+        const int v = s_own[w][lane];
+        s_own[w][lane] = run;
+        run += v;
+      }
+    }
+    const int kept = (lane < E) ? ((cap > 0 && total > cap) ? cap : total) : 0;
+    int inc = kept;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int n = __shfl_up_sync(0xffffffffu, inc, o);
+      if (lane >= o) inc += n;
+    }
+    if (lane < E) {
+      s_off[lane] = inc - kept;
+      if (blockIdx.x == 0) {
+        counts[lane] = total;
+        offsets[lane] = inc - kept;
+      }
+    }
+    if (blockIdx.x == 0 && lane == E - 1) offsets[E] = inc;
+  }
+  __syncthreads();
+  // 3. stable ranks of this CTA's assignments
+  if (oa < a1) {
+    int row = -1;
+    if (ook) {
+      const int rank = s_own[warp][oe] + __popc(opeers & lt);
+      if (cap <= 0 || rank < cap) {
+        row = s_off[oe] + rank;
+        row_src[row] = oa;
+      }
+    }
+    inv[oa] = row;
+    s_row[oa - a0] = row;
+  }
+  __syncthreads();
+  // 4. copy: warp w copies tokens 4w .. 4w+3 of the CTA's 32; each lane keeps 4 tokens x 4
+  //    chunks (256 bytes) of loads in flight before it stores them to the expert rows
+  const int tw = blockIdx.x * kOnePassTokens + warp * 4;
+  int rows[4][kOnePassMaxK];
+#pragma unroll
+  for (int u = 0; u < 4; ++u)
+#pragma unroll
+    for (int jj = 0; jj < kOnePassMaxK; ++jj)
+      rows[u][jj] = (tw + u < T && jj < k) ? s_row[(warp * 4 + u) * k + jj] : -1;
+  int v = lane;
+  for (; v + 96 < nvec; v += 128) {
+    uint4 q[4][4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+        q[u][c] = (tw + u < T) ? __ldcs(x + (int64_t)(tw + u) * nvec + v + 32 * c)
+                               : make_uint4(0u, 0u, 0u, 0u);
+#pragma unroll
+    for (int u = 0; u < 4; ++u)
+#pragma unroll
+      for (int jj = 0; jj < kOnePassMaxK; ++jj) {
+        const int r = rows[u][jj];
+        if (r < 0) continue;
+        uint4* dst = xp + (int64_t)r * nvec + v;
+#pragma unroll
+        for (int c = 0; c < 4; ++c) dst[32 * c] = q[u][c];
+      }
+  }
+  for (; v < nvec; v += 32) {
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (tw + u >= T) break;
+      const uint4 q0 = __ldcs(x + (int64_t)(tw + u) * nvec + v);
+#pragma unroll
+      for (int jj = 0; jj < kOnePassMaxK; ++jj)
+        if (rows[u][jj] >= 0) xp[(int64_t)rows[u][jj] * nvec + v] = q0;
+    }
+  }
+}
+
 // One warp per token: copy x[t] (D elements of `esz` bytes) to each kept row.
 __global__ void __launch_bounds__(256)
 gather_tc_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_t* inv,
@@ -322,6 +490,16 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
   const int A = d.T * d.k;
   const int nblk = permute_blocks(d);
   const int E = d.E;
+  const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
+  const int nvec = d.D * esz / 16;
+  if (A > 0 && A <= kOnePassMaxItems && E <= kOnePassMaxE && d.k <= kOnePassMaxK) {
+    const int grid = (d.T + kOnePassTokens - 1) / kOnePassTokens;
+    permute_onepass_kernel<<<grid, 256, 0, s>>>(ids, d.T, d.k, E, cap,
+                                                static_cast<const uint4*>(x), nvec,
+                                                static_cast<uint4*>(x_perm), counts, offsets,
+                                                row_src, inv);
+    return cudaGetLastError();
+  }
   if (A <= kFusedMaxItems) {
     const size_t smem = ((size_t)33 * E + A) * sizeof(int);
     if (smem > 48 * 1024)
@@ -335,8 +513,6 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
         ids, A, E, cap, block_hist, offsets, row_src, inv);
   }
   if (nblk > 0) {
-    const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
-    const int nvec = d.D * esz / 16;
     const int blocks = (d.T * 32 + 255) / 256;
     gather_tc_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
                                             static_cast<uint4*>(x_perm));

@@ -1,0 +1,60 @@
+"""The multi-replica logic of bench.py on 2 gloo ranks (CPU): barrier, the max over ranks of
+the timed region, and the whole-job throughput (every rank's tokens over the slowest time)."""
+
+import os
+import socket
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+import bench
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    return port
+
+
+def _rank_main(rank, world, port, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        bench.barrier(world)
+        local_ms = 100.0 + 25.0 * rank          # rank 1 is the slower replica
+        total = bench.max_over_ranks(local_ms, world, torch.device("cpu"))
+        value = bench.job_throughput(4096, world, 10, total)
+        out[rank] = (total, value)
+        bench.barrier(world)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_two_replicas_agree_on_the_slowest_time_and_job_throughput():
+    world = 2
+    port = _free_port()
+    with mp.Manager() as mgr:
+        out = mgr.dict()
+        mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True,
+                           start_method="spawn")
+        res = dict(out)
+    assert res[0] == res[1]
+    total, value = res[0]
+    assert total == 125.0
+    assert value == pytest.approx(4096 * 2 * 10 / 0.125)
+
+
+def test_single_process_needs_no_process_group():
+    assert bench.max_over_ranks(3.5, 1, torch.device("cpu")) == 3.5
+    bench.barrier(1)
+    assert bench.job_throughput(4096, 1, 100, 250.0) == pytest.approx(4096 * 100 / 0.25)
+
+
+def test_reference_arm_runs_on_rank_zero_only():
+    class A:
+        steps, warmup, workload, tokens, ref_budget = 1, 3, "mixtral", 0, 1.0
+    assert bench.run_reference(A(), rank=1, world=2) is None     # returns without work
