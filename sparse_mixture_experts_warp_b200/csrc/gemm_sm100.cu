@@ -39,6 +39,7 @@
 // the device error word and makes the CTA drain its in-flight copies and MMAs and exit.
 #include <cuda.h>
 #include <stdlib.h>
+#include <string.h>
 
 #include <mutex>
 
@@ -48,12 +49,8 @@ namespace moe {
 namespace {
 
 constexpr int BM = 128;
-constexpr int BK = 64;                      // 64 bf16 = 128 bytes = one swizzle-atom row
 constexpr int MMA_N = 256;
 constexpr int MMA_K = 16;
-constexpr int STAGES = 4;
-constexpr int A_BYTES = BM * BK * 2;        // 16 KB
-constexpr int B_BYTES = MMA_N * BK * 2;     // 32 KB
 constexpr int ACC_COLS = MMA_N;             // fp32 accumulator columns per tile
 constexpr int TMEM_COLS = 2 * ACC_COLS;     // two accumulators
 constexpr uint64_t TIMEOUT_NS = 2000000000ull;   // 2 s per wait
@@ -131,14 +128,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
-// Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row core groups 1024 B apart.
-__device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr) {
+// Shared-memory matrix descriptor, K-major, rows of KB bf16 (KB = 64: 128-byte swizzle, 8-row
+// core groups 1024 B apart; KB = 32: 64-byte swizzle, groups 512 B apart).
+template <int KB>
+__device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);        // start address
   d |= (uint64_t)1 << 16;                           // leading byte offset (unused here), 16 B
-  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset: 8 rows x 128 B
+  d |= (uint64_t)((8 * KB * 2) >> 4) << 32;         // stride byte offset: 8 rows
   d |= (uint64_t)1 << 46;                           // descriptor version for tcgen05
-  d |= (uint64_t)2 << 61;                           // 128-byte swizzle
+  d |= (uint64_t)(KB == 64 ? 2 : 4) << 61;          // 128-byte or 64-byte swizzle
   return d;
 }
 
@@ -188,14 +187,16 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 // HALVES = 2: 256-row tiles made of two M=128 MMAs that share every B stage (a third fewer
 //             L2->SMEM bytes per FLOP), 3-stage ring of 64 KB, one 512-column accumulator set,
 //             8 epilogue warps; a tile with <= 128 live rows loads and multiplies one half only.
-template <int EPI, int HALVES>
+template <int EPI, int HALVES, int KB, int NSTAGES>
 __global__ void __launch_bounds__(64 + 128 * HALVES, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
   constexpr int TBM = BM * HALVES;
-  constexpr int TSTAGES = HALVES == 1 ? STAGES : 3;
-  constexpr int TA_BYTES = TBM * BK * 2;
+  constexpr int TSTAGES = NSTAGES;
+  constexpr int HA_BYTES = BM * KB * 2;              // one 128-row half of A per stage
+  constexpr int TA_BYTES = HALVES * HA_BYTES;
+  constexpr int TB_BYTES = MMA_N * KB * 2;           // B per stage
   constexpr int NBUF = HALVES == 1 ? 2 : 1;          // TMEM accumulator buffers
   constexpr int BUF_COLS = HALVES * ACC_COLS;        // columns per buffer
   constexpr int N_EPI = 4 * HALVES;                  // epilogue warps
@@ -204,7 +205,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + TSTAGES * TA_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TSTAGES * (TA_BYTES + B_BYTES));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TSTAGES * (TA_BYTES + TB_BYTES));
   uint64_t* full = bars;
   uint64_t* empty = bars + TSTAGES;
   uint64_t* tfull = bars + 2 * TSTAGES;
@@ -275,7 +276,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = tile_pre[p.G];
-  const int nkb = (p.K + BK - 1) / BK;
+  const int nkb = (p.K + KB - 1) / KB;
 
   if (warp == 0) {
     if (lane == 0) {
@@ -300,16 +301,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             ok = false;
             break;
           }
-          mbar_expect_tx(&full[stage], (two ? 2 * A_BYTES : A_BYTES) + B_BYTES);
-          const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * B_BYTES;
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * BK, a_row);
-          if (two) tma_load_2d(a_dst + A_BYTES, &tmA, &full[stage], kb * BK, a_row + BM);
+          mbar_expect_tx(&full[stage], (two ? 2 * HA_BYTES : HA_BYTES) + TB_BYTES);
+          const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
+          tma_load_2d(a_dst, &tmA, &full[stage], kb * KB, a_row);
+          if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kb * KB, a_row + BM);
           if (EPI == EPI_SWIGLU) {
-            tma_load_2d(b_dst, &tmB0, &full[stage], kb * BK, b_row);
-            tma_load_2d(b_dst + B_BYTES / 2, &tmB1, &full[stage], kb * BK, b_row);
+            tma_load_2d(b_dst, &tmB0, &full[stage], kb * KB, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kb * KB, b_row);
           } else {
-            tma_load_2d(b_dst, &tmB0, &full[stage], kb * BK, b_row);
-            tma_load_2d(b_dst + B_BYTES / 2, &tmB0, &full[stage], kb * BK, b_row + 128);
+            tma_load_2d(b_dst, &tmB0, &full[stage], kb * KB, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB0, &full[stage], kb * KB, b_row + 128);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -356,14 +357,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           tc_fence_after();
-          const uint32_t a0 = sA + stage * TA_BYTES, b0 = sB + stage * B_BYTES;
+          const uint32_t a0 = sA + stage * TA_BYTES, b0 = sB + stage * TB_BYTES;
 #pragma unroll
-          for (int k = 0; k < BK / MMA_K; ++k) {
-            const uint64_t bdesc = sdesc_sw128(b0 + k * MMA_K * 2);
+          for (int k = 0; k < KB / MMA_K; ++k) {
+            const uint64_t bdesc = sdesc<KB>(b0 + k * MMA_K * 2);
             const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
-            umma_bf16(d_tmem, sdesc_sw128(a0 + k * MMA_K * 2), bdesc, accum);
+            umma_bf16(d_tmem, sdesc<KB>(a0 + k * MMA_K * 2), bdesc, accum);
             if (two)
-              umma_bf16(d_tmem + ACC_COLS, sdesc_sw128(a0 + A_BYTES + k * MMA_K * 2), bdesc,
+              umma_bf16(d_tmem + ACC_COLS, sdesc<KB>(a0 + HA_BYTES + k * MMA_K * 2), bdesc,
                         accum);
           }
           umma_commit(&empty[stage]);       // frees the stage once these MMAs have read it
@@ -421,6 +422,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           tmem_ld32(taddr + c, gv);
           tmem_ld32(taddr + 128 + c, uv);
           tmem_wait_ld();
+          if (c == 96) {                     // last TMEM read of the tile: release the buffer
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
           const int col = n_idx * p.n_out_tile + c;
           if (valid && col < p.N) {
             uint32_t pk[16];
@@ -445,6 +450,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           uint32_t v[32];
           tmem_ld32(taddr + c, v);
           tmem_wait_ld();
+          if (c == MMA_N - 32) {             // last TMEM read of the tile: release the buffer
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
           const int col = n_idx * p.n_out_tile + c;
           if (valid && col < p.N) {
             uint32_t pk[16];
@@ -465,8 +474,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       }
-      tc_fence_before();
-      mbar_arrive(&tempty[acc]);
     }
   }
   __syncwarp();
@@ -502,29 +509,34 @@ EncodeTiledFn encode_fn() {
 }
 
 // 2D bf16 tensor [rows, cols] row-major; box = 64 columns x box_rows rows, 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows) {
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
+              int kb) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[2] = {cols, rows};
   const cuuint64_t strides[1] = {cols * 2};
-  const cuuint32_t box[2] = {(cuuint32_t)BK, box_rows};
+  const cuuint32_t box[2] = {(cuuint32_t)kb, box_rows};
   const cuuint32_t estr[2] = {1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box,
-             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             kb == 64 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Tile height in 128-row halves: 256-row tiles (a third fewer L2 bytes per FLOP) for every
-// epilogue; measured on the Mixtral layer shape they beat 128-row tiles for both the gate/up and
-// the down projection.  MOE_GEMM_HALVES=1 selects the 128-row tile with its double TMEM buffer
-// (kept for comparison measurements; both heights are tested).
-int gemm_halves(int epi) {
-  (void)epi;
-  static int h = [] {
-    const char* v = getenv("MOE_GEMM_HALVES");
-    return (v && v[0] == '1') ? 1 : 2;
+// Tile shape.  Default: 256-row tiles (two M=128 MMAs sharing each B stage: a third fewer L2
+// bytes per FLOP than 128-row tiles) with 64-element k-blocks in a 3-stage ring.
+// MOE_GEMM_TILE selects another shape for comparison measurements (all are tested):
+//   "128"      128-row tiles, 4 stages, double TMEM buffer;
+//   "256k32"   256-row tiles with 32-element k-blocks (64-byte swizzle) in a 6-7 stage ring.
+enum GemmTile { TILE_128 = 0, TILE_256 = 1, TILE_256_K32 = 2 };
+GemmTile gemm_tile() {
+  static GemmTile t = [] {
+    const char* v = getenv("MOE_GEMM_TILE");
+    if (v && !strcmp(v, "128")) return TILE_128;
+    if (v && !strcmp(v, "256k32")) return TILE_256_K32;
+    return TILE_256;
   }();
-  return h;
+  return t;
 }
 
 int sm_count() {
@@ -534,14 +546,32 @@ int sm_count() {
   return n > 0 ? n : 148;
 }
 
-template <int EPI, int HALVES>
+template <int EPI, int HALVES, int KB, int NSTAGES>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int grid, size_t smem, cudaStream_t s) {
-  cudaError_t e = cudaFuncSetAttribute(grouped_gemm_kernel<EPI, HALVES>,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kern = grouped_gemm_kernel<EPI, HALVES, KB, NSTAGES>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
   if (e != cudaSuccess) return e;
-  grouped_gemm_kernel<EPI, HALVES><<<grid, 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
+  kern<<<grid, 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
   return cudaGetLastError();
+}
+
+template <int HALVES, int KB, int NSTAGES>
+cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
+                       const CUtensorMap& b1, const GemmParams& p, int grid, size_t smem,
+                       cudaStream_t s) {
+  switch (epi) {
+    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    case EPI_RELU: return launch_epi<EPI_RELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    default: return launch_epi<EPI_NONE, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+  }
+}
+
+// Dynamic shared memory of one configuration (ring + barriers + group tables + alignment).
+size_t gemm_smem(int halves, int kb, int nstages, int n_groups) {
+  const size_t ring = (size_t)nstages * ((size_t)halves * BM * kb * 2 + (size_t)MMA_N * kb * 2);
+  return 1024 + ring + (2 * nstages + 5) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
 }
 
 }  // namespace
@@ -552,13 +582,6 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
   alignas(64) CUtensorMap ta, tb0, tb1;
   const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
-  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&tb0, B0, brows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
-  if (epi == EPI_SWIGLU) {
-    if (!make_map(&tb1, B1, brows, (uint64_t)K, 128)) return cudaErrorInvalidValue;
-  } else {
-    tb1 = tb0;
-  }
   GemmParams p;
   p.offsets = offsets;
   p.out = static_cast<__nv_bfloat16*>(out);
@@ -570,24 +593,29 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.K = K;
   p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
   p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
-  const int halves = gemm_halves(epi);
+  const GemmTile tile = gemm_tile();
+  const int halves = tile == TILE_128 ? 1 : 2;
+  const int kb = tile == TILE_256_K32 ? 32 : 64;
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
+  if (!make_map(&tb0, B0, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
+  if (epi == EPI_SWIGLU) {
+    if (!make_map(&tb1, B1, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
+  } else {
+    tb1 = tb0;
+  }
   const int tbm = BM * halves;
   const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
-  const int tstages = halves == 1 ? STAGES : 3;
-  const size_t smem = 1024 + (size_t)tstages * ((size_t)tbm * BK * 2 + B_BYTES) +
-                      (2 * tstages + 5) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
-  if (halves == 2) {
-    switch (epi) {
-      case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 2>(ta, tb0, tb1, p, grid, smem, s);
-      case EPI_RELU: return launch_epi<EPI_RELU, 2>(ta, tb0, tb1, p, grid, smem, s);
-      default: return launch_epi<EPI_NONE, 2>(ta, tb0, tb1, p, grid, smem, s);
-    }
-  }
-  switch (epi) {
-    case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, 1>(ta, tb0, tb1, p, grid, smem, s);
-    case EPI_RELU: return launch_epi<EPI_RELU, 1>(ta, tb0, tb1, p, grid, smem, s);
-    default: return launch_epi<EPI_NONE, 1>(ta, tb0, tb1, p, grid, smem, s);
+  constexpr size_t kMaxSmem = 232448;          // 227 KB of dynamic shared memory per block
+  switch (tile) {
+    case TILE_128:
+      return launch_cfg<1, 64, 4>(epi, ta, tb0, tb1, p, grid, gemm_smem(1, 64, 4, n_groups), s);
+    case TILE_256_K32:
+      if (gemm_smem(2, 32, 7, n_groups) <= kMaxSmem)
+        return launch_cfg<2, 32, 7>(epi, ta, tb0, tb1, p, grid, gemm_smem(2, 32, 7, n_groups), s);
+      return launch_cfg<2, 32, 6>(epi, ta, tb0, tb1, p, grid, gemm_smem(2, 32, 6, n_groups), s);
+    default:
+      return launch_cfg<2, 64, 3>(epi, ta, tb0, tb1, p, grid, gemm_smem(2, 64, 3, n_groups), s);
   }
 }
 

@@ -85,13 +85,15 @@ def test_grouped_gemm_repeatable():
     assert torch.equal(y1[:n], y[:n])
 
 
-def test_grouped_gemm_128_row_tiles_in_subprocess():
-    """The 128-row tile variant (double TMEM buffer) is selected per process by
-    MOE_GEMM_HALVES=1; run this file's ragged cases under it in a child process."""
+@pytest.mark.parametrize("tile", ["128", "256k32"])
+def test_grouped_gemm_other_tiles_in_subprocess(tile):
+    """The other tile shapes (128-row tiles with a double TMEM buffer; 256-row tiles with
+    32-element k-blocks) are selected per process by MOE_GEMM_TILE; run this file's ragged
+    cases under each in a child process."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, MOE_GEMM_HALVES="1")
+    env = dict(os.environ, MOE_GEMM_TILE=tile)
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__,
                         "-k", "ragged or repeatable"],
                        env=env, capture_output=True, text=True, timeout=600)
