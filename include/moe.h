@@ -231,6 +231,15 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
  * *code receives the raw word (0 = none).  Returns MOE_OK when the word was 0. */
 moe_status_t moe_get_device_error(moe_stream_t stream, int32_t* code);
 
+/* Test hook for the bounded device waits (failure detection without a GPU fault).  fault = 1:
+ * in every following bf16 expert projection, CTA 0 of the grouped GEMM arms its first ring
+ * stage without loading it, so the MMA issuer's bounded wait runs out (about 2 s); the CTA
+ * records MOE_ERR_TIMEOUT in the device error word, drains what is in flight, frees its tensor
+ * memory and exits, the other CTAs finish, and the context stays usable.  fault = 0 restores
+ * normal operation.  Not for production use: the affected call's outputs are incomplete.
+ * Host state only (not thread-safe); returns MOE_ERR_INVALID_ARG for other values. */
+moe_status_t moe_debug_inject(int32_t fault);
+
 #ifdef __cplusplus
 }
 #endif

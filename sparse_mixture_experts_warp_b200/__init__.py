@@ -95,6 +95,7 @@ _SIGS = {
     "moe_layer_forward": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                           ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
+    "moe_debug_inject": ([_I32], ctypes.c_int),
 }
 
 
@@ -313,6 +314,19 @@ def moe_layer_forward(d, x, Wg, sel_bias, W_gate, W_up, W_down, Ws_gate, Ws_up, 
 
 
 def get_device_error(stream=None) -> int:
+    """Synchronises the stream and returns (and clears) the raw device error word."""
     code = _I32()
     lib().moe_get_device_error(_stream(stream), ctypes.byref(code))
     return code.value
+
+
+def device_error_status(stream=None):
+    """(moe_status_t, raw word) of moe_get_device_error."""
+    code = _I32()
+    st = lib().moe_get_device_error(_stream(stream), ctypes.byref(code))
+    return st, code.value
+
+
+def debug_inject(fault: int):
+    """Test hook of the bounded device waits (see moe_debug_inject in include/moe.h)."""
+    _check("moe_debug_inject", lib().moe_debug_inject(fault))

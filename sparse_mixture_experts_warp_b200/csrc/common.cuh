@@ -59,6 +59,9 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s);
 
+// Test hook of the grouped GEMM's bounded waits (see moe_debug_inject).
+void set_gemm_fault(int kind);
+
 // ffn_simt.cu (fp32 experts)
 cudaError_t launch_ffn_up_f32(int act, const float* a, int64_t a_rows, int D, int F,
                               const int32_t* offsets, int n_groups, const float* Wgate,

@@ -70,6 +70,7 @@ struct GemmParams {
   int G, N, K;
   int n_out_tile;           // output columns per tile
   int nt;                   // n-tiles per group
+  int fault;                // test hook: 1 = CTA 0 arms its first stage without loading it
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -102,14 +103,17 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// Bounded wait for the phase of parity `parity` to complete.  Returns false when it gave up
-// (time limit, or another role already aborted).
+// Bounded wait for the phase of parity `parity` to complete.  Returns false when it gave up:
+// on its time limit (which records `code` and raises the CTA's abort flag) or, when
+// honor_abort, as soon as another role has aborted.  Drain waits pass honor_abort = false so
+// that they keep waiting (bounded) for work already in flight.
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                       int* err, int code, uint64_t limit) {
+                                       int* err, int code, uint64_t limit,
+                                       bool honor_abort = true) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = gtimer();
   while (!mbar_try_wait(bar, parity)) {
-    if (*abort_flag) return false;
+    if (honor_abort && *abort_flag) return false;
     if (gtimer() - t0 > limit) {
       *abort_flag = 1;
       atomicCAS(err, 0, code);
@@ -302,6 +306,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           mbar_expect_tx(&full[stage], (two ? 2 * HA_BYTES : HA_BYTES) + TB_BYTES);
+          if (p.fault == 1 && blockIdx.x == 0 && tile == (int)blockIdx.x && kb == 0) {
+            // test hook: the stage is armed but never loaded, so the MMA issuer's bounded
+            // wait on it runs out; nothing is in flight for this stage
+            issued |= 1u << stage;
+            issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+            if (++stage == TSTAGES) {
+              stage = 0;
+              phase ^= 1u;
+            }
+            continue;
+          }
           const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
           tma_load_2d(a_dst, &tmA, &full[stage], kb * KB, a_row);
           if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kb * KB, a_row + BM);
@@ -325,7 +340,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         for (int s = 0; s < TSTAGES; ++s)
           if (issued & (1u << s))
             mbar_wait(&full[s], (issued_par >> s) & 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
-                      DRAIN_NS);
+                      DRAIN_NS, /*honor_abort=*/false);
       }
     }
   } else if (warp == 1) {
@@ -377,7 +392,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       // all MMAs issued by this thread complete before the CTA releases TMEM
       umma_commit(drain);
-      mbar_wait(drain, 0u, abort_flag, p.err, DEVERR_TIMEOUT_MMA, ok ? TIMEOUT_NS : DRAIN_NS);
+      mbar_wait(drain, 0u, abort_flag, p.err, DEVERR_TIMEOUT_MMA, ok ? TIMEOUT_NS : DRAIN_NS,
+                /*honor_abort=*/false);
     }
   } else {
     // ---------------- epilogue (warps 2 .. 2 + N_EPI) ----------------
@@ -529,6 +545,8 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 //   "128"      128-row tiles, 4 stages, double TMEM buffer;
 //   "256k32"   256-row tiles with 32-element k-blocks (64-byte swizzle) in a 6-7 stage ring.
 enum GemmTile { TILE_128 = 0, TILE_256 = 1, TILE_256_K32 = 2 };
+
+int g_gemm_fault = 0;       // set through moe_debug_inject (tests of the bounded waits)
 GemmTile gemm_tile() {
   static GemmTile t = [] {
     const char* v = getenv("MOE_GEMM_TILE");
@@ -593,6 +611,7 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.K = K;
   p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
   p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
+  p.fault = g_gemm_fault;
   const GemmTile tile = gemm_tile();
   const int halves = tile == TILE_128 ? 1 : 2;
   const int kb = tile == TILE_256_K32 ? 32 : 64;
@@ -618,5 +637,7 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
       return launch_cfg<2, 64, 3>(epi, ta, tb0, tb1, p, grid, gemm_smem(2, 64, 3, n_groups), s);
   }
 }
+
+void set_gemm_fault(int kind) { g_gemm_fault = kind; }
 
 }  // namespace moe

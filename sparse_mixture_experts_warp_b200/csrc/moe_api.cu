@@ -389,6 +389,12 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.f, v.stats, stream);
 }
 
+moe_status_t moe_debug_inject(int32_t fault) {
+  if (fault != 0 && fault != 1) return MOE_ERR_INVALID_ARG;
+  set_gemm_fault(fault);
+  return MOE_OK;
+}
+
 moe_status_t moe_get_device_error(moe_stream_t stream, int32_t* code) {
   int* w = device_error_word();
   if (!w) return MOE_ERR_CUDA;
