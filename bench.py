@@ -43,6 +43,7 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "grouped_gemm_traffic.json")
 GEMM_SRC = os.path.join(ROOT, "sparse_mixture_experts_warp_b200", "csrc", "gemm_sm100.cu")
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 STAGES = ["route", "permute", "expert_up", "expert_down", "combine", "stats"]
+# "expert_down" includes the shared experts (both projections) when the workload has them.
 
 
 # ------------------------------------------------------------------ helpers ----
@@ -170,16 +171,6 @@ def job_throughput(tokens_per_rank, world, steps, max_total_ms):
     return tokens_per_rank * world * steps / (max_total_ms / 1e3)
 
 
-def launches_per_step(w):
-    """Kernels the library launches per layer step (its own kernels only)."""
-    n = 2 + (1 if w.select == "expert" else 0)            # router, importance reduce, ec select
-    n += 3 if w.select == "expert" else 4                  # permute
-    n += 2                                                 # grouped GEMM up + down
-    n += (1 + 2 * w.n_shared) if w.n_shared else 0         # shared experts (+ offsets kernel)
-    n += 2                                                 # combine, stats
-    return n
-
-
 def stage_work(w, rows_exec):
     """Algorithmic bytes (HBM-bound stages) or FLOPs (GEMMs) per launch; rows_exec = A_exec."""
     es = 2 if w.dtype == "bf16" else 4
@@ -193,9 +184,9 @@ def stage_work(w, rows_exec):
         # ids read; x read once; x_perm written; row_src and inv written
         "permute": ("hbm", T * K * 4 + T * D * es + A * D * es + A * 4 + T * K * 4),
         "expert_up": ("tensor", 2.0 * A * D * F * n_up),
-        "expert_down": ("tensor", 2.0 * A * F * D),
+        "expert_down": ("tensor", 2.0 * A * F * D + w.n_shared * 2.0 * T * D * w.F_shared * 3),
         # expert rows read once; out written once; inv and gates read
-        "combine": ("hbm", A * D * es + T * D * es + T * K * 8),
+        "combine": ("hbm", A * D * es + (1 + w.n_shared) * T * D * es + T * K * 8),
         "stats": ("hbm", E * 16),
     }
 
@@ -215,8 +206,6 @@ def run_cuda(args, rank, world, local):
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     w = workload_of(args)
-    if w.n_shared:
-        raise SystemExit("the step benchmark covers workloads without shared experts")
     inp = make_inputs(w, seed=rank, device=dev)
     d = M.desc_of(w)
     ws = M.empty_workspace(d, dev)
@@ -224,6 +213,12 @@ def run_cuda(args, rank, world, local):
     scratch = v["scratch"]
     out = torch.empty_like(inp.x)
     stream = torch.cuda.current_stream(dev)
+    if w.n_shared:
+        # shared experts: one group over all T tokens, SwiGLU of width F_shared
+        d_sh = M.desc_of(w)
+        d_sh.act = M.SWIGLU
+        sh_off = torch.tensor([0, w.T], dtype=torch.int32, device=dev)
+        h_sh = torch.empty(w.T, w.F_shared, dtype=inp.x.dtype, device=dev)
 
     def step(ev=None):
         M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
@@ -239,9 +234,13 @@ def run_cuda(args, rank, world, local):
         if ev is not None:
             ev[3].record(stream)
         M.moe_expert_down(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], stream)
+        for i in range(w.n_shared):
+            M.moe_expert_ffn(d_sh, 1, w.F_shared, inp.x, sh_off, inp.Ws_gate[i], inp.Ws_up[i],
+                             inp.Ws_down[i], h_sh, v["y_shared"][i], stream)
         if ev is not None:
             ev[4].record(stream)
-        M.moe_combine(d, v["y"], v["inv"], v["gates"], None, out, stream)
+        M.moe_combine(d, v["y"], v["inv"], v["gates"], v["y_shared"] if w.n_shared else None,
+                      out, stream)
         if ev is not None:
             ev[5].record(stream)
         M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
@@ -262,11 +261,13 @@ def run_cuda(args, rank, world, local):
         barrier(world)
         torch.cuda.synchronize(dev)
         with ClockSampler(nvml_index) as clk:
+            n0 = M.kernel_launches()
             start.record(stream)
             for i in range(args.steps):
                 evs[i][0].record(stream)
                 step(evs[i])
             end.record(stream)
+            launches = M.kernel_launches() - n0
             torch.cuda.synchronize(dev)
         barrier(world)
         total = start.elapsed_time(end)
@@ -274,12 +275,12 @@ def run_cuda(args, rank, world, local):
         for i in range(args.steps):
             for j, s in enumerate(STAGES):
                 per_stage[s] += evs[i][j].elapsed_time(evs[i][j + 1])
-        return total, {s: per_stage[s] / args.steps for s in STAGES}, clk
+        return total, {s: per_stage[s] / args.steps for s in STAGES}, clk, launches
 
-    total_ms, per_stage, clk = timed()
+    total_ms, per_stage, clk, launches = timed()
     remeasured = False
     if clk.rejected():
-        total_ms, per_stage, clk = timed()
+        total_ms, per_stage, clk, launches = timed()
         remeasured = True
     total_ms = max_over_ranks(total_ms, world, dev)
     ms_per_step = total_ms / args.steps
@@ -367,7 +368,7 @@ def run_cuda(args, rank, world, local):
                 "ms_per_step": round(e2e_ms / args.steps, 4),
                 "h2d_bytes_per_step": x_host.numel() * x_host.element_size(),
                 "d2h_bytes_per_step": out_host.numel() * out_host.element_size()},
-        "gpu_launches": launches_per_step(w) * args.steps,
+        "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if remeasured:
@@ -488,7 +489,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=200)
     ap.add_argument("--warmup", type=int, default=10)
-    ap.add_argument("--workload", default="mixtral", choices=["mixtral", "switch", "ec"])
+    ap.add_argument("--workload", default="mixtral", choices=["mixtral", "switch", "v3", "ec"])
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch size T (smaller cases for profiling)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])

@@ -231,6 +231,10 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
  * *code receives the raw word (0 = none).  Returns MOE_OK when the word was 0. */
 moe_status_t moe_get_device_error(moe_stream_t stream, int32_t* code);
 
+/* Number of kernels this library has enqueued since it was loaded (all entry points, all
+ * streams).  Host counter; useful to attribute launches in a timed region. */
+int64_t moe_kernel_launches(void);
+
 /* Test hook for the bounded device waits (failure detection without a GPU fault).  fault = 1:
  * in every following bf16 expert projection, CTA 0 of the grouped GEMM arms its first ring
  * stage without loading it, so the MMA issuer's bounded wait runs out (about 2 s); the CTA

@@ -96,6 +96,7 @@ _SIGS = {
                           ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
     "moe_debug_inject": ([_I32], ctypes.c_int),
+    "moe_kernel_launches": ([], ctypes.c_int64),
 }
 
 
@@ -325,6 +326,11 @@ def device_error_status(stream=None):
     code = _I32()
     st = lib().moe_get_device_error(_stream(stream), ctypes.byref(code))
     return st, code.value
+
+
+def kernel_launches() -> int:
+    """Kernels the library has enqueued since it was loaded."""
+    return int(lib().moe_kernel_launches())
 
 
 def debug_inject(fault: int):

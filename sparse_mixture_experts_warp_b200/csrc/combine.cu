@@ -198,20 +198,20 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
     const uint4* yy = static_cast<const uint4*>(y);
     uint4* oo = static_cast<uint4*>(out);
     if (d.dtype == MOE_BF16) {
-      if (K == 1) combine_small_k_kernel<true, 1><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
-      else combine_small_k_kernel<true, 2><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) combine_small_k_kernel<true, 1><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      else combine_small_k_kernel<true, 2><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
     } else {
-      if (K == 1) combine_small_k_kernel<false, 1><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
-      else combine_small_k_kernel<false, 2><<<blocks, kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) combine_small_k_kernel<false, 1><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      else combine_small_k_kernel<false, 2><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
     }
     return cudaGetLastError();
   }
   if (d.dtype == MOE_BF16)
-    combine_kernel<true><<<blocks, kWarps * 32, 0, s>>>(
+    combine_kernel<true><<<counted(blocks), kWarps * 32, 0, s>>>(
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
         K, nvec, static_cast<uint4*>(out));
   else
-    combine_kernel<false><<<blocks, kWarps * 32, 0, s>>>(
+    combine_kernel<false><<<counted(blocks), kWarps * 32, 0, s>>>(
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
         K, nvec, static_cast<uint4*>(out));
   return cudaGetLastError();
@@ -221,7 +221,7 @@ cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance, float* f,
                                  moe_stats_t* stats, cudaStream_t s) {
   const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
-  stats_kernel<<<1, 256, 0, s>>>(counts, offsets, importance, d.E, n_routes, d.aux_alpha, f,
+  stats_kernel<<<counted(1), 256, 0, s>>>(counts, offsets, importance, d.E, n_routes, d.aux_alpha, f,
                                  stats);
   return cudaGetLastError();
 }

@@ -23,21 +23,33 @@ int* device_error_word();
 
 inline bool is_aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
+// Kernels this library has enqueued since it was loaded (every launch site passes its grid
+// through counted()).
+void note_launch();
+template <typename G>
+inline G counted(G grid) {
+  note_launch();
+  return grid;
+}
+
 // ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
 
 // route.cu
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
                                        float* logits, float* imp_partials, int* n_partials,
-                                       cudaStream_t s);
+                                       float* lpart, cudaStream_t s);
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, int* n_partials, cudaStream_t s);
+                                        float* imp_partials, int* n_partials, float* lpart,
+                                        cudaStream_t s);
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s);
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
                                      float* importance, cudaStream_t s);
 int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer (upper bound)
+bool router_uses_gemm(const moe_desc_t& d);
+size_t router_gemm_scratch_bytes(const moe_desc_t& d);   // partial logits of the GEMM router
 
 // Streaming multiprocessors of the current device.
 int num_sms();
@@ -54,10 +66,16 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
                                          cudaStream_t s);
 
 // gemm_sm100.cu (bf16 grouped GEMM on tcgen05)
-enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2 };
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3 };
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s);
+
+// Router product on the same engine: one group of T rows, N = E, fp32 partial logits of
+// ksplit k-ranges in partials[ksplit][T][E] (E % 32 == 0, E <= 256).
+int router_gemm_splits(int T, int D);
+cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg, int E,
+                                    float* partials, int ksplit, cudaStream_t s);
 
 // Test hook of the grouped GEMM's bounded waits (see moe_debug_inject).
 void set_gemm_fault(int kind);

@@ -71,7 +71,7 @@ cudaError_t launch_ffn_up_f32(int act, const float* a, int64_t a_rows, int D, in
   const size_t smem = (size_t)D * sizeof(float);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(ffn_up_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  ffn_up_f32_kernel<<<(unsigned)a_rows, 128, smem, s>>>(a, D, F, offsets, n_groups, Wgate, Wup,
+  ffn_up_f32_kernel<<<counted((unsigned)a_rows), 128, smem, s>>>(a, D, F, offsets, n_groups, Wgate, Wup,
                                                         act, h);
   return cudaGetLastError();
 }
@@ -83,7 +83,7 @@ cudaError_t launch_ffn_down_f32(const float* h, int64_t a_rows, int D, int F,
   const size_t smem = (size_t)F * sizeof(float);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(ffn_down_f32_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-  ffn_down_f32_kernel<<<(unsigned)a_rows, 128, smem, s>>>(h, D, F, offsets, n_groups, Wdown, y);
+  ffn_down_f32_kernel<<<counted((unsigned)a_rows), 128, smem, s>>>(h, D, F, offsets, n_groups, Wdown, y);
   return cudaGetLastError();
 }
 

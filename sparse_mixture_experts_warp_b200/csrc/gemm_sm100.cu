@@ -71,6 +71,9 @@ struct GemmParams {
   int n_out_tile;           // output columns per tile
   int nt;                   // n-tiles per group
   int fault;                // test hook: 1 = CTA 0 arms its first stage without loading it
+  int ksplit;               // k-range splits (EPI_F32 only; 1 otherwise)
+  int kchunk;               // k-blocks per split
+  int64_t split_stride;     // EPI_F32: elements between the partial outputs of two splits
 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -253,14 +256,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // group row starts and the tile prefix (tiles of group g = ceil(rows_g / BM) * nt)
     int carry = 0;
     if (lane == 0) {
-      grp_off[0] = p.offsets[0];
+      grp_off[0] = p.offsets ? p.offsets[0] : 0;
       tile_pre[0] = 0;
     }
     for (int g0 = 0; g0 < p.G; g0 += 32) {
       const int g = g0 + lane;
       int tiles = 0;
       if (g < p.G) {
-        const int lo = p.offsets[g], hi = p.offsets[g + 1];
+        // no offsets array: one group of all allocated rows
+        const int lo = p.offsets ? p.offsets[g] : 0;
+        const int hi = p.offsets ? p.offsets[g + 1] : (int)p.rows;
         const int m = hi > lo ? hi - lo : 0;
         tiles = ((m + TBM - 1) / TBM) * p.nt;
         grp_off[g + 1] = hi;
@@ -280,6 +285,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = tile_pre[p.G];
+  const int total_all = total * p.ksplit;          // k-splits are the slowest tile index
   const int nkb = (p.K + KB - 1) / KB;
 
   if (warp == 0) {
@@ -290,7 +296,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t issued = 0, issued_par = 0;     // per stage: has a load, parity of the last one
       bool ok = true;
       int g = 0;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
+        const int split = t / total, tile = t - split * total;
+        if (tile < tile_pre[g]) g = 0;
         while (tile >= tile_pre[g + 1]) ++g;
         const int m = grp_off[g + 1] - grp_off[g];
         const int mt = (m + TBM - 1) / TBM;
@@ -299,14 +307,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int a_row = grp_off[g] + m_idx * TBM;
         const int b_row = g * p.N + n_idx * p.n_out_tile;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
-        for (int kb = 0; kb < nkb; ++kb) {
+        const int kb0 = split * p.kchunk, kb1 = min(nkb, kb0 + p.kchunk);
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
                          TIMEOUT_NS)) {
             ok = false;
             break;
           }
           mbar_expect_tx(&full[stage], (two ? 2 * HA_BYTES : HA_BYTES) + TB_BYTES);
-          if (p.fault == 1 && blockIdx.x == 0 && tile == (int)blockIdx.x && kb == 0) {
+          if (p.fault == 1 && blockIdx.x == 0 && t == (int)blockIdx.x && kb == kb0) {
             // test hook: the stage is armed but never loaded, so the MMA issuer's bounded
             // wait on it runs out; nothing is in flight for this stage
             issued |= 1u << stage;
@@ -350,12 +359,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t phase = 0;
       bool ok = true;
       int it = 0, g = 0;
-      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x, ++it) {
+        const int split = t / total, tile = t - split * total;
+        if (tile < tile_pre[g]) g = 0;
         while (tile >= tile_pre[g + 1]) ++g;
         const int m = grp_off[g + 1] - grp_off[g];
         const int mt = (m + TBM - 1) / TBM;
         const int m_idx = (tile - tile_pre[g]) % mt;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
+        const int kb0 = split * p.kchunk, kb1 = min(nkb, kb0 + p.kchunk);
         const int acc = it % NBUF;
         const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
@@ -365,7 +377,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + (uint32_t)(acc * BUF_COLS);
-        for (int kb = 0; kb < nkb; ++kb) {
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!mbar_wait(&full[stage], phase, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
                          TIMEOUT_NS)) {
             ok = false;
@@ -376,7 +388,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
 #pragma unroll
           for (int k = 0; k < KB / MMA_K; ++k) {
             const uint64_t bdesc = sdesc<KB>(b0 + k * MMA_K * 2);
-            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+            const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
             umma_bf16(d_tmem, sdesc<KB>(a0 + k * MMA_K * 2), bdesc, accum);
             if (two)
               umma_bf16(d_tmem + ACC_COLS, sdesc<KB>(a0 + HA_BYTES + k * MMA_K * 2), bdesc,
@@ -401,7 +413,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
     const int row = half * BM + q * 32 + lane;
     int g = 0, it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+    for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
+      const int split = t / total, tile = t - split * total;
+      if (tile < tile_pre[g]) g = 0;
       while (tile >= tile_pre[g + 1]) ++g;
       const int m = grp_off[g + 1] - grp_off[g];
       const int mt = (m + TBM - 1) / TBM;
@@ -458,6 +472,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
             dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
             dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+          }
+        }
+      } else if (EPI == EPI_F32) {
+        // fp32 partial of this k-split, rows of out32 + split * split_stride
+        float* orow32 = reinterpret_cast<float*>(p.out) + split * p.split_stride + orow * p.ldo +
+                        (int64_t)n_idx * p.n_out_tile;
+#pragma unroll 1
+        for (int c = 0; c < MMA_N; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (c == MMA_N - 32) {             // last TMEM read of the tile: release the buffer
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          const int col = n_idx * p.n_out_tile + c;
+          if (valid && col < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
       } else {
@@ -547,6 +582,7 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 enum GemmTile { TILE_128 = 0, TILE_256 = 1, TILE_256_K32 = 2 };
 
 int g_gemm_fault = 0;       // set through moe_debug_inject (tests of the bounded waits)
+constexpr int kRouterMaxSplits = 8;
 GemmTile gemm_tile() {
   static GemmTile t = [] {
     const char* v = getenv("MOE_GEMM_TILE");
@@ -571,7 +607,7 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<grid, 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
+  kern<<<counted(grid), 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
   return cudaGetLastError();
 }
 
@@ -582,6 +618,7 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
   switch (epi) {
     case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_RELU: return launch_epi<EPI_RELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    case EPI_F32: return launch_epi<EPI_F32, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     default: return launch_epi<EPI_NONE, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
   }
 }
@@ -612,6 +649,9 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
   p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
   p.fault = g_gemm_fault;
+  p.ksplit = 1;
+  p.kchunk = 1 << 30;
+  p.split_stride = 0;
   const GemmTile tile = gemm_tile();
   const int halves = tile == TILE_128 ? 1 : 2;
   const int kb = tile == TILE_256_K32 ? 32 : 64;
@@ -639,5 +679,45 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
 }
 
 void set_gemm_fault(int kind) { g_gemm_fault = kind; }
+
+// k-splits of the router product: enough (m-tile, split) pairs to cover the SMs, at most
+// kRouterMaxSplits, and every split non-empty (ks = ceil(nkb / ceil(nkb / ks))).
+int router_gemm_splits(int T, int D) {
+  const int mt = (T + BM - 1) / BM;
+  const int nkb = (D + 63) / 64;
+  int ks = sm_count() / (mt > 0 ? mt : 1);
+  if (ks > kRouterMaxSplits) ks = kRouterMaxSplits;
+  if (ks > nkb) ks = nkb;
+  if (ks < 1) ks = 1;
+  const int kchunk = (nkb + ks - 1) / ks;
+  return (nkb + kchunk - 1) / kchunk;
+}
+
+cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg, int E,
+                                    float* partials, int ksplit, cudaStream_t s) {
+  if (T <= 0) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb;
+  if (!make_map(&ta, x, (uint64_t)T, (uint64_t)D, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, Wg, (uint64_t)E, (uint64_t)D, 128, 64)) return cudaErrorInvalidValue;
+  GemmParams p;
+  p.offsets = nullptr;                        // one group: all T token rows
+  p.out = reinterpret_cast<__nv_bfloat16*>(partials);
+  p.err = device_error_word();
+  p.rows = T;
+  p.ldo = E;
+  p.G = 1;
+  p.N = E;
+  p.K = D;
+  p.n_out_tile = 256;
+  p.nt = 1;
+  p.fault = 0;
+  const int nkb = (D + 63) / 64;
+  p.ksplit = ksplit;
+  p.kchunk = (nkb + ksplit - 1) / ksplit;
+  p.split_stride = (int64_t)T * E;
+  const int64_t tiles = (int64_t)((T + BM - 1) / BM) * ksplit;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, 1), s);
+}
 
 }  // namespace moe

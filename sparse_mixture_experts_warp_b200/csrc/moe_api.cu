@@ -6,11 +6,16 @@
 #include <math.h>
 #include <string.h>
 
+#include <atomic>
+
 #include "common.cuh"
 
 namespace moe {
 
 static __device__ int g_device_error = 0;
+
+static std::atomic<int64_t> g_launches{0};
+void note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int num_sms() {
   int dev = 0, n = 0;
@@ -83,6 +88,7 @@ size_t esize(const moe_desc_t* d) { return d->dtype == MOE_BF16 ? 2 : 4; }
 size_t route_scratch(const moe_desc_t* d) {
   size_t b = up((size_t)router_partials(*d) * d->E * sizeof(float));
   if (d->select == MOE_EXPERT_CHOICE) b += up((size_t)d->E * d->T * sizeof(float));
+  b += up(router_gemm_scratch_bytes(*d));
   return b;
 }
 size_t permute_scratch(const moe_desc_t* d) {
@@ -221,15 +227,17 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
   uint8_t* sc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(scratch) + kAlign - 1) &
                                            ~(uintptr_t)(kAlign - 1));
   float* partials = reinterpret_cast<float*>(sc);
+  const size_t pbytes = up((size_t)router_partials(*d) * d->E * sizeof(float));
+  const size_t tbytes = d->select == MOE_EXPERT_CHOICE ? up((size_t)d->E * d->T * sizeof(float)) : 0;
+  float* lpart = router_uses_gemm(*d) ? reinterpret_cast<float*>(sc + pbytes + tbytes) : nullptr;
   int np = 0;
   cudaError_t e;
   if (d->select == MOE_TOKEN_CHOICE) {
     e = launch_router_token_choice(*d, x, Wg, d->score == MOE_SCORE_SIGMOID ? sel_bias : nullptr,
-                                   expert_ids, gates, logits, partials, &np, s);
+                                   expert_ids, gates, logits, partials, &np, lpart, s);
   } else {
-    const size_t pbytes = up((size_t)router_partials(*d) * d->E * sizeof(float));
     float* probsT = reinterpret_cast<float*>(sc + pbytes);
-    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, s);
+    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, lpart, s);
     if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
   }
   if (e == cudaSuccess && importance)
@@ -367,7 +375,7 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   if (st != MOE_OK) return st;
   if (d->n_shared > 0) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    set_offsets_kernel<<<1, 1, 0, s>>>(v.shared_offsets, d->T);
+    set_offsets_kernel<<<counted(1), 1, 0, s>>>(v.shared_offsets, d->T);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     // shared experts always use SwiGLU
     moe_desc_t ds = *d;
@@ -388,6 +396,8 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   if (st != MOE_OK) return st;
   return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.f, v.stats, stream);
 }
+
+int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 moe_status_t moe_debug_inject(int32_t fault) {
   if (fault != 0 && fault != 1) return MOE_ERR_INVALID_ARG;

@@ -494,7 +494,7 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
   const int nvec = d.D * esz / 16;
   if (A > 0 && A <= kOnePassMaxItems && E <= kOnePassMaxE && d.k <= kOnePassMaxK) {
     const int grid = (d.T + kOnePassTokens - 1) / kOnePassTokens;
-    permute_onepass_kernel<<<grid, 256, 0, s>>>(ids, d.T, d.k, E, cap,
+    permute_onepass_kernel<<<counted(grid), 256, 0, s>>>(ids, d.T, d.k, E, cap,
                                                 static_cast<const uint4*>(x), nvec,
                                                 static_cast<uint4*>(x_perm), counts, offsets,
                                                 row_src, inv);
@@ -505,16 +505,16 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(perm_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
-    perm_index_fused_kernel<<<1, 1024, smem, s>>>(ids, A, E, cap, counts, offsets, row_src, inv);
+    perm_index_fused_kernel<<<counted(1), 1024, smem, s>>>(ids, A, E, cap, counts, offsets, row_src, inv);
   } else {
-    perm_hist_kernel<<<nblk, kThreads, E * sizeof(int), s>>>(ids, A, E, block_hist);
-    perm_scan_kernel<<<1, 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
-    perm_rank_kernel<<<nblk, kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
+    perm_hist_kernel<<<counted(nblk), kThreads, E * sizeof(int), s>>>(ids, A, E, block_hist);
+    perm_scan_kernel<<<counted(1), 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
+    perm_rank_kernel<<<counted(nblk), kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
         ids, A, E, cap, block_hist, offsets, row_src, inv);
   }
   if (nblk > 0) {
     const int blocks = (d.T * 32 + 255) / 256;
-    gather_tc_kernel<<<blocks, 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
+    gather_tc_kernel<<<counted(blocks), 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
                                             static_cast<uint4*>(x_perm));
   }
   return cudaGetLastError();
@@ -525,15 +525,15 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
                                          int32_t* offsets, int32_t* row_src, int32_t* inv,
                                          cudaStream_t s) {
   const int64_t n = (int64_t)d.T * d.E;
-  if (n > 0) ec_fill_kernel<<<(unsigned)((n + 255) / 256), 256, 0, s>>>(inv, n);
+  if (n > 0) ec_fill_kernel<<<counted((unsigned)((n + 255) / 256)), 256, 0, s>>>(inv, n);
   const int rows = d.E * d.c;
   const int m = (rows > d.E + 1 ? rows : d.E + 1);
-  ec_index_kernel<<<(m + 255) / 256, 256, 0, s>>>(picked, d.E, d.c, d.T, counts, offsets,
+  ec_index_kernel<<<counted((m + 255) / 256), 256, 0, s>>>(picked, d.E, d.c, d.T, counts, offsets,
                                                   row_src, inv);
   const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
   const int nvec = d.D * esz / 16;
   if (rows > 0)
-    gather_rows_kernel<<<(rows * 32 + 255) / 256, 256, 0, s>>>(
+    gather_rows_kernel<<<counted((rows * 32 + 255) / 256), 256, 0, s>>>(
         static_cast<const uint4*>(x), d.T, nvec, picked, rows, static_cast<uint4*>(x_perm));
   return cudaGetLastError();
 }

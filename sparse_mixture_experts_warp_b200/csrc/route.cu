@@ -60,6 +60,8 @@ struct RouterArgs {
   const void* x; const void* Wg; const float* bias;
   int32_t* ids; float* gates; float* logits; float* probsT; float* partials;
   int T, D, E, k, score, gate, expert_choice;
+  const float* lpart;       // when set: logits are the sum of ksplit partials [ksplit][T][E]
+  int ksplit;
 };
 
 // logits of the warp's TPW tokens for all experts -> s_log[TPW][E]
@@ -117,7 +119,22 @@ router_kernel(RouterArgs a) {
   const int t0 = gw * kTPW;
   float* s_log = s_all + warp * kTPW * a.E;
 
-  warp_logits<BF16>(a, t0, s_log, lane);
+  if (a.lpart) {
+    // logits from the tensor-core router product: fixed-order sum of the k-split partials
+    for (int t = 0; t < kTPW; ++t) {
+      const int tok = t0 + t;
+      if (tok >= a.T) break;
+      for (int e = lane; e < a.E; e += 32) {
+        float v = 0.f;
+        for (int sp = 0; sp < a.ksplit; ++sp)
+          v += a.lpart[((int64_t)sp * a.T + tok) * a.E + e];
+        s_log[t * a.E + e] = v;
+      }
+    }
+    __syncwarp();
+  } else {
+    warp_logits<BF16>(a, t0, s_log, lane);
+  }
 
   const int E = a.E;
   float imp[kMaxEPL];
@@ -504,13 +521,24 @@ static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStre
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<true><<<blocks, kWarps * 32, smem, s>>>(a);
+    router_kernel<true><<<counted(blocks), kWarps * 32, smem, s>>>(a);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<false><<<blocks, kWarps * 32, smem, s>>>(a);
+    router_kernel<false><<<counted(blocks), kWarps * 32, smem, s>>>(a);
   }
   return cudaGetLastError();
+}
+
+// Router product on tensor cores (the grouped GEMM engine, fp32 partial logits) for bf16
+// inputs with many experts; the SIMT dot products of the generic kernel re-read x per block of 8
+// experts and W_g per 4 tokens, which is far from the HBM roofline at E >= 32.
+bool router_uses_gemm(const moe_desc_t& d) {
+  return d.dtype == MOE_BF16 && d.E >= 32 && d.E % 32 == 0 && d.E <= 256 && d.D % 64 == 0;
+}
+
+size_t router_gemm_scratch_bytes(const moe_desc_t& d) {
+  return router_uses_gemm(d) ? (size_t)8 * d.T * d.E * sizeof(float) : 0;
 }
 
 static bool fast_router_ok(const moe_desc_t& d) {
@@ -521,16 +549,23 @@ static bool fast_router_ok(const moe_desc_t& d) {
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
                                        float* logits, float* imp_partials, int* n_partials,
-                                       cudaStream_t s) {
+                                       float* lpart, cudaStream_t s) {
   RouterArgs a{x, Wg, bias, ids, gates, logits, nullptr, imp_partials,
-               d.T, d.D, d.E, d.k, d.score, d.gate, 0};
+               d.T, d.D, d.E, d.k, d.score, d.gate, 0, nullptr, 1};
+  if (router_uses_gemm(d) && lpart) {
+    const int ks = router_gemm_splits(d.T, d.D);
+    cudaError_t e = launch_router_gemm_bf16(x, d.T, d.D, Wg, d.E, lpart, ks, s);
+    if (e != cudaSuccess) return e;
+    a.lpart = lpart;
+    a.ksplit = ks;
+  }
   if (fast_router_ok(d)) {
     const int sms = num_sms() < 1024 ? num_sms() : 1024;
     const int tpc = (d.T + sms - 1) / sms;
     const int grid = tpc > 0 ? (d.T + tpc - 1) / tpc : 0;
     *n_partials = grid;
     if (grid == 0) return cudaSuccess;
-    router_fast_kernel<<<grid, (d.D / 256) * 32, 0, s>>>(a, tpc);
+    router_fast_kernel<<<counted(grid), (d.D / 256) * 32, 0, s>>>(a, tpc);
     return cudaGetLastError();
   }
   *n_partials = generic_partials(d);
@@ -539,22 +574,30 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
 
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, int* n_partials, cudaStream_t s) {
+                                        float* imp_partials, int* n_partials, float* lpart,
+                                        cudaStream_t s) {
   *n_partials = generic_partials(d);
   RouterArgs a{x, Wg, nullptr, nullptr, probs, logits, probsT, imp_partials,
-               d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1};
+               d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1, nullptr, 1};
+  if (router_uses_gemm(d) && lpart) {
+    const int ks = router_gemm_splits(d.T, d.D);
+    cudaError_t e = launch_router_gemm_bf16(x, d.T, d.D, Wg, d.E, lpart, ks, s);
+    if (e != cudaSuccess) return e;
+    a.lpart = lpart;
+    a.ksplit = ks;
+  }
   return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s) {
-  ec_select_kernel<<<d.E, 1024, 0, s>>>(probsT, d.T, d.c, picked);
+  ec_select_kernel<<<counted(d.E), 1024, 0, s>>>(probsT, d.T, d.c, picked);
   return cudaGetLastError();
 }
 
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
                                      float* importance, cudaStream_t s) {
-  importance_reduce_kernel<<<E, 256, 0, s>>>(partials, n_partials, E, T, importance);
+  importance_reduce_kernel<<<counted(E), 256, 0, s>>>(partials, n_partials, E, T, importance);
   return cudaGetLastError();
 }
 

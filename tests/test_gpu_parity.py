@@ -38,6 +38,10 @@ SMALL = {
     "fast_router_T300_E6": scaled(W["mixtral"], T=300, D=2048, E=6, F=256),
     "fast_router_switch_k1": scaled(W["switch"], T=500, D=1024, E=8, F=256),
     "fast_router_sigmoid_shared": scaled(W["v3"], T=200, D=1024, E=8, k=2, F=256, F_shared=256),
+    # router product on the tensor-core engine (bf16, E >= 32): ragged T, k-splits
+    "gemm_router_switch_E32": scaled(W["switch"], T=300, D=256, E=32, F=256),
+    "gemm_router_v3_E64": scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
+    "gemm_router_ec_E64": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
     # more than 65536 assignments: the multi-block permute path
     "large_A": scaled(W["mixtral"], T=33000, D=128, F=128),
 }
