@@ -146,7 +146,7 @@ perm_rank_kernel(const int32_t* ids, int A, int E, int cap, const int32_t* block
 // groups from __match_any_sync, leader adds), the per-expert exclusive scan over warps gives
 // each warp its base, a block scan over experts gives the offsets, and pass 2 assigns ranks in
 // the same order.  One launch instead of three.
-constexpr int kFusedMaxItems = 1 << 15;
+constexpr int kFusedMaxItems = 1 << 13;
 
 __global__ void __launch_bounds__(1024)
 perm_index_fused_kernel(const int32_t* ids, int A, int E, int cap, int32_t* counts,
