@@ -60,6 +60,10 @@ constexpr uint64_t DRAIN_NS = 200000000ull;      // 0.2 s to drain after an abor
 // (bits 10-12 = 1), both K-major (bits 15, 16 = 0), N >> 3 at bits 17-22, M >> 4 at 24-28.
 constexpr uint32_t kIdesc = (1u << 4) | (1u << 7) | (1u << 10) |
                             ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+// The same with M = 64, for a 128-row half that holds at most 64 live rows.  Its accumulator
+// rows 16q .. 16q+15 sit in TMEM lanes 32q .. 32q+15 (16 lanes of each lane quarter).
+constexpr uint32_t kIdesc64 = (1u << 4) | (1u << 7) | (1u << 10) |
+                              ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(64 >> 4) << 24);
 
 struct GemmParams {
   const int32_t* offsets;   // [G+1] device
@@ -148,12 +152,13 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   return d;
 }
 
-__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc) {
+__device__ __forceinline__ void umma_bf16(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t acc,
+                                          uint32_t idesc) {
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "setp.ne.b32 p, %4, 0;\n\t"
       "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(kIdesc), "r"(acc));
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
 }
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile(
@@ -368,6 +373,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int m_idx = (tile - tile_pre[g]) % mt;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
         const int kb0 = split * p.kchunk, kb1 = min(nkb, kb0 + p.kchunk);
+        // M = 64 for a half with at most 64 live rows
+        const int live0 = min(BM, m - m_idx * TBM), live1 = min(BM, m - m_idx * TBM - BM);
+        const uint32_t idesc0 = live0 <= 64 ? kIdesc64 : kIdesc;
+        const uint32_t idesc1 = live1 <= 64 ? kIdesc64 : kIdesc;
         const int acc = it % NBUF;
         const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
@@ -389,10 +398,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           for (int k = 0; k < KB / MMA_K; ++k) {
             const uint64_t bdesc = sdesc<KB>(b0 + k * MMA_K * 2);
             const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
-            umma_bf16(d_tmem, sdesc<KB>(a0 + k * MMA_K * 2), bdesc, accum);
+            umma_bf16(d_tmem, sdesc<KB>(a0 + k * MMA_K * 2), bdesc, accum, idesc0);
             if (two)
               umma_bf16(d_tmem + ACC_COLS, sdesc<KB>(a0 + HA_BYTES + k * MMA_K * 2), bdesc,
-                        accum);
+                        accum, idesc1);
           }
           umma_commit(&empty[stage]);       // frees the stage once these MMAs have read it
           if (++stage == TSTAGES) {
@@ -411,7 +420,6 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     // ---------------- epilogue (warps 2 .. 2 + N_EPI) ----------------
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
-    const int row = half * BM + q * 32 + lane;
     int g = 0, it = 0;
     for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
       const int split = t / total, tile = t - split * total;
@@ -435,9 +443,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         mbar_arrive(&tempty[acc]);
         continue;
       }
+      // rows of this half: M = 128 -> lane quarter q holds rows 32q + lane; M = 64 (at most 64
+      // live rows) -> rows 16q + lane in the quarter's first 16 lanes
+      const int live = min(BM, m - m_idx * TBM - half * BM);
+      const bool m64 = live <= 64;
+      const int row = half * BM + (m64 ? 16 * q + lane : 32 * q + lane);
       const int r = m_idx * TBM + row;
       const int64_t orow = (int64_t)grp_off[g] + r;
-      bool valid = r < m;
+      bool valid = r < m && (!m64 || lane < 16);
       if (valid && (orow < 0 || orow >= p.rows)) {
         atomicCAS(p.err, 0, DEVERR_BOUNDS);
         valid = false;
