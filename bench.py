@@ -191,13 +191,14 @@ def stage_work(w, rows_exec):
     }
 
 
-def gemm_hbm_bytes(w, rows_exec):
-    """Bytes the expert GEMMs must move at least: every weight once, the grouped rows in and
-    out of each projection (x_perm read, h written and read, y written) and the shared experts'
-    weights and activations."""
+def gemm_hbm_bytes(w, rows_exec, active_experts=None):
+    """Bytes the expert GEMMs must move at least: the weights of every expert that has rows,
+    once, the grouped rows in and out of each projection (x_perm read, h written and read, y
+    written) and the shared experts' weights and activations."""
     es = 2 if w.dtype == "bf16" else 4
     n_up = 2 if w.act == "swiglu" else 1
-    weights = w.E * (n_up + 1) * w.F * w.D * es
+    n_active = w.E if active_experts is None else active_experts
+    weights = n_active * (n_up + 1) * w.F * w.D * es
     acts = rows_exec * (w.D + 2 * w.F + w.D) * es
     shared = w.n_shared * (3 * w.F_shared * w.D + w.T * (w.D + 2 * w.F_shared + w.D)) * es
     return weights + acts + shared
@@ -405,7 +406,9 @@ def run_cuda(args, rank, world, local):
     # whole-layer roofline: the expert GEMMs at the slower of their FLOPs at the tensor peak and
     # their weight + activation bytes at the HBM peak, plus the HBM-bound stages' bytes
     hbm_bytes = sum(work[s][1] for s in ("route", "permute", "combine", "stats"))
-    gemm_bytes = gemm_hbm_bytes(w, rows_exec)
+    offs = v["offsets"].cpu()
+    active = int(((offs[1:] - offs[:-1]) > 0).sum().item())
+    gemm_bytes = gemm_hbm_bytes(w, rows_exec, active)
     gemm_roof_s = max(gemm_flops / (tc_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
     layer_roof_s = gemm_roof_s + hbm_bytes / (peaks["hbm_gbs"] * 1e9)
     roofline = {

@@ -53,7 +53,7 @@ enum { MOE_SCORE_SOFTMAX = 0, MOE_SCORE_SIGMOID = 1 };   /* affinity */
 enum { MOE_TOKEN_CHOICE = 0, MOE_EXPERT_CHOICE = 1 };    /* who selects */
 enum { MOE_GATE_RENORM = 0, MOE_GATE_RAW = 1 };          /* merge weights */
 enum { MOE_DROPLESS = 0, MOE_CAPACITY_DROP = 1 };        /* overflow policy */
-enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU = 1 };           /* expert FFN */
+enum { MOE_ACT_SWIGLU = 0, MOE_ACT_RELU = 1, MOE_ACT_GELU = 2 };   /* expert FFN */
 enum { MOE_F32 = 0, MOE_BF16 = 1 };                      /* operand dtype */
 
 /* Problem statement of one layer call.
@@ -180,10 +180,11 @@ moe_status_t moe_permute_noalloc(const moe_desc_t* desc, const int32_t* expert_i
                                  int32_t* row_src, int32_t* inv, moe_stream_t stream);
 
 /* Expert compute on grouped rows (Tiny MoE section 3, SwiGLU: down(SiLU(x W_gate^T) * x W_up^T);
- * ReLU: down(ReLU(x W_up^T))).  Group g owns rows [offsets[g], offsets[g+1]) of `a`
+ * the classic two-matrix FFN D -> F -> D: down(ReLU(x W_up^T)) or down(GELU(x W_up^T)) with the
+ * exact GELU(z) = z * (1 + erf(z / sqrt 2)) / 2).  Group g owns rows [offsets[g], offsets[g+1]) of `a`
  * (offsets is a device array of n_groups+1 ints, read on the device).
  *   a [a_rows, D], h [a_rows, F], y [a_rows, D] (dtype; h, y rows outside the groups are not
- *   written).  W_gate (NULL for ReLU), W_up [n_groups, F, D], W_down [n_groups, D, F].
+ *   written).  W_gate (NULL for ReLU / GELU), W_up [n_groups, F, D], W_down [n_groups, D, F].
  *   D comes from desc; act and dtype too.  For routed experts: n_groups = E, F = desc->F,
  *   a = x_perm, a_rows = moe_rows_max.  For a shared expert: n_groups = 1, F = F_shared,
  *   a = x, a_rows = T, offsets = {0, T}.

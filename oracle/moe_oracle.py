@@ -50,7 +50,7 @@ __all__ = [
     "router_logits", "softmax_rows", "sigmoid", "routing_keys",
     "topk_desc", "route_token_choice", "route_expert_choice",
     "capacity", "dispatch_token_choice", "dispatch_expert_choice",
-    "swiglu_expert", "relu_expert", "expert_rows",
+    "swiglu_expert", "relu_expert", "gelu", "gelu_expert", "expert_rows",
     "combine", "balance_stats", "layer_forward", "layer_forward_rows",
     "dense_masked_forward", "soft_routing_forward",
 ]
@@ -282,11 +282,27 @@ def relu_expert(xr, Wup, Wdown):
     return h @ np.asarray(Wdown, dtype=np.float64).T
 
 
+def gelu(z):
+    """Exact GELU, z * Phi(z) = z * (1 + erf(z / sqrt 2)) / 2 ([TINY] section 3: the classic
+    FFN's nn.GELU(), whose default is this erf form)."""
+    from scipy.special import erf
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * z * (1.0 + erf(z / math.sqrt(2.0)))
+
+
+def gelu_expert(xr, Wup, Wdown):
+    """Classic two-matrix FFN D -> F -> D with GELU in between ([TINY] section 3)."""
+    xr = np.asarray(xr, dtype=np.float64)
+    return gelu(xr @ np.asarray(Wup, dtype=np.float64).T) @ np.asarray(Wdown, dtype=np.float64).T
+
+
 def expert_rows(act, xr, e, W_gate, W_up, W_down):
     if act == "swiglu":
         return swiglu_expert(xr, W_gate[e], W_up[e], W_down[e])
     if act == "relu":
         return relu_expert(xr, W_up[e], W_down[e])
+    if act == "gelu":
+        return gelu_expert(xr, W_up[e], W_down[e])
     raise ValueError(act)
 
 
@@ -457,6 +473,8 @@ def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
         ts = [t for t, _ in need[e]]
         if g["act"] == "swiglu":
             ye = swiglu_expert(x[ts], wg_e, wu_e, wd_e)
+        elif g["act"] == "gelu":
+            ye = gelu_expert(x[ts], wu_e, wd_e)
         else:
             ye = relu_expert(x[ts], wu_e, wd_e)
         for i, (t, j) in enumerate(need[e]):

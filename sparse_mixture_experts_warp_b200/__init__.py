@@ -32,7 +32,7 @@ SOFTMAX, SIGMOID = 0, 1
 TOKEN_CHOICE, EXPERT_CHOICE = 0, 1
 RENORM, RAW = 0, 1
 DROPLESS, CAPACITY_DROP = 0, 1
-SWIGLU, RELU = 0, 1
+SWIGLU, RELU, GELU = 0, 1, 2
 F32, BF16 = 0, 1
 
 
@@ -147,7 +147,7 @@ def desc_of(w, T=None) -> MoeDesc:
         select=TOKEN_CHOICE if w.select == "token" else EXPERT_CHOICE,
         gate=RENORM if w.gate == "renorm" else RAW,
         overflow=DROPLESS if w.overflow == "dropless" else CAPACITY_DROP,
-        act=SWIGLU if w.act == "swiglu" else RELU,
+        act={"swiglu": SWIGLU, "relu": RELU, "gelu": GELU}[w.act],
         dtype=BF16 if w.dtype == "bf16" else F32,
         capacity_factor=w.capacity_factor, aux_alpha=w.aux_alpha)
 

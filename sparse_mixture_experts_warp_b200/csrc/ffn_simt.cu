@@ -3,7 +3,7 @@
 //
 // "从 Dense FFN 到 MoE：用一个 Tiny Transformer 理解 Router、Top-K 与负载均衡" (f3dlife),
 // section 3: a SwiGLU expert is down(SiLU(x W_gate) * (x W_up)); the classic FFN uses one
-// up matrix and an activation (ReLU here).  Group g owns rows [offsets[g], offsets[g+1]).
+// up matrix and an activation (ReLU, or the page's GELU).  Group g owns rows [offsets[g], offsets[g+1]).
 #include "common.cuh"
 
 namespace moe {
@@ -38,6 +38,8 @@ ffn_up_f32_kernel(const float* __restrict__ a, int D, int F, const int32_t* offs
       float g = 0.f;
       for (int d = 0; d < D; ++d) g = fmaf(wg[d], s_x[d], g);
       out = g / (1.0f + expf(-g)) * u;
+    } else if (act == MOE_ACT_GELU) {
+      out = 0.5f * u * (1.0f + erff(u * 0.70710678118654752f));
     } else {
       out = fmaxf(u, 0.f);
     }

@@ -12,6 +12,7 @@
 //   EPI_SWIGLU: B0 = W_gate, B1 = W_up; one 128x256 MMA tile holds 128 gate columns and the
 //               same 128 up columns side by side in TMEM; out = SiLU(gate) * up.
 //   EPI_RELU:   out = max(acc, 0) with B0 = W_up.
+//   EPI_GELU:   out = acc * (1 + erf(acc / sqrt 2)) / 2 with B0 = W_up.
 //   EPI_NONE:   out = acc with B0 = W_down.
 //
 // Design (one persistent CTA per SM, warp-specialised; two tile heights, see grouped_gemm_kernel):
@@ -527,6 +528,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               if (EPI == EPI_RELU) {
                 a0 = fmaxf(a0, 0.f);
                 a1 = fmaxf(a1, 0.f);
+              } else if (EPI == EPI_GELU) {
+                a0 = 0.5f * a0 * (1.0f + erff(a0 * 0.70710678118654752f));
+                a1 = 0.5f * a1 * (1.0f + erff(a1 * 0.70710678118654752f));
               }
               pk[i] = pack_bf16(a0, a1);
             }
@@ -632,6 +636,7 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
     case EPI_SWIGLU: return launch_epi<EPI_SWIGLU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_RELU: return launch_epi<EPI_RELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_F32: return launch_epi<EPI_F32, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    case EPI_GELU: return launch_epi<EPI_GELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     default: return launch_epi<EPI_NONE, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
   }
 }

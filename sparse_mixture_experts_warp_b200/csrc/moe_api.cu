@@ -42,7 +42,8 @@ moe_status_t validate(const moe_desc_t* d) {
   if (d->select != MOE_TOKEN_CHOICE && d->select != MOE_EXPERT_CHOICE) return MOE_ERR_INVALID_ARG;
   if (d->gate != MOE_GATE_RENORM && d->gate != MOE_GATE_RAW) return MOE_ERR_INVALID_ARG;
   if (d->overflow != MOE_DROPLESS && d->overflow != MOE_CAPACITY_DROP) return MOE_ERR_INVALID_ARG;
-  if (d->act != MOE_ACT_SWIGLU && d->act != MOE_ACT_RELU) return MOE_ERR_INVALID_ARG;
+  if (d->act != MOE_ACT_SWIGLU && d->act != MOE_ACT_RELU && d->act != MOE_ACT_GELU)
+    return MOE_ERR_INVALID_ARG;
   if (d->dtype != MOE_F32 && d->dtype != MOE_BF16) return MOE_ERR_INVALID_ARG;
   if (d->n_shared < 0 || (d->n_shared > 0 && d->F_shared <= 0)) return MOE_ERR_INVALID_ARG;
   if (d->E > 256) return MOE_ERR_UNSUPPORTED;
@@ -293,7 +294,8 @@ moe_status_t moe_expert_up(const moe_desc_t* d, int32_t G, int32_t F, const void
     if (d->act == MOE_ACT_SWIGLU)
       e = launch_grouped_gemm_bf16(EPI_SWIGLU, a, a_rows, d->D, W_gate, W_up, G, F, offsets, h, s);
     else
-      e = launch_grouped_gemm_bf16(EPI_RELU, a, a_rows, d->D, W_up, nullptr, G, F, offsets, h, s);
+      e = launch_grouped_gemm_bf16(d->act == MOE_ACT_GELU ? EPI_GELU : EPI_RELU, a, a_rows, d->D,
+                                   W_up, nullptr, G, F, offsets, h, s);
   } else {
     e = launch_ffn_up_f32(d->act, static_cast<const float*>(a), a_rows, d->D, F, offsets, G,
                           static_cast<const float*>(W_gate), static_cast<const float*>(W_up),

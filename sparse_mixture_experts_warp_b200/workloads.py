@@ -44,7 +44,7 @@ class Workload:
     gate: str = "renorm"       # "renorm" | "raw"
     overflow: str = "dropless"  # "dropless" | "drop"
     capacity_factor: float = 0.0
-    act: str = "swiglu"        # "swiglu" | "relu"
+    act: str = "swiglu"        # "swiglu" | "relu" | "gelu"
     dtype: str = "bf16"        # "bf16" | "f32"
     n_shared: int = 0
     F_shared: int = 0

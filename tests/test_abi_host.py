@@ -65,6 +65,7 @@ def _bad(**kw):
     (dict(score=7), 1), (dict(dtype=3), 1), (dict(E=300, k=2), 2), (dict(D=4100), 2),
     (dict(F=100), 2), (dict(overflow=1, capacity_factor=0.0), 1),
     (dict(select=1, c=0), 1), (dict(select=1, c=5000), 1), (dict(select=1, c=8, score=1), 2),
+    (dict(act=3), 1),
 ])
 def test_invalid_descriptors_are_rejected(kw, status):
     v = ctypes.c_size_t()

@@ -42,6 +42,10 @@ SMALL = {
     "gemm_router_switch_E32": scaled(W["switch"], T=300, D=256, E=32, F=256),
     "gemm_router_v3_E64": scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
     "gemm_router_ec_E64": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
+    # the classic D -> F -> D expert with GELU (bf16 tensor-core epilogue, fp32 CUDA cores)
+    "gelu_bf16": scaled(W["switch"], act="gelu", T=500, D=256, E=16, F=512, overflow="dropless",
+                        gate="renorm", k=2, zipf_s=0.0),
+    "gelu_f32": scaled(W["tiny"], act="gelu", T=40),
     # more than 65536 assignments: the multi-block permute path
     "large_A": scaled(W["mixtral"], T=33000, D=128, F=128),
 }
@@ -111,3 +115,15 @@ def test_full_size_workload(name):
         tokens += np.nonzero(ref["inv"] < 0)[0][:2].tolist()   # k = 1: assignment == token
     tokens = sorted(set(tokens))
     C.check_sampled_output(w, inp, out, v, tokens)
+
+
+# small-T (decode) regime at the full Mixtral layer shape: a few rows per expert, every weight
+# tile streamed for them; all tokens are checked against the oracle
+@pytest.mark.parametrize("T", [1, 8, 64, 200])
+def test_decode_regime_mixtral_shape(T):
+    w = scaled(W["mixtral"], T=T)
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    C.check_logits(w, inp, v)
+    C.check_routing(w, inp, v)
+    C.check_sampled_output(w, inp, out, v, list(range(T)))

@@ -396,3 +396,26 @@ def test_sampled_rows_agree_with_full_layer(kw):
     full = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown, *(S or ()))
     rows = O.layer_forward_rows(c, [0, 3, 7, 9], x, Wg, b, Wgate, Wup, Wdown, *(S or ()))
     np.testing.assert_allclose(rows["out_rows"], full["out"][[0, 3, 7, 9]], rtol=1e-12, atol=1e-14)
+
+
+# ---------------------------------------------------------------- GELU ----
+
+def test_gelu_closed_forms():
+    # GELU(z) = z * Phi(z); Phi(1) = 0.8413447460685429 (standard normal table value).
+    phi1 = 0.8413447460685429
+    np.testing.assert_allclose(O.gelu(np.array([0.0, 1.0, -1.0])),
+                               [0.0, phi1, -(1.0 - phi1)], rtol=1e-14, atol=1e-16)
+    big = np.array([8.0, -8.0])
+    np.testing.assert_allclose(O.gelu(big), [8.0, 0.0], atol=1e-12)
+    # classic FFN with GELU, D = F = 1: out = w_down * GELU(w_up * x)
+    np.testing.assert_allclose(O.gelu_expert(np.array([[2.0]]), [[0.5]], [[3.0]]),
+                               [[3.0 * phi1]], rtol=1e-14)
+
+
+def test_gelu_layer_is_dense_masked():
+    c = cfg(T=10, D=6, E=4, F=5, k=2, act="gelu")
+    rng = np.random.default_rng(21)
+    x, Wg, _, _, Wup, Wdown = rand_layer(rng, c)
+    r = O.layer_forward(c, x, Wg, None, None, Wup, Wdown)
+    dense = O.dense_masked_forward(c, x, Wg, None, None, Wup, Wdown)
+    np.testing.assert_allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
