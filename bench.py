@@ -325,7 +325,7 @@ def run_cuda(args, rank, world, local):
         if ev is not None:
             ev[5].record(stream)
         M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
-                            stream)
+                            stream, logits=v["logits"])
         if ev is not None:
             ev[6].record(stream)
 

@@ -86,6 +86,10 @@ typedef struct moe_stats {
     int32_t n_kept;        /* rows the experts execute */
     int32_t n_dropped;     /* n_routes - n_kept */
     int32_t reserved;
+    float entropy;         /* mean over tokens of -sum_e p log p (NaN when no logits given) */
+    float count_p95;       /* 95th / 99th percentile of the per-expert counts, linear */
+    float count_p99;       /*   interpolation between order statistics */
+    float reserved2;
 } moe_stats_t;
 
 /* Device views into a moe_layer_forward workspace (see moe_layer_views). */
@@ -209,12 +213,16 @@ moe_status_t moe_combine(const moe_desc_t* desc, const void* y, const int32_t* i
                          moe_stream_t stream);
 
 /* Balance statistics ("Top-k 路由" load-balancing loss; Tiny MoE section 8; moe-comparison
- * [9,4,2,1] imbalance example): f_e = counts_e / n_routes, aux = alpha * E * sum f_e P_e,
- * max/mean of counts, kept and dropped routes.  counts [E] and offsets [E+1] from
- * moe_permute, importance [E] from moe_route; f [E] and one moe_stats_t are written. */
+ * [9,4,2,1] imbalance example and its monitoring list): f_e = counts_e / n_routes,
+ * aux = alpha * E * sum f_e P_e, max/mean of counts, kept and dropped routes, the 95th/99th
+ * percentiles of the per-expert counts and, when logits [T,E] (fp32, from moe_route) are
+ * given, the mean router entropy over tokens of the probabilities the importance averages
+ * (softmax, or sigmoid affinities normalised over experts).  counts [E] and offsets [E+1]
+ * from moe_permute, importance [E] from moe_route; f [E] and one moe_stats_t are written. */
 moe_status_t moe_balance_stats(const moe_desc_t* desc, const int32_t* counts,
-                               const int32_t* offsets, const float* importance, float* f,
-                               moe_stats_t* stats, moe_stream_t stream);
+                               const int32_t* offsets, const float* importance,
+                               const float* logits, float* f, moe_stats_t* stats,
+                               moe_stream_t stream);
 
 /* The whole layer: route -> permute -> expert_ffn (+ shared experts) -> combine -> stats,
  * enqueued on one stream with no host synchronisation.  Intermediates live in `ws`

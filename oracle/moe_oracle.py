@@ -343,7 +343,10 @@ def balance_stats(importance_rows, counts, n_kept, n_routes, alpha):
     [TINY] section 8: one_hot(topk).mean over (tokens, k)); aux = alpha * E *
     sum_e f_e P_e ([TKR] "負載均衡" formula, [TINY] section 8).  Also
     max/mean of the counts ([CMP] "先数 assignments": [9,4,2,1] -> 2.25) and
-    the number of dropped routes (n_routes - n_kept).
+    the number of dropped routes (n_routes - n_kept).  Monitoring figures of
+    [CMP] "监控至少要覆盖分布、容量与网络": the mean router entropy -sum p log p of
+    the importance rows, and the 95th/99th percentiles of the counts (linear
+    interpolation between order statistics).
     """
     counts = np.asarray(counts, dtype=np.float64)
     E = counts.shape[0]
@@ -351,10 +354,17 @@ def balance_stats(importance_rows, counts, n_kept, n_routes, alpha):
     f = counts / float(n_routes)
     aux = alpha * E * float(np.sum(f * P))
     mean = counts.sum() / E
+    rows = np.asarray(importance_rows, dtype=np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        plogp = np.where(rows > 0, rows * np.log(rows), 0.0)
     return {
         "P": P, "f": f, "aux": aux,
         "max_over_mean": float(counts.max() / mean) if mean > 0 else 0.0,
         "n_dropped": int(n_routes - n_kept),
+        # [CMP] monitoring list: router entropy and P95/P99 of the per-expert counts
+        "entropy": float(-plogp.sum(axis=1).mean()),
+        "count_p95": float(np.percentile(counts, 95)),
+        "count_p99": float(np.percentile(counts, 99)),
     }
 
 

@@ -48,7 +48,9 @@ class MoeDesc(ctypes.Structure):
 class MoeStats(ctypes.Structure):
     _fields_ = [("aux", ctypes.c_float), ("max_over_mean", ctypes.c_float),
                 ("n_routes", ctypes.c_int32), ("n_kept", ctypes.c_int32),
-                ("n_dropped", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("n_dropped", ctypes.c_int32), ("reserved", ctypes.c_int32),
+                ("entropy", ctypes.c_float), ("count_p95", ctypes.c_float),
+                ("count_p99", ctypes.c_float), ("reserved2", ctypes.c_float)]
 
 
 class MoeLayerViews(ctypes.Structure):
@@ -91,7 +93,7 @@ _SIGS = {
     "moe_expert_down": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_combine": ([_DP, _P, _P, _P, _P, _P, _P], ctypes.c_int),
-    "moe_balance_stats": ([_DP, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_balance_stats": ([_DP, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_layer_forward": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                           ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
@@ -247,7 +249,8 @@ def stats_of(raw: torch.Tensor) -> dict:
     b = bytes(raw.cpu().numpy().tobytes())
     s = MoeStats.from_buffer_copy(b)
     return dict(aux=s.aux, max_over_mean=s.max_over_mean, n_routes=s.n_routes,
-                n_kept=s.n_kept, n_dropped=s.n_dropped)
+                n_kept=s.n_kept, n_dropped=s.n_dropped, entropy=s.entropy,
+                count_p95=s.count_p95, count_p99=s.count_p99)
 
 
 # ---------------------------------------------------------------- steps ----
@@ -300,10 +303,10 @@ def moe_combine(d, y, inv, gates, y_shared, out, stream=None):
         _stream(stream)))
 
 
-def moe_balance_stats(d, counts, offsets, importance, f, stats, stream=None):
+def moe_balance_stats(d, counts, offsets, importance, f, stats, stream=None, logits=None):
     _check("moe_balance_stats", lib().moe_balance_stats(
-        ctypes.byref(d), _ptr(counts), _ptr(offsets), _ptr(importance), _ptr(f), _ptr(stats),
-        _stream(stream)))
+        ctypes.byref(d), _ptr(counts), _ptr(offsets), _ptr(importance), _ptr(logits), _ptr(f),
+        _ptr(stats), _stream(stream)))
 
 
 def moe_layer_forward(d, x, Wg, sel_bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, out,

@@ -10,7 +10,8 @@
 //
 // Statistics: "Top-k 路由" load-balancing loss L = alpha * N * sum_i f_i P_i; Tiny MoE section 8
 // (importance before top-k, load after top-k; E * sum p_e f_e = 1 at balance); "别只比较
-// Top-k" section "先数 assignments" (max/mean imbalance, [9,4,2,1] -> 2.25).
+// Top-k" section "先数 assignments" (max/mean imbalance, [9,4,2,1] -> 2.25) and its monitoring
+// list (per-expert counts, max/mean and P95/P99, router entropy).
 #include "common.cuh"
 
 namespace moe {
@@ -145,31 +146,73 @@ combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ 
   }
 }
 
-__global__ void __launch_bounds__(256)
-stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance, int E,
-             int n_routes, float alpha, float* f, moe_stats_t* st) {
-  __shared__ float s_fp[256];
-  __shared__ int s_max[256];
-  const int e = threadIdx.x;
+// One block of 1024 threads: f, aux, max/mean, kept/dropped, count percentiles (ranks by
+// counting, E <= 256), and the mean router entropy over tokens (thread i takes tokens i,
+// i + 1024, ...; fixed-order tree sums, so the result is deterministic).
+__global__ void __launch_bounds__(1024)
+stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance,
+             const float* logits, int T, int E, int sigmoid, int n_routes, float alpha, float* f,
+             moe_stats_t* st) {
+  __shared__ float s_fp[1024];
+  __shared__ int s_max[1024];
+  __shared__ float s_h[1024];
+  __shared__ int s_sorted[256];
+  const int tid = threadIdx.x;
   float fp = 0.f;
   int c = 0;
-  if (e < E) {
-    c = counts[e];
+  if (tid < E) {
+    c = counts[tid];
     const float fe = (float)c / (float)n_routes;
-    f[e] = fe;
-    fp = fe * importance[e];
+    f[tid] = fe;
+    fp = fe * importance[tid];
+    // rank of this count among all (ties by expert id): its slot in ascending order
+    int rank = 0;
+    for (int e = 0; e < E; ++e) {
+      const int ce = counts[e];
+      rank += (ce < c) || (ce == c && e < tid);
+    }
+    s_sorted[rank] = c;
   }
-  s_fp[e] = fp;
-  s_max[e] = c;
+  // router entropy of each token's probabilities
+  float h = 0.f;
+  if (logits) {
+    for (int t = tid; t < T; t += blockDim.x) {
+      const float* s = logits + (int64_t)t * E;
+      if (!sigmoid) {
+        float m = -INFINITY;
+        for (int e = 0; e < E; ++e) m = fmaxf(m, s[e]);
+        float z = 0.f, zs = 0.f;
+        for (int e = 0; e < E; ++e) {
+          const float ex = expf(s[e] - m);
+          z += ex;
+          zs += ex * (s[e] - m);
+        }
+        h += logf(z) - zs / z;                // -sum p log p with p = e^{s-m} / z
+      } else {
+        float sa = 0.f;
+        for (int e = 0; e < E; ++e) sa += 1.0f / (1.0f + expf(-s[e]));
+        float he = 0.f;
+        for (int e = 0; e < E; ++e) {
+          const float q = 1.0f / (1.0f + expf(-s[e])) / sa;
+          if (q > 0.f) he -= q * logf(q);
+        }
+        h += he;
+      }
+    }
+  }
+  s_fp[tid] = fp;
+  s_max[tid] = c;
+  s_h[tid] = h;
   __syncthreads();
-  for (int h = 128; h > 0; h >>= 1) {       // fixed-order tree
-    if (e < h) {
-      s_fp[e] += s_fp[e + h];
-      s_max[e] = max(s_max[e], s_max[e + h]);
+  for (int hw = 512; hw > 0; hw >>= 1) {        // fixed-order tree
+    if (tid < hw) {
+      s_fp[tid] += s_fp[tid + hw];
+      s_max[tid] = max(s_max[tid], s_max[tid + hw]);
+      s_h[tid] += s_h[tid + hw];
     }
     __syncthreads();
   }
-  if (e == 0) {
+  if (tid == 0) {
     const int kept = offsets[E];
     moe_stats_t r;
     r.aux = alpha * (float)E * s_fp[0];
@@ -179,6 +222,19 @@ stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importa
     r.n_kept = kept;
     r.n_dropped = n_routes - kept;
     r.reserved = 0;
+    r.entropy = logits ? s_h[0] / (float)T : __int_as_float(0x7fc00000);
+    float q[2];
+    const double pct[2] = {0.95, 0.99};
+    for (int i = 0; i < 2; ++i) {
+      const double pos = pct[i] * (double)(E - 1);
+      const int lo = (int)pos;
+      const int hi = lo + 1 < E ? lo + 1 : lo;
+      const double fr = pos - lo;
+      q[i] = (float)(s_sorted[lo] + fr * (double)(s_sorted[hi] - s_sorted[lo]));
+    }
+    r.count_p95 = q[0];
+    r.count_p99 = q[1];
+    r.reserved2 = 0.f;
     *st = r;
   }
 }
@@ -218,11 +274,13 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
 }
 
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
-                                 const int32_t* offsets, const float* importance, float* f,
-                                 moe_stats_t* stats, cudaStream_t s) {
+                                 const int32_t* offsets, const float* importance,
+                                 const float* logits, float* f, moe_stats_t* stats,
+                                 cudaStream_t s) {
   const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
-  stats_kernel<<<counted(1), 256, 0, s>>>(counts, offsets, importance, d.E, n_routes, d.aux_alpha, f,
-                                 stats);
+  const int sig = (d.select == MOE_TOKEN_CHOICE && d.score == MOE_SCORE_SIGMOID) ? 1 : 0;
+  stats_kernel<<<counted(1), 1024, 0, s>>>(counts, offsets, importance, logits, d.T, d.E, sig,
+                                           n_routes, d.aux_alpha, f, stats);
   return cudaGetLastError();
 }
 

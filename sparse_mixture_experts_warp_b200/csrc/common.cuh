@@ -93,7 +93,8 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
                            const float* gates, const void* y_shared, void* out,
                            cudaStream_t s);
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
-                                 const int32_t* offsets, const float* importance, float* f,
-                                 moe_stats_t* stats, cudaStream_t s);
+                                 const int32_t* offsets, const float* importance,
+                                 const float* logits, float* f, moe_stats_t* stats,
+                                 cudaStream_t s);
 
 }  // namespace moe

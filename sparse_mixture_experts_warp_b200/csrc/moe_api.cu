@@ -344,13 +344,13 @@ moe_status_t moe_combine(const moe_desc_t* d, const void* y, const int32_t* inv,
 }
 
 moe_status_t moe_balance_stats(const moe_desc_t* d, const int32_t* counts, const int32_t* offsets,
-                               const float* importance, float* f, moe_stats_t* stats,
-                               moe_stream_t stream) {
+                               const float* importance, const float* logits, float* f,
+                               moe_stats_t* stats, moe_stream_t stream) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
   if (!counts || !offsets || !importance || !f || !stats) return MOE_ERR_INVALID_ARG;
   if (d->select == MOE_TOKEN_CHOICE ? d->T * d->k == 0 : d->E * d->c == 0) return MOE_OK;
-  return cuda_status(launch_balance_stats(*d, counts, offsets, importance, f, stats,
+  return cuda_status(launch_balance_stats(*d, counts, offsets, importance, logits, f, stats,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -396,7 +396,7 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   }
   st = moe_combine(d, v.y, v.inv, v.gates, d->n_shared > 0 ? v.y_shared : nullptr, out, stream);
   if (st != MOE_OK) return st;
-  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.f, v.stats, stream);
+  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.logits, v.f, v.stats, stream);
 }
 
 int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -113,6 +113,10 @@ def check_routing(w, inp, v):
     np.testing.assert_allclose(s["max_over_mean"], st["max_over_mean"], rtol=1e-6)
     assert s["n_dropped"] == st["n_dropped"]
     assert s["n_kept"] == int(ref["kept"].sum())
+    np.testing.assert_allclose(s["count_p95"], st["count_p95"], rtol=1e-6)
+    np.testing.assert_allclose(s["count_p99"], st["count_p99"], rtol=1e-6)
+    # entropy from fp32 logits: fp32 exp/log over E terms per token, averaged over T
+    np.testing.assert_allclose(s["entropy"], st["entropy"], rtol=1e-4, atol=1e-6)
     return ref
 
 

@@ -419,3 +419,27 @@ def test_gelu_layer_is_dense_masked():
     r = O.layer_forward(c, x, Wg, None, None, Wup, Wdown)
     dense = O.dense_masked_forward(c, x, Wg, None, None, Wup, Wdown)
     np.testing.assert_allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------- monitoring statistics ----
+
+def test_router_entropy_closed_forms():
+    # uniform probabilities over E experts: entropy ln E; a one-hot row: 0
+    for E in (2, 8, 64):
+        st = O.balance_stats(np.full((3, E), 1.0 / E), [1] * E, E, E, 0.01)
+        np.testing.assert_allclose(st["entropy"], math.log(E), rtol=1e-14)
+    st = O.balance_stats(np.array([[1.0, 0.0, 0.0], [0.0, 0.0, 1.0]]), [1, 0, 1], 2, 2, 0.01)
+    assert st["entropy"] == 0.0
+    # two tokens, p = [1/2, 1/2] and [1/4, 3/4]: mean of ln 2 and H(1/4)
+    h2 = -(0.25 * math.log(0.25) + 0.75 * math.log(0.75))
+    st = O.balance_stats(np.array([[0.5, 0.5], [0.25, 0.75]]), [1, 1], 2, 2, 0.01)
+    np.testing.assert_allclose(st["entropy"], (math.log(2) + h2) / 2, rtol=1e-14)
+
+
+def test_count_percentiles_of_the_page_example():
+    # [9,4,2,1] sorted = [1,2,4,9]; position q*(E-1): 0.95*3 = 2.85 -> 4 + 0.85*5 = 8.25,
+    # 0.99*3 = 2.97 -> 4 + 0.97*5 = 8.85 (linear interpolation between order statistics)
+    g = gold("moe_comparison_imbalance.json")
+    st = O.balance_stats(np.full((1, 4), 0.25), g["counts"], g["total"], g["total"], 1e-2)
+    np.testing.assert_allclose(st["count_p95"], 8.25, rtol=1e-12)
+    np.testing.assert_allclose(st["count_p99"], 8.85, rtol=1e-12)
