@@ -303,7 +303,7 @@ def run_cuda(args, rank, world, local):
 
     def step(ev=None):
         M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
-                    v["importance"], scratch, stream)
+                    v["importance"], scratch, stream, entropy=v["entropy"])
         if ev is not None:
             ev[1].record(stream)
         M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
@@ -325,7 +325,7 @@ def run_cuda(args, rank, world, local):
         if ev is not None:
             ev[5].record(stream)
         M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
-                            stream, logits=v["logits"])
+                            stream, entropy=v["entropy"])
         if ev is not None:
             ev[6].record(stream)
 

@@ -86,7 +86,7 @@ typedef struct moe_stats {
     int32_t n_kept;        /* rows the experts execute */
     int32_t n_dropped;     /* n_routes - n_kept */
     int32_t reserved;
-    float entropy;         /* mean over tokens of -sum_e p log p (NaN when no logits given) */
+    float entropy;         /* mean over tokens of -sum_e p log p (NaN when not given) */
     float count_p95;       /* 95th / 99th percentile of the per-expert counts, linear */
     float count_p99;       /*   interpolation between order statistics */
     float reserved2;
@@ -98,6 +98,7 @@ typedef struct moe_layer_views {
     float* gates;          /* TC [T,k] merge weights;  EC [T,E] softmax probabilities */
     float* logits;         /* [T,E] fp32 router logits */
     float* importance;     /* [E]   P_e */
+    float* entropy;        /* [1]   mean router entropy over tokens */
     int32_t* counts;       /* [E]   nominal assignments per expert */
     int32_t* offsets;      /* [E+1] first row of each expert in the grouped buffers */
     int32_t* row_src;      /* [A]   assignment id of each row: t*k+j (TC) or t*E+e (EC) */
@@ -147,11 +148,12 @@ moe_status_t moe_layer_views(const moe_desc_t* desc, void* ws, size_t ws_bytes,
  *   Expert choice: expert_ids [E,c] = each expert's c most probable tokens (ties to the lower
  *   token id) in ascending order; gates [T,E] = softmax probabilities (merge weights).
  *   logits [T,E] (fp32) and importance [E] (P_e = mean_t of the softmax probabilities, or of
- *   the sigmoid affinities normalised over experts) are optional (NULL).
+ *   the sigmoid affinities normalised over experts) and entropy [1] (mean over tokens of
+ *   -sum_e p log p of those probabilities; moe-comparison monitoring list) are optional (NULL).
  *   scratch: moe_scratch_size bytes. */
 moe_status_t moe_route(const moe_desc_t* desc, const void* x, const void* Wg,
                        const float* sel_bias, int32_t* expert_ids, float* gates,
-                       float* logits, float* importance,
+                       float* logits, float* importance, float* entropy,
                        void* scratch, size_t scratch_bytes, moe_stream_t stream);
 
 /* Dispatch: counting-sort permutation of assignments into expert-contiguous rows.
@@ -215,13 +217,12 @@ moe_status_t moe_combine(const moe_desc_t* desc, const void* y, const int32_t* i
 /* Balance statistics ("Top-k 路由" load-balancing loss; Tiny MoE section 8; moe-comparison
  * [9,4,2,1] imbalance example and its monitoring list): f_e = counts_e / n_routes,
  * aux = alpha * E * sum f_e P_e, max/mean of counts, kept and dropped routes, the 95th/99th
- * percentiles of the per-expert counts and, when logits [T,E] (fp32, from moe_route) are
- * given, the mean router entropy over tokens of the probabilities the importance averages
- * (softmax, or sigmoid affinities normalised over experts).  counts [E] and offsets [E+1]
- * from moe_permute, importance [E] from moe_route; f [E] and one moe_stats_t are written. */
+ * percentiles of the per-expert counts, and the router entropy when `entropy` (a device scalar
+ * written by moe_route) is given.  counts [E] and offsets [E+1] from moe_permute, importance
+ * [E] from moe_route; f [E] and one moe_stats_t are written. */
 moe_status_t moe_balance_stats(const moe_desc_t* desc, const int32_t* counts,
                                const int32_t* offsets, const float* importance,
-                               const float* logits, float* f, moe_stats_t* stats,
+                               const float* entropy, float* f, moe_stats_t* stats,
                                moe_stream_t stream);
 
 /* The whole layer: route -> permute -> expert_ffn (+ shared experts) -> combine -> stats,

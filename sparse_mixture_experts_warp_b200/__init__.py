@@ -56,6 +56,7 @@ class MoeStats(ctypes.Structure):
 class MoeLayerViews(ctypes.Structure):
     _fields_ = [("expert_ids", ctypes.c_void_p), ("gates", ctypes.c_void_p),
                 ("logits", ctypes.c_void_p), ("importance", ctypes.c_void_p),
+                ("entropy", ctypes.c_void_p),
                 ("counts", ctypes.c_void_p), ("offsets", ctypes.c_void_p),
                 ("row_src", ctypes.c_void_p), ("inv", ctypes.c_void_p),
                 ("x_perm", ctypes.c_void_p), ("h", ctypes.c_void_p), ("y", ctypes.c_void_p),
@@ -86,7 +87,7 @@ _SIGS = {
     "moe_scratch_size": ([_DP, ctypes.POINTER(_SZ)], ctypes.c_int),
     "moe_workspace_size": ([_DP, ctypes.POINTER(_SZ)], ctypes.c_int),
     "moe_layer_views": ([_DP, _P, _SZ, ctypes.POINTER(MoeLayerViews)], ctypes.c_int),
-    "moe_route": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
+    "moe_route": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_permute_noalloc": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_up": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P], ctypes.c_int),
@@ -228,6 +229,7 @@ def layer_views(d: MoeDesc, ws: torch.Tensor) -> dict:
         gates=view(v.gates, torch.float32, (d.T, K)),
         logits=view(v.logits, torch.float32, (d.T, d.E)),
         importance=view(v.importance, torch.float32, (d.E,)),
+        entropy=view(v.entropy, torch.float32, (1,)),
         counts=view(v.counts, torch.int32, (d.E,)),
         offsets=view(v.offsets, torch.int32, (d.E + 1,)),
         row_src=view(v.row_src, torch.int32, (A,)),
@@ -256,11 +258,12 @@ def stats_of(raw: torch.Tensor) -> dict:
 # ---------------------------------------------------------------- steps ----
 
 def moe_route(d, x, Wg, sel_bias, expert_ids, gates, logits=None, importance=None,
-              scratch=None, stream=None):
+              scratch=None, stream=None, entropy=None):
     scratch = empty_scratch(d, x.device) if scratch is None else scratch
     _check("moe_route", lib().moe_route(
         ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(sel_bias), _ptr(expert_ids), _ptr(gates),
-        _ptr(logits), _ptr(importance), _ptr(scratch), scratch.numel(), _stream(stream)))
+        _ptr(logits), _ptr(importance), _ptr(entropy), _ptr(scratch), scratch.numel(),
+        _stream(stream)))
 
 
 def moe_permute(d, expert_ids, x, x_perm, counts, offsets, row_src, inv, scratch=None,
@@ -303,9 +306,9 @@ def moe_combine(d, y, inv, gates, y_shared, out, stream=None):
         _stream(stream)))
 
 
-def moe_balance_stats(d, counts, offsets, importance, f, stats, stream=None, logits=None):
+def moe_balance_stats(d, counts, offsets, importance, f, stats, stream=None, entropy=None):
     _check("moe_balance_stats", lib().moe_balance_stats(
-        ctypes.byref(d), _ptr(counts), _ptr(offsets), _ptr(importance), _ptr(logits), _ptr(f),
+        ctypes.byref(d), _ptr(counts), _ptr(offsets), _ptr(importance), _ptr(entropy), _ptr(f),
         _ptr(stats), _stream(stream)))
 
 

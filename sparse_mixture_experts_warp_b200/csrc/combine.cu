@@ -146,16 +146,13 @@ combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ 
   }
 }
 
-// One block of 1024 threads: f, aux, max/mean, kept/dropped, count percentiles (ranks by
-// counting, E <= 256), and the mean router entropy over tokens (thread i takes tokens i,
-// i + 1024, ...; fixed-order tree sums, so the result is deterministic).
-__global__ void __launch_bounds__(1024)
+// One block of 256 threads: f, aux, max/mean, kept/dropped, count percentiles (ranks by
+// counting, E <= 256) and the router's mean entropy; fixed-order tree sums (deterministic).
+__global__ void __launch_bounds__(256)
 stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance,
-             const float* logits, int T, int E, int sigmoid, int n_routes, float alpha, float* f,
-             moe_stats_t* st) {
-  __shared__ float s_fp[1024];
-  __shared__ int s_max[1024];
-  __shared__ float s_h[1024];
+             const float* entropy, int E, int n_routes, float alpha, float* f, moe_stats_t* st) {
+  __shared__ float s_fp[256];
+  __shared__ int s_max[256];
   __shared__ int s_sorted[256];
   const int tid = threadIdx.x;
   float fp = 0.f;
@@ -173,42 +170,13 @@ stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importa
     }
     s_sorted[rank] = c;
   }
-  // router entropy of each token's probabilities
-  float h = 0.f;
-  if (logits) {
-    for (int t = tid; t < T; t += blockDim.x) {
-      const float* s = logits + (int64_t)t * E;
-      if (!sigmoid) {
-        float m = -INFINITY;
-        for (int e = 0; e < E; ++e) m = fmaxf(m, s[e]);
-        float z = 0.f, zs = 0.f;
-        for (int e = 0; e < E; ++e) {
-          const float ex = expf(s[e] - m);
-          z += ex;
-          zs += ex * (s[e] - m);
-        }
-        h += logf(z) - zs / z;                // -sum p log p with p = e^{s-m} / z
-      } else {
-        float sa = 0.f;
-        for (int e = 0; e < E; ++e) sa += 1.0f / (1.0f + expf(-s[e]));
-        float he = 0.f;
-        for (int e = 0; e < E; ++e) {
-          const float q = 1.0f / (1.0f + expf(-s[e])) / sa;
-          if (q > 0.f) he -= q * logf(q);
-        }
-        h += he;
-      }
-    }
-  }
   s_fp[tid] = fp;
   s_max[tid] = c;
-  s_h[tid] = h;
   __syncthreads();
-  for (int hw = 512; hw > 0; hw >>= 1) {        // fixed-order tree
+  for (int hw = 128; hw > 0; hw >>= 1) {        // fixed-order tree
     if (tid < hw) {
       s_fp[tid] += s_fp[tid + hw];
       s_max[tid] = max(s_max[tid], s_max[tid + hw]);
-      s_h[tid] += s_h[tid + hw];
     }
     __syncthreads();
   }
@@ -222,7 +190,7 @@ stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importa
     r.n_kept = kept;
     r.n_dropped = n_routes - kept;
     r.reserved = 0;
-    r.entropy = logits ? s_h[0] / (float)T : __int_as_float(0x7fc00000);
+    r.entropy = entropy ? *entropy : __int_as_float(0x7fc00000);
     float q[2];
     const double pct[2] = {0.95, 0.99};
     for (int i = 0; i < 2; ++i) {
@@ -275,12 +243,11 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
 
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance,
-                                 const float* logits, float* f, moe_stats_t* stats,
+                                 const float* entropy, float* f, moe_stats_t* stats,
                                  cudaStream_t s) {
   const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
-  const int sig = (d.select == MOE_TOKEN_CHOICE && d.score == MOE_SCORE_SIGMOID) ? 1 : 0;
-  stats_kernel<<<counted(1), 1024, 0, s>>>(counts, offsets, importance, logits, d.T, d.E, sig,
-                                           n_routes, d.aux_alpha, f, stats);
+  stats_kernel<<<counted(1), 256, 0, s>>>(counts, offsets, importance, entropy, d.E, n_routes,
+                                          d.aux_alpha, f, stats);
   return cudaGetLastError();
 }
 

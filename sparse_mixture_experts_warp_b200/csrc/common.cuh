@@ -46,7 +46,7 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s);
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
-                                     float* importance, cudaStream_t s);
+                                     float* importance, float* entropy, cudaStream_t s);
 int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer (upper bound)
 bool router_uses_gemm(const moe_desc_t& d);
 size_t router_gemm_scratch_bytes(const moe_desc_t& d);   // partial logits of the GEMM router
@@ -94,7 +94,7 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
                            cudaStream_t s);
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance,
-                                 const float* logits, float* f, moe_stats_t* stats,
+                                 const float* entropy, float* f, moe_stats_t* stats,
                                  cudaStream_t s);
 
 }  // namespace moe

@@ -87,7 +87,7 @@ int64_t rows_of(const moe_desc_t* d) {
 size_t esize(const moe_desc_t* d) { return d->dtype == MOE_BF16 ? 2 : 4; }
 
 size_t route_scratch(const moe_desc_t* d) {
-  size_t b = up((size_t)router_partials(*d) * d->E * sizeof(float));
+  size_t b = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   if (d->select == MOE_EXPERT_CHOICE) b += up((size_t)d->E * d->T * sizeof(float));
   b += up(router_gemm_scratch_bytes(*d));
   return b;
@@ -119,6 +119,7 @@ size_t carve(const moe_desc_t* d, uint8_t* base, moe_layer_views_t* v) {
   w.expert_ids = static_cast<int32_t*>(take((ec ? E * d->c : T * K) * 4));
   w.gates = static_cast<float*>(take(T * K * 4));
   w.importance = static_cast<float*>(take(E * 4));
+  w.entropy = static_cast<float*>(take(4));
   w.counts = static_cast<int32_t*>(take(E * 4));
   w.offsets = static_cast<int32_t*>(take((E + 1) * 4));
   w.row_src = static_cast<int32_t*>(take(A * 4));
@@ -217,7 +218,8 @@ moe_status_t moe_layer_views(const moe_desc_t* d, void* ws, size_t ws_bytes,
 
 moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const float* sel_bias,
                        int32_t* expert_ids, float* gates, float* logits, float* importance,
-                       void* scratch, size_t scratch_bytes_, moe_stream_t stream) {
+                       float* entropy, void* scratch, size_t scratch_bytes_,
+                       moe_stream_t stream) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
   if (d->T == 0) return MOE_OK;
@@ -228,7 +230,7 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
   uint8_t* sc = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(scratch) + kAlign - 1) &
                                            ~(uintptr_t)(kAlign - 1));
   float* partials = reinterpret_cast<float*>(sc);
-  const size_t pbytes = up((size_t)router_partials(*d) * d->E * sizeof(float));
+  const size_t pbytes = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   const size_t tbytes = d->select == MOE_EXPERT_CHOICE ? up((size_t)d->E * d->T * sizeof(float)) : 0;
   float* lpart = router_uses_gemm(*d) ? reinterpret_cast<float*>(sc + pbytes + tbytes) : nullptr;
   int np = 0;
@@ -241,8 +243,8 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
     e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, lpart, s);
     if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
   }
-  if (e == cudaSuccess && importance)
-    e = launch_importance_reduce(partials, np, d->E, d->T, importance, s);
+  if (e == cudaSuccess && (importance || entropy))
+    e = launch_importance_reduce(partials, np, d->E, d->T, importance, entropy, s);
   return cuda_status(e);
 }
 
@@ -344,13 +346,13 @@ moe_status_t moe_combine(const moe_desc_t* d, const void* y, const int32_t* inv,
 }
 
 moe_status_t moe_balance_stats(const moe_desc_t* d, const int32_t* counts, const int32_t* offsets,
-                               const float* importance, const float* logits, float* f,
+                               const float* importance, const float* entropy, float* f,
                                moe_stats_t* stats, moe_stream_t stream) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
   if (!counts || !offsets || !importance || !f || !stats) return MOE_ERR_INVALID_ARG;
   if (d->select == MOE_TOKEN_CHOICE ? d->T * d->k == 0 : d->E * d->c == 0) return MOE_OK;
-  return cuda_status(launch_balance_stats(*d, counts, offsets, importance, logits, f, stats,
+  return cuda_status(launch_balance_stats(*d, counts, offsets, importance, entropy, f, stats,
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -366,8 +368,8 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   if (d->act == MOE_ACT_SWIGLU && !W_gate) return MOE_ERR_INVALID_ARG;
   if (d->n_shared > 0 && (!Ws_gate || !Ws_up || !Ws_down)) return MOE_ERR_INVALID_ARG;
   if (d->T == 0) return MOE_OK;
-  st = moe_route(d, x, Wg, sel_bias, v.expert_ids, v.gates, v.logits, v.importance, v.scratch,
-                 v.scratch_bytes, stream);
+  st = moe_route(d, x, Wg, sel_bias, v.expert_ids, v.gates, v.logits, v.importance, v.entropy,
+                 v.scratch, v.scratch_bytes, stream);
   if (st != MOE_OK) return st;
   st = moe_permute(d, v.expert_ids, x, v.x_perm, v.counts, v.offsets, v.row_src, v.inv,
                    v.scratch, v.scratch_bytes, stream);
@@ -396,7 +398,7 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   }
   st = moe_combine(d, v.y, v.inv, v.gates, d->n_shared > 0 ? v.y_shared : nullptr, out, stream);
   if (st != MOE_OK) return st;
-  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.logits, v.f, v.stats, stream);
+  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.entropy, v.f, v.stats, stream);
 }
 
 int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -140,6 +140,7 @@ router_kernel(RouterArgs a) {
   float imp[kMaxEPL];
 #pragma unroll
   for (int i = 0; i < kMaxEPL; ++i) imp[i] = 0.f;
+  float ent = 0.f;                 // this lane's share of the tokens' -sum p log p
 
   for (int t = 0; t < kTPW; ++t) {
     const int tok = t0 + t;
@@ -177,6 +178,7 @@ router_kernel(RouterArgs a) {
         key[i] = s[i];             // softmax is monotone in the logit within a row
         sel_w[i] = p[i];
         imp[i] += p[i];
+        if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
       }
     } else {
       float asum = 0.f;
@@ -191,7 +193,11 @@ router_kernel(RouterArgs a) {
       asum = warp_sum(asum);
       const float inv = 1.0f / asum;
 #pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) { p[i] = sel_w[i] * inv; imp[i] += p[i]; }
+      for (int i = 0; i < kMaxEPL; ++i) {
+        p[i] = sel_w[i] * inv;
+        imp[i] += p[i];
+        if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
+      }
     }
 
     if (a.expert_choice) {
@@ -246,19 +252,26 @@ router_kernel(RouterArgs a) {
   }
 
   if (a.partials) {
+    // row gw of the partials: E importance sums, then the entropy sum
 #pragma unroll
     for (int i = 0; i < kMaxEPL; ++i) {
       const int e = lane + 32 * i;
-      if (e < E) a.partials[(int64_t)gw * E + e] = imp[i];
+      if (e < E) a.partials[(int64_t)gw * (E + 1) + e] = imp[i];
     }
+    ent = warp_sum(ent);
+    if (lane == 0) a.partials[(int64_t)gw * (E + 1) + E] = ent;
   }
 }
 
-// importance[e] = (sum over partial rows, fixed order) / T.  One block per expert.
-__global__ void importance_reduce_kernel(const float* partials, int n, int E, int T, float* out) {
+// importance[e] = (sum over partial rows, fixed order) / T, one block per expert; block E
+// reduces the entropy column into *entropy (mean over tokens).
+__global__ void importance_reduce_kernel(const float* partials, int n, int E, int T,
+                                         float* importance, float* entropy) {
   const int e = blockIdx.x;
+  float* out = (e < E) ? importance : entropy;
+  if (!out) return;
   float s = 0.f;
-  for (int i = threadIdx.x; i < n; i += blockDim.x) s += partials[(int64_t)i * E + e];
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += partials[(int64_t)i * (E + 1) + e];
   __shared__ float red[32];
   s = warp_sum(s);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
@@ -266,7 +279,7 @@ __global__ void importance_reduce_kernel(const float* partials, int n, int E, in
   if (threadIdx.x < 32) {
     float v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
     v = warp_sum(v);
-    if (threadIdx.x == 0) out[e] = v / (float)T;
+    if (threadIdx.x == 0) out[e < E ? e : 0] = v / (float)T;
   }
 }
 
@@ -400,7 +413,7 @@ __device__ __forceinline__ void load_rows(uint4 (&r0)[8], uint4 (&r1)[8],
 }
 
 __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float sv, bool live,
-                                             int lane, float& imp) {
+                                             int lane, float& imp, float& ent) {
   const int E = a.E;
   if (a.logits && live) a.logits[(int64_t)tok * E + lane] = sv;
   float selw, key;
@@ -411,11 +424,14 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float
     selw = p;
     key = sv;                    // softmax is monotone in the logit within a row
     imp += p;
+    if (p > 0.f) ent -= p * logf(p);
   } else {
     const float af = live ? 1.0f / (1.0f + expf(-sv)) : 0.f;
     selw = af;
     key = live ? af + (a.bias ? a.bias[lane] : 0.f) : -INFINITY;
-    imp += af / warp_sum(af);
+    const float q = af / warp_sum(af);
+    imp += q;
+    if (q > 0.f) ent -= q * logf(q);
   }
   bool taken = !live;
   int my_id = -1;
@@ -445,6 +461,7 @@ router_fast_kernel(RouterArgs a, int tokens_per_cta) {
   __shared__ float s_red[kFastMaxNW][kFastTB][kFastE];
   __shared__ float s_log[kFastTB][kFastE];
   __shared__ float s_imp[kFastTB][kFastE];
+  __shared__ float s_ent[kFastTB];
   const int NW = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
@@ -459,7 +476,7 @@ router_fast_kernel(RouterArgs a, int tokens_per_cta) {
                     : make_uint4(0u, 0u, 0u, 0u);
   const int t_begin = blockIdx.x * tokens_per_cta;
   const int t_end = min(a.T, t_begin + tokens_per_cta);
-  float imp = 0.f;
+  float imp = 0.f, ent = 0.f;
   uint4 r0[8], r1[8];
   load_rows(r0, r1, x, a.D, t_begin, t_end, g, kbase);
   for (int t0 = t_begin; t0 < t_end; t0 += kFastTB) {
@@ -486,17 +503,19 @@ router_fast_kernel(RouterArgs a, int tokens_per_cta) {
     for (int jj = warp; jj < kFastTB; jj += NW) {
       if (t0 + jj >= t_end) break;
       const bool live = lane < E;
-      select_token(a, t0 + jj, live ? s_log[jj][lane] : -INFINITY, live, lane, imp);
+      select_token(a, t0 + jj, live ? s_log[jj][lane] : -INFINITY, live, lane, imp, ent);
     }
   }
   // CTA importance partial: sum over the selection warps in a fixed order
   const int n_sel = NW < kFastTB ? NW : kFastTB;
   if (warp < n_sel && lane < kFastE) s_imp[warp][lane] = imp;
+  ent = warp_sum(ent);
+  if (warp < n_sel && lane == 0) s_ent[warp] = ent;
   __syncthreads();
-  if (a.partials && threadIdx.x < E) {
+  if (a.partials && threadIdx.x <= E) {      // row: E importance sums, then the entropy sum
     float sum = 0.f;
-    for (int j = 0; j < n_sel; ++j) sum += s_imp[j][threadIdx.x];
-    a.partials[(int64_t)blockIdx.x * E + threadIdx.x] = sum;
+    for (int j = 0; j < n_sel; ++j) sum += (threadIdx.x < E) ? s_imp[j][threadIdx.x] : s_ent[j];
+    a.partials[(int64_t)blockIdx.x * (E + 1) + threadIdx.x] = sum;
   }
 }
 
@@ -596,8 +615,9 @@ cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* 
 }
 
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
-                                     float* importance, cudaStream_t s) {
-  importance_reduce_kernel<<<counted(E), 256, 0, s>>>(partials, n_partials, E, T, importance);
+                                     float* importance, float* entropy, cudaStream_t s) {
+  importance_reduce_kernel<<<counted(E + 1), 256, 0, s>>>(partials, n_partials, E, T, importance,
+                                                          entropy);
   return cudaGetLastError();
 }
 

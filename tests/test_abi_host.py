@@ -75,7 +75,8 @@ def test_invalid_descriptors_are_rejected(kw, status):
 def test_null_pointers_rejected_before_launch():
     d = M.desc_of(WORKLOADS["mixtral"])
     L = M.lib()
-    st = L.moe_route(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None)
+    st = L.moe_route(ctypes.byref(d), None, None, None, None, None, None, None, None, None, 0,
+                     None)
     assert st == 1
     st = L.moe_permute(ctypes.byref(d), None, None, None, None, None, None, None, None, 0, None)
     assert st == 1
@@ -98,8 +99,8 @@ def test_workspace_too_small_or_misaligned():
     assert L.moe_layer_views(ctypes.byref(d), 0x10010, need, ctypes.byref(v)) == 3
     assert L.moe_layer_views(ctypes.byref(d), 0x10000, need, ctypes.byref(v)) == 0
     # views are laid out inside the workspace, 256-byte aligned, in range
-    ptrs = [v.logits, v.expert_ids, v.gates, v.importance, v.counts, v.offsets, v.row_src,
-            v.inv, v.x_perm, v.h, v.y, v.f, v.stats, v.scratch]
+    ptrs = [v.logits, v.expert_ids, v.gates, v.importance, v.entropy, v.counts, v.offsets,
+            v.row_src, v.inv, v.x_perm, v.h, v.y, v.f, v.stats, v.scratch]
     for p in ptrs:
         assert 0x10000 <= p < 0x10000 + need and p % 256 == 0
     assert len(set(ptrs)) == len(ptrs)
