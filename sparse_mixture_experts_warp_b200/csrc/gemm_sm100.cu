@@ -100,27 +100,39 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// kCluster: acquire at cluster scope, for barriers that the peer CTA of a pair arrives on.
+template <bool kCluster = false>
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
+  if (kCluster)
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+  else
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
   return ok != 0;
 }
 // Bounded wait for the phase of parity `parity` to complete.  Returns false when it gave up:
 // on its time limit (which records `code` and raises the CTA's abort flag) or, when
 // honor_abort, as soon as another role has aborted.  Drain waits pass honor_abort = false so
 // that they keep waiting (bounded) for work already in flight.
+template <bool kCluster = false>
 __device__ __noinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
                                        int* err, int code, uint64_t limit,
                                        bool honor_abort = true) {
-  if (mbar_try_wait(bar, parity)) return true;
+  if (mbar_try_wait<kCluster>(bar, parity)) return true;
   const uint64_t t0 = gtimer();
-  while (!mbar_try_wait(bar, parity)) {
+  while (!mbar_try_wait<kCluster>(bar, parity)) {
     if (honor_abort && *abort_flag) return false;
     if (gtimer() - t0 > limit) {
       *abort_flag = 1;
@@ -193,6 +205,103 @@ __device__ __forceinline__ void tmem_wait_ld() {
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
+}
+
+// SiLU(gate) * up of 32 accumulator columns -> 32 bf16 at dst (16-byte aligned).
+__device__ __forceinline__ void store_swiglu32(const uint32_t (&gv)[32], const uint32_t (&uv)[32],
+                                               __nv_bfloat16* dst) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+    const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
+    const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;
+    const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
+    pk[i] = pack_bf16(h0, h1);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  d[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+  d[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+}
+
+// act(acc) of 32 accumulator columns -> 32 bf16 at dst (EPI_RELU, EPI_GELU or EPI_NONE).
+template <int EPI>
+__device__ __forceinline__ void store_act32(const uint32_t (&v)[32], __nv_bfloat16* dst) {
+  uint32_t pk[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
+    if (EPI == EPI_RELU) {
+      a0 = fmaxf(a0, 0.f);
+      a1 = fmaxf(a1, 0.f);
+    } else if (EPI == EPI_GELU) {
+      a0 = 0.5f * a0 * (1.0f + erff(a0 * 0.70710678118654752f));
+      a1 = 0.5f * a1 * (1.0f + erff(a1 * 0.70710678118654752f));
+    }
+    pk[i] = pack_bf16(a0, a1);
+  }
+  uint4* d = reinterpret_cast<uint4*>(dst);
+  d[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+  d[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+  d[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
+  d[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
+}
+
+// ---- CTA-pair (cluster of two) primitives ----
+__device__ __forceinline__ uint32_t cluster_cta_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+// Address of this CTA's shared variable at `saddr` in CTA `rank` of the cluster.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile(
+      "barrier.cluster.arrive.release.aligned;\n\t"
+      "barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cl_addr) {
+  asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cl_addr)
+               : "memory");
+}
+// TMA box into this CTA's shared memory; completion is counted on the mbarrier at cluster
+// address bar_cl, which may be the peer CTA's (the pair's leader).  No multicast.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap* map,
+                                                 uint32_t bar_cl, int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cl), "r"(x), "r"(y)
+      : "memory");
+}
+__device__ __forceinline__ void umma_bf16_pair(uint32_t d_tmem, uint64_t a, uint64_t b,
+                                               uint32_t acc, uint32_t idesc) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+// Arrive on the mbarrier at this offset in both CTAs of the pair once the MMAs issued so far
+// have completed.
+__device__ __forceinline__ void umma_commit_both(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+      " [%0], %1;" ::"r"(smem_u32(bar)),
+      "h"((unsigned short)3)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
+  asm volatile(
+      "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+          smem_u32(bar))
+      : "memory");
 }
 
 // HALVES = 1: 128-row tiles, 4-stage ring of 48 KB, two 256-column TMEM accumulators (the
@@ -460,33 +569,22 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                              (uint32_t)(acc * BUF_COLS + half * ACC_COLS);
       __nv_bfloat16* orow_ptr = p.out + orow * p.ldo + (int64_t)n_idx * p.n_out_tile;
       if (EPI == EPI_SWIGLU) {
+        // two 32-column chunks of gate and up per TMEM wait
 #pragma unroll 1
-        for (int c = 0; c < 128; c += 32) {
-          uint32_t gv[32], uv[32];
-          tmem_ld32(taddr + c, gv);
-          tmem_ld32(taddr + 128 + c, uv);
+        for (int c = 0; c < 128; c += 64) {
+          uint32_t g0[32], u0[32], g1[32], u1[32];
+          tmem_ld32(taddr + c, g0);
+          tmem_ld32(taddr + 128 + c, u0);
+          tmem_ld32(taddr + c + 32, g1);
+          tmem_ld32(taddr + 160 + c, u1);
           tmem_wait_ld();
-          if (c == 96) {                     // last TMEM read of the tile: release the buffer
+          if (c == 64) {                     // last TMEM read of the tile: release the buffer
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
           }
           const int col = n_idx * p.n_out_tile + c;
-          if (valid && col < p.N) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
-              const float u0 = __uint_as_float(uv[2 * i]), u1 = __uint_as_float(uv[2 * i + 1]);
-              const float h0 = __fdividef(g0, 1.0f + __expf(-g0)) * u0;   // SiLU(g) * u
-              const float h1 = __fdividef(g1, 1.0f + __expf(-g1)) * u1;
-              pk[i] = pack_bf16(h0, h1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
-          }
+          if (valid && col < p.N) store_swiglu32(g0, u0, orow_ptr + c);   // SiLU(g) * u
+          if (valid && col + 32 < p.N) store_swiglu32(g1, u1, orow_ptr + c + 32);
         }
       } else if (EPI == EPI_F32) {
         // fp32 partial of this k-split, rows of out32 + split * split_stride
@@ -510,36 +608,24 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
         }
       } else {
+        // four 32-column chunks per TMEM wait
 #pragma unroll 1
-        for (int c = 0; c < MMA_N; c += 32) {
-          uint32_t v[32];
-          tmem_ld32(taddr + c, v);
+        for (int c = 0; c < MMA_N; c += 128) {
+          uint32_t v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(taddr + c, v0);
+          tmem_ld32(taddr + c + 32, v1);
+          tmem_ld32(taddr + c + 64, v2);
+          tmem_ld32(taddr + c + 96, v3);
           tmem_wait_ld();
-          if (c == MMA_N - 32) {             // last TMEM read of the tile: release the buffer
+          if (c == MMA_N - 128) {            // last TMEM read of the tile: release the buffer
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
           }
           const int col = n_idx * p.n_out_tile + c;
-          if (valid && col < p.N) {
-            uint32_t pk[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              float a0 = __uint_as_float(v[2 * i]), a1 = __uint_as_float(v[2 * i + 1]);
-              if (EPI == EPI_RELU) {
-                a0 = fmaxf(a0, 0.f);
-                a1 = fmaxf(a1, 0.f);
-              } else if (EPI == EPI_GELU) {
-                a0 = 0.5f * a0 * (1.0f + erff(a0 * 0.70710678118654752f));
-                a1 = 0.5f * a1 * (1.0f + erff(a1 * 0.70710678118654752f));
-              }
-              pk[i] = pack_bf16(a0, a1);
-            }
-            uint4* dst = reinterpret_cast<uint4*>(orow_ptr + c);
-            dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
-            dst[2] = make_uint4(pk[8], pk[9], pk[10], pk[11]);
-            dst[3] = make_uint4(pk[12], pk[13], pk[14], pk[15]);
-          }
+          if (valid && col < p.N) store_act32<EPI>(v0, orow_ptr + c);
+          if (valid && col + 32 < p.N) store_act32<EPI>(v1, orow_ptr + c + 32);
+          if (valid && col + 64 < p.N) store_act32<EPI>(v2, orow_ptr + c + 64);
+          if (valid && col + 96 < p.N) store_act32<EPI>(v3, orow_ptr + c + 96);
         }
       }
     }
@@ -550,6 +636,348 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 1) {
     tc_fence_after();
     asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
+                 "r"(TMEM_COLS)
+                 : "memory");
+  }
+}
+
+// ---------------- CTA-pair variant: tcgen05 cta_group::2, 256 x 512 tiles ----------------
+//
+// A cluster of two CTAs on neighbouring SMs computes each tile of 256 rows x 512 accumulator
+// columns with pairs of N=256 MMAs (M=256: CTA r supplies tile rows 128r .. 128r+127 of A; the
+// B operand of each MMA is split by rows, 128 per CTA); the leader (r = 0) issues the MMAs,
+// which read both CTAs' stages and leave each CTA's 128 rows x 512 fp32 columns in that CTA's
+// tensor memory.  Per SM and 64-element k-block the ring then moves 48 KB (128 A rows + 256 B
+// rows) for 128 x 512 x 64 multiply-adds: three quarters of the operand bytes per FLOP of a
+// 256 x 256 tile, which matters because the TMA/L2 path feeds an SM only ~30 B per clock while
+// a 256 x 256 tile needs 44 B per clock at the full tensor rate.  TMEM is full, so the epilogue
+// (8 warps: 4 lane quarters x 2 column halves) is not overlapped with the next tile's MMAs.
+// A tile with at most 128 live rows runs M=128 MMAs (64 rows per CTA) instead; their
+// accumulator holds a CTA's 64 rows in TMEM lanes 0-63 for the MMA's columns [0,128) and again
+// in lanes 64-127 for its columns [128,256), both at TMEM columns [0,128) of the MMA.
+// MMA j (j = 0, 1) writes TMEM columns [256j, 256j + 256); its B rows, 128 from each CTA, are
+//   SwiGLU:    for features f = n0 + 128j + 64r .. +63 of CTA r, 64 W_gate rows then the same
+//              64 W_up rows (64-row boxes), so that gate and up of a feature share a TMEM lane
+//              in both accumulator layouts: MMA column 128r + x is gate and 128r + 64 + x up
+//              of feature n0 + 128j + 64r + x;
+//   otherwise: W rows n0 + 256j + 128r .. +127 of CTA r: MMA column c is output column
+//              n0 + 256j + c.
+// Barriers: full[s] is used on the leader (its producer arms it with both CTAs' bytes, and both
+// CTAs' TMA loads complete on it); empty[s] and tfull exist in both CTAs and the leader's
+// tcgen05.commit arrives on both; tempty is used on the leader and takes one arrive per
+// epilogue warp of both CTAs.  Waits on barriers the peer arrives on acquire at cluster scope.
+constexpr uint32_t kIdescPair256 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                   ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(256 >> 4) << 24);
+constexpr uint32_t kIdescPair128 = (1u << 4) | (1u << 7) | (1u << 10) |
+                                   ((uint32_t)(MMA_N >> 3) << 17) | ((uint32_t)(128 >> 4) << 24);
+constexpr int kPairEpiWarps = 8;
+constexpr int kPairThreads = 64 + 32 * kPairEpiWarps;
+
+template <int EPI, int NSTAGES>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+grouped_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB0,
+                         const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
+  constexpr int KB = 64;
+  constexpr int TBM = 2 * BM;                      // rows of a pair tile
+  constexpr int A_BYTES = BM * KB * 2;             // this CTA's A box per stage
+  constexpr int BH_BYTES = 128 * KB * 2;           // one 128-row B box
+  constexpr int B_BYTES = 2 * BH_BYTES;            // this CTA's B rows of both MMAs
+  constexpr uint32_t STAGE_TX = 2 * (A_BYTES + B_BYTES);   // both CTAs, counted on the leader
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  const uint32_t sA = smem_u32(smem);
+  const uint32_t sB = sA + NSTAGES * A_BYTES;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + NSTAGES * (A_BYTES + B_BYTES));
+  uint64_t* full = bars;
+  uint64_t* empty = bars + NSTAGES;
+  uint64_t* tfull = bars + 2 * NSTAGES;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  int* grp_off = reinterpret_cast<int*>(tmem_holder + 2);   // [G+1]
+  int* tile_pre = grp_off + (p.G + 1);                      // [G+1]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_cta_rank();
+  const int pair = blockIdx.x >> 1, n_pairs = gridDim.x >> 1;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NSTAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(tfull, 1);
+    mbar_init(tempty, 2 * kPairEpiWarps);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+  }
+  if (warp == 0 && lane == 0) {
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB0)) : "memory");
+    if (EPI == EPI_SWIGLU)
+      asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB1)) : "memory");
+  }
+  if (warp == 1) {
+    // both CTAs allocate together: the pair's MMAs write the same columns in each
+    asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                     smem_u32(tmem_holder)),
+                 "r"(TMEM_COLS)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+  }
+  if (warp == 2) {
+    int carry = 0;
+    if (lane == 0) {
+      grp_off[0] = p.offsets[0];
+      tile_pre[0] = 0;
+    }
+    for (int g0 = 0; g0 < p.G; g0 += 32) {
+      const int g = g0 + lane;
+      int tiles = 0;
+      if (g < p.G) {
+        const int lo = p.offsets[g], hi = p.offsets[g + 1];
+        const int m = hi > lo ? hi - lo : 0;
+        tiles = ((m + TBM - 1) / TBM) * p.nt;
+        grp_off[g + 1] = hi;
+      }
+      int inc = tiles;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (g < p.G) tile_pre[g + 1] = carry + inc;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+  }
+  // barriers initialised and TMEM allocated in both CTAs before either touches the other
+  tc_fence_before();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_holder;
+  const int total = tile_pre[p.G];
+  const int nkb = (p.K + KB - 1) / KB;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ---------------- TMA producer (both CTAs) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued = 0, issued_par = 0;
+      bool ok = true;
+      int g = 0;
+      for (int t = pair; t < total && ok; t += n_pairs) {
+        if (t < tile_pre[g]) g = 0;
+        while (t >= tile_pre[g + 1]) ++g;
+        const int m = grp_off[g + 1] - grp_off[g];
+        const int mt = (m + TBM - 1) / TBM;
+        const int local = t - tile_pre[g];
+        const int n_idx = local / mt, m_idx = local - n_idx * mt;
+        const bool m128 = m - m_idx * TBM <= BM;        // M=128 MMAs: 64 rows per CTA
+        const int a_row = grp_off[g] + m_idx * TBM + (int)rank * (m128 ? 64 : BM);
+        // SwiGLU: first feature of this CTA's rows of MMA 0 (MMA 1: + 128); otherwise the
+        // first W row of this CTA's rows of MMA 0 (MMA 1: + 256)
+        const int b_row0 = g * p.N + n_idx * p.n_out_tile + (int)rank * (EPI == EPI_SWIGLU ? 64 : 128);
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait<true>(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
+                               TIMEOUT_NS)) {
+            ok = false;
+            break;
+          }
+          if (rank == 0) mbar_expect_tx(&full[stage], STAGE_TX);
+          issued |= 1u << stage;
+          issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+          if (!(p.fault == 1 && rank == 0 && pair == 0 && t == pair && kb == 0)) {
+            // (test hook: the leader of pair 0 arms its first stage without loading its
+            // share, so the MMA issuer's bounded wait on that stage runs out)
+            const uint32_t bar = cluster_map(smem_u32(&full[stage]), 0);
+            const uint32_t b_dst = sB + stage * B_BYTES;
+            tma_load_2d_pair(sA + stage * A_BYTES, &tmA, bar, kb * KB, a_row);
+            if (EPI == EPI_SWIGLU) {          // 64-row boxes: gate, up of MMA 0, then MMA 1
+              tma_load_2d_pair(b_dst, &tmB0, bar, kb * KB, b_row0);
+              tma_load_2d_pair(b_dst + BH_BYTES / 2, &tmB1, bar, kb * KB, b_row0);
+              tma_load_2d_pair(b_dst + BH_BYTES, &tmB0, bar, kb * KB, b_row0 + 128);
+              tma_load_2d_pair(b_dst + 3 * BH_BYTES / 2, &tmB1, bar, kb * KB, b_row0 + 128);
+            } else {
+              tma_load_2d_pair(b_dst, &tmB0, bar, kb * KB, b_row0);
+              tma_load_2d_pair(b_dst + BH_BYTES, &tmB0, bar, kb * KB, b_row0 + 256);
+            }
+          }
+          if (++stage == NSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        if (rank == 0) {
+          // let the copies already in flight land before the CTA moves on
+          for (int s = 0; s < NSTAGES; ++s)
+            if (issued & (1u << s))
+              mbar_wait<true>(&full[s], (issued_par >> s) & 1u, abort_flag, p.err,
+                              DEVERR_TIMEOUT_TMA, DRAIN_NS, /*honor_abort=*/false);
+        } else {
+          // this CTA's copies complete on the leader's barriers: give them a fixed time
+          const uint64_t t0 = gtimer();
+          while (gtimer() - t0 < DRAIN_NS / 100) {
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && rank == 0) {
+      // ---------------- MMA issuer (leader only) ----------------
+      int stage = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      int it = 0, g = 0;
+      for (int t = pair; t < total && ok; t += n_pairs, ++it) {
+        if (t < tile_pre[g]) g = 0;
+        while (t >= tile_pre[g + 1]) ++g;
+        const int m = grp_off[g + 1] - grp_off[g];
+        const int mt = (m + TBM - 1) / TBM;
+        const int m_idx = (t - tile_pre[g]) % mt;
+        const uint32_t idesc = (m - m_idx * TBM <= BM) ? kIdescPair128 : kIdescPair256;
+        if (!mbar_wait<true>(tempty, ((uint32_t)it & 1u) ^ 1u, abort_flag, p.err,
+                             DEVERR_TIMEOUT_MMA, TIMEOUT_NS)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < nkb; ++kb) {
+          if (!mbar_wait<true>(&full[stage], phase, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
+                               TIMEOUT_NS)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a0 = sA + stage * A_BYTES, b0 = sB + stage * B_BYTES;
+#pragma unroll
+          for (int k = 0; k < KB / MMA_K; ++k) {
+            const uint64_t adesc = sdesc<KB>(a0 + k * MMA_K * 2);
+            const uint32_t accum = (kb > 0 || k > 0) ? 1u : 0u;
+            umma_bf16_pair(tmem_base, adesc, sdesc<KB>(b0 + k * MMA_K * 2), accum, idesc);
+            umma_bf16_pair(tmem_base + ACC_COLS, adesc,
+                           sdesc<KB>(b0 + BH_BYTES + k * MMA_K * 2), accum, idesc);
+          }
+          umma_commit_both(&empty[stage]);  // frees the stage in both CTAs once read
+          if (++stage == NSTAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (ok) umma_commit_both(tfull);    // both CTAs' accumulators are ready
+      }
+      umma_commit_pair_local(drain);
+      mbar_wait(drain, 0u, abort_flag, p.err, DEVERR_TIMEOUT_MMA, ok ? TIMEOUT_NS : DRAIN_NS,
+                /*honor_abort=*/false);
+    }
+  } else {
+    // ---------------- epilogue (warps 2..9 of both CTAs) ----------------
+    // warp (q, j): TMEM lane quarter q = warp % 4 of MMA j's accumulator columns.
+    //   M=256: rows 32q + lane of this CTA's 128; SwiGLU features n0 + 128j .. +127 (gate at
+    //          MMA columns x and 64 + x for x < 64, 128 + x' and 192 + x' for the next 64),
+    //          otherwise output columns n0 + 256j .. +255.
+    //   M=128: rows 32(q % 2) + lane of this CTA's 64; quarters 2 and 3 hold the MMA's upper
+    //          128 columns: SwiGLU features n0 + 128j + 64(q / 2) .. +63, otherwise output
+    //          columns n0 + 256j + 128(q / 2) .. +127.
+    const int q = warp & 3;
+    const int j = (warp - 2) >> 2;
+    int g = 0, it = 0;
+    for (int t = pair; t < total; t += n_pairs, ++it) {
+      if (t < tile_pre[g]) g = 0;
+      while (t >= tile_pre[g + 1]) ++g;
+      const int m = grp_off[g + 1] - grp_off[g];
+      const int mt = (m + TBM - 1) / TBM;
+      const int local = t - tile_pre[g];
+      const int n_idx = local / mt, m_idx = local - n_idx * mt;
+      int okw = 1;
+      if (lane == 0)
+        okw = mbar_wait<true>(tfull, (uint32_t)it & 1u, abort_flag, p.err, DEVERR_TIMEOUT_EPI,
+                              TIMEOUT_NS);
+      okw = __shfl_sync(0xffffffffu, okw, 0);
+      if (!okw) break;
+      tc_fence_after();
+      const uint32_t release = cluster_map(smem_u32(tempty), 0);
+      const bool m128 = m - m_idx * TBM <= BM;
+      const int r0 = m_idx * TBM + (int)rank * (m128 ? 64 : BM);
+      if (r0 >= m) {                                    // no live rows here: nothing to read
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(release);
+        continue;
+      }
+      const int r = r0 + 32 * (m128 ? (q & 1) : q) + lane;
+      const int64_t orow = (int64_t)grp_off[g] + r;
+      bool valid = r < m;
+      if (valid && (orow < 0 || orow >= p.rows)) {
+        atomicCAS(p.err, 0, DEVERR_BOUNDS);
+        valid = false;
+      }
+      const uint32_t taddr = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(j * ACC_COLS);
+      __nv_bfloat16* orow_ptr = p.out + orow * p.ldo;
+      if (EPI == EPI_SWIGLU) {
+        const int nch = m128 ? 2 : 4;
+        const int f0 = n_idx * p.n_out_tile + 128 * j + (m128 ? 64 * (q >> 1) : 0);
+        // chunks i, i+1 (gate at MMA column 32i (+64 from i = 2), up 64 further) per wait
+#pragma unroll 1
+        for (int i = 0; i < nch; i += 2) {
+          const int gc = 32 * i + (i >= 2 ? 64 : 0);
+          uint32_t g0[32], u0[32], g1[32], u1[32];
+          tmem_ld32(taddr + gc, g0);
+          tmem_ld32(taddr + gc + 64, u0);
+          tmem_ld32(taddr + gc + 32, g1);
+          tmem_ld32(taddr + gc + 96, u1);
+          tmem_wait_ld();
+          if (i + 2 >= nch) {                // last TMEM read of the tile: release it
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(release);
+          }
+          const int f = f0 + 32 * i;
+          if (valid && f < p.N) store_swiglu32(g0, u0, orow_ptr + f);
+          if (valid && f + 32 < p.N) store_swiglu32(g1, u1, orow_ptr + f + 32);
+        }
+      } else {
+        const int nch = m128 ? 4 : 8;
+        const int c0 = n_idx * p.n_out_tile + 256 * j + (m128 ? 128 * (q >> 1) : 0);
+        // four 32-column chunks per wait
+#pragma unroll 1
+        for (int i = 0; i < nch; i += 4) {
+          uint32_t v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(taddr + 32 * i, v0);
+          tmem_ld32(taddr + 32 * i + 32, v1);
+          tmem_ld32(taddr + 32 * i + 64, v2);
+          tmem_ld32(taddr + 32 * i + 96, v3);
+          tmem_wait_ld();
+          if (i + 4 >= nch) {
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive_cluster(release);
+          }
+          const int c = c0 + 32 * i;
+          if (valid && c < p.N) store_act32<EPI>(v0, orow_ptr + c);
+          if (valid && c + 32 < p.N) store_act32<EPI>(v1, orow_ptr + c + 32);
+          if (valid && c + 64 < p.N) store_act32<EPI>(v2, orow_ptr + c + 64);
+          if (valid && c + 96 < p.N) store_act32<EPI>(v3, orow_ptr + c + 96);
+        }
+      }
+    }
+  }
+  // neither CTA leaves (or frees TMEM) while the other may still touch its shared or tensor
+  // memory: the leader's MMAs read the peer's stages and write its TMEM, the peer's loads and
+  // arrives target the leader's barriers
+  __syncwarp();
+  tc_fence_before();
+  cluster_sync_all();
+  if (warp == 1) {
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem_base),
                  "r"(TMEM_COLS)
                  : "memory");
   }
@@ -595,8 +1023,10 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uin
 // bytes per FLOP than 128-row tiles) with 64-element k-blocks in a 3-stage ring.
 // MOE_GEMM_TILE selects another shape for comparison measurements (all are tested):
 //   "128"      128-row tiles, 4 stages, double TMEM buffer;
-//   "256k32"   256-row tiles with 32-element k-blocks (64-byte swizzle) in a 6-7 stage ring.
-enum GemmTile { TILE_128 = 0, TILE_256 = 1, TILE_256_K32 = 2 };
+//   "256k32"   256-row tiles with 32-element k-blocks (64-byte swizzle) in a 6-7 stage ring;
+//   "pair"     256 x 512 accumulator tiles on a CTA pair (cta_group::2), 4 stages of 48 KB
+//              per CTA.
+enum GemmTile { TILE_128 = 0, TILE_256 = 1, TILE_256_K32 = 2, TILE_PAIR = 3 };
 
 int g_gemm_fault = 0;       // set through moe_debug_inject (tests of the bounded waits)
 constexpr int kRouterMaxSplits = 8;
@@ -605,6 +1035,7 @@ GemmTile gemm_tile() {
     const char* v = getenv("MOE_GEMM_TILE");
     if (v && !strcmp(v, "128")) return TILE_128;
     if (v && !strcmp(v, "256k32")) return TILE_256_K32;
+    if (v && !strcmp(v, "pair")) return TILE_PAIR;
     return TILE_256;
   }();
   return t;
@@ -647,6 +1078,62 @@ size_t gemm_smem(int halves, int kb, int nstages, int n_groups) {
   return 1024 + ring + (2 * nstages + 5) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
 }
 
+constexpr int kPairStages = 4;
+size_t pair_smem(int nstages, int n_groups) {
+  const size_t ring = (size_t)nstages * (3 * (size_t)128 * 64 * 2);   // A box + two B boxes
+  return 1024 + ring + (2 * nstages + 3) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
+}
+
+// Co-resident CTA pairs of one pair-kernel instance (queried once per device).
+template <int EPI>
+int pair_slots(size_t smem) {
+  constexpr int kMaxDev = 64;
+  static int cached[kMaxDev] = {};
+  static std::mutex mu;
+  int dev = 0;
+  cudaGetDevice(&dev);
+  std::lock_guard<std::mutex> lock(mu);
+  if (dev >= 0 && dev < kMaxDev && cached[dev] > 0) return cached[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * (sm_count() / 2));
+  cfg.blockDim = dim3(kPairThreads);
+  cfg.dynamicSmemBytes = smem;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, grouped_gemm_pair_kernel<EPI, kPairStages>, &cfg) !=
+          cudaSuccess ||
+      n <= 0) {
+    cudaGetLastError();
+    n = sm_count() / 2;
+  }
+  if (dev >= 0 && dev < kMaxDev) cached[dev] = n;
+  return n;
+}
+
+template <int EPI>
+cudaError_t launch_pair_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
+                            const GemmParams& p, int64_t max_tiles, cudaStream_t s) {
+  auto kern = grouped_gemm_pair_kernel<EPI, kPairStages>;
+  const size_t smem = pair_smem(kPairStages, p.G);
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int slots = pair_slots<EPI>(smem);
+  const int pairs = (int)(max_tiles < slots ? max_tiles : slots);
+  kern<<<counted(2 * pairs), kPairThreads, smem, s>>>(a, b0, b1, p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0,
+                        const CUtensorMap& b1, const GemmParams& p, int64_t max_tiles,
+                        cudaStream_t s) {
+  switch (epi) {
+    case EPI_SWIGLU: return launch_pair_epi<EPI_SWIGLU>(a, b0, b1, p, max_tiles, s);
+    case EPI_RELU: return launch_pair_epi<EPI_RELU>(a, b0, b1, p, max_tiles, s);
+    case EPI_GELU: return launch_pair_epi<EPI_GELU>(a, b0, b1, p, max_tiles, s);
+    default: return launch_pair_epi<EPI_NONE>(a, b0, b1, p, max_tiles, s);
+  }
+}
+
 }  // namespace
 
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
@@ -680,8 +1167,19 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   } else {
     tb1 = tb0;
   }
-  const int tbm = BM * halves;
+  const int tbm = tile == TILE_PAIR ? 2 * BM : BM * halves;
   const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
+  if (tile == TILE_PAIR && offsets) {
+    // 256 x 512 accumulator tiles: 256 SwiGLU features (gate + up) or 512 output columns;
+    // the SwiGLU weights go in 64-row boxes
+    if (epi == EPI_SWIGLU && (!make_map(&tb0, B0, brows, (uint64_t)K, 64, kb) ||
+                              !make_map(&tb1, B1, brows, (uint64_t)K, 64, kb)))
+      return cudaErrorInvalidValue;
+    p.n_out_tile = (epi == EPI_SWIGLU) ? 256 : 512;
+    p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
+    const int64_t pair_tiles = ((a_rows + 2 * BM - 1) / (2 * BM) + n_groups) * (int64_t)p.nt;
+    return launch_pair(epi, ta, tb0, tb1, p, pair_tiles, s);
+  }
   const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
   constexpr size_t kMaxSmem = 232448;          // 227 KB of dynamic shared memory per block
   switch (tile) {

@@ -85,11 +85,11 @@ def test_grouped_gemm_repeatable():
     assert torch.equal(y1[:n], y[:n])
 
 
-@pytest.mark.parametrize("tile", ["128", "256k32"])
+@pytest.mark.parametrize("tile", ["128", "256k32", "pair"])
 def test_grouped_gemm_other_tiles_in_subprocess(tile):
     """The other tile shapes (128-row tiles with a double TMEM buffer; 256-row tiles with
-    32-element k-blocks) are selected per process by MOE_GEMM_TILE; run this file's ragged
-    cases under each in a child process."""
+    32-element k-blocks; 256 x 256 tiles on a CTA pair) are selected per process by
+    MOE_GEMM_TILE; run this file's ragged cases under each in a child process."""
     import os
     import subprocess
     import sys
