@@ -127,3 +127,16 @@ def test_decode_regime_mixtral_shape(T):
     C.check_logits(w, inp, v)
     C.check_routing(w, inp, v)
     C.check_sampled_output(w, inp, out, v, list(range(T)))
+
+
+# The bf16 fast router at larger token counts: each CTA routes several 16-token batches, the
+# last one ragged (T=5000, D=4096: 34 tokens per CTA; T=9000, D=1024: 61; T=12000, D=4096:
+# 82).  Logits of every token, the whole routing, permutation and statistics are compared
+# with the oracle.
+@pytest.mark.parametrize("T,D", [(5000, 4096), (9000, 1024), (12000, 4096)])
+def test_fast_router_many_batches(T, D):
+    w = scaled(W["mixtral"], T=T, D=D, F=256)
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    C.check_logits(w, inp, v)
+    C.check_routing(w, inp, v)
