@@ -33,7 +33,10 @@ Readings where the pages are silent (each one is listed in the design notes):
     normalised to sum 1 over experts;
   * under expert choice the merge weight is the softmax probability, a token
     taken by several experts sums their contributions, an untaken token gets 0;
-  * shared experts are added with weight 1.
+  * shared experts are added with weight 1;
+  * group-limited selection scores a group by its largest selection key and
+    keeps each token's topk_group best groups (ties -> lower group index)
+    before the top-k.
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (worked examples of the pages, closed forms, brute force and reductions to
@@ -48,7 +51,7 @@ import numpy as np
 
 __all__ = [
     "router_logits", "softmax_rows", "sigmoid", "routing_keys",
-    "topk_desc", "route_token_choice", "route_expert_choice",
+    "topk_desc", "group_limit_mask", "route_token_choice", "route_expert_choice",
     "capacity", "dispatch_token_choice", "dispatch_expert_choice",
     "swiglu_expert", "relu_expert", "gelu", "gelu_expert", "expert_rows",
     "combine", "balance_stats", "layer_forward", "layer_forward_rows",
@@ -127,7 +130,33 @@ def topk_desc(keys, k):
     return order[:, :k]
 
 
-def route_token_choice(logits, k, score="softmax", gate="renorm", bias=None):
+def group_limit_mask(keys, n_group, topk_group):
+    """Experts each token may select under group-limited routing.
+
+    [RAT] routing variant (c): groups are chosen first, then experts inside
+    the chosen groups; [CMP] "Group/node limited" row (the candidate set
+    shrinks to the experts of the allowed devices or nodes) and its
+    DeepSeek-V3 note (256 experts on 8 nodes, a token's top-8 on at most 4
+    nodes).  The experts are split into n_group contiguous groups of
+    E / n_group.  The pages do not say how a group is scored; the reading
+    here: a group scores its largest selection key, and each token keeps its
+    topk_group highest-scoring groups (ties -> lower group index).
+    Returns a boolean [T, E] mask.
+    """
+    keys = np.asarray(keys, dtype=np.float64)
+    T, E = keys.shape
+    if E % n_group:
+        raise ValueError("n_group must divide E")
+    size = E // n_group
+    scores = keys.reshape(T, n_group, size).max(axis=2)
+    best = topk_desc(scores, topk_group)
+    allowed = np.zeros((T, n_group), dtype=bool)
+    np.put_along_axis(allowed, best, True, axis=1)
+    return np.repeat(allowed, size, axis=1)
+
+
+def route_token_choice(logits, k, score="softmax", gate="renorm", bias=None,
+                       n_group=1, topk_group=1):
     """Token-choice routing from router logits.
 
     Returns (ids[T,k] int, gates[T,k], probs_for_importance[T,E]).
@@ -141,22 +170,28 @@ def route_token_choice(logits, k, score="softmax", gate="renorm", bias=None):
     * sigmoid (+ optional selection-only bias): select on sigma(s) + b,
       merge weight sigma(s_j) / sum_sel sigma(s)  (bias excluded) --
       [CMP] "Select" / "Merge" steps, DeepSeek-V3 row of the family table.
+    * n_group > 1 and topk_group < n_group: the top-k runs over the experts of
+      the token's topk_group best groups only (group_limit_mask); merge
+      weights and importance are unchanged in form.
     """
     s = np.asarray(logits, dtype=np.float64)
     T, E = s.shape
     if score == "softmax":
         p = softmax_rows(s)
-        ids = topk_desc(s, k)
-        psel = np.take_along_axis(p, ids, axis=1)
+        key = s
+        weight = p
         imp = p
     elif score == "sigmoid":
         a = sigmoid(s)
         key = a + (np.asarray(bias, dtype=np.float64)[None, :] if bias is not None else 0.0)
-        ids = topk_desc(key, k)
-        psel = np.take_along_axis(a, ids, axis=1)
+        weight = a
         imp = a / a.sum(axis=1, keepdims=True)
     else:
         raise ValueError(score)
+    if n_group > 1 and topk_group < n_group:
+        key = np.where(group_limit_mask(key, n_group, topk_group), key, -np.inf)
+    ids = topk_desc(key, k)
+    psel = np.take_along_axis(weight, ids, axis=1)
     if gate == "renorm":
         g = psel / psel.sum(axis=1, keepdims=True)
     elif gate == "raw":
@@ -389,7 +424,8 @@ def route(w, logits, bias=None):
     """
     g = _get(w)
     if g["select"] == "token":
-        ids, gates, imp = route_token_choice(logits, g["k"], g["score"], g["gate"], bias)
+        ids, gates, imp = route_token_choice(logits, g["k"], g["score"], g["gate"], bias,
+                                             g["n_group"], g["topk_group"])
         cap = capacity(g["capacity_factor"], g["T"], g["k"], g["E"]) if g["overflow"] == "drop" else None
         counts, kept, offsets, row_src, inv = dispatch_token_choice(ids, g["E"], cap)
         K = g["k"]
@@ -409,9 +445,14 @@ def route(w, logits, bias=None):
 def _get(w):
     keys = ["T", "D", "E", "F", "k", "c", "score", "select", "gate", "overflow",
             "capacity_factor", "act", "n_shared", "F_shared", "aux_alpha"]
+    optional = {"n_group": 1, "topk_group": 1}      # no group limit unless given
     if isinstance(w, dict):
-        return {k: w[k] for k in keys}
-    return {k: getattr(w, k) for k in keys}
+        out = {k: w[k] for k in keys}
+        out.update({k: w.get(k, v) for k, v in optional.items()})
+        return out
+    out = {k: getattr(w, k) for k in keys}
+    out.update({k: getattr(w, k, v) for k, v in optional.items()})
+    return out
 
 
 def layer_forward(w, x, Wg, bias, W_gate, W_up, W_down,
@@ -510,7 +551,8 @@ def dense_masked_forward(w, x, Wg, bias, W_gate, W_up, W_down):
     g = _get(w)
     x = _np(x)
     s = router_logits(x, _np(Wg))
-    ids, gates, _ = route_token_choice(s, g["k"], g["score"], g["gate"], _np(bias))
+    ids, gates, _ = route_token_choice(s, g["k"], g["score"], g["gate"], _np(bias),
+                                       g["n_group"], g["topk_group"])
     Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
     T = x.shape[0]
     allout = np.stack([expert_rows(g["act"], x, e, Wgt, Wu, Wd) for e in range(g["E"])], 1)

@@ -443,3 +443,75 @@ def test_count_percentiles_of_the_page_example():
     st = O.balance_stats(np.full((1, 4), 0.25), g["counts"], g["total"], g["total"], 1e-2)
     np.testing.assert_allclose(st["count_p95"], 8.25, rtol=1e-12)
     np.testing.assert_allclose(st["count_p99"], 8.85, rtol=1e-12)
+
+
+# ------------------------------------------------ group-limited selection ----
+# [RAT] variant (c) (choose groups, then experts inside them); [CMP] "Group/node limited" row
+# and the DeepSeek-V3 note (256 experts on 8 nodes, a token's top-8 on at most 4 nodes).
+
+def test_group_limit_hand_example():
+    # E = 4 in 2 groups {0,1} {2,3}; keys [0.9, 0.1 | 0.89, 0.88], k = 2.  Plain top-2 is
+    # {0, 2} (two groups).  With one group allowed, group 0 (best key 0.9 > 0.89) is kept and
+    # the top-2 inside it is [0, 1] -- the limit trades expert 2 (0.89) for expert 1 (0.1).
+    s = np.array([[0.9, 0.1, 0.89, 0.88]])
+    ids, _, _ = O.route_token_choice(s, 2, "softmax", "renorm")
+    assert ids.tolist() == [[0, 2]]
+    ids, gates, _ = O.route_token_choice(s, 2, "softmax", "renorm", n_group=2, topk_group=1)
+    assert ids.tolist() == [[0, 1]]
+    p = np.exp(s[0]) / np.exp(s[0]).sum()
+    np.testing.assert_allclose(gates[0], [p[0] / (p[0] + p[1]), p[1] / (p[0] + p[1])], rtol=1e-14)
+    assert O.group_limit_mask(s, 2, 1).tolist() == [[True, True, False, False]]
+    # equal group scores go to the lower group index
+    t = np.array([[0.5, 0.1, 0.5, 0.2]])
+    assert O.group_limit_mask(t, 2, 1).tolist() == [[True, True, False, False]]
+
+
+def test_group_limit_reduces_to_plain_topk():
+    rng = np.random.default_rng(31)
+    s = rng.normal(size=(50, 16))
+    b = rng.normal(scale=0.1, size=16)
+    for score, bias in (("softmax", None), ("sigmoid", b)):
+        plain = O.route_token_choice(s, 3, score, "renorm", bias)
+        for n_group, topk_group in ((1, 1), (4, 4), (16, 16)):
+            lim = O.route_token_choice(s, 3, score, "renorm", bias, n_group, topk_group)
+            assert np.array_equal(plain[0], lim[0])
+            np.testing.assert_array_equal(plain[1], lim[1])
+
+
+def test_group_limit_invariants_at_the_node_shape():
+    # V3 node shape: E = 256 in 8 groups of 32, top-8 on at most 4 groups
+    rng = np.random.default_rng(32)
+    s = rng.normal(size=(300, 256))
+    b = rng.normal(scale=0.1, size=256)
+    a = O.sigmoid(s)
+    key = a + b
+    plain, _, _ = O.route_token_choice(s, 8, "sigmoid", "renorm", b)
+    ids, gates, _ = O.route_token_choice(s, 8, "sigmoid", "renorm", b, n_group=8, topk_group=4)
+    groups = ids // 32
+    assert all(len(set(row)) <= 4 for row in groups.tolist())
+    # the token's best expert is always kept (its group has the largest score)
+    assert np.array_equal(ids[:, 0], np.argmax(key, axis=1))
+    # with distinct keys, a plain top-k that already spans <= 4 groups is unchanged
+    spans = np.array([len(set(row)) for row in (plain // 32).tolist()])
+    same = spans <= 4
+    assert same.any() and (~same).any()
+    assert np.array_equal(ids[same], plain[same])
+    # otherwise the limited set is the top-8 inside the 4 groups of largest best key
+    for t in np.nonzero(~same)[0][:20]:
+        gbest = key[t].reshape(8, 32).max(axis=1)
+        keep = sorted(np.argsort(-gbest, kind="stable")[:4].tolist())
+        cand = [e for e in range(256) if e // 32 in keep]
+        want = sorted(cand, key=lambda e: (-key[t, e], e))[:8]
+        assert ids[t].tolist() == want
+    np.testing.assert_allclose(gates.sum(axis=1), 1.0, rtol=1e-14)
+
+
+def test_group_limited_dropless_layer_is_dense_masked():
+    c = cfg(T=12, D=6, E=8, F=5, k=2)
+    c.update(n_group=4, topk_group=1)
+    rng = np.random.default_rng(33)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    r = O.layer_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    dense = O.dense_masked_forward(c, x, Wg, None, Wgate, Wup, Wdown)
+    np.testing.assert_allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
+    assert all(len(set(row)) == 1 for row in (r["ids"] // 2).tolist())
