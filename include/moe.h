@@ -67,7 +67,16 @@ enum { MOE_F32 = 0, MOE_BF16 = 1 };                      /* operand dtype */
  *   overflow : DROPLESS, or CAPACITY_DROP with C = ceil(capacity_factor * T * k / E) slots per
  *              expert, evaluated in double ("Top-k 路由" capacity factor formula); the first C
  *              assignments of an expert in (token, slot) order keep a slot, later ones add 0;
- *   aux_alpha: alpha of the balance loss alpha * E * sum_e f_e P_e. */
+ *   aux_alpha: alpha of the balance loss alpha * E * sum_e f_e P_e;
+ *   n_group, topk_group : group-limited token choice (talentme M4-080 routing variant (c):
+ *              groups first, then experts inside them; moe-comparison "Group/node limited" row,
+ *              DeepSeek-V3: 256 experts on 8 nodes, a token's top-8 on at most 4).  The experts
+ *              are split into n_group contiguous groups of E / n_group; a group scores its
+ *              largest selection key and each token keeps its topk_group best groups (ties to the
+ *              lower group index) before the top-k.  n_group <= 1 or topk_group == n_group:
+ *              no limit.  Limits: n_group <= 32 and divides E, E / n_group a power of two
+ *              <= 32 or a multiple of 32, 1 <= topk_group <= n_group, topk_group * E / n_group
+ *              >= k; token choice only. */
 typedef struct moe_desc {
     int32_t T, D, E, F;
     int32_t k;
@@ -76,6 +85,7 @@ typedef struct moe_desc {
     int32_t score, select, gate, overflow, act, dtype;
     float capacity_factor;
     float aux_alpha;
+    int32_t n_group, topk_group;
 } moe_desc_t;
 
 /* Scalars of the balance statistics (written to device memory by moe_balance_stats). */

@@ -42,7 +42,8 @@ class MoeDesc(ctypes.Structure):
                 ("n_shared", ctypes.c_int32), ("F_shared", ctypes.c_int32),
                 ("score", ctypes.c_int32), ("select", ctypes.c_int32), ("gate", ctypes.c_int32),
                 ("overflow", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("capacity_factor", ctypes.c_float), ("aux_alpha", ctypes.c_float)]
+                ("capacity_factor", ctypes.c_float), ("aux_alpha", ctypes.c_float),
+                ("n_group", ctypes.c_int32), ("topk_group", ctypes.c_int32)]
 
 
 class MoeStats(ctypes.Structure):
@@ -152,7 +153,8 @@ def desc_of(w, T=None) -> MoeDesc:
         overflow=DROPLESS if w.overflow == "dropless" else CAPACITY_DROP,
         act={"swiglu": SWIGLU, "relu": RELU, "gelu": GELU}[w.act],
         dtype=BF16 if w.dtype == "bf16" else F32,
-        capacity_factor=w.capacity_factor, aux_alpha=w.aux_alpha)
+        capacity_factor=w.capacity_factor, aux_alpha=w.aux_alpha,
+        n_group=getattr(w, "n_group", 1), topk_group=getattr(w, "topk_group", 1))
 
 
 def _ptr(t):

@@ -59,6 +59,16 @@ moe_status_t validate(const moe_desc_t* d) {
     if ((int64_t)d->T * d->E >= (int64_t)1 << 31) return MOE_ERR_UNSUPPORTED;
   }
   if (!(d->aux_alpha >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (d->n_group < 0 || d->topk_group < 0) return MOE_ERR_INVALID_ARG;
+  if (d->n_group > 1) {
+    if (d->select != MOE_TOKEN_CHOICE) return MOE_ERR_UNSUPPORTED;
+    if (d->E % d->n_group || d->topk_group < 1 || d->topk_group > d->n_group)
+      return MOE_ERR_INVALID_ARG;
+    const int size = d->E / d->n_group;
+    if ((int64_t)d->topk_group * size < d->k) return MOE_ERR_INVALID_ARG;
+    const bool pow2 = (size & (size - 1)) == 0;
+    if (d->n_group > 32 || !((pow2 && size <= 32) || size % 32 == 0)) return MOE_ERR_UNSUPPORTED;
+  }
   if (d->dtype == MOE_BF16) {
     if (d->D % 64 || d->F % 64) return MOE_ERR_UNSUPPORTED;
     if (d->n_shared > 0 && d->F_shared % 64) return MOE_ERR_UNSUPPORTED;

@@ -62,7 +62,56 @@ struct RouterArgs {
   int T, D, E, k, score, gate, expert_choice;
   const float* lpart;       // when set: logits are the sum of ksplit partials [ksplit][T][E]
   int ksplit;
+  int n_group = 1, topk_group = 1;   // group-limited selection (n_group <= 1: none)
 };
+
+// Group-limited selection ("Mixture of Experts (MoE)" routing variant (c): groups first, then
+// experts inside them; moe-comparison "Group/node limited" row).  The experts form n_group
+// contiguous groups of size = E / n_group; a group scores its largest key, the token keeps its
+// topk_group best groups (ties to the lower group) and every other expert's key becomes -inf.
+// Lane l holds experts l + 32 i in key[i].  size is a power of two <= 32 (a group lies inside
+// one register slot: a segmented shuffle max) or a multiple of 32 (a slot lies inside one
+// group: a warp max); n_group <= 32, so lane g can hold group g's score.
+template <int NS>
+__device__ __forceinline__ void group_limit(float (&key)[NS], int E, int n_group, int topk_group,
+                                            int lane) {
+  if (n_group <= 1 || topk_group >= n_group) return;
+  const int size = E / n_group;
+  float gs = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    if (32 * i >= E) break;
+    float v = (lane + 32 * i < E) ? key[i] : -INFINITY;
+    if (size < 32) {
+      for (int o = size >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+      const int src = lane * size - 32 * i;     // first lane of group `lane` in slot i
+      const float w = __shfl_sync(0xffffffffu, v, src & 31);
+      if (lane < n_group && src >= 0 && src < 32) gs = fmaxf(gs, w);
+    } else {
+      v = warp_max(v);
+      if (lane == (32 * i) / size) gs = fmaxf(gs, v);
+    }
+  }
+  uint32_t kept = 0;
+  bool used = lane >= n_group;
+  for (int r = 0; r < topk_group; ++r) {
+    float bk = used ? -INFINITY : gs;
+    int bi = used ? 0x7fffffff : lane;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
+      if (ok > bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
+    }
+    kept |= 1u << (bi & 31);
+    if (lane == bi) used = true;
+  }
+#pragma unroll
+  for (int i = 0; i < NS; ++i) {
+    const int e = lane + 32 * i;
+    if (e < E && !((kept >> (e / size)) & 1u)) key[i] = -INFINITY;
+  }
+}
 
 // logits of the warp's TPW tokens for all experts -> s_log[TPW][E]
 template <bool BF16>
@@ -212,6 +261,8 @@ router_kernel(RouterArgs a) {
       }
       continue;
     }
+
+    group_limit<kMaxEPL>(key, E, a.n_group, a.topk_group, lane);
 
     // top-k: k rounds of a warp arg-max over (key desc, expert id asc)
     bool taken[kMaxEPL];
@@ -433,6 +484,11 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float
     imp += q;
     if (q > 0.f) ent -= q * logf(q);
   }
+  {
+    float kk[1] = {key};
+    group_limit<1>(kk, E, a.n_group, a.topk_group, lane);
+    key = kk[0];
+  }
   bool taken = !live;
   int my_id = -1;
   float my_w = 0.f, wsum = 0.f;
@@ -571,6 +627,8 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
                                        float* lpart, cudaStream_t s) {
   RouterArgs a{x, Wg, bias, ids, gates, logits, nullptr, imp_partials,
                d.T, d.D, d.E, d.k, d.score, d.gate, 0, nullptr, 1};
+  a.n_group = d.n_group;
+  a.topk_group = d.topk_group;
   if (router_uses_gemm(d) && lpart) {
     const int ks = router_gemm_splits(d.T, d.D);
     cudaError_t e = launch_router_gemm_bf16(x, d.T, d.D, Wg, d.E, lpart, ks, s);

@@ -49,6 +49,8 @@ class Workload:
     n_shared: int = 0
     F_shared: int = 0
     aux_alpha: float = 1e-2
+    n_group: int = 1           # group-limited selection: expert groups (1 = no limit)
+    topk_group: int = 1        # groups each token may use
     x_std: float = 1.0
     w_std: float = 0.02
     wg_std: float = 0.02
@@ -146,6 +148,8 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", experts: bool = True,
     is the caller's routing-key function.  When it is given with key_gap > 0
     (token choice), every token whose k+1 largest keys are not pairwise
     separated by key_gap has its x row redrawn from a sub-seed until they are.
+    key_fn may instead return a list of (scores[n,m], j) pairs: then the j
+    largest scores of every row of every pair must be pairwise separated.
     With ec_gap > 0 (expert choice, key_fn returning probabilities), the
     tokens sitting at each expert's c-th / (c+1)-th boundary are redrawn
     until the boundary gap is at least ec_gap.
@@ -224,10 +228,14 @@ def _separate_keys(w, inp, seed, key_fn, key_gap, ec_gap, max_rounds):
     for rnd in range(max_rounds):
         bad = []
         if w.select == "token" and key_gap > 0:
-            m = min(w.k + 1, w.E)
-            top = -np.sort(-keys, axis=1)[:, :m]
-            gaps = top[:, :-1] - top[:, 1:]
-            bad = np.nonzero((gaps < key_gap).any(axis=1))[0].tolist()
+            pairs = keys if isinstance(keys, list) else [(keys, w.k + 1)]
+            worst = np.zeros(pairs[0][0].shape[0], dtype=bool)
+            for sc, j in pairs:
+                m = min(j, sc.shape[1])
+                top = -np.sort(-sc, axis=1)[:, :m]
+                gaps = top[:, :-1] - top[:, 1:]
+                worst |= (gaps < key_gap).any(axis=1)
+            bad = np.nonzero(worst)[0].tolist()
         elif w.select == "expert" and ec_gap > 0 and w.c < w.T:
             c = w.c
             order = np.argsort(-keys, axis=0, kind="stable")   # per expert column
@@ -242,6 +250,11 @@ def _separate_keys(w, inp, seed, key_fn, key_gap, ec_gap, max_rounds):
         redrawn.update(bad)
         _redraw(w, inp, bad, seed, rnd)
         idx = torch.as_tensor(bad, dtype=torch.long, device=inp.x.device)
-        keys[bad] = key_fn(inp.x[idx].float().cpu().double().numpy(), Wg, b)
+        new = key_fn(inp.x[idx].float().cpu().double().numpy(), Wg, b)
+        if isinstance(keys, list):
+            for (sc, _), (nsc, _) in zip(keys, new):
+                sc[bad] = nsc
+        else:
+            keys[bad] = new
     raise RuntimeError(f"could not separate router keys of workload {w.name} "
                        f"in {max_rounds} rounds")

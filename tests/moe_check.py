@@ -29,6 +29,15 @@ TOL_GATES = 1e-5
 def key_fn_for(w):
     if w.select == "expert":
         return lambda x, Wg, b: O.softmax_probs_of(x, Wg)
+    if w.n_group > 1 and w.topk_group < w.n_group:
+        # group-limited: separate the k+1 best keys, the topk_group+1 best group scores and
+        # the k+1 best keys inside the kept groups
+        def fn(x, Wg, b):
+            key = O.routing_keys(x, Wg, b, w.score)
+            gs = key.reshape(key.shape[0], w.n_group, -1).max(axis=2)
+            inside = np.where(O.group_limit_mask(key, w.n_group, w.topk_group), key, -1e30)
+            return [(key, w.k + 1), (gs, w.topk_group + 1), (inside, w.k + 1)]
+        return fn
     return lambda x, Wg, b: O.routing_keys(x, Wg, b, w.score)
 
 
@@ -79,7 +88,8 @@ def check_logits(w, inp, v, rows=None):
 def wdict(w):
     return dict(T=w.T, D=w.D, E=w.E, F=w.F, k=w.k, c=w.c, score=w.score, select=w.select,
                 gate=w.gate, overflow=w.overflow, capacity_factor=w.capacity_factor, act=w.act,
-                n_shared=w.n_shared, F_shared=w.F_shared, aux_alpha=w.aux_alpha)
+                n_shared=w.n_shared, F_shared=w.F_shared, aux_alpha=w.aux_alpha,
+                n_group=w.n_group, topk_group=w.topk_group)
 
 
 def check_routing(w, inp, v):

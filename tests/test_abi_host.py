@@ -66,10 +66,24 @@ def _bad(**kw):
     (dict(F=100), 2), (dict(overflow=1, capacity_factor=0.0), 1),
     (dict(select=1, c=0), 1), (dict(select=1, c=5000), 1), (dict(select=1, c=8, score=1), 2),
     (dict(act=3), 1),
+    # group-limited selection (Mixtral: E = 8, k = 2)
+    (dict(n_group=3, topk_group=1), 1),              # 3 does not divide 8
+    (dict(n_group=4, topk_group=0), 1), (dict(n_group=4, topk_group=5), 1),
+    (dict(n_group=8, topk_group=1), 1),              # 1 group of 1 expert < k = 2
+    (dict(n_group=-1), 1), (dict(select=1, c=8, n_group=2, topk_group=1), 2),
+    (dict(E=96, n_group=32, topk_group=4), 2),       # groups of 3 experts
 ])
 def test_invalid_descriptors_are_rejected(kw, status):
     v = ctypes.c_size_t()
     assert M.lib().moe_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == status
+
+
+def test_group_limited_descriptors_are_accepted():
+    v = ctypes.c_size_t()
+    for kw in (dict(n_group=4, topk_group=1), dict(n_group=2, topk_group=2),
+               dict(n_group=0, topk_group=0), dict(E=256, k=8, n_group=8, topk_group=4),
+               dict(E=64, k=6, n_group=2, topk_group=1)):
+        assert M.lib().moe_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == 0, kw
 
 
 def test_null_pointers_rejected_before_launch():

@@ -48,6 +48,20 @@ SMALL = {
     "gelu_f32": scaled(W["tiny"], act="gelu", T=40),
     # more than 65536 assignments: the multi-block permute path
     "large_A": scaled(W["mixtral"], T=33000, D=128, F=128),
+    # group-limited selection: fast router (groups of 2 experts, softmax; groups of 2, sigmoid
+    # with selection bias), generic fp32 router (groups of 4), tensor-core router (groups of
+    # 32 = one register slot, and of 64 = two slots)
+    "groups_fast_softmax": scaled(W["mixtral"], T=300, D=1024, E=8, k=2, F=256, n_group=4,
+                                  topk_group=1),
+    "groups_fast_sigmoid": scaled(W["v3"], T=200, D=1024, E=8, k=3, F=256, F_shared=256,
+                                  n_group=4, topk_group=2),
+    "groups_f32_generic": scaled(W["v3"], dtype="f32", T=90, D=64, E=16, F=32, k=3,
+                                 n_shared=1, F_shared=40, w_std=0.1, wg_std=0.1, n_group=4,
+                                 topk_group=2),
+    "groups_gemm_router_32": scaled(W["v3"], T=300, D=512, E=64, F=256, F_shared=256,
+                                    n_group=2, topk_group=1),
+    "groups_gemm_router_64": scaled(W["v3"], T=300, D=512, E=128, k=4, F=256, F_shared=256,
+                                    n_group=2, topk_group=1),
 }
 
 
@@ -140,3 +154,29 @@ def test_fast_router_many_batches(T, D):
     out, v = C.run_layer(w, inp)
     C.check_logits(w, inp, v)
     C.check_routing(w, inp, v)
+
+
+
+# Group-limited routing: every token's experts lie in at most topk_group groups, and the full
+# DeepSeek-V3 node shape (256 experts on 8 groups, top-8 on at most 4) matches the oracle.
+@pytest.mark.parametrize("name", [n for n in SMALL if n.startswith("groups_")])
+def test_group_limit_spans_at_most_topk_group_groups(name):
+    w = SMALL[name]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    ids = v["expert_ids"].cpu().numpy()
+    size = w.E // w.n_group
+    assert max(len(set(row)) for row in (ids // size).tolist()) <= w.topk_group
+
+
+def test_v3_node_limited_full_size():
+    w = scaled(W["v3"], n_group=8, topk_group=4)
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    C.check_logits(w, inp, v)
+    ref = C.check_routing(w, inp, v)
+    groups = ref["ids"] // 32
+    assert max(len(set(row)) for row in groups.tolist()) <= 4
+    rng = np.random.default_rng(124)
+    tokens = sorted(rng.choice(w.T, size=6, replace=False).tolist())
+    C.check_sampled_output(w, inp, out, v, tokens)
