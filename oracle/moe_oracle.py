@@ -55,6 +55,7 @@ __all__ = [
     "capacity", "dispatch_token_choice", "dispatch_expert_choice",
     "swiglu_expert", "relu_expert", "gelu", "gelu_expert", "expert_rows",
     "combine", "balance_stats", "layer_forward", "layer_forward_rows",
+    "silu_grad", "gelu_grad", "expert_backward", "gate_logit_grad", "layer_backward",
     "dense_masked_forward", "soft_routing_forward",
 ]
 
@@ -539,6 +540,175 @@ def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
     r.update(logits=s, out_rows=np.stack([out[t] for t in tokens]) if tokens else
              np.zeros((0, g["D"])))
     return r
+
+
+# --------------------------------------------------------------------------
+# Backward pass with the selection fixed
+# --------------------------------------------------------------------------
+# [TKR] "門控網路的梯度流": the discrete top-k is not differentiated; the gate
+# scores of the selected experts carry the gradient, unselected experts get
+# none from the gates.  [TINY] section 9: total loss = task loss + weight x
+# router aux loss; selected experts' gate/up/down matrices, the selected route
+# weights (task loss) and the soft importance (balance loss) get gradients;
+# the expert indices are fixed integers.  The loss here is
+#   L = <dout, out> + aux_grad * aux,
+# i.e. dout = dL/dout and aux_grad = dL/daux are given.  The selection-only
+# bias is not trained by gradients (the pages update it by a rule).
+
+def silu_grad(z):
+    """d/dz of z * sigma(z) = sigma(z) * (1 + z * (1 - sigma(z)))."""
+    z = np.asarray(z, dtype=np.float64)
+    sg = 1.0 / (1.0 + np.exp(-z))
+    return sg * (1.0 + z * (1.0 - sg))
+
+
+def gelu_grad(z):
+    """d/dz of z * Phi(z) = Phi(z) + z * phi(z)."""
+    from scipy.special import erf
+    z = np.asarray(z, dtype=np.float64)
+    return 0.5 * (1.0 + erf(z / math.sqrt(2.0))) + z * np.exp(-0.5 * z * z) / math.sqrt(2.0 * math.pi)
+
+
+def expert_backward(act, xr, dy, Wgate, Wup, Wdown):
+    """Gradients of one expert FFN on its rows xr, given dy = dL/dy_rows.
+
+    Returns (dx_rows, dW_gate or None, dW_up, dW_down).  Chain rule through
+    [TINY] section 3's expert (SwiGLU: h = SiLU(x W_gate^T) * (x W_up^T),
+    y = h W_down^T; the classic FFN with ReLU or GELU).
+    """
+    xr = np.asarray(xr, dtype=np.float64)
+    dy = np.asarray(dy, dtype=np.float64)
+    Wu = np.asarray(Wup, dtype=np.float64)
+    Wd = np.asarray(Wdown, dtype=np.float64)
+    if act == "swiglu":
+        Wg = np.asarray(Wgate, dtype=np.float64)
+        a = xr @ Wg.T
+        b = xr @ Wu.T
+        h = silu(a) * b
+        dh = dy @ Wd
+        da = dh * b * silu_grad(a)
+        db = dh * silu(a)
+        return da @ Wg + db @ Wu, da.T @ xr, db.T @ xr, dy.T @ h
+    z = xr @ Wu.T
+    if act == "relu":
+        h, dz_dh = np.maximum(z, 0.0), (z > 0).astype(np.float64)
+    elif act == "gelu":
+        h, dz_dh = gelu(z), gelu_grad(z)
+    else:
+        raise ValueError(act)
+    dz = (dy @ Wd) * dz_dh
+    return dz @ Wu, None, dz.T @ xr, dy.T @ h
+
+
+def gate_logit_grad(logits, ids, dgates, score="softmax", gate="renorm", bias=None):
+    """dL/ds from dL/dg of the merge weights, the selection ids held fixed.
+
+    softmax + renorm: g_j = softmax over the selected logits ([TKR] masked
+    softmax), so ds_i = g_i (dg_i - sum_j g_j dg_j) for selected i, 0
+    otherwise ([TKR]: unselected experts' gate derivative is 0).
+    softmax + raw: g_j = p_{id_j}, p = softmax over all E:
+    ds = p (.) (dp - <p, dp>), dp scattered from dg.
+    sigmoid + renorm: g_j = a_j / sum_sel a (a = sigma(s)):
+    da_i = (dg_i - sum_j g_j dg_j) / sum_sel a, ds = da a (1 - a).
+    sigmoid + raw: da_i = dg_i, ds = da a (1 - a).
+    """
+    s = np.asarray(logits, dtype=np.float64)
+    T, E = s.shape
+    ids = np.asarray(ids)
+    dg = np.asarray(dgates, dtype=np.float64)
+    ds = np.zeros((T, E), dtype=np.float64)
+    for t in range(T):
+        sel = ids[t]
+        if score == "softmax":
+            if gate == "renorm":
+                z = np.exp(s[t, sel] - s[t, sel].max())
+                g = z / z.sum()
+                ds[t, sel] = g * (dg[t] - np.dot(g, dg[t]))
+            else:
+                p = softmax_rows(s[t:t + 1])[0]
+                dp = np.zeros(E)
+                np.add.at(dp, sel, dg[t])
+                ds[t] = p * (dp - np.dot(p, dp))
+        else:
+            a = sigmoid(s[t])
+            da = np.zeros(E)
+            if gate == "renorm":
+                asel = a[sel]
+                g = asel / asel.sum()
+                np.add.at(da, sel, (dg[t] - np.dot(g, dg[t])) / asel.sum())
+            else:
+                np.add.at(da, sel, dg[t])
+            ds[t] = da * a * (1.0 - a)
+    return ds
+
+
+def layer_backward(w, x, Wg, bias, W_gate, W_up, W_down, dout, aux_grad=1.0, logits=None):
+    """Gradients of L = <dout, out> + aux_grad * aux for one MoE layer, the
+    routing of layer_forward held fixed (no shared experts).
+
+    Per kept assignment (t, j) -> row r of expert e: dy_r = g[t,j] dout[t] and
+    dg[t,j] = <dout[t], y_r>; a dropped assignment has neither.  Experts:
+    expert_backward on their rows.  Router: ds = gate_logit_grad(dg) plus the
+    balance-loss term: aux = alpha E sum_e f_e P_e with f fixed (counts) and
+    P_e = mean_t of the importance rows, so dP_e = aux_grad alpha E f_e / T,
+    pushed through softmax over all E (ds = p (dq - <p, dq>)) or through
+    q = a / sum_e a under sigmoid (da = (dq - <q, dq>) / sum a, ds = da a (1-a)).
+    dW_g = ds^T x, and dx = sum_j dx_rows[r(t, j)] + ds W_g.
+    """
+    g = _get(w)
+    if g["n_shared"] or g["select"] != "token":
+        raise ValueError("backward: token choice without shared experts")
+    x = _np(x)
+    Wg = _np(Wg)
+    r = layer_forward(w, x, Wg, bias, W_gate, W_up, W_down, logits=logits)
+    s, K, T, E = r["logits"], r["K"], g["T"], g["E"]
+    dout = np.asarray(dout, dtype=np.float64)
+    inv = np.asarray(r["inv"]).reshape(T, K)
+    gates = np.asarray(r["gates"], dtype=np.float64).reshape(T, K)
+    y = r["y_rows"]
+    A = len(r["row_src"])
+    dy = np.zeros((A, g["D"]), dtype=np.float64)
+    dgates = np.zeros((T, K), dtype=np.float64)
+    for t in range(T):
+        for j in range(K):
+            row = inv[t, j]
+            if row >= 0:
+                dy[row] = gates[t, j] * dout[t]
+                dgates[t, j] = float(np.dot(dout[t], y[row]))
+    Wgt, Wu, Wd = _np(W_gate), _np(W_up), _np(W_down)
+    dWgate = np.zeros_like(Wgt) if Wgt is not None else None
+    dWup, dWdown = np.zeros_like(Wu), np.zeros_like(Wd)
+    dx_rows = np.zeros((A, g["D"]), dtype=np.float64)
+    off = r["offsets"]
+    for e in range(E):
+        rows = slice(off[e], off[e + 1])
+        if off[e + 1] == off[e]:
+            continue
+        xr = x[r["row_src"][rows] // K]
+        dxr, dge, due, dde = expert_backward(g["act"], xr, dy[rows],
+                                             Wgt[e] if Wgt is not None else None, Wu[e], Wd[e])
+        dx_rows[rows] = dxr
+        if dge is not None:
+            dWgate[e] = dge
+        dWup[e], dWdown[e] = due, dde
+    ds = gate_logit_grad(s, r["ids"], dgates, g["score"], g["gate"], _np(bias))
+    f = r["stats"]["f"]
+    dq = np.broadcast_to(aux_grad * g["aux_alpha"] * E * f / T, (T, E))
+    if g["score"] == "softmax":
+        p = softmax_rows(s)
+        ds = ds + p * (dq - np.sum(p * dq, axis=1, keepdims=True))
+    else:
+        a = sigmoid(s)
+        q = a / a.sum(axis=1, keepdims=True)
+        da = (dq - np.sum(q * dq, axis=1, keepdims=True)) / a.sum(axis=1, keepdims=True)
+        ds = ds + da * a * (1.0 - a)
+    dx = ds @ Wg
+    for t in range(T):
+        for j in range(K):
+            if inv[t, j] >= 0:
+                dx[t] += dx_rows[inv[t, j]]
+    return dict(forward=r, dx=dx, dWg=ds.T @ x, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown,
+                dgates=dgates, dlogits=ds, dy_rows=dy)
 
 
 # --------------------------------------------------------------------------

@@ -515,3 +515,86 @@ def test_group_limited_dropless_layer_is_dense_masked():
     dense = O.dense_masked_forward(c, x, Wg, None, Wgate, Wup, Wdown)
     np.testing.assert_allclose(r["out"], dense, rtol=1e-12, atol=1e-13)
     assert all(len(set(row)) == 1 for row in (r["ids"] // 2).tolist())
+
+
+# ------------------------------------------------------------- backward ----
+# [TKR] "門控網路的梯度流" (selection fixed; selected gate scores carry the gradient, unselected
+# experts none) and [TINY] section 9 (task loss + weight x aux loss).  The backward is pinned
+# against central finite differences of the (separately pinned) forward oracle.
+
+def _loss(c, x, Wg, b, Wgate, Wup, Wdown, dout, aux_grad):
+    r = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown)
+    return float(np.sum(dout * r["out"])) + aux_grad * r["stats"]["aux"], r["ids"]
+
+
+@pytest.mark.parametrize("kw", [
+    dict(score="softmax", gate="renorm", act="swiglu"),
+    dict(score="softmax", gate="raw", act="relu", k=1, overflow="drop", capacity_factor=1.0),
+    dict(score="sigmoid", gate="renorm", act="gelu", k=3),
+    dict(score="sigmoid", gate="raw", act="swiglu", k=2),
+])
+def test_backward_matches_finite_differences(kw):
+    c = cfg(T=9, D=6, E=5, F=4, aux_alpha=0.05)
+    c.update(kw)
+    rng = np.random.default_rng(41)
+    x, Wg, b, Wgate, Wup, Wdown = rand_layer(rng, c, with_bias=(c["score"] == "sigmoid"))
+    if c["act"] != "swiglu":
+        Wgate = None
+    dout = rng.standard_normal((c["T"], c["D"]))
+    aux_grad = 0.7
+    gr = O.layer_backward(c, x, Wg, b, Wgate, Wup, Wdown, dout, aux_grad)
+    if c["overflow"] == "drop":
+        assert (np.asarray(gr["forward"]["inv"]) < 0).any()      # some assignments dropped
+    params = {"x": x, "Wg": Wg, "Wgate": Wgate, "Wup": Wup, "Wdown": Wdown}
+    grads = {"x": gr["dx"], "Wg": gr["dWg"], "Wgate": gr["dW_gate"], "Wup": gr["dW_up"],
+             "Wdown": gr["dW_down"]}
+    eps = 1e-6
+    for name, val in params.items():
+        if val is None:
+            continue
+        for _ in range(3):
+            v = rng.standard_normal(val.shape)
+            plus, minus = dict(params), dict(params)
+            plus[name], minus[name] = val + eps * v, val - eps * v
+            lp, ids_p = _loss(c, plus["x"], plus["Wg"], b, plus["Wgate"], plus["Wup"],
+                              plus["Wdown"], dout, aux_grad)
+            lm, ids_m = _loss(c, minus["x"], minus["Wg"], b, minus["Wgate"], minus["Wup"],
+                              minus["Wdown"], dout, aux_grad)
+            assert np.array_equal(ids_p, ids_m)                   # the selection did not move
+            fd = (lp - lm) / (2 * eps)
+            an = float(np.sum(grads[name] * v))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
+
+
+def test_backward_gate_path_reaches_selected_logits_only():
+    # softmax + renorm: the gate gradient is a softmax Jacobian over the selected logits --
+    # zero on unselected experts ([TKR]) and summing to zero over the selected ones
+    rng = np.random.default_rng(42)
+    s = rng.standard_normal((20, 8))
+    ids, _, _ = O.route_token_choice(s, 3)
+    dg = rng.standard_normal((20, 3))
+    ds = O.gate_logit_grad(s, ids, dg, "softmax", "renorm")
+    mask = np.zeros_like(ds, dtype=bool)
+    np.put_along_axis(mask, ids, True, axis=1)
+    assert np.all(ds[~mask] == 0.0)
+    np.testing.assert_allclose(ds.sum(axis=1), 0.0, atol=1e-14)
+
+
+def test_backward_single_expert_is_the_dense_ffn_backward():
+    # E = 1, k = 1: the gate is 1 and the layer is the dense FFN; with aux_grad = 0 the layer
+    # gradients are the FFN's: dW_down = dout^T h, dx = (dh . u . SiLU'(a)) W_gate + ... .
+    c = cfg(T=7, D=5, E=1, F=3, k=1)
+    rng = np.random.default_rng(43)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    dout = rng.standard_normal((7, 5))
+    gr = O.layer_backward(c, x, Wg, None, Wgate, Wup, Wdown, dout, aux_grad=0.0)
+    a, u = x @ Wgate[0].T, x @ Wup[0].T
+    h = O.silu(a) * u
+    dh = dout @ Wdown[0]
+    sg = 1 / (1 + np.exp(-a))
+    da = dh * u * (sg * (1 + a * (1 - sg)))
+    np.testing.assert_allclose(gr["dW_down"][0], dout.T @ h, rtol=1e-12)
+    np.testing.assert_allclose(gr["dW_gate"][0], da.T @ x, rtol=1e-12)
+    np.testing.assert_allclose(gr["dx"], da @ Wgate[0] + (dh * O.silu(a)) @ Wup[0], rtol=1e-12,
+                               atol=1e-13)
+    assert np.all(gr["dWg"] == 0.0)
