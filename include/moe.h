@@ -246,6 +246,25 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
                                const void* Ws_down, void* out, void* ws, size_t ws_bytes,
                                moe_stream_t stream);
 
+/* Backward of moe_layer_forward with the selection held fixed ("Top-k 路由" section
+ * "門控網路的梯度流": the selected experts' gate scores carry the gradient, unselected experts
+ * none; Tiny MoE section 9: task loss + weight x aux loss, fixed expert indices).
+ * Loss L = <dout, out> + aux_grad * aux; the routing, permutation, logits, gates, x_perm, h, y
+ * and f of the forward call are read from its workspace `fwd_ws` (same desc and inputs).
+ *   Outputs: dx [T, D] (bf16); dWg [E, D], dW_gate and dW_up [E, F, D] (dW_gate NULL unless
+ *   SwiGLU), dW_down [E, D, F], all fp32, overwritten.  The selection-only bias gets no
+ *   gradient.  Merge weights: softmax over the selected logits (RENORM) or the softmax value
+ *   (RAW); sigmoid affinities likewise; the balance loss reaches the logits through P.
+ *   bwd_ws: moe_backward_workspace_size bytes, 256-byte aligned.
+ * Limits: bf16, token choice, no shared experts (MOE_ERR_UNSUPPORTED otherwise). */
+moe_status_t moe_backward_workspace_size(const moe_desc_t* desc, size_t* bytes);
+moe_status_t moe_layer_backward(const moe_desc_t* desc, const void* x, const void* Wg,
+                                const void* W_gate, const void* W_up, const void* W_down,
+                                const void* dout, float aux_grad, void* fwd_ws,
+                                size_t fwd_ws_bytes, void* dx, float* dWg, float* dW_gate,
+                                float* dW_up, float* dW_down, void* bwd_ws,
+                                size_t bwd_ws_bytes, moe_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that kernels set when
  * a bounded wait gives up (MOE_ERR_TIMEOUT) or a device-side check fires (MOE_ERR_DEVICE).
  * *code receives the raw word (0 = none).  Returns MOE_OK when the word was 0. */

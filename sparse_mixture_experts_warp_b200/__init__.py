@@ -98,6 +98,9 @@ _SIGS = {
     "moe_balance_stats": ([_DP, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_layer_forward": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
                           ctypes.c_int),
+    "moe_backward_workspace_size": ([_DP, ctypes.POINTER(_SZ)], ctypes.c_int),
+    "moe_layer_backward": ([_DP, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _SZ, _P, _P, _P,
+                            _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
     "moe_debug_inject": ([_I32], ctypes.c_int),
     "moe_kernel_launches": ([], ctypes.c_int64),
@@ -320,6 +323,25 @@ def moe_layer_forward(d, x, Wg, sel_bias, W_gate, W_up, W_down, Ws_gate, Ws_up, 
         ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(sel_bias), _ptr(W_gate), _ptr(W_up),
         _ptr(W_down), _ptr(Ws_gate), _ptr(Ws_up), _ptr(Ws_down), _ptr(out), _ptr(ws),
         ws.numel(), _stream(stream)))
+
+
+def backward_workspace_size(d: MoeDesc) -> int:
+    n = _SZ()
+    _check("moe_backward_workspace_size",
+           lib().moe_backward_workspace_size(ctypes.byref(d), ctypes.byref(n)))
+    return n.value
+
+
+def empty_backward_workspace(d: MoeDesc, device="cuda"):
+    return torch.empty(backward_workspace_size(d), dtype=torch.uint8, device=device)
+
+
+def moe_layer_backward(d, x, Wg, W_gate, W_up, W_down, dout, aux_grad, fwd_ws, dx, dWg, dW_gate,
+                       dW_up, dW_down, bwd_ws, stream=None):
+    _check("moe_layer_backward", lib().moe_layer_backward(
+        ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(dout),
+        float(aux_grad), _ptr(fwd_ws), fwd_ws.numel(), _ptr(dx), _ptr(dWg), _ptr(dW_gate),
+        _ptr(dW_up), _ptr(dW_down), _ptr(bwd_ws), bwd_ws.numel(), _stream(stream)))
 
 
 def get_device_error(stream=None) -> int:

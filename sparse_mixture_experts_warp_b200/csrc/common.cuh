@@ -66,7 +66,8 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
                                          cudaStream_t s);
 
 // gemm_sm100.cu (bf16 grouped GEMM on tcgen05)
-enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI_GELU = 4 };
+enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI_GELU = 4,
+                    EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */ };
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s);
@@ -76,6 +77,35 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
 int router_gemm_splits(int T, int D);
 cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg, int E,
                                     float* partials, int ksplit, cudaStream_t s);
+
+// out[g] = A[:, K_g] B[:, K_g]^T (fp32 [M, N] per group) for groups along K: group g owns the
+// k columns [kgroup[g], kgroup[g+1]) of A [M, k_total] and B [N, k_total] (bf16, K-major,
+// kgroup a device array of multiples of 64).
+cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B, int N, int G,
+                                            const int32_t* kgroup, int64_t k_total, float* out,
+                                            cudaStream_t s);
+// backward.cu (layer backward with the selection fixed: memory-bound pieces)
+int backward_dwg_chunks(int T);
+cudaError_t launch_pad_offsets(const int32_t* offsets, int E, int32_t* pad_off, cudaStream_t s);
+cudaError_t launch_gather_dy(const void* dout, const void* y, const int32_t* row_src,
+                             const float* gates, const int32_t* offsets, int E, int K, int D,
+                             int64_t rows_max, void* dY, float* dgates, cudaStream_t s);
+cudaError_t launch_act_backward(int act, const void* dH, const void* gu, int64_t ldg,
+                                const int32_t* offsets, int E, int F, int64_t rows_max,
+                                void* dAB, cudaStream_t s);
+cudaError_t launch_transpose(const void* src, int64_t src_bstride, int R, int C, int64_t lds,
+                             void* dst, int64_t dst_bstride, int64_t ldd, int dcol0, int batch,
+                             cudaStream_t s);
+cudaError_t launch_transpose_pad(const void* src, int64_t lds, int C, const int32_t* offsets,
+                                 const int32_t* pad_off, int E, int64_t pad_cols, void* dst,
+                                 int64_t ldd, cudaStream_t s);
+cudaError_t launch_router_backward(const moe_desc_t& d, const float* logits, const int32_t* ids,
+                                   const float* gates, const float* dgates, const int32_t* inv,
+                                   const float* f, float aux_grad, float* ds, cudaStream_t s);
+cudaError_t launch_dx(const void* dX, const int32_t* inv, const float* ds, const void* Wg, int T,
+                      int D, int E, int K, void* dx, cudaStream_t s);
+cudaError_t launch_dwg(const float* ds, const void* x, int T, int D, int E, float* part,
+                       float* dWg, cudaStream_t s);
 
 // Test hook of the grouped GEMM's bounded waits (see moe_debug_inject).
 void set_gemm_fault(int kind);

@@ -79,7 +79,49 @@ struct GemmParams {
   int ksplit;               // k-range splits (EPI_F32 only; 1 otherwise)
   int kchunk;               // k-blocks per split
   int64_t split_stride;     // EPI_F32: elements between the partial outputs of two splits
+  // groups along K (weight gradients): group g owns k columns [kgroup[g], kgroup[g+1]) of both
+  // operands (device array, multiples of the k-block) and writes out + g * out_gstride
+  // ([rows, N], fp32 with EPI_F32); nullptr: groups along M (rows of A) as usual
+  const int32_t* kgroup;
+  int64_t out_gstride;
 };
+
+// One work item of the persistent schedule.
+struct Tile {
+  int g, m, n_idx, m_idx, kb0, kb1, split;
+  int64_t row0;   // first A row (and output row) of the group
+  int kcol0;      // first k column of the group (groups along K)
+};
+
+// Work item t (k-split slowest, then group, n-tile, m-tile); g caches the group search.
+template <int TBM, int KB>
+__device__ __forceinline__ Tile locate(int t, int total, int nkb, const GemmParams& p,
+                                       const int* grp_off, const int* tile_pre, int& g) {
+  Tile r;
+  r.split = t / total;
+  const int tile = t - r.split * total;
+  if (tile < tile_pre[g]) g = 0;
+  while (tile >= tile_pre[g + 1]) ++g;
+  r.g = g;
+  if (p.kgroup) {
+    r.m = (int)p.rows;
+    r.row0 = 0;
+    r.kcol0 = grp_off[g];
+    r.kb0 = 0;
+    r.kb1 = (grp_off[g + 1] - grp_off[g]) / KB;
+  } else {
+    r.m = grp_off[g + 1] - grp_off[g];
+    r.row0 = grp_off[g];
+    r.kcol0 = 0;
+    r.kb0 = r.split * p.kchunk;
+    r.kb1 = min(nkb, r.kb0 + p.kchunk);
+  }
+  const int mt = (r.m + TBM - 1) / TBM;
+  const int local = tile - tile_pre[g];
+  r.n_idx = local / mt;
+  r.m_idx = local - r.n_idx * mt;
+  return r;
+}
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -357,7 +399,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB0)) : "memory");
-    if (EPI == EPI_SWIGLU)
+    if (EPI == EPI_SWIGLU || EPI == EPI_RAW)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB1)) : "memory");
   }
   if (warp == 1) {
@@ -367,7 +409,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
-  if (warp == 2) {
+  if (warp == 2 && p.kgroup) {
+    // groups along K: every group has the same ceil(rows / TBM) * nt tiles
+    const int per = (int)((p.rows + TBM - 1) / TBM) * p.nt;
+    for (int g = lane; g <= p.G; g += 32) {
+      grp_off[g] = p.kgroup[g];
+      tile_pre[g] = g * per;
+    }
+  } else if (warp == 2) {
     // group row starts and the tile prefix (tiles of group g = ceil(rows_g / BM) * nt)
     int carry = 0;
     if (lane == 0) {
@@ -412,18 +461,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int g = 0;
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-        const int split = t / total, tile = t - split * total;
-        if (tile < tile_pre[g]) g = 0;
-        while (tile >= tile_pre[g + 1]) ++g;
-        const int m = grp_off[g + 1] - grp_off[g];
-        const int mt = (m + TBM - 1) / TBM;
-        const int local = tile - tile_pre[g];
-        const int n_idx = local / mt, m_idx = local - n_idx * mt;
-        const int a_row = grp_off[g] + m_idx * TBM;
-        const int b_row = g * p.N + n_idx * p.n_out_tile;
-        const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
-        const int kb0 = split * p.kchunk, kb1 = min(nkb, kb0 + p.kchunk);
+        const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+        const int a_row = (int)tl.row0 + tl.m_idx * TBM;
+        const int b_row = (p.kgroup ? 0 : tl.g * p.N) + tl.n_idx * p.n_out_tile;
+        const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
+        const int kb0 = tl.kb0, kb1 = tl.kb1;
         for (int kb = kb0; kb < kb1; ++kb) {
+          const int kx = tl.kcol0 + kb * KB;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
                          TIMEOUT_NS)) {
             ok = false;
@@ -442,14 +486,14 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             continue;
           }
           const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
-          tma_load_2d(a_dst, &tmA, &full[stage], kb * KB, a_row);
-          if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kb * KB, a_row + BM);
-          if (EPI == EPI_SWIGLU) {
-            tma_load_2d(b_dst, &tmB0, &full[stage], kb * KB, b_row);
-            tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kb * KB, b_row);
+          tma_load_2d(a_dst, &tmA, &full[stage], kx, a_row);
+          if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kx, a_row + BM);
+          if (EPI == EPI_SWIGLU || EPI == EPI_RAW) {
+            tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kx, b_row);
           } else {
-            tma_load_2d(b_dst, &tmB0, &full[stage], kb * KB, b_row);
-            tma_load_2d(b_dst + TB_BYTES / 2, &tmB0, &full[stage], kb * KB, b_row + 128);
+            tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB0, &full[stage], kx, b_row + 128);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -475,14 +519,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int it = 0, g = 0;
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x, ++it) {
-        const int split = t / total, tile = t - split * total;
-        if (tile < tile_pre[g]) g = 0;
-        while (tile >= tile_pre[g + 1]) ++g;
-        const int m = grp_off[g + 1] - grp_off[g];
-        const int mt = (m + TBM - 1) / TBM;
-        const int m_idx = (tile - tile_pre[g]) % mt;
+        const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+        const int m = tl.m, m_idx = tl.m_idx;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
-        const int kb0 = split * p.kchunk, kb1 = min(nkb, kb0 + p.kchunk);
+        const int kb0 = tl.kb0, kb1 = tl.kb1;      // kb0 == kb1: an empty group along K
         // M = 64 for a half with at most 64 live rows
         const int live0 = min(BM, m - m_idx * TBM), live1 = min(BM, m - m_idx * TBM - BM);
         const uint32_t idesc0 = live0 <= 64 ? kIdesc64 : kIdesc;
@@ -532,13 +572,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
     int g = 0, it = 0;
     for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
-      const int split = t / total, tile = t - split * total;
-      if (tile < tile_pre[g]) g = 0;
-      while (tile >= tile_pre[g + 1]) ++g;
-      const int m = grp_off[g + 1] - grp_off[g];
-      const int mt = (m + TBM - 1) / TBM;
-      const int local = tile - tile_pre[g];
-      const int n_idx = local / mt, m_idx = local - n_idx * mt;
+      const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+      const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
+      const bool zero = tl.kb1 <= tl.kb0;    // no k-blocks (empty group along K): the sum is 0
       const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
       const int acc = it % NBUF;
       const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
@@ -559,7 +595,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const bool m64 = live <= 64;
       const int row = half * BM + (m64 ? 16 * q + lane : 32 * q + lane);
       const int r = m_idx * TBM + row;
-      const int64_t orow = (int64_t)grp_off[g] + r;
+      const int64_t orow = tl.row0 + r;
       bool valid = r < m && (!m64 || lane < 16);
       if (valid && (orow < 0 || orow >= p.rows)) {
         atomicCAS(p.err, 0, DEVERR_BOUNDS);
@@ -586,15 +622,43 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (valid && col < p.N) store_swiglu32(g0, u0, orow_ptr + c);   // SiLU(g) * u
           if (valid && col + 32 < p.N) store_swiglu32(g1, u1, orow_ptr + c + 32);
         }
+      } else if (EPI == EPI_RAW) {
+        // the raw gate | up accumulators of the tile as bf16: row pitch ldo, tile n at 256 n
+        __nv_bfloat16* o = p.out + orow * p.ldo + (int64_t)n_idx * 2 * p.n_out_tile;
+#pragma unroll 1
+        for (int c = 0; c < MMA_N; c += 128) {
+          uint32_t v0[32], v1[32], v2[32], v3[32];
+          tmem_ld32(taddr + c, v0);
+          tmem_ld32(taddr + c + 32, v1);
+          tmem_ld32(taddr + c + 64, v2);
+          tmem_ld32(taddr + c + 96, v3);
+          tmem_wait_ld();
+          if (c == MMA_N - 128) {            // last TMEM read of the tile: release the buffer
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          const int f = n_idx * p.n_out_tile + (c & 127);   // feature of the chunk's first column
+          if (valid && f < p.N) store_act32<EPI_NONE>(v0, o + c);
+          if (valid && f + 32 < p.N) store_act32<EPI_NONE>(v1, o + c + 32);
+          if (valid && f + 64 < p.N) store_act32<EPI_NONE>(v2, o + c + 64);
+          if (valid && f + 96 < p.N) store_act32<EPI_NONE>(v3, o + c + 96);
+        }
       } else if (EPI == EPI_F32) {
-        // fp32 partial of this k-split, rows of out32 + split * split_stride
-        float* orow32 = reinterpret_cast<float*>(p.out) + split * p.split_stride + orow * p.ldo +
+        // fp32 partial of this k-split, rows of out32 + split * split_stride (+ the group's
+        // output block when groups run along K)
+        float* orow32 = reinterpret_cast<float*>(p.out) + split * p.split_stride +
+                        (p.kgroup ? (int64_t)tl.g * p.out_gstride : 0) + orow * p.ldo +
                         (int64_t)n_idx * p.n_out_tile;
 #pragma unroll 1
         for (int c = 0; c < MMA_N; c += 32) {
           uint32_t v[32];
-          tmem_ld32(taddr + c, v);
-          tmem_wait_ld();
+          if (!zero) {
+            tmem_ld32(taddr + c, v);
+            tmem_wait_ld();
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0u;
+          }
           if (c == MMA_N - 32) {             // last TMEM read of the tile: release the buffer
             tc_fence_before();
             mbar_arrive(&tempty[acc]);
@@ -1068,6 +1132,7 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
     case EPI_RELU: return launch_epi<EPI_RELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_F32: return launch_epi<EPI_F32, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_GELU: return launch_epi<EPI_GELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    case EPI_RAW: return launch_epi<EPI_RAW, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     default: return launch_epi<EPI_NONE, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
   }
 }
@@ -1151,8 +1216,11 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.G = n_groups;
   p.N = N;
   p.K = K;
-  p.n_out_tile = (epi == EPI_SWIGLU) ? 128 : 256;
+  p.n_out_tile = (epi == EPI_SWIGLU || epi == EPI_RAW) ? 128 : 256;
   p.nt = (N + p.n_out_tile - 1) / p.n_out_tile;
+  if (epi == EPI_RAW) p.ldo = (int64_t)p.nt * 256;     // gate | up blocks of 128 per n-tile
+  p.kgroup = nullptr;
+  p.out_gstride = 0;
   p.fault = g_gemm_fault;
   p.ksplit = 1;
   p.kchunk = 1 << 30;
@@ -1162,14 +1230,14 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   const int kb = tile == TILE_256_K32 ? 32 : 64;
   if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
   if (!make_map(&tb0, B0, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
-  if (epi == EPI_SWIGLU) {
+  if (epi == EPI_SWIGLU || epi == EPI_RAW) {
     if (!make_map(&tb1, B1, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
   } else {
     tb1 = tb0;
   }
   const int tbm = tile == TILE_PAIR ? 2 * BM : BM * halves;
   const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
-  if (tile == TILE_PAIR && offsets) {
+  if (tile == TILE_PAIR && offsets && epi != EPI_RAW) {
     // 256 x 512 accumulator tiles: 256 SwiGLU features (gate + up) or 512 output columns;
     // the SwiGLU weights go in 64-row boxes
     if (epi == EPI_SWIGLU && (!make_map(&tb0, B0, brows, (uint64_t)K, 64, kb) ||
@@ -1195,6 +1263,35 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
 }
 
 void set_gemm_fault(int kind) { g_gemm_fault = kind; }
+
+cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B, int N, int G,
+                                            const int32_t* kgroup, int64_t k_total, float* out,
+                                            cudaStream_t s) {
+  if (M <= 0 || N <= 0 || G <= 0) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb;
+  if (!make_map(&ta, A, (uint64_t)M, (uint64_t)k_total, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, B, (uint64_t)N, (uint64_t)k_total, 128, 64)) return cudaErrorInvalidValue;
+  GemmParams p;
+  p.offsets = nullptr;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  p.rows = M;
+  p.ldo = N;
+  p.G = G;
+  p.N = N;
+  p.K = (int)k_total;
+  p.n_out_tile = 256;
+  p.nt = (N + 255) / 256;
+  p.fault = 0;
+  p.ksplit = 1;
+  p.kchunk = 1 << 30;
+  p.split_stride = 0;
+  p.kgroup = kgroup;
+  p.out_gstride = (int64_t)M * N;
+  const int64_t tiles = (int64_t)G * ((M + 2 * BM - 1) / (2 * BM)) * p.nt;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch_epi<EPI_F32, 2, 64, 3>(ta, tb, tb, p, grid, gemm_smem(2, 64, 3, G), s);
+}
 
 // k-splits of the router product: enough (m-tile, split) pairs to cover the SMs, at most
 // kRouterMaxSplits, and every split non-empty (ks = ceil(nkb / ceil(nkb / ks))).
@@ -1231,6 +1328,8 @@ cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg,
   p.ksplit = ksplit;
   p.kchunk = (nkb + ksplit - 1) / ksplit;
   p.split_stride = (int64_t)T * E;
+  p.kgroup = nullptr;
+  p.out_gstride = 0;
   const int64_t tiles = (int64_t)((T + BM - 1) / BM) * ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, 1), s);

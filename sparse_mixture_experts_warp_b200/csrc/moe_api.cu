@@ -411,6 +411,156 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.entropy, v.f, v.stats, stream);
 }
 
+// ---------------- backward ----------------
+
+namespace {
+
+struct BwdViews {
+  int32_t* pad_off;
+  void *dY, *gu, *dH, *dAB, *dXp, *WdT, *WguT, *dYT, *hT, *xpT, *dABT;
+  float *dgates, *ds, *dwg_part;
+  int64_t ldg, nab, pad_cols;
+};
+
+moe_status_t check_backward(const moe_desc_t* d) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (d->dtype != MOE_BF16 || d->select != MOE_TOKEN_CHOICE || d->n_shared > 0)
+    return MOE_ERR_UNSUPPORTED;
+  if (d->E > 256) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+// Backward workspace layout; with base == nullptr only the size is computed.
+size_t carve_bwd(const moe_desc_t* d, uint8_t* base, BwdViews* v) {
+  const int64_t T = d->T, D = d->D, E = d->E, F = d->F, A = rows_of(d);
+  const bool glu = d->act == MOE_ACT_SWIGLU;
+  v->ldg = glu ? (F + 127) / 128 * 256 : F;
+  v->nab = glu ? 2 * F : F;
+  v->pad_cols = (A + 64 * E + 63) / 64 * 64;
+  size_t off = 0;
+  auto take = [&](size_t bytes) -> void* {
+    void* p = base ? base + off : nullptr;
+    off += up(bytes);
+    return p;
+  };
+  v->pad_off = static_cast<int32_t*>(take((E + 1) * 4));
+  v->dY = take(A * D * 2);
+  v->dgates = static_cast<float*>(take(T * d->k * 4));
+  v->gu = take(A * v->ldg * 2);
+  v->dH = take(A * F * 2);
+  v->dAB = take(A * v->nab * 2);
+  v->dXp = take(A * D * 2);
+  v->ds = static_cast<float*>(take(T * E * 4));
+  v->WdT = take(E * F * D * 2);
+  v->WguT = take(E * D * v->nab * 2);
+  v->dYT = take(D * v->pad_cols * 2);
+  v->hT = take(F * v->pad_cols * 2);
+  v->xpT = take(D * v->pad_cols * 2);
+  v->dABT = take(v->nab * v->pad_cols * 2);
+  v->dwg_part = static_cast<float*>(take((size_t)backward_dwg_chunks(d->T) * E * D * 4));
+  return off;
+}
+
+}  // namespace
+
+moe_status_t moe_backward_workspace_size(const moe_desc_t* d, size_t* bytes) {
+  moe_status_t st = check_backward(d);
+  if (st != MOE_OK) return st;
+  if (!bytes) return MOE_ERR_INVALID_ARG;
+  BwdViews v;
+  *bytes = carve_bwd(d, nullptr, &v);
+  return MOE_OK;
+}
+
+moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* Wg,
+                                const void* W_gate, const void* W_up, const void* W_down,
+                                const void* dout, float aux_grad, void* fwd_ws,
+                                size_t fwd_ws_bytes, void* dx, float* dWg, float* dW_gate,
+                                float* dW_up, float* dW_down, void* bwd_ws,
+                                size_t bwd_ws_bytes, moe_stream_t stream) {
+  moe_status_t st = check_backward(d);
+  if (st != MOE_OK) return st;
+  moe_layer_views_t v;
+  st = moe_layer_views(d, fwd_ws, fwd_ws_bytes, &v);
+  if (st != MOE_OK) return st;
+  const bool glu = d->act == MOE_ACT_SWIGLU;
+  if (!x || !Wg || !W_up || !W_down || !dout || !dx || !dWg || !dW_up || !dW_down || !bwd_ws)
+    return MOE_ERR_INVALID_ARG;
+  if (glu && (!W_gate || !dW_gate)) return MOE_ERR_INVALID_ARG;
+  for (const void* p : {x, Wg, W_up, W_down, dout, (const void*)dx, (const void*)dWg,
+                        (const void*)dW_up, (const void*)dW_down})
+    if (!is_aligned16(p)) return MOE_ERR_INVALID_ARG;
+  if (glu && (!is_aligned16(W_gate) || !is_aligned16(dW_gate))) return MOE_ERR_INVALID_ARG;
+  if (!(aux_grad == aux_grad)) return MOE_ERR_INVALID_ARG;      // NaN
+  BwdViews b;
+  if (bwd_ws_bytes < carve_bwd(d, nullptr, &b)) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
+  carve_bwd(d, static_cast<uint8_t*>(bwd_ws), &b);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int T = d->T, D = d->D, E = d->E, F = d->F, K = d->k;
+  const int64_t A = v.rows;
+  const int nab = (int)b.nab;
+  if (T == 0) {
+    // no tokens: every gradient is zero
+    cudaError_t e = cudaMemsetAsync(dWg, 0, (size_t)E * D * 4, s);
+    if (e == cudaSuccess && glu) e = cudaMemsetAsync(dW_gate, 0, (size_t)E * F * D * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dW_up, 0, (size_t)E * F * D * 4, s);
+    if (e == cudaSuccess) e = cudaMemsetAsync(dW_down, 0, (size_t)E * D * F * 4, s);
+    return cuda_status(e);
+  }
+  cudaError_t e = launch_pad_offsets(v.offsets, E, b.pad_off, s);
+  // dY = g dout on the executed rows, dg = <dout, y>
+  if (e == cudaSuccess)
+    e = launch_gather_dy(dout, v.y, v.row_src, v.gates, v.offsets, E, K, D, A, b.dY, b.dgates, s);
+  // pre-activations recomputed: SwiGLU gate | up blocks, or z = x W_up^T
+  if (e == cudaSuccess)
+    e = glu ? launch_grouped_gemm_bf16(EPI_RAW, v.x_perm, A, D, W_gate, W_up, E, F, v.offsets,
+                                       b.gu, s)
+            : launch_grouped_gemm_bf16(EPI_NONE, v.x_perm, A, D, W_up, nullptr, E, F, v.offsets,
+                                       b.gu, s);
+  // dH = dY W_down: B = W_down^T per expert ([F, D], K-major)
+  if (e == cudaSuccess)
+    e = launch_transpose(W_down, (int64_t)D * F, D, F, F, b.WdT, (int64_t)F * D, D, 0, E, s);
+  if (e == cudaSuccess)
+    e = launch_grouped_gemm_bf16(EPI_NONE, b.dY, A, D, b.WdT, nullptr, E, F, v.offsets, b.dH, s);
+  // activation backward -> [da | db] (SwiGLU) or dz
+  if (e == cudaSuccess)
+    e = launch_act_backward(d->act, b.dH, b.gu, b.ldg, v.offsets, E, F, A, b.dAB, s);
+  // dX = [da | db] [W_gate ; W_up]: B = [W_gate^T | W_up^T] per expert ([D, 2F])
+  if (e == cudaSuccess && glu)
+    e = launch_transpose(W_gate, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab, 0, E, s);
+  if (e == cudaSuccess)
+    e = launch_transpose(W_up, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab,
+                         glu ? F : 0, E, s);
+  if (e == cudaSuccess)
+    e = launch_grouped_gemm_bf16(EPI_NONE, b.dAB, A, nab, b.WguT, nullptr, E, D, v.offsets,
+                                 b.dXp, s);
+  // router: ds, then dx = sum_j dX[inv] + ds W_g and dW_g = ds^T x
+  if (e == cudaSuccess)
+    e = launch_router_backward(*d, v.logits, v.expert_ids, v.gates, b.dgates, v.inv, v.f,
+                               aux_grad, b.ds, s);
+  if (e == cudaSuccess) e = launch_dx(b.dXp, v.inv, b.ds, Wg, T, D, E, K, dx, s);
+  if (e == cudaSuccess) e = launch_dwg(b.ds, x, T, D, E, b.dwg_part, dWg, s);
+  // weight gradients: groups along K over the experts' row blocks, transposed and padded
+  const int64_t pc = b.pad_cols;
+  if (e == cudaSuccess) e = launch_transpose_pad(b.dY, D, D, v.offsets, b.pad_off, E, pc, b.dYT, pc, s);
+  if (e == cudaSuccess) e = launch_transpose_pad(v.h, F, F, v.offsets, b.pad_off, E, pc, b.hT, pc, s);
+  if (e == cudaSuccess)
+    e = launch_grouped_gemm_kgroups_f32(b.dYT, D, b.hT, F, E, b.pad_off, pc, dW_down, s);
+  if (e == cudaSuccess)
+    e = launch_transpose_pad(v.x_perm, D, D, v.offsets, b.pad_off, E, pc, b.xpT, pc, s);
+  if (e == cudaSuccess)
+    e = launch_transpose_pad(b.dAB, nab, nab, v.offsets, b.pad_off, E, pc, b.dABT, pc, s);
+  if (e == cudaSuccess && glu)
+    e = launch_grouped_gemm_kgroups_f32(b.dABT, F, b.xpT, D, E, b.pad_off, pc, dW_gate, s);
+  if (e == cudaSuccess)
+    e = launch_grouped_gemm_kgroups_f32(static_cast<const __nv_bfloat16*>(b.dABT) +
+                                            (glu ? (int64_t)F * pc : 0),
+                                        F, b.xpT, D, E, b.pad_off, pc, dW_up, s);
+  return cuda_status(e);
+}
+
 int64_t moe_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 moe_status_t moe_debug_inject(int32_t fault) {
