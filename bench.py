@@ -281,6 +281,48 @@ def e2e_pipelined(M, d, inp, ws, stream, dev, steps, warmup, world):
     return pipelined_ms, s0.elapsed_time(s1)
 
 
+def time_backward(M, w, d, inp, ws, stream, dev, steps, warmup, tc_peak, world):
+    """moe_layer_backward (selection fixed) on the forward workspace of the same inputs: the
+    device time per call, its GEMM FLOPs (pre-activation recompute 1x the up projection, dgrad
+    and wgrad 2x the up and down projections) and their rate against the tensor peak."""
+    bws = M.empty_backward_workspace(d, dev)
+    g = torch.Generator(device=dev)
+    g.manual_seed(7)
+    dout = torch.randn(w.T, w.D, generator=g, device=dev).to(torch.bfloat16)
+    dx = torch.empty_like(inp.x)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dWg = torch.empty(w.E, w.D, **f32)
+    dWgate = torch.empty(w.E, w.F, w.D, **f32) if w.act == "swiglu" else None
+    dWup = torch.empty(w.E, w.F, w.D, **f32)
+    dWdown = torch.empty(w.E, w.D, w.F, **f32)
+
+    def call():
+        M.moe_layer_backward(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, dout, 1.0, ws,
+                             dx, dWg, dWgate, dWup, dWdown, bws, stream)
+
+    for _ in range(warmup):
+        call()
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(steps):
+        call()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    rows = int(M.layer_views(d, ws)["offsets"][-1].item())
+    n_up = 2 if w.act == "swiglu" else 1
+    up, down = 2.0 * rows * w.D * w.F * n_up, 2.0 * rows * w.F * w.D
+    flops = 3 * up + 2 * down
+    tf = flops / (ms * 1e-3) / 1e12
+    return {"ms_per_step": round(ms, 4), "tokens_per_s": round(w.T * world / (ms * 1e-3), 1),
+            "gemm_tflop_per_step": round(flops / 1e12, 3), "tflops": round(tf, 1),
+            "frac_of_tensor_peak": round(tf / tc_peak, 3), "steps": steps,
+            "what": "moe_layer_backward: dx, dW_g, dW_gate/up/down (fp32) with the selection "
+                    "of the forward call fixed; dout ~ N(0,1) bf16"}
+
+
 def run_cuda(args, rank, world, local):
     import sparse_mixture_experts_warp_b200 as M
 
@@ -446,6 +488,10 @@ def run_cuda(args, rank, world, local):
     }
     if remeasured:
         res["clocks"]["remeasured"] = True
+    if (not args.no_backward and w.dtype == "bf16" and w.select == "token"
+            and not w.n_shared):
+        res["backward"] = time_backward(M, w, d, inp, ws, stream, dev, min(args.steps, 20),
+                                        max(args.warmup, 3), tc_peak, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         res["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
     if rank == 0:
@@ -567,6 +613,8 @@ def main():
                     help="override the batch size T (smaller cases for profiling)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-backward", action="store_true",
+                    help="skip the backward-pass timing that follows the forward measurement")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     args = ap.parse_args()

@@ -138,55 +138,63 @@ __global__ void act_backward_kernel(const uint4* __restrict__ dH, const __nv_bfl
   }
 }
 
-// Batched bf16 transpose through shared memory: dst[b][c][dcol0 + r] = src[b][r][c]
-// (src rows of pitch lds, dst rows of pitch ldd).  32 x 32 tiles, 32 x 8 threads.
-__global__ void transpose_kernel(const __nv_bfloat16* __restrict__ src, int64_t src_bstride,
-                                 int R, int C, int64_t lds, __nv_bfloat16* __restrict__ dst,
-                                 int64_t dst_bstride, int64_t ldd, int dcol0) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int b = blockIdx.z;
-  const int r0 = blockIdx.y * 32, c0 = blockIdx.x * 32;
-  const __nv_bfloat16* s = src + b * src_bstride;
-  __nv_bfloat16* d = dst + b * dst_bstride;
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int r = r0 + i, c = c0 + threadIdx.x;
-    if (r < R && c < C) tile[i][threadIdx.x] = s[(int64_t)r * lds + c];
+// 64 x 64 bf16 tile transpose, 256 threads: 16-byte global loads along the source rows and
+// 16-byte global stores along the destination rows, scalar accesses to a shared tile of pitch
+// 65 elements (spreads a column read over the banks).
+//   plain (PAD = false): dst[b][c][dcol0 + r] = src[b][r][c], r < R, c < C;
+//   padded (PAD = true): dst[c][j] for the 64-column block j0.. inside expert e's padded block:
+//     src row offsets[e] + (j - pad_off[e]) when that is below offsets[e + 1], else 0.
+template <bool PAD>
+__global__ void __launch_bounds__(256)
+transpose64_kernel(const __nv_bfloat16* __restrict__ src, int64_t src_bstride, int R, int C,
+                   int64_t lds, __nv_bfloat16* __restrict__ dst, int64_t dst_bstride,
+                   int64_t ldd, int dcol0, const int32_t* __restrict__ offsets,
+                   const int32_t* __restrict__ pad_off, int E) {
+  __shared__ __nv_bfloat16 tile[64][65];
+  const int c0 = blockIdx.y * 64;
+  int r0 = blockIdx.x * 64, j0 = r0, rlim = R;
+  const __nv_bfloat16* s = src + (int64_t)blockIdx.z * src_bstride;
+  __nv_bfloat16* d = dst + (int64_t)blockIdx.z * dst_bstride;
+  if (PAD) {
+    if (j0 >= pad_off[E]) return;
+    int lo = 0, hi = E;                      // expert e with pad_off[e] <= j0 < pad_off[e + 1]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pad_off[mid] <= j0) lo = mid; else hi = mid;
+    }
+    r0 = offsets[lo] + (j0 - pad_off[lo]);   // first source row of the tile
+    rlim = offsets[lo + 1];                  // rows from rlim on are padding
+  }
+  const int tid = threadIdx.x;
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int idx = tid + 256 * k;
+    const int row = idx >> 3, cv = (idx & 7) * 8;
+    uint4 u = make_uint4(0u, 0u, 0u, 0u);
+    if (r0 + row < rlim && c0 + cv < C)
+      u = *reinterpret_cast<const uint4*>(s + (int64_t)(r0 + row) * lds + c0 + cv);
+    const __nv_bfloat16* h = reinterpret_cast<const __nv_bfloat16*>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) tile[row][cv + i] = h[i];
   }
   __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int c = c0 + i, r = r0 + threadIdx.x;
-    if (r < R && c < C) d[(int64_t)c * ldd + dcol0 + r] = tile[threadIdx.x][i];
-  }
-}
-
-// Per-expert row blocks transposed and zero-padded: dst[c][pad_off[e] + i] = src[off[e] + i][c]
-// for i < count_e, 0 for count_e <= i < padded count (src rows of pitch lds, C columns;
-// dst [C, ldd]).  A 32-column tile of dst lies inside one expert (pad_off are multiples of 64).
-__global__ void transpose_pad_kernel(const __nv_bfloat16* __restrict__ src, int64_t lds, int C,
-                                     const int32_t* __restrict__ offsets,
-                                     const int32_t* __restrict__ pad_off, int E,
-                                     __nv_bfloat16* __restrict__ dst, int64_t ldd) {
-  __shared__ __nv_bfloat16 tile[32][33];
-  const int j0 = blockIdx.x * 32, c0 = blockIdx.y * 32;
-  if (j0 >= pad_off[E]) return;
-  int lo = 0, hi = E;                        // expert e with pad_off[e] <= j0 < pad_off[e + 1]
-  while (hi - lo > 1) {
-    const int mid = (lo + hi) >> 1;
-    if (pad_off[mid] <= j0) lo = mid; else hi = mid;
-  }
-  const int e = lo;
-  const int base = offsets[e], cnt = offsets[e + 1] - offsets[e];
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int k = j0 + i - pad_off[e];       // row of the expert
-    const int c = c0 + threadIdx.x;
-    __nv_bfloat16 v = __float2bfloat16(0.f);
-    if (k < cnt && c < C) v = src[(int64_t)(base + k) * lds + c];
-    tile[i][threadIdx.x] = v;
-  }
-  __syncthreads();
-  for (int i = threadIdx.y; i < 32; i += 8) {
-    const int c = c0 + i;
-    if (c < C) dst[(int64_t)c * ldd + j0 + threadIdx.x] = tile[threadIdx.x][i];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int idx = tid + 256 * k;
+    const int col = idx >> 3, rv = (idx & 7) * 8;
+    if (c0 + col >= C) continue;
+    if (!PAD && r0 + rv >= R) continue;
+    uint4 u;
+    __nv_bfloat16* h = reinterpret_cast<__nv_bfloat16*>(&u);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = tile[rv + i][col];
+    if (PAD) {
+      *reinterpret_cast<uint4*>(d + (int64_t)(c0 + col) * ldd + j0 + rv) = u;
+    } else if (r0 + rv + 8 <= R) {
+      *reinterpret_cast<uint4*>(d + (int64_t)(c0 + col) * ldd + dcol0 + r0 + rv) = u;
+    } else {
+      for (int i = 0; r0 + rv + i < R; ++i) d[(int64_t)(c0 + col) * ldd + dcol0 + r0 + rv + i] = h[i];
+    }
   }
 }
 
@@ -417,10 +425,10 @@ cudaError_t launch_transpose(const void* src, int64_t src_bstride, int R, int C,
                              void* dst, int64_t dst_bstride, int64_t ldd, int dcol0, int batch,
                              cudaStream_t s) {
   if (R <= 0 || C <= 0 || batch <= 0) return cudaSuccess;
-  const dim3 grid((C + 31) / 32, (R + 31) / 32, batch);
-  transpose_kernel<<<counted(grid), dim3(32, 8), 0, s>>>(
+  const dim3 grid((R + 63) / 64, (C + 63) / 64, batch);
+  transpose64_kernel<false><<<counted(grid), 256, 0, s>>>(
       static_cast<const __nv_bfloat16*>(src), src_bstride, R, C, lds,
-      static_cast<__nv_bfloat16*>(dst), dst_bstride, ldd, dcol0);
+      static_cast<__nv_bfloat16*>(dst), dst_bstride, ldd, dcol0, nullptr, nullptr, 0);
   return cudaGetLastError();
 }
 
@@ -428,10 +436,10 @@ cudaError_t launch_transpose_pad(const void* src, int64_t lds, int C, const int3
                                  const int32_t* pad_off, int E, int64_t pad_cols, void* dst,
                                  int64_t ldd, cudaStream_t s) {
   if (C <= 0 || pad_cols <= 0) return cudaSuccess;
-  const dim3 grid((unsigned)((pad_cols + 31) / 32), (C + 31) / 32);
-  transpose_pad_kernel<<<counted(grid), dim3(32, 8), 0, s>>>(
-      static_cast<const __nv_bfloat16*>(src), lds, C, offsets, pad_off, E,
-      static_cast<__nv_bfloat16*>(dst), ldd);
+  const dim3 grid((unsigned)((pad_cols + 63) / 64), (C + 63) / 64, 1);
+  transpose64_kernel<true><<<counted(grid), 256, 0, s>>>(
+      static_cast<const __nv_bfloat16*>(src), 0, 0, C, lds, static_cast<__nv_bfloat16*>(dst), 0,
+      ldd, 0, offsets, pad_off, E);
   return cudaGetLastError();
 }
 

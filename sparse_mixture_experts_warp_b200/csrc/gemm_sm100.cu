@@ -1288,9 +1288,11 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   p.split_stride = 0;
   p.kgroup = kgroup;
   p.out_gstride = (int64_t)M * N;
-  const int64_t tiles = (int64_t)G * ((M + 2 * BM - 1) / (2 * BM)) * p.nt;
+  // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (256 KB) overlaps
+  // the next tile's main loop, which is short here (one expert's rows)
+  const int64_t tiles = (int64_t)G * ((M + BM - 1) / BM) * p.nt;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  return launch_epi<EPI_F32, 2, 64, 3>(ta, tb, tb, p, grid, gemm_smem(2, 64, 3, G), s);
+  return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, G), s);
 }
 
 // k-splits of the router product: enough (m-tile, split) pairs to cover the SMs, at most
