@@ -282,9 +282,10 @@ def e2e_pipelined(M, d, inp, ws, stream, dev, steps, warmup, world):
 
 
 def time_backward(M, w, d, inp, ws, stream, dev, steps, warmup, tc_peak, world):
-    """moe_layer_backward (selection fixed) on the forward workspace of the same inputs: the
-    device time per call, its GEMM FLOPs (pre-activation recompute 1x the up projection, dgrad
-    and wgrad 2x the up and down projections) and their rate against the tensor peak."""
+    """Training step: moe_layer_forward_train (saves the expert pre-activations) then
+    moe_layer_backward with the selection fixed.  Reports the backward's device time per call,
+    its GEMM FLOPs (dgrad and wgrad: 2x the up and down projections) and their rate against the
+    tensor peak, and the time of the whole forward + backward step."""
     bws = M.empty_backward_workspace(d, dev)
     g = torch.Generator(device=dev)
     g.manual_seed(7)
@@ -296,31 +297,47 @@ def time_backward(M, w, d, inp, ws, stream, dev, steps, warmup, tc_peak, world):
     dWup = torch.empty(w.E, w.F, w.D, **f32)
     dWdown = torch.empty(w.E, w.D, w.F, **f32)
 
-    def call():
+    out = torch.empty_like(inp.x)
+
+    def fwd():
+        M.moe_layer_forward_train(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                                  out, ws, bws, stream)
+
+    def bwd():
         M.moe_layer_backward(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, dout, 1.0, ws,
-                             dx, dWg, dWgate, dWup, dWdown, bws, stream)
+                             dx, dWg, dWgate, dWup, dWdown, bws, stream,
+                             flags=M.BWD_PREACT_SAVED)
 
     for _ in range(warmup):
-        call()
+        fwd()
+        bwd()
     barrier(world)
     torch.cuda.synchronize(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(stream)
-    for _ in range(steps):
-        call()
-    e1.record(stream)
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps + 1)]
+    ev[0].record(stream)
+    for i in range(steps):
+        fwd()
+        ev[2 * i + 1].record(stream)
+        bwd()
+        ev[2 * i + 2].record(stream)
     torch.cuda.synchronize(dev)
-    ms = max_over_ranks(e0.elapsed_time(e1), world, dev) / steps
+    f_ms = sum(ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)) / steps
+    b_ms = sum(ev[2 * i + 1].elapsed_time(ev[2 * i + 2]) for i in range(steps)) / steps
+    ms = max_over_ranks(b_ms, world, dev)
+    train_ms = max_over_ranks(f_ms + b_ms, world, dev)
     rows = int(M.layer_views(d, ws)["offsets"][-1].item())
     n_up = 2 if w.act == "swiglu" else 1
     up, down = 2.0 * rows * w.D * w.F * n_up, 2.0 * rows * w.F * w.D
-    flops = 3 * up + 2 * down
+    flops = 2 * up + 2 * down          # dgrad and wgrad of both projections
     tf = flops / (ms * 1e-3) / 1e12
     return {"ms_per_step": round(ms, 4), "tokens_per_s": round(w.T * world / (ms * 1e-3), 1),
             "gemm_tflop_per_step": round(flops / 1e12, 3), "tflops": round(tf, 1),
             "frac_of_tensor_peak": round(tf / tc_peak, 3), "steps": steps,
-            "what": "moe_layer_backward: dx, dW_g, dW_gate/up/down (fp32) with the selection "
-                    "of the forward call fixed; dout ~ N(0,1) bf16"}
+            "train_step_ms": round(train_ms, 4),
+            "train_tokens_per_s": round(w.T * world / (train_ms * 1e-3), 1),
+            "what": "moe_layer_forward_train (saves the expert pre-activations) then "
+                    "moe_layer_backward: dx, dW_g, dW_gate/up/down (fp32) with the selection "
+                    "fixed; dout ~ N(0,1) bf16; ms_per_step is the backward alone"}
 
 
 def run_cuda(args, rank, world, local):

@@ -256,14 +256,28 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
  *   gradient.  Merge weights: softmax over the selected logits (RENORM) or the softmax value
  *   (RAW); sigmoid affinities likewise; the balance loss reaches the logits through P.
  *   bwd_ws: moe_backward_workspace_size bytes, 256-byte aligned.
+ *   flags: MOE_BWD_PREACT_SAVED when moe_layer_forward_train wrote the expert
+ *   pre-activations into this bwd_ws for this forward (the backward then skips recomputing
+ *   them with a third up projection); 0 otherwise.
  * Limits: bf16, token choice, no shared experts (MOE_ERR_UNSUPPORTED otherwise). */
+enum { MOE_BWD_PREACT_SAVED = 1 };
 moe_status_t moe_backward_workspace_size(const moe_desc_t* desc, size_t* bytes);
 moe_status_t moe_layer_backward(const moe_desc_t* desc, const void* x, const void* Wg,
                                 const void* W_gate, const void* W_up, const void* W_down,
                                 const void* dout, float aux_grad, void* fwd_ws,
                                 size_t fwd_ws_bytes, void* dx, float* dWg, float* dW_gate,
                                 float* dW_up, float* dW_down, void* bwd_ws,
-                                size_t bwd_ws_bytes, moe_stream_t stream);
+                                size_t bwd_ws_bytes, int32_t flags, moe_stream_t stream);
+
+/* moe_layer_forward (same limits as moe_layer_backward) that also stores the routed expert
+ * pre-activations (SwiGLU gate and up, or the ReLU/GELU input) into bwd_ws, for a following
+ * moe_layer_backward with MOE_BWD_PREACT_SAVED.  Results and the workspace `ws` are those of
+ * moe_layer_forward. */
+moe_status_t moe_layer_forward_train(const moe_desc_t* desc, const void* x, const void* Wg,
+                                     const float* sel_bias, const void* W_gate,
+                                     const void* W_up, const void* W_down, void* out, void* ws,
+                                     size_t ws_bytes, void* bwd_ws, size_t bwd_ws_bytes,
+                                     moe_stream_t stream);
 
 /* Synchronises `stream`, then reads and clears the device error word that kernels set when
  * a bounded wait gives up (MOE_ERR_TIMEOUT) or a device-side check fires (MOE_ERR_DEVICE).

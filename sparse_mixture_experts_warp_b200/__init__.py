@@ -100,7 +100,9 @@ _SIGS = {
                           ctypes.c_int),
     "moe_backward_workspace_size": ([_DP, ctypes.POINTER(_SZ)], ctypes.c_int),
     "moe_layer_backward": ([_DP, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _SZ, _P, _P, _P,
-                            _P, _P, _P, _SZ, _P], ctypes.c_int),
+                            _P, _P, _P, _SZ, _I32, _P], ctypes.c_int),
+    "moe_layer_forward_train": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _SZ, _P],
+                                ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
     "moe_debug_inject": ([_I32], ctypes.c_int),
     "moe_kernel_launches": ([], ctypes.c_int64),
@@ -336,12 +338,23 @@ def empty_backward_workspace(d: MoeDesc, device="cuda"):
     return torch.empty(backward_workspace_size(d), dtype=torch.uint8, device=device)
 
 
+BWD_PREACT_SAVED = 1
+
+
 def moe_layer_backward(d, x, Wg, W_gate, W_up, W_down, dout, aux_grad, fwd_ws, dx, dWg, dW_gate,
-                       dW_up, dW_down, bwd_ws, stream=None):
+                       dW_up, dW_down, bwd_ws, stream=None, flags=0):
     _check("moe_layer_backward", lib().moe_layer_backward(
         ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(dout),
         float(aux_grad), _ptr(fwd_ws), fwd_ws.numel(), _ptr(dx), _ptr(dWg), _ptr(dW_gate),
-        _ptr(dW_up), _ptr(dW_down), _ptr(bwd_ws), bwd_ws.numel(), _stream(stream)))
+        _ptr(dW_up), _ptr(dW_down), _ptr(bwd_ws), bwd_ws.numel(), int(flags), _stream(stream)))
+
+
+def moe_layer_forward_train(d, x, Wg, sel_bias, W_gate, W_up, W_down, out, ws, bwd_ws,
+                            stream=None):
+    _check("moe_layer_forward_train", lib().moe_layer_forward_train(
+        ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(sel_bias), _ptr(W_gate), _ptr(W_up),
+        _ptr(W_down), _ptr(out), _ptr(ws), ws.numel(), _ptr(bwd_ws), bwd_ws.numel(),
+        _stream(stream)))
 
 
 def get_device_error(stream=None) -> int:

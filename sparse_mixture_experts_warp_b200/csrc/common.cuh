@@ -70,7 +70,8 @@ enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI
                     EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */ };
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
-                                     const int32_t* offsets, void* out, cudaStream_t s);
+                                     const int32_t* offsets, void* out, cudaStream_t s,
+                                     void* out2 = nullptr);
 
 // Router product on the same engine: one group of T rows, N = E, fp32 partial logits of
 // ksplit k-ranges in partials[ksplit][T][E] (E % 32 == 0, E <= 256).

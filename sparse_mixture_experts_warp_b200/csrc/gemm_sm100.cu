@@ -84,6 +84,10 @@ struct GemmParams {
   // ([rows, N], fp32 with EPI_F32); nullptr: groups along M (rows of A) as usual
   const int32_t* kgroup;
   int64_t out_gstride;
+  // optional second output: the raw accumulators as bf16 (SwiGLU: gate | up blocks of 128 per
+  // n-tile, row pitch ldo2 = nt * 256; others: [rows, N]), saved for the backward pass
+  __nv_bfloat16* out2;
+  int64_t ldo2;
 };
 
 // One work item of the persistent schedule.
@@ -621,6 +625,17 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const int col = n_idx * p.n_out_tile + c;
           if (valid && col < p.N) store_swiglu32(g0, u0, orow_ptr + c);   // SiLU(g) * u
           if (valid && col + 32 < p.N) store_swiglu32(g1, u1, orow_ptr + c + 32);
+          if (p.out2 && valid) {             // pre-activations for the backward pass
+            __nv_bfloat16* o2 = p.out2 + orow * p.ldo2 + (int64_t)n_idx * 256 + c;
+            if (col < p.N) {
+              store_act32<EPI_NONE>(g0, o2);
+              store_act32<EPI_NONE>(u0, o2 + 128);
+            }
+            if (col + 32 < p.N) {
+              store_act32<EPI_NONE>(g1, o2 + 32);
+              store_act32<EPI_NONE>(u1, o2 + 160);
+            }
+          }
         }
       } else if (EPI == EPI_RAW) {
         // the raw gate | up accumulators of the tile as bf16: row pitch ldo, tile n at 256 n
@@ -690,6 +705,13 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (valid && col + 32 < p.N) store_act32<EPI>(v1, orow_ptr + c + 32);
           if (valid && col + 64 < p.N) store_act32<EPI>(v2, orow_ptr + c + 64);
           if (valid && col + 96 < p.N) store_act32<EPI>(v3, orow_ptr + c + 96);
+          if (p.out2 && valid) {             // pre-activations for the backward pass
+            __nv_bfloat16* o2 = p.out2 + orow * p.ldo2 + (int64_t)n_idx * p.n_out_tile + c;
+            if (col < p.N) store_act32<EPI_NONE>(v0, o2);
+            if (col + 32 < p.N) store_act32<EPI_NONE>(v1, o2 + 32);
+            if (col + 64 < p.N) store_act32<EPI_NONE>(v2, o2 + 64);
+            if (col + 96 < p.N) store_act32<EPI_NONE>(v3, o2 + 96);
+          }
         }
       }
     }
@@ -1203,7 +1225,8 @@ cudaError_t launch_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0,
 
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
-                                     const int32_t* offsets, void* out, cudaStream_t s) {
+                                     const int32_t* offsets, void* out, cudaStream_t s,
+                                     void* out2) {
   if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
   alignas(64) CUtensorMap ta, tb0, tb1;
   const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
@@ -1221,6 +1244,8 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   if (epi == EPI_RAW) p.ldo = (int64_t)p.nt * 256;     // gate | up blocks of 128 per n-tile
   p.kgroup = nullptr;
   p.out_gstride = 0;
+  p.out2 = static_cast<__nv_bfloat16*>(out2);
+  p.ldo2 = (epi == EPI_SWIGLU) ? (int64_t)p.nt * 256 : N;
   p.fault = g_gemm_fault;
   p.ksplit = 1;
   p.kchunk = 1 << 30;
@@ -1237,7 +1262,7 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   }
   const int tbm = tile == TILE_PAIR ? 2 * BM : BM * halves;
   const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
-  if (tile == TILE_PAIR && offsets && epi != EPI_RAW) {
+  if (tile == TILE_PAIR && offsets && epi != EPI_RAW && !out2) {
     // 256 x 512 accumulator tiles: 256 SwiGLU features (gate + up) or 512 output columns;
     // the SwiGLU weights go in 64-row boxes
     if (epi == EPI_SWIGLU && (!make_map(&tb0, B0, brows, (uint64_t)K, 64, kb) ||
@@ -1288,6 +1313,8 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   p.split_stride = 0;
   p.kgroup = kgroup;
   p.out_gstride = (int64_t)M * N;
+  p.out2 = nullptr;
+  p.ldo2 = 0;
   // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (256 KB) overlaps
   // the next tile's main loop, which is short here (one expert's rows)
   const int64_t tiles = (int64_t)G * ((M + BM - 1) / BM) * p.nt;
@@ -1332,6 +1359,8 @@ cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg,
   p.split_stride = (int64_t)T * E;
   p.kgroup = nullptr;
   p.out_gstride = 0;
+  p.out2 = nullptr;
+  p.ldo2 = 0;
   const int64_t tiles = (int64_t)((T + BM - 1) / BM) * ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, 1), s);

@@ -366,11 +366,28 @@ moe_status_t moe_balance_stats(const moe_desc_t* d, const int32_t* counts, const
                                           reinterpret_cast<cudaStream_t>(stream)));
 }
 
+static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void* Wg,
+                                 const float* sel_bias, const void* W_gate, const void* W_up,
+                                 const void* W_down, const void* Ws_gate, const void* Ws_up,
+                                 const void* Ws_down, void* out, void* ws, size_t ws_bytes,
+                                 void* preact, moe_stream_t stream);
+
 moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* Wg,
                                const float* sel_bias, const void* W_gate, const void* W_up,
                                const void* W_down, const void* Ws_gate, const void* Ws_up,
                                const void* Ws_down, void* out, void* ws, size_t ws_bytes,
                                moe_stream_t stream) {
+  return forward_impl(d, x, Wg, sel_bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down, out,
+                      ws, ws_bytes, nullptr, stream);
+}
+
+// preact != nullptr (bf16 token choice, from moe_layer_forward_train): the routed up
+// projection also stores its raw accumulators there for the backward pass.
+static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void* Wg,
+                                 const float* sel_bias, const void* W_gate, const void* W_up,
+                                 const void* W_down, const void* Ws_gate, const void* Ws_up,
+                                 const void* Ws_down, void* out, void* ws, size_t ws_bytes,
+                                 void* preact, moe_stream_t stream) {
   moe_layer_views_t v;
   moe_status_t st = moe_layer_views(d, ws, ws_bytes, &v);
   if (st != MOE_OK) return st;
@@ -384,8 +401,18 @@ moe_status_t moe_layer_forward(const moe_desc_t* d, const void* x, const void* W
   st = moe_permute(d, v.expert_ids, x, v.x_perm, v.counts, v.offsets, v.row_src, v.inv,
                    v.scratch, v.scratch_bytes, stream);
   if (st != MOE_OK) return st;
-  st = moe_expert_ffn(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, W_down, v.h, v.y,
-                      stream);
+  if (preact) {
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const bool glu = d->act == MOE_ACT_SWIGLU;
+    cudaError_t e = launch_grouped_gemm_bf16(
+        glu ? EPI_SWIGLU : (d->act == MOE_ACT_GELU ? EPI_GELU : EPI_RELU), v.x_perm, v.rows,
+        d->D, glu ? W_gate : W_up, glu ? W_up : nullptr, d->E, d->F, v.offsets, v.h, s, preact);
+    if (e != cudaSuccess) return MOE_ERR_CUDA;
+    st = moe_expert_down(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, stream);
+  } else {
+    st = moe_expert_ffn(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, W_down, v.h,
+                        v.y, stream);
+  }
   if (st != MOE_OK) return st;
   if (d->n_shared > 0) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -473,12 +500,27 @@ moe_status_t moe_backward_workspace_size(const moe_desc_t* d, size_t* bytes) {
   return MOE_OK;
 }
 
+moe_status_t moe_layer_forward_train(const moe_desc_t* d, const void* x, const void* Wg,
+                                     const float* sel_bias, const void* W_gate,
+                                     const void* W_up, const void* W_down, void* out, void* ws,
+                                     size_t ws_bytes, void* bwd_ws, size_t bwd_ws_bytes,
+                                     moe_stream_t stream) {
+  moe_status_t st = check_backward(d);
+  if (st != MOE_OK) return st;
+  BwdViews b;
+  if (!bwd_ws || bwd_ws_bytes < carve_bwd(d, nullptr, &b)) return MOE_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
+  carve_bwd(d, static_cast<uint8_t*>(bwd_ws), &b);
+  return forward_impl(d, x, Wg, sel_bias, W_gate, W_up, W_down, nullptr, nullptr, nullptr, out,
+                      ws, ws_bytes, b.gu, stream);
+}
+
 moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* Wg,
                                 const void* W_gate, const void* W_up, const void* W_down,
                                 const void* dout, float aux_grad, void* fwd_ws,
                                 size_t fwd_ws_bytes, void* dx, float* dWg, float* dW_gate,
                                 float* dW_up, float* dW_down, void* bwd_ws,
-                                size_t bwd_ws_bytes, moe_stream_t stream) {
+                                size_t bwd_ws_bytes, int32_t flags, moe_stream_t stream) {
   moe_status_t st = check_backward(d);
   if (st != MOE_OK) return st;
   moe_layer_views_t v;
@@ -493,6 +535,7 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
     if (!is_aligned16(p)) return MOE_ERR_INVALID_ARG;
   if (glu && (!is_aligned16(W_gate) || !is_aligned16(dW_gate))) return MOE_ERR_INVALID_ARG;
   if (!(aux_grad == aux_grad)) return MOE_ERR_INVALID_ARG;      // NaN
+  if (flags & ~MOE_BWD_PREACT_SAVED) return MOE_ERR_INVALID_ARG;
   BwdViews b;
   if (bwd_ws_bytes < carve_bwd(d, nullptr, &b)) return MOE_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
@@ -513,8 +556,9 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
   // dY = g dout on the executed rows, dg = <dout, y>
   if (e == cudaSuccess)
     e = launch_gather_dy(dout, v.y, v.row_src, v.gates, v.offsets, E, K, D, A, b.dY, b.dgates, s);
-  // pre-activations recomputed: SwiGLU gate | up blocks, or z = x W_up^T
-  if (e == cudaSuccess)
+  // pre-activations (SwiGLU gate | up blocks, or z = x W_up^T): saved by
+  // moe_layer_forward_train, else recomputed
+  if (e == cudaSuccess && !(flags & MOE_BWD_PREACT_SAVED))
     e = glu ? launch_grouped_gemm_bf16(EPI_RAW, v.x_perm, A, D, W_gate, W_up, E, F, v.offsets,
                                        b.gu, s)
             : launch_grouped_gemm_bf16(EPI_NONE, v.x_perm, A, D, W_up, nullptr, E, F, v.offsets,

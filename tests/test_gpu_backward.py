@@ -40,13 +40,19 @@ def _rel(got, ref):
     return float(np.abs(got - ref).max() / den) if den > 0 else float(np.abs(got).max())
 
 
-def run_backward(w, inp, dout, aux_grad):
+def run_backward(w, inp, dout, aux_grad, train=False, with_out=False):
+    """Forward (moe_layer_forward, or moe_layer_forward_train that saves the expert
+    pre-activations) then moe_layer_backward."""
     d = M.desc_of(w)
     ws = M.empty_workspace(d, "cuda")
     out = torch.empty_like(inp.x)
-    M.moe_layer_forward(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down, None,
-                        None, None, out, ws)
     bws = M.empty_backward_workspace(d, "cuda")
+    if train:
+        M.moe_layer_forward_train(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                                  out, ws, bws)
+    else:
+        M.moe_layer_forward(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down, None,
+                            None, None, out, ws)
     E, D, F = w.E, w.D, w.F
     dx = torch.empty_like(inp.x)
     dWg = torch.empty(E, D, dtype=torch.float32, device="cuda")
@@ -54,10 +60,14 @@ def run_backward(w, inp, dout, aux_grad):
     dWup = torch.empty(E, F, D, dtype=torch.float32, device="cuda")
     dWdown = torch.empty(E, D, F, dtype=torch.float32, device="cuda")
     M.moe_layer_backward(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, dout, aux_grad, ws,
-                         dx, dWg, dWgate, dWup, dWdown, bws)
+                         dx, dWg, dWgate, dWup, dWdown, bws,
+                         flags=M.BWD_PREACT_SAVED if train else 0)
     torch.cuda.synchronize()
     assert M.get_device_error() == 0
-    return M.layer_views(d, ws), dict(dx=dx, dWg=dWg, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown)
+    grads = dict(dx=dx, dWg=dWg, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown)
+    if with_out:
+        grads["out"] = out
+    return M.layer_views(d, ws), grads
 
 
 @pytest.mark.parametrize("name", list(CASES))
@@ -92,5 +102,21 @@ def test_backward_is_deterministic():
     _, a = run_backward(w, inp, dout, 1.0)
     a = {k: v.clone() for k, v in a.items() if v is not None}
     _, b = run_backward(w, inp, dout, 1.0)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+
+
+@pytest.mark.parametrize("name", ["swiglu_softmax_renorm", "gelu_sigmoid_bias_k3"])
+def test_saved_preactivations_give_identical_results(name):
+    # moe_layer_forward_train stores the up projection's accumulators; the backward then skips
+    # its recompute -- the same GEMM on the same operands, so every result is bit-identical
+    w = CASES[name]
+    inp = C.inputs_for(w)
+    g = torch.Generator(device="cuda")
+    g.manual_seed(12)
+    dout = torch.randn(w.T, w.D, generator=g, device="cuda").to(torch.bfloat16)
+    _, a = run_backward(w, inp, dout, 0.3, train=False, with_out=True)
+    a = {k: v.clone() for k, v in a.items() if v is not None}
+    _, b = run_backward(w, inp, dout, 0.3, train=True, with_out=True)
     for k in a:
         assert torch.equal(a[k], b[k]), k
