@@ -125,3 +125,22 @@ def test_header_entry_points_cite_the_pages():
     text = open(M.HEADER).read()
     for title in ("Top-k 路由", "Tiny MoE", "moe-comparison"):
         assert title in text
+
+
+def test_backward_validation_before_launch():
+    v = ctypes.c_size_t()
+    L = M.lib()
+    # bf16 token choice without shared experts only
+    for kw, st in ((dict(dtype=0), 2), (dict(select=1, c=8), 2), (dict(n_shared=1, F_shared=64), 2),
+                   (dict(k=0), 1)):
+        assert L.moe_backward_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == st, kw
+    d = M.desc_of(WORKLOADS["mixtral"])
+    assert L.moe_backward_workspace_size(ctypes.byref(d), ctypes.byref(v)) == 0
+    assert v.value > 0
+    # null pointers and unknown flags are rejected before anything is launched
+    st = L.moe_layer_backward(ctypes.byref(d), None, None, None, None, None, None, 1.0, None, 0,
+                              None, None, None, None, None, None, 0, 0, None)
+    assert st in (1, 3)
+    st = L.moe_layer_forward_train(ctypes.byref(d), None, None, None, None, None, None, None,
+                                   None, 0, None, 0, None)
+    assert st == 3                     # MOE_ERR_WORKSPACE: no backward workspace
