@@ -360,41 +360,62 @@ def run_cuda(args, rank, world, local):
         sh_off = torch.tensor([0, w.T], dtype=torch.int32, device=dev)
         h_sh = torch.empty(w.T, w.F_shared, dtype=inp.x.dtype, device=dev)
 
-    def step(ev=None):
+    def step(ev=None, st=None):
+        stream_ = st if st is not None else stream
         M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
-                    v["importance"], scratch, stream, entropy=v["entropy"])
+                    v["importance"], scratch, stream_, entropy=v["entropy"])
         if ev is not None:
-            ev[1].record(stream)
+            ev[1].record(stream_)
         M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
-                      v["row_src"], v["inv"], scratch, stream)
+                      v["row_src"], v["inv"], scratch, stream_)
         if ev is not None:
-            ev[2].record(stream)
+            ev[2].record(stream_)
         M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
-                        stream)
+                        stream_)
         if ev is not None:
-            ev[3].record(stream)
-        M.moe_expert_down(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], stream)
+            ev[3].record(stream_)
+        M.moe_expert_down(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], stream_)
         for i in range(w.n_shared):
             M.moe_expert_ffn(d_sh, 1, w.F_shared, inp.x, sh_off, inp.Ws_gate[i], inp.Ws_up[i],
-                             inp.Ws_down[i], h_sh, v["y_shared"][i], stream)
+                             inp.Ws_down[i], h_sh, v["y_shared"][i], stream_)
         if ev is not None:
-            ev[4].record(stream)
+            ev[4].record(stream_)
         M.moe_combine(d, v["y"], v["inv"], v["gates"], v["y_shared"] if w.n_shared else None,
-                      out, stream)
+                      out, stream_)
         if ev is not None:
-            ev[5].record(stream)
+            ev[5].record(stream_)
         M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
-                            stream, entropy=v["entropy"])
+                            stream_, entropy=v["entropy"])
         if ev is not None:
-            ev[6].record(stream)
+            ev[6].record(stream_)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
+
+    # the step captured once in a CUDA graph (the library allocates and synchronises nothing,
+    # so its calls capture as they are); replays remove the host launch gaps between kernels
+    graph, graph_launches, graph_error = None, 0, None
+    if not args.no_graph:
+        try:
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(stream)
+            g = torch.cuda.CUDAGraph()
+            n0 = M.kernel_launches()
+            with torch.cuda.graph(g, stream=cap):
+                step(st=cap)
+            graph_launches = M.kernel_launches() - n0
+            stream.wait_stream(cap)
+            for _ in range(max(args.warmup, 3)):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            graph = g
+        except Exception as e:          # capture not possible here: time the eager calls
+            graph_error = str(e).splitlines()[0][:200]
     nvml_index = local if "CUDA_VISIBLE_DEVICES" not in os.environ else \
         int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
 
-    def timed():
+    def timed(use_graph):
         evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)]
                for _ in range(args.steps)]
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -404,25 +425,39 @@ def run_cuda(args, rank, world, local):
             n0 = M.kernel_launches()
             start.record(stream)
             for i in range(args.steps):
-                evs[i][0].record(stream)
-                step(evs[i])
+                if use_graph:
+                    graph.replay()
+                else:
+                    evs[i][0].record(stream)
+                    step(evs[i])
             end.record(stream)
-            launches = M.kernel_launches() - n0
+            launches = (graph_launches * args.steps if use_graph
+                        else M.kernel_launches() - n0)
             torch.cuda.synchronize(dev)
         barrier(world)
         total = start.elapsed_time(end)
+        if use_graph:
+            return total, None, clk, launches
         per_stage = {s: 0.0 for s in STAGES}
         for i in range(args.steps):
             for j, s in enumerate(STAGES):
                 per_stage[s] += evs[i][j].elapsed_time(evs[i][j + 1])
         return total, {s: per_stage[s] / args.steps for s in STAGES}, clk, launches
 
-    total_ms, per_stage, clk, launches = timed()
+    # the headline from graph replays (timed first), per-stage times from the eager calls
+    # (events between stages)
+    use_graph = graph is not None
+    total_ms, per_stage, clk, launches = timed(use_graph)
     remeasured = False
     if clk.rejected():
-        total_ms, per_stage, clk, launches = timed()
+        total_ms, per_stage, clk, launches = timed(use_graph)
         remeasured = True
+    if use_graph:
+        eager_ms, per_stage, _, _ = timed(False)
+    else:
+        eager_ms = total_ms
     total_ms = max_over_ranks(total_ms, world, dev)
+    eager_ms = max_over_ranks(eager_ms, world, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(w.T, world, args.steps, total_ms)
 
@@ -502,6 +537,11 @@ def run_cuda(args, rank, world, local):
                 "serial_value": round(job_throughput(w.T, world, args.steps, e2e_serial_ms), 1)},
         "gpu_launches": launches,
         "clocks": clk.summary(),
+        "timing": ("CUDA-graph replay of the step (%d library kernels per step); per-stage "
+                   "times from eager calls" % graph_launches) if use_graph else
+                  ("eager calls" + (" (graph capture failed: %s)" % graph_error
+                                    if graph_error else "")),
+        "eager_value": round(job_throughput(w.T, world, args.steps, eager_ms), 1),
     }
     if remeasured:
         res["clocks"]["remeasured"] = True
@@ -630,6 +670,8 @@ def main():
                     help="override the batch size T (smaller cases for profiling)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time eager calls instead of a CUDA-graph replay of the step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass timing that follows the forward measurement")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
