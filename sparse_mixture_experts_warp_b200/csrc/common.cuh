@@ -67,7 +67,8 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
 
 // gemm_sm100.cu (bf16 grouped GEMM on tcgen05)
 enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI_GELU = 4,
-                    EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */ };
+                    EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */,
+                    EPI_NONE_BMN = 6 /* EPI_NONE with an MN-major B operand */ };
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,
@@ -79,6 +80,13 @@ int router_gemm_splits(int T, int D);
 cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg, int E,
                                     float* partials, int ksplit, cudaStream_t s);
 
+// out = A B per group along M with B stored MN-major ([K, N], N contiguous; the layout of
+// nn.Linear weights used as the right operand of a backward product): group g reads its K rows
+// at g * bk_group of B0 for k-blocks below kb_split and of B1 above it (B1 may be null).
+cudaError_t launch_grouped_gemm_bf16_bmn(const void* A, int64_t a_rows, int K, const void* B0,
+                                         const void* B1, int kb_split, int bk_group,
+                                         int n_groups, int N, const int32_t* offsets, void* out,
+                                         cudaStream_t s);
 // out[g] = A[:, K_g] B[:, K_g]^T (fp32 [M, N] per group) for groups along K: group g owns the
 // k columns [kgroup[g], kgroup[g+1]) of A [M, k_total] and B [N, k_total] (bf16, K-major,
 // kgroup a device array of multiples of 64).

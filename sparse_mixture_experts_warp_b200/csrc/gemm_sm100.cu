@@ -88,6 +88,10 @@ struct GemmParams {
   // n-tile, row pitch ldo2 = nt * 256; others: [rows, N]), saved for the backward pass
   __nv_bfloat16* out2;
   int64_t ldo2;
+  // MN-major B (EPI_NONE_BMN): k-blocks below kb_split come from tmB0, the rest from tmB1;
+  // group g's K rows start at row g * bk_group of either tensor
+  int kb_split;
+  int bk_group;
 };
 
 // One work item of the persistent schedule.
@@ -208,6 +212,19 @@ __device__ __forceinline__ uint64_t sdesc(uint32_t saddr) {
   d |= (uint64_t)((8 * KB * 2) >> 4) << 32;         // stride byte offset: 8 rows
   d |= (uint64_t)1 << 46;                           // descriptor version for tcgen05
   d |= (uint64_t)(KB == 64 ? 2 : 4) << 61;          // 128-byte or 64-byte swizzle
+  return d;
+}
+
+// Shared-memory matrix descriptor, MN-major operand with 128-byte swizzle: 64 MN-elements
+// (128 B) per row, 8-row (K) groups 1024 B apart (stride byte offset), 64-element MN blocks
+// 8192 B apart (leading byte offset: one 64 x 64 TMA box each).
+__device__ __forceinline__ uint64_t sdesc_mn(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);        // start address
+  d |= (uint64_t)(8192 >> 4) << 16;                 // leading byte offset: next MN block
+  d |= (uint64_t)(1024 >> 4) << 32;                 // stride byte offset: next 8 K rows
+  d |= (uint64_t)1 << 46;                           // descriptor version for tcgen05
+  d |= (uint64_t)2 << 61;                           // 128-byte swizzle
   return d;
 }
 
@@ -492,7 +509,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
           tma_load_2d(a_dst, &tmA, &full[stage], kx, a_row);
           if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kx, a_row + BM);
-          if (EPI == EPI_SWIGLU || EPI == EPI_RAW) {
+          if (EPI == EPI_NONE_BMN) {
+            // [K, N] boxes of 64 x 64: four N blocks of 64 for this k-block
+            const bool hi = kb >= p.kb_split;
+            const int krow = tl.g * p.bk_group + (hi ? kb - p.kb_split : kb) * KB;
+            const int n0 = tl.n_idx * p.n_out_tile;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              tma_load_2d(b_dst + j * (TB_BYTES / 4), hi ? &tmB1 : &tmB0, &full[stage], n0 + 64 * j,
+                          krow);
+          } else if (EPI == EPI_SWIGLU || EPI == EPI_RAW) {
             tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
             tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kx, b_row);
           } else {
@@ -529,8 +555,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const int kb0 = tl.kb0, kb1 = tl.kb1;      // kb0 == kb1: an empty group along K
         // M = 64 for a half with at most 64 live rows
         const int live0 = min(BM, m - m_idx * TBM), live1 = min(BM, m - m_idx * TBM - BM);
-        const uint32_t idesc0 = live0 <= 64 ? kIdesc64 : kIdesc;
-        const uint32_t idesc1 = live1 <= 64 ? kIdesc64 : kIdesc;
+        // MN-major B: the transpose-B bit (16) of the instruction descriptor
+        const uint32_t bmaj = EPI == EPI_NONE_BMN ? (1u << 16) : 0u;
+        const uint32_t idesc0 = (live0 <= 64 ? kIdesc64 : kIdesc) | bmaj;
+        const uint32_t idesc1 = (live1 <= 64 ? kIdesc64 : kIdesc) | bmaj;
         const int acc = it % NBUF;
         const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
         if (!mbar_wait(&tempty[acc], acc_par ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_MMA,
@@ -550,7 +578,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const uint32_t a0 = sA + stage * TA_BYTES, b0 = sB + stage * TB_BYTES;
 #pragma unroll
           for (int k = 0; k < KB / MMA_K; ++k) {
-            const uint64_t bdesc = sdesc<KB>(b0 + k * MMA_K * 2);
+            // K-major: the k-step moves 32 bytes along each row; MN-major: 16 rows of 128 B
+            const uint64_t bdesc = EPI == EPI_NONE_BMN ? sdesc_mn(b0 + k * MMA_K * 128)
+                                                       : sdesc<KB>(b0 + k * MMA_K * 2);
             const uint32_t accum = (kb > kb0 || k > 0) ? 1u : 0u;
             umma_bf16(d_tmem, sdesc<KB>(a0 + k * MMA_K * 2), bdesc, accum, idesc0);
             if (two)
@@ -1155,6 +1185,8 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
     case EPI_F32: return launch_epi<EPI_F32, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_GELU: return launch_epi<EPI_GELU, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     case EPI_RAW: return launch_epi<EPI_RAW, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
+    case EPI_NONE_BMN:
+      return launch_epi<EPI_NONE_BMN, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
     default: return launch_epi<EPI_NONE, HALVES, KB, NSTAGES>(a, b0, b1, p, grid, smem, s);
   }
 }
@@ -1246,6 +1278,8 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.out_gstride = 0;
   p.out2 = static_cast<__nv_bfloat16*>(out2);
   p.ldo2 = (epi == EPI_SWIGLU) ? (int64_t)p.nt * 256 : N;
+  p.kb_split = 0;
+  p.bk_group = 0;
   p.fault = g_gemm_fault;
   p.ksplit = 1;
   p.kchunk = 1 << 30;
@@ -1289,6 +1323,47 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
 
 void set_gemm_fault(int kind) { g_gemm_fault = kind; }
 
+cudaError_t launch_grouped_gemm_bf16_bmn(const void* A, int64_t a_rows, int K, const void* B0,
+                                         const void* B1, int kb_split, int bk_group,
+                                         int n_groups, int N, const int32_t* offsets, void* out,
+                                         cudaStream_t s) {
+  if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb0, tb1;
+  const uint64_t brows = (uint64_t)n_groups * (uint64_t)bk_group;
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb0, B0, brows, (uint64_t)N, 64, 64)) return cudaErrorInvalidValue;
+  if (B1) {
+    if (!make_map(&tb1, B1, brows, (uint64_t)N, 64, 64)) return cudaErrorInvalidValue;
+  } else {
+    tb1 = tb0;
+  }
+  GemmParams p;
+  p.offsets = offsets;
+  p.out = static_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  p.rows = a_rows;
+  p.ldo = N;
+  p.G = n_groups;
+  p.N = N;
+  p.K = K;
+  p.n_out_tile = 256;
+  p.nt = (N + 255) / 256;
+  p.fault = g_gemm_fault;
+  p.ksplit = 1;
+  p.kchunk = 1 << 30;
+  p.split_stride = 0;
+  p.kgroup = nullptr;
+  p.out_gstride = 0;
+  p.out2 = nullptr;
+  p.ldo2 = 0;
+  p.kb_split = kb_split;
+  p.bk_group = bk_group;
+  const int64_t max_tiles = ((a_rows + 2 * BM - 1) / (2 * BM) + n_groups) * (int64_t)p.nt;
+  const int grid = (int)(max_tiles < sm_count() ? max_tiles : sm_count());
+  return launch_epi<EPI_NONE_BMN, 2, 64, 3>(ta, tb0, tb1, p, grid, gemm_smem(2, 64, 3, n_groups),
+                                            s);
+}
+
 cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B, int N, int G,
                                             const int32_t* kgroup, int64_t k_total, float* out,
                                             cudaStream_t s) {
@@ -1315,6 +1390,8 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   p.out_gstride = (int64_t)M * N;
   p.out2 = nullptr;
   p.ldo2 = 0;
+  p.kb_split = 0;
+  p.bk_group = 0;
   // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (256 KB) overlaps
   // the next tile's main loop, which is short here (one expert's rows)
   const int64_t tiles = (int64_t)G * ((M + BM - 1) / BM) * p.nt;
@@ -1361,6 +1438,8 @@ cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg,
   p.out_gstride = 0;
   p.out2 = nullptr;
   p.ldo2 = 0;
+  p.kb_split = 0;
+  p.bk_group = 0;
   const int64_t tiles = (int64_t)((T + BM - 1) / BM) * ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, 1), s);

@@ -4,6 +4,7 @@
 // moe-comparison), Score -> Select -> Merge -> Execute.  No entry point allocates, frees or
 // synchronises (moe_get_device_error excepted); all work goes on the caller's stream.
 #include <math.h>
+#include <stdlib.h>
 #include <string.h>
 
 #include <atomic>
@@ -449,6 +450,14 @@ struct BwdViews {
   int64_t ldg, nab, pad_cols;
 };
 
+bool bwd_weight_transpose() {
+  static const bool v = [] {
+    const char* s = getenv("MOE_BWD_WEIGHT_TRANSPOSE");
+    return s && s[0] == '1';
+  }();
+  return v;
+}
+
 moe_status_t check_backward(const moe_desc_t* d) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
@@ -479,8 +488,9 @@ size_t carve_bwd(const moe_desc_t* d, uint8_t* base, BwdViews* v) {
   v->dAB = take(A * v->nab * 2);
   v->dXp = take(A * D * 2);
   v->ds = static_cast<float*>(take(T * E * 4));
-  v->WdT = take(E * F * D * 2);
-  v->WguT = take(E * D * v->nab * 2);
+  const bool tw = bwd_weight_transpose();
+  v->WdT = take(tw ? E * F * D * 2 : 0);
+  v->WguT = take(tw ? E * D * v->nab * 2 : 0);
   v->dYT = take(D * v->pad_cols * 2);
   v->hT = take(F * v->pad_cols * 2);
   v->xpT = take(D * v->pad_cols * 2);
@@ -563,23 +573,36 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
                                        b.gu, s)
             : launch_grouped_gemm_bf16(EPI_NONE, v.x_perm, A, D, W_up, nullptr, E, F, v.offsets,
                                        b.gu, s);
-  // dH = dY W_down: B = W_down^T per expert ([F, D], K-major)
-  if (e == cudaSuccess)
+  // dH = dY W_down and dX = [da | db] [W_gate ; W_up]: the weights are the right operands
+  // in their stored layout ([K, N], MN-major B); MOE_BWD_WEIGHT_TRANSPOSE=1 selects the
+  // alternative that first transposes them into K-major copies
+  const bool transpose = bwd_weight_transpose();
+  if (e == cudaSuccess && transpose) {
     e = launch_transpose(W_down, (int64_t)D * F, D, F, F, b.WdT, (int64_t)F * D, D, 0, E, s);
-  if (e == cudaSuccess)
-    e = launch_grouped_gemm_bf16(EPI_NONE, b.dY, A, D, b.WdT, nullptr, E, F, v.offsets, b.dH, s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_bf16(EPI_NONE, b.dY, A, D, b.WdT, nullptr, E, F, v.offsets, b.dH,
+                                   s);
+  } else if (e == cudaSuccess) {
+    e = launch_grouped_gemm_bf16_bmn(b.dY, A, D, W_down, nullptr, D / 64, D, E, F, v.offsets,
+                                     b.dH, s);
+  }
   // activation backward -> [da | db] (SwiGLU) or dz
   if (e == cudaSuccess)
     e = launch_act_backward(d->act, b.dH, b.gu, b.ldg, v.offsets, E, F, A, b.dAB, s);
-  // dX = [da | db] [W_gate ; W_up]: B = [W_gate^T | W_up^T] per expert ([D, 2F])
-  if (e == cudaSuccess && glu)
-    e = launch_transpose(W_gate, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab, 0, E, s);
-  if (e == cudaSuccess)
-    e = launch_transpose(W_up, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab,
-                         glu ? F : 0, E, s);
-  if (e == cudaSuccess)
-    e = launch_grouped_gemm_bf16(EPI_NONE, b.dAB, A, nab, b.WguT, nullptr, E, D, v.offsets,
-                                 b.dXp, s);
+  if (e == cudaSuccess && transpose) {
+    if (glu)
+      e = launch_transpose(W_gate, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab, 0, E,
+                           s);
+    if (e == cudaSuccess)
+      e = launch_transpose(W_up, (int64_t)F * D, F, D, D, b.WguT, (int64_t)D * nab, nab,
+                           glu ? F : 0, E, s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_bf16(EPI_NONE, b.dAB, A, nab, b.WguT, nullptr, E, D, v.offsets,
+                                   b.dXp, s);
+  } else if (e == cudaSuccess) {
+    e = launch_grouped_gemm_bf16_bmn(b.dAB, A, nab, glu ? W_gate : W_up, glu ? W_up : nullptr,
+                                     F / 64, F, E, D, v.offsets, b.dXp, s);
+  }
   // router: ds, then dx = sum_j dX[inv] + ds W_g and dW_g = ds^T x
   if (e == cudaSuccess)
     e = launch_router_backward(*d, v.logits, v.expert_ids, v.gates, b.dgates, v.inv, v.f,

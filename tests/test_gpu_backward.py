@@ -120,3 +120,16 @@ def test_saved_preactivations_give_identical_results(name):
     _, b = run_backward(w, inp, dout, 0.3, train=True, with_out=True)
     for k in a:
         assert torch.equal(a[k], b[k]), k
+
+
+def test_backward_with_transposed_weight_copies_in_subprocess():
+    """MOE_BWD_WEIGHT_TRANSPOSE=1 makes the dgrad products use K-major transposed copies of the
+    weights instead of reading them MN-major; run this file's parity cases under it."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_BWD_WEIGHT_TRANSPOSE="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__,
+                        "-k", "matches_oracle and not mixtral_width"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
