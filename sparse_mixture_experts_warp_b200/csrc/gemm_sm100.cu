@@ -14,11 +14,22 @@
 //   EPI_RELU:   out = max(acc, 0) with B0 = W_up.
 //   EPI_GELU:   out = acc * (1 + erf(acc / sqrt 2)) / 2 with B0 = W_up.
 //   EPI_NONE:   out = acc with B0 = W_down.
+//   Also used by the layer backward:
+//   EPI_RAW:      SwiGLU operand staging, out = the raw gate | up accumulators (bf16);
+//   EPI_NONE_BMN: out = acc with B stored MN-major ([K, N], N contiguous: a weight used as the
+//                 right operand of a backward product, read as stored); K rows of group g at
+//                 g * bk_group of B0 below k-block kb_split and of B1 above it;
+//   EPI_F32:      fp32 out; with `kgroup` the groups run along K instead of M (weight
+//                 gradients: group g owns k columns [kgroup[g], kgroup[g+1]) of A [M, Ktot]
+//                 and B [N, Ktot] and writes its own [M, N] block), without it k-splits of one
+//                 group write fp32 partials (the router product).
+//   An optional second output (out2) receives the raw accumulators of the SwiGLU / activation
+//   epilogues as bf16: the pre-activations a training forward saves for the backward.
 //
 // Design (one persistent CTA per SM, warp-specialised; two tile heights, see grouped_gemm_kernel):
 //   warp 0 (one thread)  TMA producer: 128-byte-swizzled K-major boxes of A (128 x 64, one or two
-//                        per stage) and B (2 x 128 x 64) into a shared-memory ring, mbarrier
-//                        complete_tx; no multicast.
+//                        per stage) and B (2 x 128 x 64; MN-major B: 4 x 64 x 64) into a
+//                        shared-memory ring, mbarrier complete_tx; no multicast.
 //   warp 1 (one thread)  MMA issuer: tcgen05.mma.cta_group::1.kind::f16, M=128 N=256 K=16, fp32
 //                        accumulators in TMEM (512 columns); tcgen05.commit frees ring stages and
 //                        hands finished accumulators to the epilogue.  Warp 1 also owns the TMEM
