@@ -32,6 +32,10 @@ CASES = {
                                    F_shared=0, act="gelu"),
     "empty_expert": scaled(W["mixtral"], T=5, D=128, E=16, k=2, F=128),
     "mixtral_width_T64": scaled(W["mixtral"], T=64),
+    # DeepSeek-V3 routing (256 experts, top-8, sigmoid + selection bias) without the shared
+    # expert, at D = 256, F = 128 so the fp64 oracle stays small: 256 groups along K in the
+    # weight gradients, E = 256 in the router backward and dW_g
+    "v3_routing_E256": scaled(W["v3"], T=128, D=256, F=128, n_shared=0, F_shared=0),
 }
 
 
