@@ -303,14 +303,23 @@ router_kernel(RouterArgs a) {
   }
 
   if (a.partials) {
-    // row gw of the partials: E importance sums, then the entropy sum
+    // one partial row per block: E importance sums, then the entropy sum, over the block's
+    // warps in a fixed order (s_all held the logits; every warp is past its last use of it)
+    ent = warp_sum(ent);
+    __syncthreads();
+    float* s_part = s_all + warp * (E + 1);
 #pragma unroll
     for (int i = 0; i < kMaxEPL; ++i) {
       const int e = lane + 32 * i;
-      if (e < E) a.partials[(int64_t)gw * (E + 1) + e] = imp[i];
+      if (e < E) s_part[e] = imp[i];
     }
-    ent = warp_sum(ent);
-    if (lane == 0) a.partials[(int64_t)gw * (E + 1) + E] = ent;
+    if (lane == 0) s_part[E] = ent;
+    __syncthreads();
+    for (int c = threadIdx.x; c <= E; c += blockDim.x) {
+      float sum = 0.f;
+      for (int w = 0; w < kWarps; ++w) sum += s_all[w * (E + 1) + c];
+      a.partials[(int64_t)blockIdx.x * (E + 1) + c] = sum;
+    }
   }
 }
 
@@ -577,10 +586,9 @@ router_fast_kernel(RouterArgs a, int tokens_per_cta) {
 
 }  // namespace
 
-// Rows of importance partials the generic kernel writes (one per warp).
+// Rows of importance partials the generic kernel writes (one per block).
 static int generic_partials(const moe_desc_t& d) {
-  const int blocks = (d.T + kWarps * kTPW - 1) / (kWarps * kTPW);
-  return blocks * kWarps;
+  return (d.T + kWarps * kTPW - 1) / (kWarps * kTPW);
 }
 
 int router_partials(const moe_desc_t& d) {
