@@ -372,10 +372,25 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
   return before + inc - v;
 }
 
+// staged: the expert's T keys are first copied to shared memory (dynamic, T * 4 bytes) in one
+// pass with 16-byte loads, so the four histogram passes and the compaction read them from
+// there instead of going back to L2 with one dependent load per thread and pass.
+template <bool STAGED>
 __global__ void __launch_bounds__(1024)
 ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
   const int e = blockIdx.x;
-  const uint32_t* keys = reinterpret_cast<const uint32_t*>(probsT + (int64_t)e * T);
+  const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(probsT + (int64_t)e * T);
+  extern __shared__ uint32_t s_keys[];
+  const uint32_t* keys = gkeys;
+  if (STAGED) {
+    // T * 4 bytes from a row start of probsT: 16-byte aligned when T % 4 == 0 (the launcher
+    // stages only then)
+    const uint4* src = reinterpret_cast<const uint4*>(gkeys);
+    uint4* dst = reinterpret_cast<uint4*>(s_keys);
+    for (int i = threadIdx.x; i < T / 4; i += blockDim.x) dst[i] = src[i];
+    __syncthreads();
+    keys = s_keys;
+  }
   __shared__ int hist[256];
   __shared__ int s_digit, s_need;
   __shared__ int s_warp[32];
@@ -676,7 +691,17 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
 
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s) {
-  ec_select_kernel<<<counted(d.E), 1024, 0, s>>>(probsT, d.T, d.c, picked);
+  const size_t smem = (size_t)d.T * sizeof(float);
+  if (d.T % 4 == 0 && smem <= 200 * 1024) {
+    if (smem > 48 * 1024) {
+      cudaError_t e = cudaFuncSetAttribute(ec_select_kernel<true>,
+                                           cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+      if (e != cudaSuccess) return e;
+    }
+    ec_select_kernel<true><<<counted(d.E), 1024, smem, s>>>(probsT, d.T, d.c, picked);
+  } else {
+    ec_select_kernel<false><<<counted(d.E), 1024, 0, s>>>(probsT, d.T, d.c, picked);
+  }
   return cudaGetLastError();
 }
 
