@@ -522,9 +522,8 @@ def run_cuda(args, rank, world, local):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random-init)",
-        "config": {"workload": w.name, "model": w.description, "T": w.T,
-                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "global_batch": w.T * world,
-                   "seq_len": w.T,
+        "config": {"workload": w.name, "shape": w.description, "T": w.T,
+                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "tokens_per_step": w.T * world,
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
                    "rows_executed": rows_exec,
                    "l2": "inputs larger than L2: %.2f GB of expert weights stream per step"
@@ -649,9 +648,9 @@ def run_reference(args, rank, world):
         "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded N(0,1) tokens, N(0,0.02) weights, random-init)",
-        "config": {"workload": w.name, "model": w.description, "T": w.T,
-                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "global_batch": w.T,
-                   "seq_len": w.T, "parallelism": "CPU oracle (rank 0)"},
+        "config": {"workload": w.name, "shape": w.description, "T": w.T,
+                   "D": w.D, "E": w.E, "k": w.k, "F": w.F, "tokens_per_step": w.T,
+                   "parallelism": "CPU oracle (rank 0)"},
         "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(),
                          "kind": "oracle", "sample": desc},
         "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
