@@ -14,8 +14,9 @@
 //   dX = da W_gate + db W_up,  dW_down = dY^T h,  dW_gate = da^T x,  dW_up = db^T x;
 // router: ds from dg through the merge weights, plus the balance-loss term through P;
 //   dW_g = ds^T x,  dx[t] = sum_j dX[r(t, j)] + ds[t] W_g.
-// The big products run on the tcgen05 grouped GEMM: dgrad with transposed weights (K-major B),
-// wgrad with groups along K over per-expert row blocks transposed and zero-padded to 64.
+// The big products run on the tcgen05 grouped GEMM: dgrad reads the weights as stored, an
+// MN-major B operand (or K-major transposed copies when MOE_BWD_WEIGHT_TRANSPOSE=1), wgrad runs
+// with groups along K over per-expert row blocks transposed and zero-padded to 64.
 // This file holds the memory-bound pieces.
 #include "common.cuh"
 
