@@ -58,3 +58,27 @@ def test_reference_arm_runs_on_rank_zero_only():
     class A:
         steps, warmup, workload, tokens, ref_budget = 1, 3, "mixtral", 0, 1.0
     assert bench.run_reference(A(), rank=1, world=2) is None     # returns without work
+
+
+def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
+    # a small Mixtral-shaped layer so that the fp64 oracle steps take well under a second
+    import json
+    from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, scaled
+    small = scaled(WORKLOADS["mixtral"], T=64, D=128, F=128)
+    monkeypatch.setattr(bench, "workload_of", lambda args: small)
+
+    class A:
+        steps, warmup, workload, tokens, ref_budget = 2, 3, "mixtral", 0, 0.5
+    bench.run_reference(A(), rank=0, world=1)
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1
+    r = json.loads(lines[0])
+    assert r["impl"] == "reference" and r["metric"] == bench.METRIC
+    assert r["unit"] == "tokens/s" and r["higher_is_better"] is True
+    assert r["steps"] == 2 and r["warmup"] == 3 and r["n_gpus"] == 1
+    assert r["value"] > 0 and r["dtype"] == "f64"
+    assert r["config"]["workload"] == small.name and "model" not in r["config"]
+    assert r["cpu_baseline"]["kind"] == "oracle" and r["cpu_baseline"]["value"] == r["value"]
+    assert r["cpu_baseline"]["cores"] >= 1 and r["cpu_baseline"]["sample"]
+    assert r["e2e"] == {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
