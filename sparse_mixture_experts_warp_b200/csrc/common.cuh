@@ -68,7 +68,8 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
 // gemm_sm100.cu (bf16 grouped GEMM on tcgen05)
 enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI_GELU = 4,
                     EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */,
-                    EPI_NONE_BMN = 6 /* EPI_NONE with an MN-major B operand */ };
+                    EPI_NONE_BMN = 6 /* EPI_NONE with an MN-major B operand */,
+                    EPI_F32_TMA = 7 /* EPI_F32 written by TMA stores from shared memory */ };
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,

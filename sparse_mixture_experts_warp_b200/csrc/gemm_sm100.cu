@@ -22,7 +22,13 @@
 //   EPI_F32:      fp32 out; with `kgroup` the groups run along K instead of M (weight
 //                 gradients: group g owns k columns [kgroup[g], kgroup[g+1]) of A [M, Ktot]
 //                 and B [N, Ktot] and writes its own [M, N] block), without it k-splits of one
-//                 group write fp32 partials (the router product).
+//                 group write fp32 partials (the router product);
+//   EPI_F32_TMA:  EPI_F32 with groups along K, written through shared memory: each epilogue
+//                 warp stages a 32 x 32 fp32 block (128-byte swizzle, two buffers per warp) and
+//                 one lane stores it with a 3-D TMA store (columns, rows, group) that clips at
+//                 the group's bounds.  A weight-gradient tile has a short main loop (one
+//                 expert's rows) and 128 KB of fp32 output; per-thread row stores would touch 32
+//                 rows per instruction and hold the tensor pipe back.
 //   An optional second output (out2) receives the raw accumulators of the SwiGLU / activation
 //   epilogues as bf16: the pre-activations a training forward saves for the backward.
 //
@@ -213,6 +219,33 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Shared -> global tile store through a 3-D tensor map (x = column, y = row, z = group); the
+// copy joins the issuing thread's current bulk group.
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y,
+                                             int z) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.global.shared::cta.bulk_group [%0, {%2, %3, %4}], [%1];" ::"l"(
+          reinterpret_cast<uint64_t>(map)),
+      "r"(src), "r"(x), "r"(y), "r"(z)
+      : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+// Wait until at most N of this thread's bulk groups are still reading shared memory.
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+  asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+// Wait until all of this thread's bulk groups have completed (their writes are done).
+__device__ __forceinline__ void bulk_wait_all() {
+  asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+// Make this thread's generic-proxy shared-memory writes visible to the TMA (async proxy).
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, rows of KB bf16 (KB = 64: 128-byte swizzle, 8-row
 // core groups 1024 B apart; KB = 32: 64-byte swizzle, groups 512 B apart).
 template <int KB>
@@ -383,6 +416,8 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
 // HALVES = 2: 256-row tiles made of two M=128 MMAs that share every B stage (a third fewer
 //             L2->SMEM bytes per FLOP), 3-stage ring of 64 KB, one 512-column accumulator set,
 //             8 epilogue warps; a tile with <= 128 live rows loads and multiplies one half only.
+// tmB1 is the second B operand (SwiGLU, EPI_RAW, EPI_NONE_BMN) or, for EPI_F32_TMA, the fp32
+// output map: [groups][rows][N], boxes of 32 columns x 32 rows, 128-byte swizzle.
 template <int EPI, int HALVES, int KB, int NSTAGES>
 __global__ void __launch_bounds__(64 + 128 * HALVES, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -396,12 +431,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr int NBUF = HALVES == 1 ? 2 : 1;          // TMEM accumulator buffers
   constexpr int BUF_COLS = HALVES * ACC_COLS;        // columns per buffer
   constexpr int N_EPI = 4 * HALVES;                  // epilogue warps
+  // EPI_F32_TMA: two 4 KB staging buffers (32 rows x 32 fp32) per epilogue warp
+  constexpr int STG_BYTES = EPI == EPI_F32_TMA ? N_EPI * 2 * 4096 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   const uint32_t sA = smem_u32(smem);
   const uint32_t sB = sA + TSTAGES * TA_BYTES;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + TSTAGES * (TA_BYTES + TB_BYTES));
+  const uint32_t sStg = sB + TSTAGES * TB_BYTES;     // 1024-byte aligned (the ring is)
+  uint64_t* bars =
+      reinterpret_cast<uint64_t*>(smem + TSTAGES * (TA_BYTES + TB_BYTES) + STG_BYTES);
   uint64_t* full = bars;
   uint64_t* empty = bars + TSTAGES;
   uint64_t* tfull = bars + 2 * TSTAGES;
@@ -431,7 +470,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   if (warp == 0 && lane == 0) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmA)) : "memory");
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB0)) : "memory");
-    if (EPI == EPI_SWIGLU || EPI == EPI_RAW)
+    if (EPI == EPI_SWIGLU || EPI == EPI_RAW || EPI == EPI_F32_TMA)
       asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmB1)) : "memory");
   }
   if (warp == 1) {
@@ -616,6 +655,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
     int g = 0, it = 0;
+    uint32_t nstored = 0;                    // EPI_F32_TMA: staged chunks this warp has stored
     for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
       const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
       const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
@@ -699,12 +739,15 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           if (valid && f + 64 < p.N) store_act32<EPI_NONE>(v2, o + c + 64);
           if (valid && f + 96 < p.N) store_act32<EPI_NONE>(v3, o + c + 96);
         }
-      } else if (EPI == EPI_F32) {
+      } else if (EPI == EPI_F32 || EPI == EPI_F32_TMA) {
         // fp32 partial of this k-split, rows of out32 + split * split_stride (+ the group's
         // output block when groups run along K)
         float* orow32 = reinterpret_cast<float*>(p.out) + split * p.split_stride +
                         (p.kgroup ? (int64_t)tl.g * p.out_gstride : 0) + orow * p.ldo +
                         (int64_t)n_idx * p.n_out_tile;
+        // TMA stores need the warp's 32 rows in its 32 lanes: a tile of at most 64 live rows
+        // (M = 64 MMA, 16 rows per lane quarter) keeps the per-thread stores
+        const bool staged = EPI == EPI_F32_TMA && !m64;
 #pragma unroll 1
         for (int c = 0; c < MMA_N; c += 32) {
           uint32_t v[32];
@@ -720,7 +763,30 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             mbar_arrive(&tempty[acc]);
           }
           const int col = n_idx * p.n_out_tile + c;
-          if (valid && col < p.N) {
+          if (staged) {
+            if (col >= p.N) continue;        // warp-uniform: the chunk lies past the last column
+            // buffer (nstored & 1) of this warp; the store that used it two chunks ago must
+            // have finished reading it
+            const uint32_t buf = sStg + (uint32_t)((((warp - 2) << 1) | (nstored & 1)) << 12);
+            if (lane == 0) bulk_wait_read<1>();
+            __syncwarp();
+            // row `lane`, 16-byte chunk i at chunk position i ^ (lane % 8): the 128-byte swizzle
+            // the tensor map names (conflict-free: 8 lanes of a phase hit 8 different chunks)
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              const uint32_t a = buf + (uint32_t)(lane << 7) + (uint32_t)((i ^ (lane & 7)) << 4);
+              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[4 * i]),
+                           "r"(v[4 * i + 1]), "r"(v[4 * i + 2]), "r"(v[4 * i + 3])
+                           : "memory");
+            }
+            fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_3d(&tmB1, buf, col, m_idx * TBM + half * BM + 32 * q, tl.g);
+              bulk_commit();
+            }
+            ++nstored;
+          } else if (valid && col < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -756,6 +822,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         }
       }
     }
+    // the TMA stores this warp issued complete before the kernel ends
+    if (EPI == EPI_F32_TMA && lane == 0) bulk_wait_all();
   }
   __syncwarp();
   tc_fence_before();
@@ -1131,6 +1199,20 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+// 3D fp32 tensor [groups][rows][cols] (dense); box = 32 columns x 32 rows x 1 group, 128-byte
+// swizzle (one 128-byte row of the box per swizzle row): the EPI_F32_TMA output.
+bool make_map_f32_out(CUtensorMap* m, void* ptr, uint64_t groups, uint64_t rows, uint64_t cols) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[3] = {cols, rows, groups};
+  const cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
+  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 // 2D bf16 tensor [rows, cols] row-major; box = 64 columns x box_rows rows, 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,
               int kb) {
@@ -1203,9 +1285,11 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
 }
 
 // Dynamic shared memory of one configuration (ring + barriers + group tables + alignment).
-size_t gemm_smem(int halves, int kb, int nstages, int n_groups) {
+// `staging`: the EPI_F32_TMA store buffers between the ring and the barriers.
+size_t gemm_smem(int halves, int kb, int nstages, int n_groups, size_t staging = 0) {
   const size_t ring = (size_t)nstages * ((size_t)halves * BM * kb * 2 + (size_t)MMA_N * kb * 2);
-  return 1024 + ring + (2 * nstages + 5) * 8 + 8 + (size_t)2 * (n_groups + 1) * sizeof(int);
+  return 1024 + ring + staging + (2 * nstages + 5) * 8 + 8 +
+         (size_t)2 * (n_groups + 1) * sizeof(int);
 }
 
 constexpr int kPairStages = 4;
@@ -1403,11 +1487,23 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   p.ldo2 = 0;
   p.kb_split = 0;
   p.bk_group = 0;
-  // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (256 KB) overlaps
-  // the next tile's main loop, which is short here (one expert's rows)
+  // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (128 KB, written by
+  // TMA stores from shared memory) overlaps the next tile's main loop, which is short here (one
+  // expert's rows).  The output needs 16-byte aligned rows: N a multiple of 4.
+  if (N % 4 || (reinterpret_cast<uintptr_t>(out) & 15)) return cudaErrorInvalidValue;
+  alignas(64) CUtensorMap to;
+  if (!make_map_f32_out(&to, out, (uint64_t)G, (uint64_t)M, (uint64_t)N))
+    return cudaErrorInvalidValue;
   const int64_t tiles = (int64_t)G * ((M + BM - 1) / BM) * p.nt;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, G), s);
+  constexpr size_t kMaxSmem = 232448;          // 227 KB of dynamic shared memory per block
+  constexpr size_t kStaging = 4 * 2 * 4096;    // two 4 KB buffers per epilogue warp
+  // four ring stages unless the group tables of many experts leave no room for them
+  if (gemm_smem(1, 64, 4, G, kStaging) <= kMaxSmem)
+    return launch_epi<EPI_F32_TMA, 1, 64, 4>(ta, tb, to, p, grid,
+                                             gemm_smem(1, 64, 4, G, kStaging), s);
+  return launch_epi<EPI_F32_TMA, 1, 64, 3>(ta, tb, to, p, grid, gemm_smem(1, 64, 3, G, kStaging),
+                                           s);
 }
 
 // k-splits of the router product: enough (m-tile, split) pairs to cover the SMs, at most
