@@ -70,9 +70,12 @@ def file_sha(path):
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
 
-def load_traffic(workload):
-    """DRAM bytes per launch of the gate/up grouped GEMM from a committed ncu capture; null
-    once the kernel source has changed since the capture."""
+def load_traffic(workload, w):
+    """DRAM bytes per launch of the gate/up grouped GEMM from a committed ncu capture of the
+    full-size workload; null once the kernel source has changed since the capture, and for a
+    shape that differs from the captured one (--tokens / --ffn overrides)."""
+    if w != WORKLOADS.get(workload):
+        return None
     try:
         with open(TRAFFIC_FILE) as f:
             t = json.load(f)
@@ -208,6 +211,8 @@ def workload_of(args):
     w = WORKLOADS[args.workload]
     if args.tokens:
         w = scaled(w, T=args.tokens)
+    if getattr(args, "ffn", 0):
+        w = scaled(w, F=args.ffn, description=w.description + f" (expert width F={args.ffn})")
     return w
 
 
@@ -510,7 +515,7 @@ def run_cuda(args, rank, world, local):
         "kernel": "grouped_gemm_kernel<EPI_SWIGLU> (expert up: gate+up, SiLU*up epilogue)",
         "achieved": round(achieved, 1), "peak": tc_peak, "unit": "TFLOP/s",
         "frac": round(achieved / tc_peak, 3),
-        "traffic": load_traffic(args.workload),
+        "traffic": load_traffic(args.workload, w),
         "peak_source": f"{peaks_kind} {tc_key} (MEASURED_PEAKS.json)",
         "flops_per_launch": up_flops,
         "grouped_gemm_up_down_tflops": round(gemm_tflops, 1),
@@ -667,6 +672,8 @@ def main():
     ap.add_argument("--workload", default="mixtral", choices=["mixtral", "switch", "v3", "ec"])
     ap.add_argument("--tokens", type=int, default=0,
                     help="override the batch size T (smaller cases for profiling)")
+    ap.add_argument("--ffn", type=int, default=0,
+                    help="override the expert width F (smaller cases for profiling)")
     ap.add_argument("--impl", default="cuda", choices=["cuda", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-graph", action="store_true",

@@ -82,3 +82,13 @@ def test_reference_arm_prints_the_contract_line(monkeypatch, capsys):
     assert r["cpu_baseline"]["cores"] >= 1 and r["cpu_baseline"]["sample"]
     assert r["e2e"] == {"value": r["value"], "unit": "tokens/s", "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
+
+
+def test_traffic_is_null_for_shapes_other_than_the_captured_one():
+    import argparse
+    from sparse_mixture_experts_warp_b200.workloads import WORKLOADS
+    full = bench.workload_of(argparse.Namespace(workload="mixtral", tokens=0, ffn=0))
+    assert full == WORKLOADS["mixtral"]
+    for tokens, ffn in ((1024, 0), (0, 3584)):
+        w = bench.workload_of(argparse.Namespace(workload="mixtral", tokens=tokens, ffn=ffn))
+        assert w != full and bench.load_traffic("mixtral", w) is None
