@@ -24,9 +24,9 @@
 //                 and B [N, Ktot] and writes its own [M, N] block), without it k-splits of one
 //                 group write fp32 partials (the router product);
 //   EPI_F32_TMA:  EPI_F32 with groups along K, written through shared memory: each epilogue
-//                 warp stages a 32 x 32 fp32 block (128-byte swizzle, two buffers per warp) and
-//                 one lane stores it with a 3-D TMA store (columns, rows, group) that clips at
-//                 the group's bounds.  A weight-gradient tile has a short main loop (one
+//                 warp stages 32 x 16 fp32 blocks (64-byte swizzle, two 2 KB buffers per warp)
+//                 and one lane stores each with a 3-D TMA store (columns, rows, group) that
+//                 clips at the group's bounds.  A weight-gradient tile has a short main loop (one
 //                 expert's rows) and 128 KB of fp32 output; per-thread row stores would touch 32
 //                 rows per instruction and hold the tensor pipe back.
 //   An optional second output (out2) receives the raw accumulators of the SwiGLU / activation
@@ -417,7 +417,7 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
 //             L2->SMEM bytes per FLOP), 3-stage ring of 64 KB, one 512-column accumulator set,
 //             8 epilogue warps; a tile with <= 128 live rows loads and multiplies one half only.
 // tmB1 is the second B operand (SwiGLU, EPI_RAW, EPI_NONE_BMN) or, for EPI_F32_TMA, the fp32
-// output map: [groups][rows][N], boxes of 32 columns x 32 rows, 128-byte swizzle.
+// output map: [groups][rows][N], boxes of 16 columns x 32 rows, 64-byte swizzle.
 template <int EPI, int HALVES, int KB, int NSTAGES>
 __global__ void __launch_bounds__(64 + 128 * HALVES, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
@@ -431,8 +431,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   constexpr int NBUF = HALVES == 1 ? 2 : 1;          // TMEM accumulator buffers
   constexpr int BUF_COLS = HALVES * ACC_COLS;        // columns per buffer
   constexpr int N_EPI = 4 * HALVES;                  // epilogue warps
-  // EPI_F32_TMA: two 4 KB staging buffers (32 rows x 32 fp32) per epilogue warp
-  constexpr int STG_BYTES = EPI == EPI_F32_TMA ? N_EPI * 2 * 4096 : 0;
+  // EPI_F32_TMA: two 2 KB staging buffers (32 rows x 16 fp32) per epilogue warp
+  constexpr int STG_BYTES = EPI == EPI_F32_TMA ? N_EPI * 2 * 2048 : 0;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
@@ -655,7 +655,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int q = warp & 3;                  // TMEM lane quarter this warp may access
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
     int g = 0, it = 0;
-    uint32_t nstored = 0;                    // EPI_F32_TMA: staged chunks this warp has stored
+    uint32_t nstored = 0;                    // EPI_F32_TMA: staged blocks this warp has stored
     for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
       const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
       const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
@@ -765,27 +765,34 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           const int col = n_idx * p.n_out_tile + c;
           if (staged) {
             if (col >= p.N) continue;        // warp-uniform: the chunk lies past the last column
-            // buffer (nstored & 1) of this warp; the store that used it two chunks ago must
-            // have finished reading it
-            const uint32_t buf = sStg + (uint32_t)((((warp - 2) << 1) | (nstored & 1)) << 12);
-            if (lane == 0) bulk_wait_read<1>();
-            __syncwarp();
-            // row `lane`, 16-byte chunk i at chunk position i ^ (lane % 8): the 128-byte swizzle
-            // the tensor map names (conflict-free: 8 lanes of a phase hit 8 different chunks)
+            // two 16-column halves, each staged in buffer (nstored & 1) of this warp (2 KB: 32
+            // rows of 64 B) and written by one TMA store; the store that used the buffer two
+            // halves ago must have finished reading it
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint32_t a = buf + (uint32_t)(lane << 7) + (uint32_t)((i ^ (lane & 7)) << 4);
-              asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(v[4 * i]),
-                           "r"(v[4 * i + 1]), "r"(v[4 * i + 2]), "r"(v[4 * i + 3])
-                           : "memory");
+            for (int h = 0; h < 2; ++h) {
+              const uint32_t buf = sStg + (uint32_t)((((warp - 2) << 1) | (nstored & 1)) << 11);
+              if (lane == 0) bulk_wait_read<1>();
+              __syncwarp();
+              // row `lane`, 16-byte chunk i at chunk position i ^ ((lane / 2) % 4): the 64-byte
+              // swizzle the tensor map names (conflict-free: a phase of 8 lanes covers the 8
+              // distinct 16-byte bank groups)
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const uint32_t a =
+                    buf + (uint32_t)(lane << 6) + (uint32_t)((i ^ ((lane >> 1) & 3)) << 4);
+                asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(a),
+                             "r"(v[16 * h + 4 * i]), "r"(v[16 * h + 4 * i + 1]),
+                             "r"(v[16 * h + 4 * i + 2]), "r"(v[16 * h + 4 * i + 3])
+                             : "memory");
+              }
+              fence_proxy_async_smem();
+              __syncwarp();
+              if (lane == 0) {
+                tma_store_3d(&tmB1, buf, col + 16 * h, m_idx * TBM + half * BM + 32 * q, tl.g);
+                bulk_commit();
+              }
+              ++nstored;
             }
-            fence_proxy_async_smem();
-            __syncwarp();
-            if (lane == 0) {
-              tma_store_3d(&tmB1, buf, col, m_idx * TBM + half * BM + 32 * q, tl.g);
-              bulk_commit();
-            }
-            ++nstored;
           } else if (valid && col < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
 #pragma unroll
@@ -1199,17 +1206,17 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
-// 3D fp32 tensor [groups][rows][cols] (dense); box = 32 columns x 32 rows x 1 group, 128-byte
-// swizzle (one 128-byte row of the box per swizzle row): the EPI_F32_TMA output.
+// 3D fp32 tensor [groups][rows][cols] (dense); box = 16 columns x 32 rows x 1 group, 64-byte
+// swizzle (one 64-byte row of the box per swizzle row): the EPI_F32_TMA output.
 bool make_map_f32_out(CUtensorMap* m, void* ptr, uint64_t groups, uint64_t rows, uint64_t cols) {
   EncodeTiledFn enc = encode_fn();
   if (!enc) return false;
   const cuuint64_t dims[3] = {cols, rows, groups};
   const cuuint64_t strides[2] = {cols * 4, rows * cols * 4};
-  const cuuint32_t box[3] = {32, 32, 1};
+  const cuuint32_t box[3] = {16, 32, 1};
   const cuuint32_t estr[3] = {1, 1, 1};
   return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, ptr, dims, strides, box, estr,
-             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
              CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
@@ -1459,13 +1466,37 @@ cudaError_t launch_grouped_gemm_bf16_bmn(const void* A, int64_t a_rows, int K, c
                                             s);
 }
 
+// Weight-gradient tile shape.  Default: 256-row tiles (two M=128 MMAs share each B stage, so a
+// k-block moves 64 B of operands per MMA clock instead of 96; one accumulator set, the epilogue
+// is not overlapped).  MOE_WGRAD_TILE=128 selects 128-row tiles with two TMEM accumulators (the
+// epilogue overlaps the next tile; tested, kept for comparison measurements).
+bool wgrad_tile_128() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_WGRAD_TILE");
+    return e && !strcmp(e, "128");
+  }();
+  return v;
+}
+
 cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B, int N, int G,
                                             const int32_t* kgroup, int64_t k_total, float* out,
                                             cudaStream_t s) {
   if (M <= 0 || N <= 0 || G <= 0) return cudaSuccess;
-  alignas(64) CUtensorMap ta, tb;
-  if (!make_map(&ta, A, (uint64_t)M, (uint64_t)k_total, 128, 64)) return cudaErrorInvalidValue;
-  if (!make_map(&tb, B, (uint64_t)N, (uint64_t)k_total, 128, 64)) return cudaErrorInvalidValue;
+  // The output needs 16-byte aligned rows: N a multiple of 4.
+  if (N % 4 || (reinterpret_cast<uintptr_t>(out) & 15)) return cudaErrorInvalidValue;
+  constexpr size_t kMaxSmem = 232448;          // 227 KB of dynamic shared memory per block
+  const bool t128 = wgrad_tile_128();
+  const int halves = t128 ? 1 : 2;
+  const size_t staging = (size_t)4 * halves * 2 * 2048;   // two 2 KB buffers per epilogue warp
+  // 64-element k-blocks unless the group tables of many experts leave no room for the ring;
+  // then 32-element k-blocks (64-byte swizzle) in a deeper ring of smaller stages
+  const bool k32 = !t128 && gemm_smem(2, 64, 3, G, staging) > kMaxSmem;
+  const int kb = k32 ? 32 : 64;
+  alignas(64) CUtensorMap ta, tb, to;
+  if (!make_map(&ta, A, (uint64_t)M, (uint64_t)k_total, 128, kb)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, B, (uint64_t)N, (uint64_t)k_total, 128, kb)) return cudaErrorInvalidValue;
+  if (!make_map_f32_out(&to, out, (uint64_t)G, (uint64_t)M, (uint64_t)N))
+    return cudaErrorInvalidValue;
   GemmParams p;
   p.offsets = nullptr;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
@@ -1487,22 +1518,20 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   p.ldo2 = 0;
   p.kb_split = 0;
   p.bk_group = 0;
-  // 128-row tiles: two TMEM accumulators, so the fp32 epilogue of one tile (128 KB, written by
-  // TMA stores from shared memory) overlaps the next tile's main loop, which is short here (one
-  // expert's rows).  The output needs 16-byte aligned rows: N a multiple of 4.
-  if (N % 4 || (reinterpret_cast<uintptr_t>(out) & 15)) return cudaErrorInvalidValue;
-  alignas(64) CUtensorMap to;
-  if (!make_map_f32_out(&to, out, (uint64_t)G, (uint64_t)M, (uint64_t)N))
-    return cudaErrorInvalidValue;
-  const int64_t tiles = (int64_t)G * ((M + BM - 1) / BM) * p.nt;
+  const int tbm = BM * halves;
+  const int64_t tiles = (int64_t)G * ((M + tbm - 1) / tbm) * p.nt;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
-  constexpr size_t kMaxSmem = 232448;          // 227 KB of dynamic shared memory per block
-  constexpr size_t kStaging = 4 * 2 * 4096;    // two 4 KB buffers per epilogue warp
-  // four ring stages unless the group tables of many experts leave no room for them
-  if (gemm_smem(1, 64, 4, G, kStaging) <= kMaxSmem)
-    return launch_epi<EPI_F32_TMA, 1, 64, 4>(ta, tb, to, p, grid,
-                                             gemm_smem(1, 64, 4, G, kStaging), s);
-  return launch_epi<EPI_F32_TMA, 1, 64, 3>(ta, tb, to, p, grid, gemm_smem(1, 64, 3, G, kStaging),
+  if (t128) {
+    if (gemm_smem(1, 64, 4, G, staging) <= kMaxSmem)
+      return launch_epi<EPI_F32_TMA, 1, 64, 4>(ta, tb, to, p, grid,
+                                               gemm_smem(1, 64, 4, G, staging), s);
+    return launch_epi<EPI_F32_TMA, 1, 64, 3>(ta, tb, to, p, grid,
+                                             gemm_smem(1, 64, 3, G, staging), s);
+  }
+  if (!k32)
+    return launch_epi<EPI_F32_TMA, 2, 64, 3>(ta, tb, to, p, grid,
+                                             gemm_smem(2, 64, 3, G, staging), s);
+  return launch_epi<EPI_F32_TMA, 2, 32, 5>(ta, tb, to, p, grid, gemm_smem(2, 32, 5, G, staging),
                                            s);
 }
 

@@ -137,3 +137,17 @@ def test_backward_with_transposed_weight_copies_in_subprocess():
                         "-k", "matches_oracle and not mixtral_width"],
                        env=env, capture_output=True, text=True, timeout=600)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+def test_backward_with_128_row_weight_gradient_tiles_in_subprocess():
+    """MOE_WGRAD_TILE=128 runs the weight-gradient products on 128-row tiles with two TMEM
+    accumulators instead of the default 256-row tiles; run this file's parity cases under it
+    (the E = 256 case takes 64-element k-blocks there, 32-element ones by default)."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_WGRAD_TILE="128")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__,
+                        "-k", "matches_oracle and not mixtral_width"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
