@@ -139,7 +139,8 @@ moe_status_t moe_rows_max(const moe_desc_t* desc, int64_t* rows);
 /* C, the slots per expert under MOE_CAPACITY_DROP (0 otherwise). */
 moe_status_t moe_capacity(const moe_desc_t* desc, int32_t* capacity);
 
-/* Bytes of scratch that moe_route, moe_permute and moe_balance_stats need. */
+/* Bytes of scratch that moe_route, moe_permute and moe_balance_stats need, and the routed
+ * experts' k-split partials of moe_expert_up_ws / moe_expert_down_ws (a few executed rows). */
 moe_status_t moe_scratch_size(const moe_desc_t* desc, size_t* bytes);
 
 /* Bytes of workspace moe_layer_forward needs (every intermediate plus scratch). */
@@ -215,6 +216,27 @@ moe_status_t moe_expert_ffn(const moe_desc_t* desc, int32_t n_groups, int32_t F,
                             const void* a, int64_t a_rows, const int32_t* offsets,
                             const void* W_gate, const void* W_up, const void* W_down,
                             void* h, void* y, moe_stream_t stream);
+
+/* moe_expert_up / moe_expert_down with a scratch area for the small-batch (decode) schedule
+ * ("别只比较 Top-k" expert-work account: a small decode batch leaves each expert's products
+ * with very few rows, so they stream the weights).  Same arguments and results (up to fp32
+ * summation order), plus scratch (device, 16-byte aligned, scratch_bytes long; may be NULL with
+ * scratch_bytes = 0).  bf16 only: when the fused grouped product would keep fewer than 80% of
+ * the SMs busy (a_rows <= 256 for the down product, <= 16 for the up product; active groups
+ * bounded by min(n_groups, a_rows)), the product is split along K into 2..8 parts whose fp32
+ * partials [S][a_rows][N] go to scratch and are summed in a fixed order (deterministic) before
+ * the activation and the bf16 rounding.  When scratch is too small for the partials, or
+ * MOE_DECODE_SPLITK=0 is set in the environment, the fused product runs.  moe_scratch_size
+ * covers the routed experts' partials; moe_layer_forward uses this schedule for the routed and
+ * the shared experts. */
+moe_status_t moe_expert_up_ws(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                              const void* a, int64_t a_rows, const int32_t* offsets,
+                              const void* W_gate, const void* W_up, void* h, void* scratch,
+                              size_t scratch_bytes, moe_stream_t stream);
+moe_status_t moe_expert_down_ws(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                                const void* h, int64_t a_rows, const int32_t* offsets,
+                                const void* W_down, void* y, void* scratch, size_t scratch_bytes,
+                                moe_stream_t stream);
 
 /* Merge: out[t] = sum_j gates[t,j] * y[inv[t,j]] + sum_s y_shared[s,t], fp32 accumulation in
  * slot order, no atomics; inv = -1 contributes 0.  "Top-k 路由" Combine; Tiny MoE section 6.

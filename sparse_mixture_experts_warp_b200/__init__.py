@@ -5,7 +5,8 @@ PyTorch supplies device memory and the stream.  There is no fallback: if the lib
 missing, every call raises.
 
 The functions keep the C names (moe_route, moe_permute, moe_expert_up, moe_expert_down,
-moe_expert_ffn, moe_combine, moe_balance_stats, moe_layer_forward) and take torch tensors.
+moe_expert_ffn, moe_expert_up_ws, moe_expert_down_ws, moe_combine, moe_balance_stats,
+moe_layer_forward) and take torch tensors.
 """
 
 from __future__ import annotations
@@ -20,7 +21,8 @@ __all__ = [
     "MoeDesc", "MoeStats", "MoeLayerViews", "MoeError", "lib", "library_path", "desc_of",
     "header_functions", "status_string", "rows_max", "capacity", "scratch_size",
     "workspace_size", "layer_views", "moe_route", "moe_permute", "moe_expert_up",
-    "moe_expert_down", "moe_expert_ffn", "moe_permute_noalloc", "moe_combine", "moe_balance_stats",
+    "moe_expert_down", "moe_expert_ffn", "moe_expert_up_ws", "moe_expert_down_ws",
+    "moe_permute_noalloc", "moe_combine", "moe_balance_stats",
     "moe_layer_forward", "get_device_error", "empty_scratch", "empty_workspace",
 ]
 
@@ -94,6 +96,9 @@ _SIGS = {
     "moe_expert_up": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_down": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_expert_up_ws": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P],
+                         ctypes.c_int),
+    "moe_expert_down_ws": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
     "moe_combine": ([_DP, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_balance_stats": ([_DP, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_layer_forward": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P],
@@ -305,6 +310,19 @@ def moe_expert_ffn(d, n_groups, F, a, offsets, W_gate, W_up, W_down, h, y, strea
     _check("moe_expert_ffn", lib().moe_expert_ffn(
         ctypes.byref(d), n_groups, F, _ptr(a), a.shape[0], _ptr(offsets), _ptr(W_gate),
         _ptr(W_up), _ptr(W_down), _ptr(h), _ptr(y), _stream(stream)))
+
+
+def moe_expert_up_ws(d, n_groups, F, a, offsets, W_gate, W_up, h, scratch, stream=None):
+    _check("moe_expert_up_ws", lib().moe_expert_up_ws(
+        ctypes.byref(d), n_groups, F, _ptr(a), a.shape[0], _ptr(offsets), _ptr(W_gate),
+        _ptr(W_up), _ptr(h), _ptr(scratch), 0 if scratch is None else scratch.numel(),
+        _stream(stream)))
+
+
+def moe_expert_down_ws(d, n_groups, F, h, offsets, W_down, y, scratch, stream=None):
+    _check("moe_expert_down_ws", lib().moe_expert_down_ws(
+        ctypes.byref(d), n_groups, F, _ptr(h), h.shape[0], _ptr(offsets), _ptr(W_down), _ptr(y),
+        _ptr(scratch), 0 if scratch is None else scratch.numel(), _stream(stream)))
 
 
 def moe_combine(d, y, inv, gates, y_shared, out, stream=None):

@@ -70,6 +70,19 @@ enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI
                     EPI_RAW = 5 /* bf16 gate | up accumulators, SwiGLU operand staging */,
                     EPI_NONE_BMN = 6 /* EPI_NONE with an MN-major B operand */,
                     EPI_F32_TMA = 7 /* EPI_F32 written by TMA stores from shared memory */ };
+// k-split fp32 partials [ksplit][a_rows][N] of a grouped product (groups along M); the number
+// of non-empty splits is ceil(nkb / ceil(nkb / ksplit)) for nkb = ceil(K / 64).
+cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
+                                           int G, int N, const int32_t* offsets, int ksplit,
+                                           float* out, cudaStream_t s);
+int gemm_sm_count();
+int splitk_count(int K, int ksplit);   // non-empty splits of K (64-element k-blocks)
+// splitk.cu: the sums of k-split partials of the small-batch schedule (rows below *n_rows)
+cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S,
+                              int64_t rows, int F, const int32_t* n_rows, void* h,
+                              cudaStream_t s);
+cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N,
+                              const int32_t* n_rows, void* y, cudaStream_t s);
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,

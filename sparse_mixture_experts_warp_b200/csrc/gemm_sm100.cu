@@ -1535,6 +1535,54 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
                                            s);
 }
 
+// k-split fp32 partials of a grouped product with groups along M (the small-batch schedule,
+// when a handful of executed rows leaves most SMs without a tile): out[s][r][n] = the sum over
+// the k-blocks of split s of A[r, k] * B[g * N + n, k] for every row r of group g; split s
+// covers k-blocks [s * kchunk, (s + 1) * kchunk), every split non-empty.  out is
+// [ksplit][a_rows][N] fp32; only rows below offsets[G] are written.
+cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
+                                           int G, int N, const int32_t* offsets, int ksplit,
+                                           float* out, cudaStream_t s) {
+  if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb;
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb, B, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  GemmParams p;
+  p.offsets = offsets;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  p.rows = a_rows;
+  p.ldo = N;
+  p.G = G;
+  p.N = N;
+  p.K = K;
+  p.n_out_tile = 256;
+  p.nt = (N + 255) / 256;
+  p.fault = 0;
+  const int nkb = (K + 63) / 64;
+  p.kchunk = (nkb + ksplit - 1) / ksplit;
+  p.ksplit = splitk_count(K, ksplit);
+  p.split_stride = a_rows * (int64_t)N;
+  p.kgroup = nullptr;
+  p.out_gstride = 0;
+  p.out2 = nullptr;
+  p.ldo2 = 0;
+  p.kb_split = 0;
+  p.bk_group = 0;
+  const int64_t tiles = ((a_rows + BM - 1) / BM + G) * (int64_t)p.nt * p.ksplit;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, G), s);
+}
+
+int gemm_sm_count() { return sm_count(); }
+
+int splitk_count(int K, int ksplit) {
+  const int nkb = (K + 63) / 64;
+  if (nkb <= 0 || ksplit < 1) return 1;
+  const int kchunk = (nkb + ksplit - 1) / ksplit;
+  return (nkb + kchunk - 1) / kchunk;
+}
+
 // k-splits of the router product: enough (m-tile, split) pairs to cover the SMs, at most
 // kRouterMaxSplits, and every split non-empty (ks = ceil(nkb / ceil(nkb / ks))).
 int router_gemm_splits(int T, int D) {

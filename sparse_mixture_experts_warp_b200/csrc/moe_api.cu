@@ -107,9 +107,69 @@ size_t permute_scratch(const moe_desc_t* d) {
   if (d->select == MOE_EXPERT_CHOICE) return 0;
   return up((size_t)(permute_blocks(*d) > 0 ? permute_blocks(*d) : 1) * d->E * sizeof(int32_t));
 }
+// Small-batch (decode) schedule of the routed experts.  With few executed rows the grouped
+// GEMM has fewer tiles than SMs (one token of the Mixtral layer: 2 experts x 16 output tiles of
+// the down projection for 148 SMs), so the products are split along K into fp32 partials in
+// the step scratch (free once the permutation is done) and summed by splitk.cu.  At most
+// kMaxSplits splits; the up projection only for A <= kSplitUpRows, the down projection for
+// A <= kSplitDownRows.  MOE_DECODE_SPLITK=0 turns the schedule off (comparison measurements).
+constexpr int kMaxSplits = 8;
+constexpr int64_t kSplitUpRows = 16, kSplitDownRows = 256;
+
+bool decode_splitk_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_DECODE_SPLITK");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+size_t splitk_up_bytes(const moe_desc_t* d, int64_t A) {     // one partial set
+  return up((size_t)kMaxSplits * A * d->F * sizeof(float));
+}
+size_t splitk_scratch(const moe_desc_t* d) {
+  if (d->dtype != MOE_BF16) return 0;
+  const int64_t A = rows_of(d);
+  size_t b = 0;
+  if (A <= kSplitDownRows) b = up((size_t)kMaxSplits * A * d->D * sizeof(float));
+  if (A <= kSplitUpRows) {
+    const size_t u = (d->act == MOE_ACT_SWIGLU ? 2 : 1) * splitk_up_bytes(d, A);
+    if (u > b) b = u;
+  }
+  return b;
+}
+
 size_t scratch_bytes(const moe_desc_t* d) {
-  const size_t a = route_scratch(d), b = permute_scratch(d);
-  return (a > b ? a : b) + kAlign;
+  size_t a = route_scratch(d);
+  const size_t b = permute_scratch(d), c = splitk_scratch(d);
+  if (b > a) a = b;
+  if (c > a) a = c;
+  return a + kAlign;
+}
+
+// Fraction of the SM slots that a persistent launch of `units` equal work items keeps busy.
+double sm_fill(int64_t units, int sms) {
+  const int64_t waves = (units + sms - 1) / sms;
+  return waves > 0 ? (double)units / (double)(waves * sms) : 0.0;
+}
+
+// Split count for a product of `units` output tiles over K: 1 when the unsplit launch fills
+// at least 80% of the SM slots; otherwise the (effective) count in 2..kMaxSplits, each split
+// at least 4 k-blocks, that fills the most slots (fewer splits unless 2 points better).
+int choose_splits(int64_t units, int K, int sms) {
+  const int nkb = (K + 63) / 64;
+  double best_fill = sm_fill(units, sms);
+  if (units <= 0 || best_fill >= 0.8) return 1;
+  int best = 1;
+  for (int S = 2; S <= kMaxSplits && S * 4 <= nkb; ++S) {
+    const int se = splitk_count(K, S);
+    const double f = sm_fill(units * se, sms);
+    if (f > best_fill + 0.02) {
+      best_fill = f;
+      best = se;
+    }
+  }
+  return best;
 }
 
 // Workspace layout of moe_layer_forward; with base == nullptr only the size is computed.
@@ -343,6 +403,77 @@ moe_status_t moe_expert_ffn(const moe_desc_t* d, int32_t G, int32_t F, const voi
   return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
 }
 
+// ---- the small-batch (decode) schedule: k-split products, see kMaxSplits ----
+
+// Scratch of at least `need` bytes at a 256-byte boundary inside [scratch, +bytes), or null.
+static float* splitk_space(void* scratch, size_t bytes, size_t need) {
+  if (!scratch) return nullptr;
+  const uintptr_t b = reinterpret_cast<uintptr_t>(scratch);
+  const uintptr_t a = (b + kAlign - 1) & ~(uintptr_t)(kAlign - 1);
+  if (a - b > bytes || bytes - (a - b) < need) return nullptr;
+  return reinterpret_cast<float*>(a);
+}
+
+moe_status_t moe_expert_up_ws(const moe_desc_t* d, int32_t G, int32_t F, const void* a,
+                              int64_t a_rows, const int32_t* offsets, const void* W_gate,
+                              const void* W_up, void* h, void* scratch, size_t scratch_bytes,
+                              moe_stream_t stream) {
+  moe_status_t st = check_ffn(d, G, F, a, a_rows, offsets);
+  if (st != MOE_OK) return st;
+  const bool glu = d->act == MOE_ACT_SWIGLU;
+  int S = 1;
+  if (d->dtype == MOE_BF16 && decode_splitk_enabled() && a_rows > 0 && a_rows <= kSplitUpRows &&
+      h && W_up && is_aligned16(W_up) && is_aligned16(h) &&
+      (!glu || (W_gate && is_aligned16(W_gate)))) {
+    // fused: SwiGLU tiles hold 128 features (gate and up side by side), others 256 columns;
+    // split: gate and up are separate products of 256-column tiles
+    const int sms = gemm_sm_count();
+    const int64_t active = a_rows < G ? a_rows : G;
+    const int64_t fused = active * ((F + (glu ? 127 : 255)) / (glu ? 128 : 256));
+    const int64_t units = active * ((F + 255) / 256);
+    const double fill_fused = sm_fill(fused, sms);
+    const int c = choose_splits(units, d->D, sms);
+    if (c > 1 && fill_fused < 0.8 && sm_fill(units * c, sms) > fill_fused + 0.05) S = c;
+  }
+  const size_t one = (size_t)S * a_rows * F * sizeof(float);
+  const size_t step = up(one);
+  float* part = S > 1 ? splitk_space(scratch, scratch_bytes, (glu ? step : 0) + one) : nullptr;
+  if (!part)
+    return moe_expert_up(d, G, F, a, a_rows, offsets, W_gate, W_up, h, stream);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  float* pu = glu ? part + step / sizeof(float) : part;
+  cudaError_t e = cudaSuccess;
+  if (glu) e = launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_gate, G, F, offsets, S, part, s);
+  if (e == cudaSuccess)
+    e = launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_up, G, F, offsets, S, pu, s);
+  if (e == cudaSuccess)
+    e = launch_splitk_act(d->act, part, pu, S, a_rows, F, offsets + G, h, s);
+  return cuda_status(e);
+}
+
+moe_status_t moe_expert_down_ws(const moe_desc_t* d, int32_t G, int32_t F, const void* h,
+                                int64_t a_rows, const int32_t* offsets, const void* W_down,
+                                void* y, void* scratch, size_t scratch_bytes,
+                                moe_stream_t stream) {
+  moe_status_t st = check_ffn(d, G, F, h, a_rows, offsets);
+  if (st != MOE_OK) return st;
+  int S = 1;
+  if (d->dtype == MOE_BF16 && decode_splitk_enabled() && a_rows > 0 &&
+      a_rows <= kSplitDownRows && W_down && y && is_aligned16(W_down) && is_aligned16(y)) {
+    const int64_t active = a_rows < G ? a_rows : G;
+    S = choose_splits(active * ((d->D + 255) / 256), F, gemm_sm_count());
+  }
+  float* part = S > 1 ? splitk_space(scratch, scratch_bytes,
+                                     (size_t)S * a_rows * d->D * sizeof(float))
+                      : nullptr;
+  if (!part) return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  cudaError_t e = launch_grouped_gemm_f32_splitk(h, a_rows, F, W_down, G, d->D, offsets, S, part,
+                                                 s);
+  if (e == cudaSuccess) e = launch_splitk_sum(part, S, a_rows, d->D, offsets + G, y, s);
+  return cuda_status(e);
+}
+
 moe_status_t moe_combine(const moe_desc_t* d, const void* y, const int32_t* inv,
                          const float* gates, const void* y_shared, void* out,
                          moe_stream_t stream) {
@@ -411,8 +542,13 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
     if (e != cudaSuccess) return MOE_ERR_CUDA;
     st = moe_expert_down(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, stream);
   } else {
-    st = moe_expert_ffn(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, W_down, v.h,
-                        v.y, stream);
+    // the step scratch is free once the permutation is done: the small-batch schedule's
+    // partials go there
+    st = moe_expert_up_ws(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, v.h,
+                          v.scratch, v.scratch_bytes, stream);
+    if (st == MOE_OK)
+      st = moe_expert_down_ws(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
+                              v.scratch_bytes, stream);
   }
   if (st != MOE_OK) return st;
   if (d->n_shared > 0) {
@@ -429,8 +565,11 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
       const uint8_t* uw = static_cast<const uint8_t*>(Ws_up) + i * wstride_up;
       const uint8_t* dw = static_cast<const uint8_t*>(Ws_down) + i * wstride_up;
       uint8_t* ys = static_cast<uint8_t*>(v.y_shared) + (int64_t)i * d->T * d->D * es;
-      st = moe_expert_ffn(&ds, 1, d->F_shared, x, d->T, v.shared_offsets, gw, uw, dw, v.h_shared,
-                          ys, stream);
+      st = moe_expert_up_ws(&ds, 1, d->F_shared, x, d->T, v.shared_offsets, gw, uw, v.h_shared,
+                            v.scratch, v.scratch_bytes, stream);
+      if (st == MOE_OK)
+        st = moe_expert_down_ws(&ds, 1, d->F_shared, v.h_shared, d->T, v.shared_offsets, dw, ys,
+                                v.scratch, v.scratch_bytes, stream);
       if (st != MOE_OK) return st;
     }
   }

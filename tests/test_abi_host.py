@@ -99,9 +99,36 @@ def test_null_pointers_rejected_before_launch():
     st = L.moe_expert_ffn(ctypes.byref(d), 8, 14336, None, 8192, None, None, None, None, None,
                           None, None)
     assert st == 1
+    st = L.moe_expert_up_ws(ctypes.byref(d), 8, 14336, None, 8192, None, None, None, None,
+                            None, 0, None)
+    assert st == 1
+    st = L.moe_expert_down_ws(ctypes.byref(d), 8, 14336, None, 8192, None, None, None, None, 0,
+                              None)
+    assert st == 1
     # misaligned pointers are refused too
     st = L.moe_combine(ctypes.byref(d), 0x1001, 0x2000, 0x3000, None, 0x4000, None)
     assert st == 1
+
+
+def test_scratch_holds_the_small_batch_partials():
+    # the routed experts' k-split partials (at most 8 splits, fp32) fit in moe_scratch_size
+    # whenever the schedule may run: A <= 256 for the down product, A <= 16 for the up product
+    # (gate and up partial sets for SwiGLU, each rounded to 256 bytes), plus the alignment slack
+    from sparse_mixture_experts_warp_b200.workloads import scaled
+    for T in (1, 2, 8, 64, 128):
+        w = scaled(WORKLOADS["mixtral"], T=T)
+        d = M.desc_of(w)
+        A = rows_max(w)
+        need = 0
+        if A <= 256:
+            need = 8 * A * w.D * 4
+        if A <= 16:
+            one = -(-8 * A * w.F * 4 // 256) * 256
+            need = max(need, 2 * one)
+        assert M.scratch_size(d) >= need + 256, T
+    # large batches do not pay for it
+    big = M.desc_of(WORKLOADS["mixtral"])
+    assert M.scratch_size(big) < 8 * 2 * 4096 * 4
 
 
 def test_workspace_too_small_or_misaligned():

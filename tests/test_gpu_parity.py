@@ -143,6 +143,41 @@ def test_decode_regime_mixtral_shape(T):
     C.check_sampled_output(w, inp, out, v, list(range(T)))
 
 
+# A few executed rows (bf16) take the k-split expert schedule: fp32 partials of the up and down
+# products summed by splitk.cu.  ReLU at the full Switch layer with its capacity limit (up split
+# 3, down split 8) and GELU (splits 4 and 2); SwiGLU is covered by fast_router_T1 (up split 7)
+# and T = 1 above (up 5, down 4).  Every token against the oracle, which evaluates only the
+# experts in use.
+DECODE = {
+    "switch_relu_T2": scaled(W["switch"], T=2),
+    "gelu_T3": scaled(W["switch"], act="gelu", T=3, D=1024, E=16, F=512, overflow="dropless",
+                      gate="renorm", k=2, zipf_s=0.0),
+}
+
+
+@pytest.mark.parametrize("name", list(DECODE))
+def test_decode_split_schedule(name):
+    w = DECODE[name]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    C.check_logits(w, inp, v)
+    C.check_routing(w, inp, v)
+    C.check_sampled_output(w, inp, out, v, list(range(w.T)))
+
+
+def test_decode_split_schedule_matches_fused_path_in_subprocess():
+    """MOE_DECODE_SPLITK=0 keeps the fused grouped GEMMs at every size; the decode cases pass
+    there too."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_DECODE_SPLITK="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "decode_split_schedule and not subprocess or decode_regime and 1]"],
+                       env=env, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
 # The bf16 fast router at larger token counts: each CTA routes several 16-token batches, the
 # last one ragged (T=5000, D=4096: 34 tokens per CTA; T=9000, D=1024: 61; T=12000, D=4096:
 # 82).  Logits of every token, the whole routing, permutation and statistics are compared

@@ -1,0 +1,95 @@
+"""moe_expert_up_ws / moe_expert_down_ws: the small-batch (decode) schedule of the expert
+products.  With a few executed rows the products are split along K into fp32 partials in the
+scratch and summed in a fixed order before the activation; the result equals the fused grouped
+GEMM up to fp32 summation order (both round the same fp32 value to bf16 once), the split path
+really runs (kernel launch count), and without scratch the fused product runs (bit-identical).
+Layer-level parity of the schedule against the oracle is in test_gpu_parity.py (decode cases).
+"""
+
+import pytest
+import torch
+
+import sparse_mixture_experts_warp_b200 as M
+from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, scaled
+import moe_check as C
+
+pytestmark = pytest.mark.gpu
+
+# bf16 ulp is 2^-8 relative; two roundings of values that differ only in fp32 summation order
+TOL = 2.0 ** -7
+
+CASES = {
+    # one token of a SwiGLU layer: up split 4 (gate and up), down split 8
+    "swiglu_T1": scaled(WORKLOADS["mixtral"], T=1, D=1024, F=2048),
+    # ReLU, two tokens over 16 experts: up split, down split
+    "relu_T2": scaled(WORKLOADS["switch"], T=2, D=1024, E=16, F=1024, zipf_s=0.0),
+    # GELU
+    "gelu_T3": scaled(WORKLOADS["switch"], act="gelu", T=3, D=1024, E=16, F=512,
+                      overflow="dropless", gate="renorm", k=2, zipf_s=0.0),
+}
+
+
+def _rel(a, b):
+    den = b.abs().max().item()
+    return (a - b).abs().max().item() / den if den > 0 else (a - b).abs().max().item()
+
+
+@pytest.mark.parametrize("name", list(CASES))
+def test_ws_products_match_fused_products(name):
+    w = CASES[name]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    n = int(v["offsets"][w.E].item())              # executed rows
+    assert n > 0
+    scratch = v["scratch"]
+    h0 = torch.zeros_like(v["h"])
+    h1 = torch.zeros_like(v["h"])
+    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
+    k0 = M.kernel_launches()
+    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1, scratch)
+    up_launches = M.kernel_launches() - k0
+    y0 = torch.zeros_like(v["y"])
+    y1 = torch.zeros_like(v["y"])
+    M.moe_expert_down(d, w.E, w.F, h0, v["offsets"], inp.W_down, y0)
+    k0 = M.kernel_launches()
+    M.moe_expert_down_ws(d, w.E, w.F, h0, v["offsets"], inp.W_down, y1, scratch)
+    down_launches = M.kernel_launches() - k0
+    torch.cuda.synchronize()
+    assert M.get_device_error() == 0
+    # split products (gate and up for SwiGLU) plus the summing pass
+    assert up_launches == (3 if w.act == "swiglu" else 2)
+    assert down_launches == 2
+    assert _rel(h1[:n].float(), h0[:n].float()) <= TOL
+    assert _rel(y1[:n].float(), y0[:n].float()) <= TOL
+
+
+def test_ws_without_scratch_runs_the_fused_products():
+    w = CASES["swiglu_T1"]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    h0, h1 = torch.zeros_like(v["h"]), torch.zeros_like(v["h"])
+    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
+    k0 = M.kernel_launches()
+    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1, None)
+    assert M.kernel_launches() - k0 == 1
+    y0, y1 = torch.zeros_like(v["y"]), torch.zeros_like(v["y"])
+    M.moe_expert_down(d, w.E, w.F, h0, v["offsets"], inp.W_down, y0)
+    M.moe_expert_down_ws(d, w.E, w.F, h0, v["offsets"], inp.W_down, y1, None)
+    torch.cuda.synchronize()
+    assert torch.equal(h0, h1) and torch.equal(y0, y1)
+
+
+def test_ws_with_many_rows_runs_the_fused_products():
+    # 700 tokens x top-2: far more rows than the schedule's limits
+    w = scaled(WORKLOADS["mixtral"], T=700, D=512, F=1024)
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    h0, h1 = torch.zeros_like(v["h"]), torch.zeros_like(v["h"])
+    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
+    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1,
+                       v["scratch"])
+    torch.cuda.synchronize()
+    assert torch.equal(h0, h1)
