@@ -1,8 +1,9 @@
 /* A plain C caller of the library's C ABI (include/moe.h): no Python, no torch.
  * It fills the descriptor of the Mixtral-shaped layer ("Top-k 路由" gate Steps 1-3; Tiny MoE
  * sections 3-8: D = 4096, E = 8 SwiGLU experts of width 14336, softmax top-2 renormalised,
- * dropless) and exercises the host-side entry points that need no GPU: sizing, the Switch
- * capacity rule C = ceil(CF T k / E), and argument validation.  Exit status 0 when every
+ * dropless) and exercises the host-side entry points that need no GPU: sizing (including the
+ * scratch of the small-batch schedule), the Switch capacity rule C = ceil(CF T k / E), and
+ * argument validation.  Exit status 0 when every
  * check holds; prints one line per check. */
 #include <stdio.h>
 #include <string.h>
@@ -59,6 +60,16 @@ int main(void) {
           "fp32 backward unsupported");
     check(moe_layer_forward(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
                             NULL, 0, NULL) != MOE_OK, "null buffers refused");
+    check(moe_expert_up_ws(&d, 8, 14336, NULL, 8192, NULL, NULL, NULL, NULL, NULL, 0, NULL) ==
+              MOE_ERR_INVALID_ARG, "expert up (scratch form): null buffers refused");
+    check(moe_expert_down_ws(&d, 8, 14336, NULL, 8192, NULL, NULL, NULL, NULL, 0, NULL) ==
+              MOE_ERR_INVALID_ARG, "expert down (scratch form): null buffers refused");
+    /* one token: the scratch also holds the small-batch schedule's k-split partials */
+    moe_desc_t one = d;
+    one.T = 1;
+    size_t sc1 = 0;
+    check(moe_scratch_size(&one, &sc1) == MOE_OK && sc1 >= (size_t)8 * 2 * 4096 * 4,
+          "one-token scratch holds the down product's partials");
     check(strlen(moe_status_string(MOE_ERR_TIMEOUT)) > 0, "status strings");
     printf("library %s\n", moe_version());
     return failures == 0 ? 0 : 1;
