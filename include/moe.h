@@ -26,6 +26,10 @@
  *     with moe_get_device_error.
  *   - Limits: 1 <= E <= 256; token choice 1 <= k <= min(E, 32); expert choice 1 <= c <= T;
  *     T * max(k, E) < 2^31.  bf16: D, F and F_shared multiples of 64.  fp32: D multiple of 4.
+ *   - An empty batch (T = 0, token choice) is valid: moe_layer_forward, moe_route, moe_combine
+ *     and moe_balance_stats check their arguments and return MOE_OK without launching anything
+ *     or writing any output (views and statistics keep their previous contents); moe_permute
+ *     writes zero counts and offsets; the expert products have no rows to compute.
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H

@@ -171,3 +171,26 @@ def test_backward_validation_before_launch():
     st = L.moe_layer_forward_train(ctypes.byref(d), None, None, None, None, None, None, None,
                                    None, 0, None, 0, None)
     assert st == 3                     # MOE_ERR_WORKSPACE: no backward workspace
+
+
+def test_empty_batch_returns_before_any_launch():
+    # T = 0: argument checks only, no kernel is enqueued (the pointers are never dereferenced)
+    from sparse_mixture_experts_warp_b200.workloads import scaled
+    w = scaled(WORKLOADS["mixtral"], T=0)
+    d = M.desc_of(w)
+    assert M.rows_max(d) == 0
+    need = M.workspace_size(d)
+    L = M.lib()
+    n0 = L.moe_kernel_launches()
+    st = L.moe_layer_forward(ctypes.byref(d), 0x1000, 0x2000, None, 0x3000, 0x4000, 0x5000, None,
+                             None, None, 0x6000, 0x10000, need, None)
+    assert st == 0
+    st = L.moe_route(ctypes.byref(d), 0x1000, 0x2000, None, 0x3000, 0x4000, None, None, None,
+                     0x10000, M.scratch_size(d), None)
+    assert st == 0
+    st = L.moe_combine(ctypes.byref(d), 0x1000, 0x2000, 0x3000, None, 0x4000, None)
+    assert st == 0
+    assert L.moe_kernel_launches() == n0
+    # the workspace check still applies
+    assert L.moe_layer_forward(ctypes.byref(d), 0x1000, 0x2000, None, 0x3000, 0x4000, 0x5000,
+                               None, None, None, 0x6000, 0x10000, need - 1, None) == 3
