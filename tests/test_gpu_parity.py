@@ -46,6 +46,13 @@ SMALL = {
     "gelu_bf16": scaled(W["switch"], act="gelu", T=500, D=256, E=16, F=512, overflow="dropless",
                         gate="renorm", k=2, zipf_s=0.0),
     "gelu_f32": scaled(W["tiny"], act="gelu", T=40),
+    # degenerate and extreme shapes: one expert (the layer is the dense FFN, every gate 1), the
+    # largest top-k (k = 32 of 64 experts: tensor-core router, 32 arg-max rounds, the general
+    # combine), and the smallest bf16 widths (D = F = 64: one k-block, 64 live features in a
+    # 128-feature SwiGLU tile)
+    "single_expert_E1": scaled(W["mixtral"], T=100, D=256, E=1, k=1, F=256),
+    "max_k32": scaled(W["mixtral"], T=64, D=256, E=64, k=32, F=128),
+    "bf16_D64_F64": scaled(W["mixtral"], T=50, D=64, F=64),
     # more than 65536 assignments: the multi-block permute path
     "large_A": scaled(W["mixtral"], T=33000, D=128, F=128),
     # group-limited selection: fast router (groups of 2 experts, softmax; groups of 2, sigmoid
