@@ -375,7 +375,7 @@ def run_cuda(args, rank, world, local):
                       v["row_src"], v["inv"], scratch, stream_)
         if ev is not None:
             ev[2].record(stream_)
-        # (with a few executed rows the expert products take the k-split schedule, its
+        # (with a few executed rows the routed experts' products take the k-split schedule, its
         # partials in the step scratch, as in moe_layer_forward)
         M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
                            scratch, stream_)
@@ -384,10 +384,8 @@ def run_cuda(args, rank, world, local):
         M.moe_expert_down_ws(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], scratch,
                              stream_)
         for i in range(w.n_shared):
-            M.moe_expert_up_ws(d_sh, 1, w.F_shared, inp.x, sh_off, inp.Ws_gate[i], inp.Ws_up[i],
-                               h_sh, scratch, stream_)
-            M.moe_expert_down_ws(d_sh, 1, w.F_shared, h_sh, sh_off, inp.Ws_down[i],
-                                 v["y_shared"][i], scratch, stream_)
+            M.moe_expert_ffn(d_sh, 1, w.F_shared, inp.x, sh_off, inp.Ws_gate[i], inp.Ws_up[i],
+                             inp.Ws_down[i], h_sh, v["y_shared"][i], stream_)
         if ev is not None:
             ev[4].record(stream_)
         M.moe_combine(d, v["y"], v["inv"], v["gates"], v["y_shared"] if w.n_shared else None,

@@ -231,8 +231,8 @@ moe_status_t moe_expert_ffn(const moe_desc_t* desc, int32_t n_groups, int32_t F,
  * partials [S][a_rows][N] go to scratch and are summed in a fixed order (deterministic) before
  * the activation and the bf16 rounding.  When scratch is too small for the partials, or
  * MOE_DECODE_SPLITK=0 is set in the environment, the fused product runs.  moe_scratch_size
- * covers the routed experts' partials; moe_layer_forward uses this schedule for the routed and
- * the shared experts. */
+ * covers the routed experts' partials; moe_layer_forward uses this schedule for the routed
+ * experts (the shared experts keep the fused products). */
 moe_status_t moe_expert_up_ws(const moe_desc_t* desc, int32_t n_groups, int32_t F,
                               const void* a, int64_t a_rows, const int32_t* offsets,
                               const void* W_gate, const void* W_up, void* h, void* scratch,

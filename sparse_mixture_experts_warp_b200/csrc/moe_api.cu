@@ -565,11 +565,8 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
       const uint8_t* uw = static_cast<const uint8_t*>(Ws_up) + i * wstride_up;
       const uint8_t* dw = static_cast<const uint8_t*>(Ws_down) + i * wstride_up;
       uint8_t* ys = static_cast<uint8_t*>(v.y_shared) + (int64_t)i * d->T * d->D * es;
-      st = moe_expert_up_ws(&ds, 1, d->F_shared, x, d->T, v.shared_offsets, gw, uw, v.h_shared,
-                            v.scratch, v.scratch_bytes, stream);
-      if (st == MOE_OK)
-        st = moe_expert_down_ws(&ds, 1, d->F_shared, v.h_shared, d->T, v.shared_offsets, dw, ys,
-                                v.scratch, v.scratch_bytes, stream);
+      st = moe_expert_ffn(&ds, 1, d->F_shared, x, d->T, v.shared_offsets, gw, uw, dw, v.h_shared,
+                          ys, stream);
       if (st != MOE_OK) return st;
     }
   }
