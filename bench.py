@@ -1,6 +1,7 @@
 """Throughput of the sparse MoE FFN layer forward pass on B200 (one JSON line on rank 0).
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload mixtral] [--impl cuda|reference]
+                    [--tokens T] [--ffn F] [--no-graph] [--no-backward] [--no-cpu-baseline]
 
 A step is one pass of the whole layer -- route, permute, expert up (gate/up + SiLU*up),
 expert down, combine, balance statistics -- over one batch of synthetic tokens of the
@@ -16,6 +17,11 @@ slowest rank's time (weak scaling).
 
 `--impl reference` times the CPU oracle (fp64) on the host cores on bounded samples of the
 same workload: each step routes the whole batch and evaluates a sample of its tokens.
+
+After the forward, a training step (moe_layer_forward_train + moe_layer_backward) is timed
+too, reported under "backward" (`--no-backward` skips it).  `--tokens` and `--ffn` shrink the
+batch or the expert width for profiling cases and the small-batch (decode) regime; the DRAM
+traffic figure is then null (it is taken from an ncu capture of the full-size workload only).
 """
 
 from __future__ import annotations
