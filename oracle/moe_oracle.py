@@ -40,7 +40,10 @@ Readings where the pages are silent (each one is listed in the design notes):
 
 Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
 (worked examples of the pages, closed forms, brute force and reductions to
-dense/soft routing); none is "parity unpinned".
+dense/soft routing; the backward by central finite differences of the forward);
+none is "parity unpinned".  ``tests/test_oracle_mutations.py`` plants plausible
+mistakes in these functions, one at a time, and checks that a pin of the same
+stage catches each.
 """
 
 from __future__ import annotations
