@@ -70,6 +70,17 @@ int main(void) {
     size_t sc1 = 0;
     check(moe_scratch_size(&one, &sc1) == MOE_OK && sc1 >= (size_t)8 * 2 * 4096 * 4,
           "one-token scratch holds the down product's partials");
+    /* an empty batch: arguments checked, nothing launched, MOE_OK (the pointers below are
+     * never dereferenced; the workspace is carved on the host only) */
+    moe_desc_t none = d;
+    none.T = 0;
+    size_t ws0 = 0;
+    check(moe_workspace_size(&none, &ws0) == MOE_OK, "empty batch: workspace size");
+    const int64_t n0 = moe_kernel_launches();
+    void* fake = (void*)(uintptr_t)0x100000;
+    check(moe_layer_forward(&none, fake, fake, NULL, fake, fake, fake, NULL, NULL, NULL, fake,
+                            fake, ws0, NULL) == MOE_OK && moe_kernel_launches() == n0,
+          "empty batch: layer forward returns before any launch");
     check(strlen(moe_status_string(MOE_ERR_TIMEOUT)) > 0, "status strings");
     printf("library %s\n", moe_version());
     return failures == 0 ? 0 : 1;
