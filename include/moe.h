@@ -187,12 +187,17 @@ moe_status_t moe_permute(const moe_desc_t* desc, const int32_t* expert_ids, cons
  * host code that must not call cudaMalloc at that point).  The pages have no counterpart: this
  * is a property of the library, not of the method.
  *   Same arguments, outputs and results as moe_permute, minus scratch.  Its scratch is a fixed
- *   file-scope device array of MOE_PERMUTE_NOALLOC_MAX_INTS int32 (256 KiB) that every GPU
- *   loading the library holds until exit.  Token choice needs ceil(T*k/1024)*E of them; larger
- *   problems return MOE_ERR_UNSUPPORTED before anything is launched.  Allocates nothing (no
- *   cudaMalloc, cudaFree or allocating library call).
- *   The first call on a device looks up the array's device address (cudaGetSymbolAddress) with
- *   that device current and caches it: make that first call before any stream capture.
+ *   file-scope device array of MOE_PERMUTE_NOALLOC_MAX_INTS int32 (256 KiB), held until exit on
+ *   every GPU where the library's module is loaded.  Token choice needs ceil(T*k/1024)*E of
+ *   them; larger problems return MOE_ERR_UNSUPPORTED before any pointer is examined and before
+ *   anything is launched.  Allocates nothing (no cudaMalloc, cudaFree or allocating library
+ *   call).
+ *   The first call in each CUDA context looks up the array's device address
+ *   (cudaGetSymbolAddress) with that context current and caches it under the context's unique
+ *   id, so a device reset is followed by a fresh look-up: make that first call before any
+ *   stream capture.  Under lazy module loading that first call is also when the array is
+ *   committed to the GPU: make it before the caller reserves the GPU's memory (a GPU with no
+ *   room left gives MOE_ERR_CUDA).
  *   All calls share the array and each overwrites the last one's contents; calls whose work
  *   overlaps on the GPU (other streams, other threads) race on it -- serialise them. */
 #define MOE_PERMUTE_NOALLOC_MAX_INTS 65536

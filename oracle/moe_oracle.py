@@ -501,7 +501,9 @@ def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
     earlier tokens); only the sampled tokens' expert rows are evaluated.
     `weights_of(e)` (optional) returns (W_gate[e], W_up[e], W_down[e]) as fp64
     arrays, so that a caller can stream expert weights from device memory one
-    expert at a time.
+    expert at a time.  Besides out_rows, the result holds each evaluated
+    assignment's expert output before its gate (y_assign[(t, j)]) and each
+    shared expert's output on the sampled tokens (shared_rows[i]).
     """
     g = _get(w)
     x = _np(x)
@@ -523,6 +525,7 @@ def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
             return (Wgt[e] if Wgt is not None else None), Wu[e], Wd[e]
     out = {t: np.zeros(g["D"], dtype=np.float64) for t in tokens}
     gates = np.asarray(r["gates"], dtype=np.float64).reshape(g["T"], K)
+    y_assign = {}
     for e in sorted(need):
         wg_e, wu_e, wd_e = weights_of(e)
         ts = [t for t, _ in need[e]]
@@ -534,14 +537,17 @@ def layer_forward_rows(w, tokens, x, Wg, bias, W_gate, W_up, W_down,
             ye = relu_expert(x[ts], wu_e, wd_e)
         for i, (t, j) in enumerate(need[e]):
             out[t] += gates[t, j] * ye[i]
+            y_assign[(t, j)] = ye[i]
+    shared_rows = []
     if g["n_shared"]:
         Sg, Su, Sd = _np(Ws_gate), _np(Ws_up), _np(Ws_down)
         for i in range(g["n_shared"]):
             ys = swiglu_expert(x[tokens], Sg[i], Su[i], Sd[i])
+            shared_rows.append(ys)
             for n, t in enumerate(tokens):
                 out[t] += ys[n]
     r.update(logits=s, out_rows=np.stack([out[t] for t in tokens]) if tokens else
-             np.zeros((0, g["D"])))
+             np.zeros((0, g["D"])), y_assign=y_assign, shared_rows=shared_rows)
     return r
 
 

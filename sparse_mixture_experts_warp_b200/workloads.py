@@ -199,6 +199,15 @@ def make_inputs(w: Workload, seed: int = 0, device="cpu", experts: bool = True,
     return inp
 
 
+def separate_keys(w: Workload, inp: Inputs, seed: int, key_fn, key_gap: float = 0.0,
+                  ec_gap: float = 0.0, max_rounds: int = 64) -> Inputs:
+    """The key-separation step of make_inputs on inputs a caller has already edited (for
+    example router rows made equal on purpose, whose tied keys key_fn leaves out)."""
+    if key_fn is not None and (key_gap > 0 or ec_gap > 0):
+        _separate_keys(w, inp, seed, key_fn, key_gap, ec_gap, max_rounds)
+    return inp
+
+
 def _redraw(w, inp, rows, seed, rnd):
     """Redraw x rows `rows` (sorted) from sub-seed (seed, round)."""
     device = inp.x.device

@@ -4,8 +4,10 @@ the CPU oracle on the same seeded inputs.
 Tolerances (from the layer's arithmetic):
   * routing (expert ids, counts, offsets, row order, inverse permutation, dropped sets) is
     compared bit-exactly, the oracle routing from the GPU's own fp32 logits;
-  * router logits: per token max_e |gpu - oracle| / max_e |oracle| <= 1e-5 (fp32 accumulation
-    of exact bf16/fp32 products over D terms);
+  * router logits: for every token t and expert e, |gpu - oracle| / sum_d |x[t,d] Wg[e,d]|
+    <= 1e-5.  The denominator is the condition number of the fp32 dot product: its rounding
+    error is bounded relative to the sum of the magnitudes of its terms, so the bound holds per
+    logit whatever the logit's own size (a logit near zero, or E = 1);
   * gates / probabilities: relative 1e-5 (fp32 exp and division);
   * layer output: max |gpu - oracle| / max |oracle| over the compared rows <= 2e-2 for bf16
     operands (bf16 rounding of h, y and out, each 2^-9 relative), <= 1e-5 for fp32; rows the
@@ -72,20 +74,29 @@ def max_rel(a, b):
     return float(np.max(np.abs(a - b)) / den)
 
 
+def logit_condition(x, Wg):
+    """cond[t, e] = sum_d |x[t, d] * Wg[e, d]|, the scale of one fp32 dot product's rounding
+    error (each of its D products and partial sums is rounded relative to this sum)."""
+    return np.abs(x) @ np.abs(Wg).T
+
+
 def check_logits(w, inp, v, rows=None):
-    """GPU fp32 logits against the oracle's fp64 router product (optionally sampled rows):
-    max |gpu - oracle| / max |oracle| over the whole (sampled) logits tensor, the reading of
-    "max relative error" every other check here uses.  (Normalising each row by its own
-    largest logit is ill-conditioned when a row holds one or a few small logits: with E = 1 it
-    divides one fp32 dot product by itself, whose rounding error is bounded relative to
-    sum_i |x_i w_i|, not to the sum.)"""
+    """GPU fp32 logits against the oracle's fp64 router product (optionally sampled rows),
+    per token and expert: |gpu - oracle| <= 1e-5 * sum_d |x_d Wg[e, d]|.  A logit whose terms
+    are all zero (cond = 0) must be exactly zero."""
     x = np64(inp.x) if rows is None else np64(inp.x[torch.as_tensor(rows, device=inp.x.device)])
-    ref = O.router_logits(x, np64(inp.Wg))
+    Wg = np64(inp.Wg)
+    ref = O.router_logits(x, Wg)
     got = v["logits"].double().cpu().numpy()
     if rows is not None:
         got = got[rows]
-    err = max_rel(got, ref)
-    assert err <= TOL_LOGITS, f"router logits max rel err {err:.3e}"
+    cond = logit_condition(x, Wg)
+    diff = np.abs(got - ref)
+    zero = cond == 0.0
+    assert np.all(diff[zero] == 0.0), "a logit with no nonzero term is not exactly zero"
+    rel = diff[~zero] / cond[~zero]
+    err = float(rel.max()) if rel.size else 0.0
+    assert err <= TOL_LOGITS, f"router logit error {err:.3e} of sum|x*Wg| (tolerance 1e-5)"
     return err
 
 
@@ -175,3 +186,70 @@ def check_sampled_output(w, inp, out, v, tokens):
         if np.all(ref[i] == 0.0):
             assert np.all(got[i] == 0.0)
     return err
+
+
+def stratified_rows(offsets, rng, every_slice=True):
+    """Executed rows to check at full size.  The grouped GEMM tiles each expert's rows from the
+    expert's first row in 256-row tiles made of two 128-row MMA halves, whose rows sit in the
+    four 32-lane quarters of the TMEM accumulator; so the 32-row slices of each expert, counted
+    from its first row, are exactly its (tile, half, lane quarter) cells.  One random row from
+    every slice (or, with every_slice=False, from one random slice per expert), plus each
+    expert's last row (the ragged tail of its last tile)."""
+    rows = set()
+    for e in range(len(offsets) - 1):
+        lo, hi = int(offsets[e]), int(offsets[e + 1])
+        if hi <= lo:
+            continue
+        starts = list(range(lo, hi, 32))
+        if not every_slice:
+            starts = [starts[int(rng.integers(len(starts)))]]
+        for s in starts:
+            rows.add(int(rng.integers(s, min(s + 32, hi))))
+        rows.add(hi - 1)
+    return sorted(rows)
+
+
+def check_stratified_output(w, inp, out, v, seed=123, every_slice=True, extra_tokens=()):
+    """Full-size output parity on a tile-stratified sample (stratified_rows).
+
+    Each sampled executed row's expert output y (before its gate) is compared with the
+    oracle's evaluation of that assignment; every token owning a sampled row, every token of
+    one row per 32-token slice of the shared experts' group (the tokens themselves) and
+    `extra_tokens` are compared on the whole layer output, the oracle routing the batch from
+    the GPU's fp32 logits.  Returns (rows checked, tokens checked, y error, output error)."""
+    rng = np.random.default_rng(seed)
+    offsets = v["offsets"].cpu().numpy()
+    row_src = v["row_src"].cpu().numpy()
+    K = w.E if w.select == "expert" else w.k
+    rows = stratified_rows(offsets, rng, every_slice)
+    tokens = {int(row_src[r]) // K for r in rows}
+    if w.n_shared:
+        tokens.update(stratified_rows(np.array([0, w.T]), rng, every_slice))
+    tokens.update(int(t) for t in extra_tokens)
+    tokens = sorted(tokens)
+    logits = v["logits"].double().cpu().numpy()
+    tk = torch.as_tensor(tokens, device=inp.x.device, dtype=torch.long)
+    x_rows = np.zeros((w.T, w.D))
+    x_rows[tokens] = np64(inp.x[tk])
+    r = O.layer_forward_rows(wdict(w), tokens, x_rows, None, np64(inp.bias), None, None, None,
+                             np64(inp.Ws_gate), np64(inp.Ws_up), np64(inp.Ws_down),
+                             logits=logits, weights_of=expert_weights_streamer(inp))
+    # expert outputs of the sampled rows
+    ref_y = np.stack([r["y_assign"][(int(row_src[q]) // K, int(row_src[q]) % K)] for q in rows])
+    got_y = np64(v["y"][torch.as_tensor(rows, device=inp.x.device, dtype=torch.long)])
+    err_y = max_rel(got_y, ref_y)
+    assert err_y <= TOL_OUT[w.dtype], f"sampled expert rows max rel err {err_y:.3e}"
+    if w.n_shared:
+        for i in range(w.n_shared):
+            got_s = np64(v["y_shared"][i][tk])
+            err_s = max_rel(got_s, r["shared_rows"][i])
+            assert err_s <= TOL_OUT[w.dtype], f"shared expert {i} rows max rel err {err_s:.3e}"
+    # whole-layer output of the tokens
+    got = out[tk].double().cpu().numpy()
+    ref = r["out_rows"]
+    err = max_rel(got, ref)
+    assert err <= TOL_OUT[w.dtype], f"sampled output max rel err {err:.3e}"
+    for i in range(len(tokens)):
+        if np.all(ref[i] == 0.0):
+            assert np.all(got[i] == 0.0)
+    return len(rows), len(tokens), err_y, err

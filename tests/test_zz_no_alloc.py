@@ -6,7 +6,8 @@ entry point keeps that scratch in a fixed device array inside the library instea
 calls it through the C ABI twice in a row, on two different routings, and checks each result
 against moe_permute's: the permutation is integer work, so they must agree bit for bit (the
 tolerance of the other permute checks).  The second call reuses the shared array the first one
-left behind.  It also checks the size limit is refused before anything runs.
+left behind.  A host-only test (no GPU needed) checks that a problem beyond the array's size is
+refused before any pointer is looked at or anything is launched.
 
 The file name sorts last so that a run stopping at its first failure has run every other test.
 """
@@ -18,8 +19,6 @@ import torch
 
 import sparse_mixture_experts_warp_b200 as M
 from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, make_inputs, scaled
-
-pytestmark = pytest.mark.gpu
 
 
 def _route(w, seed):
@@ -61,13 +60,18 @@ def _compare(w, d, x, ids):
     assert torch.equal(got["x_perm"][:n], ref["x_perm"][:n])
 
 
+# The permute takes its one-pass path (E <= 8 and at most 16384 assignments) or its one-CTA
+# index path (at most 8192 assignments otherwise) without touching the scratch array; above
+# those sizes it builds per-block histograms in it.
+@pytest.mark.gpu
 @pytest.mark.parametrize("name,shape", [
-    ("mixtral", dict(T=700, D=512, F=1024)),
-    ("switch", dict(T=3000, D=256, E=16, F=512)),     # capacity drop
+    ("mixtral", dict(T=700, D=512, F=1024)),            # one-pass path
+    ("switch", dict(T=3000, D=256, E=16, F=512)),      # index path, capacity drop
     ("v3", dict(T=300, D=512, E=64, F=256, F_shared=256)),
-    # more than 65536 assignments: the histogram path that uses the fixed scratch array
-    ("mixtral", dict(T=40000, D=128, F=128)),
-    ("v3", dict(T=9000, D=128, E=64, F=128, F_shared=128)),
+    # histogram paths, in the fixed scratch array
+    ("mixtral", dict(T=40000, D=128, F=128)),           # 80000 assignments, E = 8
+    ("v3", dict(T=9000, D=128, E=64, F=128, F_shared=128)),   # 72000 assignments
+    ("switch", dict(T=20000, D=256, E=16, F=512)),     # 20000 assignments, capacity clamp
 ])
 def test_noalloc_permute_matches_permute_on_two_calls(name, shape):
     w = scaled(WORKLOADS[name], **shape)
@@ -77,9 +81,14 @@ def test_noalloc_permute_matches_permute_on_two_calls(name, shape):
 
 
 def test_noalloc_permute_rejects_oversized_problems_before_launch():
+    """Host-only: the size check comes before the pointer checks, so with every pointer NULL an
+    oversized problem still answers MOE_ERR_UNSUPPORTED, and a size that fits answers
+    MOE_ERR_INVALID_ARG; neither launches anything (no GPU is needed)."""
     w = scaled(WORKLOADS["v3"], T=300_000, D=512, F=256, F_shared=256)
     d = M.desc_of(w)
     # ceil(300000*8/1024) * 256 histogram entries exceed the fixed array
     assert -(-w.T * w.k // 1024) * w.E > 65536
-    st = M.lib().moe_permute_noalloc(ctypes.byref(d), 16, 16, 16, 16, 16, 16, 16, None)
-    assert st == 2      # MOE_ERR_UNSUPPORTED
+    nulls = [None] * 7
+    assert M.lib().moe_permute_noalloc(ctypes.byref(d), *nulls, None) == 2  # UNSUPPORTED
+    small = M.desc_of(scaled(WORKLOADS["v3"], T=300, D=512, F=256, F_shared=256))
+    assert M.lib().moe_permute_noalloc(ctypes.byref(small), *nulls, None) == 1  # INVALID_ARG
