@@ -18,8 +18,12 @@ slowest rank's time (weak scaling).
 `--impl reference` times the CPU oracle (fp64) on the host cores on bounded samples of the
 same workload: each step routes the whole batch and evaluates a sample of its tokens.
 
-After the forward, a training step (moe_layer_forward_train + moe_layer_backward) is timed
-too, reported under "backward" (`--no-backward` skips it).  `--tokens` and `--ffn` shrink the
+After the forward, the same graph is replayed for about a second ("sustained": the clock the
+1 kW power cap settles at), and a training step (moe_layer_forward_train + moe_layer_backward)
+is timed, reported under "backward" (`--no-backward` skips it).  At one GPU the other layer
+shapes the pages name -- Switch top-1, DeepSeek-V3, expert choice at the DeepSeekMoE-16B shape
+and a one-token Mixtral decode step -- are then timed for a few graph-replayed steps each and
+reported under "per_workload", each with its dominant stage and the fraction of its roofline.  `--tokens` and `--ffn` shrink the
 batch or the expert width for profiling cases and the small-batch (decode) regime; the DRAM
 traffic figure is then null (it is taken from an ncu capture of the full-size workload only).
 """
@@ -29,6 +33,7 @@ from __future__ import annotations
 import argparse
 import hashlib
 import json
+import math
 import os
 import statistics
 import sys
@@ -93,7 +98,7 @@ def load_traffic(workload, w):
 
 
 class ClockSampler:
-    """Samples the SM clock and clock-event reasons of one GPU in a thread (NVML, 20 ms)."""
+    """Samples the SM clock and clock-event reasons of one GPU in a thread (NVML, every 5 ms)."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -134,7 +139,7 @@ class ClockSampler:
                         self.reasons.add(name)
             except Exception as e:  # pragma: no cover
                 self.error = str(e)
-            self._stop.wait(0.02)
+            self._stop.wait(0.005)
 
     def __exit__(self, *a):
         self._stop.set()
@@ -351,6 +356,225 @@ def time_backward(M, w, d, inp, ws, stream, dev, steps, warmup, tc_peak, world):
                     "fixed; dout ~ N(0,1) bf16; ms_per_step is the backward alone"}
 
 
+class LayerStep:
+    """One step of the layer through the library's step entry points, in the order
+    moe_layer_forward chains them, with optional CUDA events between the stages."""
+
+    def __init__(self, M, w, inp, dev, stream):
+        self.M, self.w, self.inp, self.dev, self.stream = M, w, inp, dev, stream
+        self.d = M.desc_of(w)
+        self.ws = M.empty_workspace(self.d, dev)
+        self.v = M.layer_views(self.d, self.ws)
+        self.out = torch.empty_like(inp.x)
+        if w.n_shared:
+            # shared experts: one group over all T tokens, SwiGLU of width F_shared
+            self.d_sh = M.desc_of(w)
+            self.d_sh.act = M.SWIGLU
+            self.sh_off = torch.tensor([0, w.T], dtype=torch.int32, device=dev)
+            self.h_sh = torch.empty(w.T, w.F_shared, dtype=inp.x.dtype, device=dev)
+        self.graph, self.graph_launches, self.graph_error = None, 0, None
+
+    def __call__(self, ev=None, st=None):
+        M, w, inp, v = self.M, self.w, self.inp, self.v
+        d, scratch = self.d, v["scratch"]
+        s = st if st is not None else self.stream
+        M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
+                    v["importance"], scratch, s, entropy=v["entropy"])
+        if ev is not None:
+            ev[1].record(s)
+        M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
+                      v["row_src"], v["inv"], scratch, s)
+        if ev is not None:
+            ev[2].record(s)
+        # (with a few executed rows the routed experts' products take the k-split schedule, its
+        # partials in the step scratch, as in moe_layer_forward)
+        M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
+                           scratch, s)
+        if ev is not None:
+            ev[3].record(s)
+        M.moe_expert_down_ws(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], scratch, s)
+        for i in range(w.n_shared):
+            M.moe_expert_ffn(self.d_sh, 1, w.F_shared, inp.x, self.sh_off, inp.Ws_gate[i],
+                             inp.Ws_up[i], inp.Ws_down[i], self.h_sh, v["y_shared"][i], s)
+        if ev is not None:
+            ev[4].record(s)
+        M.moe_combine(d, v["y"], v["inv"], v["gates"], v["y_shared"] if w.n_shared else None,
+                      self.out, s)
+        if ev is not None:
+            ev[5].record(s)
+        M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
+                            s, entropy=v["entropy"])
+        if ev is not None:
+            ev[6].record(s)
+
+    def capture(self, warmup):
+        """The step captured once in a CUDA graph (the library allocates and synchronises
+        nothing, so its calls capture as they are); replays remove the host launch gaps."""
+        M, dev = self.M, self.dev
+        try:
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(self.stream)
+            g = torch.cuda.CUDAGraph()
+            n0 = M.kernel_launches()
+            with torch.cuda.graph(g, stream=cap):
+                self(st=cap)
+            self.graph_launches = M.kernel_launches() - n0
+            self.stream.wait_stream(cap)
+            for _ in range(max(warmup, 3)):
+                g.replay()
+            torch.cuda.synchronize(dev)
+            self.graph = g
+        except Exception as e:          # capture not possible here: time the eager calls
+            self.graph_error = str(e).splitlines()[0][:200]
+
+    def staged_times(self, steps):
+        """Per-stage device times from replays of a second graph of the step that holds event
+        record nodes between the stages (no host launch gaps); None if that capture fails."""
+        M, dev = self.M, self.dev
+        try:
+            evs = [torch.cuda.Event(enable_timing=True, external=True) for _ in range(7)]
+            cap = torch.cuda.Stream(dev)
+            cap.wait_stream(self.stream)
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap):
+                evs[0].record(cap)
+                self(evs, st=cap)
+            self.stream.wait_stream(cap)
+            g.replay()
+            torch.cuda.synchronize(dev)
+            acc = {s: 0.0 for s in STAGES}
+            for _ in range(steps):
+                g.replay()
+                torch.cuda.synchronize(dev)
+                for j, s in enumerate(STAGES):
+                    acc[s] += evs[j].elapsed_time(evs[j + 1])
+            del g
+            return {s: acc[s] / steps for s in STAGES}
+        except Exception:
+            return None
+
+    def timed(self, steps, use_graph, nvml_index, world):
+        """(total ms, per-stage ms or None, clock sampler, kernel launches) of `steps` steps."""
+        M, dev, stream = self.M, self.dev, self.stream
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)] for _ in range(steps)]
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(dev)
+        with ClockSampler(nvml_index) as clk:
+            n0 = M.kernel_launches()
+            start.record(stream)
+            for i in range(steps):
+                if use_graph:
+                    self.graph.replay()
+                else:
+                    evs[i][0].record(stream)
+                    self(evs[i])
+            end.record(stream)
+            launches = self.graph_launches * steps if use_graph else M.kernel_launches() - n0
+            torch.cuda.synchronize(dev)
+        barrier(world)
+        total = start.elapsed_time(end)
+        if use_graph:
+            return total, None, clk, launches
+        per_stage = {s: 0.0 for s in STAGES}
+        for i in range(steps):
+            for j, s in enumerate(STAGES):
+                per_stage[s] += evs[i][j].elapsed_time(evs[i][j + 1])
+        return total, {s: per_stage[s] / steps for s in STAGES}, clk, launches
+
+    def release(self):
+        self.graph = None
+        self.ws = self.v = self.out = None
+
+
+def stage_rooflines(w, per_stage, rows_exec, active, peaks, tc_peak):
+    """Per stage: achieved rate and the fraction of its own roofline time (GEMM stages: the
+    slower of FLOPs at the tensor peak and weight + activation bytes at the HBM peak; the
+    others: bytes at the HBM peak), plus the whole layer's roofline."""
+    work = stage_work(w, rows_exec)
+    es = 2 if w.dtype == "bf16" else 4
+    n_up = 2 if w.act == "swiglu" else 1
+    gemm_bytes = {
+        "expert_up": active * n_up * w.F * w.D * es + rows_exec * (w.D + w.F) * es,
+        "expert_down": active * w.F * w.D * es + rows_exec * (w.F + w.D) * es
+        + w.n_shared * (3 * w.F_shared * w.D + w.T * (w.D + 2 * w.F_shared + w.D)) * es,
+    }
+    hbm = peaks["hbm_gbs"] * 1e9
+    stages = {}
+    for s in STAGES:
+        kind, amount = work[s]
+        t = per_stage[s] * 1e-3
+        if kind == "tensor":
+            roof = max(amount / (tc_peak * 1e12), gemm_bytes[s] / hbm)
+            bound = "tensor" if amount / (tc_peak * 1e12) >= gemm_bytes[s] / hbm else "hbm"
+            ach = amount / t / 1e12
+            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "tflops": round(ach, 1),
+                         "gbs": round(gemm_bytes[s] / t / 1e9, 1), "bound": bound,
+                         "frac": round(ach / tc_peak, 3), "roof_frac": round(roof / t, 3)}
+        else:
+            ach = amount / t / 1e9
+            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "gbs": round(ach, 1),
+                         "bound": "hbm", "frac": round(ach / peaks["hbm_gbs"], 3),
+                         "roof_frac": round(amount / hbm / t, 3)}
+    gemm_flops = work["expert_up"][1] + work["expert_down"][1]
+    hbm_bytes = sum(work[s][1] for s in ("route", "permute", "combine", "stats"))
+    gemm_roof_s = max(gemm_flops / (tc_peak * 1e12),
+                      gemm_hbm_bytes(w, rows_exec, active) / hbm)
+    layer_roof_s = gemm_roof_s + hbm_bytes / hbm
+    return stages, work, gemm_flops, layer_roof_s
+
+
+def rows_and_active(v):
+    offs = v["offsets"].cpu()
+    return int(offs[-1].item()), int(((offs[1:] - offs[:-1]) > 0).sum().item())
+
+
+def measure_workload(M, w, seed, dev, stream, steps, warmup, nvml_index, peaks):
+    """A shorter measurement of another workload shape (graph replays for the step time,
+    eager calls for the stage times), reported beside the headline."""
+    inp = make_inputs(w, seed=seed, device=dev)
+    st = LayerStep(M, w, inp, dev, stream)
+    for _ in range(warmup):
+        st()
+    torch.cuda.synchronize(dev)
+    st.capture(warmup)
+    use_graph = st.graph is not None
+    total, _, clk, launches = st.timed(steps, use_graph, nvml_index, 1)
+    eager_total, per_stage, _, _ = st.timed(steps, False, nvml_index, 1)
+    staged = st.staged_times(steps) if use_graph else None
+    if staged is not None:
+        per_stage = staged
+    err = M.get_device_error(stream)
+    if err:
+        raise RuntimeError(f"device error word {err:#x} ({w.name})")
+    ms = (total if use_graph else eager_total) / steps
+    tc_key = "bf16_tflops_sustained" if "sw_power_cap" in clk.reasons else "bf16_tflops"
+    rows_exec, active = rows_and_active(st.v)
+    stages, work, gemm_flops, layer_roof_s = stage_rooflines(w, per_stage, rows_exec, active,
+                                                             peaks, peaks[tc_key])
+    top = max(STAGES, key=lambda s: per_stage[s])
+    res = {
+        "shape": w.description, "T": w.T, "ms_per_step": round(ms, 4),
+        "tokens_per_s": round(w.T / (ms * 1e-3), 1), "steps": steps,
+        "timing": "CUDA-graph replay" if use_graph else "eager calls",
+        "stage_timing": "graph replays, event nodes between stages" if staged is not None
+        else "eager calls, events between stages",
+        "rows_executed": rows_exec, "active_experts": active,
+        "dominant": {"stage": top, **stages[top]},
+        "layer_frac_of_roofline": round(layer_roof_s / (ms * 1e-3), 3),
+        "layer_roofline_ms": round(layer_roof_s * 1e3, 4),
+        "stages": stages, "tc_peak": tc_key, "clocks": clk.summary(),
+    }
+    st.release()
+    del inp
+    torch.cuda.empty_cache()
+    return res
+
+
+# the other layer shapes timed beside the headline (name, batch override)
+PER_WORKLOAD = [("switch", None), ("v3", None), ("ec", None), ("mixtral_T1", 1)]
+
+
 def run_cuda(args, rank, world, local):
     import sparse_mixture_experts_warp_b200 as M
 
@@ -358,122 +582,47 @@ def run_cuda(args, rank, world, local):
     dev = torch.device("cuda", local)
     w = workload_of(args)
     inp = make_inputs(w, seed=rank, device=dev)
-    d = M.desc_of(w)
-    ws = M.empty_workspace(d, dev)
-    v = M.layer_views(d, ws)
-    scratch = v["scratch"]
-    out = torch.empty_like(inp.x)
     stream = torch.cuda.current_stream(dev)
-    if w.n_shared:
-        # shared experts: one group over all T tokens, SwiGLU of width F_shared
-        d_sh = M.desc_of(w)
-        d_sh.act = M.SWIGLU
-        sh_off = torch.tensor([0, w.T], dtype=torch.int32, device=dev)
-        h_sh = torch.empty(w.T, w.F_shared, dtype=inp.x.dtype, device=dev)
-
-    def step(ev=None, st=None):
-        stream_ = st if st is not None else stream
-        M.moe_route(d, inp.x, inp.Wg, inp.bias, v["expert_ids"], v["gates"], v["logits"],
-                    v["importance"], scratch, stream_, entropy=v["entropy"])
-        if ev is not None:
-            ev[1].record(stream_)
-        M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
-                      v["row_src"], v["inv"], scratch, stream_)
-        if ev is not None:
-            ev[2].record(stream_)
-        # (with a few executed rows the routed experts' products take the k-split schedule, its
-        # partials in the step scratch, as in moe_layer_forward)
-        M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
-                           scratch, stream_)
-        if ev is not None:
-            ev[3].record(stream_)
-        M.moe_expert_down_ws(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], scratch,
-                             stream_)
-        for i in range(w.n_shared):
-            M.moe_expert_ffn(d_sh, 1, w.F_shared, inp.x, sh_off, inp.Ws_gate[i], inp.Ws_up[i],
-                             inp.Ws_down[i], h_sh, v["y_shared"][i], stream_)
-        if ev is not None:
-            ev[4].record(stream_)
-        M.moe_combine(d, v["y"], v["inv"], v["gates"], v["y_shared"] if w.n_shared else None,
-                      out, stream_)
-        if ev is not None:
-            ev[5].record(stream_)
-        M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], v["f"], v["stats"],
-                            stream_, entropy=v["entropy"])
-        if ev is not None:
-            ev[6].record(stream_)
+    step = LayerStep(M, w, inp, dev, stream)
+    d, ws, v = step.d, step.ws, step.v
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize(dev)
-
-    # the step captured once in a CUDA graph (the library allocates and synchronises nothing,
-    # so its calls capture as they are); replays remove the host launch gaps between kernels
-    graph, graph_launches, graph_error = None, 0, None
     if not args.no_graph:
-        try:
-            cap = torch.cuda.Stream(dev)
-            cap.wait_stream(stream)
-            g = torch.cuda.CUDAGraph()
-            n0 = M.kernel_launches()
-            with torch.cuda.graph(g, stream=cap):
-                step(st=cap)
-            graph_launches = M.kernel_launches() - n0
-            stream.wait_stream(cap)
-            for _ in range(max(args.warmup, 3)):
-                g.replay()
-            torch.cuda.synchronize(dev)
-            graph = g
-        except Exception as e:          # capture not possible here: time the eager calls
-            graph_error = str(e).splitlines()[0][:200]
+        step.capture(args.warmup)
     nvml_index = local if "CUDA_VISIBLE_DEVICES" not in os.environ else \
         int(os.environ["CUDA_VISIBLE_DEVICES"].split(",")[local])
 
-    def timed(use_graph):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(7)]
-               for _ in range(args.steps)]
-        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize(dev)
-        with ClockSampler(nvml_index) as clk:
-            n0 = M.kernel_launches()
-            start.record(stream)
-            for i in range(args.steps):
-                if use_graph:
-                    graph.replay()
-                else:
-                    evs[i][0].record(stream)
-                    step(evs[i])
-            end.record(stream)
-            launches = (graph_launches * args.steps if use_graph
-                        else M.kernel_launches() - n0)
-            torch.cuda.synchronize(dev)
-        barrier(world)
-        total = start.elapsed_time(end)
-        if use_graph:
-            return total, None, clk, launches
-        per_stage = {s: 0.0 for s in STAGES}
-        for i in range(args.steps):
-            for j, s in enumerate(STAGES):
-                per_stage[s] += evs[i][j].elapsed_time(evs[i][j + 1])
-        return total, {s: per_stage[s] / args.steps for s in STAGES}, clk, launches
-
     # the headline from graph replays (timed first), per-stage times from the eager calls
     # (events between stages)
-    use_graph = graph is not None
-    total_ms, per_stage, clk, launches = timed(use_graph)
+    use_graph = step.graph is not None
+    total_ms, per_stage, clk, launches = step.timed(args.steps, use_graph, nvml_index, world)
     remeasured = False
     if clk.rejected():
-        total_ms, per_stage, clk, launches = timed(use_graph)
+        total_ms, per_stage, clk, launches = step.timed(args.steps, use_graph, nvml_index, world)
         remeasured = True
     if use_graph:
-        eager_ms, per_stage, _, _ = timed(False)
+        eager_ms, eager_stage, _, _ = step.timed(args.steps, False, nvml_index, world)
+        graph_stage = step.staged_times(args.steps)
+        per_stage = graph_stage if graph_stage is not None else eager_stage
     else:
-        eager_ms = total_ms
+        eager_ms, eager_stage, graph_stage = total_ms, per_stage, None
     total_ms = max_over_ranks(total_ms, world, dev)
     eager_ms = max_over_ranks(eager_ms, world, dev)
     ms_per_step = total_ms / args.steps
     value = job_throughput(w.T, world, args.steps, total_ms)
+
+    # sustained: the same graph replayed for about a second, where the 1 kW power cap sets the
+    # clock, reported beside the headline
+    sustained = None
+    if use_graph and not args.no_sustained:
+        n_sus = max(args.steps, int(math.ceil(1000.0 / max(ms_per_step, 1e-3))))
+        sus_ms, _, sus_clk, _ = step.timed(n_sus, True, nvml_index, world)
+        sus_ms = max_over_ranks(sus_ms, world, dev)
+        sustained = {"steps": n_sus, "ms_per_step": round(sus_ms / n_sus, 4),
+                     "value": round(job_throughput(w.T, world, n_sus, sus_ms), 1),
+                     "clocks": sus_clk.summary()}
 
     # e2e: the public call with host buffers; every step copies its own tokens in from pinned
     # host memory and its output back, inside the timed region.  Copies run on their own
@@ -489,36 +638,16 @@ def run_cuda(args, rank, world, local):
         raise RuntimeError(f"device error word {err:#x}")
 
     # roofline of the dominant kernel (gate/up grouped GEMM launch)
-    rows_exec = int(v["offsets"][-1].item())
-    work = stage_work(w, rows_exec)
+    rows_exec, active = rows_and_active(v)
     peaks, peaks_kind = load_peaks()
     power_capped = "sw_power_cap" in clk.reasons
     tc_key = "bf16_tflops_sustained" if power_capped else "bf16_tflops"
     tc_peak = peaks[tc_key]
-    stages = {}
-    for s in STAGES:
-        kind, amount = work[s]
-        t = per_stage[s] * 1e-3
-        if kind == "tensor":
-            ach = amount / t / 1e12
-            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "tflops": round(ach, 1),
-                         "frac": round(ach / tc_peak, 3)}
-        else:
-            ach = amount / t / 1e9
-            stages[s] = {"us": round(per_stage[s] * 1e3, 2), "gbs": round(ach, 1),
-                         "frac": round(ach / peaks["hbm_gbs"], 3)}
+    stages, work, gemm_flops, layer_roof_s = stage_rooflines(w, per_stage, rows_exec, active,
+                                                             peaks, tc_peak)
     up_flops = work["expert_up"][1]
     achieved = up_flops / (per_stage["expert_up"] * 1e-3) / 1e12
-    gemm_flops = work["expert_up"][1] + work["expert_down"][1]
     gemm_tflops = gemm_flops / ((per_stage["expert_up"] + per_stage["expert_down"]) * 1e-3) / 1e12
-    # whole-layer roofline: the expert GEMMs at the slower of their FLOPs at the tensor peak and
-    # their weight + activation bytes at the HBM peak, plus the HBM-bound stages' bytes
-    hbm_bytes = sum(work[s][1] for s in ("route", "permute", "combine", "stats"))
-    offs = v["offsets"].cpu()
-    active = int(((offs[1:] - offs[:-1]) > 0).sum().item())
-    gemm_bytes = gemm_hbm_bytes(w, rows_exec, active)
-    gemm_roof_s = max(gemm_flops / (tc_peak * 1e12), gemm_bytes / (peaks["hbm_gbs"] * 1e9))
-    layer_roof_s = gemm_roof_s + hbm_bytes / (peaks["hbm_gbs"] * 1e9)
     roofline = {
         "bound": "tensor",
         "kernel": "grouped_gemm_kernel<EPI_SWIGLU> (expert up: gate+up, SiLU*up epilogue)",
@@ -543,6 +672,9 @@ def run_cuda(args, rank, world, local):
                    "l2": "inputs larger than L2: %.2f GB of expert weights stream per step"
                          % ((w.E * 3 * w.F * w.D * 2) / 1e9)},
         "roofline": roofline, "stages": stages,
+        "stage_timing": ("graph replays with event record nodes between the stages"
+                         if graph_stage is not None else "eager calls, events between stages"),
+        "eager_stage_us": {s: round(eager_stage[s] * 1e3, 2) for s in STAGES},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms / args.steps, 4),
                 "h2d_bytes_per_step": x_bytes, "d2h_bytes_per_step": x_bytes,
@@ -551,19 +683,36 @@ def run_cuda(args, rank, world, local):
         "gpu_launches": launches,
         "clocks": clk.summary(),
         "timing": ("CUDA-graph replay of the step (%d library kernels per step); per-stage "
-                   "times from eager calls" % graph_launches) if use_graph else
-                  ("eager calls" + (" (graph capture failed: %s)" % graph_error
-                                    if graph_error else "")),
+                   "times from eager calls" % step.graph_launches) if use_graph else
+                  ("eager calls" + (" (graph capture failed: %s)" % step.graph_error
+                                    if step.graph_error else "")),
         "eager_value": round(job_throughput(w.T, world, args.steps, eager_ms), 1),
     }
+    if sustained:
+        res["sustained"] = sustained
     if remeasured:
         res["clocks"]["remeasured"] = True
     if (not args.no_backward and w.dtype == "bf16" and w.select == "token"
             and not w.n_shared):
         res["backward"] = time_backward(M, w, d, inp, ws, stream, dev, min(args.steps, 20),
                                         max(args.warmup, 3), tc_peak, world)
+    step.release()
+    del inp
+    torch.cuda.empty_cache()
+    if world == 1 and not args.no_per_workload and args.workload == "mixtral" \
+            and not args.tokens and not args.ffn:
+        per = {}
+        for name, T in PER_WORKLOAD:
+            wk = WORKLOADS[name.split("_")[0]]
+            if T:
+                wk = scaled(wk, T=T)
+            per[name] = measure_workload(M, wk, rank, dev, stream, min(args.steps, 20), 3,
+                                         nvml_index, peaks)
+        res["per_workload"] = per
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        res["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.cpu_budget)
+        w_cpu = workload_of(args)
+        inp_cpu = make_inputs(w_cpu, seed=rank, device=dev)
+        res["cpu_baseline"] = cpu_baseline(w_cpu, inp_cpu, budget_s=args.cpu_budget)
     if rank == 0:
         print(json.dumps(res), flush=True)
 
@@ -689,6 +838,10 @@ def main():
                     help="time eager calls instead of a CUDA-graph replay of the step")
     ap.add_argument("--no-backward", action="store_true",
                     help="skip the backward-pass timing that follows the forward measurement")
+    ap.add_argument("--no-sustained", action="store_true",
+                    help="skip the one-second replay of the step reported as 'sustained'")
+    ap.add_argument("--no-per-workload", action="store_true",
+                    help="skip the shorter measurements of the other layer shapes")
     ap.add_argument("--cpu-budget", type=float, default=15.0)
     ap.add_argument("--ref-budget", type=float, default=90.0)
     args = ap.parse_args()

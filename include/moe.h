@@ -310,6 +310,38 @@ moe_status_t moe_layer_forward_train(const moe_desc_t* desc, const void* x, cons
                                      size_t ws_bytes, void* bwd_ws, size_t bwd_ws_bytes,
                                      moe_stream_t stream);
 
+/* Expert parallelism ("Top-k 路由" section "通訊拓撲：All-to-All": rows go to the device that
+ * holds their expert and their outputs come back, two All-to-All exchanges per layer;
+ * "别只比较 Top-k", "两次 All-to-All 是常见 dispatcher 的前向合同").  G ranks, rank r holds the
+ * Eg = E / G experts [r Eg, (r+1) Eg).  A rank's permuted rows are already grouped by expert,
+ * so the rows for rank r are the contiguous range of its experts' rows.
+ *
+ * moe_ep_plan (host only, no GPU needed) turns the row counts into the exchange plan.
+ *   rows_send [G*Eg]: this rank's rows per expert (kept rows, offsets[e+1] - offsets[e]),
+ *     entry r*Eg + e for expert r*Eg + e.
+ *   rows_recv [G*Eg]: rows_recv[s*Eg + e] = rows source rank s sends for local expert e (its
+ *     rows_send entry r*Eg + e, received through a count exchange).
+ *   Outputs (caller arrays): send_rows / send_offsets [G] and recv_rows / recv_offsets [G]
+ *   (rows per peer and their start, in rows, in the send buffer = the permuted rows and in the
+ *   source-major receive buffer); local_offsets [Eg+1], the expert-major layout the grouped
+ *   GEMM runs on (local expert e: its rows from source 0, then 1, ...); block (s, e) at index
+ *   s*Eg + e: block_recv (start in the receive buffer), block_local (start in the local
+ *   layout), block_rows; *max_block_rows.  Negative counts or G*Eg > 65536 give
+ *   MOE_ERR_INVALID_ARG.
+ * moe_ep_reorder moves row blocks on `stream`: dst[dst_start[b] + i] = src[src_start[b] + i]
+ *   for i < block_rows[b], rows of desc->D elements of desc->dtype; the three block arrays are
+ *   device arrays of n_blocks int64; 16-byte aligned src and dst.  Receive buffer -> local
+ *   layout with (block_recv, block_local); back with the two swapped. */
+moe_status_t moe_ep_plan(int32_t G, int32_t Eg, const int32_t* rows_send,
+                         const int32_t* rows_recv, int64_t* send_rows, int64_t* send_offsets,
+                         int64_t* recv_rows, int64_t* recv_offsets, int32_t* local_offsets,
+                         int64_t* block_recv, int64_t* block_local, int64_t* block_rows,
+                         int64_t* max_block_rows);
+moe_status_t moe_ep_reorder(const moe_desc_t* desc, int32_t n_blocks, const int64_t* src_start,
+                            const int64_t* dst_start, const int64_t* block_rows,
+                            int64_t max_block_rows, const void* src, void* dst,
+                            moe_stream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that kernels set when
  * a bounded wait gives up (MOE_ERR_TIMEOUT) or a device-side check fires (MOE_ERR_DEVICE).
  * *code receives the raw word (0 = none).  Returns MOE_OK when the word was 0. */

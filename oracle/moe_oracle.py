@@ -651,25 +651,31 @@ def gate_logit_grad(logits, ids, dgates, score="softmax", gate="renorm", bias=No
     return ds
 
 
-def layer_backward(w, x, Wg, bias, W_gate, W_up, W_down, dout, aux_grad=1.0, logits=None):
+def layer_backward(w, x, Wg, bias, W_gate, W_up, W_down, dout, aux_grad=1.0, logits=None,
+                   Ws_gate=None, Ws_up=None, Ws_down=None):
     """Gradients of L = <dout, out> + aux_grad * aux for one MoE layer, the
-    routing of layer_forward held fixed (no shared experts).
+    routing of layer_forward held fixed.
 
     Per kept assignment (t, j) -> row r of expert e: dy_r = g[t,j] dout[t] and
-    dg[t,j] = <dout[t], y_r>; a dropped assignment has neither.  Experts:
-    expert_backward on their rows.  Router: ds = gate_logit_grad(dg) plus the
+    dg[t,j] = <dout[t], y_r>; a dropped (or, under expert choice, unpicked)
+    assignment has neither.  Experts: expert_backward on their rows.
+    Router: token choice -- ds = gate_logit_grad(dg); expert choice -- the
+    merge weight of (t, e) is the softmax probability p[t, e] itself, so
+    ds = p (.) (dp - <p, dp>) with dp[t, e] = dg[t, e] on picked pairs, 0
+    elsewhere (the picked sets are held fixed, as the top-k is).  Plus the
     balance-loss term: aux = alpha E sum_e f_e P_e with f fixed (counts) and
     P_e = mean_t of the importance rows, so dP_e = aux_grad alpha E f_e / T,
     pushed through softmax over all E (ds = p (dq - <p, dq>)) or through
     q = a / sum_e a under sigmoid (da = (dq - <q, dq>) / sum a, ds = da a (1-a)).
-    dW_g = ds^T x, and dx = sum_j dx_rows[r(t, j)] + ds W_g.
+    Shared experts ([CMP] "shared direct path", weight 1) see dout on every
+    token: dx gains their input gradient and dWs_* their weight gradients.
+    dW_g = ds^T x, and dx = sum_j dx_rows[r(t, j)] + ds W_g (+ shared).
     """
     g = _get(w)
-    if g["n_shared"] or g["select"] != "token":
-        raise ValueError("backward: token choice without shared experts")
     x = _np(x)
     Wg = _np(Wg)
-    r = layer_forward(w, x, Wg, bias, W_gate, W_up, W_down, logits=logits)
+    r = layer_forward(w, x, Wg, bias, W_gate, W_up, W_down, Ws_gate, Ws_up, Ws_down,
+                      logits=logits)
     s, K, T, E = r["logits"], r["K"], g["T"], g["E"]
     dout = np.asarray(dout, dtype=np.float64)
     inv = np.asarray(r["inv"]).reshape(T, K)
@@ -700,7 +706,12 @@ def layer_backward(w, x, Wg, bias, W_gate, W_up, W_down, dout, aux_grad=1.0, log
         if dge is not None:
             dWgate[e] = dge
         dWup[e], dWdown[e] = due, dde
-    ds = gate_logit_grad(s, r["ids"], dgates, g["score"], g["gate"], _np(bias))
+    if g["select"] == "token":
+        ds = gate_logit_grad(s, r["ids"], dgates, g["score"], g["gate"], _np(bias))
+    else:
+        p = softmax_rows(s)
+        dp = np.where(inv >= 0, dgates, 0.0)
+        ds = p * (dp - np.sum(p * dp, axis=1, keepdims=True))
     f = r["stats"]["f"]
     dq = np.broadcast_to(aux_grad * g["aux_alpha"] * E * f / T, (T, E))
     if g["score"] == "softmax":
@@ -716,8 +727,17 @@ def layer_backward(w, x, Wg, bias, W_gate, W_up, W_down, dout, aux_grad=1.0, log
         for j in range(K):
             if inv[t, j] >= 0:
                 dx[t] += dx_rows[inv[t, j]]
+    dWs = None
+    if g["n_shared"]:
+        Sg, Su, Sd = _np(Ws_gate), _np(Ws_up), _np(Ws_down)
+        dWs = (np.zeros_like(Sg), np.zeros_like(Su), np.zeros_like(Sd))
+        for i in range(g["n_shared"]):
+            dxs, dgs, dus, dds = expert_backward("swiglu", x, dout, Sg[i], Su[i], Sd[i])
+            dx += dxs
+            dWs[0][i], dWs[1][i], dWs[2][i] = dgs, dus, dds
     return dict(forward=r, dx=dx, dWg=ds.T @ x, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown,
-                dgates=dgates, dlogits=ds, dy_rows=dy)
+                dWs_gate=dWs[0] if dWs else None, dWs_up=dWs[1] if dWs else None,
+                dWs_down=dWs[2] if dWs else None, dgates=dgates, dlogits=ds, dy_rows=dy)
 
 
 # --------------------------------------------------------------------------

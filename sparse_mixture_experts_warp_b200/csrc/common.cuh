@@ -35,18 +35,19 @@ inline G counted(G grid) {
 // ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
 
 // route.cu
+// With ticket (an int in the scratch, zeroed here before the launch) and importance / entropy
+// given, the router's last CTA reduces the importance partials into them (fixed order).
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
-                                       float* logits, float* imp_partials, int* n_partials,
-                                       float* lpart, cudaStream_t s);
+                                       float* logits, float* imp_partials, float* lpart,
+                                       int* ticket, float* importance, float* entropy,
+                                       cudaStream_t s);
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, int* n_partials, float* lpart,
-                                        cudaStream_t s);
+                                        float* imp_partials, float* lpart, int* ticket,
+                                        float* importance, float* entropy, cudaStream_t s);
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s);
-cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
-                                     float* importance, float* entropy, cudaStream_t s);
 int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer (upper bound)
 bool router_uses_gemm(const moe_desc_t& d);
 size_t router_gemm_scratch_bytes(const moe_desc_t& d);   // partial logits of the GEMM router

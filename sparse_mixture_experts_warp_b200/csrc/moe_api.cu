@@ -101,6 +101,7 @@ size_t route_scratch(const moe_desc_t* d) {
   size_t b = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   if (d->select == MOE_EXPERT_CHOICE) b += up((size_t)d->E * d->T * sizeof(float));
   b += up(router_gemm_scratch_bytes(*d));
+  b += kAlign;                    // the router's ticket (last-CTA reduction)
   return b;
 }
 size_t permute_scratch(const moe_desc_t* d) {
@@ -304,18 +305,18 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
   const size_t pbytes = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   const size_t tbytes = d->select == MOE_EXPERT_CHOICE ? up((size_t)d->E * d->T * sizeof(float)) : 0;
   float* lpart = router_uses_gemm(*d) ? reinterpret_cast<float*>(sc + pbytes + tbytes) : nullptr;
-  int np = 0;
+  int* ticket = reinterpret_cast<int*>(sc + pbytes + tbytes + up(router_gemm_scratch_bytes(*d)));
   cudaError_t e;
   if (d->select == MOE_TOKEN_CHOICE) {
     e = launch_router_token_choice(*d, x, Wg, d->score == MOE_SCORE_SIGMOID ? sel_bias : nullptr,
-                                   expert_ids, gates, logits, partials, &np, lpart, s);
+                                   expert_ids, gates, logits, partials, lpart, ticket,
+                                   importance, entropy, s);
   } else {
     float* probsT = reinterpret_cast<float*>(sc + pbytes);
-    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, lpart, s);
+    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, lpart, ticket,
+                                    importance, entropy, s);
     if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
   }
-  if (e == cudaSuccess && (importance || entropy))
-    e = launch_importance_reduce(partials, np, d->E, d->T, importance, entropy, s);
   return cuda_status(e);
 }
 

@@ -37,7 +37,7 @@ def _rank_main(rank, world, port, out):
 def test_two_replicas_agree_on_the_slowest_time_and_job_throughput():
     world = 2
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.start_processes(_rank_main, args=(world, port, out), nprocs=world, join=True,
                            start_method="spawn")

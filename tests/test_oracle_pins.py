@@ -522,9 +522,33 @@ def test_group_limited_dropless_layer_is_dense_masked():
 # experts none) and [TINY] section 9 (task loss + weight x aux loss).  The backward is pinned
 # against central finite differences of the (separately pinned) forward oracle.
 
-def _loss(c, x, Wg, b, Wgate, Wup, Wdown, dout, aux_grad):
-    r = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown)
+def _loss(c, x, Wg, b, Wgate, Wup, Wdown, dout, aux_grad, Ws=(None, None, None)):
+    r = O.layer_forward(c, x, Wg, b, Wgate, Wup, Wdown, *Ws)
     return float(np.sum(dout * r["out"])) + aux_grad * r["stats"]["aux"], r["ids"]
+
+
+def _check_fd(c, params, grads, b, dout, aux_grad, rng, shared=()):
+    """Directional derivatives of the loss along 3 random directions per parameter, by
+    central differences, against the analytic gradients; the selection must not move."""
+    eps = 1e-6
+    names = ["x", "Wg", "Wgate", "Wup", "Wdown"]
+    for name, val in params.items():
+        if val is None:
+            continue
+        for _ in range(3):
+            v = rng.standard_normal(val.shape)
+            plus, minus = dict(params), dict(params)
+            plus[name], minus[name] = val + eps * v, val - eps * v
+            args_p = [plus[n] for n in names]
+            args_m = [minus[n] for n in names]
+            sp = tuple(plus.get(n) for n in shared) if shared else (None, None, None)
+            sm = tuple(minus.get(n) for n in shared) if shared else (None, None, None)
+            lp, ids_p = _loss(c, args_p[0], args_p[1], b, *args_p[2:], dout, aux_grad, sp)
+            lm, ids_m = _loss(c, args_m[0], args_m[1], b, *args_m[2:], dout, aux_grad, sm)
+            assert np.array_equal(ids_p, ids_m)                   # the selection did not move
+            fd = (lp - lm) / (2 * eps)
+            an = float(np.sum(grads[name] * v))
+            assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), (name, fd, an)
 
 
 @pytest.mark.parametrize("kw", [
@@ -598,3 +622,73 @@ def test_backward_single_expert_is_the_dense_ffn_backward():
     np.testing.assert_allclose(gr["dx"], da @ Wgate[0] + (dh * O.silu(a)) @ Wup[0], rtol=1e-12,
                                atol=1e-13)
     assert np.all(gr["dWg"] == 0.0)
+
+
+def test_backward_shared_experts_match_finite_differences():
+    # DeepSeek-style layer: sigmoid top-3 with a selection bias plus two always-on shared
+    # experts ([CMP] "shared direct path", weight 1); the shared weights get gradients too
+    c = cfg(T=9, D=6, E=6, F=4, k=3, score="sigmoid", n_shared=2, F_shared=5, aux_alpha=0.05)
+    rng = np.random.default_rng(44)
+    x, Wg, b, Wgate, Wup, Wdown = rand_layer(rng, c, with_bias=True)
+    Sg = rng.standard_normal((2, 5, 6)) / math.sqrt(6)
+    Su = rng.standard_normal((2, 5, 6)) / math.sqrt(6)
+    Sd = rng.standard_normal((2, 6, 5)) / math.sqrt(5)
+    dout = rng.standard_normal((c["T"], c["D"]))
+    gr = O.layer_backward(c, x, Wg, b, Wgate, Wup, Wdown, dout, 0.7, Ws_gate=Sg, Ws_up=Su,
+                          Ws_down=Sd)
+    params = {"x": x, "Wg": Wg, "Wgate": Wgate, "Wup": Wup, "Wdown": Wdown, "Sg": Sg,
+              "Su": Su, "Sd": Sd}
+    grads = {"x": gr["dx"], "Wg": gr["dWg"], "Wgate": gr["dW_gate"], "Wup": gr["dW_up"],
+             "Wdown": gr["dW_down"], "Sg": gr["dWs_gate"], "Su": gr["dWs_up"],
+             "Sd": gr["dWs_down"]}
+    _check_fd(c, params, grads, b, dout, 0.7, rng, shared=("Sg", "Su", "Sd"))
+
+
+def test_backward_shared_expert_alone_is_the_dense_ffn_backward():
+    # the shared expert's weight gradients are those of the dense SwiGLU FFN on all tokens
+    c = cfg(T=7, D=5, E=3, F=4, k=1, n_shared=1, F_shared=3)
+    rng = np.random.default_rng(45)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    Sg = rng.standard_normal((1, 3, 5))
+    Su = rng.standard_normal((1, 3, 5))
+    Sd = rng.standard_normal((1, 5, 3))
+    dout = rng.standard_normal((7, 5))
+    gr = O.layer_backward(c, x, Wg, None, Wgate, Wup, Wdown, dout, 0.0, Ws_gate=Sg, Ws_up=Su,
+                          Ws_down=Sd)
+    a, u = x @ Sg[0].T, x @ Su[0].T
+    np.testing.assert_allclose(gr["dWs_down"][0], dout.T @ (O.silu(a) * u), rtol=1e-12)
+    dh = dout @ Sd[0]
+    np.testing.assert_allclose(gr["dWs_up"][0], (dh * O.silu(a)).T @ x, rtol=1e-12)
+
+
+@pytest.mark.parametrize("act", ["swiglu", "relu"])
+def test_backward_expert_choice_matches_finite_differences(act):
+    # expert choice: each expert keeps its top-c tokens (held fixed); the merge weight of a
+    # picked (token, expert) is its softmax probability
+    c = cfg(T=10, D=6, E=4, F=4, k=0, c=4, select="expert", act=act, aux_alpha=0.05)
+    rng = np.random.default_rng(46)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    if act != "swiglu":
+        Wgate = None
+    dout = rng.standard_normal((c["T"], c["D"]))
+    gr = O.layer_backward(c, x, Wg, None, Wgate, Wup, Wdown, dout, 0.7)
+    inv = np.asarray(gr["forward"]["inv"]).reshape(10, 4)
+    assert (inv < 0).any() and (inv >= 0).sum(axis=1).max() > 1   # unpicked and multi-picked
+    params = {"x": x, "Wg": Wg, "Wgate": Wgate, "Wup": Wup, "Wdown": Wdown}
+    grads = {"x": gr["dx"], "Wg": gr["dWg"], "Wgate": gr["dW_gate"], "Wup": gr["dW_up"],
+             "Wdown": gr["dW_down"]}
+    _check_fd(c, params, grads, None, dout, 0.7, rng)
+
+
+def test_backward_expert_choice_unpicked_token_gets_router_gradient_only():
+    # a token no expert picked contributes nothing to out: its dx is the router term ds W_g
+    # alone, and with aux_grad = 0 its ds is zero (no merge weight of its own)
+    c = cfg(T=12, D=5, E=3, F=4, k=0, c=3, select="expert")
+    rng = np.random.default_rng(47)
+    x, Wg, _, Wgate, Wup, Wdown = rand_layer(rng, c)
+    dout = rng.standard_normal((12, 5))
+    gr = O.layer_backward(c, x, Wg, None, Wgate, Wup, Wdown, dout, 0.0)
+    inv = np.asarray(gr["forward"]["inv"]).reshape(12, 3)
+    un = np.nonzero((inv < 0).all(axis=1))[0]
+    assert len(un) > 0
+    assert np.all(gr["dlogits"][un] == 0.0) and np.all(gr["dx"][un] == 0.0)
