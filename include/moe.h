@@ -277,6 +277,16 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
                                const void* Ws_down, void* out, void* ws, size_t ws_bytes,
                                moe_stream_t stream);
 
+/* Shared experts' weights and gradient outputs for moe_layer_backward_ex (see below). */
+typedef struct moe_bwd_shared {
+    const void* Ws_gate;   /* [S, Fs, D] bf16, as given to moe_layer_forward */
+    const void* Ws_up;     /* [S, Fs, D] */
+    const void* Ws_down;   /* [S, D, Fs] */
+    float* dWs_gate;       /* [S, Fs, D] fp32, overwritten */
+    float* dWs_up;         /* [S, Fs, D] fp32, overwritten */
+    float* dWs_down;       /* [S, D, Fs] fp32, overwritten */
+} moe_bwd_shared_t;
+
 /* Backward of moe_layer_forward with the selection held fixed ("Top-k 路由" section
  * "門控網路的梯度流": the selected experts' gate scores carry the gradient, unselected experts
  * none; Tiny MoE section 9: task loss + weight x aux loss, fixed expert indices).
@@ -290,7 +300,10 @@ moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void
  *   flags: MOE_BWD_PREACT_SAVED when moe_layer_forward_train wrote the expert
  *   pre-activations into this bwd_ws for this forward (the backward then skips recomputing
  *   them with a third up projection); 0 otherwise.
- * Limits: bf16, token choice, no shared experts (MOE_ERR_UNSUPPORTED otherwise). */
+ * Token choice or expert choice (the merge weight of a picked (token, expert) pair is its
+ * softmax probability, so its logit gradient is the softmax Jacobian applied to the pairs' dg;
+ * the picked sets are held fixed like the top-k).  Layers with shared experts use
+ * moe_layer_backward_ex.  Limits: bf16 (MOE_ERR_UNSUPPORTED otherwise). */
 enum { MOE_BWD_PREACT_SAVED = 1 };
 moe_status_t moe_backward_workspace_size(const moe_desc_t* desc, size_t* bytes);
 moe_status_t moe_layer_backward(const moe_desc_t* desc, const void* x, const void* Wg,
@@ -300,10 +313,26 @@ moe_status_t moe_layer_backward(const moe_desc_t* desc, const void* x, const voi
                                 float* dW_up, float* dW_down, void* bwd_ws,
                                 size_t bwd_ws_bytes, int32_t flags, moe_stream_t stream);
 
+/* moe_layer_backward for any layer, shared experts included ("别只比较 Top-k" family table,
+ * DeepSeek rows: always-on shared experts on the direct path with weight 1, so each sees dout on
+ * every token).  `shared` (NULL when n_shared = 0) holds their weights and receives their
+ * gradients: dWs_down[i] = dout^T h_i, dWs_gate[i] = da_i^T x, dWs_up[i] = db_i^T x, and their
+ * input gradients are added into dx.  Their pre-activations are recomputed.  The other
+ * arguments, results and limits are those of moe_layer_backward; bwd_ws is
+ * moe_backward_workspace_size bytes of the same desc. */
+moe_status_t moe_layer_backward_ex(const moe_desc_t* desc, const void* x, const void* Wg,
+                                   const void* W_gate, const void* W_up, const void* W_down,
+                                   const moe_bwd_shared_t* shared, const void* dout,
+                                   float aux_grad, void* fwd_ws, size_t fwd_ws_bytes, void* dx,
+                                   float* dWg, float* dW_gate, float* dW_up, float* dW_down,
+                                   void* bwd_ws, size_t bwd_ws_bytes, int32_t flags,
+                                   moe_stream_t stream);
+
 /* moe_layer_forward (same limits as moe_layer_backward) that also stores the routed expert
  * pre-activations (SwiGLU gate and up, or the ReLU/GELU input) into bwd_ws, for a following
  * moe_layer_backward with MOE_BWD_PREACT_SAVED.  Results and the workspace `ws` are those of
- * moe_layer_forward. */
+ * moe_layer_forward.  Layers with shared experts: MOE_ERR_UNSUPPORTED (run moe_layer_forward,
+ * then moe_layer_backward_ex with flags 0). */
 moe_status_t moe_layer_forward_train(const moe_desc_t* desc, const void* x, const void* Wg,
                                      const float* sel_bias, const void* W_gate,
                                      const void* W_up, const void* W_down, void* out, void* ws,

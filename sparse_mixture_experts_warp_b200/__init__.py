@@ -22,7 +22,8 @@ __all__ = [
     "header_functions", "status_string", "rows_max", "capacity", "scratch_size",
     "workspace_size", "layer_views", "moe_route", "moe_permute", "moe_expert_up",
     "moe_expert_down", "moe_expert_ffn", "moe_expert_up_ws", "moe_expert_down_ws",
-    "moe_permute_noalloc", "moe_combine", "moe_balance_stats",
+    "moe_permute_noalloc", "moe_combine", "moe_balance_stats", "moe_layer_backward_ex",
+    "MoeBwdShared",
     "moe_layer_forward", "get_device_error", "empty_scratch", "empty_workspace",
 ]
 
@@ -69,6 +70,12 @@ class MoeLayerViews(ctypes.Structure):
                 ("scratch_bytes", ctypes.c_size_t), ("rows", ctypes.c_int64)]
 
 
+class MoeBwdShared(ctypes.Structure):
+    _fields_ = [("Ws_gate", ctypes.c_void_p), ("Ws_up", ctypes.c_void_p),
+                ("Ws_down", ctypes.c_void_p), ("dWs_gate", ctypes.c_void_p),
+                ("dWs_up", ctypes.c_void_p), ("dWs_down", ctypes.c_void_p)]
+
+
 class MoeError(RuntimeError):
     def __init__(self, fn, status):
         self.status = status
@@ -106,6 +113,9 @@ _SIGS = {
     "moe_backward_workspace_size": ([_DP, ctypes.POINTER(_SZ)], ctypes.c_int),
     "moe_layer_backward": ([_DP, _P, _P, _P, _P, _P, _P, ctypes.c_float, _P, _SZ, _P, _P, _P,
                             _P, _P, _P, _SZ, _I32, _P], ctypes.c_int),
+    "moe_layer_backward_ex": ([_DP, _P, _P, _P, _P, _P, ctypes.POINTER(MoeBwdShared), _P,
+                               ctypes.c_float, _P, _SZ, _P, _P, _P, _P, _P, _P, _SZ, _I32, _P],
+                              ctypes.c_int),
     "moe_layer_forward_train": ([_DP, _P, _P, _P, _P, _P, _P, _P, _P, _SZ, _P, _SZ, _P],
                                 ctypes.c_int),
     "moe_get_device_error": ([_P, ctypes.POINTER(_I32)], ctypes.c_int),
@@ -365,6 +375,20 @@ def moe_layer_backward(d, x, Wg, W_gate, W_up, W_down, dout, aux_grad, fwd_ws, d
         ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(W_gate), _ptr(W_up), _ptr(W_down), _ptr(dout),
         float(aux_grad), _ptr(fwd_ws), fwd_ws.numel(), _ptr(dx), _ptr(dWg), _ptr(dW_gate),
         _ptr(dW_up), _ptr(dW_down), _ptr(bwd_ws), bwd_ws.numel(), int(flags), _stream(stream)))
+
+
+def moe_layer_backward_ex(d, x, Wg, W_gate, W_up, W_down, shared, dout, aux_grad, fwd_ws, dx,
+                          dWg, dW_gate, dW_up, dW_down, bwd_ws, stream=None, flags=0):
+    """moe_layer_backward for any layer; `shared` = (Ws_gate, Ws_up, Ws_down, dWs_gate, dWs_up,
+    dWs_down) tensors, or None without shared experts."""
+    sh = None
+    if shared is not None:
+        sh = MoeBwdShared(*[_ptr(t) for t in shared])
+    _check("moe_layer_backward_ex", lib().moe_layer_backward_ex(
+        ctypes.byref(d), _ptr(x), _ptr(Wg), _ptr(W_gate), _ptr(W_up), _ptr(W_down),
+        ctypes.byref(sh) if sh is not None else None, _ptr(dout), float(aux_grad), _ptr(fwd_ws),
+        fwd_ws.numel(), _ptr(dx), _ptr(dWg), _ptr(dW_gate), _ptr(dW_up), _ptr(dW_down),
+        _ptr(bwd_ws), bwd_ws.numel(), int(flags), _stream(stream)))
 
 
 def moe_layer_forward_train(d, x, Wg, sel_bias, W_gate, W_up, W_down, out, ws, bwd_ws,

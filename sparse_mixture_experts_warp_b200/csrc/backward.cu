@@ -1,4 +1,5 @@
-// Backward pass of the MoE layer with the selection held fixed (bf16 operands, fp32 math).
+// Backward pass of the MoE layer with the selection held fixed (bf16 operands, fp32 math):
+// token choice or expert choice, with or without shared experts.
 //
 // "Top-k 路由（Top-k Routing）" (compassingai), "門控網路的梯度流": the discrete top-k is not
 // differentiated; the selected experts' gate scores carry the gradient (softmax normalised over
@@ -93,12 +94,13 @@ __global__ void gather_dy_kernel(const uint4* __restrict__ dout, const uint4* __
 
 // Activation backward on the executed rows, 8 features per thread.
 //   SwiGLU (ACT 0): gu row = blocks of [128 gate | 128 up] per 128 features (pitch ldg);
-//                   dAB row = [da (F) | db (F)].
+//                   dAB row = [da (F) | db (F)]; with h_out also h = SiLU(a) b (bf16 [rows, F]).
 //   ReLU (1), GELU (2): gu = z [rows, F]; dAB = dz [rows, F].
 template <int ACT>
 __global__ void act_backward_kernel(const uint4* __restrict__ dH, const __nv_bfloat16* __restrict__ gu,
                                     const int32_t* __restrict__ offsets, int E, int F,
-                                    int64_t ldg, int64_t rows_max, __nv_bfloat16* __restrict__ dAB) {
+                                    int64_t ldg, int64_t rows_max, __nv_bfloat16* __restrict__ dAB,
+                                    __nv_bfloat16* __restrict__ h_out) {
   const int nv = F / 8;
   const int64_t rows = min((int64_t)offsets[E], rows_max);
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < rows * nv;
@@ -109,7 +111,7 @@ __global__ void act_backward_kernel(const uint4* __restrict__ dH, const __nv_bfl
     unpack8(dH[i], dh);
     if (ACT == 0) {
       const int64_t gcol = (int64_t)(f / 128) * 256 + (f % 128);
-      float a[8], b[8], da[8], db[8];
+      float a[8], b[8], da[8], db[8], hv[8];
       unpack8(*reinterpret_cast<const uint4*>(gu + r * ldg + gcol), a);
       unpack8(*reinterpret_cast<const uint4*>(gu + r * ldg + gcol + 128), b);
 #pragma unroll
@@ -117,9 +119,11 @@ __global__ void act_backward_kernel(const uint4* __restrict__ dH, const __nv_bfl
         const float s = 1.0f / (1.0f + expf(-a[k]));
         da[k] = dh[k] * b[k] * (s * (1.0f + a[k] * (1.0f - s)));
         db[k] = dh[k] * a[k] * s;
+        hv[k] = a[k] * s * b[k];
       }
       *reinterpret_cast<uint4*>(dAB + r * 2 * F + f) = pack8(da);
       *reinterpret_cast<uint4*>(dAB + r * 2 * F + F + f) = pack8(db);
+      if (h_out) *reinterpret_cast<uint4*>(h_out + r * F + f) = pack8(hv);
     } else {
       float z[8], dz[8];
       unpack8(*reinterpret_cast<const uint4*>(gu + r * ldg + f), z);
@@ -200,7 +204,9 @@ transpose64_kernel(const __nv_bfloat16* __restrict__ src, int64_t src_bstride, i
 }
 
 // One warp per token: ds[t, :] = dL/ds from the merge-weight gradients (selection fixed) plus
-// the balance-loss term.  Lane l holds experts l + 32 i.
+// the balance-loss term.  Lane l holds experts l + 32 i.  Under expert choice (ec) the merge
+// weight of a picked (token, expert) pair is the softmax probability itself: the raw-gate form
+// with K = E slots, slot j being expert j ("Top-k 路由" Token-Choice vs Expert-Choice table).
 constexpr int kMaxEL = 8;   // E <= 256
 __global__ void router_backward_kernel(const float* __restrict__ logits,
                                        const int32_t* __restrict__ ids,
@@ -208,7 +214,7 @@ __global__ void router_backward_kernel(const float* __restrict__ logits,
                                        const float* __restrict__ dgates,
                                        const int32_t* __restrict__ inv,
                                        const float* __restrict__ f, int T, int E, int K,
-                                       int sigmoid_score, int renorm, float aux_coef,
+                                       int sigmoid_score, int renorm, int ec, float aux_coef,
                                        float* __restrict__ ds) {
   const int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
@@ -250,7 +256,7 @@ __global__ void router_backward_kernel(const float* __restrict__ logits,
     const int64_t a = (int64_t)t * K + j;
     const float dg = inv[a] >= 0 ? dgates[a] : 0.f;
     dot += gates[a] * dg;
-    const int e = ids[a];
+    const int e = ec ? j : ids[a];           // expert choice: slot j of a token is expert j
 #pragma unroll
     for (int i = 0; i < kMaxEL; ++i)
       if (lane + 32 * i == e) selw += w[i];
@@ -259,7 +265,7 @@ __global__ void router_backward_kernel(const float* __restrict__ logits,
   for (int j = 0; j < K; ++j) {
     const int64_t a = (int64_t)t * K + j;
     const float dg = inv[a] >= 0 ? dgates[a] : 0.f;
-    const int e = ids[a];
+    const int e = ec ? j : ids[a];
 #pragma unroll
     for (int i = 0; i < kMaxEL; ++i) {
       if (lane + 32 * i != e) continue;
@@ -312,11 +318,12 @@ __global__ void router_backward_kernel(const float* __restrict__ logits,
   }
 }
 
-// dx[t] = sum_j dX[inv[t, j]] (fixed slot order) + sum_e ds[t, e] W_g[e]; one block per token,
-// 8 columns per thread.
+// dx[t] = sum_j dX[inv[t, j]] (fixed slot order) + sum_e ds[t, e] W_g[e] + sum_i dXs[i][t] (the
+// shared experts' input gradients, when given); one block per token, 8 columns per thread.
 __global__ void dx_kernel(const uint4* __restrict__ dX, const int32_t* __restrict__ inv,
                           const float* __restrict__ ds, const uint4* __restrict__ Wg, int T,
-                          int D, int E, int K, uint4* __restrict__ dx) {
+                          int D, int E, int K, const uint4* __restrict__ dXs, int n_add,
+                          uint4* __restrict__ dx) {
   extern __shared__ float s_ds[];
   const int t = blockIdx.x;
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_ds[e] = ds[(int64_t)t * E + e];
@@ -338,6 +345,12 @@ __global__ void dx_kernel(const uint4* __restrict__ dX, const int32_t* __restric
       const float c = s_ds[e];
 #pragma unroll
       for (int i = 0; i < 8; ++i) acc[i] += c * wv[i];
+    }
+    for (int j = 0; j < n_add; ++j) {        // shared experts' input gradients
+      float a[8];
+      unpack8(dXs[((int64_t)j * T + t) * nv + v], a);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) acc[i] += a[i];
     }
     dx[(int64_t)t * nv + v] = pack8(acc);
   }
@@ -407,18 +420,22 @@ cudaError_t launch_gather_dy(const void* dout, const void* y, const int32_t* row
 
 cudaError_t launch_act_backward(int act, const void* dH, const void* gu, int64_t ldg,
                                 const int32_t* offsets, int E, int F, int64_t rows_max,
-                                void* dAB, cudaStream_t s) {
+                                void* dAB, cudaStream_t s, void* h_out) {
   if (rows_max <= 0) return cudaSuccess;
   const int grid = grid_of(rows_max * (F / 8), 256);
   const uint4* h = static_cast<const uint4*>(dH);
   const __nv_bfloat16* g = static_cast<const __nv_bfloat16*>(gu);
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(dAB);
+  __nv_bfloat16* ho = static_cast<__nv_bfloat16*>(h_out);
   if (act == MOE_ACT_SWIGLU)
-    act_backward_kernel<0><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o);
+    act_backward_kernel<0><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o,
+                                                         ho);
   else if (act == MOE_ACT_RELU)
-    act_backward_kernel<1><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o);
+    act_backward_kernel<1><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o,
+                                                         nullptr);
   else
-    act_backward_kernel<2><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o);
+    act_backward_kernel<2><<<counted(grid), 256, 0, s>>>(h, g, offsets, E, F, ldg, rows_max, o,
+                                                         nullptr);
   return cudaGetLastError();
 }
 
@@ -450,18 +467,21 @@ cudaError_t launch_router_backward(const moe_desc_t& d, const float* logits, con
   if (d.T <= 0) return cudaSuccess;
   const int warps = 8;
   const float coef = aux_grad * d.aux_alpha * (float)d.E / (float)d.T;
+  const bool ec = d.select == MOE_EXPERT_CHOICE;
   router_backward_kernel<<<counted((d.T + warps - 1) / warps), warps * 32, 0, s>>>(
-      logits, ids, gates, dgates, inv, f, d.T, d.E, d.k, d.score == MOE_SCORE_SIGMOID ? 1 : 0,
-      d.gate == MOE_GATE_RENORM ? 1 : 0, coef, ds);
+      logits, ids, gates, dgates, inv, f, d.T, d.E, ec ? d.E : d.k,
+      d.score == MOE_SCORE_SIGMOID ? 1 : 0, (!ec && d.gate == MOE_GATE_RENORM) ? 1 : 0,
+      ec ? 1 : 0, coef, ds);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dx(const void* dX, const int32_t* inv, const float* ds, const void* Wg, int T,
-                      int D, int E, int K, void* dx, cudaStream_t s) {
+                      int D, int E, int K, void* dx, cudaStream_t s, const void* dXs,
+                      int n_add) {
   if (T <= 0) return cudaSuccess;
   dx_kernel<<<counted(T), 256, E * sizeof(float), s>>>(
       static_cast<const uint4*>(dX), inv, ds, static_cast<const uint4*>(Wg), T, D, E, K,
-      static_cast<uint4*>(dx));
+      static_cast<const uint4*>(dXs), dXs ? n_add : 0, static_cast<uint4*>(dx));
   return cudaGetLastError();
 }
 

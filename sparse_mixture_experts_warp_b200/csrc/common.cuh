@@ -116,7 +116,7 @@ cudaError_t launch_gather_dy(const void* dout, const void* y, const int32_t* row
                              int64_t rows_max, void* dY, float* dgates, cudaStream_t s);
 cudaError_t launch_act_backward(int act, const void* dH, const void* gu, int64_t ldg,
                                 const int32_t* offsets, int E, int F, int64_t rows_max,
-                                void* dAB, cudaStream_t s);
+                                void* dAB, cudaStream_t s, void* h_out = nullptr);
 cudaError_t launch_transpose(const void* src, int64_t src_bstride, int R, int C, int64_t lds,
                              void* dst, int64_t dst_bstride, int64_t ldd, int dcol0, int batch,
                              cudaStream_t s);
@@ -127,7 +127,8 @@ cudaError_t launch_router_backward(const moe_desc_t& d, const float* logits, con
                                    const float* gates, const float* dgates, const int32_t* inv,
                                    const float* f, float aux_grad, float* ds, cudaStream_t s);
 cudaError_t launch_dx(const void* dX, const int32_t* inv, const float* ds, const void* Wg, int T,
-                      int D, int E, int K, void* dx, cudaStream_t s);
+                      int D, int E, int K, void* dx, cudaStream_t s, const void* dXs = nullptr,
+                      int n_add = 0);
 cudaError_t launch_dwg(const float* ds, const void* x, int T, int D, int E, float* part,
                        float* dWg, cudaStream_t s);
 

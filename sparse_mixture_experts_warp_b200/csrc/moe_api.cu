@@ -585,6 +585,10 @@ struct BwdViews {
   void *dY, *gu, *dH, *dAB, *dXp, *WdT, *WguT, *dYT, *hT, *xpT, *dABT;
   float *dgates, *ds, *dwg_part;
   int64_t ldg, nab, pad_cols;
+  // shared experts (n_shared > 0): one group of all T tokens each
+  int32_t* pad_off_s;
+  void *gu_s, *dH_s, *dAB_s, *h_s, *dXs, *doutT, *xT, *hT_s, *dABT_s;
+  int64_t ldg_s, pad_cols_s;
 };
 
 bool bwd_weight_transpose() {
@@ -598,8 +602,7 @@ bool bwd_weight_transpose() {
 moe_status_t check_backward(const moe_desc_t* d) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
-  if (d->dtype != MOE_BF16 || d->select != MOE_TOKEN_CHOICE || d->n_shared > 0)
-    return MOE_ERR_UNSUPPORTED;
+  if (d->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (d->E > 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
@@ -617,9 +620,10 @@ size_t carve_bwd(const moe_desc_t* d, uint8_t* base, BwdViews* v) {
     off += up(bytes);
     return p;
   };
+  const int64_t K = d->select == MOE_EXPERT_CHOICE ? E : d->k;
   v->pad_off = static_cast<int32_t*>(take((E + 1) * 4));
   v->dY = take(A * D * 2);
-  v->dgates = static_cast<float*>(take(T * d->k * 4));
+  v->dgates = static_cast<float*>(take(T * K * 4));
   v->gu = take(A * v->ldg * 2);
   v->dH = take(A * F * 2);
   v->dAB = take(A * v->nab * 2);
@@ -633,7 +637,73 @@ size_t carve_bwd(const moe_desc_t* d, uint8_t* base, BwdViews* v) {
   v->xpT = take(D * v->pad_cols * 2);
   v->dABT = take(v->nab * v->pad_cols * 2);
   v->dwg_part = static_cast<float*>(take((size_t)backward_dwg_chunks(d->T) * E * D * 4));
+  const int64_t S = d->n_shared, Fs = d->F_shared;
+  v->ldg_s = S ? (Fs + 127) / 128 * 256 : 0;
+  v->pad_cols_s = S ? (T + 63) / 64 * 64 : 0;
+  const int64_t pcs = v->pad_cols_s;
+  v->pad_off_s = static_cast<int32_t*>(take(S ? 2 * 4 : 0));
+  v->gu_s = take(S ? T * v->ldg_s * 2 : 0);
+  v->dH_s = take(S ? T * Fs * 2 : 0);
+  v->dAB_s = take(S ? T * 2 * Fs * 2 : 0);
+  v->h_s = take(S ? T * Fs * 2 : 0);
+  v->dXs = take(S * T * D * 2);
+  v->doutT = take(S ? D * pcs * 2 : 0);
+  v->xT = take(S ? D * pcs * 2 : 0);
+  v->hT_s = take(S ? Fs * pcs * 2 : 0);
+  v->dABT_s = take(S ? 2 * Fs * pcs * 2 : 0);
   return off;
+}
+
+// The shared experts' backward ("别只比较 Top-k" family table, DeepSeek rows: always-on shared
+// experts on the direct path, weight 1): for expert i, with the recomputed pre-activations
+// a | b = x [Ws_gate[i] ; Ws_up[i]]^T, dH = dout Ws_down[i], [da | db] and h from the SwiGLU
+// derivative, dXs[i] = [da | db] [Ws_gate[i] ; Ws_up[i]], dWs_down[i] = dout^T h,
+// dWs_gate[i] = da^T x, dWs_up[i] = db^T x (fp32, groups along K of one group).
+cudaError_t shared_backward(const moe_desc_t* d, const moe_layer_views_t& v, const BwdViews& b,
+                            const void* x, const moe_bwd_shared_t* sh, const void* dout,
+                            cudaStream_t s) {
+  const int T = d->T, D = d->D, Fs = d->F_shared, S = d->n_shared;
+  const int64_t pcs = b.pad_cols_s;
+  const int64_t wst = (int64_t)Fs * D;           // elements per shared weight matrix
+  cudaError_t e = launch_pad_offsets(v.shared_offsets, 1, b.pad_off_s, s);
+  if (e == cudaSuccess)
+    e = launch_transpose_pad(dout, D, D, v.shared_offsets, b.pad_off_s, 1, pcs, b.doutT, pcs, s);
+  if (e == cudaSuccess)
+    e = launch_transpose_pad(x, D, D, v.shared_offsets, b.pad_off_s, 1, pcs, b.xT, pcs, s);
+  for (int i = 0; i < S && e == cudaSuccess; ++i) {
+    const __nv_bfloat16* wg = static_cast<const __nv_bfloat16*>(sh->Ws_gate) + i * wst;
+    const __nv_bfloat16* wu = static_cast<const __nv_bfloat16*>(sh->Ws_up) + i * wst;
+    const __nv_bfloat16* wd = static_cast<const __nv_bfloat16*>(sh->Ws_down) + i * wst;
+    void* dxs = static_cast<__nv_bfloat16*>(b.dXs) + (int64_t)i * T * D;
+    e = launch_grouped_gemm_bf16(EPI_RAW, x, T, D, wg, wu, 1, Fs, v.shared_offsets, b.gu_s, s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_bf16_bmn(dout, T, D, wd, nullptr, D / 64, D, 1, Fs,
+                                       v.shared_offsets, b.dH_s, s);
+    if (e == cudaSuccess)
+      e = launch_act_backward(MOE_ACT_SWIGLU, b.dH_s, b.gu_s, b.ldg_s, v.shared_offsets, 1, Fs,
+                              T, b.dAB_s, s, b.h_s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_bf16_bmn(b.dAB_s, T, 2 * Fs, wg, wu, Fs / 64, Fs, 1, D,
+                                       v.shared_offsets, dxs, s);
+    if (e == cudaSuccess)
+      e = launch_transpose_pad(b.h_s, Fs, Fs, v.shared_offsets, b.pad_off_s, 1, pcs, b.hT_s, pcs,
+                               s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_kgroups_f32(b.doutT, D, b.hT_s, Fs, 1, b.pad_off_s, pcs,
+                                          sh->dWs_down + i * wst, s);
+    if (e == cudaSuccess)
+      e = launch_transpose_pad(b.dAB_s, 2 * Fs, 2 * Fs, v.shared_offsets, b.pad_off_s, 1, pcs,
+                               b.dABT_s, pcs, s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_kgroups_f32(b.dABT_s, Fs, b.xT, D, 1, b.pad_off_s, pcs,
+                                          sh->dWs_gate + i * wst, s);
+    if (e == cudaSuccess)
+      e = launch_grouped_gemm_kgroups_f32(static_cast<const __nv_bfloat16*>(b.dABT_s) +
+                                              (int64_t)Fs * pcs,
+                                          Fs, b.xT, D, 1, b.pad_off_s, pcs,
+                                          sh->dWs_up + i * wst, s);
+  }
+  return e;
 }
 
 }  // namespace
@@ -654,6 +724,7 @@ moe_status_t moe_layer_forward_train(const moe_desc_t* d, const void* x, const v
                                      moe_stream_t stream) {
   moe_status_t st = check_backward(d);
   if (st != MOE_OK) return st;
+  if (d->n_shared > 0) return MOE_ERR_UNSUPPORTED;   // use moe_layer_forward, flags 0
   BwdViews b;
   if (!bwd_ws || bwd_ws_bytes < carve_bwd(d, nullptr, &b)) return MOE_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
@@ -668,8 +739,30 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
                                 size_t fwd_ws_bytes, void* dx, float* dWg, float* dW_gate,
                                 float* dW_up, float* dW_down, void* bwd_ws,
                                 size_t bwd_ws_bytes, int32_t flags, moe_stream_t stream) {
+  return moe_layer_backward_ex(d, x, Wg, W_gate, W_up, W_down, nullptr, dout, aux_grad, fwd_ws,
+                               fwd_ws_bytes, dx, dWg, dW_gate, dW_up, dW_down, bwd_ws,
+                               bwd_ws_bytes, flags, stream);
+}
+
+moe_status_t moe_layer_backward_ex(const moe_desc_t* d, const void* x, const void* Wg,
+                                   const void* W_gate, const void* W_up, const void* W_down,
+                                   const moe_bwd_shared_t* shared, const void* dout,
+                                   float aux_grad, void* fwd_ws, size_t fwd_ws_bytes, void* dx,
+                                   float* dWg, float* dW_gate, float* dW_up, float* dW_down,
+                                   void* bwd_ws, size_t bwd_ws_bytes, int32_t flags,
+                                   moe_stream_t stream) {
   moe_status_t st = check_backward(d);
   if (st != MOE_OK) return st;
+  const int S = d->n_shared;
+  if (S > 0) {
+    if (!shared || !shared->Ws_gate || !shared->Ws_up || !shared->Ws_down ||
+        !shared->dWs_gate || !shared->dWs_up || !shared->dWs_down)
+      return MOE_ERR_INVALID_ARG;
+    for (const void* p : {shared->Ws_gate, shared->Ws_up, shared->Ws_down,
+                          (const void*)shared->dWs_gate, (const void*)shared->dWs_up,
+                          (const void*)shared->dWs_down})
+      if (!is_aligned16(p)) return MOE_ERR_INVALID_ARG;
+  }
   moe_layer_views_t v;
   st = moe_layer_views(d, fwd_ws, fwd_ws_bytes, &v);
   if (st != MOE_OK) return st;
@@ -688,15 +781,21 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
   if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
   carve_bwd(d, static_cast<uint8_t*>(bwd_ws), &b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  const int T = d->T, D = d->D, E = d->E, F = d->F, K = d->k;
+  const int T = d->T, D = d->D, E = d->E, F = d->F;
+  const int K = d->select == MOE_EXPERT_CHOICE ? E : d->k;
   const int64_t A = v.rows;
   const int nab = (int)b.nab;
+  const int Fs = d->F_shared;
   if (T == 0) {
     // no tokens: every gradient is zero
     cudaError_t e = cudaMemsetAsync(dWg, 0, (size_t)E * D * 4, s);
     if (e == cudaSuccess && glu) e = cudaMemsetAsync(dW_gate, 0, (size_t)E * F * D * 4, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dW_up, 0, (size_t)E * F * D * 4, s);
     if (e == cudaSuccess) e = cudaMemsetAsync(dW_down, 0, (size_t)E * D * F * 4, s);
+    const size_t sb = (size_t)S * Fs * D * 4;
+    if (e == cudaSuccess && S) e = cudaMemsetAsync(shared->dWs_gate, 0, sb, s);
+    if (e == cudaSuccess && S) e = cudaMemsetAsync(shared->dWs_up, 0, sb, s);
+    if (e == cudaSuccess && S) e = cudaMemsetAsync(shared->dWs_down, 0, sb, s);
     return cuda_status(e);
   }
   cudaError_t e = launch_pad_offsets(v.offsets, E, b.pad_off, s);
@@ -744,7 +843,12 @@ moe_status_t moe_layer_backward(const moe_desc_t* d, const void* x, const void* 
   if (e == cudaSuccess)
     e = launch_router_backward(*d, v.logits, v.expert_ids, v.gates, b.dgates, v.inv, v.f,
                                aux_grad, b.ds, s);
-  if (e == cudaSuccess) e = launch_dx(b.dXp, v.inv, b.ds, Wg, T, D, E, K, dx, s);
+  // shared experts: one group of all T tokens each, weight 1, so dY_s = dout; their input
+  // gradients dXs[i] go into dx with the routed ones
+  if (e == cudaSuccess && S > 0)
+    e = shared_backward(d, v, b, x, shared, dout, s);
+  if (e == cudaSuccess)
+    e = launch_dx(b.dXp, v.inv, b.ds, Wg, T, D, E, K, dx, s, S > 0 ? b.dXs : nullptr, S);
   if (e == cudaSuccess) e = launch_dwg(b.ds, x, T, D, E, b.dwg_part, dWg, s);
   // weight gradients: groups along K over the experts' row blocks, transposed and padded
   const int64_t pc = b.pad_cols;

@@ -157,10 +157,18 @@ def test_header_entry_points_cite_the_pages():
 def test_backward_validation_before_launch():
     v = ctypes.c_size_t()
     L = M.lib()
-    # bf16 token choice without shared experts only
-    for kw, st in ((dict(dtype=0), 2), (dict(select=1, c=8), 2), (dict(n_shared=1, F_shared=64), 2),
+    # bf16 layers: token choice or expert choice, with or without shared experts
+    for kw, st in ((dict(dtype=0), 2), (dict(select=1, c=8), 0), (dict(n_shared=1, F_shared=64), 0),
                    (dict(k=0), 1)):
         assert L.moe_backward_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == st, kw
+    # shared experts need moe_layer_backward_ex's weights (moe_layer_backward passes none) and
+    # the plain forward (moe_layer_forward_train does not run them)
+    sh = _bad(n_shared=1, F_shared=64)
+    p = 0x10000
+    assert L.moe_layer_backward(ctypes.byref(sh), p, p, p, p, p, p, 1.0, p, 1 << 30, p, p, p, p,
+                                p, p, 1 << 30, 0, None) == 1
+    assert L.moe_layer_forward_train(ctypes.byref(sh), p, p, None, p, p, p, p, p, 1 << 30, p,
+                                     1 << 30, None) == 2
     d = M.desc_of(WORKLOADS["mixtral"])
     assert L.moe_backward_workspace_size(ctypes.byref(d), ctypes.byref(v)) == 0
     assert v.value > 0

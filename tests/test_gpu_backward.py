@@ -7,7 +7,8 @@ relative), so gradients are compared by max |gpu - oracle| / max |oracle| over e
 <= 3e-2.  Cases: SwiGLU with softmax + renormalised gates; Switch-style top-1 with raw gates,
 ReLU experts and a capacity limit (dropped assignments carry no gradient); sigmoid +
 selection bias + GELU with k = 3; an expert that receives no rows (its weight gradients are
-exactly zero); and the full Mixtral layer width at T = 64.
+exactly zero); the full Mixtral layer width at T = 64; expert choice; and layers with one or two
+shared experts (moe_layer_backward_ex, whose shared weights get gradients too).
 """
 
 import numpy as np
@@ -36,6 +37,13 @@ CASES = {
     # expert, at D = 256, F = 128 so the fp64 oracle stays small: 256 groups along K in the
     # weight gradients, E = 256 in the router backward and dW_g
     "v3_routing_E256": scaled(W["v3"], T=128, D=256, F=128, n_shared=0, F_shared=0),
+    # expert choice: every expert keeps its top-c tokens; a picked pair's merge weight is its
+    # softmax probability (tokens picked by several experts and by none)
+    "expert_choice": scaled(W["ec"], T=500, D=256, E=16, F=256, c=62),
+    # shared experts (weight 1 on every token): DeepSeek-style sigmoid + bias top-4 with one
+    # shared expert, and softmax top-2 with two of them
+    "v3_shared": scaled(W["v3"], T=200, D=256, E=16, k=4, F=128, F_shared=256),
+    "two_shared": scaled(W["mixtral"], T=150, D=128, E=8, F=128, n_shared=2, F_shared=192),
 }
 
 
@@ -55,20 +63,29 @@ def run_backward(w, inp, dout, aux_grad, train=False, with_out=False):
         M.moe_layer_forward_train(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
                                   out, ws, bws)
     else:
-        M.moe_layer_forward(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down, None,
-                            None, None, out, ws)
+        M.moe_layer_forward(d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                            inp.Ws_gate, inp.Ws_up, inp.Ws_down, out, ws)
     E, D, F = w.E, w.D, w.F
+    f32 = dict(dtype=torch.float32, device="cuda")
     dx = torch.empty_like(inp.x)
-    dWg = torch.empty(E, D, dtype=torch.float32, device="cuda")
-    dWgate = torch.empty(E, F, D, dtype=torch.float32, device="cuda") if w.act == "swiglu" else None
-    dWup = torch.empty(E, F, D, dtype=torch.float32, device="cuda")
-    dWdown = torch.empty(E, D, F, dtype=torch.float32, device="cuda")
-    M.moe_layer_backward(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, dout, aux_grad, ws,
-                         dx, dWg, dWgate, dWup, dWdown, bws,
-                         flags=M.BWD_PREACT_SAVED if train else 0)
+    dWg = torch.empty(E, D, **f32)
+    dWgate = torch.empty(E, F, D, **f32) if w.act == "swiglu" else None
+    dWup = torch.empty(E, F, D, **f32)
+    dWdown = torch.empty(E, D, F, **f32)
+    grads = dict(dx=dx, dWg=dWg, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown)
+    if w.n_shared:
+        S, Fs = w.n_shared, w.F_shared
+        sh = (inp.Ws_gate, inp.Ws_up, inp.Ws_down, torch.empty(S, Fs, D, **f32),
+              torch.empty(S, Fs, D, **f32), torch.empty(S, D, Fs, **f32))
+        grads.update(dWs_gate=sh[3], dWs_up=sh[4], dWs_down=sh[5])
+        M.moe_layer_backward_ex(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, sh, dout,
+                                aux_grad, ws, dx, dWg, dWgate, dWup, dWdown, bws)
+    else:
+        M.moe_layer_backward(d, inp.x, inp.Wg, inp.W_gate, inp.W_up, inp.W_down, dout, aux_grad,
+                             ws, dx, dWg, dWgate, dWup, dWdown, bws,
+                             flags=M.BWD_PREACT_SAVED if train else 0)
     torch.cuda.synchronize()
     assert M.get_device_error() == 0
-    grads = dict(dx=dx, dWg=dWg, dW_gate=dWgate, dW_up=dWup, dW_down=dWdown)
     if with_out:
         grads["out"] = out
     return M.layer_views(d, ws), grads
@@ -85,9 +102,11 @@ def test_backward_matches_oracle(name):
     v, got = run_backward(w, inp, dout, aux_grad)
     ref = O.layer_backward(C.wdict(w), C.np64(inp.x), C.np64(inp.Wg), C.np64(inp.bias),
                            C.np64(inp.W_gate), C.np64(inp.W_up), C.np64(inp.W_down),
-                           C.np64(dout), aux_grad, logits=v["logits"].double().cpu().numpy())
-    for key in ("dx", "dWg", "dW_gate", "dW_up", "dW_down"):
-        if ref[key] is None:
+                           C.np64(dout), aux_grad, logits=v["logits"].double().cpu().numpy(),
+                           Ws_gate=C.np64(inp.Ws_gate), Ws_up=C.np64(inp.Ws_up),
+                           Ws_down=C.np64(inp.Ws_down))
+    for key in ("dx", "dWg", "dW_gate", "dW_up", "dW_down", "dWs_gate", "dWs_up", "dWs_down"):
+        if ref.get(key) is None:
             continue
         err = _rel(C.np64(got[key]), ref[key])
         assert err <= TOL, f"{name}: {key} max rel err {err:.3e}"
