@@ -185,8 +185,9 @@ def job_throughput(tokens_per_rank, world, steps, max_total_ms):
     return tokens_per_rank * world * steps / (max_total_ms / 1e3)
 
 
-def stage_work(w, rows_exec):
-    """Algorithmic bytes (HBM-bound stages) or FLOPs (GEMMs) per launch; rows_exec = A_exec."""
+def stage_work(w, rows_exec, gather=False):
+    """Algorithmic bytes (HBM-bound stages) or FLOPs (GEMMs) per launch; rows_exec = A_exec.
+    With the gathering up projection the permutation moves indices only."""
     es = 2 if w.dtype == "bf16" else 4
     T, D, E, F = w.T, w.D, w.E, w.F
     K = w.E if w.select == "expert" else w.k
@@ -196,7 +197,8 @@ def stage_work(w, rows_exec):
         # x and W_g read once; logits, ids and gates written
         "route": ("hbm", T * D * es + E * D * es + T * E * 4 + T * K * 8),
         # ids read; x read once; x_perm written; row_src and inv written
-        "permute": ("hbm", T * K * 4 + T * D * es + A * D * es + A * 4 + T * K * 4),
+        "permute": ("hbm", T * K * 4 + (0 if gather else T * D * es + A * D * es) + A * 4
+                    + T * K * 4),
         "expert_up": ("tensor", 2.0 * A * D * F * n_up),
         "expert_down": ("tensor", 2.0 * A * F * D + w.n_shared * 2.0 * T * D * w.F_shared * 3),
         # expert rows read once; out written once; inv and gates read
@@ -373,6 +375,9 @@ class LayerStep:
             self.sh_off = torch.tensor([0, w.T], dtype=torch.int32, device=dev)
             self.h_sh = torch.empty(w.T, w.F_shared, dtype=inp.x.dtype, device=dev)
         self.graph, self.graph_launches, self.graph_error = None, 0, None
+        # as in moe_layer_forward: with enough rows the up projection gathers the token rows
+        # itself and the permutation writes indices only
+        self.gather = M.gather_fusion(self.d)
 
     def __call__(self, ev=None, st=None):
         M, w, inp, v = self.M, self.w, self.inp, self.v
@@ -382,14 +387,18 @@ class LayerStep:
                     v["importance"], scratch, s, entropy=v["entropy"])
         if ev is not None:
             ev[1].record(s)
-        M.moe_permute(d, v["expert_ids"], inp.x, v["x_perm"], v["counts"], v["offsets"],
-                      v["row_src"], v["inv"], scratch, s)
+        M.moe_permute(d, v["expert_ids"], inp.x, None if self.gather else v["x_perm"],
+                      v["counts"], v["offsets"], v["row_src"], v["inv"], scratch, s)
         if ev is not None:
             ev[2].record(s)
         # (with a few executed rows the routed experts' products take the k-split schedule, its
         # partials in the step scratch, as in moe_layer_forward)
-        M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, v["h"],
-                           scratch, s)
+        if self.gather:
+            M.moe_expert_up_gather(d, w.E, w.F, inp.x, v["row_src"], v["rows"], v["offsets"],
+                                   inp.W_gate, inp.W_up, v["h"], s)
+        else:
+            M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up,
+                               v["h"], scratch, s)
         if ev is not None:
             ev[3].record(s)
         M.moe_expert_down_ws(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, v["y"], scratch, s)
@@ -487,11 +496,11 @@ class LayerStep:
         self.ws = self.v = self.out = None
 
 
-def stage_rooflines(w, per_stage, rows_exec, active, peaks, tc_peak):
+def stage_rooflines(w, per_stage, rows_exec, active, peaks, tc_peak, gather=False):
     """Per stage: achieved rate and the fraction of its own roofline time (GEMM stages: the
     slower of FLOPs at the tensor peak and weight + activation bytes at the HBM peak; the
     others: bytes at the HBM peak), plus the whole layer's roofline."""
-    work = stage_work(w, rows_exec)
+    work = stage_work(w, rows_exec, gather)
     es = 2 if w.dtype == "bf16" else 4
     n_up = 2 if w.act == "swiglu" else 1
     gemm_bytes = {
@@ -551,7 +560,7 @@ def measure_workload(M, w, seed, dev, stream, steps, warmup, nvml_index, peaks):
     tc_key = "bf16_tflops_sustained" if "sw_power_cap" in clk.reasons else "bf16_tflops"
     rows_exec, active = rows_and_active(st.v)
     stages, work, gemm_flops, layer_roof_s = stage_rooflines(w, per_stage, rows_exec, active,
-                                                             peaks, peaks[tc_key])
+                                                             peaks, peaks[tc_key], st.gather)
     top = max(STAGES, key=lambda s: per_stage[s])
     res = {
         "shape": w.description, "T": w.T, "ms_per_step": round(ms, 4),
@@ -559,7 +568,7 @@ def measure_workload(M, w, seed, dev, stream, steps, warmup, nvml_index, peaks):
         "timing": "CUDA-graph replay" if use_graph else "eager calls",
         "stage_timing": "graph replays, event nodes between stages" if staged is not None
         else "eager calls, events between stages",
-        "rows_executed": rows_exec, "active_experts": active,
+        "rows_executed": rows_exec, "active_experts": active, "gather_fusion": st.gather,
         "dominant": {"stage": top, **stages[top]},
         "layer_frac_of_roofline": round(layer_roof_s / (ms * 1e-3), 3),
         "layer_roofline_ms": round(layer_roof_s * 1e3, 4),
@@ -644,7 +653,7 @@ def run_cuda(args, rank, world, local):
     tc_key = "bf16_tflops_sustained" if power_capped else "bf16_tflops"
     tc_peak = peaks[tc_key]
     stages, work, gemm_flops, layer_roof_s = stage_rooflines(w, per_stage, rows_exec, active,
-                                                             peaks, tc_peak)
+                                                             peaks, tc_peak, step.gather)
     up_flops = work["expert_up"][1]
     achieved = up_flops / (per_stage["expert_up"] * 1e-3) / 1e12
     gemm_tflops = gemm_flops / ((per_stage["expert_up"] + per_stage["expert_down"]) * 1e-3) / 1e12
@@ -668,7 +677,7 @@ def run_cuda(args, rank, world, local):
         "config": {"workload": w.name, "shape": w.description, "T": w.T,
                    "D": w.D, "E": w.E, "k": w.k, "F": w.F, "tokens_per_step": w.T * world,
                    "parallelism": f"replicas x{world}" if world > 1 else "1 GPU",
-                   "rows_executed": rows_exec,
+                   "rows_executed": rows_exec, "gather_fusion": step.gather,
                    "l2": "inputs larger than L2: %.2f GB of expert weights stream per step"
                          % ((w.E * 3 * w.F * w.D * 2) / 1e9)},
         "roofline": roofline, "stages": stages,

@@ -117,7 +117,8 @@ typedef struct moe_layer_views {
     int32_t* offsets;      /* [E+1] first row of each expert in the grouped buffers */
     int32_t* row_src;      /* [A]   assignment id of each row: t*k+j (TC) or t*E+e (EC) */
     int32_t* inv;          /* TC [T*k], EC [T*E]: row of each assignment, -1 if dropped / not picked */
-    void* x_perm;          /* [A, D]  token rows grouped by expert */
+    void* x_perm;          /* [A, D]  token rows grouped by expert (not written by a
+                                         moe_layer_forward that gathers, see moe_gather_fusion) */
     void* h;               /* [A, F]  expert hidden activations */
     void* y;               /* [A, D]  expert outputs, grouped */
     void* y_shared;        /* [S, T, D] shared expert outputs (NULL when S = 0) */
@@ -176,7 +177,8 @@ moe_status_t moe_route(const moe_desc_t* desc, const void* x, const void* Wg,
  * order); "Top-k 路由" capacity factor; moe-comparison capacity/overflow table.
  *   counts [E] nominal assignments; offsets [E+1] exclusive scan of kept rows;
  *   row_src [A] assignment id per row; inv [T*k] (TC) / [T*E] (EC) row per assignment or -1;
- *   x_perm [A, D] (dtype) rows gathered from x.  Rows of one expert are ordered by (token,
+ *   x_perm [A, D] (dtype) rows gathered from x; x_perm = NULL computes the indices only (the
+ *   rows are then read by moe_expert_up_gather).  Rows of one expert are ordered by (token,
  *   slot).  All outputs are deterministic.  scratch: moe_scratch_size bytes. */
 moe_status_t moe_permute(const moe_desc_t* desc, const int32_t* expert_ids, const void* x,
                          void* x_perm, int32_t* counts, int32_t* offsets, int32_t* row_src,
@@ -225,6 +227,23 @@ moe_status_t moe_expert_ffn(const moe_desc_t* desc, int32_t n_groups, int32_t F,
                             const void* a, int64_t a_rows, const int32_t* offsets,
                             const void* W_gate, const void* W_up, const void* W_down,
                             void* h, void* y, moe_stream_t stream);
+
+/* moe_expert_up that reads its rows straight from the tokens: Tiny MoE section 12.1's fusion of
+ * the token permutation into the grouped GEMM.  Row r of the grouped operand is token
+ * row_src[r] / K of x (K = k for token choice, E for expert choice; row_src from moe_permute,
+ * which then needs no x_perm); the up projection's A tiles are loaded with 4-row TMA gathers,
+ * so the grouped copy of x is never written or read.  Same results as moe_permute with x_perm
+ * followed by moe_expert_up on it.  x [T, D] bf16; a_rows = moe_rows_max; bf16 only, and the
+ * default or 128-row GEMM tile (MOE_ERR_UNSUPPORTED otherwise). */
+moe_status_t moe_expert_up_gather(const moe_desc_t* desc, int32_t n_groups, int32_t F,
+                                  const void* x, const int32_t* row_src, int64_t a_rows,
+                                  const int32_t* offsets, const void* W_gate, const void* W_up,
+                                  void* h, moe_stream_t stream);
+
+/* Whether moe_layer_forward uses that fusion for this desc (*on = 1): bf16, more than 16
+ * grouped rows (fewer take the small-batch schedule on x_perm), and not disabled by
+ * MOE_GATHER_FUSION=0 in the environment.  Host only. */
+moe_status_t moe_gather_fusion(const moe_desc_t* desc, int32_t* on);
 
 /* moe_expert_up / moe_expert_down with a scratch area for the small-batch (decode) schedule
  * ("别只比较 Top-k" expert-work account: a small decode batch leaves each expert's products
@@ -290,9 +309,9 @@ typedef struct moe_bwd_shared {
 /* Backward of moe_layer_forward with the selection held fixed ("Top-k 路由" section
  * "門控網路的梯度流": the selected experts' gate scores carry the gradient, unselected experts
  * none; Tiny MoE section 9: task loss + weight x aux loss, fixed expert indices).
- * Loss L = <dout, out> + aux_grad * aux; the routing, permutation, logits, gates, x_perm, h, y
+ * Loss L = <dout, out> + aux_grad * aux; the routing, permutation, logits, gates, h, y
  * and f of the forward call are read from its workspace `fwd_ws` (same desc and inputs).
- *   Outputs: dx [T, D] (bf16); dWg [E, D], dW_gate and dW_up [E, F, D] (dW_gate NULL unless
+ *   Outputs: dx [T, D] (the layer dtype); dWg [E, D], dW_gate and dW_up [E, F, D] (dW_gate NULL unless
  *   SwiGLU), dW_down [E, D, F], all fp32, overwritten.  The selection-only bias gets no
  *   gradient.  Merge weights: softmax over the selected logits (RENORM) or the softmax value
  *   (RAW); sigmoid affinities likewise; the balance loss reaches the logits through P.
@@ -303,7 +322,10 @@ typedef struct moe_bwd_shared {
  * Token choice or expert choice (the merge weight of a picked (token, expert) pair is its
  * softmax probability, so its logit gradient is the softmax Jacobian applied to the pairs' dg;
  * the picked sets are held fixed like the top-k).  Layers with shared experts use
- * moe_layer_backward_ex.  Limits: bf16 (MOE_ERR_UNSUPPORTED otherwise). */
+ * moe_layer_backward_ex.  bf16 layers run the products on the tensor-core grouped GEMM (bf16
+ * operands, fp32 accumulation); fp32 layers (Tiny MoE section 9 trains in fp32) run them in
+ * fp32 on CUDA cores, always recompute the pre-activations (flags ignored) and write dx in
+ * fp32. */
 enum { MOE_BWD_PREACT_SAVED = 1 };
 moe_status_t moe_backward_workspace_size(const moe_desc_t* desc, size_t* bytes);
 moe_status_t moe_layer_backward(const moe_desc_t* desc, const void* x, const void* Wg,
@@ -331,8 +353,8 @@ moe_status_t moe_layer_backward_ex(const moe_desc_t* desc, const void* x, const 
 /* moe_layer_forward (same limits as moe_layer_backward) that also stores the routed expert
  * pre-activations (SwiGLU gate and up, or the ReLU/GELU input) into bwd_ws, for a following
  * moe_layer_backward with MOE_BWD_PREACT_SAVED.  Results and the workspace `ws` are those of
- * moe_layer_forward.  Layers with shared experts: MOE_ERR_UNSUPPORTED (run moe_layer_forward,
- * then moe_layer_backward_ex with flags 0). */
+ * moe_layer_forward.  Layers with shared experts and fp32 layers: MOE_ERR_UNSUPPORTED (run
+ * moe_layer_forward, then the backward with flags 0). */
 moe_status_t moe_layer_forward_train(const moe_desc_t* desc, const void* x, const void* Wg,
                                      const float* sel_bias, const void* W_gate,
                                      const void* W_up, const void* W_down, void* out, void* ws,

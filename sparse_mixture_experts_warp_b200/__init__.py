@@ -23,6 +23,7 @@ __all__ = [
     "workspace_size", "layer_views", "moe_route", "moe_permute", "moe_expert_up",
     "moe_expert_down", "moe_expert_ffn", "moe_expert_up_ws", "moe_expert_down_ws",
     "moe_permute_noalloc", "moe_combine", "moe_balance_stats", "moe_layer_backward_ex",
+    "moe_expert_up_gather", "gather_fusion",
     "MoeBwdShared",
     "moe_layer_forward", "get_device_error", "empty_scratch", "empty_workspace",
 ]
@@ -103,6 +104,8 @@ _SIGS = {
     "moe_expert_up": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_down": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P], ctypes.c_int),
     "moe_expert_ffn": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_expert_up_gather": ([_DP, _I32, _I32, _P, _P, _I64, _P, _P, _P, _P, _P], ctypes.c_int),
+    "moe_gather_fusion": ([_DP, ctypes.POINTER(_I32)], ctypes.c_int),
     "moe_expert_up_ws": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _P, _SZ, _P],
                          ctypes.c_int),
     "moe_expert_down_ws": ([_DP, _I32, _I32, _P, _I64, _P, _P, _P, _P, _SZ, _P], ctypes.c_int),
@@ -308,6 +311,21 @@ def moe_expert_up(d, n_groups, F, a, offsets, W_gate, W_up, h, stream=None):
     _check("moe_expert_up", lib().moe_expert_up(
         ctypes.byref(d), n_groups, F, _ptr(a), a.shape[0], _ptr(offsets), _ptr(W_gate),
         _ptr(W_up), _ptr(h), _stream(stream)))
+
+
+def moe_expert_up_gather(d, n_groups, F, x, row_src, a_rows, offsets, W_gate, W_up, h,
+                         stream=None):
+    """moe_expert_up reading its rows from the tokens x through row_src (no x_perm)."""
+    _check("moe_expert_up_gather", lib().moe_expert_up_gather(
+        ctypes.byref(d), n_groups, F, _ptr(x), _ptr(row_src), int(a_rows), _ptr(offsets),
+        _ptr(W_gate), _ptr(W_up), _ptr(h), _stream(stream)))
+
+
+def gather_fusion(d: MoeDesc) -> bool:
+    """Whether moe_layer_forward gathers the token rows inside the up projection."""
+    v = _I32()
+    _check("moe_gather_fusion", lib().moe_gather_fusion(ctypes.byref(d), ctypes.byref(v)))
+    return bool(v.value)
 
 
 def moe_expert_down(d, n_groups, F, h, offsets, W_down, y, stream=None):

@@ -35,19 +35,18 @@ inline G counted(G grid) {
 // ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
 
 // route.cu
-// With ticket (an int in the scratch, zeroed here before the launch) and importance / entropy
-// given, the router's last CTA reduces the importance partials into them (fixed order).
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
-                                       float* logits, float* imp_partials, float* lpart,
-                                       int* ticket, float* importance, float* entropy,
-                                       cudaStream_t s);
+                                       float* logits, float* imp_partials, int* n_partials,
+                                       float* lpart, cudaStream_t s);
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, float* lpart, int* ticket,
-                                        float* importance, float* entropy, cudaStream_t s);
+                                        float* imp_partials, int* n_partials, float* lpart,
+                                        cudaStream_t s);
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s);
+cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
+                                     float* importance, float* entropy, cudaStream_t s);
 int router_partials(const moe_desc_t& d);   // rows of the importance partials buffer (upper bound)
 bool router_uses_gemm(const moe_desc_t& d);
 size_t router_gemm_scratch_bytes(const moe_desc_t& d);   // partial logits of the GEMM router
@@ -61,6 +60,11 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
                                         void* x_perm, int32_t* counts, int32_t* offsets,
                                         int32_t* row_src, int32_t* inv, int32_t* block_hist,
                                         int32_t cap, cudaStream_t s);
+// The grouped copy of the token rows alone (x_perm[row] = x[token of row]), from the
+// permutation's inv (token choice) or picked lists (expert choice).
+cudaError_t launch_gather_permuted_rows(const moe_desc_t& d, const int32_t* ids,
+                                        const int32_t* inv, const void* x, void* x_perm,
+                                        cudaStream_t s);
 cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* picked,
                                          const void* x, void* x_perm, int32_t* counts,
                                          int32_t* offsets, int32_t* row_src, int32_t* inv,
@@ -84,10 +88,14 @@ cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S,
                               cudaStream_t s);
 cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N,
                               const int32_t* n_rows, void* y, cudaStream_t s);
+// With gather_src, A is the token tensor [src_rows, K] and row r of the grouped operand is its
+// row gather_src[r] / gather_div (4-row TMA gathers; the grouped copy is never written).
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,
-                                     void* out2 = nullptr);
+                                     void* out2 = nullptr, const int32_t* gather_src = nullptr,
+                                     int gather_div = 1, int64_t src_rows = 0);
+bool gemm_gather_ok();   // the selected tile shape can gather A rows
 
 // Router product on the same engine: one group of T rows, N = E, fp32 partial logits of
 // ksplit k-ranges in partials[ksplit][T][E] (E % 32 == 0, E <= 256).
@@ -134,6 +142,15 @@ cudaError_t launch_dwg(const float* ds, const void* x, int T, int D, int E, floa
 
 // Test hook of the grouped GEMM's bounded waits (see moe_debug_inject).
 void set_gemm_fault(int kind);
+
+// backward_f32.cu (fp32 layer backward on CUDA cores)
+size_t backward_f32_workspace(const moe_desc_t& d, int64_t rows);
+cudaError_t launch_backward_f32(const moe_desc_t& d, const moe_layer_views_t& v,
+                                const float* x, const float* Wg, const float* W_gate,
+                                const float* W_up, const float* W_down,
+                                const moe_bwd_shared_t* sh, const float* dout, float aux_grad,
+                                float* dx, float* dWg, float* dW_gate, float* dW_up,
+                                float* dW_down, void* ws, cudaStream_t s);
 
 // ffn_simt.cu (fp32 experts)
 cudaError_t launch_ffn_up_f32(int act, const float* a, int64_t a_rows, int D, int F,

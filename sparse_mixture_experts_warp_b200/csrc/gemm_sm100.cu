@@ -110,6 +110,11 @@ struct GemmParams {
   // group g's K rows start at row g * bk_group of either tensor
   int kb_split;
   int bk_group;
+  // row gather (groups along M): when set, row r of the grouped operand A is row
+  // gather_src[r] / gather_div of the tensor tmA maps (the tokens x, with 1-row boxes), read
+  // with 4-row gathers straight into the ring: the grouped copy of the rows is never written
+  const int32_t* gather_src;
+  int gather_div;
 };
 
 // One work item of the persistent schedule.
@@ -155,6 +160,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
       " [%0], [%1, {%3, %4}], [%2];" ::"r"(dst),
       "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y)
+      : "memory");
+}
+
+// Four rows (y0..y3) of 64 (or 32) columns from x on, through a tensor map whose box is one row
+// high, into four consecutive 128-byte (64-byte) rows of shared memory; the map's swizzle
+// applies as for a tiled box.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y0, int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+      "r"(y2), "r"(y3)
       : "memory");
 }
 
@@ -462,7 +480,77 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   const int total_all = total * p.ksplit;          // k-splits are the slowest tile index
   const int nkb = (p.K + KB - 1) / KB;
 
-  if (warp == 0) {
+  if (warp == 0 && p.gather_src) {
+    // ---------------- TMA producer, gathered rows of A ----------------
+    // All 32 lanes walk the schedule.  Lane 0 waits for a free stage, arms it and loads B;
+    // lane l loads rows 8 l .. 8 l + 7 of the tile's A block with two 4-row gathers (rows past
+    // the group end read token row 0: computed, then discarded by the epilogue).
+    constexpr int ROWB = KB * 2;                 // bytes of one A row in a stage
+    int stage = 0;
+    uint32_t phase = 0;
+    uint32_t issued = 0, issued_par = 0;
+    bool ok = true;
+    int g = 0;
+    for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
+      const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+      const int a_row = (int)tl.row0 + tl.m_idx * TBM;
+      const int row_end = (int)tl.row0 + tl.m;
+      const int b_row = tl.g * p.N + tl.n_idx * p.n_out_tile;
+      const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
+      const bool mine = 8 * lane < (two ? 2 * BM : BM);
+      int src[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const int r = a_row + 8 * lane + i;
+        src[i] = (mine && r < row_end) ? __ldg(p.gather_src + r) / p.gather_div : 0;
+      }
+      for (int kb = tl.kb0; kb < tl.kb1; ++kb) {
+        const int kx = kb * KB;
+        int go = 1;
+        if (lane == 0) {
+          go = mbar_wait(&empty[stage], phase ^ 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
+                         TIMEOUT_NS);
+          if (go) mbar_expect_tx(&full[stage], (two ? 2 * HA_BYTES : HA_BYTES) + TB_BYTES);
+        }
+        go = __shfl_sync(0xffffffffu, go, 0);
+        if (!go) {
+          ok = false;
+          break;
+        }
+        const bool withhold = p.fault == 1 && blockIdx.x == 0 && t == (int)blockIdx.x &&
+                              kb == tl.kb0;     // test hook, as in the tiled producer below
+        const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
+        if (mine && !withhold) {
+          tma_gather4(a_dst + (8 * lane) * ROWB, &tmA, &full[stage], kx, src[0], src[1], src[2],
+                      src[3]);
+          tma_gather4(a_dst + (8 * lane + 4) * ROWB, &tmA, &full[stage], kx, src[4], src[5],
+                      src[6], src[7]);
+        }
+        if (lane == 0 && !withhold) {
+          if (EPI == EPI_SWIGLU || EPI == EPI_RAW) {
+            tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kx, b_row);
+          } else {
+            tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, &tmB0, &full[stage], kx, b_row + 128);
+          }
+        }
+        issued |= 1u << stage;
+        issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
+        if (++stage == TSTAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      // let the copies already in flight land before the CTA exits
+      for (int s = 0; s < TSTAGES; ++s)
+        if (issued & (1u << s))
+          mbar_wait(&full[s], (issued_par >> s) & 1u, abort_flag, p.err, DEVERR_TIMEOUT_TMA,
+                    DRAIN_NS, /*honor_abort=*/false);
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ---------------- TMA producer ----------------
       int stage = 0;
@@ -1296,14 +1384,23 @@ cudaError_t launch_pair(int epi, const CUtensorMap& a, const CUtensorMap& b0,
 
 }  // namespace
 
+bool gemm_gather_ok() {
+  const GemmTile t = gemm_tile();
+  return t == TILE_256 || t == TILE_128;
+}
+
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,
-                                     void* out2) {
+                                     void* out2, const int32_t* gather_src, int gather_div,
+                                     int64_t src_rows) {
   if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
+  if (gather_src && (!offsets || !gemm_gather_ok() || epi == EPI_NONE_BMN || gather_div < 1 ||
+                     src_rows <= 0))
+    return cudaErrorInvalidValue;
   alignas(64) CUtensorMap ta, tb0, tb1;
   const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
-  GemmParams p;
+  GemmParams p{};
   p.offsets = offsets;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = device_error_word();
@@ -1325,10 +1422,17 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.ksplit = 1;
   p.kchunk = 1 << 30;
   p.split_stride = 0;
+  p.gather_src = gather_src;
+  p.gather_div = gather_div;
   const GemmTile tile = gemm_tile();
   const int halves = tile == TILE_128 ? 1 : 2;
   const int kb = tile == TILE_256_K32 ? 32 : 64;
-  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
+  if (gather_src) {
+    // A rows come from the token rows of A itself ([src_rows, K]) by 4-row gathers
+    if (!make_map(&ta, A, (uint64_t)src_rows, (uint64_t)K, 1, kb)) return cudaErrorInvalidValue;
+  } else if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, kb)) {
+    return cudaErrorInvalidValue;
+  }
   if (!make_map(&tb0, B0, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
   if (epi == EPI_SWIGLU || epi == EPI_RAW) {
     if (!make_map(&tb1, B1, brows, (uint64_t)K, 128, kb)) return cudaErrorInvalidValue;
@@ -1337,7 +1441,7 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   }
   const int tbm = tile == TILE_PAIR ? 2 * BM : BM * halves;
   const int64_t max_tiles = ((a_rows + tbm - 1) / tbm + n_groups) * (int64_t)p.nt;
-  if (tile == TILE_PAIR && offsets && epi != EPI_RAW && !out2) {
+  if (tile == TILE_PAIR && offsets && epi != EPI_RAW && !out2 && !gather_src) {
     // 256 x 512 accumulator tiles: 256 SwiGLU features (gate + up) or 512 output columns;
     // the SwiGLU weights go in 64-row boxes
     if (epi == EPI_SWIGLU && (!make_map(&tb0, B0, brows, (uint64_t)K, 64, kb) ||
@@ -1378,7 +1482,7 @@ cudaError_t launch_grouped_gemm_bf16_bmn(const void* A, int64_t a_rows, int K, c
   } else {
     tb1 = tb0;
   }
-  GemmParams p;
+  GemmParams p{};
   p.offsets = offsets;
   p.out = static_cast<__nv_bfloat16*>(out);
   p.err = device_error_word();
@@ -1436,7 +1540,7 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
   if (!make_map(&tb, B, (uint64_t)N, (uint64_t)k_total, 128, kb)) return cudaErrorInvalidValue;
   if (!make_map_f32_out(&to, out, (uint64_t)G, (uint64_t)M, (uint64_t)N))
     return cudaErrorInvalidValue;
-  GemmParams p;
+  GemmParams p{};
   p.offsets = nullptr;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.err = device_error_word();
@@ -1486,7 +1590,7 @@ cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K,
   alignas(64) CUtensorMap ta, tb;
   if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&tb, B, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
-  GemmParams p;
+  GemmParams p{};
   p.offsets = offsets;
   p.out = reinterpret_cast<__nv_bfloat16*>(out);
   p.err = device_error_word();
@@ -1541,7 +1645,7 @@ cudaError_t launch_router_gemm_bf16(const void* x, int T, int D, const void* Wg,
   alignas(64) CUtensorMap ta, tb;
   if (!make_map(&ta, x, (uint64_t)T, (uint64_t)D, 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&tb, Wg, (uint64_t)E, (uint64_t)D, 128, 64)) return cudaErrorInvalidValue;
-  GemmParams p;
+  GemmParams p{};
   p.offsets = nullptr;                        // one group: all T token rows
   p.out = reinterpret_cast<__nv_bfloat16*>(partials);
   p.err = device_error_word();

@@ -101,7 +101,6 @@ size_t route_scratch(const moe_desc_t* d) {
   size_t b = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   if (d->select == MOE_EXPERT_CHOICE) b += up((size_t)d->E * d->T * sizeof(float));
   b += up(router_gemm_scratch_bytes(*d));
-  b += kAlign;                    // the router's ticket (last-CTA reduction)
   return b;
 }
 size_t permute_scratch(const moe_desc_t* d) {
@@ -305,18 +304,18 @@ moe_status_t moe_route(const moe_desc_t* d, const void* x, const void* Wg, const
   const size_t pbytes = up((size_t)router_partials(*d) * (d->E + 1) * sizeof(float));
   const size_t tbytes = d->select == MOE_EXPERT_CHOICE ? up((size_t)d->E * d->T * sizeof(float)) : 0;
   float* lpart = router_uses_gemm(*d) ? reinterpret_cast<float*>(sc + pbytes + tbytes) : nullptr;
-  int* ticket = reinterpret_cast<int*>(sc + pbytes + tbytes + up(router_gemm_scratch_bytes(*d)));
+  int np = 0;
   cudaError_t e;
   if (d->select == MOE_TOKEN_CHOICE) {
     e = launch_router_token_choice(*d, x, Wg, d->score == MOE_SCORE_SIGMOID ? sel_bias : nullptr,
-                                   expert_ids, gates, logits, partials, lpart, ticket,
-                                   importance, entropy, s);
+                                   expert_ids, gates, logits, partials, &np, lpart, s);
   } else {
     float* probsT = reinterpret_cast<float*>(sc + pbytes);
-    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, lpart, ticket,
-                                    importance, entropy, s);
+    e = launch_router_expert_choice(*d, x, Wg, gates, probsT, logits, partials, &np, lpart, s);
     if (e == cudaSuccess) e = launch_ec_select(*d, probsT, expert_ids, s);
   }
+  if (e == cudaSuccess && (importance || entropy))
+    e = launch_importance_reduce(partials, np, d->E, d->T, importance, entropy, s);
   return cuda_status(e);
 }
 
@@ -326,9 +325,9 @@ moe_status_t moe_permute(const moe_desc_t* d, const int32_t* expert_ids, const v
                          moe_stream_t stream) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
-  if (!expert_ids || !x || !x_perm || !counts || !offsets || !row_src || !inv)
-    return MOE_ERR_INVALID_ARG;
-  if (!is_aligned16(x) || !is_aligned16(x_perm)) return MOE_ERR_INVALID_ARG;
+  // x_perm == NULL: indices only (the rows are gathered later, by moe_expert_up_gather)
+  if (!expert_ids || !x || !counts || !offsets || !row_src || !inv) return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(x) || (x_perm && !is_aligned16(x_perm))) return MOE_ERR_INVALID_ARG;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e;
   if (d->select == MOE_TOKEN_CHOICE) {
@@ -402,6 +401,46 @@ moe_status_t moe_expert_ffn(const moe_desc_t* d, int32_t G, int32_t F, const voi
   moe_status_t st = moe_expert_up(d, G, F, a, a_rows, offsets, W_gate, W_up, h, stream);
   if (st != MOE_OK) return st;
   return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
+}
+
+static bool gather_fusion_enabled() {
+  static const bool v = [] {
+    const char* s = getenv("MOE_GATHER_FUSION");
+    return !(s && s[0] == '0');
+  }();
+  return v;
+}
+
+moe_status_t moe_gather_fusion(const moe_desc_t* d, int32_t* on) {
+  moe_status_t st = validate(d);
+  if (st != MOE_OK) return st;
+  if (!on) return MOE_ERR_INVALID_ARG;
+  *on = (d->dtype == MOE_BF16 && gather_fusion_enabled() && gemm_gather_ok() &&
+         rows_of(d) > kSplitUpRows)
+            ? 1
+            : 0;
+  return MOE_OK;
+}
+
+moe_status_t moe_expert_up_gather(const moe_desc_t* d, int32_t G, int32_t F, const void* x,
+                                  const int32_t* row_src, int64_t a_rows,
+                                  const int32_t* offsets, const void* W_gate, const void* W_up,
+                                  void* h, moe_stream_t stream) {
+  moe_status_t st = check_ffn(d, G, F, x, a_rows, offsets);
+  if (st != MOE_OK) return st;
+  if (d->dtype != MOE_BF16 || !gemm_gather_ok()) return MOE_ERR_UNSUPPORTED;
+  if (!row_src || !W_up || !h || (d->act == MOE_ACT_SWIGLU && !W_gate))
+    return MOE_ERR_INVALID_ARG;
+  if (!is_aligned16(W_up) || !is_aligned16(h) || (W_gate && !is_aligned16(W_gate)))
+    return MOE_ERR_INVALID_ARG;
+  if (d->T == 0 || a_rows == 0) return MOE_OK;
+  const int div = d->select == MOE_EXPERT_CHOICE ? d->E : d->k;
+  const bool glu = d->act == MOE_ACT_SWIGLU;
+  const int epi = glu ? EPI_SWIGLU : (d->act == MOE_ACT_GELU ? EPI_GELU : EPI_RELU);
+  return cuda_status(launch_grouped_gemm_bf16(epi, x, a_rows, d->D, glu ? W_gate : W_up,
+                                              glu ? W_up : nullptr, G, F, offsets, h,
+                                              reinterpret_cast<cudaStream_t>(stream), nullptr,
+                                              row_src, div, d->T));
 }
 
 // ---- the small-batch (decode) schedule: k-split products, see kMaxSplits ----
@@ -531,10 +570,20 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
   st = moe_route(d, x, Wg, sel_bias, v.expert_ids, v.gates, v.logits, v.importance, v.entropy,
                  v.scratch, v.scratch_bytes, stream);
   if (st != MOE_OK) return st;
-  st = moe_permute(d, v.expert_ids, x, v.x_perm, v.counts, v.offsets, v.row_src, v.inv,
-                   v.scratch, v.scratch_bytes, stream);
+  // with enough rows (bf16), the up projection gathers the token rows itself and the
+  // permutation writes indices only
+  int32_t gather = 0;
+  if (!preact) moe_gather_fusion(d, &gather);
+  st = moe_permute(d, v.expert_ids, x, gather ? nullptr : v.x_perm, v.counts, v.offsets,
+                   v.row_src, v.inv, v.scratch, v.scratch_bytes, stream);
   if (st != MOE_OK) return st;
-  if (preact) {
+  if (gather) {
+    st = moe_expert_up_gather(d, d->E, d->F, x, v.row_src, v.rows, v.offsets, W_gate, W_up, v.h,
+                              stream);
+    if (st == MOE_OK)
+      st = moe_expert_down_ws(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
+                              v.scratch_bytes, stream);
+  } else if (preact) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool glu = d->act == MOE_ACT_SWIGLU;
     cudaError_t e = launch_grouped_gemm_bf16(
@@ -602,13 +651,17 @@ bool bwd_weight_transpose() {
 moe_status_t check_backward(const moe_desc_t* d) {
   moe_status_t st = validate(d);
   if (st != MOE_OK) return st;
-  if (d->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   if (d->E > 256) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
-// Backward workspace layout; with base == nullptr only the size is computed.
+// Backward workspace layout; with base == nullptr only the size is computed.  fp32 layers use
+// their own layout (backward_f32.cu); only its size is returned here.
 size_t carve_bwd(const moe_desc_t* d, uint8_t* base, BwdViews* v) {
+  if (d->dtype == MOE_F32) {
+    memset(v, 0, sizeof *v);
+    return backward_f32_workspace(*d, rows_of(d));
+  }
   const int64_t T = d->T, D = d->D, E = d->E, F = d->F, A = rows_of(d);
   const bool glu = d->act == MOE_ACT_SWIGLU;
   v->ldg = glu ? (F + 127) / 128 * 256 : F;
@@ -724,7 +777,8 @@ moe_status_t moe_layer_forward_train(const moe_desc_t* d, const void* x, const v
                                      moe_stream_t stream) {
   moe_status_t st = check_backward(d);
   if (st != MOE_OK) return st;
-  if (d->n_shared > 0) return MOE_ERR_UNSUPPORTED;   // use moe_layer_forward, flags 0
+  // shared experts and fp32 layers: moe_layer_forward, then the backward with flags 0
+  if (d->n_shared > 0 || d->dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
   BwdViews b;
   if (!bwd_ws || bwd_ws_bytes < carve_bwd(d, nullptr, &b)) return MOE_ERR_WORKSPACE;
   if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
@@ -781,6 +835,12 @@ moe_status_t moe_layer_backward_ex(const moe_desc_t* d, const void* x, const voi
   if ((reinterpret_cast<uintptr_t>(bwd_ws) % kAlign) != 0) return MOE_ERR_WORKSPACE;
   carve_bwd(d, static_cast<uint8_t*>(bwd_ws), &b);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d->dtype == MOE_F32)
+    return cuda_status(launch_backward_f32(
+        *d, v, static_cast<const float*>(x), static_cast<const float*>(Wg),
+        static_cast<const float*>(W_gate), static_cast<const float*>(W_up),
+        static_cast<const float*>(W_down), shared, static_cast<const float*>(dout), aux_grad,
+        static_cast<float*>(dx), dWg, dW_gate, dW_up, dW_down, bwd_ws, s));
   const int T = d->T, D = d->D, E = d->E, F = d->F;
   const int K = d->select == MOE_EXPERT_CHOICE ? E : d->k;
   const int64_t A = v.rows;
@@ -798,7 +858,9 @@ moe_status_t moe_layer_backward_ex(const moe_desc_t* d, const void* x, const voi
     if (e == cudaSuccess && S) e = cudaMemsetAsync(shared->dWs_down, 0, sb, s);
     return cuda_status(e);
   }
-  cudaError_t e = launch_pad_offsets(v.offsets, E, b.pad_off, s);
+  // the grouped copy of x (a forward with the gathering up projection does not write it)
+  cudaError_t e = launch_gather_permuted_rows(*d, v.expert_ids, v.inv, x, v.x_perm, s);
+  if (e == cudaSuccess) e = launch_pad_offsets(v.offsets, E, b.pad_off, s);
   // dY = g dout on the executed rows, dg = <dout, y>
   if (e == cudaSuccess)
     e = launch_gather_dy(dout, v.y, v.row_src, v.gates, v.offsets, E, K, D, A, b.dY, b.dgates, s);

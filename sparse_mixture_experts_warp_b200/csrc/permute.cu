@@ -359,6 +359,7 @@ permute_onepass_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int
     s_row[oa - a0] = row;
   }
   __syncthreads();
+  if (xp == nullptr) return;      // indices only: the up projection gathers the rows itself
   // 4. copy: warp w copies tokens 4w .. 4w+3 of the CTA's 32; each lane keeps 4 tokens x 4
   //    chunks (256 bytes) of loads in flight before it stores them to the expert rows
   const int tw = blockIdx.x * kOnePassTokens + warp * 4;
@@ -512,10 +513,28 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
     perm_rank_kernel<<<counted(nblk), kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
         ids, A, E, cap, block_hist, offsets, row_src, inv);
   }
-  if (nblk > 0) {
+  if (nblk > 0 && x_perm) {
     const int blocks = (d.T * 32 + 255) / 256;
     gather_tc_kernel<<<counted(blocks), 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
                                             static_cast<uint4*>(x_perm));
+  }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_gather_permuted_rows(const moe_desc_t& d, const int32_t* ids,
+                                        const int32_t* inv, const void* x, void* x_perm,
+                                        cudaStream_t s) {
+  const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
+  const int nvec = d.D * esz / 16;
+  if (d.select == MOE_TOKEN_CHOICE) {
+    if (d.T > 0)
+      gather_tc_kernel<<<counted((d.T * 32 + 255) / 256), 256, 0, s>>>(
+          static_cast<const uint4*>(x), d.T, nvec, d.k, inv, static_cast<uint4*>(x_perm));
+  } else {
+    const int rows = d.E * d.c;
+    if (rows > 0)
+      gather_rows_kernel<<<counted((rows * 32 + 255) / 256), 256, 0, s>>>(
+          static_cast<const uint4*>(x), d.T, nvec, ids, rows, static_cast<uint4*>(x_perm));
   }
   return cudaGetLastError();
 }
@@ -532,7 +551,7 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
                                                   row_src, inv);
   const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
   const int nvec = d.D * esz / 16;
-  if (rows > 0)
+  if (rows > 0 && x_perm)
     gather_rows_kernel<<<counted((rows * 32 + 255) / 256), 256, 0, s>>>(
         static_cast<const uint4*>(x), d.T, nvec, picked, rows, static_cast<uint4*>(x_perm));
   return cudaGetLastError();

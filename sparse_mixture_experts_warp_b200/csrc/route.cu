@@ -14,7 +14,6 @@
 // arg-max for top-k, and the merge weights.  Everything stays on chip except x, W_g and the
 // outputs.
 #include "common.cuh"
-#include "mbar.cuh"
 
 namespace moe {
 namespace {
@@ -114,29 +113,6 @@ __device__ __forceinline__ void group_limit(float (&key)[NS], int E, int n_group
   }
 }
 
-// Sum of the partial rows (E importance sums, then the entropy sum) over the n CTAs, each
-// column by one warp in a fixed order (lane-strided sums, then a shuffle tree).
-__device__ __forceinline__ void reduce_partials(const float* partials, int n, int E, int T,
-                                                float* importance, float* entropy, int warp,
-                                                int lane, int nwarps) {
-  for (int c = warp; c <= E; c += nwarps) {
-    float v = 0.f;
-    for (int b = lane; b < n; b += 32) v += __ldcg(partials + (int64_t)b * (E + 1) + c);
-    v = warp_sum(v);
-    if (lane == 0) {
-      if (c < E && importance) importance[c] = v / (float)T;
-      if (c == E && entropy) *entropy = v / (float)T;
-    }
-  }
-}
-
-struct ReduceExtra {
-  int* ticket;           // zeroed before the launch; null: no in-kernel reduction
-  float* importance;
-  float* entropy;
-  int* err;              // device error word
-};
-
 // logits of the warp's TPW tokens for all experts -> s_log[TPW][E]
 template <bool BF16>
 __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* s_log, int lane) {
@@ -185,7 +161,7 @@ __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* 
 
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
-router_kernel(RouterArgs a, ReduceExtra ex) {
+router_kernel(RouterArgs a) {
   extern __shared__ float s_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + warp;
@@ -344,22 +320,26 @@ router_kernel(RouterArgs a, ReduceExtra ex) {
       for (int w = 0; w < kWarps; ++w) sum += s_all[w * (E + 1) + c];
       a.partials[(int64_t)blockIdx.x * (E + 1) + c] = sum;
     }
-    // the last block to finish reduces every block's row (fixed order)
-    if (ex.ticket) {
-      __shared__ int s_last;
-      __syncthreads();
-      if (threadIdx.x == 0) {
-        __threadfence();
-        s_last = atomicAdd(ex.ticket, 1) == (int)gridDim.x - 1;
-      }
-      __syncthreads();
-      if (s_last) {
-        __threadfence();
-        reduce_partials(a.partials, gridDim.x, E, a.T, ex.importance, ex.entropy, warp, lane,
-                        kWarps);
-        if (threadIdx.x == 0) *ex.ticket = 0;
-      }
-    }
+  }
+}
+
+// importance[e] = (sum over partial rows, fixed order) / T, one block per expert; block E
+// reduces the entropy column into *entropy (mean over tokens).
+__global__ void importance_reduce_kernel(const float* partials, int n, int E, int T,
+                                         float* importance, float* entropy) {
+  const int e = blockIdx.x;
+  float* out = (e < E) ? importance : entropy;
+  if (!out) return;
+  float s = 0.f;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s += partials[(int64_t)i * (E + 1) + e];
+  __shared__ float red[32];
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = s;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = (threadIdx.x < (blockDim.x >> 5)) ? red[threadIdx.x] : 0.f;
+    v = warp_sum(v);
+    if (threadIdx.x == 0) out[e < E ? e : 0] = v / (float)T;
   }
 }
 
@@ -465,28 +445,19 @@ ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
 
 // ---- fast path: bf16 token choice, E <= 8, D = 256 * NW with 4 <= NW <= 16 ----
 //
-// The router product is an HBM-bound contraction with at most 8 experts: the FMAs (and the
-// bf16 -> fp32 conversions a CUDA-core dot product needs) go to the tensor cores through
-// mma.sync m16n8k16 with W_g as the A operand (experts on rows 0..7, rows 8..15 zero) and 8
-// tokens as N, and the kernel is left with streaming x.  One CTA per SM owns a contiguous range
-// of tokens; a producer warp copies its token rows from HBM into a shared-memory ring with bulk
-// copies (8 rows per stage, each row padded by 64 bytes so the 16-byte fragment reads of a warp
-// hit distinct banks), so the copy engine, not the load/store units, keeps up to 3 x 64 KB in
-// flight per SM.  Consumer warp w owns the hidden slice [256 w, 256 w + 256).  The k order inside
-// the slice is permuted (the same permutation for x and W_g, which leaves the sum unchanged) so
-// that each thread's B fragments over the 16 k-steps are eight 16-byte chunks of one token row
-// and its A fragments the same eight chunks of one W_g row, W_g held in registers.  Partial
-// logits of the warps are summed in a fixed order through shared memory; warps 0..7 then do the
-// affinity, top-k and gates of one token each.  The CTAs' importance / entropy partial rows are
-// reduced by the last CTA to finish (a ticket in the scratch, zeroed before the launch), in a
-// fixed order, so the result is deterministic and no second kernel is launched.
-constexpr int kFastE = 8;        // experts (zero-padded): rows of the MMA's A operand
-constexpr int kFastTB = 8;       // MMA N: tokens per group = rows per ring stage
+// The router product is an HBM-bound contraction with N = E <= 8 experts: exactly the N of
+// mma.sync m16n8k16, so the FMAs (and the bf16 -> fp32 conversions a CUDA-core dot product
+// needs) go to the tensor cores and the kernel is left with streaming x.  One CTA of NW warps
+// owns a contiguous range of tokens; warp w owns the hidden slice [256w, 256w + 256).  The k
+// order inside the slice is permuted (the same permutation for x and W_g, which leaves the sum
+// unchanged) so that each thread's A fragments over the 16 k-steps are eight 16-byte chunks of
+// two token rows and its B fragments the same eight chunks of one W_g row: every global load is
+// a 16-byte vector load, and the 4 threads of a row read 64 contiguous bytes together.  Per 16-token batch a warp issues 16 MMAs; partial
+// logits of the NW warps are summed in a fixed order through shared memory, the next batch's
+// loads are already in flight while warps do the per-token affinity / top-k / gates.
+constexpr int kFastE = 8;        // MMA N: experts (zero-padded)
+constexpr int kFastTB = 16;      // MMA M: tokens per batch
 constexpr int kFastMaxNW = 16;
-constexpr int kFastStages = 3;
-constexpr int kRowPad = 64;      // bytes after each staged row
-constexpr uint64_t kRouterTimeoutNs = 2000000000ull;
-constexpr uint64_t kRouterDrainNs = 200000000ull;
 
 __device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint32_t a1,
                                                uint32_t a2, uint32_t a3, uint32_t b0,
@@ -496,6 +467,24 @@ __device__ __forceinline__ void mma_16816_bf16(float (&c)[4], uint32_t a0, uint3
       "{%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Two token rows (g, g + 8 of the batch): this thread's 8 chunks of 8 elements, chunk i at
+// element kbase + 32 i (kbase = 256 w + 8 tig), so the 4 threads of a row read 64 contiguous
+// bytes per load instruction.
+__device__ __forceinline__ void load_rows(uint4 (&r0)[8], uint4 (&r1)[8],
+                                          const __nv_bfloat16* x, int D, int t0, int t_end,
+                                          int g, int kbase) {
+  const int ta = t0 + g, tb = t0 + g + 8;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r0[i] = (ta < t_end)
+                ? __ldcs(reinterpret_cast<const uint4*>(x + (int64_t)ta * D + kbase + 32 * i))
+                : make_uint4(0u, 0u, 0u, 0u);
+    r1[i] = (tb < t_end)
+                ? __ldcs(reinterpret_cast<const uint4*>(x + (int64_t)tb * D + kbase + 32 * i))
+                : make_uint4(0u, 0u, 0u, 0u);
+  }
 }
 
 __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float sv, bool live,
@@ -547,130 +536,66 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float
   }
 }
 
-__global__ void __launch_bounds__((kFastMaxNW + 1) * 32, 1)
-router_fast_kernel(RouterArgs a, ReduceExtra ex, int tokens_per_cta) {
-  extern __shared__ __align__(128) uint8_t s_dyn[];
-  __shared__ uint64_t full[kFastStages], empty[kFastStages];
-  __shared__ float s_red[2][kFastMaxNW][kFastTB][kFastE];
+__global__ void __launch_bounds__(kFastMaxNW * 32, 1)
+router_fast_kernel(RouterArgs a, int tokens_per_cta) {
+  __shared__ float s_red[kFastMaxNW][kFastTB][kFastE];
+  __shared__ float s_log[kFastTB][kFastE];
   __shared__ float s_imp[kFastTB][kFastE];
   __shared__ float s_ent[kFastTB];
-  __shared__ int s_abort, s_last;
-  const int NW = (blockDim.x >> 5) - 1;         // consumer warps; warp NW produces
+  const int NW = blockDim.x >> 5;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, tig = lane & 3;
-  const int E = a.E, D = a.D;
-  const uint32_t row_bytes = (uint32_t)D * 2u;
-  const uint32_t row_stride = row_bytes + kRowPad;
-  const uint32_t stage_bytes = kFastTB * row_stride;
-  volatile int* abort_flag = &s_abort;
+  const int E = a.E;
+  const int kbase = warp * 256 + tig * 8;    // this thread's chunks: kbase + 32 i, i < 8
+  const __nv_bfloat16* x = static_cast<const __nv_bfloat16*>(a.x);
+  const __nv_bfloat16* Wg = static_cast<const __nv_bfloat16*>(a.Wg);
+  uint4 wv[8];                               // W_g[g][kbase + 32 i .. + 8)
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+    wv[i] = (g < E) ? __ldg(reinterpret_cast<const uint4*>(Wg + (int64_t)g * a.D + kbase + 32 * i))
+                    : make_uint4(0u, 0u, 0u, 0u);
   const int t_begin = blockIdx.x * tokens_per_cta;
   const int t_end = min(a.T, t_begin + tokens_per_cta);
-  const int n_groups = t_end > t_begin ? (t_end - t_begin + kFastTB - 1) / kFastTB : 0;
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kFastStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], NW);
-    }
-    s_abort = 0;
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  __syncthreads();
   float imp = 0.f, ent = 0.f;
-
-  if (warp == NW) {
-    // producer: one lane issues the bulk copies of each group's rows
-    if (lane == 0) {
-      const char* xb = static_cast<const char*>(a.x);
-      int issued = 0;
-      for (int gi = 0; gi < n_groups; ++gi) {
-        const int s = gi % kFastStages;
-        if (gi >= kFastStages &&
-            !mbar_wait(&empty[s], ((gi / kFastStages) - 1) & 1u, abort_flag, ex.err,
-                       DEVERR_TIMEOUT_TMA, kRouterTimeoutNs))
-          break;
-        const int t0 = t_begin + gi * kFastTB;
-        const int n = min(kFastTB, t_end - t0);
-        mbar_expect_tx(&full[s], (uint32_t)n * row_bytes);
-        uint8_t* dst = s_dyn + (size_t)s * stage_bytes;
-        for (int j = 0; j < n; ++j)
-          bulk_load(dst + (size_t)j * row_stride, xb + (int64_t)(t0 + j) * row_bytes, row_bytes,
-                    &full[s]);
-        issued = gi + 1;
-      }
-      // every copy issued has landed before the CTA may exit (bounded, also after an abort)
-      for (int gi = issued > kFastStages ? issued - kFastStages : 0; gi < issued; ++gi)
-        mbar_wait(&full[gi % kFastStages], (gi / kFastStages) & 1u, abort_flag, ex.err,
-                  DEVERR_TIMEOUT_TMA, kRouterDrainNs, /*honor_abort=*/false);
+  uint4 r0[8], r1[8];
+  load_rows(r0, r1, x, a.D, t_begin, t_end, g, kbase);
+  for (int t0 = t_begin; t0 < t_end; t0 += kFastTB) {
+    float c[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      // k-steps 2i (chunk elements 0..3) and 2i+1 (chunk elements 4..7)
+      mma_16816_bf16(c, r0[i].x, r1[i].x, r0[i].y, r1[i].y, wv[i].x, wv[i].y);
+      mma_16816_bf16(c, r0[i].z, r1[i].z, r0[i].w, r1[i].w, wv[i].z, wv[i].w);
     }
-  } else {
-    // consumer warp: W_g rows g (zero for g >= E) of this warp's slice, held in registers
-    const int kbase = warp * 256 + tig * 8;      // this thread's chunks: kbase + 32 i, i < 8
-    const __nv_bfloat16* Wg = static_cast<const __nv_bfloat16*>(a.Wg);
-    uint4 wv[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      wv[i] = (g < E) ? __ldg(reinterpret_cast<const uint4*>(Wg + (int64_t)g * D + kbase + 32 * i))
-                      : make_uint4(0u, 0u, 0u, 0u);
-    for (int gi = 0; gi < n_groups; ++gi) {
-      const int s = gi % kFastStages, par = gi & 1;
-      const int t0 = t_begin + gi * kFastTB;
-      const bool ok = mbar_wait(&full[s], (gi / kFastStages) & 1u, abort_flag, ex.err,
-                                DEVERR_TIMEOUT_TMA, kRouterTimeoutNs);
-      if (ok) {
-        // B fragments: token g of the group, this thread's 8 chunks of the warp's slice
-        const uint8_t* row = s_dyn + (size_t)s * stage_bytes + (size_t)g * row_stride +
-                             (size_t)kbase * 2;
-        float c[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const uint4 xv = *reinterpret_cast<const uint4*>(row + 64 * i);
-          // k-steps 2i (chunk elements 0..3) and 2i+1 (chunk elements 4..7)
-          mma_16816_bf16(c, wv[i].x, 0u, wv[i].y, 0u, xv.x, xv.y);
-          mma_16816_bf16(c, wv[i].z, 0u, wv[i].w, 0u, xv.z, xv.w);
-        }
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&empty[s]);   // this warp no longer reads the stage
-        // c[0], c[1]: expert g, tokens 2 tig and 2 tig + 1 of the group
-        s_red[par][warp][2 * tig][g] = c[0];
-        s_red[par][warp][2 * tig + 1][g] = c[1];
-      }
-      asm volatile("bar.sync 1, %0;" ::"r"(NW * 32) : "memory");
-      if (*abort_flag) break;
-      for (int j = warp; j < kFastTB && t0 + j < t_end; j += NW) {
-        const bool live = lane < E;
-        float sv = -INFINITY;
-        if (live) {
-          sv = 0.f;
-          for (int ww = 0; ww < NW; ++ww) sv += s_red[par][ww][j][lane];
-        }
-        select_token(a, t0 + j, sv, live, lane, imp, ent);
-      }
+    if (t0 + kFastTB < t_end) load_rows(r0, r1, x, a.D, t0 + kFastTB, t_end, g, kbase);
+    s_red[warp][g][2 * tig] = c[0];
+    s_red[warp][g][2 * tig + 1] = c[1];
+    s_red[warp][g + 8][2 * tig] = c[2];
+    s_red[warp][g + 8][2 * tig + 1] = c[3];
+    __syncthreads();
+    if (threadIdx.x < kFastTB * kFastE) {
+      const int j = threadIdx.x / kFastE, e = threadIdx.x % kFastE;
+      float sum = 0.f;
+      for (int ww = 0; ww < NW; ++ww) sum += s_red[ww][j][e];
+      s_log[j][e] = sum;
+    }
+    __syncthreads();
+    for (int jj = warp; jj < kFastTB; jj += NW) {
+      if (t0 + jj >= t_end) break;
+      const bool live = lane < E;
+      select_token(a, t0 + jj, live ? s_log[jj][lane] : -INFINITY, live, lane, imp, ent);
     }
   }
-  // CTA importance partial: sum over the selection warps (consumer warps below 8) in a fixed
-  // order
-  const int nsel = NW < kFastTB ? NW : kFastTB;
-  if (warp < nsel && lane < kFastE) s_imp[warp][lane] = imp;
+  // CTA importance partial: sum over the selection warps in a fixed order
+  const int n_sel = NW < kFastTB ? NW : kFastTB;
+  if (warp < n_sel && lane < kFastE) s_imp[warp][lane] = imp;
   ent = warp_sum(ent);
-  if (warp < nsel && lane == 0) s_ent[warp] = ent;
+  if (warp < n_sel && lane == 0) s_ent[warp] = ent;
   __syncthreads();
   if (a.partials && threadIdx.x <= E) {      // row: E importance sums, then the entropy sum
     float sum = 0.f;
-    for (int j = 0; j < nsel; ++j) sum += (threadIdx.x < E) ? s_imp[j][threadIdx.x] : s_ent[j];
+    for (int j = 0; j < n_sel; ++j) sum += (threadIdx.x < E) ? s_imp[j][threadIdx.x] : s_ent[j];
     a.partials[(int64_t)blockIdx.x * (E + 1) + threadIdx.x] = sum;
-  }
-  if (!ex.ticket) return;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    __threadfence();
-    s_last = atomicAdd(ex.ticket, 1) == (int)gridDim.x - 1;
-  }
-  __syncthreads();
-  if (s_last) {
-    __threadfence();
-    reduce_partials(a.partials, gridDim.x, E, a.T, ex.importance, ex.entropy, warp, lane,
-                    blockDim.x >> 5);
-    if (threadIdx.x == 0) *ex.ticket = 0;
   }
 }
 
@@ -687,23 +612,18 @@ int router_partials(const moe_desc_t& d) {
   return generic > 1024 ? generic : 1024;
 }
 
-static cudaError_t launch_router(const RouterArgs& a, ReduceExtra ex, bool bf16, int T,
-                                 cudaStream_t s) {
+static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStream_t s) {
   const int blocks = (T + kWarps * kTPW - 1) / (kWarps * kTPW);
   if (blocks == 0) return cudaSuccess;
-  if (ex.ticket) {
-    cudaError_t e = cudaMemsetAsync(ex.ticket, 0, sizeof(int), s);
-    if (e != cudaSuccess) return e;
-  }
   const size_t smem = (size_t)kWarps * kTPW * a.E * sizeof(float);
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<true><<<counted(blocks), kWarps * 32, smem, s>>>(a, ex);
+    router_kernel<true><<<counted(blocks), kWarps * 32, smem, s>>>(a);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<false><<<counted(blocks), kWarps * 32, smem, s>>>(a, ex);
+    router_kernel<false><<<counted(blocks), kWarps * 32, smem, s>>>(a);
   }
   return cudaGetLastError();
 }
@@ -724,15 +644,10 @@ static bool fast_router_ok(const moe_desc_t& d) {
          d.D % 256 == 0 && d.D / 256 >= 4 && d.D / 256 <= kFastMaxNW && d.k <= 32;
 }
 
-size_t fast_router_smem(const moe_desc_t& d) {
-  return (size_t)kFastStages * kFastTB * ((size_t)d.D * 2 + kRowPad);
-}
-
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
-                                       float* logits, float* imp_partials, float* lpart,
-                                       int* ticket, float* importance, float* entropy,
-                                       cudaStream_t s) {
+                                       float* logits, float* imp_partials, int* n_partials,
+                                       float* lpart, cudaStream_t s) {
   RouterArgs a{x, Wg, bias, ids, gates, logits, nullptr, imp_partials,
                d.T, d.D, d.E, d.k, d.score, d.gate, 0, nullptr, 1};
   a.n_group = d.n_group;
@@ -748,29 +663,20 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
     const int sms = num_sms() < 1024 ? num_sms() : 1024;
     const int tpc = (d.T + sms - 1) / sms;
     const int grid = tpc > 0 ? (d.T + tpc - 1) / tpc : 0;
+    *n_partials = grid;
     if (grid == 0) return cudaSuccess;
-    ReduceExtra ex{nullptr, importance, entropy, device_error_word()};
-    if (ticket && imp_partials && (importance || entropy)) {
-      cudaError_t e = cudaMemsetAsync(ticket, 0, sizeof(int), s);
-      if (e != cudaSuccess) return e;
-      ex.ticket = ticket;
-    }
-    const size_t smem = fast_router_smem(d);
-    cudaError_t e = cudaFuncSetAttribute(router_fast_kernel,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    router_fast_kernel<<<counted(grid), (d.D / 256 + 1) * 32, smem, s>>>(a, ex, tpc);
+    router_fast_kernel<<<counted(grid), (d.D / 256) * 32, 0, s>>>(a, tpc);
     return cudaGetLastError();
   }
-  ReduceExtra ex{nullptr, importance, entropy, device_error_word()};
-  if (ticket && imp_partials && (importance || entropy)) ex.ticket = ticket;
-  return launch_router(a, ex, d.dtype == MOE_BF16, d.T, s);
+  *n_partials = generic_partials(d);
+  return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
 cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                         float* probs, float* probsT, float* logits,
-                                        float* imp_partials, float* lpart, int* ticket,
-                                        float* importance, float* entropy, cudaStream_t s) {
+                                        float* imp_partials, int* n_partials, float* lpart,
+                                        cudaStream_t s) {
+  *n_partials = generic_partials(d);
   RouterArgs a{x, Wg, nullptr, nullptr, probs, logits, probsT, imp_partials,
                d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1, nullptr, 1};
   if (router_uses_gemm(d) && lpart) {
@@ -780,9 +686,7 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
     a.lpart = lpart;
     a.ksplit = ks;
   }
-  ReduceExtra ex{nullptr, importance, entropy, device_error_word()};
-  if (ticket && imp_partials && (importance || entropy)) ex.ticket = ticket;
-  return launch_router(a, ex, d.dtype == MOE_BF16, d.T, s);
+  return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
@@ -798,6 +702,13 @@ cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* 
   } else {
     ec_select_kernel<false><<<counted(d.E), 1024, 0, s>>>(probsT, d.T, d.c, picked);
   }
+  return cudaGetLastError();
+}
+
+cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
+                                     float* importance, float* entropy, cudaStream_t s) {
+  importance_reduce_kernel<<<counted(E + 1), 256, 0, s>>>(partials, n_partials, E, T, importance,
+                                                          entropy);
   return cudaGetLastError();
 }
 

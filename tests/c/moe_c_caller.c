@@ -54,10 +54,13 @@ int main(void) {
     bad = d;
     bad.n_group = 3; bad.topk_group = 1;
     check(moe_workspace_size(&bad, &ws) == MOE_ERR_INVALID_ARG, "n_group must divide E");
-    bad = d;
-    bad.dtype = MOE_F32;
-    check(moe_backward_workspace_size(&bad, &bws) == MOE_ERR_UNSUPPORTED,
-          "fp32 backward unsupported");
+    moe_desc_t f32 = d;
+    f32.dtype = MOE_F32;
+    check(moe_backward_workspace_size(&f32, &bws) == MOE_OK && bws > 0,
+          "fp32 backward workspace size");
+    check(moe_layer_forward_train(&f32, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, 0, NULL,
+                                  0, NULL) == MOE_ERR_UNSUPPORTED,
+          "fp32 training forward refused (the plain forward serves fp32 backward)");
     check(moe_layer_forward(&d, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL, NULL,
                             NULL, 0, NULL) != MOE_OK, "null buffers refused");
     check(moe_expert_up_ws(&d, 8, 14336, NULL, 8192, NULL, NULL, NULL, NULL, NULL, 0, NULL) ==

@@ -157,9 +157,9 @@ def test_header_entry_points_cite_the_pages():
 def test_backward_validation_before_launch():
     v = ctypes.c_size_t()
     L = M.lib()
-    # bf16 layers: token choice or expert choice, with or without shared experts
-    for kw, st in ((dict(dtype=0), 2), (dict(select=1, c=8), 0), (dict(n_shared=1, F_shared=64), 0),
-                   (dict(k=0), 1)):
+    # bf16 and fp32 layers: token choice or expert choice, with or without shared experts
+    for kw, st in ((dict(dtype=0), 0), (dict(select=1, c=8), 0), (dict(n_shared=1, F_shared=64), 0),
+                   (dict(k=0), 1), (dict(E=300, k=2), 2)):
         assert L.moe_backward_workspace_size(ctypes.byref(_bad(**kw)), ctypes.byref(v)) == st, kw
     # shared experts need moe_layer_backward_ex's weights (moe_layer_backward passes none) and
     # the plain forward (moe_layer_forward_train does not run them)

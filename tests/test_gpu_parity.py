@@ -13,6 +13,7 @@ import torch
 
 from sparse_mixture_experts_warp_b200.workloads import WORKLOADS, scaled
 import moe_check as C
+import sparse_mixture_experts_warp_b200 as M
 
 pytestmark = pytest.mark.gpu
 
@@ -224,3 +225,44 @@ def test_v3_node_limited_full_size():
     assert max(len(set(row)) for row in groups.tolist()) <= 4
     # every expert that received rows: one row from one of its 32-row slices, and its last row
     C.check_stratified_output(w, inp, out, v, seed=124, every_slice=False)
+
+
+def test_layer_without_gather_fusion_in_subprocess():
+    """MOE_GATHER_FUSION=0 makes moe_layer_forward write the grouped copy x_perm and run the up
+    projection on it (instead of gathering the token rows inside it); the small-case parity
+    tests pass there too, x_perm checked row by row against the tokens."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_GATHER_FUSION="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "small_layer_matches_oracle"], env=env, capture_output=True, text=True,
+                       timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+
+
+@pytest.mark.parametrize("name", ["mixtral_small", "switch_small", "v3_small", "ec_small"])
+def test_gathering_up_projection_matches_the_permuted_one(name):
+    """moe_permute without x_perm + moe_expert_up_gather gives the same h, bit for bit, as
+    moe_permute with x_perm + moe_expert_up (the same products in the same k order; only the
+    way the A rows reach shared memory differs), and moe_permute's x_perm rows are the tokens'."""
+    w = SMALL[name]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    A = M.rows_max(d)
+    x_perm = torch.empty(A, w.D, dtype=inp.x.dtype, device="cuda")
+    M.moe_permute(d, v["expert_ids"], inp.x, x_perm, v["counts"], v["offsets"], v["row_src"],
+                  v["inv"])
+    n = int(v["offsets"][-1].item())
+    K = w.E if w.select == "expert" else w.k
+    tok = (v["row_src"][:n] // K).long()
+    assert torch.equal(x_perm[:n], inp.x[tok])
+    h1 = torch.zeros(A, w.F, dtype=inp.x.dtype, device="cuda")
+    h2 = torch.zeros(A, w.F, dtype=inp.x.dtype, device="cuda")
+    M.moe_expert_up(d, w.E, w.F, x_perm, v["offsets"], inp.W_gate, inp.W_up, h1)
+    M.moe_expert_up_gather(d, w.E, w.F, inp.x, v["row_src"], A, v["offsets"], inp.W_gate,
+                           inp.W_up, h2)
+    torch.cuda.synchronize()
+    assert M.get_device_error() == 0
+    assert torch.equal(h1[:n], h2[:n])
