@@ -65,6 +65,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                const float* __restrict__ gates, const uint4* __restrict__ ys, int S, int T,
                int K, int nvec, uint4* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   using R = Row<BF16>;
   __shared__ int s_row[kWarps][kMaxList];
   __shared__ float s_g[kWarps][kMaxList];
@@ -104,6 +106,8 @@ __global__ void __launch_bounds__(kWarps * 32)
 combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                        const float* __restrict__ gates, int T, int nvec,
                        uint4* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
   using R = Row<BF16>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
@@ -151,6 +155,8 @@ combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ 
 __global__ void __launch_bounds__(256)
 stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance,
              const float* entropy, int E, int n_routes, float alpha, float* f, moe_stats_t* st) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_fp[256];
   __shared__ int s_max[256];
   __shared__ int s_sorted[256];
@@ -222,20 +228,20 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
     const uint4* yy = static_cast<const uint4*>(y);
     uint4* oo = static_cast<uint4*>(out);
     if (d.dtype == MOE_BF16) {
-      if (K == 1) combine_small_k_kernel<true, 1><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
-      else combine_small_k_kernel<true, 2><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<true, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
+      else (void)launch_pdl(combine_small_k_kernel<true, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
     } else {
-      if (K == 1) combine_small_k_kernel<false, 1><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
-      else combine_small_k_kernel<false, 2><<<counted(blocks), kWarps * 32, 0, s>>>(yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<false, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
+      else (void)launch_pdl(combine_small_k_kernel<false, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
     }
     return cudaGetLastError();
   }
   if (d.dtype == MOE_BF16)
-    combine_kernel<true><<<counted(blocks), kWarps * 32, 0, s>>>(
+    (void)launch_pdl(combine_kernel<true>, dim3(blocks), dim3(kWarps * 32), 0, s, 
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
         K, nvec, static_cast<uint4*>(out));
   else
-    combine_kernel<false><<<counted(blocks), kWarps * 32, 0, s>>>(
+    (void)launch_pdl(combine_kernel<false>, dim3(blocks), dim3(kWarps * 32), 0, s, 
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
         K, nvec, static_cast<uint4*>(out));
   return cudaGetLastError();
@@ -246,7 +252,7 @@ cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const float* entropy, float* f, moe_stats_t* stats,
                                  cudaStream_t s) {
   const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
-  stats_kernel<<<counted(1), 256, 0, s>>>(counts, offsets, importance, entropy, d.E, n_routes,
+  (void)launch_pdl(stats_kernel, dim3(1), dim3(256), 0, s, counts, offsets, importance, entropy, d.E, n_routes,
                                           d.aux_alpha, f, stats);
   return cudaGetLastError();
 }

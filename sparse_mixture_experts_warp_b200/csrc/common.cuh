@@ -32,6 +32,37 @@ inline G counted(G grid) {
   return grid;
 }
 
+// ---- programmatic dependent launch ----
+// The forward path's kernels are launched with programmatic stream serialization: the next
+// kernel in the stream may be scheduled while this one finishes (its launch and set-up overlap
+// the tail), and every such kernel starts with pdl_trigger() (its dependents may launch) and
+// calls pdl_wait() -- which returns once the preceding grid has completed and its memory is
+// visible -- before it touches anything an earlier kernel wrote or reads.  Without the launch
+// attribute both are no-ops.  MOE_PDL=0 in the environment turns the attribute off.
+bool pdl_enabled();
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// Launch of a kernel that calls pdl_wait() before its first dependent access.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  note_launch();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = pdl_enabled() ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
 
 // route.cu

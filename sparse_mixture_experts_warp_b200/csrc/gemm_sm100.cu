@@ -437,6 +437,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                  : "memory");
     asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
   }
+  // everything above is set-up of this CTA's own shared memory and tensor memory; the group
+  // table and the operands were written by earlier kernels
+  pdl_trigger();
+  pdl_wait();
   if (warp == 2 && p.kgroup) {
     // groups along K: every group has the same ceil(rows / TBM) * nt tiles
     const int per = (int)((p.rows + TBM - 1) / TBM) * p.nt;
@@ -1298,8 +1302,7 @@ cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtens
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  kern<<<counted(grid), 64 + 128 * HALVES, smem, s>>>(a, b0, b1, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(64 + 128 * HALVES), smem, s, a, b0, b1, p);
 }
 
 template <int HALVES, int KB, int NSTAGES>

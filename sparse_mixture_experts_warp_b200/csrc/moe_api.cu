@@ -25,6 +25,14 @@ int num_sms() {
   return n > 0 ? n : 148;
 }
 
+bool pdl_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_PDL");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 int* device_error_word() {
   void* p = nullptr;
   if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
@@ -218,6 +226,8 @@ inline moe_status_t cuda_status(cudaError_t e) {
 }
 
 __global__ void set_offsets_kernel(int32_t* o, int T) {
+  pdl_trigger();
+  pdl_wait();
   o[0] = 0;
   o[1] = T;
 }
@@ -603,7 +613,7 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
   if (st != MOE_OK) return st;
   if (d->n_shared > 0) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    set_offsets_kernel<<<counted(1), 1, 0, s>>>(v.shared_offsets, d->T);
+    (void)launch_pdl(set_offsets_kernel, dim3(1), dim3(1), 0, s, v.shared_offsets, d->T);
     if (cudaGetLastError() != cudaSuccess) return MOE_ERR_CUDA;
     // shared experts always use SwiGLU
     moe_desc_t ds = *d;

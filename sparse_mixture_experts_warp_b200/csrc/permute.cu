@@ -30,6 +30,8 @@ constexpr int kWarpsPerBlock = kThreads / 32;
 
 __global__ void __launch_bounds__(kThreads)
 perm_hist_kernel(const int32_t* ids, int A, int E, int32_t* block_hist) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int s_hist[];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_hist[e] = 0;
   __syncthreads();
@@ -49,6 +51,8 @@ perm_hist_kernel(const int32_t* ids, int A, int E, int32_t* block_hist) {
 __global__ void __launch_bounds__(1024)
 perm_scan_kernel(int32_t* block_hist, int nblk, int E, int cap, int32_t* counts,
                  int32_t* offsets) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_warp[32];
   const int e = threadIdx.x;
   int total = 0;
@@ -89,6 +93,8 @@ perm_scan_kernel(int32_t* block_hist, int nblk, int E, int cap, int32_t* counts,
 __global__ void __launch_bounds__(kThreads)
 perm_rank_kernel(const int32_t* ids, int A, int E, int cap, const int32_t* block_base,
                  const int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int s_mem[];
   int* s_cnt = s_mem;                             // [warps][E] per-warp counts, then bases
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -151,6 +157,8 @@ constexpr int kFusedMaxItems = 1 << 13;
 __global__ void __launch_bounds__(1024)
 perm_index_fused_kernel(const int32_t* ids, int A, int E, int cap, int32_t* counts,
                         int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ int s_mem[];
   int* s_cnt = s_mem;                    // [32][E]
   int* s_off = s_mem + 32 * E;           // [E]
@@ -257,6 +265,8 @@ __global__ void __launch_bounds__(256)
 permute_onepass_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int cap,
                        const uint4* __restrict__ x, int nvec, uint4* __restrict__ xp,
                        int32_t* counts, int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ int s_all[8][kOnePassMaxE];       // per warp: all assignments
   __shared__ int s_pre[8][kOnePassMaxE];       // per warp: assignments before this CTA's
   __shared__ int s_own[8][kOnePassMaxE];       // per warp: this CTA's, then exclusive bases
@@ -405,6 +415,8 @@ permute_onepass_kernel(const int32_t* __restrict__ ids, int T, int k, int E, int
 __global__ void __launch_bounds__(256)
 gather_tc_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int32_t* inv,
                  uint4* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
   const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (warp >= T) return;
   int rows[8];
@@ -442,12 +454,16 @@ gather_tc_kernel(const uint4* __restrict__ x, int T, int nvec, int k, const int3
 
 // Expert choice: row r = e*c + i takes token picked[r]; inv[t*E + e] = r.
 __global__ void ec_fill_kernel(int32_t* inv, int64_t n) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i < n) inv[i] = -1;
 }
 
 __global__ void ec_index_kernel(const int32_t* picked, int E, int c, int T, int32_t* counts,
                                 int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  pdl_trigger();
+  pdl_wait();
   const int r = blockIdx.x * blockDim.x + threadIdx.x;
   if (r <= E) {
     offsets[r] = r * c;
@@ -468,6 +484,8 @@ __global__ void ec_index_kernel(const int32_t* picked, int E, int c, int T, int3
 __global__ void __launch_bounds__(256)
 gather_rows_kernel(const uint4* __restrict__ x, int T, int nvec, const int32_t* picked, int rows,
                    uint4* __restrict__ xp) {
+  pdl_trigger();
+  pdl_wait();
   const int r = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
   if (r >= rows) return;
   const int t = picked[r];
@@ -495,7 +513,7 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
   const int nvec = d.D * esz / 16;
   if (A > 0 && A <= kOnePassMaxItems && E <= kOnePassMaxE && d.k <= kOnePassMaxK) {
     const int grid = (d.T + kOnePassTokens - 1) / kOnePassTokens;
-    permute_onepass_kernel<<<counted(grid), 256, 0, s>>>(ids, d.T, d.k, E, cap,
+    (void)launch_pdl(permute_onepass_kernel, dim3(grid), dim3(256), 0, s, ids, d.T, d.k, E, cap,
                                                 static_cast<const uint4*>(x), nvec,
                                                 static_cast<uint4*>(x_perm), counts, offsets,
                                                 row_src, inv);
@@ -506,16 +524,16 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(perm_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                            (int)smem);
-    perm_index_fused_kernel<<<counted(1), 1024, smem, s>>>(ids, A, E, cap, counts, offsets, row_src, inv);
+    (void)launch_pdl(perm_index_fused_kernel, dim3(1), dim3(1024), smem, s, ids, A, E, cap, counts, offsets, row_src, inv);
   } else {
-    perm_hist_kernel<<<counted(nblk), kThreads, E * sizeof(int), s>>>(ids, A, E, block_hist);
-    perm_scan_kernel<<<counted(1), 1024, 0, s>>>(block_hist, nblk, E, cap, counts, offsets);
-    perm_rank_kernel<<<counted(nblk), kThreads, kWarpsPerBlock * E * sizeof(int), s>>>(
+    (void)launch_pdl(perm_hist_kernel, dim3(nblk), dim3(kThreads), E * sizeof(int), s, ids, A, E, block_hist);
+    (void)launch_pdl(perm_scan_kernel, dim3(1), dim3(1024), 0, s, block_hist, nblk, E, cap, counts, offsets);
+    (void)launch_pdl(perm_rank_kernel, dim3(nblk), dim3(kThreads), kWarpsPerBlock * E * sizeof(int), s, 
         ids, A, E, cap, block_hist, offsets, row_src, inv);
   }
   if (nblk > 0 && x_perm) {
     const int blocks = (d.T * 32 + 255) / 256;
-    gather_tc_kernel<<<counted(blocks), 256, 0, s>>>(static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
+    (void)launch_pdl(gather_tc_kernel, dim3(blocks), dim3(256), 0, s, static_cast<const uint4*>(x), d.T, nvec, d.k, inv,
                                             static_cast<uint4*>(x_perm));
   }
   return cudaGetLastError();
@@ -528,12 +546,12 @@ cudaError_t launch_gather_permuted_rows(const moe_desc_t& d, const int32_t* ids,
   const int nvec = d.D * esz / 16;
   if (d.select == MOE_TOKEN_CHOICE) {
     if (d.T > 0)
-      gather_tc_kernel<<<counted((d.T * 32 + 255) / 256), 256, 0, s>>>(
+      (void)launch_pdl(gather_tc_kernel, dim3((d.T * 32 + 255) / 256), dim3(256), 0, s, 
           static_cast<const uint4*>(x), d.T, nvec, d.k, inv, static_cast<uint4*>(x_perm));
   } else {
     const int rows = d.E * d.c;
     if (rows > 0)
-      gather_rows_kernel<<<counted((rows * 32 + 255) / 256), 256, 0, s>>>(
+      (void)launch_pdl(gather_rows_kernel, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, 
           static_cast<const uint4*>(x), d.T, nvec, ids, rows, static_cast<uint4*>(x_perm));
   }
   return cudaGetLastError();
@@ -544,15 +562,15 @@ cudaError_t launch_permute_expert_choice(const moe_desc_t& d, const int32_t* pic
                                          int32_t* offsets, int32_t* row_src, int32_t* inv,
                                          cudaStream_t s) {
   const int64_t n = (int64_t)d.T * d.E;
-  if (n > 0) ec_fill_kernel<<<counted((unsigned)((n + 255) / 256)), 256, 0, s>>>(inv, n);
+  if (n > 0) (void)launch_pdl(ec_fill_kernel, dim3((unsigned)((n + 255) / 256)), dim3(256), 0, s, inv, n);
   const int rows = d.E * d.c;
   const int m = (rows > d.E + 1 ? rows : d.E + 1);
-  ec_index_kernel<<<counted((m + 255) / 256), 256, 0, s>>>(picked, d.E, d.c, d.T, counts, offsets,
+  (void)launch_pdl(ec_index_kernel, dim3((m + 255) / 256), dim3(256), 0, s, picked, d.E, d.c, d.T, counts, offsets,
                                                   row_src, inv);
   const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
   const int nvec = d.D * esz / 16;
   if (rows > 0 && x_perm)
-    gather_rows_kernel<<<counted((rows * 32 + 255) / 256), 256, 0, s>>>(
+    (void)launch_pdl(gather_rows_kernel, dim3((rows * 32 + 255) / 256), dim3(256), 0, s, 
         static_cast<const uint4*>(x), d.T, nvec, picked, rows, static_cast<uint4*>(x_perm));
   return cudaGetLastError();
 }

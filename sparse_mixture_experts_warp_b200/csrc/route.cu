@@ -162,6 +162,8 @@ __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* 
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
 router_kernel(RouterArgs a) {
+  pdl_trigger();
+  pdl_wait();
   extern __shared__ float s_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + warp;
@@ -327,6 +329,8 @@ router_kernel(RouterArgs a) {
 // reduces the entropy column into *entropy (mean over tokens).
 __global__ void importance_reduce_kernel(const float* partials, int n, int E, int T,
                                          float* importance, float* entropy) {
+  pdl_trigger();
+  pdl_wait();
   const int e = blockIdx.x;
   float* out = (e < E) ? importance : entropy;
   if (!out) return;
@@ -372,13 +376,28 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
   return before + inc - v;
 }
 
-// staged: the expert's T keys are first copied to shared memory (dynamic, T * 4 bytes) in one
-// pass with 16-byte loads, so the four histogram passes and the compaction read them from
-// there instead of going back to L2 with one dependent load per thread and pass.
+// One block per expert.  staged: the expert's T keys are first copied to shared memory
+// (dynamic, T * 4 bytes) with 16-byte loads, so the radix passes and the compaction read them
+// from there.
+//
+// Radix select of the c-th largest key.  Probabilities are >= 0, so their IEEE bit patterns order
+// like the values.  The bits above the highest bit in which the largest and smallest key differ
+// are common to all keys and are skipped; the rest is resolved 8 bits per pass, most significant
+// first, each pass counting the digit of the keys that still match the prefix into one
+// 256-bin histogram per warp (lanes of different warps never contend), the bins then summed in
+// a fixed order.  Compaction: thread i owns the keys [i * per, (i+1) * per) in token order; one
+// block scan of its (above-threshold, equal-to-threshold) counts gives every thread its output
+// position and the number of equal keys before it, so the output holds all keys above the
+// threshold and the first `need` equal ones, in ascending token order.  Shared memory: the
+// keys (T * 4 bytes, when staged) and 32 KB of per-warp histograms.
 template <bool STAGED>
 __global__ void __launch_bounds__(1024)
 ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
+  pdl_trigger();
+  pdl_wait();
+  constexpr int NW = 32;                     // warps (blockDim.x == 1024)
   const int e = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t* gkeys = reinterpret_cast<const uint32_t*>(probsT + (int64_t)e * T);
   extern __shared__ uint32_t s_keys[];
   const uint32_t* keys = gkeys;
@@ -391,57 +410,102 @@ ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
     __syncthreads();
     keys = s_keys;
   }
-  __shared__ int hist[256];
+  __shared__ int hist[NW][256];
+  __shared__ uint32_t s_max[NW], s_min[NW];
   __shared__ int s_digit, s_need;
   __shared__ int s_warp[32];
-  uint32_t prefix = 0, mask = 0;
+  // common high bits of all keys
+  uint32_t kmax = 0u, kmin = 0xffffffffu;
+  for (int t = threadIdx.x; t < T; t += blockDim.x) {
+    const uint32_t kk = keys[t];
+    kmax = kk > kmax ? kk : kmax;
+    kmin = kk < kmin ? kk : kmin;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const uint32_t a = __shfl_xor_sync(0xffffffffu, kmax, o);
+    const uint32_t b = __shfl_xor_sync(0xffffffffu, kmin, o);
+    kmax = a > kmax ? a : kmax;
+    kmin = b < kmin ? b : kmin;
+  }
+  if (lane == 0) {
+    s_max[warp] = kmax;
+    s_min[warp] = kmin;
+  }
+  __syncthreads();
+  kmax = 0u;
+  kmin = 0xffffffffu;
+  for (int w = 0; w < NW; ++w) {
+    kmax = s_max[w] > kmax ? s_max[w] : kmax;
+    kmin = s_min[w] < kmin ? s_min[w] : kmin;
+  }
+  const uint32_t diff = kmax ^ kmin;
+  const int top = diff ? 31 - __clz(diff) : -1;      // highest differing bit
+  uint32_t mask = top >= 31 ? 0u : ~((2u << top) - 1u);   // bits above `top`
+  if (top < 0) mask = 0xffffffffu;
+  uint32_t prefix = kmax & mask;
   int need = c;
-  // Radix select of the c-th largest key, 8 bits per pass, most significant first.
-  // Probabilities are >= 0, so their IEEE bit patterns order like the values.
-  for (int pass = 0; pass < 4; ++pass) {
-    const int shift = 24 - 8 * pass;
-    for (int i = threadIdx.x; i < 256; i += blockDim.x) hist[i] = 0;
-    __syncthreads();
+  for (int lo = top - 7; top >= 0; lo -= 8) {
+    const int shift = lo > 0 ? lo : 0;
+    const int width = (lo + 7) - shift + 1;            // bits in this digit (<= 8)
+    const uint32_t dmask = (1u << width) - 1u;
+    for (int i = lane; i < 256; i += 32) hist[warp][i] = 0;
+    __syncwarp();
     for (int t = threadIdx.x; t < T; t += blockDim.x) {
       const uint32_t kk = keys[t];
-      if ((kk & mask) == prefix) atomicAdd(&hist[(kk >> shift) & 0xffu], 1);
+      if ((kk & mask) == prefix) atomicAdd(&hist[warp][(kk >> shift) & dmask], 1);
     }
     __syncthreads();
+    // bin totals (fixed order over the warps), thread b < 256 holds bin b
+    int tot = 0;
+    if (threadIdx.x < 256)
+      for (int w = 0; w < NW; ++w) tot += hist[w][threadIdx.x];
+    __syncthreads();
+    if (threadIdx.x < 256) hist[0][threadIdx.x] = tot;
+    __syncthreads();
     if (threadIdx.x == 0) {
-      int cum = 0, d = 255;
+      int cum = 0, d = (int)dmask;
       for (; d > 0; --d) {
-        if (cum + hist[d] >= need) break;
-        cum += hist[d];
+        if (cum + hist[0][d] >= need) break;
+        cum += hist[0][d];
       }
       s_digit = d;
       s_need = need - cum;
     }
     __syncthreads();
     prefix |= (uint32_t)s_digit << shift;
-    mask |= 0xffu << shift;
+    mask |= dmask << shift;
     need = s_need;
     __syncthreads();
+    if (shift == 0) break;
   }
-  // Ordered compaction: every key above the threshold, plus the first `need` keys equal to
-  // it in ascending token order.
-  int out_base = 0, eq_seen = 0;
-  for (int base = 0; base < T; base += blockDim.x) {
-    const int t = base + threadIdx.x;
-    const uint32_t kk = (t < T) ? keys[t] : 0u;
-    const int gt = (t < T && kk > prefix) ? 1 : 0;
-    const int eq = (t < T && kk == prefix) ? 1 : 0;
-    int eq_total;
-    const int eq_rank = block_exclusive_scan(eq, s_warp, &eq_total);
-    const int take = gt | (eq && (eq_seen + eq_rank < need));
-    int take_total;
-    const int pos = block_exclusive_scan(take, s_warp, &take_total);
-    if (take && out_base + pos < c) picked[(int64_t)e * c + out_base + pos] = t;
-    out_base += take_total;
-    eq_seen += eq_total;
-    __syncthreads();
+  // prefix is now the c-th largest key; take everything above it and the first `need` equal
+  // keys in token order
+  const int per = (T + blockDim.x - 1) / blockDim.x;
+  const int t0 = threadIdx.x * per, t1 = min(T, t0 + per);
+  int gt = 0, eq = 0;
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t kk = keys[t];
+    gt += kk > prefix;
+    eq += kk == prefix;
+  }
+  int total;
+  const int gt_before = block_exclusive_scan(gt, s_warp, &total);
+  int eq_before = block_exclusive_scan(eq, s_warp, &total);
+  int pos = gt_before + min(eq_before, need);
+  for (int t = t0; t < t1; ++t) {
+    const uint32_t kk = keys[t];
+    bool take = kk > prefix;
+    if (kk == prefix) {
+      take = eq_before < need;
+      ++eq_before;
+    }
+    if (take) {
+      if (pos < c) picked[(int64_t)e * c + pos] = t;
+      ++pos;
+    }
   }
 }
-
 
 // ---- fast path: bf16 token choice, E <= 8, D = 256 * NW with 4 <= NW <= 16 ----
 //
@@ -538,6 +602,8 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, float
 
 __global__ void __launch_bounds__(kFastMaxNW * 32, 1)
 router_fast_kernel(RouterArgs a, int tokens_per_cta) {
+  pdl_trigger();
+  pdl_wait();
   __shared__ float s_red[kFastMaxNW][kFastTB][kFastE];
   __shared__ float s_log[kFastTB][kFastE];
   __shared__ float s_imp[kFastTB][kFastE];
@@ -619,11 +685,11 @@ static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStre
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<true><<<counted(blocks), kWarps * 32, smem, s>>>(a);
+    (void)launch_pdl(router_kernel<true>, dim3(blocks), dim3(kWarps * 32), smem, s, a);
   } else {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    router_kernel<false><<<counted(blocks), kWarps * 32, smem, s>>>(a);
+    (void)launch_pdl(router_kernel<false>, dim3(blocks), dim3(kWarps * 32), smem, s, a);
   }
   return cudaGetLastError();
 }
@@ -665,7 +731,7 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
     const int grid = tpc > 0 ? (d.T + tpc - 1) / tpc : 0;
     *n_partials = grid;
     if (grid == 0) return cudaSuccess;
-    router_fast_kernel<<<counted(grid), (d.D / 256) * 32, 0, s>>>(a, tpc);
+    (void)launch_pdl(router_fast_kernel, dim3(grid), dim3((d.D / 256) * 32), 0, s, a, tpc);
     return cudaGetLastError();
   }
   *n_partials = generic_partials(d);
@@ -692,22 +758,22 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
 cudaError_t launch_ec_select(const moe_desc_t& d, const float* probsT, int32_t* picked,
                              cudaStream_t s) {
   const size_t smem = (size_t)d.T * sizeof(float);
-  if (d.T % 4 == 0 && smem <= 200 * 1024) {
+  if (d.T % 4 == 0 && smem <= 180 * 1024) {      // + 33 KB of static shared memory
     if (smem > 48 * 1024) {
       cudaError_t e = cudaFuncSetAttribute(ec_select_kernel<true>,
                                            cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
       if (e != cudaSuccess) return e;
     }
-    ec_select_kernel<true><<<counted(d.E), 1024, smem, s>>>(probsT, d.T, d.c, picked);
+    (void)launch_pdl(ec_select_kernel<true>, dim3(d.E), dim3(1024), smem, s, probsT, d.T, d.c, picked);
   } else {
-    ec_select_kernel<false><<<counted(d.E), 1024, 0, s>>>(probsT, d.T, d.c, picked);
+    (void)launch_pdl(ec_select_kernel<false>, dim3(d.E), dim3(1024), 0, s, probsT, d.T, d.c, picked);
   }
   return cudaGetLastError();
 }
 
 cudaError_t launch_importance_reduce(const float* partials, int n_partials, int E, int T,
                                      float* importance, float* entropy, cudaStream_t s) {
-  importance_reduce_kernel<<<counted(E + 1), 256, 0, s>>>(partials, n_partials, E, T, importance,
+  (void)launch_pdl(importance_reduce_kernel, dim3(E + 1), dim3(256), 0, s, partials, n_partials, E, T, importance,
                                                           entropy);
   return cudaGetLastError();
 }

@@ -53,6 +53,8 @@ __global__ void __launch_bounds__(kThreads)
 splitk_act_kernel(const float* __restrict__ pg, const float* __restrict__ pu, int S,
                   int64_t rows, int F, const int32_t* __restrict__ n_rows,
                   __nv_bfloat16* __restrict__ h) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t live = min((int64_t)__ldg(n_rows), rows);
   const int q = F / 4;                       // four columns per item
   const int64_t items = live * q;
@@ -79,6 +81,8 @@ splitk_act_kernel(const float* __restrict__ pg, const float* __restrict__ pu, in
 __global__ void __launch_bounds__(kThreads)
 splitk_sum_kernel(const float* __restrict__ p, int S, int64_t rows, int N,
                   const int32_t* __restrict__ n_rows, __nv_bfloat16* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
   const int64_t live = min((int64_t)__ldg(n_rows), rows);
   const int q = N / 4;
   const int64_t items = live * q;
@@ -110,13 +114,13 @@ cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S, 
   const int grid = grid_for(rows, F);
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(h);
   if (act == MOE_ACT_SWIGLU)
-    splitk_act_kernel<MOE_ACT_SWIGLU><<<counted(grid), kThreads, 0, s>>>(pg, pu, S, rows, F,
+    (void)launch_pdl(splitk_act_kernel<MOE_ACT_SWIGLU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
                                                                         n_rows, o);
   else if (act == MOE_ACT_GELU)
-    splitk_act_kernel<MOE_ACT_GELU><<<counted(grid), kThreads, 0, s>>>(pg, pu, S, rows, F,
+    (void)launch_pdl(splitk_act_kernel<MOE_ACT_GELU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
                                                                       n_rows, o);
   else
-    splitk_act_kernel<MOE_ACT_RELU><<<counted(grid), kThreads, 0, s>>>(pg, pu, S, rows, F,
+    (void)launch_pdl(splitk_act_kernel<MOE_ACT_RELU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
                                                                       n_rows, o);
   return cudaGetLastError();
 }
@@ -125,7 +129,7 @@ cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N, const 
                               void* y, cudaStream_t s) {
   if (rows <= 0 || N <= 0) return cudaSuccess;
   if (N % 4 || S < 1) return cudaErrorInvalidValue;
-  splitk_sum_kernel<<<counted(grid_for(rows, N)), kThreads, 0, s>>>(
+  (void)launch_pdl(splitk_sum_kernel, dim3(grid_for(rows, N)), dim3(kThreads), 0, s, 
       p, S, rows, N, n_rows, static_cast<__nv_bfloat16*>(y));
   return cudaGetLastError();
 }

@@ -266,3 +266,17 @@ def test_gathering_up_projection_matches_the_permuted_one(name):
     torch.cuda.synchronize()
     assert M.get_device_error() == 0
     assert torch.equal(h1[:n], h2[:n])
+
+
+def test_layer_without_programmatic_dependent_launch_in_subprocess():
+    """MOE_PDL=0 launches every kernel without programmatic stream serialization (each waits
+    for the previous one to finish before it is scheduled); the small-case parity tests pass
+    there too."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_PDL="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "small_layer_matches_oracle or full_size_workload and mixtral"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
