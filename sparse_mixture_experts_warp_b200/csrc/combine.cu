@@ -88,7 +88,36 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
     n += __popc(live);
   }
   __syncwarp();
-  for (int v = lane; v < nvec; v += 32) {
+  // four 16-byte chunks per lane at a time: the loads of one assignment row are all in flight
+  // before they are accumulated (the same fixed order of the sum as one chunk at a time)
+  int v = lane;
+  for (; v + 96 < nvec; v += 128) {
+    float a[4][R::N];
+#pragma unroll
+    for (int c = 0; c < 4; ++c)
+#pragma unroll
+      for (int i = 0; i < R::N; ++i) a[c][i] = 0.f;
+    for (int q = 0; q < n; ++q) {
+      const uint4* src = y + (int64_t)s_row[warp][q] * nvec + v;
+      const float gq = s_g[warp][q];
+      uint4 u[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) u[c] = __ldcs(src + 32 * c);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) R::acc_val(u[c], gq, a[c]);
+    }
+    for (int s = 0; s < S; ++s) {
+      const uint4* src = ys + ((int64_t)s * T + t) * nvec + v;
+      uint4 u[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) u[c] = __ldcs(src + 32 * c);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) R::acc_val(u[c], 1.0f, a[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < 4; ++c) R::store(out + (int64_t)t * nvec + v + 32 * c, a[c]);
+  }
+  for (; v < nvec; v += 32) {
     float a[R::N];
 #pragma unroll
     for (int i = 0; i < R::N; ++i) a[i] = 0.f;
