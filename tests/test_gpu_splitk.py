@@ -29,6 +29,16 @@ CASES = {
 }
 
 
+def _x_perm(w, inp, v):
+    """The grouped token rows, by moe_permute (a layer forward that gathers its rows inside the
+    up projection leaves the workspace's x_perm unwritten)."""
+    d = M.desc_of(w)
+    xp = torch.empty_like(v["x_perm"])
+    M.moe_permute(d, v["expert_ids"], inp.x, xp, v["counts"], v["offsets"], v["row_src"],
+                  v["inv"], v["scratch"])
+    return xp
+
+
 def _rel(a, b):
     den = b.abs().max().item()
     return (a - b).abs().max().item() / den if den > 0 else (a - b).abs().max().item()
@@ -45,9 +55,10 @@ def test_ws_products_match_fused_products(name):
     scratch = v["scratch"]
     h0 = torch.zeros_like(v["h"])
     h1 = torch.zeros_like(v["h"])
-    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
+    xp = _x_perm(w, inp, v)
+    M.moe_expert_up(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h0)
     k0 = M.kernel_launches()
-    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1, scratch)
+    M.moe_expert_up_ws(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h1, scratch)
     up_launches = M.kernel_launches() - k0
     y0 = torch.zeros_like(v["y"])
     y1 = torch.zeros_like(v["y"])
@@ -70,9 +81,10 @@ def test_ws_without_scratch_runs_the_fused_products():
     out, v = C.run_layer(w, inp)
     d = M.desc_of(w)
     h0, h1 = torch.zeros_like(v["h"]), torch.zeros_like(v["h"])
-    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
+    xp = _x_perm(w, inp, v)
+    M.moe_expert_up(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h0)
     k0 = M.kernel_launches()
-    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1, None)
+    M.moe_expert_up_ws(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h1, None)
     assert M.kernel_launches() - k0 == 1
     y0, y1 = torch.zeros_like(v["y"]), torch.zeros_like(v["y"])
     M.moe_expert_down(d, w.E, w.F, h0, v["offsets"], inp.W_down, y0)
@@ -88,8 +100,9 @@ def test_ws_with_many_rows_runs_the_fused_products():
     out, v = C.run_layer(w, inp)
     d = M.desc_of(w)
     h0, h1 = torch.zeros_like(v["h"]), torch.zeros_like(v["h"])
-    M.moe_expert_up(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h0)
-    M.moe_expert_up_ws(d, w.E, w.F, v["x_perm"], v["offsets"], inp.W_gate, inp.W_up, h1,
+    xp = _x_perm(w, inp, v)
+    M.moe_expert_up(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h0)
+    M.moe_expert_up_ws(d, w.E, w.F, xp, v["offsets"], inp.W_gate, inp.W_up, h1,
                        v["scratch"])
     torch.cuda.synchronize()
     assert torch.equal(h0, h1)
