@@ -240,9 +240,10 @@ moe_status_t moe_expert_up_gather(const moe_desc_t* desc, int32_t n_groups, int3
                                   const int32_t* offsets, const void* W_gate, const void* W_up,
                                   void* h, moe_stream_t stream);
 
-/* Whether moe_layer_forward uses that fusion for this desc (*on = 1): bf16, more than 16
- * grouped rows (fewer take the small-batch schedule on x_perm), and not disabled by
- * MOE_GATHER_FUSION=0 in the environment.  Host only. */
+/* Whether moe_layer_forward uses that fusion for this desc (*on = 1): MOE_GATHER_FUSION=1 in the
+ * environment (it is off by default: measured slower than the tiled loads of x_perm, whose
+ * write it saves), bf16, more than 16 grouped rows (fewer take the small-batch schedule on
+ * x_perm).  Host only. */
 moe_status_t moe_gather_fusion(const moe_desc_t* desc, int32_t* on);
 
 /* moe_expert_up / moe_expert_down with a scratch area for the small-batch (decode) schedule

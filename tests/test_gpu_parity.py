@@ -227,14 +227,14 @@ def test_v3_node_limited_full_size():
     C.check_stratified_output(w, inp, out, v, seed=124, every_slice=False)
 
 
-def test_layer_without_gather_fusion_in_subprocess():
-    """MOE_GATHER_FUSION=0 makes moe_layer_forward write the grouped copy x_perm and run the up
-    projection on it (instead of gathering the token rows inside it); the small-case parity
-    tests pass there too, x_perm checked row by row against the tokens."""
+def test_layer_with_gather_fusion_in_subprocess():
+    """MOE_GATHER_FUSION=1 makes moe_layer_forward gather the token rows inside the up
+    projection (the permutation writes indices only, x_perm stays unwritten); the small-case
+    parity tests pass there too."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, MOE_GATHER_FUSION="0")
+    env = dict(os.environ, MOE_GATHER_FUSION="1")
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
                         "small_layer_matches_oracle"], env=env, capture_output=True, text=True,
                        timeout=900)
