@@ -252,13 +252,16 @@ router_kernel(RouterArgs a) {
     }
 
     if (a.expert_choice) {
-      // merge weights are the softmax probabilities; selection happens per expert later
+      // merge weights are the softmax probabilities; selection happens per expert later.  The
+      // transposed copy goes through shared memory ([token][E+1]) so that it leaves as rows of
+      // the block's 32 consecutive tokens (below)
+      float* s_pT = s_all + kWarps * kTPW * E;
 #pragma unroll
       for (int i = 0; i < kMaxEPL; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
           a.gates[(int64_t)tok * E + e] = p[i];
-          a.probsT[(int64_t)e * a.T + tok] = p[i];
+          s_pT[(warp * kTPW + t) * (E + 1) + e] = p[i];
         }
       }
       continue;
@@ -301,6 +304,18 @@ router_kernel(RouterArgs a) {
       const float g = (a.gate == MOE_GATE_RENORM) ? my_w / wsum : my_w;
       a.ids[(int64_t)tok * a.k + lane] = my_id;
       a.gates[(int64_t)tok * a.k + lane] = g;
+    }
+  }
+
+  if (a.expert_choice) {
+    // probsT[e][t] for the block's 32 tokens: 128-byte rows per expert (conflict-free reads:
+    // the row pitch E + 1 puts the 32 tokens of one expert in 32 different banks)
+    const float* s_pT = s_all + kWarps * kTPW * E;
+    const int tb = blockIdx.x * kWarps * kTPW;
+    __syncthreads();
+    for (int i = threadIdx.x; i < E * kWarps * kTPW; i += blockDim.x) {
+      const int e = i / (kWarps * kTPW), j = i % (kWarps * kTPW);
+      if (tb + j < a.T) a.probsT[(int64_t)e * a.T + tb + j] = s_pT[j * (E + 1) + e];
     }
   }
 
@@ -681,7 +696,8 @@ int router_partials(const moe_desc_t& d) {
 static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStream_t s) {
   const int blocks = (T + kWarps * kTPW - 1) / (kWarps * kTPW);
   if (blocks == 0) return cudaSuccess;
-  const size_t smem = (size_t)kWarps * kTPW * a.E * sizeof(float);
+  size_t smem = (size_t)kWarps * kTPW * a.E * sizeof(float);
+  if (a.expert_choice) smem += (size_t)kWarps * kTPW * (a.E + 1) * sizeof(float);
   if (bf16) {
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
