@@ -114,21 +114,21 @@ __device__ __forceinline__ void group_limit(float (&key)[NS], int E, int n_group
 }
 
 // logits of the warp's TPW tokens for all experts -> s_log[TPW][E]
-template <bool BF16>
+template <bool BF16, int TPW>
 __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* s_log, int lane) {
   using C = Chunk<BF16>;
   const int nvec = a.D / C::N;
   for (int e0 = 0; e0 < a.E; e0 += kEB) {
-    float acc[kTPW][kEB];
+    float acc[TPW][kEB];
 #pragma unroll
-    for (int t = 0; t < kTPW; ++t)
+    for (int t = 0; t < TPW; ++t)
 #pragma unroll
       for (int e = 0; e < kEB; ++e) acc[t][e] = 0.f;
     const int ne = min(kEB, a.E - e0);
     for (int v = lane; v < nvec; v += 32) {
-      float xv[kTPW][C::N];
+      float xv[TPW][C::N];
 #pragma unroll
-      for (int t = 0; t < kTPW; ++t) {
+      for (int t = 0; t < TPW; ++t) {
         if (t0 + t < a.T) {
           C::load(a.x, (int64_t)(t0 + t) * a.D + (int64_t)v * C::N, xv[t]);
         } else {
@@ -142,14 +142,14 @@ __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* 
           float wv[C::N];
           C::load(a.Wg, (int64_t)(e0 + e) * a.D + (int64_t)v * C::N, wv);
 #pragma unroll
-          for (int t = 0; t < kTPW; ++t)
+          for (int t = 0; t < TPW; ++t)
 #pragma unroll
             for (int i = 0; i < C::N; ++i) acc[t][e] = fmaf(xv[t][i], wv[i], acc[t][e]);
         }
       }
     }
 #pragma unroll
-    for (int t = 0; t < kTPW; ++t)
+    for (int t = 0; t < TPW; ++t)
 #pragma unroll
       for (int e = 0; e < kEB; ++e) {
         float v = warp_sum(acc[t][e]);
@@ -159,7 +159,9 @@ __device__ __forceinline__ void warp_logits(const RouterArgs& a, int t0, float* 
   __syncwarp();
 }
 
-template <bool BF16>
+// TPW tokens per warp: 4 when the warp computes the logits itself (W_g loads shared by 4
+// tokens), 1 when they come from the tensor-core product (more warps in flight).
+template <bool BF16, int TPW>
 __global__ void __launch_bounds__(kWarps * 32)
 router_kernel(RouterArgs a) {
   pdl_trigger();
@@ -167,12 +169,12 @@ router_kernel(RouterArgs a) {
   extern __shared__ float s_all[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gw = blockIdx.x * kWarps + warp;
-  const int t0 = gw * kTPW;
-  float* s_log = s_all + warp * kTPW * a.E;
+  const int t0 = gw * TPW;
+  float* s_log = s_all + warp * TPW * a.E;
 
   if (a.lpart) {
     // logits from the tensor-core router product: fixed-order sum of the k-split partials
-    for (int t = 0; t < kTPW; ++t) {
+    for (int t = 0; t < TPW; ++t) {
       const int tok = t0 + t;
       if (tok >= a.T) break;
       for (int e = lane; e < a.E; e += 32) {
@@ -184,7 +186,7 @@ router_kernel(RouterArgs a) {
     }
     __syncwarp();
   } else {
-    warp_logits<BF16>(a, t0, s_log, lane);
+    warp_logits<BF16, TPW>(a, t0, s_log, lane);
   }
 
   const int E = a.E;
@@ -193,7 +195,7 @@ router_kernel(RouterArgs a) {
   for (int i = 0; i < kMaxEPL; ++i) imp[i] = 0.f;
   float ent = 0.f;                 // this lane's share of the tokens' -sum p log p
 
-  for (int t = 0; t < kTPW; ++t) {
+  for (int t = 0; t < TPW; ++t) {
     const int tok = t0 + t;
     if (tok >= a.T) break;
     float s[kMaxEPL], p[kMaxEPL], key[kMaxEPL];
@@ -255,13 +257,13 @@ router_kernel(RouterArgs a) {
       // merge weights are the softmax probabilities; selection happens per expert later.  The
       // transposed copy goes through shared memory ([token][E+1]) so that it leaves as rows of
       // the block's 32 consecutive tokens (below)
-      float* s_pT = s_all + kWarps * kTPW * E;
+      float* s_pT = s_all + kWarps * TPW * E;
 #pragma unroll
       for (int i = 0; i < kMaxEPL; ++i) {
         const int e = lane + 32 * i;
         if (e < E) {
           a.gates[(int64_t)tok * E + e] = p[i];
-          s_pT[(warp * kTPW + t) * (E + 1) + e] = p[i];
+          s_pT[(warp * TPW + t) * (E + 1) + e] = p[i];
         }
       }
       continue;
@@ -310,11 +312,11 @@ router_kernel(RouterArgs a) {
   if (a.expert_choice) {
     // probsT[e][t] for the block's 32 tokens: 128-byte rows per expert (conflict-free reads:
     // the row pitch E + 1 puts the 32 tokens of one expert in 32 different banks)
-    const float* s_pT = s_all + kWarps * kTPW * E;
-    const int tb = blockIdx.x * kWarps * kTPW;
+    const float* s_pT = s_all + kWarps * TPW * E;
+    const int tb = blockIdx.x * kWarps * TPW;
     __syncthreads();
-    for (int i = threadIdx.x; i < E * kWarps * kTPW; i += blockDim.x) {
-      const int e = i / (kWarps * kTPW), j = i % (kWarps * kTPW);
+    for (int i = threadIdx.x; i < E * kWarps * TPW; i += blockDim.x) {
+      const int e = i / (kWarps * TPW), j = i % (kWarps * TPW);
       if (tb + j < a.T) a.probsT[(int64_t)e * a.T + tb + j] = s_pT[j * (E + 1) + e];
     }
   }
@@ -682,31 +684,41 @@ router_fast_kernel(RouterArgs a, int tokens_per_cta) {
 
 }  // namespace
 
+// Tokens per warp of the generic kernel: 1 when the logits come from the tensor-core product.
+static int router_tpw(bool lpart) { return lpart ? 1 : kTPW; }
+
 // Rows of importance partials the generic kernel writes (one per block).
-static int generic_partials(const moe_desc_t& d) {
-  return (d.T + kWarps * kTPW - 1) / (kWarps * kTPW);
+static int generic_partials(const moe_desc_t& d, bool lpart) {
+  const int per_block = kWarps * router_tpw(lpart);
+  return (d.T + per_block - 1) / per_block;
 }
 
 int router_partials(const moe_desc_t& d) {
-  // capacity for either kernel: generic = one row per warp; fast = one row per CTA (<= 1024)
-  const int generic = generic_partials(d);
+  // capacity for either kernel: generic = one row per block of 8 (or 32) tokens; fast = one
+  // row per CTA (<= 1024)
+  const int generic = generic_partials(d, true);
   return generic > 1024 ? generic : 1024;
 }
 
+template <bool BF16, int TPW>
+static void launch_router_tpw(const RouterArgs& a, int T, cudaStream_t s) {
+  const int blocks = (T + kWarps * TPW - 1) / (kWarps * TPW);
+  size_t smem = (size_t)kWarps * TPW * a.E * sizeof(float);
+  if (a.expert_choice) smem += (size_t)kWarps * TPW * (a.E + 1) * sizeof(float);
+  if (smem > 48 * 1024)
+    cudaFuncSetAttribute(router_kernel<BF16, TPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                         (int)smem);
+  (void)launch_pdl(router_kernel<BF16, TPW>, dim3(blocks), dim3(kWarps * 32), smem, s, a);
+}
+
 static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStream_t s) {
-  const int blocks = (T + kWarps * kTPW - 1) / (kWarps * kTPW);
-  if (blocks == 0) return cudaSuccess;
-  size_t smem = (size_t)kWarps * kTPW * a.E * sizeof(float);
-  if (a.expert_choice) smem += (size_t)kWarps * kTPW * (a.E + 1) * sizeof(float);
-  if (bf16) {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(router_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    (void)launch_pdl(router_kernel<true>, dim3(blocks), dim3(kWarps * 32), smem, s, a);
-  } else {
-    if (smem > 48 * 1024)
-      cudaFuncSetAttribute(router_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    (void)launch_pdl(router_kernel<false>, dim3(blocks), dim3(kWarps * 32), smem, s, a);
-  }
+  if (T <= 0) return cudaSuccess;
+  if (a.lpart)
+    launch_router_tpw<true, 1>(a, T, s);        // the tensor-core product is bf16-only
+  else if (bf16)
+    launch_router_tpw<true, kTPW>(a, T, s);
+  else
+    launch_router_tpw<false, kTPW>(a, T, s);
   return cudaGetLastError();
 }
 
@@ -750,7 +762,7 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
     (void)launch_pdl(router_fast_kernel, dim3(grid), dim3((d.D / 256) * 32), 0, s, a, tpc);
     return cudaGetLastError();
   }
-  *n_partials = generic_partials(d);
+  *n_partials = generic_partials(d, a.lpart != nullptr);
   return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
@@ -758,7 +770,6 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
                                         float* probs, float* probsT, float* logits,
                                         float* imp_partials, int* n_partials, float* lpart,
                                         cudaStream_t s) {
-  *n_partials = generic_partials(d);
   RouterArgs a{x, Wg, nullptr, nullptr, probs, logits, probsT, imp_partials,
                d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1, nullptr, 1};
   if (router_uses_gemm(d) && lpart) {
@@ -768,6 +779,7 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
     a.lpart = lpart;
     a.ksplit = ks;
   }
+  *n_partials = generic_partials(d, a.lpart != nullptr);
   return launch_router(a, d.dtype == MOE_BF16, d.T, s);
 }
 
