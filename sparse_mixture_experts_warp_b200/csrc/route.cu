@@ -703,8 +703,14 @@ int router_partials(const moe_desc_t& d) {
 template <bool BF16, int TPW>
 static void launch_router_tpw(const RouterArgs& a, int T, cudaStream_t s) {
   const int blocks = (T + kWarps * TPW - 1) / (kWarps * TPW);
-  size_t smem = (size_t)kWarps * TPW * a.E * sizeof(float);
-  if (a.expert_choice) smem += (size_t)kWarps * TPW * (a.E + 1) * sizeof(float);
+  // the warps' logits [kWarps * TPW][E] (then, under expert choice, the transposed
+  // probabilities [kWarps * TPW][E + 1] after them); the partial rows [kWarps][E + 1] reuse the
+  // start of the buffer at the end, so it holds at least that many
+  size_t words = (size_t)kWarps * TPW * a.E;
+  if (a.expert_choice) words += (size_t)kWarps * TPW * (a.E + 1);
+  const size_t part_words = (size_t)kWarps * (a.E + 1);
+  if (words < part_words) words = part_words;
+  const size_t smem = words * sizeof(float);
   if (smem > 48 * 1024)
     cudaFuncSetAttribute(router_kernel<BF16, TPW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                          (int)smem);
