@@ -13,7 +13,11 @@
 // holds the token's E logits in shared memory and does the per-token affinity, a k-round warp
 // arg-max for top-k, and the merge weights.  Everything stays on chip except x, W_g and the
 // outputs.
+#include <stdlib.h>
+#include <string.h>
+
 #include "common.cuh"
+#include "route_select.cuh"
 
 namespace moe {
 namespace {
@@ -21,18 +25,6 @@ namespace {
 constexpr int kTPW = 4;          // tokens per warp
 constexpr int kWarps = 8;        // warps per block
 constexpr int kEB = 8;           // experts per accumulation block
-constexpr int kMaxEPL = 8;       // experts per lane in the selection phase (E <= 256)
-
-__device__ __forceinline__ float warp_sum(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-  return v;
-}
-__device__ __forceinline__ float warp_max(float v) {
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-  return v;
-}
 
 // 16 bytes of x or W_g as fp32 values.
 template <bool BF16> struct Chunk;
@@ -55,63 +47,6 @@ template <> struct Chunk<false> {
     out[0] = f.x; out[1] = f.y; out[2] = f.z; out[3] = f.w;
   }
 };
-
-struct RouterArgs {
-  const void* x; const void* Wg; const float* bias;
-  int32_t* ids; float* gates; float* logits; float* probsT; float* partials;
-  int T, D, E, k, score, gate, expert_choice;
-  const float* lpart;       // when set: logits are the sum of ksplit partials [ksplit][T][E]
-  int ksplit;
-  int n_group = 1, topk_group = 1;   // group-limited selection (n_group <= 1: none)
-};
-
-// Group-limited selection ("Mixture of Experts (MoE)" routing variant (c): groups first, then
-// experts inside them; moe-comparison "Group/node limited" row).  The experts form n_group
-// contiguous groups of size = E / n_group; a group scores its largest key, the token keeps its
-// topk_group best groups (ties to the lower group) and every other expert's key becomes -inf.
-// Lane l holds experts l + 32 i in key[i].  size is a power of two <= 32 (a group lies inside
-// one register slot: a segmented shuffle max) or a multiple of 32 (a slot lies inside one
-// group: a warp max); n_group <= 32, so lane g can hold group g's score.
-template <int NS>
-__device__ __forceinline__ void group_limit(float (&key)[NS], int E, int n_group, int topk_group,
-                                            int lane) {
-  if (n_group <= 1 || topk_group >= n_group) return;
-  const int size = E / n_group;
-  float gs = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < NS; ++i) {
-    if (32 * i >= E) break;
-    float v = (lane + 32 * i < E) ? key[i] : -INFINITY;
-    if (size < 32) {
-      for (int o = size >> 1; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
-      const int src = lane * size - 32 * i;     // first lane of group `lane` in slot i
-      const float w = __shfl_sync(0xffffffffu, v, src & 31);
-      if (lane < n_group && src >= 0 && src < 32) gs = fmaxf(gs, w);
-    } else {
-      v = warp_max(v);
-      if (lane == (32 * i) / size) gs = fmaxf(gs, v);
-    }
-  }
-  uint32_t kept = 0;
-  bool used = lane >= n_group;
-  for (int r = 0; r < topk_group; ++r) {
-    float bk = used ? -INFINITY : gs;
-    int bi = used ? 0x7fffffff : lane;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ok > bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-    }
-    kept |= 1u << (bi & 31);
-    if (lane == bi) used = true;
-  }
-#pragma unroll
-  for (int i = 0; i < NS; ++i) {
-    const int e = lane + 32 * i;
-    if (e < E && !((kept >> (e / size)) & 1u)) key[i] = -INFINITY;
-  }
-}
 
 // logits of the warp's TPW tokens for all experts -> s_log[TPW][E]
 template <bool BF16, int TPW>
@@ -198,114 +133,22 @@ router_kernel(RouterArgs a) {
   for (int t = 0; t < TPW; ++t) {
     const int tok = t0 + t;
     if (tok >= a.T) break;
-    float s[kMaxEPL], p[kMaxEPL], key[kMaxEPL];
-    float m = -INFINITY;
+    float s[kMaxEPL], p[kMaxEPL];
 #pragma unroll
     for (int i = 0; i < kMaxEPL; ++i) {
       const int e = lane + 32 * i;
       s[i] = (e < E) ? s_log[t * E + e] : -INFINITY;
-      m = fmaxf(m, s[i]);
     }
-    if (a.logits) {
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E) a.logits[(int64_t)tok * E + e] = s[i];
-      }
-    }
-    float sel_w[kMaxEPL];   // weight used in the merge (softmax p or sigmoid affinity)
-    if (a.score == MOE_SCORE_SOFTMAX) {
-      m = warp_max(m);
-      float z = 0.f;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        const int e = lane + 32 * i;
-        p[i] = (e < E) ? expf(s[i] - m) : 0.f;
-        z += p[i];
-      }
-      z = warp_sum(z);
-      const float inv = 1.0f / z;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        p[i] = p[i] * inv;
-        key[i] = s[i];             // softmax is monotone in the logit within a row
-        sel_w[i] = p[i];
-        imp[i] += p[i];
-        if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
-      }
-    } else {
-      float asum = 0.f;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        const int e = lane + 32 * i;
-        const float af = (e < E) ? 1.0f / (1.0f + expf(-s[i])) : 0.f;
-        sel_w[i] = af;
-        key[i] = (e < E) ? af + (a.bias ? a.bias[e] : 0.f) : -INFINITY;
-        asum += af;
-      }
-      asum = warp_sum(asum);
-      const float inv = 1.0f / asum;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        p[i] = sel_w[i] * inv;
-        imp[i] += p[i];
-        if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
-      }
-    }
-
+    select_token<kMaxEPL>(a, tok, s, imp, ent, p, lane);
     if (a.expert_choice) {
-      // merge weights are the softmax probabilities; selection happens per expert later.  The
-      // transposed copy goes through shared memory ([token][E+1]) so that it leaves as rows of
-      // the block's 32 consecutive tokens (below)
+      // the transposed copy goes through shared memory ([token][E+1]) so that it leaves as
+      // rows of the block's 32 consecutive tokens (below)
       float* s_pT = s_all + kWarps * TPW * E;
 #pragma unroll
       for (int i = 0; i < kMaxEPL; ++i) {
         const int e = lane + 32 * i;
-        if (e < E) {
-          a.gates[(int64_t)tok * E + e] = p[i];
-          s_pT[(warp * TPW + t) * (E + 1) + e] = p[i];
-        }
+        if (e < E) s_pT[(warp * TPW + t) * (E + 1) + e] = p[i];
       }
-      continue;
-    }
-
-    group_limit<kMaxEPL>(key, E, a.n_group, a.topk_group, lane);
-
-    // top-k: k rounds of a warp arg-max over (key desc, expert id asc)
-    bool taken[kMaxEPL];
-#pragma unroll
-    for (int i = 0; i < kMaxEPL; ++i) taken[i] = false;
-    int my_id = -1;        // lane j < k keeps slot j
-    float my_w = 0.f;
-    float wsum = 0.f;
-    for (int j = 0; j < a.k; ++j) {
-      float bk = -INFINITY;
-      int bi = 0x7fffffff;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i) {
-        const int e = lane + 32 * i;
-        if (e < E && !taken[i] && (key[i] > bk || (key[i] == bk && e < bi))) { bk = key[i]; bi = e; }
-      }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-        const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-        if (ok > bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-      }
-      // owner lane marks it and broadcasts its merge weight
-      const int owner = bi & 31, slot = bi >> 5;
-      float w = 0.f;
-#pragma unroll
-      for (int i = 0; i < kMaxEPL; ++i)
-        if (lane == owner && i == slot) { taken[i] = true; w = sel_w[i]; }
-      w = __shfl_sync(0xffffffffu, w, owner);
-      wsum += w;
-      if (lane == j) { my_id = bi; my_w = w; }
-    }
-    if (lane < a.k) {
-      const float g = (a.gate == MOE_GATE_RENORM) ? my_w / wsum : my_w;
-      a.ids[(int64_t)tok * a.k + lane] = my_id;
-      a.gates[(int64_t)tok * a.k + lane] = g;
     }
   }
 
@@ -728,11 +571,30 @@ static cudaError_t launch_router(const RouterArgs& a, bool bf16, int T, cudaStre
   return cudaGetLastError();
 }
 
-// Router product on tensor cores (the grouped GEMM engine, fp32 partial logits) for bf16
-// inputs with many experts; the SIMT dot products of the generic kernel re-read x per block of 8
-// experts and W_g per 4 tokens, which is far from the HBM roofline at E >= 32.
+// Router path.  Default: for bf16 with at most 8 experts the mma.sync kernel (when D is a
+// multiple of 256 between 1024 and 4096: measured faster there), otherwise the tensor-core
+// router fused with the selection (router_tc.cu: bf16, D % 64 == 0, E <= 256), otherwise the
+// SIMT kernel.  MOE_ROUTER selects one path for comparison measurements (each is tested):
+// "tc", "fast" (mma.sync, E <= 8), "gemm" (the grouped-GEMM router product, k-split fp32
+// partial logits in the step scratch, then the SIMT selection kernel) or "simt".
+enum RouterMode { ROUTER_AUTO = -1, ROUTER_TC = 0, ROUTER_GEMM = 1, ROUTER_FAST = 2, ROUTER_SIMT = 3 };
+static int router_env() {
+  static int v = [] {
+    const char* e = getenv("MOE_ROUTER");
+    if (!e) return (int)ROUTER_AUTO;
+    if (!strcmp(e, "tc")) return (int)ROUTER_TC;
+    if (!strcmp(e, "gemm")) return (int)ROUTER_GEMM;
+    if (!strcmp(e, "fast")) return (int)ROUTER_FAST;
+    if (!strcmp(e, "simt")) return (int)ROUTER_SIMT;
+    return (int)ROUTER_AUTO;
+  }();
+  return v;
+}
+
+// The grouped-GEMM router product (MOE_ROUTER=gemm): bf16, 32 <= E <= 256, E % 32 == 0.
 bool router_uses_gemm(const moe_desc_t& d) {
-  return d.dtype == MOE_BF16 && d.E >= 32 && d.E % 32 == 0 && d.E <= 256 && d.D % 64 == 0;
+  return router_env() == ROUTER_GEMM && d.dtype == MOE_BF16 && d.E >= 32 && d.E % 32 == 0 &&
+         d.E <= 256 && d.D % 64 == 0;
 }
 
 size_t router_gemm_scratch_bytes(const moe_desc_t& d) {
@@ -744,6 +606,16 @@ static bool fast_router_ok(const moe_desc_t& d) {
          d.D % 256 == 0 && d.D / 256 >= 4 && d.D / 256 <= kFastMaxNW && d.k <= 32;
 }
 
+static bool use_router_fast(const moe_desc_t& d) {
+  const int m = router_env();
+  return (m == ROUTER_AUTO || m == ROUTER_FAST) && fast_router_ok(d);
+}
+
+static bool use_router_tc(const moe_desc_t& d) {
+  const int m = router_env();
+  return (m == ROUTER_TC || (m == ROUTER_AUTO && !fast_router_ok(d))) && router_tc_ok(d);
+}
+
 cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const void* Wg,
                                        const float* bias, int32_t* ids, float* gates,
                                        float* logits, float* imp_partials, int* n_partials,
@@ -752,6 +624,7 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
                d.T, d.D, d.E, d.k, d.score, d.gate, 0, nullptr, 1};
   a.n_group = d.n_group;
   a.topk_group = d.topk_group;
+  if (use_router_tc(d)) return launch_router_tc(d, a, n_partials, s);
   if (router_uses_gemm(d) && lpart) {
     const int ks = router_gemm_splits(d.T, d.D);
     cudaError_t e = launch_router_gemm_bf16(x, d.T, d.D, Wg, d.E, lpart, ks, s);
@@ -759,7 +632,7 @@ cudaError_t launch_router_token_choice(const moe_desc_t& d, const void* x, const
     a.lpart = lpart;
     a.ksplit = ks;
   }
-  if (fast_router_ok(d)) {
+  if (use_router_fast(d)) {
     const int sms = num_sms() < 1024 ? num_sms() : 1024;
     const int tpc = (d.T + sms - 1) / sms;
     const int grid = tpc > 0 ? (d.T + tpc - 1) / tpc : 0;
@@ -778,6 +651,7 @@ cudaError_t launch_router_expert_choice(const moe_desc_t& d, const void* x, cons
                                         cudaStream_t s) {
   RouterArgs a{x, Wg, nullptr, nullptr, probs, logits, probsT, imp_partials,
                d.T, d.D, d.E, 0, MOE_SCORE_SOFTMAX, MOE_GATE_RAW, 1, nullptr, 1};
+  if (use_router_tc(d)) return launch_router_tc(d, a, n_partials, s);
   if (router_uses_gemm(d) && lpart) {
     const int ks = router_gemm_splits(d.T, d.D);
     cudaError_t e = launch_router_gemm_bf16(x, d.T, d.D, Wg, d.E, lpart, ks, s);

@@ -33,16 +33,29 @@ SMALL = {
     "switch_small": scaled(W["switch"], T=3000, D=256, E=16, F=512),
     "v3_small": scaled(W["v3"], T=300, D=512, E=64, F=256, F_shared=256),
     "ec_small": scaled(W["ec"], T=1000, D=256, E=16, F=256, c=125),
-    # the bf16 router fast path (E <= 8, D = 256 * NW, 4 <= NW <= 16), ragged token counts
-    "fast_router_T1": scaled(W["mixtral"], T=1, D=4096, F=256),
-    "fast_router_T37": scaled(W["mixtral"], T=37, D=1024, F=256),
-    "fast_router_T300_E6": scaled(W["mixtral"], T=300, D=2048, E=6, F=256),
-    "fast_router_switch_k1": scaled(W["switch"], T=500, D=1024, E=8, F=256),
-    "fast_router_sigmoid_shared": scaled(W["v3"], T=200, D=1024, E=8, k=2, F=256, F_shared=256),
-    # router product on the tensor-core engine (bf16, E >= 32): ragged T, k-splits
-    "gemm_router_switch_E32": scaled(W["switch"], T=300, D=256, E=32, F=256),
-    "gemm_router_v3_E64": scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
-    "gemm_router_ec_E64": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
+    # router shapes.  By default bf16 with E <= 8 and D = 256 * NW (4 <= NW <= 16) runs the
+    # mma.sync router and the rest the tensor-core router; in subprocesses below the router
+    # cases also run through the tensor-core router (MOE_ROUTER=tc), the mma.sync router
+    # (MOE_ROUTER=fast), the grouped-GEMM router product (E % 32 == 0: MOE_ROUTER=gemm) and
+    # the CUDA-core router (MOE_ROUTER=simt).  E <= 8, ragged token counts
+    "router_E8_T1": scaled(W["mixtral"], T=1, D=4096, F=256),
+    "router_E8_T37": scaled(W["mixtral"], T=37, D=1024, F=256),
+    "router_E6_T300": scaled(W["mixtral"], T=300, D=2048, E=6, F=256),
+    "router_E8_switch_k1": scaled(W["switch"], T=500, D=1024, E=8, F=256),
+    "router_E8_sigmoid_shared": scaled(W["v3"], T=200, D=1024, E=8, k=2, F=256, F_shared=256),
+    # E >= 32: ragged T, one to four k-ranges per 128-token tile
+    "router_E32_switch": scaled(W["switch"], T=300, D=256, E=32, F=256),
+    "router_E64_v3": scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
+    "router_E64_ec": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
+    # tensor-core router: E not a multiple of 16 (N = 48 of which 40 live, 64 TMEM columns;
+    # 8 tiles, 4 k-ranges of 3 k-blocks), one k-range per tile over more tiles than SMs, and
+    # expert choice over 256 experts (the largest E with the DeepSeek-V3 group limit is
+    # groups_E256_v3_node below)
+    "router_E40_T1000": scaled(W["switch"], T=1000, D=768, E=40, F=128, capacity_factor=2.0),
+    "groups_E256_v3_node": scaled(W["v3"], T=130, D=1024, F=128, F_shared=128, n_group=8,
+                                  topk_group=4),
+    "router_E16_T20000": scaled(W["mixtral"], T=20000, D=128, E=16, k=2, F=64),
+    "router_E256_ec": scaled(W["ec"], T=600, D=512, E=256, F=128, c=10),
     # the classic D -> F -> D expert with GELU (bf16 tensor-core epilogue, fp32 CUDA cores)
     "gelu_bf16": scaled(W["switch"], act="gelu", T=500, D=256, E=16, F=512, overflow="dropless",
                         gate="renorm", k=2, zipf_s=0.0),
@@ -59,16 +72,16 @@ SMALL = {
     # group-limited selection: fast router (groups of 2 experts, softmax; groups of 2, sigmoid
     # with selection bias), generic fp32 router (groups of 4), tensor-core router (groups of
     # 32 = one register slot, and of 64 = two slots)
-    "groups_fast_softmax": scaled(W["mixtral"], T=300, D=1024, E=8, k=2, F=256, n_group=4,
+    "groups_E8_softmax": scaled(W["mixtral"], T=300, D=1024, E=8, k=2, F=256, n_group=4,
                                   topk_group=1),
-    "groups_fast_sigmoid": scaled(W["v3"], T=200, D=1024, E=8, k=3, F=256, F_shared=256,
+    "groups_E8_sigmoid": scaled(W["v3"], T=200, D=1024, E=8, k=3, F=256, F_shared=256,
                                   n_group=4, topk_group=2),
     "groups_f32_generic": scaled(W["v3"], dtype="f32", T=90, D=64, E=16, F=32, k=3,
                                  n_shared=1, F_shared=40, w_std=0.1, wg_std=0.1, n_group=4,
                                  topk_group=2),
-    "groups_gemm_router_32": scaled(W["v3"], T=300, D=512, E=64, F=256, F_shared=256,
+    "groups_E64_size32": scaled(W["v3"], T=300, D=512, E=64, F=256, F_shared=256,
                                     n_group=2, topk_group=1),
-    "groups_gemm_router_64": scaled(W["v3"], T=300, D=512, E=128, k=4, F=256, F_shared=256,
+    "groups_E128_size64": scaled(W["v3"], T=300, D=512, E=128, k=4, F=256, F_shared=256,
                                     n_group=2, topk_group=1),
 }
 
@@ -156,7 +169,7 @@ def test_decode_regime_mixtral_shape(T):
 
 # A few executed rows (bf16) take the k-split expert schedule: fp32 partials of the up and down
 # products summed by splitk.cu.  ReLU at the full Switch layer with its capacity limit (up split
-# 3, down split 8) and GELU (splits 4 and 2); SwiGLU is covered by fast_router_T1 (up split 7)
+# 3, down split 8) and GELU (splits 4 and 2); SwiGLU is covered by router_E8_T1 (up split 7)
 # and T = 1 above (up 5, down 4).  Every token against the oracle, which evaluates only the
 # experts in use.
 DECODE = {
@@ -189,12 +202,13 @@ def test_decode_split_schedule_matches_fused_path_in_subprocess():
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
 
 
-# The bf16 fast router at larger token counts: each CTA routes several 16-token batches, the
-# last one ragged (T=5000, D=4096: 34 tokens per CTA; T=9000, D=1024: 61; T=12000, D=4096:
-# 82).  Logits of every token, the whole routing, permutation and statistics are compared
-# with the oracle.
+# The E = 8 router at larger token counts.  Tensor-core router: 40 to 94 tiles, 1 to 3
+# k-ranges, a ragged last tile.  mma.sync router (MOE_ROUTER=fast): each CTA routes several
+# 16-token batches, the last one ragged (T=5000, D=4096: 34 tokens per CTA; T=9000, D=1024:
+# 61; T=12000, D=4096: 82).  Logits of every token, the whole routing, permutation and
+# statistics are compared with the oracle.
 @pytest.mark.parametrize("T,D", [(5000, 4096), (9000, 1024), (12000, 4096)])
-def test_fast_router_many_batches(T, D):
+def test_router_many_batches(T, D):
     w = scaled(W["mixtral"], T=T, D=D, F=256)
     inp = C.inputs_for(w)
     out, v = C.run_layer(w, inp)
@@ -266,6 +280,30 @@ def test_gathering_up_projection_matches_the_permuted_one(name):
     torch.cuda.synchronize()
     assert M.get_device_error() == 0
     assert torch.equal(h1[:n], h2[:n])
+
+
+# The router paths other than the default tensor-core router, each on the router cases it
+# can take (MOE_ROUTER is read once per process).
+ROUTER_MODES = {
+    "tc": "router_E8 or router_E6_ or groups_E8 or router_many_batches or single_expert",
+    "fast": "router_E8 or router_E6_ or groups_E8 or router_many_batches",
+    "gemm": "router_E32 or router_E64 or router_E256 or groups_E64 or groups_E128 or groups_E256",
+    "simt": "router_E8_T37 or router_E6_ or router_E64_v3 or router_E40 or groups_E64 or "
+            "router_E256_ec or groups_E256",
+}
+
+
+@pytest.mark.parametrize("mode", list(ROUTER_MODES))
+def test_other_router_paths_in_subprocess(mode):
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_ROUTER=mode)
+    sel = f"(small_layer_matches_oracle or router_many_batches) and ({ROUTER_MODES[mode]})"
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k", sel],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
 
 
 def test_layer_without_programmatic_dependent_launch_in_subprocess():

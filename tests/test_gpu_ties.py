@@ -8,8 +8,10 @@ ties back on purpose:
 * token choice: two router rows W_g[a] = W_g[b] (and, under sigmoid, equal selection biases)
   give bit-identical fp32 logits for every token, so wherever a and b sit among a token's k+1
   largest keys the rule decides their order or which of them is kept.  Every router path is
-  covered: the mma.sync router (bf16, E <= 8), the tcgen05 router product (bf16, E >= 32) and
-  the CUDA-core router (fp32).
+  covered: the mma.sync router (bf16, E <= 8, by default) and the tensor-core router fused
+  with the selection (bf16, the other cases by default, E <= 8 in a subprocess), the
+  grouped-GEMM router product (bf16, E % 32 == 0, in a subprocess) and the CUDA-core router
+  (fp32 always, bf16 in a subprocess).
 * sigmoid with a selection bias: two experts whose router rows are zero have sigma(0) = 1/2
   exactly, and equal biases then make their keys equal although the merge weights leave the
   bias out.
@@ -37,21 +39,22 @@ W = WORKLOADS
 
 # name: (workload, duplicated router rows (src, dst), zero router rows with one shared bias)
 TOKEN_CASES = {
-    # mma.sync router (bf16, E <= 8): softmax top-2 renormalised; two tied pairs
-    "fast_softmax_top2": (scaled(W["mixtral"], T=300, D=1024, F=256), [(2, 5), (6, 7)], ()),
-    # mma.sync router, top-1 with the raw softmax gate: a tie at the top must go to the lower id
-    "fast_top1_raw": (scaled(W["switch"], T=400, D=1024, E=8, F=256, zipf_s=0.0,
+    # E <= 8 (the mma.sync router under MOE_ROUTER=fast): softmax top-2 renormalised; two
+    # tied pairs
+    "e8_softmax_top2": (scaled(W["mixtral"], T=300, D=1024, F=256), [(2, 5), (6, 7)], ()),
+    # E = 8, top-1 with the raw softmax gate: a tie at the top must go to the lower id
+    "e8_top1_raw": (scaled(W["switch"], T=400, D=1024, E=8, F=256, zipf_s=0.0,
                              overflow="dropless"), [(1, 4)], ()),
-    # mma.sync router, sigmoid + bias: zero router rows 1 and 6 with equal biases
-    "fast_sigmoid_bias": (scaled(W["v3"], T=200, D=1024, E=8, k=3, F=256, F_shared=256),
+    # E = 8, sigmoid + bias: zero router rows 1 and 6 with equal biases
+    "e8_sigmoid_bias": (scaled(W["v3"], T=200, D=1024, E=8, k=3, F=256, F_shared=256),
                           [], (1, 6)),
-    # tcgen05 router product (E = 64, sigmoid + bias, top-6): pairs inside one 32-expert
-    # register slot and across two
-    "gemm_sigmoid_top6": (scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
+    # E = 64 (the grouped-GEMM router product under MOE_ROUTER=gemm), sigmoid + bias, top-6:
+    # pairs inside one 32-expert register slot and across two
+    "e64_sigmoid_top6": (scaled(W["v3"], T=97, D=1024, E=64, k=6, F=256, F_shared=256),
                           [(3, 4), (10, 41)], ()),
-    # tcgen05 router product (E = 32, softmax top-1, raw gate, capacity drop)
+    # E = 32, softmax top-1, raw gate, capacity drop
     # (Zipf offsets: the most popular expert is copied onto the last one, "popular")
-    "gemm_softmax_top1_drop": (scaled(W["switch"], T=300, D=256, E=32, F=256),
+    "e32_softmax_top1_drop": (scaled(W["switch"], T=300, D=256, E=32, F=256),
                                "popular", ()),
     # CUDA-core router (fp32): tiny layer, softmax top-2
     "f32_softmax_top2": (scaled(W["tiny"], T=64), [(0, 3)], ()),
@@ -125,7 +128,7 @@ def test_token_choice_ties_go_to_the_lower_expert(name):
 EC_CASES = {
     "ec_small": scaled(W["ec"], T=1000, D=256, E=16, F=256, c=125),
     # router product on the tcgen05 engine (E = 64)
-    "ec_gemm_router": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
+    "ec_e64": scaled(W["ec"], T=777, D=512, E=64, F=256, c=50),
     "ec_f32": scaled(W["ec"], dtype="f32", T=120, D=32, E=6, F=24, c=30, clusters=4, w_std=0.2,
                      wg_std=0.2),
 }
@@ -186,3 +189,28 @@ def test_expert_choice_ties_go_to_the_lower_token(name):
     assert t1 in picked[1] and u1 not in picked[1]
     np.testing.assert_array_equal(picked, ref["ids"])
     C.check_sampled_output(w, inp, out, v, list(range(w.T)))
+
+
+# The same ties through the router paths other than the default (MOE_ROUTER is read once per
+# process): the tensor-core router takes the E = 8 cases (the mma.sync router has them by
+# default; MOE_ROUTER=fast only confirms that), the grouped-GEMM product the E = 32 and E = 64
+# ones, the CUDA-core router every bf16 case.
+ROUTER_MODES = {
+    "tc": "e8_",
+    "fast": "e8_",
+    "gemm": "e32_ or e64_ or ec_e64",
+    "simt": "e8_ or e32_ or e64_ or ec_small or ec_e64",
+}
+
+
+@pytest.mark.parametrize("mode", list(ROUTER_MODES))
+def test_ties_through_other_router_paths_in_subprocess(mode):
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_ROUTER=mode)
+    sel = f"not subprocess and ({ROUTER_MODES[mode]})"
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k", sel],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
