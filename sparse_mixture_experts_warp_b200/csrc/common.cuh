@@ -119,13 +119,24 @@ cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S,
                               cudaStream_t s);
 cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N,
                               const int32_t* n_rows, void* y, cudaStream_t s);
+// y[r, n] = sum over *ks splits of P[s][r][n] (split stride *n_rows * N) for r < *n_rows; does
+// nothing when *ks == 1 (the product wrote y itself).  rows bounds *n_rows (grid sizing).
+cudaError_t launch_splitk_sum_adaptive(const float* p, const int* ks, int64_t rows, int N,
+                                       const int32_t* n_rows, void* y, cudaStream_t s);
 // With gather_src, A is the token tensor [src_rows, K] and row r of the grouped operand is its
 // row gather_src[r] / gather_div (4-row TMA gathers; the grouped copy is never written).
+// adapt_ks_max > 1 (EPI_NONE, groups along M, no gather or out2): an adaptive k-split.  When
+// the group table on the device gives fewer tiles than half the launch's CTAs, K is split
+// (at most adapt_ks_max ways, as many as fill the CTAs and fit adapt_cap floats) into fp32
+// partials [split][offsets[G]][N] at adapt_part instead of writing out; the split count goes
+// to *adapt_ks (1: out was written), for launch_splitk_sum_adaptive.
 cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int K,
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,
                                      void* out2 = nullptr, const int32_t* gather_src = nullptr,
-                                     int gather_div = 1, int64_t src_rows = 0);
+                                     int gather_div = 1, int64_t src_rows = 0,
+                                     float* adapt_part = nullptr, int64_t adapt_cap = 0,
+                                     int adapt_ks_max = 0, int* adapt_ks = nullptr);
 bool gemm_gather_ok();   // the selected tile shape can gather A rows
 
 // Router product on the same engine: one group of T rows, N = E, fp32 partial logits of

@@ -116,6 +116,14 @@ struct GemmParams {
   // with 4-row gathers straight into the ring: the grouped copy of the rows is never written
   const int32_t* gather_src;
   int gather_div;
+  // adaptive k-split (EPI_NONE, groups along M): when the launch's tiles fill fewer than half
+  // of its CTAs, K is split (at most adapt_ks_max ways, within adapt_cap floats of fp32
+  // partials [split][offsets[G]][N] at adapt_part) and the split count goes to *adapt_ks for
+  // the summing kernel; otherwise bf16 out as usual and *adapt_ks = 1
+  float* adapt_part;
+  int64_t adapt_cap;
+  int adapt_ks_max;
+  int* adapt_ks;
 };
 
 // One work item of the persistent schedule.
@@ -127,7 +135,7 @@ struct Tile {
 
 // Work item t (k-split slowest, then group, n-tile, m-tile); g caches the group search.
 template <int TBM, int KB>
-__device__ __forceinline__ Tile locate(int t, int total, int nkb, const GemmParams& p,
+__device__ __forceinline__ Tile locate(int t, int total, int nkb, int kchunk, const GemmParams& p,
                                        const int* grp_off, const int* tile_pre, int& g) {
   Tile r;
   r.split = t / total;
@@ -145,8 +153,8 @@ __device__ __forceinline__ Tile locate(int t, int total, int nkb, const GemmPara
     r.m = grp_off[g + 1] - grp_off[g];
     r.row0 = grp_off[g];
     r.kcol0 = 0;
-    r.kb0 = r.split * p.kchunk;
-    r.kb1 = min(nkb, r.kb0 + p.kchunk);
+    r.kb0 = r.split * kchunk;
+    r.kb1 = min(nkb, r.kb0 + kchunk);
   }
   const int mt = (r.m + TBM - 1) / TBM;
   const int local = tile - tile_pre[g];
@@ -406,8 +414,28 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   tc_fence_after();
   const uint32_t tmem_base = *tmem_holder;
   const int total = tile_pre[p.G];
-  const int total_all = total * p.ksplit;          // k-splits are the slowest tile index
   const int nkb = (p.K + KB - 1) / KB;
+  int ksplit = p.ksplit, kchunk = p.kchunk;
+  int64_t split_stride = p.split_stride;
+  if (EPI == EPI_NONE && p.adapt_ks_max > 1) {
+    // the same decision in every thread of every CTA (it depends on the group table only)
+    const int64_t live = grp_off[p.G];
+    int sk = (total > 0 && 2 * total <= (int)gridDim.x) ? (int)gridDim.x / total : 1;
+    sk = min(sk, min(p.adapt_ks_max, nkb));
+    while (sk > 1 && (int64_t)sk * live * p.N > p.adapt_cap) --sk;
+    if (sk > 1) {
+      kchunk = (nkb + sk - 1) / sk;
+      sk = (nkb + kchunk - 1) / kchunk;            // every k-range non-empty
+    } else {
+      sk = 1;
+      kchunk = nkb;
+    }
+    ksplit = sk;
+    split_stride = live * p.N;
+    if (blockIdx.x == 0 && threadIdx.x == 0) *p.adapt_ks = sk;
+  }
+  const bool adapt_f32 = EPI == EPI_NONE && ksplit > 1;
+  const int total_all = total * ksplit;            // k-splits are the slowest tile index
 
   if (warp == 0 && p.gather_src) {
     // ---------------- TMA producer, gathered rows of A ----------------
@@ -421,7 +449,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     bool ok = true;
     int g = 0;
     for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-      const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+      const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
       const int a_row = (int)tl.row0 + tl.m_idx * TBM;
       const int row_end = (int)tl.row0 + tl.m;
       const int b_row = tl.g * p.N + tl.n_idx * p.n_out_tile;
@@ -488,7 +516,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int g = 0;
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-        const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+        const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
         const int a_row = (int)tl.row0 + tl.m_idx * TBM;
         const int b_row = (p.kgroup ? 0 : tl.g * p.N) + tl.n_idx * p.n_out_tile;
         const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
@@ -555,7 +583,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       bool ok = true;
       int it = 0, g = 0;
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x, ++it) {
-        const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+        const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
         const int m = tl.m, m_idx = tl.m_idx;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
         const int kb0 = tl.kb0, kb1 = tl.kb1;      // kb0 == kb1: an empty group along K
@@ -613,7 +641,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     int g = 0, it = 0;
     uint32_t nstored = 0;                    // EPI_F32_TMA: staged blocks this warp has stored
     for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
-      const Tile tl = locate<TBM, KB>(t, total, nkb, p, grp_off, tile_pre, g);
+      const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
       const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
       const bool zero = tl.kb1 <= tl.kb0;    // no k-blocks (empty group along K): the sum is 0
       const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
@@ -698,7 +726,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       } else if (EPI == EPI_F32 || EPI == EPI_F32_TMA) {
         // fp32 partial of this k-split, rows of out32 + split * split_stride (+ the group's
         // output block when groups run along K)
-        float* orow32 = reinterpret_cast<float*>(p.out) + split * p.split_stride +
+        float* orow32 = reinterpret_cast<float*>(p.out) + split * split_stride +
                         (p.kgroup ? (int64_t)tl.g * p.out_gstride : 0) + orow * p.ldo +
                         (int64_t)n_idx * p.n_out_tile;
         // TMA stores need the warp's 32 rows in its 32 lanes: a tile of at most 64 live rows
@@ -750,6 +778,27 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               ++nstored;
             }
           } else if (valid && col < p.N) {
+            uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+          }
+        }
+      } else if (EPI == EPI_NONE && adapt_f32) {
+        // adaptive k-split: this split's fp32 partial, rows of adapt_part + split * stride
+        float* orow32 = p.adapt_part + split * split_stride + orow * p.N +
+                        (int64_t)n_idx * p.n_out_tile;
+#pragma unroll 1
+        for (int c = 0; c < MMA_N; c += 32) {
+          uint32_t v[32];
+          tmem_ld32(taddr + c, v);
+          tmem_wait_ld();
+          if (c == MMA_N - 32) {             // last TMEM read of the tile: release the buffer
+            tc_fence_before();
+            mbar_arrive(&tempty[acc]);
+          }
+          const int col = n_idx * p.n_out_tile + c;
+          if (valid && col < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -1339,10 +1388,14 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
                                      const void* B0, const void* B1, int n_groups, int N,
                                      const int32_t* offsets, void* out, cudaStream_t s,
                                      void* out2, const int32_t* gather_src, int gather_div,
-                                     int64_t src_rows) {
+                                     int64_t src_rows, float* adapt_part, int64_t adapt_cap,
+                                     int adapt_ks_max, int* adapt_ks) {
   if (a_rows <= 0 || n_groups <= 0) return cudaSuccess;
   if (gather_src && (!offsets || !gemm_gather_ok() || epi == EPI_NONE_BMN || gather_div < 1 ||
                      src_rows <= 0))
+    return cudaErrorInvalidValue;
+  const bool adapt = adapt_ks_max > 1;
+  if (adapt && (epi != EPI_NONE || !offsets || out2 || gather_src || !adapt_part || !adapt_ks))
     return cudaErrorInvalidValue;
   alignas(64) CUtensorMap ta, tb0, tb1;
   const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
@@ -1370,7 +1423,12 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.split_stride = 0;
   p.gather_src = gather_src;
   p.gather_div = gather_div;
-  const GemmTile tile = tile_for(a_rows, n_groups, offsets != nullptr);
+  p.adapt_part = adapt_part;
+  p.adapt_cap = adapt_cap;
+  p.adapt_ks_max = adapt ? adapt_ks_max : 0;
+  p.adapt_ks = adapt_ks;
+  GemmTile tile = tile_for(a_rows, n_groups, offsets != nullptr);
+  if (adapt && tile == TILE_PAIR) tile = TILE_256;     // the pair kernel has no adaptive split
   const int halves = tile == TILE_128 ? 1 : 2;
   const int kb = tile == TILE_256_K32 ? 32 : 64;
   if (gather_src) {

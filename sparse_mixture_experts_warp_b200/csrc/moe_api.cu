@@ -132,6 +132,52 @@ bool decode_splitk_enabled() {
   return v;
 }
 
+// Adaptive k-split of the down projection.  Under a capacity limit the executed rows can be
+// far fewer than the host's bound (a few popular experts, each at its capacity: the Switch
+// layer runs 413 of 8192 possible rows on 9 of 128 experts), and the down projection's tiles
+// then leave most SMs idle.  The grouped GEMM reads the group table on the device and, when
+// its tiles fill fewer than half of the CTAs, splits K into fp32 partials that
+// launch_splitk_sum_adaptive sums.  Used where the smallest possible row count gives fewer
+// tiles than a B200 has SMs (148), the only case in which a launch can be under-filled;
+// MOE_ADAPTIVE_SPLIT=0 turns it off (comparison measurements).
+constexpr int kSmBound = 148;
+constexpr size_t kAdaptCapBytes = (size_t)24 << 20;   // partials of any split that fills the SMs
+
+bool adaptive_split_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_ADAPTIVE_SPLIT");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
+// Fewest rows the routed experts can execute: every token on the same k experts, each kept up
+// to its capacity; expert choice always E * c.
+int64_t min_rows_of(const moe_desc_t* d) {
+  if (d->select == MOE_EXPERT_CHOICE) return (int64_t)d->E * d->c;
+  const int64_t A = (int64_t)d->T * d->k;
+  if (d->overflow != MOE_CAPACITY_DROP) return A;
+  const int64_t cap = capacity_of(d);
+  const int64_t m = (int64_t)d->k * (d->T < cap ? d->T : cap);
+  return m < A ? m : A;
+}
+
+bool adaptive_down(const moe_desc_t* d) {
+  if (d->dtype != MOE_BF16 || !decode_splitk_enabled() || !adaptive_split_enabled()) return false;
+  if (rows_of(d) <= kSplitDownRows) return false;     // the small-batch schedule splits already
+  const int64_t min_tiles = ((min_rows_of(d) + 255) / 256) * (((int64_t)d->D + 255) / 256);
+  return min_tiles < kSmBound;
+}
+
+// fp32 partials (at most kAdaptCapBytes) and the split count after them
+size_t adaptive_part_bytes(const moe_desc_t* d) {
+  const size_t full = (size_t)kMaxSplits * rows_of(d) * d->D * sizeof(float);
+  return up(full < kAdaptCapBytes ? full : kAdaptCapBytes);
+}
+size_t adaptive_bytes(const moe_desc_t* d) {
+  return adaptive_down(d) ? adaptive_part_bytes(d) + kAlign : 0;
+}
+
 size_t splitk_up_bytes(const moe_desc_t* d, int64_t A) {     // one partial set
   return up((size_t)kMaxSplits * A * d->F * sizeof(float));
 }
@@ -144,7 +190,8 @@ size_t splitk_scratch(const moe_desc_t* d) {
     const size_t u = (d->act == MOE_ACT_SWIGLU ? 2 : 1) * splitk_up_bytes(d, A);
     if (u > b) b = u;
   }
-  return b;
+  const size_t ad = adaptive_bytes(d);
+  return ad > b ? ad : b;
 }
 
 size_t scratch_bytes(const moe_desc_t* d) {
@@ -519,8 +566,21 @@ moe_status_t moe_expert_down_ws(const moe_desc_t* d, int32_t G, int32_t F, const
   float* part = S > 1 ? splitk_space(scratch, scratch_bytes,
                                      (size_t)S * a_rows * d->D * sizeof(float))
                       : nullptr;
-  if (!part) return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (!part && adaptive_down(d) && W_down && y && is_aligned16(W_down) && is_aligned16(y) &&
+      d->D % 4 == 0) {
+    float* ap = splitk_space(scratch, scratch_bytes, adaptive_part_bytes(d) + kAlign);
+    if (ap) {
+      const size_t pb = adaptive_part_bytes(d);
+      int* ks = reinterpret_cast<int*>(reinterpret_cast<uint8_t*>(ap) + pb);
+      cudaError_t e = launch_grouped_gemm_bf16(EPI_NONE, h, a_rows, F, W_down, nullptr, G, d->D,
+                                               offsets, y, s, nullptr, nullptr, 1, 0, ap,
+                                               (int64_t)(pb / sizeof(float)), kMaxSplits, ks);
+      if (e == cudaSuccess) e = launch_splitk_sum_adaptive(ap, ks, a_rows, d->D, offsets + G, y, s);
+      return cuda_status(e);
+    }
+  }
+  if (!part) return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
   cudaError_t e = launch_grouped_gemm_f32_splitk(h, a_rows, F, W_down, G, d->D, offsets, S, part,
                                                  s);
   if (e == cudaSuccess) e = launch_splitk_sum(part, S, a_rows, d->D, offsets + G, y, s);

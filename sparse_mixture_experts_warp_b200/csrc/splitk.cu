@@ -96,6 +96,28 @@ splitk_sum_kernel(const float* __restrict__ p, int S, int64_t rows, int N,
   }
 }
 
+// The adaptive split's sum: the split count and the live rows come from the device.
+__global__ void __launch_bounds__(kThreads)
+splitk_sum_adaptive_kernel(const float* __restrict__ p, const int* __restrict__ ks, int64_t rows,
+                           int N, const int32_t* __restrict__ n_rows,
+                           __nv_bfloat16* __restrict__ y) {
+  pdl_trigger();
+  pdl_wait();
+  const int S = __ldg(ks);
+  if (S <= 1) return;                       // the product wrote y
+  const int64_t live = min((int64_t)__ldg(n_rows), rows);
+  const int q = N / 4;
+  const int64_t items = live * q;
+  const int64_t stride = live * (int64_t)N;
+  for (int64_t i = blockIdx.x * (int64_t)kThreads + threadIdx.x; i < items;
+       i += (int64_t)gridDim.x * kThreads) {
+    const int64_t r = i / q;
+    const int64_t off = r * N + (i - r * q) * 4;
+    const float4 a = sum_splits(p, S, stride, off);
+    *reinterpret_cast<uint2*>(y + off) = make_uint2(pack2(a.x, a.y), pack2(a.z, a.w));
+  }
+}
+
 // enough blocks for every item of the allocated rows, at most 4 per SM (grid-stride beyond)
 int grid_for(int64_t rows, int n) {
   const int64_t items = rows * (n / 4);
@@ -131,6 +153,16 @@ cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N, const 
   if (N % 4 || S < 1) return cudaErrorInvalidValue;
   (void)launch_pdl(splitk_sum_kernel, dim3(grid_for(rows, N)), dim3(kThreads), 0, s, 
       p, S, rows, N, n_rows, static_cast<__nv_bfloat16*>(y));
+  return cudaGetLastError();
+}
+
+cudaError_t launch_splitk_sum_adaptive(const float* p, const int* ks, int64_t rows, int N,
+                                       const int32_t* n_rows, void* y, cudaStream_t s) {
+  if (rows <= 0 || N <= 0) return cudaSuccess;
+  if (N % 4) return cudaErrorInvalidValue;
+  const int grid = grid_for(rows, N);
+  (void)launch_pdl(splitk_sum_adaptive_kernel, dim3(grid), dim3(kThreads), 0, s, p, ks, rows, N,
+                   n_rows, static_cast<__nv_bfloat16*>(y));
   return cudaGetLastError();
 }
 

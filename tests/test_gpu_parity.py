@@ -306,6 +306,23 @@ def test_other_router_paths_in_subprocess(mode):
     assert " passed" in r.stdout, r.stdout[-3000:]
 
 
+def test_switch_layer_without_adaptive_split_in_subprocess():
+    """MOE_ADAPTIVE_SPLIT=0: the down projection of capacity-limited layers writes bf16 directly
+    whatever its tile count (by default the grouped GEMM splits K on the device when the
+    executed rows leave most SMs idle, as in the Switch layer); the Switch cases pass both
+    ways."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_ADAPTIVE_SPLIT="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "(small_layer_matches_oracle or full_size_workload or capacity_drops) "
+                        "and (switch or f32_relu_drop or router_E40)"],
+                       env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
+
+
 def test_layer_without_programmatic_dependent_launch_in_subprocess():
     """MOE_PDL=0 launches every kernel without programmatic stream serialization (each waits
     for the previous one to finish before it is scheduled); the small-case parity tests pass
