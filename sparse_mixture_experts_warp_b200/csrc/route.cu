@@ -249,7 +249,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* s_warp, int* tot
 // block scan of its (above-threshold, equal-to-threshold) counts gives every thread its output
 // position and the number of equal keys before it, so the output holds all keys above the
 // threshold and the first `need` equal ones, in ascending token order.  Shared memory: the
-// keys (T * 4 bytes, when staged) and 32 KB of per-warp histograms.
+// keys (T * 4 bytes, when staged) and 32 KB of per-warp histograms.  The digit of a pass comes
+// from a scan of the 256 bin totals by 256 threads.
 template <bool STAGED>
 __global__ void __launch_bounds__(1024)
 ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
@@ -323,14 +324,27 @@ ec_select_kernel(const float* probsT, int T, int c, int32_t* picked) {
     __syncthreads();
     if (threadIdx.x < 256) hist[0][threadIdx.x] = tot;
     __syncthreads();
-    if (threadIdx.x == 0) {
-      int cum = 0, d = (int)dmask;
-      for (; d > 0; --d) {
-        if (cum + hist[0][d] >= need) break;
-        cum += hist[0][d];
+    // the digit: the largest d whose keys, with those of the digits above it, number at least
+    // `need`.  Thread j < 256 takes bin 255 - j, so an inclusive scan over j counts the keys at
+    // and above that digit; the first j to reach `need` names it.
+    if (threadIdx.x < 256) {
+      const int b = 255 - (int)threadIdx.x;
+      const int v = b <= (int)dmask ? hist[0][b] : 0;
+      int inc = v;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += n;
       }
-      s_digit = d;
-      s_need = need - cum;
+      if (lane == 31) s_warp[warp] = inc;
+      asm volatile("bar.sync 1, 256;" ::: "memory");      // the 8 warps of threads < 256
+      int before = 0;
+      for (int w = 0; w < warp; ++w) before += s_warp[w];
+      inc += before;
+      if (inc >= need && inc - v < need) {
+        s_digit = b;
+        s_need = need - (inc - v);
+      }
     }
     __syncthreads();
     prefix |= (uint32_t)s_digit << shift;
