@@ -4,9 +4,12 @@ exchange plan, the block reorder kernel, the local grouped GEMMs on Eg = E / G e
 reverse exchange and the combine all run on the device.
 
 Each rank's output is compared with the single-device layer on the same tokens and full expert
-set (moe_layer_forward): every row meets the same kernels in the same k order, so they must
-agree bit for bit; and with the oracle (routing from the GPU's fp32 logits, every token, the
-bf16 tolerance)."""
+set (moe_layer_forward): in a dropless layer every row meets the same kernels in the same k
+order, so they must agree bit for bit.  Under a capacity limit the single-device layer may
+split its down projection along K on the device (when the kept rows leave SMs idle) while the
+ranks, each with fewer experts, decide for themselves, so y's fp32 summation order can differ:
+there the outputs must agree within bf16 rounding.  Every rank is also compared with the oracle
+(routing from the GPU's fp32 logits, every token, the bf16 tolerance)."""
 
 import numpy as np
 import pytest
@@ -52,7 +55,13 @@ def test_expert_parallel_layer_matches_single_device(name):
         inp = per_rank[r]
         ref = C.run_layer(w, type(inp)(inp.x, full.Wg, full.bias, full.W_gate, full.W_up,
                                        full.W_down))[0]
-        assert torch.equal(ranks[r].out, ref), f"rank {r}: differs from the single-device layer"
+        if w.overflow == "drop":
+            diff = (ranks[r].out.float() - ref.float()).abs().max().item()
+            assert diff <= 1e-2 * ref.float().abs().max().item(), \
+                f"rank {r}: differs from the single-device layer by {diff}"
+        else:
+            assert torch.equal(ranks[r].out, ref), \
+                f"rank {r}: differs from the single-device layer"
         v = ranks[r].views
         C.check_routing(w, type(inp)(inp.x, full.Wg, full.bias, full.W_gate, full.W_up,
                                      full.W_down), v)
