@@ -111,12 +111,21 @@ enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI
 cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
                                            int G, int N, const int32_t* offsets, int ksplit,
                                            float* out, cudaStream_t s);
+// The same for two products that share A (the gate and up products of the decode schedule):
+// out[split][row][ldo] with ldo = 2 * ceil(N / 256) * 256, B0's product in columns
+// [0, N) and B1's from column ldo / 2.
+cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K, const void* B0,
+                                            const void* B1, int G, int N,
+                                            const int32_t* offsets, int ksplit, float* out,
+                                            cudaStream_t s);
 int gemm_sm_count();
 int splitk_count(int K, int ksplit);   // non-empty splits of K (64-element k-blocks)
 // splitk.cu: the sums of k-split partials of the small-batch schedule (rows below *n_rows)
+// ld: row pitch of the partials (F when gate and up are separate arrays; the two-product
+// layout's ldo otherwise).
 cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S,
                               int64_t rows, int F, const int32_t* n_rows, void* h,
-                              cudaStream_t s);
+                              cudaStream_t s, int64_t ld = 0);
 cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N,
                               const int32_t* n_rows, void* y, cudaStream_t s);
 // y[r, n] = sum over *ks splits of P[s][r][n] (split stride *n_rows * N) for r < *n_rows; does

@@ -124,6 +124,9 @@ struct GemmParams {
   int64_t adapt_cap;
   int adapt_ks_max;
   int* adapt_ks;
+  // EPI_F32 with two B tensors: n-tiles from b1_nt on read tmB1 (rows of n-tile n - b1_nt), so
+  // one launch computes both the gate and the up product (0: one B tensor)
+  int b1_nt;
 };
 
 // One work item of the persistent schedule.
@@ -518,7 +521,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
         const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
         const int a_row = (int)tl.row0 + tl.m_idx * TBM;
-        const int b_row = (p.kgroup ? 0 : tl.g * p.N) + tl.n_idx * p.n_out_tile;
+        const bool b1 = EPI == EPI_F32 && p.b1_nt > 0 && tl.n_idx >= p.b1_nt;
+        const int b_row = (p.kgroup ? 0 : tl.g * p.N) +
+                          (tl.n_idx - (b1 ? p.b1_nt : 0)) * p.n_out_tile;
         const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
         const int kb0 = tl.kb0, kb1 = tl.kb1;
         for (int kb = kb0; kb < kb1; ++kb) {
@@ -556,8 +561,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
             tma_load_2d(b_dst + TB_BYTES / 2, &tmB1, &full[stage], kx, b_row);
           } else {
-            tma_load_2d(b_dst, &tmB0, &full[stage], kx, b_row);
-            tma_load_2d(b_dst + TB_BYTES / 2, &tmB0, &full[stage], kx, b_row + 128);
+            const CUtensorMap* mb = b1 ? &tmB1 : &tmB0;
+            tma_load_2d(b_dst, mb, &full[stage], kx, b_row);
+            tma_load_2d(b_dst + TB_BYTES / 2, mb, &full[stage], kx, b_row + 128);
           }
           issued |= 1u << stage;
           issued_par = (issued_par & ~(1u << stage)) | (phase << stage);
@@ -747,6 +753,11 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             mbar_arrive(&tempty[acc]);
           }
           const int col = n_idx * p.n_out_tile + c;
+          // column within its product (two B tensors: the second product's block starts at
+          // n-tile b1_nt)
+          const int pcol = (EPI == EPI_F32 && p.b1_nt > 0 && n_idx >= p.b1_nt)
+                               ? col - p.b1_nt * p.n_out_tile
+                               : col;
           if (staged) {
             if (col >= p.N) continue;        // warp-uniform: the chunk lies past the last column
             // two 16-column halves, each staged in buffer (nstored & 1) of this warp (2 KB: 32
@@ -777,7 +788,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               }
               ++nstored;
             }
-          } else if (valid && col < p.N) {
+          } else if (valid && pcol < p.N) {
             uint4* dst = reinterpret_cast<uint4*>(orow32 + c);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -1619,6 +1630,38 @@ cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K,
   const int64_t tiles = ((a_rows + BM - 1) / BM + G) * (int64_t)p.nt * p.ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, G), s);
+}
+
+cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K, const void* B0,
+                                            const void* B1, int G, int N,
+                                            const int32_t* offsets, int ksplit, float* out,
+                                            cudaStream_t s) {
+  if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
+  alignas(64) CUtensorMap ta, tb0, tb1;
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb0, B0, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  if (!make_map(&tb1, B1, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  const int half = (N + 255) / 256;               // n-tiles of one product
+  GemmParams p{};
+  p.offsets = offsets;
+  p.out = reinterpret_cast<__nv_bfloat16*>(out);
+  p.err = device_error_word();
+  p.rows = a_rows;
+  p.ldo = (int64_t)2 * half * 256;                // [product 0 | product 1], 256-column tiles
+  p.G = G;
+  p.N = N;
+  p.K = K;
+  p.n_out_tile = 256;
+  p.nt = 2 * half;
+  p.b1_nt = half;
+  p.fault = 0;
+  const int nkb = (K + 63) / 64;
+  p.kchunk = (nkb + ksplit - 1) / ksplit;
+  p.ksplit = splitk_count(K, ksplit);
+  p.split_stride = a_rows * p.ldo;
+  const int64_t tiles = ((a_rows + BM - 1) / BM + G) * (int64_t)p.nt * p.ksplit;
+  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  return launch_epi<EPI_F32, 1, 64, 4>(ta, tb0, tb1, p, grid, gemm_smem(1, 64, 4, G), s);
 }
 
 int gemm_sm_count() { return sm_count(); }

@@ -178,8 +178,8 @@ size_t adaptive_bytes(const moe_desc_t* d) {
   return adaptive_down(d) ? adaptive_part_bytes(d) + kAlign : 0;
 }
 
-size_t splitk_up_bytes(const moe_desc_t* d, int64_t A) {     // one partial set
-  return up((size_t)kMaxSplits * A * d->F * sizeof(float));
+size_t splitk_up_bytes(const moe_desc_t* d, int64_t A) {     // one product's partials
+  return up((size_t)kMaxSplits * A * ((int64_t)(d->F + 255) / 256 * 256) * sizeof(float));
 }
 size_t splitk_scratch(const moe_desc_t* d) {
   if (d->dtype != MOE_BF16) return 0;
@@ -527,27 +527,31 @@ moe_status_t moe_expert_up_ws(const moe_desc_t* d, int32_t G, int32_t F, const v
       (!glu || (W_gate && is_aligned16(W_gate)))) {
     // fused: SwiGLU tiles hold 128 features (gate and up side by side), others 256 columns;
     // split: gate and up are separate products of 256-column tiles
+    // split: SwiGLU's gate and up products in one launch of 256-column tiles (n-tiles of W_up
+    // after those of W_gate), others one product
     const int sms = gemm_sm_count();
     const int64_t active = a_rows < G ? a_rows : G;
     const int64_t fused = active * ((F + (glu ? 127 : 255)) / (glu ? 128 : 256));
-    const int64_t units = active * ((F + 255) / 256);
+    const int64_t units = active * ((F + 255) / 256) * (glu ? 2 : 1);
     const double fill_fused = sm_fill(fused, sms);
     const int c = choose_splits(units, d->D, sms);
     if (c > 1 && fill_fused < 0.8 && sm_fill(units * c, sms) > fill_fused + 0.05) S = c;
   }
-  const size_t one = (size_t)S * a_rows * F * sizeof(float);
-  const size_t step = up(one);
-  float* part = S > 1 ? splitk_space(scratch, scratch_bytes, (glu ? step : 0) + one) : nullptr;
+  // partial rows: [gate | up] blocks of ceil(F / 256) * 256 columns each (SwiGLU), F otherwise
+  const int64_t fpad = (int64_t)(F + 255) / 256 * 256;
+  const int64_t ld = glu ? 2 * fpad : F;
+  float* part = S > 1 ? splitk_space(scratch, scratch_bytes, (size_t)S * a_rows * ld * sizeof(float))
+                      : nullptr;
   if (!part)
     return moe_expert_up(d, G, F, a, a_rows, offsets, W_gate, W_up, h, stream);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  float* pu = glu ? part + step / sizeof(float) : part;
-  cudaError_t e = cudaSuccess;
-  if (glu) e = launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_gate, G, F, offsets, S, part, s);
+  cudaError_t e = glu ? launch_grouped_gemm_f32_splitk2(a, a_rows, d->D, W_gate, W_up, G, F,
+                                                         offsets, S, part, s)
+                      : launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_up, G, F, offsets, S,
+                                                       part, s);
   if (e == cudaSuccess)
-    e = launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_up, G, F, offsets, S, pu, s);
-  if (e == cudaSuccess)
-    e = launch_splitk_act(d->act, part, pu, S, a_rows, F, offsets + G, h, s);
+    e = launch_splitk_act(d->act, part, glu ? part + fpad : part, S, a_rows, F, offsets + G, h, s,
+                          ld);
   return cuda_status(e);
 }
 

@@ -10,7 +10,8 @@
 // kernels add the S partials in a fixed order (deterministic), apply the activation and round
 // once to bf16:
 //   launch_splitk_act:  h[r, f] = act(sum_s Pg[s][r][f], sum_s Pu[s][r][f]) (SwiGLU: SiLU(g) * u;
-//                       ReLU / GELU: act(u), Pg unused);
+//                       ReLU / GELU: act(u), Pg unused); the partials' rows are ld apart (gate
+//                       and up in one buffer: Pu = Pg + ld / 2);
 //   launch_splitk_sum:  y[r, n] = sum_s P[s][r][n].
 // Rows at or past *n_rows (the executed-row count, offsets[G] on the device) are left alone:
 // nothing reads them.  Both are HBM-bound elementwise passes over S * rows * N fp32 values,
@@ -51,22 +52,24 @@ __device__ __forceinline__ float gelu(float a) {
 template <int ACT>
 __global__ void __launch_bounds__(kThreads)
 splitk_act_kernel(const float* __restrict__ pg, const float* __restrict__ pu, int S,
-                  int64_t rows, int F, const int32_t* __restrict__ n_rows,
+                  int64_t rows, int F, int64_t ld, const int32_t* __restrict__ n_rows,
                   __nv_bfloat16* __restrict__ h) {
   pdl_trigger();
   pdl_wait();
   const int64_t live = min((int64_t)__ldg(n_rows), rows);
   const int q = F / 4;                       // four columns per item
   const int64_t items = live * q;
-  const int64_t stride = rows * (int64_t)F;
+  const int64_t stride = rows * ld;
   for (int64_t i = blockIdx.x * (int64_t)kThreads + threadIdx.x; i < items;
        i += (int64_t)gridDim.x * kThreads) {
     const int64_t r = i / q;
-    const int64_t off = r * F + (i - r * q) * 4;
-    const float4 u = sum_splits(pu, S, stride, off);
+    const int64_t cidx = (i - r * q) * 4;
+    const int64_t off = r * F + cidx;          // in h
+    const int64_t poff = r * ld + cidx;        // in the partials
+    const float4 u = sum_splits(pu, S, stride, poff);
     float4 o;
     if (ACT == MOE_ACT_SWIGLU) {
-      const float4 g = sum_splits(pg, S, stride, off);
+      const float4 g = sum_splits(pg, S, stride, poff);
       o = make_float4(silu_mul(g.x, u.x), silu_mul(g.y, u.y), silu_mul(g.z, u.z),
                       silu_mul(g.w, u.w));
     } else if (ACT == MOE_ACT_GELU) {
@@ -130,20 +133,21 @@ int grid_for(int64_t rows, int n) {
 }  // namespace
 
 cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S, int64_t rows,
-                              int F, const int32_t* n_rows, void* h, cudaStream_t s) {
+                              int F, const int32_t* n_rows, void* h, cudaStream_t s, int64_t ld) {
+  if (ld <= 0) ld = F;
   if (rows <= 0 || F <= 0) return cudaSuccess;
   if (F % 4 || S < 1) return cudaErrorInvalidValue;
   const int grid = grid_for(rows, F);
   __nv_bfloat16* o = static_cast<__nv_bfloat16*>(h);
   if (act == MOE_ACT_SWIGLU)
     (void)launch_pdl(splitk_act_kernel<MOE_ACT_SWIGLU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
-                                                                        n_rows, o);
+                                                                        ld, n_rows, o);
   else if (act == MOE_ACT_GELU)
     (void)launch_pdl(splitk_act_kernel<MOE_ACT_GELU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
-                                                                      n_rows, o);
+                                                                      ld, n_rows, o);
   else
     (void)launch_pdl(splitk_act_kernel<MOE_ACT_RELU>, dim3(grid), dim3(kThreads), 0, s, pg, pu, S, rows, F,
-                                                                      n_rows, o);
+                                                                      ld, n_rows, o);
   return cudaGetLastError();
 }
 
