@@ -19,7 +19,8 @@ slowest rank's time (weak scaling).
 same workload: each step routes the whole batch and evaluates a sample of its tokens.
 
 After the forward, the same graph is replayed for about a second ("sustained": the clock the
-1 kW power cap settles at), and a training step (moe_layer_forward_train + moe_layer_backward)
+1 kW power cap settles at, the GPU's joules per step from the NVML energy counter and the
+expert GEMMs' TFLOP per joule), and a training step (moe_layer_forward_train + moe_layer_backward)
 is timed, reported under "backward" (`--no-backward` skips it).  At one GPU the other layer
 shapes the pages name -- Switch top-1, DeepSeek-V3, expert choice at the DeepSeekMoE-16B shape
 and a one-token Mixtral decode step -- are then timed for a few graph-replayed steps each and
@@ -111,6 +112,8 @@ class ClockSampler:
         self._stop = threading.Event()
         self._thread = None
         self.error = None
+        self._e0 = self._e1 = None     # NVML total energy (mJ) at start and end
+        self._t0 = self._t1 = None
 
     def __enter__(self):
         try:
@@ -122,6 +125,11 @@ class ClockSampler:
         except Exception as e:  # pragma: no cover - no NVML
             self.error = str(e)
             return self
+        try:
+            self._e0 = self._nvml.nvmlDeviceGetTotalEnergyConsumption(self._h)
+            self._t0 = time.time()
+        except Exception:  # pragma: no cover - no energy counter
+            self._e0 = None
         self._thread = threading.Thread(target=self._run, daemon=True)
         self._thread.start()
         return self
@@ -145,11 +153,26 @@ class ClockSampler:
         self._stop.set()
         if self._thread:
             self._thread.join()
+        if self._e0 is not None:
+            try:
+                self._e1 = self._nvml.nvmlDeviceGetTotalEnergyConsumption(self._h)
+                self._t1 = time.time()
+            except Exception:  # pragma: no cover
+                self._e1 = None
+
+    def energy_j(self):
+        """Joules the GPU drew while the sampler ran (NVML energy counter), or None."""
+        if self._e0 is None or self._e1 is None:
+            return None
+        return (self._e1 - self._e0) / 1000.0
 
     def summary(self):
         med = statistics.median(self.samples) if self.samples else None
         out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                "samples": len(self.samples)}
+        e = self.energy_j()
+        if e is not None and self._t1 and self._t1 > self._t0:
+            out["avg_w"] = round(e / (self._t1 - self._t0), 1)
         if self.error:
             out["error"] = self.error
         return out
@@ -632,6 +655,10 @@ def run_cuda(args, rank, world, local):
         sustained = {"steps": n_sus, "ms_per_step": round(sus_ms / n_sus, 4),
                      "value": round(job_throughput(w.T, world, n_sus, sus_ms), 1),
                      "clocks": sus_clk.summary()}
+        e = sus_clk.energy_j()
+        if e is not None:
+            # the GPU's energy over the replay (this rank's GPU), per step
+            sustained["joules_per_step"] = round(e / n_sus, 4)
 
     # e2e: the public call with host buffers; every step copies its own tokens in from pinned
     # host memory and its output back, inside the timed region.  Copies run on their own
@@ -655,6 +682,8 @@ def run_cuda(args, rank, world, local):
     stages, work, gemm_flops, layer_roof_s = stage_rooflines(w, per_stage, rows_exec, active,
                                                              peaks, tc_peak, step.gather)
     up_flops = work["expert_up"][1]
+    if sustained and sustained.get("joules_per_step"):
+        sustained["gemm_tflop_per_joule"] = round(gemm_flops / 1e12 / sustained["joules_per_step"], 3)
     achieved = up_flops / (per_stage["expert_up"] * 1e-3) / 1e12
     gemm_tflops = gemm_flops / ((per_stage["expert_up"] + per_stage["expert_down"]) * 1e-3) / 1e12
     roofline = {
