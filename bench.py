@@ -171,7 +171,8 @@ class ClockSampler:
         out = {"sm_mhz": med, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
                "samples": len(self.samples)}
         e = self.energy_j()
-        if e is not None and self._t1 and self._t1 > self._t0:
+        # the counter advances in steps: only a run of half a second or more gives a mean power
+        if e is not None and e > 0 and self._t1 and self._t1 - self._t0 >= 0.5:
             out["avg_w"] = round(e / (self._t1 - self._t0), 1)
         if self.error:
             out["error"] = self.error
@@ -656,7 +657,7 @@ def run_cuda(args, rank, world, local):
                      "value": round(job_throughput(w.T, world, n_sus, sus_ms), 1),
                      "clocks": sus_clk.summary()}
         e = sus_clk.energy_j()
-        if e is not None:
+        if e is not None and e > 0:
             # the GPU's energy over the replay (this rank's GPU), per step
             sustained["joules_per_step"] = round(e / n_sus, 4)
 
