@@ -18,7 +18,10 @@
 //   4. gather: one warp per token reads x[t] once (16-byte loads) and writes it to each of its
 //              kept rows.
 // Expert choice: row e*c + i is the i-th picked token of expert e (already in token order).
+#include <stdlib.h>
+
 #include "common.cuh"
+#include "tc_ops.cuh"
 
 namespace moe {
 namespace {
@@ -240,6 +243,122 @@ perm_index_fused_kernel(const int32_t* ids, int A, int E, int cap, int32_t* coun
   }
 }
 
+
+// Mid-sized problems (kClusterMinItems < A <= kClusterMaxItems, E <= 1024): the index kernel
+// above spread over one cluster of up to 8 CTAs.  CTA r stages and ranks the contiguous
+// assignments [r*C, (r+1)*C) (C a multiple of 1024: 32 warps x whole 32-assignment batches).
+// After its per-warp counts, every CTA reads the per-expert totals of all CTAs of the cluster
+// through distributed shared memory: the lower ranks' totals are its base, their sum the
+// expert's count.  The capacity clamp and the exclusive scan over experts then give every CTA
+// the same offsets (CTA 0 writes counts and offsets).  Ranks are global (base + the warp
+// prefix + the rank inside the batch), so rows follow the (token, slot) order across CTAs
+// exactly as in the one-CTA kernel.
+constexpr int kClusterMaxCTAs = 8;
+constexpr int kClusterMinItems = 1 << 11;
+constexpr int kClusterMaxItems = kClusterMaxCTAs * (1 << 13);
+
+__global__ void __launch_bounds__(1024)
+perm_index_cluster_kernel(const int32_t* ids, int A, int E, int cap, int chunk, int32_t* counts,
+                          int32_t* offsets, int32_t* row_src, int32_t* inv) {
+  pdl_trigger();
+  pdl_wait();
+  extern __shared__ int s_mem[];
+  int* s_cnt = s_mem;                    // [32][E]
+  int* s_tot = s_mem + 32 * E;           // [E] this CTA's totals, read by the whole cluster
+  int* s_off = s_tot + E;                // [E]
+  int* s_base = s_off + E;               // [E]
+  int* s_ids = s_base + E;               // [chunk]
+  __shared__ int s_warp[32];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = (int)cluster_cta_rank(), ncta = (int)gridDim.x;   // one cluster
+  const int a0 = rank * chunk;
+  const int n = max(0, min(A, a0 + chunk) - a0);
+  for (int i = threadIdx.x; i < 32 * E; i += blockDim.x) s_cnt[i] = 0;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s_ids[i] = ids[a0 + i];
+  __syncthreads();
+  const int per = chunk / 32;            // multiple of 32
+  const int lo = warp * per, hi = min(n, lo + per);
+  int* my = s_cnt + warp * E;
+  const unsigned lt = (1u << lane) - 1u;
+  for (int base = lo; base < hi; base += 32) {
+    const int a = base + lane;
+    const int e = (a < hi) ? s_ids[a] : -1;
+    const bool ok = (e >= 0 && e < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? e : -1);
+    if (ok && (peers & lt) == 0) my[e] += __popc(peers);
+    __syncwarp();
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  if (e < E) {
+    int run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int v = s_cnt[w * E + e];
+      s_cnt[w * E + e] = run;
+      run += v;
+    }
+    s_tot[e] = run;
+  }
+  cluster_sync_all();                    // every CTA's totals are in its shared memory
+  int kept = 0;
+  if (e < E) {
+    const uint32_t at = smem_u32(s_tot + e);
+    int base = 0, total = 0;
+    for (int r = 0; r < ncta; ++r) {
+      const int v = ld_cluster_s32(cluster_map(at, (uint32_t)r));
+      if (r < rank) base += v;
+      total += v;
+    }
+    s_base[e] = base;
+    if (rank == 0) counts[e] = total;
+    kept = (cap > 0 && total > cap) ? cap : total;
+  }
+  // exclusive scan of kept over experts (E <= 1024)
+  int inc = kept;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += v;
+  }
+  if (lane == 31) s_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int wv = s_warp[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int v = __shfl_up_sync(0xffffffffu, wv, o);
+      if (lane >= o) wv += v;
+    }
+    s_warp[lane] = wv;
+  }
+  __syncthreads();
+  const int excl = (warp > 0 ? s_warp[warp - 1] : 0) + inc - kept;
+  if (e < E) {
+    s_off[e] = excl;
+    if (rank == 0) offsets[e] = excl;
+  }
+  if (rank == 0 && e == E - 1) offsets[E] = excl + kept;
+  cluster_sync_all();                    // no CTA reads a peer's totals past here
+  for (int base = lo; base < hi; base += 32) {
+    const int a = base + lane;
+    const int ee = (a < hi) ? s_ids[a] : -1;
+    const bool ok = (ee >= 0 && ee < E);
+    const unsigned peers = __match_any_sync(0xffffffffu, ok ? ee : -1);
+    int rk = 0;
+    if (ok) rk = s_base[ee] + my[ee] + __popc(peers & lt);
+    __syncwarp();
+    if (ok && (peers & lt) == 0) my[ee] += __popc(peers);
+    __syncwarp();
+    if (a < hi) {
+      int row = -1;
+      if (ok && (cap <= 0 || rk < cap)) {
+        row = s_off[ee] + rk;
+        row_src[row] = a0 + a;
+      }
+      inv[a0 + a] = row;
+    }
+  }
+}
 
 // One-pass token-choice permute for small problems (E <= 8, k <= 8, A <= kOnePassMaxItems):
 // every CTA owns 32 consecutive tokens.  It first counts ALL assignments per expert (totals)
@@ -502,6 +621,16 @@ int permute_blocks(const moe_desc_t& d) {
   return (int)((A + kBlockItems - 1) / kBlockItems);
 }
 
+// MOE_PERMUTE_CLUSTER=0 keeps the one-CTA index kernel (A <= 8192) and the three-kernel
+// histogram path instead of the cluster kernel (comparison measurements; both are tested).
+static bool permute_cluster_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_PERMUTE_CLUSTER");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids, const void* x,
                                         void* x_perm, int32_t* counts, int32_t* offsets,
                                         int32_t* row_src, int32_t* inv, int32_t* block_hist,
@@ -519,7 +648,34 @@ cudaError_t launch_permute_token_choice(const moe_desc_t& d, const int32_t* ids,
                                                 row_src, inv);
     return cudaGetLastError();
   }
-  if (A <= kFusedMaxItems) {
+  if (A > kClusterMinItems && A <= kClusterMaxItems && E <= 1024 && permute_cluster_enabled()) {
+    int ncta = (A + 1023) / 1024;
+    if (ncta > kClusterMaxCTAs) ncta = kClusterMaxCTAs;
+    const int chunk = ((A + ncta - 1) / ncta + 1023) / 1024 * 1024;
+    ncta = (A + chunk - 1) / chunk;
+    const size_t smem = ((size_t)35 * E + chunk) * sizeof(int);
+    cudaError_t e = cudaFuncSetAttribute(perm_index_cluster_kernel,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    note_launch();
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(ncta);
+    cfg.blockDim = dim3(1024);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute at[2];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = (unsigned)ncta;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    at[1].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = at;
+    cfg.numAttrs = pdl_enabled() ? 2 : 1;
+    e = cudaLaunchKernelEx(&cfg, perm_index_cluster_kernel, ids, A, E, cap, chunk, counts,
+                           offsets, row_src, inv);
+    if (e != cudaSuccess) return e;
+  } else if (A <= kFusedMaxItems) {
     const size_t smem = ((size_t)33 * E + A) * sizeof(int);
     if (smem > 48 * 1024)
       cudaFuncSetAttribute(perm_index_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,

@@ -111,6 +111,13 @@ __device__ __forceinline__ float ld_cluster_f32(uint32_t cl_addr) {
   return v;
 }
 
+// int32 load from a cluster shared-memory address (no memory clobber, as above).
+__device__ __forceinline__ int ld_cluster_s32(uint32_t cl_addr) {
+  int v;
+  asm volatile("ld.shared::cluster.s32 %0, [%1];" : "=r"(v) : "r"(cl_addr));
+  return v;
+}
+
 // Host: 2-D bf16 tensor map [rows, cols] (row-major), box = kb columns x box_rows rows,
 // 128-byte swizzle for kb = 64, 64-byte for kb = 32; rows past the end read as zeros.
 bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, uint64_t cols, uint32_t box_rows,

@@ -323,6 +323,23 @@ def test_switch_layer_without_adaptive_split_in_subprocess():
     assert " passed" in r.stdout, r.stdout[-3000:]
 
 
+def test_permutation_without_cluster_kernel_in_subprocess():
+    """MOE_PERMUTE_CLUSTER=0: between 2048 and 65536 assignments the permutation indexes with the
+    one-CTA kernel (up to 8192) or the three-kernel histogram path instead of one cluster of up
+    to 8 CTAs; the cases in that range pass both ways."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_PERMUTE_CLUSTER="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "(small_layer_matches_oracle or full_size_workload or capacity_drops) "
+                        "and (switch or v3 or router_E16_T20000 or router_E40 or groups_E64 or "
+                        "groups_E128 or router_E256_ec)"],
+                       env=env, capture_output=True, text=True, timeout=1200)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
+
+
 def test_layer_without_programmatic_dependent_launch_in_subprocess():
     """MOE_PDL=0 launches every kernel without programmatic stream serialization (each waits
     for the previous one to finish before it is scheduled); the small-case parity tests pass

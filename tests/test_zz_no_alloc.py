@@ -60,18 +60,18 @@ def _compare(w, d, x, ids):
     assert torch.equal(got["x_perm"][:n], ref["x_perm"][:n])
 
 
-# The permute takes its one-pass path (E <= 8 and at most 16384 assignments) or its one-CTA
-# index path (at most 8192 assignments otherwise) without touching the scratch array; above
-# those sizes it builds per-block histograms in it.
+# The permute takes its one-pass path (E <= 8 and at most 16384 assignments), its one-CTA
+# index path (at most 2048 assignments otherwise) or its cluster index path (at most 65536)
+# without touching the scratch array; above those sizes it builds per-block histograms in it.
 @pytest.mark.gpu
 @pytest.mark.parametrize("name,shape", [
     ("mixtral", dict(T=700, D=512, F=1024)),            # one-pass path
-    ("switch", dict(T=3000, D=256, E=16, F=512)),      # index path, capacity drop
+    ("switch", dict(T=3000, D=256, E=16, F=512)),      # cluster index path, capacity drop
     ("v3", dict(T=300, D=512, E=64, F=256, F_shared=256)),
     # histogram paths, in the fixed scratch array
     ("mixtral", dict(T=40000, D=128, F=128)),           # 80000 assignments, E = 8
     ("v3", dict(T=9000, D=128, E=64, F=128, F_shared=128)),   # 72000 assignments
-    ("switch", dict(T=20000, D=256, E=16, F=512)),     # 20000 assignments, capacity clamp
+    ("switch", dict(T=70000, D=128, E=16, F=128)),     # 70000 assignments, capacity clamp
 ])
 def test_noalloc_permute_matches_permute_on_two_calls(name, shape):
     w = scaled(WORKLOADS[name], **shape)
