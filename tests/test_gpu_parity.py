@@ -56,6 +56,8 @@ SMALL = {
                                   topk_group=4),
     "router_E16_T20000": scaled(W["mixtral"], T=20000, D=128, E=16, k=2, F=64),
     "router_E256_ec": scaled(W["ec"], T=600, D=512, E=256, F=128, c=10),
+    # three k-blocks: a cluster of three CTAs, one k-block each; E = 24 (N = 32, 24 live)
+    "router_E24_ks3": scaled(W["mixtral"], T=130, D=192, E=24, k=3, F=128),
     # the classic D -> F -> D expert with GELU (bf16 tensor-core epilogue, fp32 CUDA cores)
     "gelu_bf16": scaled(W["switch"], act="gelu", T=500, D=256, E=16, F=512, overflow="dropless",
                         gate="renorm", k=2, zipf_s=0.0),

@@ -23,6 +23,8 @@ CASES = {
     "swiglu_T1": scaled(WORKLOADS["mixtral"], T=1, D=1024, F=2048),
     # ReLU, two tokens over 16 experts: up split, down split
     "relu_T2": scaled(WORKLOADS["switch"], T=2, D=1024, E=16, F=1024, zipf_s=0.0),
+    # F not a multiple of 256: the up product's partial block starts at column 1536
+    "swiglu_T1_F1408": scaled(WORKLOADS["mixtral"], T=1, D=1024, F=1408),
     # GELU
     "gelu_T3": scaled(WORKLOADS["switch"], act="gelu", T=3, D=1024, E=16, F=512,
                       overflow="dropless", gate="renorm", k=2, zipf_s=0.0),
