@@ -157,6 +157,10 @@ moe_status_t moe_layer_views(const moe_desc_t* desc, void* ws, size_t ws_bytes,
 
 /* Score + Select + merge weights.
  * "Top-k 路由" gate Steps 1-2; Tiny MoE section 4; moe-comparison "Score"/"Select"/"Merge".
+ *   Kernels: bf16 with E <= 8 and D a multiple of 256 in [1024, 4096]: an mma.sync router;
+ *   other bf16 with D % 64 == 0 and E <= 256: the tcgen05 router product in CTA clusters fused
+ *   with the selection; otherwise a CUDA-core router.  Every path takes the same decisions from
+ *   its fp32 logits (MOE_ROUTER=tc|fast|gemm|simt in the environment selects one).
  *   x [T,D], Wg [E,D] (dtype); sel_bias [E] fp32 or NULL (added to sigmoid affinities for
  *   selection only).
  *   Token choice: expert_ids [T,k], gates [T,k]; slot j holds the j-th largest key (the logit
@@ -253,11 +257,17 @@ moe_status_t moe_gather_fusion(const moe_desc_t* desc, int32_t* on);
  * scratch_bytes = 0).  bf16 only: when the fused grouped product would keep fewer than 80% of
  * the SMs busy (a_rows <= 256 for the down product, <= 16 for the up product; active groups
  * bounded by min(n_groups, a_rows)), the product is split along K into 2..8 parts whose fp32
- * partials [S][a_rows][N] go to scratch and are summed in a fixed order (deterministic) before
- * the activation and the bf16 rounding.  When scratch is too small for the partials, or
- * MOE_DECODE_SPLITK=0 is set in the environment, the fused product runs.  moe_scratch_size
- * covers the routed experts' partials; moe_layer_forward uses this schedule for the routed
- * experts (the shared experts keep the fused products). */
+ * partials go to scratch and are summed in a fixed order (deterministic) before the activation
+ * and the bf16 rounding; SwiGLU's gate and up products run as one launch.
+ * moe_expert_down_ws also splits on the device: for a desc under a capacity limit whose fewest
+ * possible executed rows would give fewer output tiles than a B200 has SMs, the grouped GEMM
+ * reads the group table and, when its tiles fill fewer than half of its CTAs, splits K (at most
+ * 8 ways, fp32 partials of the executed rows within at most 24 MB of scratch) and a second
+ * kernel sums them in split order; otherwise it writes y directly.  When scratch is too small
+ * for the partials, or MOE_DECODE_SPLITK=0 (both schedules) / MOE_ADAPTIVE_SPLIT=0 (the
+ * device-side one) is set in the environment, the fused product runs.  moe_scratch_size covers
+ * the routed experts' partials; moe_layer_forward uses these schedules for the routed experts
+ * (the shared experts keep the fused products). */
 moe_status_t moe_expert_up_ws(const moe_desc_t* desc, int32_t n_groups, int32_t F,
                               const void* a, int64_t a_rows, const int32_t* offsets,
                               const void* W_gate, const void* W_up, void* h, void* scratch,
