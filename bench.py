@@ -383,8 +383,10 @@ def time_backward(M, w, d, inp, ws, stream, dev, steps, warmup, tc_peak, world):
 
 
 class LayerStep:
-    """One step of the layer through the library's step entry points, in the order
-    moe_layer_forward chains them, with optional CUDA events between the stages."""
+    """One step of the layer: `layer` is one moe_layer_forward call (the headline graph);
+    calling the object runs the library's step entry points in the order moe_layer_forward
+    chains them, with optional CUDA events between the stages (the eager and per-stage
+    times)."""
 
     def __init__(self, M, w, inp, dev, stream):
         self.M, self.w, self.inp, self.dev, self.stream = M, w, inp, dev, stream
@@ -402,6 +404,14 @@ class LayerStep:
         # as in moe_layer_forward: with enough rows the up projection gathers the token rows
         # itself and the permutation writes indices only
         self.gather = M.gather_fusion(self.d)
+
+    def layer(self, st=None):
+        """The whole layer as one moe_layer_forward call."""
+        M, w, inp = self.M, self.w, self.inp
+        s = st if st is not None else self.stream
+        sh = (inp.Ws_gate, inp.Ws_up, inp.Ws_down) if w.n_shared else (None, None, None)
+        M.moe_layer_forward(self.d, inp.x, inp.Wg, inp.bias, inp.W_gate, inp.W_up, inp.W_down,
+                            *sh, self.out, self.ws, s)
 
     def __call__(self, ev=None, st=None):
         M, w, inp, v = self.M, self.w, self.inp, self.v
@@ -441,8 +451,9 @@ class LayerStep:
             ev[6].record(s)
 
     def capture(self, warmup):
-        """The step captured once in a CUDA graph (the library allocates and synchronises
-        nothing, so its calls capture as they are); replays remove the host launch gaps."""
+        """The layer (one moe_layer_forward call) captured once in a CUDA graph (the library
+        allocates and synchronises nothing, so its calls capture as they are); replays remove
+        the host launch gaps."""
         M, dev = self.M, self.dev
         try:
             cap = torch.cuda.Stream(dev)
@@ -450,7 +461,7 @@ class LayerStep:
             g = torch.cuda.CUDAGraph()
             n0 = M.kernel_launches()
             with torch.cuda.graph(g, stream=cap):
-                self(st=cap)
+                self.layer(st=cap)
             self.graph_launches = M.kernel_launches() - n0
             self.stream.wait_stream(cap)
             for _ in range(max(warmup, 3)):
@@ -721,8 +732,9 @@ def run_cuda(args, rank, world, local):
                 "serial_value": round(job_throughput(w.T, world, args.steps, e2e_serial_ms), 1)},
         "gpu_launches": launches,
         "clocks": clk.summary(),
-        "timing": ("CUDA-graph replay of the step (%d library kernels per step); per-stage "
-                   "times from eager calls" % step.graph_launches) if use_graph else
+        "timing": ("CUDA-graph replay of one moe_layer_forward call (%d library kernels per "
+                   "step); per-stage times from the step entry points" % step.graph_launches)
+                  if use_graph else
                   ("eager calls" + (" (graph capture failed: %s)" % step.graph_error
                                     if step.graph_error else "")),
         "eager_value": round(job_throughput(w.T, world, args.steps, eager_ms), 1),
