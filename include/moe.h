@@ -298,7 +298,9 @@ moe_status_t moe_balance_stats(const moe_desc_t* desc, const int32_t* counts,
 
 /* The whole layer: route -> permute -> expert_ffn (+ shared experts) -> combine -> stats,
  * enqueued on one stream with no host synchronisation.  Intermediates live in `ws`
- * (moe_workspace_size bytes); moe_layer_views gives their addresses.
+ * (moe_workspace_size bytes); moe_layer_views gives their addresses.  The last two steps run
+ * as one launch (the combine's first block computes the statistics); f and the moe_stats_t in
+ * `ws` equal, bit for bit, what moe_balance_stats computes from the same views.
  *   x [T,D], Wg [E,D], sel_bias [E] or NULL, routed weights as above, shared weights
  *   [S,Fs,D], [S,Fs,D], [S,D,Fs] (NULL when S = 0), out [T,D]. */
 moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void* Wg,

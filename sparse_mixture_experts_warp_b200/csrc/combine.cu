@@ -60,13 +60,81 @@ template <> struct Row<false> {    // 4 fp32 per 16 bytes
   }
 };
 
+// The balance statistics of one layer call, computed by one block of 256 threads (E <= 256):
+// f, aux, max/mean, kept/dropped, count percentiles (ranks by counting, ties by expert id) and
+// the router's mean entropy; fixed-order tree sums (deterministic).  Every thread of the block
+// calls it.
+__device__ __noinline__ void balance_stats_block(const StatsArgs& a) {
+  __shared__ float s_fp[256];
+  __shared__ int s_max[256];
+  __shared__ int s_sorted[256];
+  __shared__ int s_cnt[256];
+  const int tid = threadIdx.x;
+  const int E = a.E;
+  float fp = 0.f;
+  int c = 0;
+  if (tid < E) {
+    c = a.counts[tid];
+    s_cnt[tid] = c;
+  }
+  __syncthreads();
+  if (tid < E) {
+    const float fe = (float)c / (float)a.n_routes;
+    a.f[tid] = fe;
+    fp = fe * a.importance[tid];
+    // rank of this count among all (ties by expert id): its slot in ascending order
+    int rank = 0;
+    for (int e = 0; e < E; ++e) {
+      const int ce = s_cnt[e];
+      rank += (ce < c) || (ce == c && e < tid);
+    }
+    s_sorted[rank] = c;
+  }
+  s_fp[tid] = fp;
+  s_max[tid] = c;
+  __syncthreads();
+  for (int hw = 128; hw > 0; hw >>= 1) {        // fixed-order tree
+    if (tid < hw) {
+      s_fp[tid] += s_fp[tid + hw];
+      s_max[tid] = max(s_max[tid], s_max[tid + hw]);
+    }
+    __syncthreads();
+  }
+  if (tid == 0) {
+    const int kept = a.offsets[E];
+    moe_stats_t r;
+    r.aux = a.alpha * (float)E * s_fp[0];
+    const float mean = (float)a.n_routes / (float)E;
+    r.max_over_mean = mean > 0.f ? (float)s_max[0] / mean : 0.f;
+    r.n_routes = a.n_routes;
+    r.n_kept = kept;
+    r.n_dropped = a.n_routes - kept;
+    r.reserved = 0;
+    r.entropy = a.entropy ? *a.entropy : __int_as_float(0x7fc00000);
+    float q[2];
+    const double pct[2] = {0.95, 0.99};
+    for (int i = 0; i < 2; ++i) {
+      const double pos = pct[i] * (double)(E - 1);
+      const int lo = (int)pos;
+      const int hi = lo + 1 < E ? lo + 1 : lo;
+      const double fr = pos - lo;
+      q[i] = (float)(s_sorted[lo] + fr * (double)(s_sorted[hi] - s_sorted[lo]));
+    }
+    r.count_p95 = q[0];
+    r.count_p99 = q[1];
+    r.reserved2 = 0.f;
+    *a.st = r;
+  }
+}
+
 template <bool BF16>
 __global__ void __launch_bounds__(kWarps * 32)
 combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                const float* __restrict__ gates, const uint4* __restrict__ ys, int S, int T,
-               int K, int nvec, uint4* __restrict__ out) {
+               int K, int nvec, uint4* __restrict__ out, const StatsArgs sa) {
   pdl_trigger();
   pdl_wait();
+  if (sa.st && blockIdx.x == 0) balance_stats_block(sa);
   using R = Row<BF16>;
   __shared__ int s_row[kWarps][kMaxList];
   __shared__ float s_g[kWarps][kMaxList];
@@ -134,9 +202,10 @@ template <bool BF16, int K>
 __global__ void __launch_bounds__(kWarps * 32)
 combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                        const float* __restrict__ gates, int T, int nvec,
-                       uint4* __restrict__ out) {
+                       uint4* __restrict__ out, const StatsArgs sa) {
   pdl_trigger();
   pdl_wait();
+  if (sa.st && blockIdx.x == 0) balance_stats_block(sa);
   using R = Row<BF16>;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t = blockIdx.x * kWarps + warp;
@@ -179,75 +248,37 @@ combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ 
   }
 }
 
-// One block of 256 threads: f, aux, max/mean, kept/dropped, count percentiles (ranks by
-// counting, E <= 256) and the router's mean entropy; fixed-order tree sums (deterministic).
-__global__ void __launch_bounds__(256)
-stats_kernel(const int32_t* counts, const int32_t* offsets, const float* importance,
-             const float* entropy, int E, int n_routes, float alpha, float* f, moe_stats_t* st) {
+// The statistics as a kernel of their own (moe_balance_stats): one block of 256 threads.
+__global__ void __launch_bounds__(256) stats_kernel(const StatsArgs a) {
   pdl_trigger();
   pdl_wait();
-  __shared__ float s_fp[256];
-  __shared__ int s_max[256];
-  __shared__ int s_sorted[256];
-  const int tid = threadIdx.x;
-  float fp = 0.f;
-  int c = 0;
-  if (tid < E) {
-    c = counts[tid];
-    const float fe = (float)c / (float)n_routes;
-    f[tid] = fe;
-    fp = fe * importance[tid];
-    // rank of this count among all (ties by expert id): its slot in ascending order
-    int rank = 0;
-    for (int e = 0; e < E; ++e) {
-      const int ce = counts[e];
-      rank += (ce < c) || (ce == c && e < tid);
-    }
-    s_sorted[rank] = c;
-  }
-  s_fp[tid] = fp;
-  s_max[tid] = c;
-  __syncthreads();
-  for (int hw = 128; hw > 0; hw >>= 1) {        // fixed-order tree
-    if (tid < hw) {
-      s_fp[tid] += s_fp[tid + hw];
-      s_max[tid] = max(s_max[tid], s_max[tid + hw]);
-    }
-    __syncthreads();
-  }
-  if (tid == 0) {
-    const int kept = offsets[E];
-    moe_stats_t r;
-    r.aux = alpha * (float)E * s_fp[0];
-    const float mean = (float)n_routes / (float)E;
-    r.max_over_mean = mean > 0.f ? (float)s_max[0] / mean : 0.f;
-    r.n_routes = n_routes;
-    r.n_kept = kept;
-    r.n_dropped = n_routes - kept;
-    r.reserved = 0;
-    r.entropy = entropy ? *entropy : __int_as_float(0x7fc00000);
-    float q[2];
-    const double pct[2] = {0.95, 0.99};
-    for (int i = 0; i < 2; ++i) {
-      const double pos = pct[i] * (double)(E - 1);
-      const int lo = (int)pos;
-      const int hi = lo + 1 < E ? lo + 1 : lo;
-      const double fr = pos - lo;
-      q[i] = (float)(s_sorted[lo] + fr * (double)(s_sorted[hi] - s_sorted[lo]));
-    }
-    r.count_p95 = q[0];
-    r.count_p99 = q[1];
-    r.reserved2 = 0.f;
-    *st = r;
-  }
+  balance_stats_block(a);
 }
 
 }  // namespace
 
+StatsArgs stats_args(const moe_desc_t& d, const int32_t* counts, const int32_t* offsets,
+                     const float* importance, const float* entropy, float* f,
+                     moe_stats_t* stats) {
+  StatsArgs a;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.importance = importance;
+  a.entropy = entropy;
+  a.E = d.E;
+  a.n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
+  a.alpha = d.aux_alpha;
+  a.f = f;
+  a.st = stats;
+  return a;
+}
+
 cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
                            const float* gates, const void* y_shared, void* out,
-                           cudaStream_t s) {
+                           cudaStream_t s, const StatsArgs* with_stats) {
   if (d.T == 0) return cudaSuccess;
+  StatsArgs sa{};
+  if (with_stats) sa = *with_stats;
   const int K = (d.select == MOE_EXPERT_CHOICE) ? d.E : d.k;
   const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
   const int nvec = d.D * esz / 16;
@@ -257,22 +288,22 @@ cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* in
     const uint4* yy = static_cast<const uint4*>(y);
     uint4* oo = static_cast<uint4*>(out);
     if (d.dtype == MOE_BF16) {
-      if (K == 1) (void)launch_pdl(combine_small_k_kernel<true, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
-      else (void)launch_pdl(combine_small_k_kernel<true, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<true, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
+      else (void)launch_pdl(combine_small_k_kernel<true, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
     } else {
-      if (K == 1) (void)launch_pdl(combine_small_k_kernel<false, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
-      else (void)launch_pdl(combine_small_k_kernel<false, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<false, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
+      else (void)launch_pdl(combine_small_k_kernel<false, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
     }
     return cudaGetLastError();
   }
   if (d.dtype == MOE_BF16)
     (void)launch_pdl(combine_kernel<true>, dim3(blocks), dim3(kWarps * 32), 0, s, 
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
-        K, nvec, static_cast<uint4*>(out));
+        K, nvec, static_cast<uint4*>(out), sa);
   else
     (void)launch_pdl(combine_kernel<false>, dim3(blocks), dim3(kWarps * 32), 0, s, 
         static_cast<const uint4*>(y), inv, gates, static_cast<const uint4*>(y_shared), S, d.T,
-        K, nvec, static_cast<uint4*>(out));
+        K, nvec, static_cast<uint4*>(out), sa);
   return cudaGetLastError();
 }
 
@@ -280,9 +311,8 @@ cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance,
                                  const float* entropy, float* f, moe_stats_t* stats,
                                  cudaStream_t s) {
-  const int n_routes = (d.select == MOE_EXPERT_CHOICE) ? d.E * d.c : d.T * d.k;
-  (void)launch_pdl(stats_kernel, dim3(1), dim3(256), 0, s, counts, offsets, importance, entropy, d.E, n_routes,
-                                          d.aux_alpha, f, stats);
+  (void)launch_pdl(stats_kernel, dim3(1), dim3(256), 0, s,
+                   stats_args(d, counts, offsets, importance, entropy, f, stats));
   return cudaGetLastError();
 }
 

@@ -147,6 +147,16 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
                                      float* adapt_part = nullptr, int64_t adapt_cap = 0,
                                      int adapt_ks_max = 0, int* adapt_ks = nullptr);
 bool gemm_gather_ok();   // the selected tile shape can gather A rows
+// gemm_swap.cu: the same grouped product with the weights as the MMA's M side and the tokens as
+// its N side (tiles of 256 weight rows by up to 256 tokens, N rounded up to 16), for many groups
+// of a few hundred rows or fewer; EPI_SWIGLU / EPI_RELU / EPI_GELU / EPI_NONE, bf16 out
+// [a_rows, N]; gather_src as above; fault: the bounded-wait test hook.
+bool swap_epilogue_ok(int epi);
+cudaError_t launch_grouped_gemm_swap(int epi, const void* A, int64_t a_rows, int K,
+                                     const void* B0, const void* B1, int n_groups, int N,
+                                     const int32_t* offsets, void* out, cudaStream_t s,
+                                     const int32_t* gather_src, int gather_div, int64_t src_rows,
+                                     int fault);
 
 // Router product on the same engine: one group of T rows, N = E, fp32 partial logits of
 // ksplit k-ranges in partials[ksplit][T][E] (E % 32 == 0, E <= 256).
@@ -212,9 +222,26 @@ cudaError_t launch_ffn_down_f32(const float* h, int64_t a_rows, int D, int F,
                                 float* y, cudaStream_t s);
 
 // combine.cu
+// Inputs of the balance statistics (moe_balance_stats): counts / offsets from the permutation,
+// importance / entropy from the router, outputs f [E] and *st.
+struct StatsArgs {
+  const int32_t* counts;
+  const int32_t* offsets;
+  const float* importance;
+  const float* entropy;
+  int E, n_routes;
+  float alpha;
+  float* f;
+  moe_stats_t* st;
+};
+StatsArgs stats_args(const moe_desc_t& d, const int32_t* counts, const int32_t* offsets,
+                     const float* importance, const float* entropy, float* f,
+                     moe_stats_t* stats);
+// with_stats: block 0 of the combine also computes the balance statistics (the layer step's
+// last two stages in one launch; every input of the statistics was written by earlier kernels)
 cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
                            const float* gates, const void* y_shared, void* out,
-                           cudaStream_t s);
+                           cudaStream_t s, const StatsArgs* with_stats = nullptr);
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance,
                                  const float* entropy, float* f, moe_stats_t* stats,

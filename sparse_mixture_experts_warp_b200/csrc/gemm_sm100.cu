@@ -166,19 +166,6 @@ __device__ __forceinline__ Tile locate(int t, int total, int nkb, int kchunk, co
   return r;
 }
 
-// Four rows (y0..y3) of 64 (or 32) columns from x on, through a tensor map whose box is one row
-// high, into four consecutive 128-byte (64-byte) rows of shared memory; the map's swizzle
-// applies as for a tiled box.
-__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
-                                            int x, int y0, int y1, int y2, int y3) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
-      "r"(y2), "r"(y3)
-      : "memory");
-}
-
 // Shared -> global tile store through a 3-D tensor map (x = column, y = row, z = group); the
 // copy joins the issuing thread's current bulk group.
 __device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, uint32_t src, int x, int y,
@@ -1269,6 +1256,20 @@ GemmTile gemm_tile() {
 // tile a short main loop whose epilogue is not overlapped; 128-row tiles with two TMEM
 // accumulators measured faster there (V3 down projection 1.70 -> 1.61 ms).  Large groups
 // (Mixtral: 1024 rows per expert) keep the 256-row tiles.
+// Weights-as-M schedule (gemm_swap.cu), taken for every eligible call when MOE_GEMM_SWAP=1
+// (unless MOE_GEMM_TILE names a row-tile shape).  Off by default: it measured slower than the
+// row tiles at the DeepSeek-V3 shape (up 2.94 against 2.51 ms, down 1.81 against 1.72 ms) and
+// at the Mixtral shape.  An M=128 MMA reads its 4 KB weight slice from shared memory whatever
+// its N, so a token tile below ~128 rows needs more than the SM's 128 B per clock of shared
+// memory bandwidth; the row tiles always run N = 256.
+bool use_swap(int epi, bool grouped, bool out2, bool adapt) {
+  static const bool on = [] {
+    const char* e = getenv("MOE_GEMM_SWAP");
+    return e && !strcmp(e, "1");
+  }();
+  return on && grouped && !out2 && !adapt && swap_epilogue_ok(epi) && gemm_tile_env() < 0;
+}
+
 GemmTile tile_for(int64_t a_rows, int n_groups, bool grouped) {
   const int t = gemm_tile_env();
   if (t >= 0) return (GemmTile)t;
@@ -1408,6 +1409,9 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   const bool adapt = adapt_ks_max > 1;
   if (adapt && (epi != EPI_NONE || !offsets || out2 || gather_src || !adapt_part || !adapt_ks))
     return cudaErrorInvalidValue;
+  if (use_swap(epi, offsets != nullptr, out2 != nullptr, adapt))
+    return launch_grouped_gemm_swap(epi, A, a_rows, K, B0, B1, n_groups, N, offsets, out, s,
+                                    gather_src, gather_div, src_rows, g_gemm_fault);
   alignas(64) CUtensorMap ta, tb0, tb1;
   const uint64_t brows = (uint64_t)n_groups * (uint64_t)N;
   GemmParams p{};

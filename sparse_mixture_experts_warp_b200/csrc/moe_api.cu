@@ -697,9 +697,13 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
       if (st != MOE_OK) return st;
     }
   }
-  st = moe_combine(d, v.y, v.inv, v.gates, d->n_shared > 0 ? v.y_shared : nullptr, out, stream);
-  if (st != MOE_OK) return st;
-  return moe_balance_stats(d, v.counts, v.offsets, v.importance, v.entropy, v.f, v.stats, stream);
+  // the combine's first block also computes the balance statistics (the stages of
+  // moe_combine and moe_balance_stats in one launch)
+  if (!is_aligned16(out)) return MOE_ERR_INVALID_ARG;
+  const StatsArgs sa = stats_args(*d, v.counts, v.offsets, v.importance, v.entropy, v.f, v.stats);
+  return cuda_status(launch_combine(*d, v.y, v.inv, v.gates,
+                                    d->n_shared > 0 ? v.y_shared : nullptr, out,
+                                    reinterpret_cast<cudaStream_t>(stream), &sa));
 }
 
 // ---------------- backward ----------------

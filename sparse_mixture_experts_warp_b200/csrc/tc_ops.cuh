@@ -20,6 +20,19 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* map
       : "memory");
 }
 
+// Four rows (y0..y3) of 64 (or 32) columns from x on, through a tensor map whose box is one row
+// high, into four consecutive 128-byte (64-byte) rows of shared memory; the map's swizzle
+// applies as for a tiled box.
+__device__ __forceinline__ void tma_gather4(uint32_t dst, const CUtensorMap* map, uint64_t* bar,
+                                            int x, int y0, int y1, int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1),
+      "r"(y2), "r"(y3)
+      : "memory");
+}
+
 // Shared-memory matrix descriptor, K-major, rows of KB bf16 (KB = 64: 128-byte swizzle, 8-row
 // core groups 1024 B apart; KB = 32: 64-byte swizzle, groups 512 B apart).
 template <int KB>

@@ -42,6 +42,9 @@ def _case(act, D, F, counts, extra_rows=5, seed=3):
     (256, 192, [0, 1, 127, 129, 300]),
     (128, 512, [5, 0, 0, 256, 3]),
     (512, 256, [1000]),
+    # token tiles of the weights-as-M schedule: N = 16 and 32 (17 rows), three token tiles
+    # (513 rows: 256 + 256 + 1), 64 live features in the last feature tile (F = 320)
+    (256, 320, [17, 16, 513, 0, 33]),
 ])
 def test_grouped_gemm_ragged(act, D, F, counts):
     d, G, a, Wg, Wu, Wd, offsets, h, y, n, sentinel = _case(act, D, F, counts)
@@ -85,15 +88,19 @@ def test_grouped_gemm_repeatable():
     assert torch.equal(y1[:n], y[:n])
 
 
-@pytest.mark.parametrize("tile", ["128", "256k32", "pair"])
-def test_grouped_gemm_other_tiles_in_subprocess(tile):
+@pytest.mark.parametrize("var,val", [("MOE_GEMM_TILE", "128"), ("MOE_GEMM_TILE", "256k32"),
+                                     ("MOE_GEMM_TILE", "pair"), ("MOE_GEMM_SWAP", "0"),
+                                     ("MOE_GEMM_SWAP", "1")])
+def test_grouped_gemm_other_tiles_in_subprocess(var, val):
     """The other tile shapes (128-row tiles with a double TMEM buffer; 256-row tiles with
     32-element k-blocks; 256 x 256 tiles on a CTA pair) are selected per process by
-    MOE_GEMM_TILE; run this file's ragged cases under each in a child process."""
+    MOE_GEMM_TILE, and the weights-as-M schedule by MOE_GEMM_SWAP=1 (every grouped call, the
+    one-group case included; MOE_GEMM_SWAP=0 is the default, the row tiles); run this file's
+    ragged cases under each in a child process."""
     import os
     import subprocess
     import sys
-    env = dict(os.environ, MOE_GEMM_TILE=tile)
+    env = dict(os.environ, **{var: val})
     r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__,
                         "-k", "ragged or repeatable"],
                        env=env, capture_output=True, text=True, timeout=600)

@@ -108,6 +108,25 @@ def test_layer_is_deterministic():
     assert torch.equal(rs1, v2["row_src"])
 
 
+@pytest.mark.parametrize("name", ["mixtral_small", "switch_small", "v3_small", "ec_small",
+                                  "router_E8_T1"])
+def test_layer_statistics_equal_the_statistics_entry_point(name):
+    """moe_layer_forward computes the balance statistics in the combine's first block; they equal,
+    bit for bit, what moe_balance_stats computes from the same counts, offsets, importance and
+    entropy."""
+    w = SMALL[name]
+    inp = C.inputs_for(w)
+    _, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    f = torch.full_like(v["f"], float("nan"))
+    stats = torch.zeros_like(v["stats"])
+    M.moe_balance_stats(d, v["counts"], v["offsets"], v["importance"], f, stats,
+                        entropy=v["entropy"])
+    torch.cuda.synchronize()
+    assert torch.equal(f, v["f"])
+    assert torch.equal(stats, v["stats"])
+
+
 def test_capacity_drops_give_zero_rows():
     w = SMALL["switch_small"]
     inp = C.inputs_for(w)
@@ -321,6 +340,22 @@ def test_switch_layer_without_adaptive_split_in_subprocess():
                         "(small_layer_matches_oracle or full_size_workload or capacity_drops) "
                         "and (switch or f32_relu_drop or router_E40)"],
                        env=env, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
+
+
+def test_layer_with_weights_as_m_tiles_in_subprocess():
+    """MOE_GEMM_SWAP=1 runs every expert product of the layer (bf16, inference) on the
+    weights-as-M tiles instead of the row tiles: token tiles of up to 256 rows with N rounded to
+    16, gathered or tiled token loads; the layer cases pass there too."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_GEMM_SWAP="1")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "small_layer_matches_oracle or full_size_workload or decode_regime or "
+                        "gathering_up_projection or v3_node_limited"],
+                       env=env, capture_output=True, text=True, timeout=1800)
     assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
     assert " passed" in r.stdout, r.stdout[-3000:]
 
