@@ -88,64 +88,110 @@ bool router_tc_ok(const moe_desc_t& d);
 cudaError_t launch_router_tc(const moe_desc_t& d, const RouterArgs& a, int* n_partials,
                              cudaStream_t s);
 
-// One token.  Lane l holds s[i] = logit of expert l + 32 i (-inf past E).  Writes the token's
-// logits row (when a.logits), adds its probabilities to imp and its -sum p log p to ent; under
-// expert choice writes its probabilities as gates[tok][e] and leaves them in p, under token
-// choice writes its k expert ids and merge weights.
+// Order-preserving map of a float key to an unsigned integer (-0 counts as +0, so that equal
+// keys compare equal as in float compares), for warp reductions with redux.sync.
+__device__ __forceinline__ uint32_t ord_key(float f) {
+  const uint32_t b = __float_as_uint(f + 0.0f);
+  return (b & 0x80000000u) ? ~b : (b | 0x80000000u);
+}
+__device__ __forceinline__ float ord_to_float(uint32_t o) {
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+
+// NT tokens in lockstep (their dependency chains interleave: the selection is latency-bound,
+// one warp per token).  Lane l holds s[t][i] = logit of expert l + 32 i of token tok[t] (-inf
+// past E); tokens with has[t] false are computed on and discarded.  For each token: writes its
+// logits row (when a.logits), adds its probabilities to imp and its -sum p log p to ent (token
+// 0 first, then token 1, ...); under expert choice writes its probabilities as
+// gates[tok][e] and leaves them in p, under token choice writes its k expert ids and merge
+// weights.  Top-k: k rounds of a warp arg-max over (key desc, expert id asc), each two
+// redux.sync reductions: the largest key (order-preserving integers), then the smallest expert
+// id holding it.
 // NS = expert slots per lane (E <= 32 NS): the loops below cover only those.
-template <int NS>
-__device__ __forceinline__ void select_token(const RouterArgs& a, int tok, const float (&s)[NS],
-                                             float (&imp)[NS], float& ent, float (&p)[NS],
-                                             int lane) {
+template <int NS, int NT>
+__device__ __forceinline__ void select_tokens(const RouterArgs& a, const int (&tok)[NT],
+                                              const bool (&has)[NT], const float (&s)[NT][NS],
+                                              float (&imp)[NS], float& ent,
+                                              float (&p)[NT][NS], int lane) {
   const int E = a.E;
-  float key[NS];
-  float m = -INFINITY;
-#pragma unroll
-  for (int i = 0; i < NS; ++i) m = fmaxf(m, s[i]);
+  float sel_w[NT][NS];   // weight used in the merge (softmax p or sigmoid affinity)
+  float key[NT][NS];
   if (a.logits) {
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) a.logits[(int64_t)tok * E + e] = s[i];
+    for (int t = 0; t < NT; ++t) {
+      if (!has[t]) continue;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) a.logits[(int64_t)tok[t] * E + e] = s[t][i];
+      }
     }
   }
-  float sel_w[NS];   // weight used in the merge (softmax p or sigmoid affinity)
   if (a.score == MOE_SCORE_SOFTMAX) {
-    m = warp_max(m);
-    float z = 0.f;
+    float m[NT], z[NT];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      const int e = lane + 32 * i;
-      p[i] = (e < E) ? expf(s[i] - m) : 0.f;
-      z += p[i];
+    for (int t = 0; t < NT; ++t) {
+      m[t] = -INFINITY;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) m[t] = fmaxf(m[t], s[t][i]);
+      m[t] = ord_to_float(__reduce_max_sync(0xffffffffu, ord_key(m[t])));
     }
-    z = warp_sum(z);
-    const float inv = 1.0f / z;
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      p[i] = p[i] * inv;
-      key[i] = s[i];             // softmax is monotone in the logit within a row
-      sel_w[i] = p[i];
-      imp[i] += p[i];
-      if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
+    for (int t = 0; t < NT; ++t) {
+      z[t] = 0.f;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        p[t][i] = (e < E) ? expf(s[t][i] - m[t]) : 0.f;
+        z[t] += p[t][i];
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) z[t] += __shfl_xor_sync(0xffffffffu, z[t], o);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float inv = 1.0f / z[t];
+#pragma unroll
+      for (int i = 0; i < NS; ++i) {
+        p[t][i] = p[t][i] * inv;
+        key[t][i] = s[t][i];         // softmax is monotone in the logit within a row
+        sel_w[t][i] = p[t][i];
+      }
     }
   } else {
-    float asum = 0.f;
+    float asum[NT];
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      const int e = lane + 32 * i;
-      const float af = (e < E) ? 1.0f / (1.0f + expf(-s[i])) : 0.f;
-      sel_w[i] = af;
-      key[i] = (e < E) ? af + (a.bias ? a.bias[e] : 0.f) : -INFINITY;
-      asum += af;
+    for (int t = 0; t < NT; ++t) {
+      asum[t] = 0.f;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        const float af = (e < E) ? 1.0f / (1.0f + expf(-s[t][i])) : 0.f;
+        sel_w[t][i] = af;
+        key[t][i] = (e < E) ? af + (a.bias ? a.bias[e] : 0.f) : -INFINITY;
+        asum[t] += af;
+      }
     }
-    asum = warp_sum(asum);
-    const float inv = 1.0f / asum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) asum[t] += __shfl_xor_sync(0xffffffffu, asum[t], o);
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      const float inv = 1.0f / asum[t];
+#pragma unroll
+      for (int i = 0; i < NS; ++i) p[t][i] = sel_w[t][i] * inv;
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    if (!has[t]) continue;
 #pragma unroll
     for (int i = 0; i < NS; ++i) {
-      p[i] = sel_w[i] * inv;
-      imp[i] += p[i];
-      if (p[i] > 0.f) ent -= p[i] * logf(p[i]);
+      imp[i] += p[t][i];
+      if (p[t][i] > 0.f) ent -= p[t][i] * logf(p[t][i]);
     }
   }
 
@@ -153,51 +199,82 @@ __device__ __forceinline__ void select_token(const RouterArgs& a, int tok, const
     // merge weights are the softmax probabilities; selection happens per expert later (the
     // caller stages the transposed copy from p)
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E) a.gates[(int64_t)tok * E + e] = p[i];
+    for (int t = 0; t < NT; ++t) {
+      if (!has[t]) continue;
+#pragma unroll
+      for (int i = 0; i < NS; ++i) {
+        const int e = lane + 32 * i;
+        if (e < E) a.gates[(int64_t)tok[t] * E + e] = p[t][i];
+      }
     }
     return;
   }
 
-  group_limit<NS>(key, E, a.n_group, a.topk_group, lane);
+#pragma unroll
+  for (int t = 0; t < NT; ++t) group_limit<NS>(key[t], E, a.n_group, a.topk_group, lane);
 
-  // top-k: k rounds of a warp arg-max over (key desc, expert id asc)
-  bool taken[NS];
+  // top-k rounds; okey = 0 marks a slot that is taken or past E (every real key maps above 0)
+  uint32_t okey[NT][NS];
 #pragma unroll
-  for (int i = 0; i < NS; ++i) taken[i] = false;
-  int my_id = -1;        // lane j < k keeps slot j
-  float my_w = 0.f;
-  float wsum = 0.f;
+  for (int t = 0; t < NT; ++t)
+#pragma unroll
+    for (int i = 0; i < NS; ++i)   // a NaN key never wins a comparison: never a candidate
+      okey[t][i] = (lane + 32 * i < E && key[t][i] == key[t][i]) ? ord_key(key[t][i]) : 0u;
+  int my_id[NT];         // lane j < k keeps slot j
+  float my_w[NT], wsum[NT];
+#pragma unroll
+  for (int t = 0; t < NT; ++t) {
+    my_id[t] = -1;
+    my_w[t] = 0.f;
+    wsum[t] = 0.f;
+  }
   for (int j = 0; j < a.k; ++j) {
-    float bk = -INFINITY;
-    int bi = 0x7fffffff;
 #pragma unroll
-    for (int i = 0; i < NS; ++i) {
-      const int e = lane + 32 * i;
-      if (e < E && !taken[i] && (key[i] > bk || (key[i] == bk && e < bi))) { bk = key[i]; bi = e; }
+    for (int t = 0; t < NT; ++t) {
+      // this lane's best untaken slot: largest key, and among equal keys the first slot
+      // (the lowest expert id of this lane)
+      uint32_t bk = 0u;
+      int bi = 0x7fffffff;
+#pragma unroll
+      for (int i = 0; i < NS; ++i)
+        if (okey[t][i] > bk) { bk = okey[t][i]; bi = lane + 32 * i; }
+      const uint32_t wk = __reduce_max_sync(0xffffffffu, bk);
+      const int wi = (int)__reduce_min_sync(0xffffffffu, (unsigned)(bk == wk ? bi : 0x7fffffff));
+      // owner lane marks it and broadcasts its merge weight
+      const int owner = wi & 31, slot = wi >> 5;
+      float w = 0.f;
+#pragma unroll
+      for (int i = 0; i < NS; ++i)
+        if (lane == owner && i == slot) { okey[t][i] = 0u; w = sel_w[t][i]; }
+      w = __shfl_sync(0xffffffffu, w, owner);
+      wsum[t] += w;
+      if (lane == j) { my_id[t] = wi; my_w[t] = w; }
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ok = __shfl_xor_sync(0xffffffffu, bk, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ok > bk || (ok == bk && oi < bi)) { bk = ok; bi = oi; }
-    }
-    // owner lane marks it and broadcasts its merge weight
-    const int owner = bi & 31, slot = bi >> 5;
-    float w = 0.f;
-#pragma unroll
-    for (int i = 0; i < NS; ++i)
-      if (lane == owner && i == slot) { taken[i] = true; w = sel_w[i]; }
-    w = __shfl_sync(0xffffffffu, w, owner);
-    wsum += w;
-    if (lane == j) { my_id = bi; my_w = w; }
   }
   if (lane < a.k) {
-    const float g = (a.gate == MOE_GATE_RENORM) ? my_w / wsum : my_w;
-    a.ids[(int64_t)tok * a.k + lane] = my_id;
-    a.gates[(int64_t)tok * a.k + lane] = g;
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      if (!has[t]) continue;
+      const float g = (a.gate == MOE_GATE_RENORM) ? my_w[t] / wsum[t] : my_w[t];
+      a.ids[(int64_t)tok[t] * a.k + lane] = my_id[t];
+      a.gates[(int64_t)tok[t] * a.k + lane] = g;
+    }
   }
+}
+
+// One token (select_tokens with NT = 1).
+template <int NS>
+__device__ __forceinline__ void select_token(const RouterArgs& a, int tok, const float (&s)[NS],
+                                             float (&imp)[NS], float& ent, float (&p)[NS],
+                                             int lane) {
+  const int tk[1] = {tok};
+  const bool has[1] = {true};
+  float s1[1][NS], p1[1][NS];
+#pragma unroll
+  for (int i = 0; i < NS; ++i) s1[0][i] = s[i];
+  select_tokens<NS, 1>(a, tk, has, s1, imp, ent, p1, lane);
+#pragma unroll
+  for (int i = 0; i < NS; ++i) p[i] = p1[0][i];
 }
 
 }  // namespace moe

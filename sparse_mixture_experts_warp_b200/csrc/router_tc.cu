@@ -260,20 +260,32 @@ router_tc_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant_
 #pragma unroll
   for (int u = 0; u < NS; ++u) imp[u] = 0.f;
   float ent = 0.f;
-  for (int j = warp; j < n_rows; j += kRtWarps) {
-    const int i = i0 + j;
-    float* row = s_log + i * p.pitch;
-    float sv[NS], pr[NS];
+  // warp w takes tokens w, w + 16, w + 32, ... two at a time in lockstep
+  for (int j = warp; j < n_rows; j += 2 * kRtWarps) {
+    const int jt[2] = {j, j + kRtWarps};
+    const bool has[2] = {true, j + kRtWarps < n_rows};
+    int tk[2];
+    float sv[2][NS], pr[2][NS];
 #pragma unroll
-    for (int u = 0; u < NS; ++u) {
-      const int e = lane + 32 * u;
-      sv[u] = e < E ? row[e] : -INFINITY;
+    for (int t = 0; t < 2; ++t) {
+      tk[t] = m0 + i0 + jt[t];
+      const float* row = s_log + (i0 + (has[t] ? jt[t] : j)) * p.pitch;
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int e = lane + 32 * u;
+        sv[t][u] = e < E ? row[e] : -INFINITY;
+      }
     }
-    select_token<NS>(a, m0 + i, sv, imp, ent, pr, lane);
+    select_tokens<NS, 2>(a, tk, has, sv, imp, ent, pr, lane);
 #pragma unroll
-    for (int u = 0; u < NS; ++u) {
-      const int e = lane + 32 * u;
-      if (e < E) row[e] = pr[u];
+    for (int t = 0; t < 2; ++t) {
+      if (!has[t]) continue;
+      float* row = s_log + (i0 + jt[t]) * p.pitch;
+#pragma unroll
+      for (int u = 0; u < NS; ++u) {
+        const int e = lane + 32 * u;
+        if (e < E) row[e] = pr[t][u];
+      }
     }
   }
   ent = warp_sum(ent);
