@@ -1251,11 +1251,13 @@ GemmTile gemm_tile() {
   const int t = gemm_tile_env();
   return t < 0 ? TILE_256 : (GemmTile)t;
 }
-// Per call: groups of a few hundred rows at most (DeepSeek-V3: T k / E = 128 on average,
-// Switch: at most the capacity) fill a 256-row tile's second half only partly and leave each
-// tile a short main loop whose epilogue is not overlapped; 128-row tiles with two TMEM
-// accumulators measured faster there (V3 down projection 1.70 -> 1.61 ms).  Large groups
-// (Mixtral: 1024 rows per expert) keep the 256-row tiles.
+int sm_count() {
+  int dev = 0, n = 0;
+  cudaGetDevice(&dev);
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 // Weights-as-M schedule (gemm_swap.cu), taken for every eligible call when MOE_GEMM_SWAP=1
 // (unless MOE_GEMM_TILE names a row-tile shape).  Off by default: it measured slower than the
 // row tiles at the DeepSeek-V3 shape (up 2.94 against 2.51 ms, down 1.81 against 1.72 ms) and
@@ -1270,19 +1272,28 @@ bool use_swap(int epi, bool grouped, bool out2, bool adapt) {
   return on && grouped && !out2 && !adapt && swap_epilogue_ok(epi) && gemm_tile_env() < 0;
 }
 
-GemmTile tile_for(int64_t a_rows, int n_groups, bool grouped) {
+// Per call.  Groups of at most 192 rows on average (DeepSeek-V3: T k / E = 128, Switch: at most
+// the capacity) run 128-row tiles with two TMEM accumulators: they fill a 256-row tile's second
+// half only partly and give each tile a short main loop whose epilogue one accumulator set
+// cannot hide (V3 down projection 1.70 -> 1.61 ms).  Larger groups compare the two shapes by
+// whole waves of persistent CTAs: tiles ~ (a_rows / TBM + n_groups / 2) * nt (each group's last
+// tile counted as half full), a 128-row tile costing 0.6 of a 256-row one (half the rows, a
+// fifth more time per row: more L2 bytes per FLOP, measured).  The 256-row tiles keep every
+// Mixtral projection at T k >= 8192; the down projection (16 output tiles per group) takes the
+// 128-row tiles at 1024 and 2048 tokens, where 256-row tiles leave a mostly idle last wave
+// (measured: 365 -> 330 us and 531 -> 444 us).
+GemmTile tile_for(int64_t a_rows, int n_groups, bool grouped, int nt) {
   const int t = gemm_tile_env();
   if (t >= 0) return (GemmTile)t;
-  if (grouped && n_groups > 1 && a_rows / n_groups <= 192) return TILE_128;
-  return TILE_256;
+  if (!grouped || n_groups < 1) return TILE_256;
+  if (n_groups > 1 && a_rows / n_groups <= 192) return TILE_128;
+  const int64_t sms = sm_count();
+  const int64_t t256 = ((a_rows + 255) / 256 + n_groups / 2) * nt;
+  const int64_t t128 = ((a_rows + 127) / 128 + n_groups / 2) * nt;
+  const int64_t w256 = (t256 + sms - 1) / sms, w128 = (t128 + sms - 1) / sms;
+  return 6 * w128 < 10 * w256 ? TILE_128 : TILE_256;
 }
 
-int sm_count() {
-  int dev = 0, n = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
 
 template <int EPI, int HALVES, int KB, int NSTAGES>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
@@ -1442,7 +1453,7 @@ cudaError_t launch_grouped_gemm_bf16(int epi, const void* A, int64_t a_rows, int
   p.adapt_cap = adapt_cap;
   p.adapt_ks_max = adapt ? adapt_ks_max : 0;
   p.adapt_ks = adapt_ks;
-  GemmTile tile = tile_for(a_rows, n_groups, offsets != nullptr);
+  GemmTile tile = tile_for(a_rows, n_groups, offsets != nullptr, p.nt);
   if (adapt && tile == TILE_PAIR) tile = TILE_256;     // the pair kernel has no adaptive split
   const int halves = tile == TILE_128 ? 1 : 2;
   const int kb = tile == TILE_256_K32 ? 32 : 64;

@@ -188,6 +188,20 @@ def test_decode_regime_mixtral_shape(T):
     C.check_sampled_output(w, inp, out, v, list(range(T)))
 
 
+# mid-size batches at the full Mixtral layer shape: ~256 and ~512 rows per expert, where the
+# down projection takes the 128-row tiles (whole waves of CTAs) and the up projection the
+# 256-row tiles at 2048 tokens; routing bit-exact, a tile-stratified output sample
+@pytest.mark.parametrize("T", [1024, 2048])
+def test_mid_size_mixtral_shape(T):
+    w = scaled(W["mixtral"], T=T)
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    C.check_logits(w, inp, v)
+    C.check_routing(w, inp, v)
+    nrows, ntok, _, _ = C.check_stratified_output(w, inp, out, v, seed=125)
+    assert nrows > 0 and ntok > 0
+
+
 # A few executed rows (bf16) take the k-split expert schedule: fp32 partials of the up and down
 # products summed by splitk.cu.  ReLU at the full Switch layer with its capacity limit (up split
 # 3, down split 8) and GELU (splits 4 and 2); SwiGLU is covered by router_E8_T1 (up split 7)
