@@ -198,11 +198,16 @@ combine_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
 
 // K <= 2 and no shared experts (Mixtral, Switch): each lane keeps 4 chunks x K rows of loads in
 // flight before accumulating, so a warp has up to 4 KB outstanding.
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
 template <bool BF16, int K>
 __global__ void __launch_bounds__(kWarps * 32)
 combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ inv,
                        const float* __restrict__ gates, int T, int nvec,
-                       uint4* __restrict__ out, const StatsArgs sa) {
+                       uint4* __restrict__ out, const StatsArgs sa, const SplitRows sr) {
   pdl_trigger();
   pdl_wait();
   if (sa.st && blockIdx.x == 0) balance_stats_block(sa);
@@ -216,6 +221,39 @@ combine_small_k_kernel(const uint4* __restrict__ y, const int32_t* __restrict__ 
   for (int j = 0; j < K; ++j) {
     row[j] = inv[(int64_t)t * K + j];
     g[j] = row[j] >= 0 ? gates[(int64_t)t * K + j] : 0.f;
+  }
+  const int S = (BF16 && sr.part) ? __ldg(sr.ks) : 1;
+  if (BF16 && S > 1) {
+    // y rows from the k-split partials: the S partial values of 8 columns summed in split
+    // order, rounded once to bf16, stored to y and weighted into the output
+    const int64_t live = min((int64_t)__ldg(sr.n_rows), sr.rows);
+    const int64_t ncol = (int64_t)nvec * 8;
+    const int64_t stride = live * ncol;
+    uint4* yw = static_cast<uint4*>(sr.y);
+    for (int v = lane; v < nvec; v += 32) {
+      float acc[R::N];
+#pragma unroll
+      for (int i = 0; i < R::N; ++i) acc[i] = 0.f;
+#pragma unroll
+      for (int j = 0; j < K; ++j) {
+        if (row[j] < 0 || row[j] >= live) continue;
+        const float* pr = sr.part + (int64_t)row[j] * ncol + 8 * v;
+        float4 a0 = __ldcs(reinterpret_cast<const float4*>(pr));
+        float4 a1 = __ldcs(reinterpret_cast<const float4*>(pr + 4));
+        for (int sp = 1; sp < S; ++sp) {
+          const float4 b0 = __ldcs(reinterpret_cast<const float4*>(pr + sp * stride));
+          const float4 b1 = __ldcs(reinterpret_cast<const float4*>(pr + sp * stride + 4));
+          a0.x += b0.x; a0.y += b0.y; a0.z += b0.z; a0.w += b0.w;
+          a1.x += b1.x; a1.y += b1.y; a1.z += b1.z; a1.w += b1.w;
+        }
+        const uint4 yb = make_uint4(pack_bf16x2(a0.x, a0.y), pack_bf16x2(a0.z, a0.w),
+                                    pack_bf16x2(a1.x, a1.y), pack_bf16x2(a1.z, a1.w));
+        yw[(int64_t)row[j] * nvec + v] = yb;
+        R::acc_val(yb, g[j], acc);
+      }
+      R::store(out + (int64_t)t * nvec + v, acc);
+    }
+    return;
   }
   int v = lane;
   for (; v + 96 < nvec; v += 128) {
@@ -275,24 +313,38 @@ StatsArgs stats_args(const moe_desc_t& d, const int32_t* counts, const int32_t* 
 
 cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
                            const float* gates, const void* y_shared, void* out,
-                           cudaStream_t s, const StatsArgs* with_stats) {
+                           cudaStream_t s, const StatsArgs* with_stats,
+                           const SplitRows* split) {
   if (d.T == 0) return cudaSuccess;
   StatsArgs sa{};
   if (with_stats) sa = *with_stats;
+  SplitRows sr{};
+  const bool small_k = !y_shared && d.select == MOE_TOKEN_CHOICE && d.k <= 2;
+  if (split) {
+    if (small_k && d.dtype == MOE_BF16 && d.D % 8 == 0) {
+      sr = *split;
+      sr.y = const_cast<void*>(y);
+    } else {
+      // the general combine reads y: sum the partials into it first
+      cudaError_t e = launch_splitk_sum_adaptive(split->part, split->ks, split->rows, d.D,
+                                                 split->n_rows, const_cast<void*>(y), s);
+      if (e != cudaSuccess) return e;
+    }
+  }
   const int K = (d.select == MOE_EXPERT_CHOICE) ? d.E : d.k;
   const int esz = (d.dtype == MOE_BF16) ? 2 : 4;
   const int nvec = d.D * esz / 16;
   const int S = y_shared ? d.n_shared : 0;
   const int blocks = (d.T + kWarps - 1) / kWarps;
-  if (S == 0 && d.select == MOE_TOKEN_CHOICE && d.k <= 2) {
+  if (small_k) {
     const uint4* yy = static_cast<const uint4*>(y);
     uint4* oo = static_cast<uint4*>(out);
     if (d.dtype == MOE_BF16) {
-      if (K == 1) (void)launch_pdl(combine_small_k_kernel<true, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
-      else (void)launch_pdl(combine_small_k_kernel<true, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<true, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa, sr);
+      else (void)launch_pdl(combine_small_k_kernel<true, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa, sr);
     } else {
-      if (K == 1) (void)launch_pdl(combine_small_k_kernel<false, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
-      else (void)launch_pdl(combine_small_k_kernel<false, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa);
+      if (K == 1) (void)launch_pdl(combine_small_k_kernel<false, 1>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa, sr);
+      else (void)launch_pdl(combine_small_k_kernel<false, 2>, dim3(blocks), dim3(kWarps * 32), 0, s, yy, inv, gates, d.T, nvec, oo, sa, sr);
     }
     return cudaGetLastError();
   }

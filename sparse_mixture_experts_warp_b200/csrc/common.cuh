@@ -237,11 +237,23 @@ struct StatsArgs {
 StatsArgs stats_args(const moe_desc_t& d, const int32_t* counts, const int32_t* offsets,
                      const float* importance, const float* entropy, float* f,
                      moe_stats_t* stats);
+// The down projection's adaptive k-split left unsummed: fp32 partials [*ks][live][D] at part
+// (live = min(*n_rows, rows)); when *ks <= 1 the product wrote y itself.
+struct SplitRows {
+  const float* part;
+  const int* ks;
+  const int32_t* n_rows;
+  int64_t rows;
+  void* y;          // [rows, D] bf16, filled by launch_combine
+};
 // with_stats: block 0 of the combine also computes the balance statistics (the layer step's
-// last two stages in one launch; every input of the statistics was written by earlier kernels)
+// last two stages in one launch; every input of the statistics was written by earlier kernels).
+// split: the combine first forms each kept row of y from the partials (the sum and bf16
+// rounding of launch_splitk_sum_adaptive, in split order), writes it to y and uses it.
 cudaError_t launch_combine(const moe_desc_t& d, const void* y, const int32_t* inv,
                            const float* gates, const void* y_shared, void* out,
-                           cudaStream_t s, const StatsArgs* with_stats = nullptr);
+                           cudaStream_t s, const StatsArgs* with_stats = nullptr,
+                           const SplitRows* split = nullptr);
 cudaError_t launch_balance_stats(const moe_desc_t& d, const int32_t* counts,
                                  const int32_t* offsets, const float* importance,
                                  const float* entropy, float* f, moe_stats_t* stats,

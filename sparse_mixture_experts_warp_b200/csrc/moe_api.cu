@@ -555,10 +555,25 @@ moe_status_t moe_expert_up_ws(const moe_desc_t* d, int32_t G, int32_t F, const v
   return cuda_status(e);
 }
 
+// defer != nullptr: when the device-side k-split runs, its partials are left for the combine
+// (described in *defer; defer->part stays null otherwise).
+static moe_status_t down_ws_impl(const moe_desc_t* d, int32_t G, int32_t F, const void* h,
+                                 int64_t a_rows, const int32_t* offsets, const void* W_down,
+                                 void* y, void* scratch, size_t scratch_bytes,
+                                 moe_stream_t stream, SplitRows* defer);
+
 moe_status_t moe_expert_down_ws(const moe_desc_t* d, int32_t G, int32_t F, const void* h,
                                 int64_t a_rows, const int32_t* offsets, const void* W_down,
                                 void* y, void* scratch, size_t scratch_bytes,
                                 moe_stream_t stream) {
+  return down_ws_impl(d, G, F, h, a_rows, offsets, W_down, y, scratch, scratch_bytes, stream,
+                      nullptr);
+}
+
+static moe_status_t down_ws_impl(const moe_desc_t* d, int32_t G, int32_t F, const void* h,
+                                 int64_t a_rows, const int32_t* offsets, const void* W_down,
+                                 void* y, void* scratch, size_t scratch_bytes,
+                                 moe_stream_t stream, SplitRows* defer) {
   moe_status_t st = check_ffn(d, G, F, h, a_rows, offsets);
   if (st != MOE_OK) return st;
   int S = 1;
@@ -580,6 +595,10 @@ moe_status_t moe_expert_down_ws(const moe_desc_t* d, int32_t G, int32_t F, const
       cudaError_t e = launch_grouped_gemm_bf16(EPI_NONE, h, a_rows, F, W_down, nullptr, G, d->D,
                                                offsets, y, s, nullptr, nullptr, 1, 0, ap,
                                                (int64_t)(pb / sizeof(float)), kMaxSplits, ks);
+      if (e == cudaSuccess && defer) {
+        *defer = SplitRows{ap, ks, offsets + G, a_rows, nullptr};
+        return MOE_OK;
+      }
       if (e == cudaSuccess) e = launch_splitk_sum_adaptive(ap, ks, a_rows, d->D, offsets + G, y, s);
       return cuda_status(e);
     }
@@ -654,12 +673,16 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
   st = moe_permute(d, v.expert_ids, x, gather ? nullptr : v.x_perm, v.counts, v.offsets,
                    v.row_src, v.inv, v.scratch, v.scratch_bytes, stream);
   if (st != MOE_OK) return st;
+  // without shared experts the combine sums a device-side k-split of the down projection
+  // itself (one launch fewer)
+  SplitRows split{};
+  SplitRows* defer = d->n_shared == 0 ? &split : nullptr;
   if (gather) {
     st = moe_expert_up_gather(d, d->E, d->F, x, v.row_src, v.rows, v.offsets, W_gate, W_up, v.h,
                               stream);
     if (st == MOE_OK)
-      st = moe_expert_down_ws(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
-                              v.scratch_bytes, stream);
+      st = down_ws_impl(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
+                        v.scratch_bytes, stream, defer);
   } else if (preact) {
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     const bool glu = d->act == MOE_ACT_SWIGLU;
@@ -674,8 +697,8 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
     st = moe_expert_up_ws(d, d->E, d->F, v.x_perm, v.rows, v.offsets, W_gate, W_up, v.h,
                           v.scratch, v.scratch_bytes, stream);
     if (st == MOE_OK)
-      st = moe_expert_down_ws(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
-                              v.scratch_bytes, stream);
+      st = down_ws_impl(d, d->E, d->F, v.h, v.rows, v.offsets, W_down, v.y, v.scratch,
+                        v.scratch_bytes, stream, defer);
   }
   if (st != MOE_OK) return st;
   if (d->n_shared > 0) {
@@ -703,7 +726,8 @@ static moe_status_t forward_impl(const moe_desc_t* d, const void* x, const void*
   const StatsArgs sa = stats_args(*d, v.counts, v.offsets, v.importance, v.entropy, v.f, v.stats);
   return cuda_status(launch_combine(*d, v.y, v.inv, v.gates,
                                     d->n_shared > 0 ? v.y_shared : nullptr, out,
-                                    reinterpret_cast<cudaStream_t>(stream), &sa));
+                                    reinterpret_cast<cudaStream_t>(stream), &sa,
+                                    split.part ? &split : nullptr));
 }
 
 // ---------------- backward ----------------

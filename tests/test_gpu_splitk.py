@@ -109,3 +109,27 @@ def test_ws_with_many_rows_runs_the_fused_products():
                        v["scratch"])
     torch.cuda.synchronize()
     assert torch.equal(h0, h1)
+
+
+@pytest.mark.parametrize("name", ["switch_full", "switch_small_k2"])
+def test_layer_combine_sums_the_adaptive_split(name):
+    """Under a capacity limit the down projection may split K on the device (fp32 partials);
+    moe_layer_forward then lets the combine sum each kept row's partials (split order, one bf16
+    rounding), write it to y and weight it, instead of a separate summing launch.  y and the
+    layer output equal, bit for bit, those of the step entry points (moe_expert_down_ws sums
+    with its own kernel, moe_combine reads y)."""
+    w = {"switch_full": WORKLOADS["switch"],
+         "switch_small_k2": scaled(WORKLOADS["switch"], T=3000, D=256, E=16, F=512, k=2)}[name]
+    inp = C.inputs_for(w)
+    out, v = C.run_layer(w, inp)
+    d = M.desc_of(w)
+    n = int(v["offsets"][w.E].item())
+    assert n > 0
+    y1 = torch.zeros_like(v["y"])
+    M.moe_expert_down_ws(d, w.E, w.F, v["h"], v["offsets"], inp.W_down, y1, v["scratch"])
+    out1 = torch.empty_like(out)
+    M.moe_combine(d, y1, v["inv"], v["gates"], None, out1)
+    torch.cuda.synchronize()
+    assert M.get_device_error() == 0
+    assert torch.equal(y1[:n], v["y"][:n])
+    assert torch.equal(out1, out)
