@@ -300,7 +300,10 @@ moe_status_t moe_balance_stats(const moe_desc_t* desc, const int32_t* counts,
  * enqueued on one stream with no host synchronisation.  Intermediates live in `ws`
  * (moe_workspace_size bytes); moe_layer_views gives their addresses.  The last two steps run
  * as one launch (the combine's first block computes the statistics); f and the moe_stats_t in
- * `ws` equal, bit for bit, what moe_balance_stats computes from the same views.
+ * `ws` equal, bit for bit, what moe_balance_stats computes from the same views.  When the down
+ * projection splits K on the device (moe_expert_down_ws) and the layer has no shared experts
+ * and k <= 2, the combine sums the split partials into y itself; y and out are the same, bit
+ * for bit, as with the separate summing pass.
  *   x [T,D], Wg [E,D], sel_bias [E] or NULL, routed weights as above, shared weights
  *   [S,Fs,D], [S,Fs,D], [S,D,Fs] (NULL when S = 0), out [T,D]. */
 moe_status_t moe_layer_forward(const moe_desc_t* desc, const void* x, const void* Wg,
