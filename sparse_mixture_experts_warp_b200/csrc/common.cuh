@@ -237,8 +237,8 @@ struct StatsArgs {
 StatsArgs stats_args(const moe_desc_t& d, const int32_t* counts, const int32_t* offsets,
                      const float* importance, const float* entropy, float* f,
                      moe_stats_t* stats);
-// The down projection's adaptive k-split left unsummed: fp32 partials [*ks][live][D] at part
-// (live = min(*n_rows, rows)); when *ks <= 1 the product wrote y itself.
+// The down projection's device-side k-split left unsummed: fp32 partials [*ks][live][D] at
+// part (live = min(*n_rows, rows)); when *ks <= 1 the product wrote y itself.
 struct SplitRows {
   const float* part;
   const int* ks;

@@ -606,6 +606,9 @@ static moe_status_t down_ws_impl(const moe_desc_t* d, int32_t G, int32_t F, cons
   if (!part) return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
   cudaError_t e = launch_grouped_gemm_f32_splitk(h, a_rows, F, W_down, G, d->D, offsets, S, part,
                                                  s);
+  // (the decode split keeps its own summing kernel: with a handful of tokens the combine is a
+  // warp or two, and the sum needs the whole GPU's loads in flight; measured at one token:
+  // 0.160 against 0.183 ms with the sum inside the combine)
   if (e == cudaSuccess) e = launch_splitk_sum(part, S, a_rows, d->D, offsets + G, y, s);
   return cuda_status(e);
 }

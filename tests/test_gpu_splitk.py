@@ -111,15 +111,17 @@ def test_ws_with_many_rows_runs_the_fused_products():
     assert torch.equal(h0, h1)
 
 
-@pytest.mark.parametrize("name", ["switch_full", "switch_small_k2"])
-def test_layer_combine_sums_the_adaptive_split(name):
+@pytest.mark.parametrize("name", ["switch_full", "switch_small_k2", "swiglu_T1", "relu_T2"])
+def test_layer_combine_sums_the_down_split(name):
     """Under a capacity limit the down projection may split K on the device (fp32 partials);
     moe_layer_forward then lets the combine sum each kept row's partials (split order, one bf16
-    rounding), write it to y and weight it, instead of a separate summing launch.  y and the
-    layer output equal, bit for bit, those of the step entry points (moe_expert_down_ws sums
-    with its own kernel, moe_combine reads y)."""
+    rounding), write it to y and weight it, instead of a separate summing launch (the decode
+    cases keep the summing kernel of their host-side split).  Either way y and the layer output
+    equal, bit for bit, those of the step entry points (moe_expert_down_ws sums with its own
+    kernel, moe_combine reads y)."""
     w = {"switch_full": WORKLOADS["switch"],
-         "switch_small_k2": scaled(WORKLOADS["switch"], T=3000, D=256, E=16, F=512, k=2)}[name]
+         "switch_small_k2": scaled(WORKLOADS["switch"], T=3000, D=256, E=16, F=512, k=2),
+         **CASES}[name]
     inp = C.inputs_for(w)
     out, v = C.run_layer(w, inp)
     d = M.desc_of(w)
