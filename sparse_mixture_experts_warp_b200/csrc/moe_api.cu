@@ -534,8 +534,16 @@ moe_status_t moe_expert_up_ws(const moe_desc_t* d, int32_t G, int32_t F, const v
     const int64_t fused = active * ((F + (glu ? 127 : 255)) / (glu ? 128 : 256));
     const int64_t units = active * ((F + 255) / 256) * (glu ? 2 : 1);
     const double fill_fused = sm_fill(fused, sms);
-    const int c = choose_splits(units, d->D, sms);
-    if (c > 1 && fill_fused < 0.8 && sm_fill(units * c, sms) > fill_fused + 0.05) S = c;
+    if (units >= sms) {
+      // at least a full wave of split tiles already: two k-ranges when the fused product
+      // fills its last wave poorly.  Fewer, longer weight streams per tile measured faster
+      // than the fullest last wave (Mixtral width, gate + up: 1 token 0.165 -> 0.153 ms with
+      // 2 instead of 5 k-ranges, 2 tokens 0.293 -> 0.269 ms; 3 to 8 ranges all slower)
+      if (fill_fused < 0.8 && d->D / 64 >= 8) S = 2;
+    } else {
+      const int c = choose_splits(units, d->D, sms);
+      if (c > 1 && fill_fused < 0.8 && sm_fill(units * c, sms) > fill_fused + 0.05) S = c;
+    }
   }
   // partial rows: [gate | up] blocks of ceil(F / 256) * 256 columns each (SwiGLU), F otherwise
   const int64_t fpad = (int64_t)(F + 255) / 256 * 256;

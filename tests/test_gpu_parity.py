@@ -205,7 +205,7 @@ def test_mid_size_mixtral_shape(T):
 # A few executed rows (bf16) take the k-split expert schedule: fp32 partials of the up and down
 # products summed by splitk.cu.  ReLU at the full Switch layer with its capacity limit (up split
 # 3, down split 8) and GELU (splits 4 and 2); SwiGLU is covered by router_E8_T1 (up split 7)
-# and T = 1 above (up 5, down 4).  Every token against the oracle, which evaluates only the
+# and T = 1 above (up 2, down 4).  Every token against the oracle, which evaluates only the
 # experts in use.
 DECODE = {
     "switch_relu_T2": scaled(W["switch"], T=2),
