@@ -298,14 +298,16 @@ __device__ __forceinline__ void umma_commit_pair_local(uint64_t* bar) {
 //             8 epilogue warps; a tile with <= 128 live rows loads and multiplies one half only.
 // tmB1 is the second B operand (SwiGLU, EPI_RAW, EPI_NONE_BMN) or, for EPI_F32_TMA, the fp32
 // output map: [groups][rows][N], boxes of 16 columns x 32 rows, 64-byte swizzle.
-template <int EPI, int HALVES, int KB, int NSTAGES>
+// RB: A rows per half (128; 64 for products of a few rows, whose 128-row boxes would be mostly
+// rows past the end: half the A bytes per stage, one more stage of weights in flight).
+template <int EPI, int HALVES, int KB, int NSTAGES, int RB = BM>
 __global__ void __launch_bounds__(64 + 128 * HALVES, 1)
 grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB0,
                     const __grid_constant__ CUtensorMap tmB1, const GemmParams p) {
-  constexpr int TBM = BM * HALVES;
+  constexpr int TBM = RB * HALVES;
   constexpr int TSTAGES = NSTAGES;
-  constexpr int HA_BYTES = BM * KB * 2;              // one 128-row half of A per stage
+  constexpr int HA_BYTES = RB * KB * 2;              // one half of A per stage
   constexpr int TA_BYTES = HALVES * HA_BYTES;
   constexpr int TB_BYTES = MMA_N * KB * 2;           // B per stage
   constexpr int NBUF = HALVES == 1 ? 2 : 1;          // TMEM accumulator buffers
@@ -443,8 +445,8 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const int a_row = (int)tl.row0 + tl.m_idx * TBM;
       const int row_end = (int)tl.row0 + tl.m;
       const int b_row = tl.g * p.N + tl.n_idx * p.n_out_tile;
-      const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
-      const bool mine = 8 * lane < (two ? 2 * BM : BM);
+      const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > RB;
+      const bool mine = 8 * lane < (two ? 2 * RB : RB);
       int src[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
@@ -511,7 +513,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
         const bool b1 = EPI == EPI_F32 && p.b1_nt > 0 && tl.n_idx >= p.b1_nt;
         const int b_row = (p.kgroup ? 0 : tl.g * p.N) +
                           (tl.n_idx - (b1 ? p.b1_nt : 0)) * p.n_out_tile;
-        const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > BM;
+        const bool two = HALVES == 2 && (tl.m - tl.m_idx * TBM) > RB;
         const int kb0 = tl.kb0, kb1 = tl.kb1;
         for (int kb = kb0; kb < kb1; ++kb) {
           const int kx = tl.kcol0 + kb * KB;
@@ -534,7 +536,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           }
           const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
           tma_load_2d(a_dst, &tmA, &full[stage], kx, a_row);
-          if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kx, a_row + BM);
+          if (two) tma_load_2d(a_dst + HA_BYTES, &tmA, &full[stage], kx, a_row + RB);
           if (EPI == EPI_NONE_BMN) {
             // [K, N] boxes of 64 x 64: four N blocks of 64 for this k-block
             const bool hi = kb >= p.kb_split;
@@ -578,10 +580,10 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x, ++it) {
         const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
         const int m = tl.m, m_idx = tl.m_idx;
-        const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
+        const bool two = HALVES == 2 && (m - m_idx * TBM) > RB;
         const int kb0 = tl.kb0, kb1 = tl.kb1;      // kb0 == kb1: an empty group along K
         // M = 64 for a half with at most 64 live rows
-        const int live0 = min(BM, m - m_idx * TBM), live1 = min(BM, m - m_idx * TBM - BM);
+        const int live0 = min(RB, m - m_idx * TBM), live1 = min(RB, m - m_idx * TBM - RB);
         // MN-major B: the transpose-B bit (16) of the instruction descriptor
         const uint32_t bmaj = EPI == EPI_NONE_BMN ? (1u << 16) : 0u;
         const uint32_t idesc0 = (live0 <= 64 ? kIdesc64 : kIdesc) | bmaj;
@@ -637,7 +639,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
       const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
       const bool zero = tl.kb1 <= tl.kb0;    // no k-blocks (empty group along K): the sum is 0
-      const bool two = HALVES == 2 && (m - m_idx * TBM) > BM;
+      const bool two = HALVES == 2 && (m - m_idx * TBM) > RB;
       const int acc = it % NBUF;
       const uint32_t acc_par = (uint32_t)(it / NBUF) & 1u;
       int okw = 1;
@@ -653,9 +655,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       }
       // rows of this half: M = 128 -> lane quarter q holds rows 32q + lane; M = 64 (at most 64
       // live rows) -> rows 16q + lane in the quarter's first 16 lanes
-      const int live = min(BM, m - m_idx * TBM - half * BM);
+      const int live = min(RB, m - m_idx * TBM - half * RB);
       const bool m64 = live <= 64;
-      const int row = half * BM + (m64 ? 16 * q + lane : 32 * q + lane);
+      const int row = half * RB + (m64 ? 16 * q + lane : 32 * q + lane);
       const int r = m_idx * TBM + row;
       const int64_t orow = tl.row0 + r;
       bool valid = r < m && (!m64 || lane < 16);
@@ -770,7 +772,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
               fence_proxy_async_smem();
               __syncwarp();
               if (lane == 0) {
-                tma_store_3d(&tmB1, buf, col + 16 * h, m_idx * TBM + half * BM + 32 * q, tl.g);
+                tma_store_3d(&tmB1, buf, col + 16 * h, m_idx * TBM + half * RB + 32 * q, tl.g);
                 bulk_commit();
               }
               ++nstored;
@@ -1295,10 +1297,10 @@ GemmTile tile_for(int64_t a_rows, int n_groups, bool grouped, int nt) {
 }
 
 
-template <int EPI, int HALVES, int KB, int NSTAGES>
+template <int EPI, int HALVES, int KB, int NSTAGES, int RB = BM>
 cudaError_t launch_epi(const CUtensorMap& a, const CUtensorMap& b0, const CUtensorMap& b1,
                        const GemmParams& p, int grid, size_t smem, cudaStream_t s) {
-  auto kern = grouped_gemm_kernel<EPI, HALVES, KB, NSTAGES>;
+  auto kern = grouped_gemm_kernel<EPI, HALVES, KB, NSTAGES, RB>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
@@ -1323,8 +1325,9 @@ cudaError_t launch_cfg(int epi, const CUtensorMap& a, const CUtensorMap& b0,
 
 // Dynamic shared memory of one configuration (ring + barriers + group tables + alignment).
 // `staging`: the EPI_F32_TMA store buffers between the ring and the barriers.
-size_t gemm_smem(int halves, int kb, int nstages, int n_groups, size_t staging = 0) {
-  const size_t ring = (size_t)nstages * ((size_t)halves * BM * kb * 2 + (size_t)MMA_N * kb * 2);
+size_t gemm_smem(int halves, int kb, int nstages, int n_groups, size_t staging = 0,
+                 int rb = BM) {
+  const size_t ring = (size_t)nstages * ((size_t)halves * rb * kb * 2 + (size_t)MMA_N * kb * 2);
   return 1024 + ring + staging + (2 * nstages + 5) * 8 + 8 +
          (size_t)2 * (n_groups + 1) * sizeof(int);
 }
@@ -1613,12 +1616,19 @@ cudaError_t launch_grouped_gemm_kgroups_f32(const void* A, int M, const void* B,
 // the k-blocks of split s of A[r, k] * B[g * N + n, k] for every row r of group g; split s
 // covers k-blocks [s * kchunk, (s + 1) * kchunk), every split non-empty.  out is
 // [ksplit][a_rows][N] fp32; only rows below offsets[G] are written.
+// A rows per tile of the k-split products: with at most 64 rows in all (the decode schedule
+// at up to 32 tokens of top-2), 64-row A boxes and a 5-stage ring (40 KB stages: 160 KB of
+// weights in flight per SM instead of 128 KB with 128-row boxes, which are then mostly rows
+// past the end that TMA fills without a memory access); otherwise 128 rows, 4 stages.
+static int split_rows(int64_t a_rows) { return a_rows <= 64 ? 64 : BM; }
+
 cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
                                            int G, int N, const int32_t* offsets, int ksplit,
                                            float* out, cudaStream_t s) {
   if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
   alignas(64) CUtensorMap ta, tb;
-  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  const int rb = split_rows(a_rows);
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, rb, 64)) return cudaErrorInvalidValue;
   if (!make_map(&tb, B, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
   GemmParams p{};
   p.offsets = offsets;
@@ -1642,8 +1652,11 @@ cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K,
   p.ldo2 = 0;
   p.kb_split = 0;
   p.bk_group = 0;
-  const int64_t tiles = ((a_rows + BM - 1) / BM + G) * (int64_t)p.nt * p.ksplit;
+  const int64_t tiles = ((a_rows + rb - 1) / rb + G) * (int64_t)p.nt * p.ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (rb == 64)
+    return launch_epi<EPI_F32, 1, 64, 5, 64>(ta, tb, tb, p, grid,
+                                             gemm_smem(1, 64, 5, G, 0, 64), s);
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb, tb, p, grid, gemm_smem(1, 64, 4, G), s);
 }
 
@@ -1653,7 +1666,8 @@ cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K
                                             cudaStream_t s) {
   if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
   alignas(64) CUtensorMap ta, tb0, tb1;
-  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
+  const int rb = split_rows(a_rows);
+  if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, rb, 64)) return cudaErrorInvalidValue;
   if (!make_map(&tb0, B0, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
   if (!make_map(&tb1, B1, (uint64_t)G * N, (uint64_t)K, 128, 64)) return cudaErrorInvalidValue;
   const int half = (N + 255) / 256;               // n-tiles of one product
@@ -1674,8 +1688,11 @@ cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K
   p.kchunk = (nkb + ksplit - 1) / ksplit;
   p.ksplit = splitk_count(K, ksplit);
   p.split_stride = a_rows * p.ldo;
-  const int64_t tiles = ((a_rows + BM - 1) / BM + G) * (int64_t)p.nt * p.ksplit;
+  const int64_t tiles = ((a_rows + rb - 1) / rb + G) * (int64_t)p.nt * p.ksplit;
   const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  if (rb == 64)
+    return launch_epi<EPI_F32, 1, 64, 5, 64>(ta, tb0, tb1, p, grid,
+                                             gemm_smem(1, 64, 5, G, 0, 64), s);
   return launch_epi<EPI_F32, 1, 64, 4>(ta, tb0, tb1, p, grid, gemm_smem(1, 64, 4, G), s);
 }
 
