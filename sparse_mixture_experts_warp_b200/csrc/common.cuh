@@ -63,6 +63,22 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 
+// ---- stream-K schedule of the fp32 k-split products (grouped GEMM and its summing kernel) ----
+// CTA c of g takes k-blocks [c * work / g, (c + 1) * work / g) of work = tiles * nkb (tile t
+// owns [t * nkb, (t + 1) * nkb)).  CTAs used: at most grid, and few enough that every range
+// holds ceil(nkb / (slots - 1)) k-blocks or more, so that a tile meets at most `slots` ranges.
+__host__ __device__ __forceinline__ int streamk_ctas(int64_t work, int nkb, int slots, int grid) {
+  if (work <= 0) return 0;
+  const int64_t minr = slots > 1 ? (nkb + slots - 2) / (slots - 1) : nkb;
+  int64_t g = work / (minr > 0 ? minr : 1);
+  if (g > grid) g = grid;
+  return g > 0 ? (int)g : 1;
+}
+// The CTA whose range holds k-block x.
+__host__ __device__ __forceinline__ int streamk_owner(int64_t x, int64_t work, int g) {
+  return (int)(((x + 1) * g - 1) / work);
+}
+
 // ---- launchers implemented in the .cu files (all enqueue on `s`, return the launch error) ----
 
 // route.cu
@@ -108,16 +124,20 @@ enum GemmEpilogue { EPI_SWIGLU = 0, EPI_RELU = 1, EPI_NONE = 2, EPI_F32 = 3, EPI
                     EPI_F32_TMA = 7 /* EPI_F32 written by TMA stores from shared memory */ };
 // k-split fp32 partials [ksplit][a_rows][N] of a grouped product (groups along M); the number
 // of non-empty splits is ceil(nkb / ceil(nkb / ksplit)) for nkb = ceil(K / 64).
+// sk_slots > 0 (a_rows <= 64): stream-K instead of ksplit equal k-ranges per tile: every CTA
+// takes an equal contiguous range of the tiles' k-blocks, and the part of a tile in CTA c's
+// range is written as partial slot c - (the tile's first CTA), at most sk_slots per tile
+// (launch_splitk_streamk sums them).
 cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
                                            int G, int N, const int32_t* offsets, int ksplit,
-                                           float* out, cudaStream_t s);
+                                           float* out, cudaStream_t s, int sk_slots = 0);
 // The same for two products that share A (the gate and up products of the decode schedule):
 // out[split][row][ldo] with ldo = 2 * ceil(N / 256) * 256, B0's product in columns
 // [0, N) and B1's from column ldo / 2.
 cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K, const void* B0,
                                             const void* B1, int G, int N,
                                             const int32_t* offsets, int ksplit, float* out,
-                                            cudaStream_t s);
+                                            cudaStream_t s, int sk_slots = 0);
 int gemm_sm_count();
 int splitk_count(int K, int ksplit);   // non-empty splits of K (64-element k-blocks)
 // splitk.cu: the sums of k-split partials of the small-batch schedule (rows below *n_rows)
@@ -128,6 +148,15 @@ cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S,
                               cudaStream_t s, int64_t ld = 0);
 cudaError_t launch_splitk_sum(const float* p, int S, int64_t rows, int N,
                               const int32_t* n_rows, void* y, cudaStream_t s);
+// The sums of a stream-K product (launch_grouped_gemm_f32_splitk[2] with sk_slots, over the
+// grid of gemm_sm_count() CTAs, groups of at most 64 rows): out[r, c] = act(sum over the
+// segments of c's tile, in slot order) for the rows r < offsets[G].  Partials [slots][rows][ld];
+// two = 1: gate columns at [0, N), up columns at ld / 2 (the two-product layout, n-tiles of the
+// up product from ceil(N / 256)), else one product of ceil(N / 256) n-tiles.  act: MOE_ACT_* or
+// -1 (no activation: the down projection).
+cudaError_t launch_splitk_streamk(int act, const float* part, int slots, int64_t rows, int ld,
+                                  int N, int K, int two, const int32_t* offsets, int G,
+                                  void* out, cudaStream_t s);
 // y[r, n] = sum over *ks splits of P[s][r][n] (split stride *n_rows * N) for r < *n_rows; does
 // nothing when *ks == 1 (the product wrote y itself).  rows bounds *n_rows (grid sizing).
 cudaError_t launch_splitk_sum_adaptive(const float* p, const int* ks, int64_t rows, int N,

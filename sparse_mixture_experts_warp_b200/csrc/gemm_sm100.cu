@@ -127,7 +127,23 @@ struct GemmParams {
   // EPI_F32 with two B tensors: n-tiles from b1_nt on read tmB1 (rows of n-tile n - b1_nt), so
   // one launch computes both the gate and the up product (0: one B tensor)
   int b1_nt;
+  // stream-K (EPI_F32, groups along M): the tiles' k-blocks, tile by tile, are cut into equal
+  // contiguous ranges, one per CTA; the part of a tile in CTA c's range is the tile's segment
+  // c - (first CTA of the tile), written as fp32 partial slot `segment` (split_stride apart).
+  // At most sk_slots segments per tile: the CTAs used are limited so that every range holds
+  // at least ceil(nkb / (sk_slots - 1)) k-blocks.
+  int streamk;
+  int sk_slots;
 };
+
+// This CTA's stream-K range of k-blocks [lo, hi) of work = tiles * nkb, over g CTAs.
+struct SkRange {
+  bool on;
+  int64_t lo, hi, work;
+  int g;
+};
+
+
 
 // One work item of the persistent schedule.
 struct Tile {
@@ -164,6 +180,30 @@ __device__ __forceinline__ Tile locate(int t, int total, int nkb, int kchunk, co
   r.n_idx = local / mt;
   r.m_idx = local - r.n_idx * mt;
   return r;
+}
+
+// Work item j of this CTA: the tile t = blockIdx.x + j * gridDim.x of the round-robin schedule,
+// or under stream-K the j-th tile its range touches, with that segment's k-blocks and slot.
+template <int TBM, int KB>
+__device__ __forceinline__ bool item_tile(int j, const SkRange& sk, int total_all, int total,
+                                          int nkb, int kchunk, const GemmParams& p,
+                                          const int* grp_off, const int* tile_pre, int& g,
+                                          Tile& tl) {
+  if (!sk.on) {
+    const int t = (int)blockIdx.x + j * (int)gridDim.x;
+    if (t >= total_all) return false;
+    tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
+    return true;
+  }
+  if (sk.hi <= sk.lo) return false;
+  const int t = (int)(sk.lo / nkb) + j;
+  if (t > (int)((sk.hi - 1) / nkb)) return false;
+  tl = locate<TBM, KB>(t, total, nkb, nkb, p, grp_off, tile_pre, g);
+  const int64_t base = (int64_t)t * nkb;
+  tl.kb0 = (int)((sk.lo > base ? sk.lo : base) - base);
+  tl.kb1 = (int)((sk.hi < base + nkb ? sk.hi : base + nkb) - base);
+  tl.split = (int)blockIdx.x - streamk_owner(base, sk.work, sk.g);
+  return true;
 }
 
 // Shared -> global tile store through a 3-D tensor map (x = column, y = row, z = group); the
@@ -428,6 +468,16 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
   }
   const bool adapt_f32 = EPI == EPI_NONE && ksplit > 1;
   const int total_all = total * ksplit;            // k-splits are the slowest tile index
+  SkRange sk{false, 0, 0, 0, 0};
+  if (EPI == EPI_F32 && p.streamk) {
+    sk.on = true;
+    sk.work = (int64_t)total * nkb;
+    sk.g = streamk_ctas(sk.work, nkb, p.sk_slots, (int)gridDim.x);
+    if ((int)blockIdx.x < sk.g) {
+      sk.lo = (int64_t)blockIdx.x * sk.work / sk.g;
+      sk.hi = (int64_t)(blockIdx.x + 1) * sk.work / sk.g;
+    }
+  }
 
   if (warp == 0 && p.gather_src) {
     // ---------------- TMA producer, gathered rows of A ----------------
@@ -440,8 +490,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     uint32_t issued = 0, issued_par = 0;
     bool ok = true;
     int g = 0;
-    for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-      const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
+    Tile tl;
+    for (int j = 0; ok && item_tile<TBM, KB>(j, sk, total_all, total, nkb, kchunk, p, grp_off,
+                                            tile_pre, g, tl); ++j) {
       const int a_row = (int)tl.row0 + tl.m_idx * TBM;
       const int row_end = (int)tl.row0 + tl.m;
       const int b_row = tl.g * p.N + tl.n_idx * p.n_out_tile;
@@ -466,7 +517,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
           ok = false;
           break;
         }
-        const bool withhold = p.fault == 1 && blockIdx.x == 0 && t == (int)blockIdx.x &&
+        const bool withhold = p.fault == 1 && blockIdx.x == 0 && j == 0 &&
                               kb == tl.kb0;     // test hook, as in the tiled producer below
         const uint32_t a_dst = sA + stage * TA_BYTES, b_dst = sB + stage * TB_BYTES;
         if (mine && !withhold) {
@@ -507,8 +558,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t issued = 0, issued_par = 0;     // per stage: has a load, parity of the last one
       bool ok = true;
       int g = 0;
-      for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x) {
-        const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
+      Tile tl;
+      for (int j = 0; ok && item_tile<TBM, KB>(j, sk, total_all, total, nkb, kchunk, p, grp_off,
+                                              tile_pre, g, tl); ++j) {
         const int a_row = (int)tl.row0 + tl.m_idx * TBM;
         const bool b1 = EPI == EPI_F32 && p.b1_nt > 0 && tl.n_idx >= p.b1_nt;
         const int b_row = (p.kgroup ? 0 : tl.g * p.N) +
@@ -523,7 +575,7 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
             break;
           }
           mbar_expect_tx(&full[stage], (two ? 2 * HA_BYTES : HA_BYTES) + TB_BYTES);
-          if (p.fault == 1 && blockIdx.x == 0 && t == (int)blockIdx.x && kb == kb0) {
+          if (p.fault == 1 && blockIdx.x == 0 && j == 0 && kb == kb0) {
             // test hook: the stage is armed but never loaded, so the MMA issuer's bounded
             // wait on it runs out; nothing is in flight for this stage
             issued |= 1u << stage;
@@ -577,8 +629,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
       uint32_t phase = 0;
       bool ok = true;
       int it = 0, g = 0;
-      for (int t = blockIdx.x; t < total_all && ok; t += gridDim.x, ++it) {
-        const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
+      Tile tl;
+      for (int j = 0; ok && item_tile<TBM, KB>(j, sk, total_all, total, nkb, kchunk, p, grp_off,
+                                              tile_pre, g, tl); ++j, ++it) {
         const int m = tl.m, m_idx = tl.m_idx;
         const bool two = HALVES == 2 && (m - m_idx * TBM) > RB;
         const int kb0 = tl.kb0, kb1 = tl.kb1;      // kb0 == kb1: an empty group along K
@@ -635,8 +688,9 @@ grouped_gemm_kernel(const __grid_constant__ CUtensorMap tmA,
     const int half = (warp - 2) / 4;         // which 128-row half of the tile
     int g = 0, it = 0;
     uint32_t nstored = 0;                    // EPI_F32_TMA: staged blocks this warp has stored
-    for (int t = blockIdx.x; t < total_all; t += gridDim.x, ++it) {
-      const Tile tl = locate<TBM, KB>(t, total, nkb, kchunk, p, grp_off, tile_pre, g);
+    Tile tl;
+    for (int j = 0; item_tile<TBM, KB>(j, sk, total_all, total, nkb, kchunk, p, grp_off, tile_pre,
+                                       g, tl); ++j, ++it) {
       const int m = tl.m, n_idx = tl.n_idx, m_idx = tl.m_idx, split = tl.split;
       const bool zero = tl.kb1 <= tl.kb0;    // no k-blocks (empty group along K): the sum is 0
       const bool two = HALVES == 2 && (m - m_idx * TBM) > RB;
@@ -1624,8 +1678,9 @@ static int split_rows(int64_t a_rows) { return a_rows <= 64 ? 64 : BM; }
 
 cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K, const void* B,
                                            int G, int N, const int32_t* offsets, int ksplit,
-                                           float* out, cudaStream_t s) {
+                                           float* out, cudaStream_t s, int sk_slots) {
   if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
+  if (sk_slots > 0 && (split_rows(a_rows) != 64 || sk_slots < 2)) return cudaErrorInvalidValue;
   alignas(64) CUtensorMap ta, tb;
   const int rb = split_rows(a_rows);
   if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, rb, 64)) return cudaErrorInvalidValue;
@@ -1652,8 +1707,10 @@ cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K,
   p.ldo2 = 0;
   p.kb_split = 0;
   p.bk_group = 0;
+  p.streamk = sk_slots > 0;
+  p.sk_slots = sk_slots;
   const int64_t tiles = ((a_rows + rb - 1) / rb + G) * (int64_t)p.nt * p.ksplit;
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  const int grid = p.streamk ? sm_count() : (int)(tiles < sm_count() ? tiles : sm_count());
   if (rb == 64)
     return launch_epi<EPI_F32, 1, 64, 5, 64>(ta, tb, tb, p, grid,
                                              gemm_smem(1, 64, 5, G, 0, 64), s);
@@ -1663,8 +1720,9 @@ cudaError_t launch_grouped_gemm_f32_splitk(const void* A, int64_t a_rows, int K,
 cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K, const void* B0,
                                             const void* B1, int G, int N,
                                             const int32_t* offsets, int ksplit, float* out,
-                                            cudaStream_t s) {
+                                            cudaStream_t s, int sk_slots) {
   if (a_rows <= 0 || G <= 0 || N <= 0 || ksplit < 1) return cudaSuccess;
+  if (sk_slots > 0 && (split_rows(a_rows) != 64 || sk_slots < 2)) return cudaErrorInvalidValue;
   alignas(64) CUtensorMap ta, tb0, tb1;
   const int rb = split_rows(a_rows);
   if (!make_map(&ta, A, (uint64_t)a_rows, (uint64_t)K, rb, 64)) return cudaErrorInvalidValue;
@@ -1688,8 +1746,10 @@ cudaError_t launch_grouped_gemm_f32_splitk2(const void* A, int64_t a_rows, int K
   p.kchunk = (nkb + ksplit - 1) / ksplit;
   p.ksplit = splitk_count(K, ksplit);
   p.split_stride = a_rows * p.ldo;
+  p.streamk = sk_slots > 0;
+  p.sk_slots = sk_slots;
   const int64_t tiles = ((a_rows + rb - 1) / rb + G) * (int64_t)p.nt * p.ksplit;
-  const int grid = (int)(tiles < sm_count() ? tiles : sm_count());
+  const int grid = p.streamk ? sm_count() : (int)(tiles < sm_count() ? tiles : sm_count());
   if (rb == 64)
     return launch_epi<EPI_F32, 1, 64, 5, 64>(ta, tb0, tb1, p, grid,
                                              gemm_smem(1, 64, 5, G, 0, 64), s);

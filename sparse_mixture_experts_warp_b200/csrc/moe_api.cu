@@ -132,6 +132,23 @@ bool decode_splitk_enabled() {
   return v;
 }
 
+// With at most kStreamKRows rows (64-row tiles: one per group) a split product whose S equal
+// k-ranges per tile would take more than one wave of CTAs runs stream-K instead: every SM takes
+// an equal contiguous share of all tiles' k-blocks, so no partly filled last wave leaves SMs
+// idle; up to kMaxSplits partial slots per tile.  Mixtral width, one token: gate + up 94 -> 87
+// us (448 equal ranges over 148 SMs before); the down product (128 ranges, one wave) keeps its
+// equal ranges (stream-K measured 49 -> 51 us there).  MOE_STREAMK=0 keeps the equal ranges
+// everywhere (comparison measurements).
+constexpr int64_t kStreamKRows = 64;
+constexpr int kStreamKGroups = 1024;
+bool streamk_enabled() {
+  static const bool v = [] {
+    const char* e = getenv("MOE_STREAMK");
+    return !(e && e[0] == '0');
+  }();
+  return v;
+}
+
 // Adaptive k-split of the down projection.  Under a capacity limit the executed rows can be
 // far fewer than the host's bound (a few popular experts, each at its capacity: the Switch
 // layer runs 413 of 8192 possible rows on 9 of 128 experts), and the down projection's tiles
@@ -548,16 +565,28 @@ moe_status_t moe_expert_up_ws(const moe_desc_t* d, int32_t G, int32_t F, const v
   // partial rows: [gate | up] blocks of ceil(F / 256) * 256 columns each (SwiGLU), F otherwise
   const int64_t fpad = (int64_t)(F + 255) / 256 * 256;
   const int64_t ld = glu ? 2 * fpad : F;
-  float* part = S > 1 ? splitk_space(scratch, scratch_bytes, (size_t)S * a_rows * ld * sizeof(float))
+  // at most 64 rows, and S equal k-ranges per tile would take more than one wave of CTAs:
+  // stream-K over all SMs (every CTA an equal share of the tiles' k-blocks, up to kMaxSplits
+  // partial slots per tile), so that no partly filled last wave remains
+  const int64_t split_units =
+      (int64_t)(a_rows < G ? a_rows : G) * ((F + 255) / 256) * (glu ? 2 : 1);
+  const bool sk = S > 1 && streamk_enabled() && a_rows <= kStreamKRows && F % 4 == 0 &&
+                  G <= kStreamKGroups && split_units * S > gemm_sm_count();
+  const int slots = sk ? kMaxSplits : S;
+  float* part = S > 1 ? splitk_space(scratch, scratch_bytes,
+                                     (size_t)slots * a_rows * ld * sizeof(float))
                       : nullptr;
   if (!part)
     return moe_expert_up(d, G, F, a, a_rows, offsets, W_gate, W_up, h, stream);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   cudaError_t e = glu ? launch_grouped_gemm_f32_splitk2(a, a_rows, d->D, W_gate, W_up, G, F,
-                                                         offsets, S, part, s)
+                                                         offsets, S, part, s, sk ? slots : 0)
                       : launch_grouped_gemm_f32_splitk(a, a_rows, d->D, W_up, G, F, offsets, S,
-                                                       part, s);
-  if (e == cudaSuccess)
+                                                       part, s, sk ? slots : 0);
+  if (e == cudaSuccess && sk)
+    e = launch_splitk_streamk(d->act, part, slots, a_rows, (int)ld, F, d->D, glu ? 1 : 0,
+                              offsets, G, h, s);
+  else if (e == cudaSuccess)
     e = launch_splitk_act(d->act, part, glu ? part + fpad : part, S, a_rows, F, offsets + G, h, s,
                           ld);
   return cuda_status(e);
@@ -590,8 +619,12 @@ static moe_status_t down_ws_impl(const moe_desc_t* d, int32_t G, int32_t F, cons
     const int64_t active = a_rows < G ? a_rows : G;
     S = choose_splits(active * ((d->D + 255) / 256), F, gemm_sm_count());
   }
+  const int64_t split_units = (int64_t)(a_rows < G ? a_rows : G) * ((d->D + 255) / 256);
+  const bool sk = S > 1 && streamk_enabled() && a_rows <= kStreamKRows && d->D % 4 == 0 &&
+                  G <= kStreamKGroups && split_units * S > gemm_sm_count();
+  const int slots = sk ? kMaxSplits : S;
   float* part = S > 1 ? splitk_space(scratch, scratch_bytes,
-                                     (size_t)S * a_rows * d->D * sizeof(float))
+                                     (size_t)slots * a_rows * d->D * sizeof(float))
                       : nullptr;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (!part && adaptive_down(d) && W_down && y && is_aligned16(W_down) && is_aligned16(y) &&
@@ -613,11 +646,14 @@ static moe_status_t down_ws_impl(const moe_desc_t* d, int32_t G, int32_t F, cons
   }
   if (!part) return moe_expert_down(d, G, F, h, a_rows, offsets, W_down, y, stream);
   cudaError_t e = launch_grouped_gemm_f32_splitk(h, a_rows, F, W_down, G, d->D, offsets, S, part,
-                                                 s);
+                                                 s, sk ? slots : 0);
   // (the decode split keeps its own summing kernel: with a handful of tokens the combine is a
   // warp or two, and the sum needs the whole GPU's loads in flight; measured at one token:
   // 0.160 against 0.183 ms with the sum inside the combine)
-  if (e == cudaSuccess) e = launch_splitk_sum(part, S, a_rows, d->D, offsets + G, y, s);
+  if (e == cudaSuccess && sk)
+    e = launch_splitk_streamk(-1, part, slots, a_rows, d->D, d->D, F, 0, offsets, G, y, s);
+  else if (e == cudaSuccess)
+    e = launch_splitk_sum(part, S, a_rows, d->D, offsets + G, y, s);
   return cuda_status(e);
 }
 

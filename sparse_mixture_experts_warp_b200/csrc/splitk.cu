@@ -121,6 +121,91 @@ splitk_sum_adaptive_kernel(const float* __restrict__ p, const int* __restrict__ 
   }
 }
 
+// Stream-K sums: the partial slots of a tile are the segments of the CTAs whose k-block ranges
+// meet it (the schedule in common.cuh); every group has at most 64 rows, so group g's tiles are
+// tiles nt * (non-empty groups before g) + n for its n-tiles n.
+constexpr int kMaxGroups = 1024;
+
+// Sum of the nseg partial slots of 4 columns at offset off (slot order).
+__device__ __forceinline__ float4 sum_slots(const float* __restrict__ p, int nseg, int64_t stride,
+                                            int64_t off) {
+  return sum_splits(p, nseg, stride, off);
+}
+
+template <int ACT>   // MOE_ACT_*; -1: no activation
+__global__ void __launch_bounds__(kThreads)
+splitk_streamk_kernel(const float* __restrict__ part, int slots, int64_t rows, int ld, int N,
+                      int nkb, int two, const int32_t* __restrict__ offsets, int G, int grid,
+                      __nv_bfloat16* __restrict__ out) {
+  pdl_trigger();
+  pdl_wait();
+  __shared__ int s_off[kMaxGroups + 1];
+  __shared__ int s_pre[kMaxGroups + 1];
+  for (int i = threadIdx.x; i <= G; i += blockDim.x) s_off[i] = __ldg(offsets + i);
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    // exclusive prefix count of the non-empty groups, 32 at a time
+    const int lane = threadIdx.x;
+    int carry = 0;
+    for (int g0 = 0; g0 < G; g0 += 32) {
+      const int g = g0 + lane;
+      const int ne = (g < G && s_off[g + 1] > s_off[g]) ? 1 : 0;
+      int inc = ne;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int v = __shfl_up_sync(0xffffffffu, inc, o);
+        if (lane >= o) inc += v;
+      }
+      if (g < G) s_pre[g] = carry + inc - ne;
+      carry += __shfl_sync(0xffffffffu, inc, 31);
+    }
+    if (lane == 0) s_pre[G] = carry;
+  }
+  __syncthreads();
+  const int half = (N + 255) / 256;
+  const int nt = two ? 2 * half : half;
+  const int64_t work = (int64_t)nt * s_pre[G] * nkb;
+  const int gct = streamk_ctas(work, nkb, slots, grid);
+  const int64_t r_end = min((int64_t)s_off[G], rows);
+  const int64_t live = r_end > s_off[0] ? r_end - s_off[0] : 0;
+  const int q = N / 4;
+  const int64_t items = live * q;
+  const int64_t stride = rows * (int64_t)ld;
+  for (int64_t i = blockIdx.x * (int64_t)kThreads + threadIdx.x; i < items;
+       i += (int64_t)gridDim.x * kThreads) {
+    const int64_t r = i / q + s_off[0];
+    const int c = (int)(i - (i / q) * q) * 4;
+    // the group of row r: the last g with s_off[g] <= r
+    int lo = 0, hi = G - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (s_off[mid] <= r) lo = mid; else hi = mid - 1;
+    }
+    const int64_t tb = (int64_t)nt * s_pre[lo];
+    const int64_t t0 = tb + c / 256;
+    const int n0 = streamk_owner((t0 + 1) * nkb - 1, work, gct) -
+                   streamk_owner(t0 * nkb, work, gct) + 1;
+    const float4 u = sum_slots(part, n0, stride, r * ld + c);
+    float4 o;
+    if (ACT == MOE_ACT_SWIGLU) {
+      // u above is the gate (product 0); the up product's tile and columns follow
+      const int64_t t1 = tb + half + c / 256;
+      const int n1 = streamk_owner((t1 + 1) * nkb - 1, work, gct) -
+                     streamk_owner(t1 * nkb, work, gct) + 1;
+      const float4 v = sum_slots(part, n1, stride, r * ld + ld / 2 + c);
+      o = make_float4(silu_mul(u.x, v.x), silu_mul(u.y, v.y), silu_mul(u.z, v.z),
+                      silu_mul(u.w, v.w));
+    } else if (ACT == MOE_ACT_GELU) {
+      o = make_float4(gelu(u.x), gelu(u.y), gelu(u.z), gelu(u.w));
+    } else if (ACT == MOE_ACT_RELU) {
+      o = make_float4(fmaxf(u.x, 0.f), fmaxf(u.y, 0.f), fmaxf(u.z, 0.f), fmaxf(u.w, 0.f));
+    } else {
+      o = u;
+    }
+    *reinterpret_cast<uint2*>(out + r * N + c) = make_uint2(pack2(o.x, o.y), pack2(o.z, o.w));
+  }
+}
+
 // enough blocks for every item of the allocated rows, at most 4 per SM (grid-stride beyond)
 int grid_for(int64_t rows, int n) {
   const int64_t items = rows * (n / 4);
@@ -131,6 +216,31 @@ int grid_for(int64_t rows, int n) {
 }
 
 }  // namespace
+
+cudaError_t launch_splitk_streamk(int act, const float* part, int slots, int64_t rows, int ld,
+                                  int N, int K, int two, const int32_t* offsets, int G,
+                                  void* out, cudaStream_t s) {
+  if (rows <= 0 || N <= 0) return cudaSuccess;
+  if (N % 4 || slots < 2 || G < 1 || G > kMaxGroups || (two && act != MOE_ACT_SWIGLU))
+    return cudaErrorInvalidValue;
+  const int nkb = (K + 63) / 64;
+  const int grid = grid_for(rows, N);
+  const int gemm_grid = gemm_sm_count();
+  __nv_bfloat16* o = static_cast<__nv_bfloat16*>(out);
+  if (act == MOE_ACT_SWIGLU)
+    (void)launch_pdl(splitk_streamk_kernel<MOE_ACT_SWIGLU>, dim3(grid), dim3(kThreads), 0, s, part,
+                     slots, rows, ld, N, nkb, two, offsets, G, gemm_grid, o);
+  else if (act == MOE_ACT_GELU)
+    (void)launch_pdl(splitk_streamk_kernel<MOE_ACT_GELU>, dim3(grid), dim3(kThreads), 0, s, part,
+                     slots, rows, ld, N, nkb, two, offsets, G, gemm_grid, o);
+  else if (act == MOE_ACT_RELU)
+    (void)launch_pdl(splitk_streamk_kernel<MOE_ACT_RELU>, dim3(grid), dim3(kThreads), 0, s, part,
+                     slots, rows, ld, N, nkb, two, offsets, G, gemm_grid, o);
+  else
+    (void)launch_pdl(splitk_streamk_kernel<-1>, dim3(grid), dim3(kThreads), 0, s, part, slots,
+                     rows, ld, N, nkb, two, offsets, G, gemm_grid, o);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_splitk_act(int act, const float* pg, const float* pu, int S, int64_t rows,
                               int F, const int32_t* n_rows, void* h, cudaStream_t s, int64_t ld) {

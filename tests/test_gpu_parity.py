@@ -224,6 +224,21 @@ def test_decode_split_schedule(name):
     C.check_sampled_output(w, inp, out, v, list(range(w.T)))
 
 
+def test_decode_without_streamk_in_subprocess():
+    """MOE_STREAMK=0: split products whose equal k-ranges take more than one wave of SMs keep
+    them (by default they run stream-K: equal shares of all tiles' k-blocks per SM); the decode
+    cases pass both ways."""
+    import os
+    import subprocess
+    import sys
+    env = dict(os.environ, MOE_STREAMK="0")
+    r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", __file__, "-k",
+                        "(decode or router_E8_T1) and not in_subprocess"], env=env,
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stdout[-3000:] + r.stderr[-3000:]
+    assert " passed" in r.stdout, r.stdout[-3000:]
+
+
 def test_decode_split_schedule_matches_fused_path_in_subprocess():
     """MOE_DECODE_SPLITK=0 keeps the fused grouped GEMMs at every size; the decode cases pass
     there too."""

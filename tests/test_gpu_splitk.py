@@ -28,6 +28,13 @@ CASES = {
     # GELU
     "gelu_T3": scaled(WORKLOADS["switch"], act="gelu", T=3, D=1024, E=16, F=512,
                       overflow="dropless", gate="renorm", k=2, zipf_s=0.0),
+    # stream-K (the split tiles would take more than one wave of SMs): the Mixtral width at one
+    # and two tokens (gate + up: 224 and 448 tiles, two k-ranges each), and a single ReLU
+    # product of 112 tiles split five ways
+    "swiglu_T1_full": scaled(WORKLOADS["mixtral"], T=1),
+    "swiglu_T2_full": scaled(WORKLOADS["mixtral"], T=2),
+    "relu_T1_wide": scaled(WORKLOADS["switch"], act="relu", T=1, D=4096, E=8, F=14336,
+                           overflow="dropless", gate="renorm", k=2, zipf_s=0.0),
 }
 
 
