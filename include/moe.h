@@ -258,7 +258,10 @@ moe_status_t moe_gather_fusion(const moe_desc_t* desc, int32_t* on);
  * the SMs busy (a_rows <= 256 for the down product, <= 16 for the up product; active groups
  * bounded by min(n_groups, a_rows)), the product is split along K into 2..8 parts whose fp32
  * partials go to scratch and are summed in a fixed order (deterministic) before the activation
- * and the bf16 rounding; SwiGLU's gate and up products run as one launch.
+ * and the bf16 rounding; SwiGLU's gate and up products run as one launch.  With at most 64 rows,
+ * a split whose tiles x k-ranges exceed the SM count runs stream-K instead (every SM an equal
+ * contiguous share of all tiles' k-blocks, at most 8 partial slots per tile, summed in slot
+ * order); MOE_STREAMK=0 keeps equal k-ranges per tile.
  * moe_expert_down_ws also splits on the device: for a desc under a capacity limit whose fewest
  * possible executed rows would give fewer output tiles than a B200 has SMs, the grouped GEMM
  * reads the group table and, when its tiles fill fewer than half of its CTAs, splits K (at most
