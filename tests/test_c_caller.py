@@ -85,3 +85,21 @@ def test_gpu_c_program_runs_the_layer(tmp_path):
     st = M.MoeStats.from_buffer_copy((tmp_path / "stats.bin").read_bytes())
     np.testing.assert_allclose(st.aux, ref["stats"]["aux"], rtol=1e-4)
     assert st.n_routes == w.T * w.k and st.n_dropped == 0
+
+
+NVCC = os.path.join(CUDA, "bin", "nvcc")
+
+
+@pytest.mark.skipif(not os.path.exists(NVCC), reason="nvcc not installed")
+def test_streamk_schedule_closed_forms(tmp_path):
+    """The stream-K schedule of the decode k-split products (common.cuh), compiled for the
+    host: the owner of every k-block and the partial-slot bound per tile agree with a
+    brute-force table over several thousand (tiles, nkb, slots, grid)."""
+    exe = tmp_path / "streamk_schedule"
+    subprocess.run([NVCC, "-std=c++17", "-O1", "-I", os.path.join(ROOT, "include"),
+                    "-I", os.path.join(ROOT, "sparse_mixture_experts_warp_b200", "csrc"),
+                    os.path.join(ROOT, "tests", "c", "streamk_schedule.cu"), "-o", str(exe)],
+                   check=True, capture_output=True, text=True)
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert r.stdout.startswith("ok:"), r.stdout
