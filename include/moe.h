@@ -30,6 +30,22 @@
  *     and moe_balance_stats check their arguments and return MOE_OK without launching anything
  *     or writing any output (views and statistics keep their previous contents); moe_permute
  *     writes zero counts and offsets; the expert products have no rows to compute.
+ *
+ * Environment switches, read once per process.  The defaults are the paths measured fastest on
+ * B200; each switch keeps another tested path reachable for comparison measurements:
+ *   MOE_ROUTER=tc|fast|gemm|simt   router kernel (default: mma.sync for E <= 8 with
+ *                                  D = 256 * (4..16), else the tcgen05 router, else SIMT)
+ *   MOE_GEMM_TILE=128|256|256k32|pair  one grouped-GEMM tile shape for every call (default:
+ *                                  chosen per call by group size and whole waves of SMs)
+ *   MOE_GEMM_SWAP=1                grouped GEMMs with the weights as the MMA's M side
+ *   MOE_GATHER_FUSION=1            the layer's up projection gathers the token rows itself
+ *   MOE_DECODE_SPLITK=0            no k-split schedule for few executed rows
+ *   MOE_STREAMK=0                  equal k-ranges instead of stream-K in that schedule
+ *   MOE_ADAPTIVE_SPLIT=0           no device-side k-split of a capacity-limited down product
+ *   MOE_PERMUTE_CLUSTER=0          no one-cluster permutation index kernel
+ *   MOE_PDL=0                      no programmatic dependent launch between kernels
+ *   MOE_WGRAD_TILE=128             128-row weight-gradient tiles (default 256)
+ *   MOE_BWD_WEIGHT_TRANSPOSE=1     the backward's dgrad products read transposed weight copies
  */
 #ifndef MOE_B200_H
 #define MOE_B200_H
