@@ -723,7 +723,10 @@ def run_cuda(args, rank, world, local):
                          % ((w.E * 3 * w.F * w.D * 2) / 1e9)},
         "roofline": roofline, "stages": stages,
         "stage_timing": ("graph replays with event record nodes between the stages"
-                         if graph_stage is not None else "eager calls, events between stages"),
+                         if graph_stage is not None else "eager calls, events between stages")
+                        + "; each stage is its step entry point (moe_layer_forward computes the"
+                          " statistics inside the combine's launch and, under a capacity"
+                          " limit, sums the down projection's k-split there too)",
         "eager_stage_us": {s: round(eager_stage[s] * 1e3, 2) for s in STAGES},
         "e2e": {"value": round(e2e_value, 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms / args.steps, 4),
